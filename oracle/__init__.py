@@ -1,0 +1,177 @@
+"""float64 CPU oracle for the gated delta rule -- TEST INFRASTRUCTURE ONLY.
+
+Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product library never does, and
+this package imports nothing from the product.  It wraps ``gdn_oracle.c``
+(plain C, double precision, OpenMP over (batch, head)) through ctypes.
+
+What is computed follows "ATMA: Long-Context Language Modeling via Polar
+Attention and Gated-Delta Compression Memory", Sec. 3.3 (the gated-delta
+memory equation), with gamma_t renamed alpha_t, M renamed S and r renamed o:
+
+    S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,   o_t = S_t q_t.
+
+Array conventions (numpy, C-contiguous):
+    q, k [B, T, H, dk] and v [B, T, H, dv] as float32 (bf16 inputs are passed
+    as their exact float32 values); log_alpha, beta [B, T, H] float32;
+    S0 / S_final [B, H, dv, dk] float64; out [B, T, H, dv] float64.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(_HERE, "gdn_oracle.c")
+LIBRARY = os.path.join(_HERE, "libgdn_oracle.so")
+
+_i64 = ctypes.c_int64
+_ptr = ctypes.c_void_p
+
+
+def build(src: str = SOURCE, out: str = LIBRARY, force: bool = False) -> str:
+    """Compile the oracle with gcc (no fast-math: IEEE double throughout)."""
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src):
+        return out
+    tmp = out + ".tmp%d" % os.getpid()
+    cmd = ["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-Wall", "-o", tmp, src, "-lm"]
+    subprocess.run(cmd, check=True, capture_output=True, text=True)
+    os.replace(tmp, out)
+    return out
+
+
+def _f32(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float32)
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _p(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(_ptr)
+
+
+class Oracle:
+    """ctypes view of one compiled oracle library (the real one, or a test mutant)."""
+
+    def __init__(self, path: str):
+        self.path = path
+        self.lib = ctypes.CDLL(path)
+        L = self.lib
+        L.gdn_oracle_forward.argtypes = [_ptr] * 8 + [_i64] * 5 + [ctypes.c_int]
+        L.gdn_oracle_forward_chunked.argtypes = [_ptr] * 8 + [_i64] * 6 + [ctypes.c_int]
+        L.gdn_oracle_decode_step.argtypes = [_ptr] * 7 + [_i64] * 4 + [ctypes.c_int]
+        L.gdn_oracle_segment_transfer.argtypes = [_ptr] * 6 + [_i64] * 4
+        L.gdn_oracle_dense_product.argtypes = [_ptr] * 8 + [_i64] * 3
+        for f in ("gdn_oracle_forward", "gdn_oracle_forward_chunked", "gdn_oracle_decode_step",
+                  "gdn_oracle_segment_transfer", "gdn_oracle_dense_product"):
+            getattr(L, f).restype = ctypes.c_int
+
+    # -- the definition: token-by-token recurrence ---------------------------------
+    def forward(self, q, k, v, log_alpha, beta, S0=None, nthreads: int = 0, want_out: bool = True):
+        """Sequential recurrence.  Returns (out [B,T,H,dv] float64 or None, S_final float64)."""
+        q, k, v, la, be = _f32(q), _f32(k), _f32(v), _f32(log_alpha), _f32(beta)
+        B, T, H, dk = q.shape
+        dv = v.shape[-1]
+        _check_shapes(q, k, v, la, be, B, T, H, dk, dv)
+        S0 = None if S0 is None else _f64(S0)
+        if S0 is not None:
+            assert S0.shape == (B, H, dv, dk)
+        out = np.empty((B, T, H, dv), np.float64) if want_out else None
+        Sf = np.empty((B, H, dv, dk), np.float64)
+        rc = self.lib.gdn_oracle_forward(_p(q), _p(k), _p(v), _p(la), _p(be), _p(S0), _p(out), _p(Sf),
+                                         B, T, H, dk, dv, nthreads)
+        if rc != 0:
+            raise RuntimeError("gdn_oracle_forward failed (%d)" % rc)
+        return out, Sf
+
+    def decode_step(self, q, k, v, log_alpha, beta, S, nthreads: int = 0):
+        """One token for every (b, h); S [B,H,dv,dk] float64 is updated in place.
+        q, k [B,H,dk]; v [B,H,dv]; gates [B,H].  Returns out [B,H,dv] float64."""
+        q, k, v, la, be = _f32(q), _f32(k), _f32(v), _f32(log_alpha), _f32(beta)
+        B, H, dk = q.shape
+        dv = v.shape[-1]
+        assert S.dtype == np.float64 and S.flags.c_contiguous and S.shape == (B, H, dv, dk)
+        assert k.shape == (B, H, dk) and v.shape == (B, H, dv) and la.shape == (B, H) and be.shape == (B, H)
+        out = np.empty((B, H, dv), np.float64)
+        rc = self.lib.gdn_oracle_decode_step(_p(q), _p(k), _p(v), _p(la), _p(be), _p(S), _p(out),
+                                             B, H, dk, dv, nthreads)
+        if rc != 0:
+            raise RuntimeError("gdn_oracle_decode_step failed (%d)" % rc)
+        return out
+
+    # -- test-only alternative forms ----------------------------------------------
+    def forward_chunked(self, q, k, v, log_alpha, beta, S0=None, chunk: int = 64, nthreads: int = 0):
+        """Chunkwise (UT-transform) form of the same recurrence, float64."""
+        q, k, v, la, be = _f32(q), _f32(k), _f32(v), _f32(log_alpha), _f32(beta)
+        B, T, H, dk = q.shape
+        dv = v.shape[-1]
+        _check_shapes(q, k, v, la, be, B, T, H, dk, dv)
+        S0 = None if S0 is None else _f64(S0)
+        out = np.empty((B, T, H, dv), np.float64)
+        Sf = np.empty((B, H, dv, dk), np.float64)
+        rc = self.lib.gdn_oracle_forward_chunked(_p(q), _p(k), _p(v), _p(la), _p(be), _p(S0), _p(out),
+                                                 _p(Sf), B, T, H, dk, dv, chunk, nthreads)
+        if rc != 0:
+            raise RuntimeError("gdn_oracle_forward_chunked failed (%d)" % rc)
+        return out, Sf
+
+    def segment_transfer(self, k, v, log_alpha, beta, chunk: int = 64):
+        """Affine transfer (M [dk,dk], Bseg [dv,dk]) of one head's run of tokens: k [T,dk], v [T,dv]."""
+        k, v, la, be = _f32(k), _f32(v), _f32(log_alpha), _f32(beta)
+        T, dk = k.shape
+        dv = v.shape[1]
+        M = np.empty((dk, dk), np.float64)
+        Bs = np.empty((dv, dk), np.float64)
+        rc = self.lib.gdn_oracle_segment_transfer(_p(k), _p(v), _p(la), _p(be), _p(M), _p(Bs), T, dk, dv, chunk)
+        if rc != 0:
+            raise RuntimeError("gdn_oracle_segment_transfer failed (%d)" % rc)
+        return M, Bs
+
+    def dense_product(self, q, k, v, log_alpha, beta, S0=None):
+        """Brute-force product form for one head, T <= 16: q,k [T,dk], v [T,dv], S0 [dv,dk]."""
+        q, k, v, la, be = _f32(q), _f32(k), _f32(v), _f32(log_alpha), _f32(beta)
+        T, dk = q.shape
+        dv = v.shape[1]
+        S0 = None if S0 is None else _f64(S0)
+        out = np.empty((T, dv), np.float64)
+        Sf = np.empty((dv, dk), np.float64)
+        rc = self.lib.gdn_oracle_dense_product(_p(q), _p(k), _p(v), _p(la), _p(be), _p(S0), _p(out), _p(Sf),
+                                               T, dk, dv)
+        if rc != 0:
+            raise RuntimeError("gdn_oracle_dense_product failed (%d)" % rc)
+        return out, Sf
+
+
+def _check_shapes(q, k, v, la, be, B, T, H, dk, dv):
+    assert k.shape == (B, T, H, dk), (k.shape, (B, T, H, dk))
+    assert v.shape == (B, T, H, dv)
+    assert la.shape == (B, T, H) and be.shape == (B, T, H)
+
+
+_default: Optional[Oracle] = None
+
+
+def get() -> Oracle:
+    """The oracle built from the committed source (compiled on first use)."""
+    global _default
+    if _default is None:
+        _default = Oracle(build())
+    return _default
+
+
+def forward(*args, **kw):
+    return get().forward(*args, **kw)
+
+
+def decode_step(*args, **kw):
+    return get().decode_step(*args, **kw)
+
+
+def forward_chunked(*args, **kw):
+    return get().forward_chunked(*args, **kw)

@@ -1,0 +1,447 @@
+/*
+ * gdn_oracle.c -- float64 CPU oracle for the gated delta rule.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product library links, includes
+ * or calls this file; only the test suite, the smoke check and the CPU
+ * baseline leg of the benchmark load it (through oracle/__init__.py).  It
+ * shares no source with the CUDA path.
+ *
+ * What it computes (source: "ATMA: Long-Context Language Modeling via Polar
+ * Attention and Gated-Delta Compression Memory", Sec. 3.3, the gated-delta
+ * memory equation), per (batch b, head h), with the paper's symbols renamed
+ * gamma_t -> alpha_t, M -> S, r -> o:
+ *
+ *     S_t = alpha_t * S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t = S_t q_t
+ *
+ * S is d_v x d_k (row index over the value dimension, column index over the
+ * key dimension), held in double.  alpha_t = exp(log_alpha_t).
+ *
+ * Layouts (row-major, 64-bit indexing):
+ *   q, k        [B, T, H, dk]      float (exact values of the caller's inputs)
+ *   v, out      [B, T, H, dv]      float in, double out
+ *   log_alpha,
+ *   beta        [B, T, H]          float
+ *   S0, S_final [B, H, dv, dk]     double; S0 may be NULL (zero state),
+ *                                  S_final may be NULL (not written)
+ *
+ * Inputs are taken as float because every input the library accepts (fp32
+ * or bf16) converts to float exactly; all arithmetic is double.
+ *
+ * Functions:
+ *   gdn_oracle_forward          the token-by-token recurrence (the definition)
+ *   gdn_oracle_decode_step      one token for every (b, h), state in place
+ *   gdn_oracle_forward_chunked  the chunkwise (WY / UT-transform) form of the
+ *                               same recurrence, any chunk length C >= 1; the
+ *                               algebra is the one of the works the paper cites
+ *                               for the memory ("Gated delta networks",
+ *                               "Parallelizing linear transformers with the
+ *                               delta rule over sequence length"), re-derived
+ *                               from the Sec. 3.3 equation
+ *   gdn_oracle_segment_transfer the affine map S_end = S_start M + Bseg of a
+ *                               run of tokens, built chunk by chunk
+ *   gdn_oracle_dense_product    brute force: explicit d_k x d_k factors
+ *                               alpha_t (I - beta_t k_t k_t^T), tiny T only
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define IDX_TOK(b, t, h, d, T, H, D) ((((int64_t)(b) * (T) + (t)) * (H) + (h)) * (D) + (d))
+#define IDX_GATE(b, t, h, T, H) (((int64_t)(b) * (T) + (t)) * (H) + (h))
+#define IDX_STATE(b, h, H, dv, dk) (((int64_t)(b) * (H) + (h)) * (dv) * (dk))
+
+static void set_threads(int nthreads) {
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+}
+
+/* One token of the Sec. 3.3 recurrence on a single state S (dv x dk).
+ * S (I - beta k k^T) is evaluated as S - beta (S k) k^T, which is the same
+ * matrix (associativity), so the step costs O(dv dk) instead of O(dv dk^2). */
+static void recurrence_step(double *S, const float *q, const float *k, const float *v,
+                            float log_alpha, float beta, double *o, double *x,
+                            int64_t dk, int64_t dv) {
+    const double a = exp((double)log_alpha);
+    const double bt = (double)beta;
+    for (int64_t r = 0; r < dv; ++r) {          /* x = S_{t-1} k_t */
+        double acc = 0.0;
+        for (int64_t c = 0; c < dk; ++c) acc += S[r * dk + c] * (double)k[c];
+        x[r] = acc;
+    }
+    for (int64_t r = 0; r < dv; ++r) {
+        for (int64_t c = 0; c < dk; ++c) {
+            /* alpha * [S (I - beta k k^T)]_{rc} + beta v_r k_c */
+            const double sk = S[r * dk + c] - bt * x[r] * (double)k[c];
+            S[r * dk + c] = a * sk + bt * (double)v[r] * (double)k[c];
+        }
+    }
+    for (int64_t r = 0; r < dv; ++r) {          /* o_t = S_t q_t */
+        double acc = 0.0;
+        for (int64_t c = 0; c < dk; ++c) acc += S[r * dk + c] * (double)q[c];
+        o[r] = acc;
+    }
+}
+
+int gdn_oracle_forward(const float *q, const float *k, const float *v,
+                       const float *log_alpha, const float *beta, const double *S0,
+                       double *out, double *S_final, int64_t B, int64_t T, int64_t H,
+                       int64_t dk, int64_t dv, int nthreads) {
+    if (B < 0 || T < 0 || H < 0 || dk < 1 || dv < 1) return 1;
+    set_threads(nthreads);
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        const int64_t b = bh / H, h = bh % H;
+        double *S = (double *)malloc(sizeof(double) * dv * dk);
+        double *x = (double *)malloc(sizeof(double) * dv);
+        double *o = (double *)malloc(sizeof(double) * dv);
+        if (!S || !x || !o) {
+            free(S); free(x); free(o);
+#pragma omp atomic write
+            failed = 1;
+            continue;
+        }
+        if (S0) memcpy(S, S0 + IDX_STATE(b, h, H, dv, dk), sizeof(double) * dv * dk);
+        else memset(S, 0, sizeof(double) * dv * dk);
+        for (int64_t t = 0; t < T; ++t) {
+            recurrence_step(S, q + IDX_TOK(b, t, h, 0, T, H, dk), k + IDX_TOK(b, t, h, 0, T, H, dk),
+                            v + IDX_TOK(b, t, h, 0, T, H, dv), log_alpha[IDX_GATE(b, t, h, T, H)],
+                            beta[IDX_GATE(b, t, h, T, H)], o, x, dk, dv);
+            if (out) memcpy(out + IDX_TOK(b, t, h, 0, T, H, dv), o, sizeof(double) * dv);
+        }
+        if (S_final) memcpy(S_final + IDX_STATE(b, h, H, dv, dk), S, sizeof(double) * dv * dk);
+        free(S); free(x); free(o);
+    }
+    return failed ? 2 : 0;
+}
+
+/* Decode: one token per (b, h).  q, k [B, H, dk]; v, out [B, H, dv];
+ * gates [B, H]; S [B, H, dv, dk] updated in place. */
+int gdn_oracle_decode_step(const float *q, const float *k, const float *v,
+                           const float *log_alpha, const float *beta, double *S,
+                           double *out, int64_t B, int64_t H, int64_t dk, int64_t dv,
+                           int nthreads) {
+    if (B < 0 || H < 0 || dk < 1 || dv < 1) return 1;
+    set_threads(nthreads);
+    int failed = 0;
+#pragma omp parallel for schedule(static)
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        double *x = (double *)malloc(sizeof(double) * dv);
+        if (!x) {
+#pragma omp atomic write
+            failed = 1;
+            continue;
+        }
+        recurrence_step(S + bh * dv * dk, q + bh * dk, k + bh * dk, v + bh * dv, log_alpha[bh],
+                        beta[bh], out + bh * dv, x, dk, dv);
+        free(x);
+    }
+    return failed ? 2 : 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Chunkwise form.  Within a chunk of n <= C tokens with entry state S0, write
+ * the Sec. 3.3 step as S_t = alpha_t S_{t-1} + u_t k_t^T with
+ * u_t = beta_t (v_t - alpha_t S_{t-1} k_t).  Unrolling,
+ *     S_t = gamma_t S0 + sum_{s<=t} (gamma_t / gamma_s) u_s k_s^T,
+ * gamma_t = prod_{r<=t} alpha_r (chunk-local).  Putting that back into u_t
+ * gives the unit-lower-triangular system
+ *     (I + A) U = diag(beta) V - diag(beta*gamma) K S0^T,
+ *     A_ts = beta_t (gamma_t/gamma_s) (k_t . k_s)   for s < t, else 0,
+ * so with Tinv = (I + A)^{-1} (forward substitution):
+ *     W  = Tinv diag(beta*gamma) K,   Ut = Tinv diag(beta) V,   U = Ut - W S0^T
+ *     O  = diag(gamma) Q S0^T + [ (Q K^T) o (gamma_t/gamma_s) ]_{s<=t} U
+ *     S_n = gamma_n S0 + U^T Ktil,   Ktil_s = (gamma_n/gamma_s) k_s.
+ * Ratios gamma_t/gamma_s (s <= t) are formed as products of the alphas in
+ * (s, t], so an alpha of exactly 0 stays exact and nothing overflows.
+ * ---------------------------------------------------------------------- */
+
+/* decay[t][s] = prod_{r=s+1..t} alpha_r for s <= t (1 on the diagonal), 0 above. */
+static void chunk_decays(const double *alpha, int64_t n, double *decay) {
+    for (int64_t t = 0; t < n; ++t) {
+        for (int64_t s = 0; s < n; ++s) {
+            if (s > t) { decay[t * n + s] = 0.0; continue; }
+            double p = 1.0;
+            for (int64_t r = s + 1; r <= t; ++r) p *= alpha[r];
+            decay[t * n + s] = p;
+        }
+    }
+}
+
+/* One chunk: consumes entry state S (dv x dk), writes o (n x dv, may be NULL)
+ * and replaces S by the exit state.  Token rows are gathered into dense
+ * n x d matrices by the caller. */
+static void chunk_step(double *S, const double *Q, const double *K, const double *V,
+                       const double *alpha, const double *beta, int64_t n, int64_t dk,
+                       int64_t dv, double *o, double *work) {
+    double *decay = work;                  /* n*n   */
+    double *gamma = decay + n * n;         /* n     */
+    double *A = gamma + n;                 /* n*n   */
+    double *Tinv = A + n * n;              /* n*n   */
+    double *Wm = Tinv + n * n;             /* n*dk  */
+    double *Ut = Wm + n * dk;              /* n*dv  */
+    double *U = Ut + n * dv;               /* n*dv  */
+    double *Snew = U + n * dv;             /* dv*dk */
+
+    chunk_decays(alpha, n, decay);
+    for (int64_t t = 0; t < n; ++t) gamma[t] = decay[t * n + 0] * alpha[0];
+
+    /* A_ts = beta_t (gamma_t/gamma_s) (k_t . k_s), strictly lower */
+    for (int64_t t = 0; t < n; ++t)
+        for (int64_t s = 0; s < n; ++s) {
+            double a = 0.0;
+            if (s < t) {
+                double kk = 0.0;
+                for (int64_t c = 0; c < dk; ++c) kk += K[t * dk + c] * K[s * dk + c];
+                a = beta[t] * decay[t * n + s] * kk;
+            }
+            A[t * n + s] = a;
+        }
+    /* Tinv = (I + A)^{-1}: solve (I + A) X = I column by column, top to bottom */
+    for (int64_t j = 0; j < n; ++j)
+        for (int64_t t = 0; t < n; ++t) {
+            double x = (t == j) ? 1.0 : 0.0;
+            for (int64_t s = 0; s < t; ++s) x -= A[t * n + s] * Tinv[s * n + j];
+            Tinv[t * n + j] = x;
+        }
+    /* W = Tinv diag(beta*gamma) K ;  Ut = Tinv diag(beta) V */
+    for (int64_t t = 0; t < n; ++t) {
+        for (int64_t c = 0; c < dk; ++c) {
+            double acc = 0.0;
+            for (int64_t s = 0; s < n; ++s) acc += Tinv[t * n + s] * beta[s] * gamma[s] * K[s * dk + c];
+            Wm[t * dk + c] = acc;
+        }
+        for (int64_t r = 0; r < dv; ++r) {
+            double acc = 0.0;
+            for (int64_t s = 0; s < n; ++s) acc += Tinv[t * n + s] * beta[s] * V[s * dv + r];
+            Ut[t * dv + r] = acc;
+        }
+    }
+    /* U = Ut - W S0^T */
+    for (int64_t t = 0; t < n; ++t)
+        for (int64_t r = 0; r < dv; ++r) {
+            double acc = 0.0;
+            for (int64_t c = 0; c < dk; ++c) acc += Wm[t * dk + c] * S[r * dk + c];
+            U[t * dv + r] = Ut[t * dv + r] - acc;
+        }
+    /* O = diag(gamma) Q S0^T + [(Q K^T) o decay]_{s<=t} U */
+    if (o) {
+        for (int64_t t = 0; t < n; ++t)
+            for (int64_t r = 0; r < dv; ++r) {
+                double inter = 0.0;
+                for (int64_t c = 0; c < dk; ++c) inter += Q[t * dk + c] * S[r * dk + c];
+                double intra = 0.0;
+                for (int64_t s = 0; s <= t; ++s) {
+                    double qk = 0.0;
+                    for (int64_t c = 0; c < dk; ++c) qk += Q[t * dk + c] * K[s * dk + c];
+                    intra += qk * decay[t * n + s] * U[s * dv + r];
+                }
+                o[t * dv + r] = gamma[t] * inter + intra;
+            }
+    }
+    /* S_n = gamma_n S0 + U^T Ktil */
+    for (int64_t r = 0; r < dv; ++r)
+        for (int64_t c = 0; c < dk; ++c) {
+            double acc = 0.0;
+            for (int64_t s = 0; s < n; ++s) acc += U[s * dv + r] * decay[(n - 1) * n + s] * K[s * dk + c];
+            Snew[r * dk + c] = gamma[n - 1] * S[r * dk + c] + acc;
+        }
+    memcpy(S, Snew, sizeof(double) * dv * dk);
+}
+
+static size_t chunk_work_doubles(int64_t C, int64_t dk, int64_t dv) {
+    return (size_t)(3 * C * C + C + C * dk + 2 * C * dv + dv * dk);
+}
+
+/* Gather n token rows of one (b, h) into dense double matrices. */
+static void gather_chunk(const float *q, const float *k, const float *v, const float *log_alpha,
+                         const float *beta, int64_t b, int64_t h, int64_t t0, int64_t n,
+                         int64_t T, int64_t H, int64_t dk, int64_t dv, double *Q, double *K,
+                         double *V, double *al, double *be) {
+    for (int64_t i = 0; i < n; ++i) {
+        const int64_t t = t0 + i;
+        for (int64_t c = 0; c < dk; ++c) {
+            if (Q) Q[i * dk + c] = (double)q[IDX_TOK(b, t, h, c, T, H, dk)];
+            K[i * dk + c] = (double)k[IDX_TOK(b, t, h, c, T, H, dk)];
+        }
+        for (int64_t r = 0; r < dv; ++r) V[i * dv + r] = (double)v[IDX_TOK(b, t, h, r, T, H, dv)];
+        al[i] = exp((double)log_alpha[IDX_GATE(b, t, h, T, H)]);
+        be[i] = (double)beta[IDX_GATE(b, t, h, T, H)];
+    }
+}
+
+int gdn_oracle_forward_chunked(const float *q, const float *k, const float *v,
+                               const float *log_alpha, const float *beta, const double *S0,
+                               double *out, double *S_final, int64_t B, int64_t T, int64_t H,
+                               int64_t dk, int64_t dv, int64_t C, int nthreads) {
+    if (B < 0 || T < 0 || H < 0 || dk < 1 || dv < 1 || C < 1) return 1;
+    set_threads(nthreads);
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        const int64_t b = bh / H, h = bh % H;
+        double *S = (double *)malloc(sizeof(double) * dv * dk);
+        double *Q = (double *)malloc(sizeof(double) * C * dk);
+        double *K = (double *)malloc(sizeof(double) * C * dk);
+        double *V = (double *)malloc(sizeof(double) * C * dv);
+        double *al = (double *)malloc(sizeof(double) * C);
+        double *be = (double *)malloc(sizeof(double) * C);
+        double *o = (double *)malloc(sizeof(double) * C * dv);
+        double *work = (double *)malloc(sizeof(double) * chunk_work_doubles(C, dk, dv));
+        if (!S || !Q || !K || !V || !al || !be || !o || !work) {
+#pragma omp atomic write
+            failed = 1;
+        } else {
+            if (S0) memcpy(S, S0 + IDX_STATE(b, h, H, dv, dk), sizeof(double) * dv * dk);
+            else memset(S, 0, sizeof(double) * dv * dk);
+            for (int64_t t0 = 0; t0 < T; t0 += C) {
+                const int64_t n = (T - t0 < C) ? (T - t0) : C;
+                gather_chunk(q, k, v, log_alpha, beta, b, h, t0, n, T, H, dk, dv, Q, K, V, al, be);
+                chunk_step(S, Q, K, V, al, be, n, dk, dv, o, work);
+                if (out)
+                    for (int64_t i = 0; i < n; ++i)
+                        memcpy(out + IDX_TOK(b, t0 + i, h, 0, T, H, dv), o + i * dv, sizeof(double) * dv);
+            }
+            if (S_final) memcpy(S_final + IDX_STATE(b, h, H, dv, dk), S, sizeof(double) * dv * dk);
+        }
+        free(S); free(Q); free(K); free(V); free(al); free(be); free(o); free(work);
+    }
+    return failed ? 2 : 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Segment transfer.  Each chunk maps its entry state affinely:
+ *     S_n = S0 (gamma_n I - W^T Ktil) + Ut^T Ktil = S0 Mc + Bc,
+ * so a run of chunks maps S_start -> S_start Mseg + Bseg with
+ *     Mseg <- Mseg Mc,  Bseg <- Bseg Mc + Bc   (chunk by chunk).
+ * Mseg is dk x dk, Bseg is dv x dk.  Single (b, h): inputs are [T, d].
+ * ---------------------------------------------------------------------- */
+int gdn_oracle_segment_transfer(const float *k, const float *v, const float *log_alpha,
+                                const float *beta, double *Mseg, double *Bseg, int64_t T,
+                                int64_t dk, int64_t dv, int64_t C) {
+    if (T < 0 || dk < 1 || dv < 1 || C < 1) return 1;
+    double *K = (double *)malloc(sizeof(double) * C * dk);
+    double *V = (double *)malloc(sizeof(double) * C * dv);
+    double *al = (double *)malloc(sizeof(double) * C);
+    double *be = (double *)malloc(sizeof(double) * C);
+    /* the d_k transfer rows run through chunk_step as a state with d_k rows */
+    double *work = (double *)malloc(sizeof(double) * chunk_work_doubles(C, dk, dv > dk ? dv : dk));
+    double *Mc = (double *)malloc(sizeof(double) * dk * dk);
+    double *Bc = (double *)malloc(sizeof(double) * dv * dk);
+    double *tmpM = (double *)malloc(sizeof(double) * dk * dk);
+    double *tmpB = (double *)malloc(sizeof(double) * dv * dk);
+    int rc = 0;
+    if (!K || !V || !al || !be || !work || !Mc || !Bc || !tmpM || !tmpB) { rc = 2; goto done; }
+    for (int64_t i = 0; i < dk; ++i)
+        for (int64_t j = 0; j < dk; ++j) Mseg[i * dk + j] = (i == j) ? 1.0 : 0.0;
+    memset(Bseg, 0, sizeof(double) * dv * dk);
+    for (int64_t t0 = 0; t0 < T; t0 += C) {
+        const int64_t n = (T - t0 < C) ? (T - t0) : C;
+        gather_chunk(NULL, k, v, log_alpha, beta, 0, 0, t0, n, T, 1, dk, dv, NULL, K, V, al, be);
+        /* Bc = chunk applied to the zero state; Mc row i = chunk applied to e_i^T
+         * with v = 0 (rows of the state evolve independently). */
+        memset(Bc, 0, sizeof(double) * dv * dk);
+        chunk_step(Bc, NULL, K, V, al, be, n, dk, dv, NULL, work);
+        double *Vz = (double *)calloc((size_t)(n * dk), sizeof(double));
+        if (!Vz) { rc = 2; goto done; }
+        for (int64_t i = 0; i < dk; ++i)
+            for (int64_t j = 0; j < dk; ++j) Mc[i * dk + j] = (i == j) ? 1.0 : 0.0;
+        chunk_step(Mc, NULL, K, Vz, al, be, n, dk, dk, NULL, work);
+        free(Vz);
+        /* compose */
+        for (int64_t i = 0; i < dk; ++i)
+            for (int64_t j = 0; j < dk; ++j) {
+                double acc = 0.0;
+                for (int64_t l = 0; l < dk; ++l) acc += Mseg[i * dk + l] * Mc[l * dk + j];
+                tmpM[i * dk + j] = acc;
+            }
+        for (int64_t r = 0; r < dv; ++r)
+            for (int64_t j = 0; j < dk; ++j) {
+                double acc = Bc[r * dk + j];
+                for (int64_t l = 0; l < dk; ++l) acc += Bseg[r * dk + l] * Mc[l * dk + j];
+                tmpB[r * dk + j] = acc;
+            }
+        memcpy(Mseg, tmpM, sizeof(double) * dk * dk);
+        memcpy(Bseg, tmpB, sizeof(double) * dv * dk);
+    }
+done:
+    free(K); free(V); free(al); free(be); free(work); free(Mc); free(Bc); free(tmpM); free(tmpB);
+    return rc;
+}
+
+/* ------------------------------------------------------------------------
+ * Brute force for tiny T, single (b, h), inputs [T, d]: with the explicit
+ * d_k x d_k factors F_t = alpha_t (I - beta_t k_t k_t^T),
+ *     S_t = S0 F_1 ... F_t + sum_{s<=t} beta_s v_s k_s^T F_{s+1} ... F_t,
+ * every product formed from scratch for every t (no reuse between t).
+ * ---------------------------------------------------------------------- */
+int gdn_oracle_dense_product(const float *q, const float *k, const float *v,
+                             const float *log_alpha, const float *beta, const double *S0,
+                             double *out, double *S_final, int64_t T, int64_t dk, int64_t dv) {
+    if (T < 0 || T > 16 || dk < 1 || dv < 1 || dk > 64 || dv > 64) return 1;
+    double *F = (double *)malloc(sizeof(double) * (T > 0 ? T : 1) * dk * dk);
+    double *P = (double *)malloc(sizeof(double) * dk * dk);
+    double *tmp = (double *)malloc(sizeof(double) * dk * dk);
+    double *St = (double *)malloc(sizeof(double) * dv * dk);
+    if (!F || !P || !tmp || !St) { free(F); free(P); free(tmp); free(St); return 2; }
+    for (int64_t t = 0; t < T; ++t) {
+        const double a = exp((double)log_alpha[t]), bt = (double)beta[t];
+        for (int64_t i = 0; i < dk; ++i)
+            for (int64_t j = 0; j < dk; ++j)
+                F[t * dk * dk + i * dk + j] =
+                    a * (((i == j) ? 1.0 : 0.0) - bt * (double)k[t * dk + i] * (double)k[t * dk + j]);
+    }
+    for (int64_t t = 0; t < T; ++t) {
+        memset(St, 0, sizeof(double) * dv * dk);
+        /* term j = -1 is S0 F_0..F_t ; term j >= 0 is beta_j v_j k_j^T F_{j+1}..F_t */
+        for (int64_t j = -1; j <= t; ++j) {
+            for (int64_t i = 0; i < dk; ++i)
+                for (int64_t l = 0; l < dk; ++l) P[i * dk + l] = (i == l) ? 1.0 : 0.0;
+            for (int64_t m = j + 1; m <= t; ++m) {
+                for (int64_t i = 0; i < dk; ++i)
+                    for (int64_t l = 0; l < dk; ++l) {
+                        double acc = 0.0;
+                        for (int64_t x = 0; x < dk; ++x) acc += P[i * dk + x] * F[m * dk * dk + x * dk + l];
+                        tmp[i * dk + l] = acc;
+                    }
+                memcpy(P, tmp, sizeof(double) * dk * dk);
+            }
+            for (int64_t r = 0; r < dv; ++r)
+                for (int64_t l = 0; l < dk; ++l) {
+                    double acc = 0.0;
+                    if (j < 0) {
+                        if (S0)
+                            for (int64_t x = 0; x < dk; ++x) acc += S0[r * dk + x] * P[x * dk + l];
+                    } else {
+                        const double bv = (double)beta[j] * (double)v[j * dv + r];
+                        for (int64_t x = 0; x < dk; ++x) acc += bv * (double)k[j * dk + x] * P[x * dk + l];
+                    }
+                    St[r * dk + l] += acc;
+                }
+        }
+        if (out)
+            for (int64_t r = 0; r < dv; ++r) {
+                double acc = 0.0;
+                for (int64_t c = 0; c < dk; ++c) acc += St[r * dk + c] * (double)q[t * dk + c];
+                out[t * dv + r] = acc;
+            }
+    }
+    if (S_final) {
+        if (T == 0) {
+            if (S0) memcpy(S_final, S0, sizeof(double) * dv * dk);
+            else memset(S_final, 0, sizeof(double) * dv * dk);
+        } else {
+            memcpy(S_final, St, sizeof(double) * dv * dk);
+        }
+    }
+    free(F); free(P); free(tmp); free(St);
+    return 0;
+}
