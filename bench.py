@@ -1,0 +1,378 @@
+#!/usr/bin/env python
+"""Benchmark of the gated-delta-rule library on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl gdn|reference]
+
+One step = one ``gdn_forward`` call over the long-sequence workload (bf16
+q/k/v, float32 gates and state, B=1, H=16, T=65536, dk=dv=128, chunk=64,
+slow-decay gates) with inputs resident in HBM.  The single-token decode path
+(B=64, H=16, d=128, state 134 MB) is timed in its own region and reported in
+the same line under ``decode``.  Under torchrun every rank runs its own
+independent replica (the (batch, head) problems are independent: weak
+scaling, no collective on the data path); times are device times (CUDA
+events on the launching stream), max over ranks.
+
+The JSON line also carries ``e2e`` (the same metric through the C ABI with
+pinned host buffers, copies inside the timed region), ``roofline`` of the
+forward kernel, ``clocks`` sampled with nvidia-smi during the run, and
+``cpu_baseline`` (the float64 oracle on a bounded sample, host cores).
+``--impl reference`` times the float64 CPU oracle as the reference arm.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from gdn_inputs import WORKLOADS, as_f32_numpy, decode_inputs, forward_inputs  # noqa: E402
+
+FWD_WORKLOAD = "fwd_bf16_b1h16_t64k_d128"
+DEC_WORKLOAD = "decode_bf16_b64h16_d128_x1024"
+METRIC = "gated-delta forward tokens/s & TFLOP/s vs BF16 roofline; decode GB/s vs HBM peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------- unit counts
+def fwd_flop_per_token_head(dk, dv, C):
+    """Full-tile contractions of the chunkwise method per token and head:
+    K K^T, Q K^T, T.(beta gamma K), T.(beta V), P.U  (2C(3dk + 2dv))
+    and W S^T, Q S^T, U^T Ktil (6 dk dv)."""
+    return 2 * C * (3 * dk + 2 * dv) + 6 * dk * dv
+
+
+def fwd_bytes(B, T, H, dk, dv, es, s0, s_final):
+    """Compulsory HBM bytes of one forward: q, k, v, out, two float32 gates, and the states."""
+    per_tok_head = (2 * dk + 2 * dv) * es + 8
+    return B * T * H * per_tok_head + (int(s0) + int(s_final)) * B * H * dv * dk * 4
+
+
+def decode_bytes_per_head_step(dk, dv, es):
+    return 2 * dk * dv * 4 + (2 * dk + 2 * dv) * es + 8
+
+
+# ---------------------------------------------------------------- helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle sampling in the background (read-only queries)."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: torch.device):
+        try:
+            self.dev = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            self.dev = str(device.index or 0)
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = max((float(r[2]) for r in rows if r[2].replace(".", "").isdigit()), default=None)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        loaded = [x for x in sm if smax and x > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": smax,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def cpu_info():
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return model, len(os.sched_getaffinity(0))
+
+
+# ---------------------------------------------------------------- oracle timing
+def oracle_forward_sample(w, budget_s: float):
+    """Float64 oracle on a bounded prefix of the forward workload (all heads of batch row 0,
+    the first T' tokens), sized from a short calibration run to take about `budget_s`.
+    Returns (tokens/s, cores, description)."""
+    import oracle
+    _, cores = cpu_info()
+    threads = min(cores, w.B * w.H)
+
+    def run(Tp):
+        inp = forward_inputs(1, Tp, w.H, w.dk, w.dv, w.dtype, seed=w.seed, alpha_mu=w.alpha_mu)
+        args = [as_f32_numpy(inp[n]) for n in ("q", "k", "v", "log_alpha", "beta")]
+        t0 = time.perf_counter()
+        oracle.forward(*args, None, nthreads=threads)
+        return time.perf_counter() - t0
+
+    probe = 128
+    dt = max(run(probe), 1e-4)
+    Tp = int(max(probe, min(w.T, probe * budget_s / dt)))
+    dt = run(Tp)
+    return Tp / dt, threads, "oracle float64, batch row 0 of %s: H=%d, first %d of %d tokens, %d threads" % (
+        w.name, w.H, Tp, w.T, threads), Tp, dt
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    w = WORKLOADS[FWD_WORKLOAD]
+    model, cores = cpu_info()
+    for _ in range(args.warmup):
+        oracle_forward_sample(w, 0.5)
+    times, toks = [], []
+    for _ in range(args.steps):
+        tps, threads, desc, Tp, dt = oracle_forward_sample(w, args.ref_step_seconds)
+        times.append(dt)
+        toks.append(Tp)
+    value = sum(toks) / sum(times)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * statistics.mean(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
+                   "input_dtype": w.dtype, "parallelism": "replicas"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": desc + "; CPU: " + model},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+def time_region(fn, steps, stream, world):
+    barrier(world)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return start.elapsed_time(end)  # ms
+
+
+def run_gdn(args, world, rank, local):
+    import gated_delta_rule_142_b200 as gdn
+    from gated_delta_rule_142_b200 import build as gdn_build
+    if not os.path.exists(gdn.LIBRARY):
+        gdn_build.build()
+    gdn.load()
+    peaks, peak_kind = load_peaks()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    sampler = ClockSampler(dev)
+    sampler.start()
+
+    # ---- forward, inputs resident in HBM ----
+    w = WORKLOADS[FWD_WORKLOAD]
+    es = 2 if w.dtype == "bf16" else 4
+    inp = forward_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, seed=w.seed + 1000 * rank, s0_std=w.s0_std,
+                         alpha_mu=w.alpha_mu)
+    d = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}
+    out = torch.empty((w.B, w.T, w.H, w.dv), dtype=d["q"].dtype, device=dev)
+    Sf = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=dev)
+
+    def fwd_step():
+        gdn.forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"], chunk=w.chunk, out=out,
+                    S_final=Sf, stream=stream)
+
+    for _ in range(args.warmup):
+        fwd_step()
+    ms = time_region(fwd_step, args.steps, stream, world)
+    ms_step = max_over_ranks(ms / args.steps, world)
+    tokens = w.B * w.T
+    value = world * tokens / (ms_step / 1e3)
+    flop = w.B * w.T * w.H * fwd_flop_per_token_head(w.dk, w.dv, w.chunk)
+    nbytes = fwd_bytes(w.B, w.T, w.H, w.dk, w.dv, es, w.s0_std is not None, True)
+    tflops = flop / (ms_step / 1e3) / 1e12
+    gbs = nbytes / (ms_step / 1e3) / 1e9
+    launches_per_fwd = 1
+
+    # ---- decode: 1024 consecutive single-token steps, each its own launch ----
+    dec = None
+    if not args.no_decode:
+        wd = WORKLOADS[DEC_WORKLOAD]
+        dsteps = wd.steps
+        di = decode_inputs(dsteps, wd.B, wd.H, wd.dk, wd.dv, wd.dtype, seed=wd.seed + 1000 * rank,
+                           s0_std=wd.s0_std)
+        dd = {k: v.to(dev) for k, v in di.items()}
+        S = dd["S"].clone()
+        dout = torch.empty((dsteps, wd.B, wd.H, wd.dv), dtype=dd["q"].dtype, device=dev)
+
+        def dec_run():
+            for t in range(dsteps):
+                gdn.decode_step(dd["q"][t], dd["k"][t], dd["v"][t], dd["log_alpha"][t], dd["beta"][t], S,
+                                out=dout[t], stream=stream)
+
+        for _ in range(max(1, args.warmup // 3)):
+            dec_run()
+        dms = time_region(dec_run, 1, stream, world) / dsteps
+        dms = max_over_ranks(dms, world)
+        des = 2 if wd.dtype == "bf16" else 4
+        dbytes = wd.B * wd.H * decode_bytes_per_head_step(wd.dk, wd.dv, des)
+        dgbs = dbytes / (dms / 1e3) / 1e9
+        dec = {"workload": wd.name, "steps": dsteps, "us_per_step": dms * 1e3,
+               "tokens_per_s": world * wd.B / (dms / 1e3), "GB_per_s": dgbs,
+               "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                            "frac": dgbs / peaks["hbm_gbs"], "traffic": None,
+                            "peak_kind": peak_kind, "bytes_per_launch": dbytes},
+               "launches": dsteps}
+        del dd, S, dout
+    clocks = sampler.stop()
+
+    # ---- e2e: same forward through the C ABI with pinned host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        h = {k: (None if v is None else v.pin_memory()) for k, v in inp.items()}
+        hout = torch.empty((w.B, w.T, w.H, w.dv), dtype=h["q"].dtype).pin_memory()
+        hSf = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            gdn.forward(h["q"], h["k"], h["v"], h["log_alpha"], h["beta"], h["S0"], chunk=w.chunk, out=hout,
+                        S_final=hSf, stream=stream)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        ke = max(1, min(args.steps, 10))
+        ems = max_over_ranks(time_region(e2e_step, ke, stream, world) / ke, world)
+        h2d = sum(t.numel() * t.element_size() for k, t in h.items() if t is not None)
+        d2h = hout.numel() * hout.element_size() + hSf.numel() * hSf.element_size()
+        e2e = {"value": world * tokens / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": ke}
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only) ----
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        model, _ = cpu_info()
+        tps, threads, desc, _, _ = oracle_forward_sample(w, args.cpu_seconds)
+        cpu = {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc + "; CPU: " + model}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
+                       "input_dtype": w.dtype, "state_dtype": "f32", "parallelism": "replicas" if world > 1 else "single",
+                       "l2": "inputs larger than L2 (%.2f GB read+written per step)" % (nbytes / 1e9)},
+            "tflops": tflops, "gb_per_s": gbs,
+            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": tflops / peaks["bf16_tflops"], "traffic": None, "peak_kind": peak_kind,
+                         "flop_per_launch": flop, "hbm_frac": gbs / peaks["hbm_gbs"]},
+            "decode": dec, "e2e": e2e, "cpu_baseline": cpu, "clocks": clocks,
+            "gpu_launches": args.steps * launches_per_fwd,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["gdn", "reference"], default="gdn")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=8.0)
+    args = ap.parse_args()
+    if args.impl == "reference":
+        # CPU oracle arm: rank 0 alone runs and prints; other ranks exit without work.
+        return run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
+    world, rank, local = dist_setup()
+    try:
+        return run_gdn(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,171 @@
+"""Gated delta rule on NVIDIA B200 (sm_100a): Python binding of libgdn.so.
+
+This module only marshals arguments: it reads shapes and data pointers from
+torch tensors and calls the C ABI declared in ``include/gdn.h``.  Every step
+of the computation runs in the library's CUDA kernels; there is no Python or
+CPU fallback, and importing the binding fails loudly when ``libgdn.so`` has
+not been built (``python -m gated_delta_rule_142_b200.build``).
+
+The operation ("ATMA: Long-Context Language Modeling via Polar Attention and
+Gated-Delta Compression Memory", Sec. 3.3), per (batch, head):
+
+    S_t = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,   o_t = S_t q_t,
+    alpha_t = exp(log_alpha_t).
+
+Tensors may live on the current CUDA device (used in place) or on the host
+(staged by the library through stream-ordered device buffers).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIBRARY = os.path.join(_PKG, "libgdn.so")
+
+GDN_F32 = 0
+GDN_BF16 = 1
+
+STATUS = {
+    0: "GDN_OK", 1: "GDN_ERR_NULL_PTR", 2: "GDN_ERR_INVALID_SIZE", 3: "GDN_ERR_UNSUPPORTED",
+    4: "GDN_ERR_MISALIGNED", 5: "GDN_ERR_ALLOC", 6: "GDN_ERR_LAUNCH", 7: "GDN_ERR_DEVICE_TIMEOUT",
+    8: "GDN_ERR_ALIAS", 9: "GDN_ERR_DEVICE",
+}
+
+EXPORTS = ("gdn_forward", "gdn_decode_step", "gdn_status_string", "gdn_version")
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__("%s: %s (%s)" % (where, STATUS.get(status, status), status_string(status)))
+
+
+_lib = None
+
+
+def load(path: str = LIBRARY) -> ctypes.CDLL:
+    """Load libgdn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError("libgdn.so not found at %s: build it with "
+                           "`python -m gated_delta_rule_142_b200.build`" % path)
+    lib = ctypes.CDLL(path)
+    vp, i64 = ctypes.c_void_p, ctypes.c_int64
+    lib.gdn_forward.argtypes = [vp] * 8 + [i64] * 6 + [vp, ctypes.c_int]
+    lib.gdn_forward.restype = ctypes.c_int
+    lib.gdn_decode_step.argtypes = [vp] * 7 + [i64] * 4 + [vp, ctypes.c_int]
+    lib.gdn_decode_step.restype = ctypes.c_int
+    lib.gdn_status_string.argtypes = [ctypes.c_int]
+    lib.gdn_status_string.restype = ctypes.c_char_p
+    lib.gdn_version.argtypes = []
+    lib.gdn_version.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().gdn_status_string(int(status)).decode()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return GDN_F32
+    if t.dtype == torch.bfloat16:
+        return GDN_BF16
+    raise TypeError("q/k/v must be float32 or bfloat16, got %s" % t.dtype)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr()) if t.numel() > 0 else None
+
+
+def _pinned(t: torch.Tensor) -> bool:
+    return t.device.type == "cpu" and torch.cuda.is_available() and t.is_pinned()
+
+
+def _stream_handle(device: torch.device, stream) -> ctypes.c_void_p:
+    if stream is None:
+        if device.type == "cuda":
+            stream = torch.cuda.current_stream(device)
+        else:
+            stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
+            beta: torch.Tensor, S0: Optional[torch.Tensor] = None, chunk: int = 64,
+            out: Optional[torch.Tensor] = None, S_final: Optional[torch.Tensor] = None,
+            output_final_state: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunkwise forward.  q, k [B,T,H,dk], v [B,T,H,dv] (float32 or bfloat16, same dtype);
+    log_alpha, beta [B,T,H] float32; S0 [B,H,dv,dk] float32 or None.
+    Returns (out [B,T,H,dv] in the input dtype, S_final [B,H,dv,dk] float32 or None)."""
+    lib = load()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for name, t, shape in (("k", k, (B, T, H, dk)), ("v", v, (B, T, H, dv)), ("log_alpha", log_alpha, (B, T, H)),
+                           ("beta", beta, (B, T, H)), ("out", out, (B, T, H, dv))):
+        if t is not None and tuple(t.shape) != shape:
+            raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), shape))
+    _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype or (out is not None and out.dtype != q.dtype):
+        raise TypeError("q, k, v and out must share one dtype")
+    for name, t in (("log_alpha", log_alpha), ("beta", beta), ("S0", S0), ("S_final", S_final)):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError("%s must be float32" % name)
+    for name, t in (("S0", S0), ("S_final", S_final)):
+        if t is not None and tuple(t.shape) != (B, H, dv, dk):
+            raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), (B, H, dv, dk)))
+    for t in (q, k, v, log_alpha, beta, S0, out, S_final):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device, pin_memory=_pinned(q))
+    if S_final is None and output_final_state:
+        S_final = torch.empty((B, H, dv, dk), dtype=torch.float32, device=q.device, pin_memory=_pinned(q))
+    with torch.cuda.device(q.device if q.device.type == "cuda" else torch.cuda.current_device()):
+        st = lib.gdn_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(out),
+                             _ptr(S_final), B, T, H, dk, dv, int(chunk), _stream_handle(q.device, stream),
+                             _dtype_code(q))
+    if st != 0:
+        raise GdnError(st, "gdn_forward")
+    return out, S_final
+
+
+def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
+                beta: torch.Tensor, S: torch.Tensor, out: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+    """One token for every (b, h).  q, k [B,H,dk]; v [B,H,dv]; log_alpha, beta [B,H] float32;
+    S [B,H,dv,dk] float32 is updated in place.  Returns out [B,H,dv]."""
+    lib = load()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    for name, t, shape in (("k", k, (B, H, dk)), ("v", v, (B, H, dv)), ("log_alpha", log_alpha, (B, H)),
+                           ("beta", beta, (B, H)), ("S", S, (B, H, dv, dk)), ("out", out, (B, H, dv))):
+        if t is not None and tuple(t.shape) != shape:
+            raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), shape))
+    _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype or (out is not None and out.dtype != q.dtype):
+        raise TypeError("q, k, v and out must share one dtype")
+    if S.dtype != torch.float32 or log_alpha.dtype != torch.float32 or beta.dtype != torch.float32:
+        raise TypeError("S, log_alpha and beta must be float32")
+    for t in (q, k, v, log_alpha, beta, S, out):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=q.dtype, device=q.device, pin_memory=_pinned(q))
+    with torch.cuda.device(q.device if q.device.type == "cuda" else torch.cuda.current_device()):
+        st = lib.gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S), _ptr(out),
+                                 B, H, dk, dv, _stream_handle(q.device, stream), _dtype_code(q))
+    if st != 0:
+        raise GdnError(st, "gdn_decode_step")
+    return out

@@ -1,0 +1,121 @@
+// decode.cu -- single-token gated-delta step, state updated in place.
+//
+// Operation ("ATMA: Long-Context Language Modeling via Polar Attention and
+// Gated-Delta Compression Memory", Sec. 3.3, gated-delta memory equation),
+// per (b, h) and per row r of the d_v x d_k state:
+//     a_r = S_r . k,  b_r = S_r . q
+//     u_r = beta (v_r - alpha a_r)
+//     S_r <- alpha S_r + u_r k^T
+//     o_r = S'_r . q = alpha b_r + u_r (k . q)
+// which is the equation's S (I - beta k k^T) alpha + beta v k^T written row by
+// row.  The step is bound by HBM: each state row (dk float32) is read once
+// with 128-bit loads and written once; everything else is a few bytes.
+//
+// Mapping: a row is held by DK/4 consecutive lanes, four columns per lane
+// (one float4).  A warp covers 32/(DK/4) rows per step and each thread keeps
+// kUnroll rows in flight, so a CTA of 4 warps owns 4 * (32/(DK/4)) * kUnroll
+// rows of one head (32 rows at dk = 128).  Grid: (B*H) x ceil(dv / rows).
+#include "common.cuh"
+#include "gdn_internal.h"
+
+namespace gdn {
+namespace {
+
+constexpr int kDecodeThreads = 128;
+constexpr int kUnroll = 8;
+
+template <int DK>
+constexpr int decode_rows_per_cta() {
+    return (kDecodeThreads / 32) * (32 / (DK / 4)) * kUnroll;
+}
+
+template <typename Tin, int DK>
+__global__ void __launch_bounds__(kDecodeThreads)
+decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
+              const float *__restrict__ log_alpha, const float *__restrict__ beta,
+              float *__restrict__ S, Tin *__restrict__ out, int dv) {
+    constexpr int LPR = DK / 4;          // lanes per row
+    constexpr int RPW = 32 / LPR;        // rows per warp per step
+    constexpr int STRIDE = (kDecodeThreads / 32) * RPW;
+    const int64_t head = blockIdx.x;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int grp = lane / LPR, gl = lane % LPR;
+    const int row_base = blockIdx.y * decode_rows_per_cta<DK>() + warp * RPW + grp;
+
+    const float4 kf = load4(k + head * DK + 4 * gl);
+    const float4 qf = load4(q + head * DK + 4 * gl);
+    const float alpha = expf(log_alpha[head]);
+    const float bt = beta[head];
+    const float kq = group_sum<LPR>(dot4(kf, qf));
+
+    float *Sh = S + head * (int64_t)dv * DK;
+    float4 s[kUnroll];
+    float vr[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int r = row_base + u * STRIDE;
+        if (r < dv) {
+            s[u] = *reinterpret_cast<const float4 *>(Sh + (int64_t)r * DK + 4 * gl);
+            vr[u] = to_f32(v[head * dv + r]);
+        } else {
+            s[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            vr[u] = 0.f;
+        }
+    }
+    float a[kUnroll], b[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        a[u] = dot4(s[u], kf);
+        b[u] = dot4(s[u], qf);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        a[u] = group_sum<LPR>(a[u]);
+        b[u] = group_sum<LPR>(b[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int r = row_base + u * STRIDE;
+        if (r < dv) {
+            const float ur = bt * (vr[u] - alpha * a[u]);
+            float4 n;
+            n.x = fmaf(alpha, s[u].x, ur * kf.x);
+            n.y = fmaf(alpha, s[u].y, ur * kf.y);
+            n.z = fmaf(alpha, s[u].z, ur * kf.z);
+            n.w = fmaf(alpha, s[u].w, ur * kf.w);
+            *reinterpret_cast<float4 *>(Sh + (int64_t)r * DK + 4 * gl) = n;
+            if (gl == 0) out[head * dv + r] = from_f32<Tin>(fmaf(alpha, b[u], ur * kq));
+        }
+    }
+}
+
+template <typename Tin, int DK>
+cudaError_t launch_decode_t(const DecodeProblem &p, cudaStream_t stream) {
+    const int rows = decode_rows_per_cta<DK>();
+    dim3 grid((unsigned)(p.B * p.H), (unsigned)((p.dv + rows - 1) / rows));
+    decode_kernel<Tin, DK><<<grid, kDecodeThreads, 0, stream>>>(
+        static_cast<const Tin *>(p.q), static_cast<const Tin *>(p.k), static_cast<const Tin *>(p.v),
+        p.log_alpha, p.beta, p.S, static_cast<Tin *>(p.out), (int)p.dv);
+    return cudaGetLastError();
+}
+
+template <typename Tin>
+cudaError_t launch_decode_dtype(const DecodeProblem &p, cudaStream_t stream) {
+    switch (p.dk) {
+        case 16: return launch_decode_t<Tin, 16>(p, stream);
+        case 32: return launch_decode_t<Tin, 32>(p, stream);
+        case 64: return launch_decode_t<Tin, 64>(p, stream);
+        case 128: return launch_decode_t<Tin, 128>(p, stream);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeProblem &p, cudaStream_t stream) {
+    if (p.B * p.H == 0) return cudaSuccess;
+    if (p.dtype == 0) return launch_decode_dtype<float>(p, stream);
+    return launch_decode_dtype<__nv_bfloat16>(p, stream);
+}
+
+}  // namespace gdn

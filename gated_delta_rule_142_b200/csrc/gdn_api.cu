@@ -1,0 +1,275 @@
+// gdn_api.cu -- the C ABI declared in include/gdn.h: argument validation,
+// host-buffer staging and dispatch to the kernels.  No arithmetic of the
+// recurrence happens here; every step of it runs in the CUDA kernels.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "gdn.h"
+#include "gdn_internal.h"
+
+namespace {
+
+using gdn::DecodeProblem;
+using gdn::FwdProblem;
+
+// ---------------------------------------------------------------- device info
+struct DeviceInfo {
+    int sm_count = 0;
+    int major = 0;
+};
+
+// Immutable per-device properties, filled on first use (benign race: every
+// writer stores the same values).
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+std::atomic<int> g_major[kMaxDevices];
+
+int device_info(DeviceInfo *info) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+        cudaGetLastError();
+        return GDN_ERR_DEVICE;
+    }
+    if (dev < kMaxDevices && g_sm_count[dev].load(std::memory_order_relaxed) > 0) {
+        info->sm_count = g_sm_count[dev].load(std::memory_order_relaxed);
+        info->major = g_major[dev].load(std::memory_order_relaxed);
+    } else {
+        int sms = 0, major = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+            cudaGetLastError();
+            return GDN_ERR_DEVICE;
+        }
+        info->sm_count = sms;
+        info->major = major;
+        if (dev < kMaxDevices) {
+            g_major[dev].store(major, std::memory_order_relaxed);
+            g_sm_count[dev].store(sms, std::memory_order_relaxed);
+        }
+    }
+    // The kernels are built for sm_100a only.
+    if (info->major != 10) return GDN_ERR_DEVICE;
+    return GDN_OK;
+}
+
+// ---------------------------------------------------------------- validation
+bool supported_dim(int64_t d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool supported_chunk(int64_t c) { return c == 16 || c == 32 || c == 64; }
+bool aligned16(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool mul3(int64_t a, int64_t b, int64_t c, int64_t *r) {
+    int64_t t;
+    return !__builtin_mul_overflow(a, b, &t) && !__builtin_mul_overflow(t, c, r);
+}
+
+struct Span {
+    uintptr_t lo = 0, hi = 0;  // [lo, hi); empty when lo == hi
+    Span() = default;
+    Span(const void *p, int64_t bytes) {
+        if (p && bytes > 0) {
+            lo = reinterpret_cast<uintptr_t>(p);
+            hi = lo + (uintptr_t)bytes;
+        }
+    }
+    bool empty() const { return lo == hi; }
+};
+bool overlaps(const Span &a, const Span &b) { return !a.empty() && !b.empty() && a.lo < b.hi && b.lo < a.hi; }
+
+// ---------------------------------------------------------------- staging
+bool is_device_pointer(const void *p) {
+    cudaPointerAttributes attr;
+    if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged;
+}
+
+// Stream-ordered device copies of host buffers, released on the same stream.
+struct Stager {
+    cudaStream_t stream;
+    void *bufs[10];
+    int n = 0;
+    explicit Stager(cudaStream_t s) : stream(s) {}
+    ~Stager() {
+        for (int i = 0; i < n; ++i) cudaFreeAsync(bufs[i], stream);
+    }
+    // Returns a device pointer for p (p itself when it is device memory).
+    int in(const void *p, int64_t bytes, bool copy, const void **dev) {
+        if (p == nullptr || bytes <= 0 || is_device_pointer(p)) {
+            *dev = p;
+            return GDN_OK;
+        }
+        void *d = nullptr;
+        if (cudaMallocAsync(&d, (size_t)bytes, stream) != cudaSuccess) {
+            cudaGetLastError();
+            return GDN_ERR_ALLOC;
+        }
+        bufs[n++] = d;
+        if (copy && cudaMemcpyAsync(d, p, (size_t)bytes, cudaMemcpyDefault, stream) != cudaSuccess) {
+            cudaGetLastError();
+            return GDN_ERR_LAUNCH;
+        }
+        *dev = d;
+        return GDN_OK;
+    }
+    int out_back(void *host, const void *dev, int64_t bytes) {
+        if (host == nullptr || host == dev || bytes <= 0) return GDN_OK;
+        if (cudaMemcpyAsync(host, dev, (size_t)bytes, cudaMemcpyDefault, stream) != cudaSuccess) {
+            cudaGetLastError();
+            return GDN_ERR_LAUNCH;
+        }
+        return GDN_OK;
+    }
+};
+
+enum class FwdPath { Auto, Simt };
+
+FwdPath forced_path() {
+    const char *e = getenv("GDN_FORWARD_PATH");
+    if (e && strcmp(e, "simt") == 0) return FwdPath::Simt;
+    return FwdPath::Auto;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *gdn_status_string(int status) {
+    switch (status) {
+        case GDN_OK: return "ok";
+        case GDN_ERR_NULL_PTR: return "a required pointer is NULL";
+        case GDN_ERR_INVALID_SIZE: return "invalid size (negative, or the element count overflows int64)";
+        case GDN_ERR_UNSUPPORTED: return "unsupported dk/dv (16, 32, 64, 128), chunk (16, 32, 64) or dtype";
+        case GDN_ERR_MISALIGNED: return "a pointer is not 16-byte aligned";
+        case GDN_ERR_ALLOC: return "stream-ordered device allocation failed";
+        case GDN_ERR_LAUNCH: return "kernel launch or enqueued copy failed";
+        case GDN_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
+        case GDN_ERR_ALIAS: return "an output buffer overlaps an input it must not overlap";
+        case GDN_ERR_DEVICE: return "no usable sm_100 CUDA device is current";
+        default: return "unknown gdn status";
+    }
+}
+
+int gdn_version(void) { return 100; }  // 0.1.0
+
+int gdn_forward(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                const float *S0, void *out, float *S_final, int64_t B, int64_t T, int64_t H, int64_t dk,
+                int64_t dv, int64_t chunk, void *stream_, int dtype) {
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
+    if (B < 0 || T < 0 || H < 0 || dk < 0 || dv < 0 || chunk < 0) return GDN_ERR_INVALID_SIZE;
+    if (!supported_dim(dk) || !supported_dim(dv) || !supported_chunk(chunk)) return GDN_ERR_UNSUPPORTED;
+    const int64_t es = (dtype == GDN_F32) ? 4 : 2;
+    int64_t ntok, nqk, nv, nstate;
+    if (!mul3(B, T, H, &ntok) || !mul3(ntok, dk, es, &nqk) || !mul3(ntok, dv, es, &nv) ||
+        !mul3(B * H, dv, dk * 4, &nstate) || ntok > (INT64_MAX / 8))
+        return GDN_ERR_INVALID_SIZE;
+    if (B * H == 0) return GDN_OK;
+    if (ntok > 0 && (!q || !k || !v || !log_alpha || !beta || !out)) return GDN_ERR_NULL_PTR;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) || !aligned16(beta) ||
+        !aligned16(S0) || !aligned16(out) || !aligned16(S_final))
+        return GDN_ERR_MISALIGNED;
+    const Span sq(q, nqk), sk(k, nqk), sv(v, nv), sla(log_alpha, ntok * 4), sbe(beta, ntok * 4);
+    const Span s0(S0, nstate), sf(S_final, nstate), so(out, nv);
+    const Span inputs[] = {sq, sk, sv, sla, sbe, s0, sf};
+    for (const Span &x : inputs)
+        if (overlaps(so, x)) return GDN_ERR_ALIAS;
+    if (overlaps(sf, s0) && !(sf.lo == s0.lo)) return GDN_ERR_ALIAS;
+    for (const Span &x : {sq, sk, sv, sla, sbe})
+        if (overlaps(sf, x)) return GDN_ERR_ALIAS;
+
+    DeviceInfo info;
+    if (int st = device_info(&info)) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+
+    Stager stg(stream);
+    FwdProblem p;
+    int st = GDN_OK;
+    const void *dS0 = nullptr;
+    if ((st = stg.in(q, nqk, true, &p.q)) || (st = stg.in(k, nqk, true, &p.k)) || (st = stg.in(v, nv, true, &p.v)) ||
+        (st = stg.in(log_alpha, ntok * 4, true, reinterpret_cast<const void **>(&p.log_alpha))) ||
+        (st = stg.in(beta, ntok * 4, true, reinterpret_cast<const void **>(&p.beta))) ||
+        (st = stg.in(S0, nstate, true, &dS0)))
+        return st;
+    p.S0 = static_cast<const float *>(dS0);
+    const void *dout = nullptr, *dSf = nullptr;
+    if ((st = stg.in(out, nv, false, &dout))) return st;
+    if (S_final && S_final == S0) {
+        dSf = dS0;
+    } else if ((st = stg.in(S_final, nstate, false, &dSf))) {
+        return st;
+    }
+    p.out = const_cast<void *>(dout);
+    p.S_final = static_cast<float *>(const_cast<void *>(dSf));
+    p.B = B; p.T = T; p.H = H; p.dk = dk; p.dv = dv; p.chunk = chunk; p.dtype = dtype;
+
+    cudaError_t e = cudaSuccess;
+    if (T == 0) {
+        if (p.S_final && p.S_final != p.S0) {
+            e = p.S0 ? cudaMemcpyAsync(p.S_final, p.S0, (size_t)nstate, cudaMemcpyDeviceToDevice, stream)
+                     : cudaMemsetAsync(p.S_final, 0, (size_t)nstate, stream);
+        }
+    } else {
+        (void)forced_path();
+        e = gdn::launch_fwd_simt(p, info.sm_count, stream);
+    }
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_LAUNCH;
+    }
+    if ((st = stg.out_back(out, p.out, nv))) return st;
+    if ((st = stg.out_back(S_final, p.S_final, nstate))) return st;
+    return GDN_OK;
+}
+
+int gdn_decode_step(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                    float *S, void *out, int64_t B, int64_t H, int64_t dk, int64_t dv, void *stream_, int dtype) {
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
+    if (B < 0 || H < 0 || dk < 0 || dv < 0) return GDN_ERR_INVALID_SIZE;
+    if (!supported_dim(dk) || !supported_dim(dv)) return GDN_ERR_UNSUPPORTED;
+    const int64_t es = (dtype == GDN_F32) ? 4 : 2;
+    int64_t nh, nqk, nv, nstate;
+    if (__builtin_mul_overflow(B, H, &nh) || !mul3(nh, dk, es, &nqk) || !mul3(nh, dv, es, &nv) ||
+        !mul3(nh, dv, dk * 4, &nstate) || nh > (int64_t)INT32_MAX)
+        return GDN_ERR_INVALID_SIZE;
+    if (nh == 0) return GDN_OK;
+    if (!q || !k || !v || !log_alpha || !beta || !S || !out) return GDN_ERR_NULL_PTR;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) || !aligned16(beta) ||
+        !aligned16(S) || !aligned16(out))
+        return GDN_ERR_MISALIGNED;
+    const Span sq(q, nqk), sk(k, nqk), sv(v, nv), sla(log_alpha, nh * 4), sbe(beta, nh * 4);
+    const Span ss(S, nstate), so(out, nv);
+    for (const Span &x : {sq, sk, sv, sla, sbe, ss})
+        if (overlaps(so, x)) return GDN_ERR_ALIAS;
+    for (const Span &x : {sq, sk, sv, sla, sbe})
+        if (overlaps(ss, x)) return GDN_ERR_ALIAS;
+
+    DeviceInfo info;
+    if (int st = device_info(&info)) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    Stager stg(stream);
+    DecodeProblem p;
+    int st = GDN_OK;
+    const void *dS = nullptr, *dout = nullptr;
+    if ((st = stg.in(q, nqk, true, &p.q)) || (st = stg.in(k, nqk, true, &p.k)) || (st = stg.in(v, nv, true, &p.v)) ||
+        (st = stg.in(log_alpha, nh * 4, true, reinterpret_cast<const void **>(&p.log_alpha))) ||
+        (st = stg.in(beta, nh * 4, true, reinterpret_cast<const void **>(&p.beta))) ||
+        (st = stg.in(S, nstate, true, &dS)) || (st = stg.in(out, nv, false, &dout)))
+        return st;
+    p.S = static_cast<float *>(const_cast<void *>(dS));
+    p.out = const_cast<void *>(dout);
+    p.B = B; p.H = H; p.dk = dk; p.dv = dv; p.dtype = dtype;
+    if (gdn::launch_decode(p, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_LAUNCH;
+    }
+    if ((st = stg.out_back(out, p.out, nv))) return st;
+    if ((st = stg.out_back(S, p.S, nstate))) return st;
+    return GDN_OK;
+}
+
+}  // extern "C"

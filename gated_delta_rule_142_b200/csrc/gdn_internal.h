@@ -1,0 +1,39 @@
+// gdn_internal.h -- kernel launchers shared by the C-ABI host code (gdn_api.cu).
+// Not part of the public interface; see include/gdn.h for the operation and layouts.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gdn {
+
+// Floor applied to log_alpha inside the chunkwise forward: exp(-40) < 5e-18,
+// below float32 resolution of a state next to O(1) terms, and chunk-local
+// log-decay sums stay small enough for float32 differences g_t - g_s.
+constexpr float kLogAlphaFloor = -40.0f;
+
+struct FwdProblem {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta, *S0;
+    void *out;
+    float *S_final;
+    int64_t B, T, H, dk, dv, chunk;
+    int dtype;  // gdn_dtype
+};
+
+struct DecodeProblem {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta;
+    float *S;
+    void *out;
+    int64_t B, H, dk, dv;
+    int dtype;
+};
+
+// decode.cu
+cudaError_t launch_decode(const DecodeProblem &p, cudaStream_t stream);
+
+// fwd_simt.cu -- float32 SIMT chunkwise forward, any supported (dk, dv, chunk).
+cudaError_t launch_fwd_simt(const FwdProblem &p, int sm_count, cudaStream_t stream);
+
+}  // namespace gdn

@@ -1,0 +1,136 @@
+/*
+ * gdn.h -- C ABI of the B200 gated-delta-rule library (libgdn.so).
+ *
+ * The operation (source: "ATMA: Long-Context Language Modeling via Polar
+ * Attention and Gated-Delta Compression Memory", Sec. 3.3, the gated-delta
+ * memory equation, with the paper's gamma_t written alpha_t, M written S and
+ * r written o).  For every batch row b and head h independently, with a
+ * d_v x d_k float32 state S:
+ *
+ *     alpha_t = exp(log_alpha_t)
+ *     S_t     = alpha_t S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T
+ *     o_t     = S_t q_t                      (the output uses the updated state)
+ *
+ * No scale is applied to q, and q, k are used as given: callers that want
+ * the paper's unit-norm keys and queries (its App. A.2 assumes
+ * ||q_t|| = ||k_t|| = 1) normalise them before the call.
+ *
+ * Layouts (row-major, contiguous, 64-bit indexing):
+ *     q, k            [B, T, H, dk]   dtype (GDN_F32 or GDN_BF16)
+ *     v, out          [B, T, H, dv]   dtype
+ *     log_alpha, beta [B, T, H]       float32, always
+ *     S0, S_final, S  [B, H, dv, dk]  float32, always (row = value index,
+ *                                     column = key index; k contiguous)
+ * For gdn_decode_step the T axis is absent: q, k [B, H, dk], v, out [B, H, dv],
+ * log_alpha, beta [B, H].
+ *
+ * Memory: every pointer may be device memory (cudaMalloc, stream-ordered or
+ * managed) or host memory (pinned or pageable).  Device memory is used in
+ * place.  Host buffers are staged through stream-ordered device buffers:
+ * host-to-device copies are enqueued on `stream` before the kernels and
+ * device-to-host copies of the results after them; with pinned host output
+ * memory the results are valid after the stream has been synchronised,
+ * with pageable host output memory they are valid when the call returns.
+ * The library keeps no pointer after a call returns and owns no buffer.
+ *
+ * Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ * stream).  All device work of a call is enqueued on it; calls are
+ * asynchronous unless host staging forces a synchronous copy.  The library
+ * holds no global mutable state, so calls on different streams may run
+ * concurrently provided their buffers do not overlap.
+ *
+ * Errors: every entry point returns a gdn_status.  Arguments are validated
+ * on the host before anything is enqueued; a rejected call enqueues nothing
+ * and writes nothing.  A failed kernel launch returns GDN_ERR_LAUNCH.  Device
+ * code never traps; errors raised asynchronously by the device appear at the
+ * caller's next synchronisation, as for any CUDA work.
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element type of q, k, v and out.  Gates and states are always float32. */
+typedef enum {
+    GDN_F32 = 0,  /* float32: arithmetic in float32 (SIMT), for tight parity   */
+    GDN_BF16 = 1  /* bfloat16: tensor-core operands, float32 accumulation/state */
+} gdn_dtype;
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_NULL_PTR = 1,       /* a required pointer is NULL                          */
+    GDN_ERR_INVALID_SIZE = 2,   /* negative size, or sizes whose product overflows     */
+    GDN_ERR_UNSUPPORTED = 3,    /* dk, dv, chunk or dtype outside the supported set    */
+    GDN_ERR_MISALIGNED = 4,     /* a pointer is not 16-byte aligned                    */
+    GDN_ERR_ALLOC = 5,          /* stream-ordered workspace/staging allocation failed  */
+    GDN_ERR_LAUNCH = 6,         /* a kernel launch or an enqueued copy failed          */
+    GDN_ERR_DEVICE_TIMEOUT = 7, /* a bounded device-side wait gave up                  */
+    GDN_ERR_ALIAS = 8,          /* an output overlaps an input it must not overlap     */
+    GDN_ERR_DEVICE = 9          /* no usable CUDA device / not an sm_100 device        */
+} gdn_status;
+
+/*
+ * gdn_forward -- prefill / training forward over T tokens.
+ *
+ * Computes o_t for t = 1..T and, if S_final != NULL, S_T, starting from S0
+ * (S0 == NULL means the zero state).  Chunkwise-parallel: the sequence is cut
+ * into chunks of `chunk` tokens; inside a chunk the recurrence is solved in
+ * closed form (a unit-lower-triangular UT transform), and the state is passed
+ * from chunk to chunk.  The result does not depend on `chunk` beyond
+ * rounding.  T need not be a multiple of `chunk`.
+ *
+ * Arguments:
+ *   q, k, v, out   see layouts above; dtype given by `dtype`
+ *   log_alpha      log of the decay gate; alpha = exp(log_alpha) in [0, 1].
+ *                  -inf (alpha = 0) is accepted; values below -40 act as -40
+ *                  (alpha < 5e-18, below float32 resolution of the state)
+ *   beta           write strength, used as given (the paper takes [0, 1])
+ *   S0             initial state or NULL.  May equal S_final (in place)
+ *   S_final        final state or NULL (not written)
+ *   B, T, H        batch, tokens, heads.  B == 0, H == 0 or T == 0 are
+ *                  valid: with T == 0, S_final receives S0 (or zeros)
+ *   dk, dv         key / value head dims, each one of 16, 32, 64, 128
+ *   chunk          16, 32 or 64
+ *   stream         cudaStream_t
+ *   dtype          gdn_dtype of q, k, v, out
+ *
+ * Aliasing: out must not overlap q, k, v, gates, S0 or S_final; S_final
+ * must not partially overlap S0 (exact equality is allowed).
+ * Alignment: all non-NULL pointers 16-byte aligned.
+ */
+int gdn_forward(const void *q, const void *k, const void *v, const float *log_alpha,
+                const float *beta, const float *S0, void *out, float *S_final, int64_t B,
+                int64_t T, int64_t H, int64_t dk, int64_t dv, int64_t chunk, void *stream,
+                int dtype);
+
+/*
+ * gdn_decode_step -- one token for every (b, h), state updated in place.
+ *
+ * Same equation as gdn_forward with T = 1 (source: the Sec. 3.3 gated-delta
+ * memory equation): reads S, writes S_1 back into S and o_1 into out.  Each
+ * head's state is streamed from memory once and written back once.
+ *
+ * Arguments: q, k [B, H, dk]; v, out [B, H, dv]; log_alpha, beta [B, H]
+ * float32; S [B, H, dv, dk] float32, read and overwritten; dk, dv each one
+ * of 16, 32, 64, 128; dtype of q, k, v, out.  B == 0 or H == 0 is a no-op.
+ * Aliasing: out must not overlap any input or S.
+ */
+int gdn_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
+                    const float *beta, float *S, void *out, int64_t B, int64_t H, int64_t dk,
+                    int64_t dv, void *stream, int dtype);
+
+/* Static, NUL-terminated description of a gdn_status value. */
+const char *gdn_status_string(int status);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+int gdn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

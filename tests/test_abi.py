@@ -1,0 +1,138 @@
+"""C-ABI checks that need no GPU: the library builds, loads and exports every
+function declared in include/gdn.h, and host-side validation rejects bad
+arguments before anything touches a device (no compute calls here)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+import gated_delta_rule_142_b200 as gdn
+from gated_delta_rule_142_b200 import build as gdn_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER_DIR = os.path.join(ROOT, "include")
+
+OK, NULL, SIZE, UNSUP, MISAL, ALLOC, LAUNCH, TIMEOUT, ALIAS, DEVICE = range(10)
+
+
+def declared_functions():
+    names = set()
+    for h in os.listdir(HEADER_DIR):
+        if not h.endswith(".h"):
+            continue
+        text = open(os.path.join(HEADER_DIR, h)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b(gdn_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    gdn_build.build()
+    return gdn.load()
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    assert {"gdn_forward", "gdn_decode_step", "gdn_status_string", "gdn_version"} <= names
+
+
+def test_library_exports_every_declared_function(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert getattr(lib, name) is not None
+    assert set(gdn.EXPORTS) <= declared_functions()
+
+
+def test_status_strings(lib):
+    for s in range(10):
+        assert gdn.status_string(s)
+    assert gdn.status_string(0) == "ok"
+    assert "unknown" in gdn.status_string(12345)
+    assert lib.gdn_version() >= 100
+
+
+# Fake, never dereferenced addresses: every call below is rejected by the host-side
+# validation before any device or memory access.
+A = 0x10000000
+
+
+def fwd(lib, q=A, k=A + 0x1000000, v=A + 0x2000000, la=A + 0x3000000, be=A + 0x4000000, S0=None,
+        out=A + 0x5000000, Sf=None, B=1, T=8, H=2, dk=16, dv=16, chunk=16, dtype=0):
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    return lib.gdn_forward(P(q), P(k), P(v), P(la), P(be), P(S0), P(out), P(Sf), B, T, H, dk, dv, chunk, None, dtype)
+
+
+def dec(lib, q=A, k=A + 0x1000000, v=A + 0x2000000, la=A + 0x3000000, be=A + 0x4000000, S=A + 0x6000000,
+        out=A + 0x5000000, B=2, H=2, dk=16, dv=16, dtype=1):
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    return lib.gdn_decode_step(P(q), P(k), P(v), P(la), P(be), P(S), P(out), B, H, dk, dv, None, dtype)
+
+
+def test_forward_rejects_bad_arguments(lib):
+    assert fwd(lib, dtype=7) == UNSUP
+    assert fwd(lib, B=-1) == SIZE
+    assert fwd(lib, T=-5) == SIZE
+    assert fwd(lib, dk=48) == UNSUP
+    assert fwd(lib, dv=256) == UNSUP
+    assert fwd(lib, chunk=128) == UNSUP
+    assert fwd(lib, chunk=0) == UNSUP
+    assert fwd(lib, q=None) == NULL
+    assert fwd(lib, out=None) == NULL
+    assert fwd(lib, be=None) == NULL
+    assert fwd(lib, q=A + 8) == MISAL
+    assert fwd(lib, S0=A + 0x7000004) == MISAL
+    assert fwd(lib, B=1 << 40, T=1 << 40) == SIZE
+    # out overlapping an input, S_final partially overlapping S0
+    assert fwd(lib, out=A + 0x2000000) == ALIAS
+    assert fwd(lib, S0=A + 0x7000000, Sf=A + 0x7000010) == ALIAS
+    assert fwd(lib, Sf=A + 0x1000000) == ALIAS
+
+
+def test_forward_empty_problems_are_noops(lib):
+    assert fwd(lib, B=0) == OK
+    assert fwd(lib, H=0, q=None, k=None, v=None, la=None, be=None, out=None) == OK
+
+
+def test_decode_rejects_bad_arguments(lib):
+    assert dec(lib, dtype=2) == UNSUP
+    assert dec(lib, dk=8) == UNSUP
+    assert dec(lib, H=-1) == SIZE
+    assert dec(lib, S=None) == NULL
+    assert dec(lib, out=None) == NULL
+    assert dec(lib, v=A + 0x2000002) == MISAL
+    assert dec(lib, out=A + 0x6000000) == ALIAS
+    assert dec(lib, S=A) == ALIAS
+    assert dec(lib, B=0) == OK
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_valid_call_without_device_reports_device_error(lib):
+    # S0 == S_final (in place) is allowed; with no CUDA device the call stops at the device check.
+    assert fwd(lib, S0=A + 0x7000000, Sf=A + 0x7000000) == DEVICE
+    assert dec(lib) == DEVICE
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    import importlib
+    saved = gdn._lib
+    try:
+        gdn._lib = None
+        with pytest.raises(RuntimeError, match="libgdn.so not found"):
+            gdn.load(os.path.join(str(tmp_path), "missing.so"))
+    finally:
+        gdn._lib = saved
+    importlib.import_module("gated_delta_rule_142_b200")
+
+
+def test_binding_validates_shapes_and_dtypes(lib):
+    q = torch.zeros(1, 4, 2, 16)
+    with pytest.raises(ValueError):
+        gdn.forward(q, torch.zeros(1, 4, 2, 8), torch.zeros(1, 4, 2, 16), torch.zeros(1, 4, 2), torch.zeros(1, 4, 2))
+    with pytest.raises(TypeError):
+        gdn.forward(q.double(), q.double(), q.double(), torch.zeros(1, 4, 2), torch.zeros(1, 4, 2))
+    with pytest.raises(ValueError):
+        gdn.forward(q.transpose(1, 2), q, q, torch.zeros(1, 4, 2), torch.zeros(1, 4, 2))
