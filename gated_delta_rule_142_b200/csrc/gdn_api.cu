@@ -60,6 +60,7 @@ int device_info(DeviceInfo *info) {
 bool supported_dim(int64_t d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 bool supported_chunk(int64_t c) { return c == 16 || c == 32 || c == 64; }
 bool aligned16(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 bool mul3(int64_t a, int64_t b, int64_t c, int64_t *r) {
     int64_t t;
@@ -145,7 +146,7 @@ const char *gdn_status_string(int status) {
         case GDN_ERR_NULL_PTR: return "a required pointer is NULL";
         case GDN_ERR_INVALID_SIZE: return "invalid size (negative, or the element count overflows int64)";
         case GDN_ERR_UNSUPPORTED: return "unsupported dk/dv (16, 32, 64, 128), chunk (16, 32, 64) or dtype";
-        case GDN_ERR_MISALIGNED: return "a pointer is not 16-byte aligned";
+        case GDN_ERR_MISALIGNED: return "a pointer is misaligned (16 bytes; 4 bytes for log_alpha and beta)";
         case GDN_ERR_ALLOC: return "stream-ordered device allocation failed";
         case GDN_ERR_LAUNCH: return "kernel launch or enqueued copy failed";
         case GDN_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
@@ -170,7 +171,7 @@ int gdn_forward(const void *q, const void *k, const void *v, const float *log_al
         return GDN_ERR_INVALID_SIZE;
     if (B * H == 0) return GDN_OK;
     if (ntok > 0 && (!q || !k || !v || !log_alpha || !beta || !out)) return GDN_ERR_NULL_PTR;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) || !aligned16(beta) ||
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(log_alpha) || !aligned4(beta) ||
         !aligned16(S0) || !aligned16(out) || !aligned16(S_final))
         return GDN_ERR_MISALIGNED;
     const Span sq(q, nqk), sk(k, nqk), sv(v, nv), sla(log_alpha, ntok * 4), sbe(beta, ntok * 4);
@@ -238,7 +239,7 @@ int gdn_decode_step(const void *q, const void *k, const void *v, const float *lo
         return GDN_ERR_INVALID_SIZE;
     if (nh == 0) return GDN_OK;
     if (!q || !k || !v || !log_alpha || !beta || !S || !out) return GDN_ERR_NULL_PTR;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) || !aligned16(beta) ||
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(log_alpha) || !aligned4(beta) ||
         !aligned16(S) || !aligned16(out))
         return GDN_ERR_MISALIGNED;
     const Span sq(q, nqk), sk(k, nqk), sv(v, nv), sla(log_alpha, nh * 4), sbe(beta, nh * 4);

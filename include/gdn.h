@@ -65,7 +65,7 @@ typedef enum {
     GDN_ERR_NULL_PTR = 1,       /* a required pointer is NULL                          */
     GDN_ERR_INVALID_SIZE = 2,   /* negative size, or sizes whose product overflows     */
     GDN_ERR_UNSUPPORTED = 3,    /* dk, dv, chunk or dtype outside the supported set    */
-    GDN_ERR_MISALIGNED = 4,     /* a pointer is not 16-byte aligned                    */
+    GDN_ERR_MISALIGNED = 4,     /* misaligned pointer (see Alignment below)            */
     GDN_ERR_ALLOC = 5,          /* stream-ordered workspace/staging allocation failed  */
     GDN_ERR_LAUNCH = 6,         /* a kernel launch or an enqueued copy failed          */
     GDN_ERR_DEVICE_TIMEOUT = 7, /* a bounded device-side wait gave up                  */
@@ -100,7 +100,8 @@ typedef enum {
  *
  * Aliasing: out must not overlap q, k, v, gates, S0 or S_final; S_final
  * must not partially overlap S0 (exact equality is allowed).
- * Alignment: all non-NULL pointers 16-byte aligned.
+ * Alignment: q, k, v, out, S0, S_final 16-byte aligned; log_alpha and beta
+ * 4-byte aligned.
  */
 int gdn_forward(const void *q, const void *k, const void *v, const float *log_alpha,
                 const float *beta, const float *S0, void *out, float *S_final, int64_t B,
@@ -118,6 +119,8 @@ int gdn_forward(const void *q, const void *k, const void *v, const float *log_al
  * float32; S [B, H, dv, dk] float32, read and overwritten; dk, dv each one
  * of 16, 32, 64, 128; dtype of q, k, v, out.  B == 0 or H == 0 is a no-op.
  * Aliasing: out must not overlap any input or S.
+ * Alignment: q, k, v, out, S 16-byte aligned; log_alpha and beta 4-byte
+ * aligned (a per-step slice of a [steps, B, H] gate array is accepted).
  */
 int gdn_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
                     const float *beta, float *S, void *out, int64_t B, int64_t H, int64_t dk,

@@ -85,6 +85,8 @@ def test_forward_rejects_bad_arguments(lib):
     assert fwd(lib, be=None) == NULL
     assert fwd(lib, q=A + 8) == MISAL
     assert fwd(lib, S0=A + 0x7000004) == MISAL
+    assert fwd(lib, la=A + 0x3000002) == MISAL
+    assert fwd(lib, la=A + 0x3000004, B=0) == OK
     assert fwd(lib, B=1 << 40, T=1 << 40) == SIZE
     # out overlapping an input, S_final partially overlapping S0
     assert fwd(lib, out=A + 0x2000000) == ALIAS
