@@ -215,8 +215,10 @@ int gdn_forward(const void *q, const void *k, const void *v, const float *log_al
                      : cudaMemsetAsync(p.S_final, 0, (size_t)nstate, stream);
         }
     } else {
-        (void)forced_path();
-        e = gdn::launch_fwd_simt(p, info.sm_count, stream);
+        if (forced_path() != FwdPath::Simt && gdn::fwd_tc_supported(p))
+            e = gdn::launch_fwd_tc(p, stream);
+        else
+            e = gdn::launch_fwd_simt(p, info.sm_count, stream);
     }
     if (e != cudaSuccess) {
         cudaGetLastError();

@@ -36,4 +36,8 @@ cudaError_t launch_decode(const DecodeProblem &p, cudaStream_t stream);
 // fwd_simt.cu -- float32 SIMT chunkwise forward, any supported (dk, dv, chunk).
 cudaError_t launch_fwd_simt(const FwdProblem &p, int sm_count, cudaStream_t stream);
 
+// fwd_tc.cu -- tcgen05 chunkwise forward: bf16, dk = dv = 128, chunk = 64.
+bool fwd_tc_supported(const FwdProblem &p);
+cudaError_t launch_fwd_tc(const FwdProblem &p, cudaStream_t stream);
+
 }  // namespace gdn
