@@ -195,7 +195,7 @@ def oracle_forward_sample(w, budget_s: float):
 def run_reference(args, world, rank):
     if rank != 0:
         return 0
-    w = WORKLOADS[FWD_WORKLOAD]
+    w = WORKLOADS[args.workload]
     model, cores = cpu_info()
     for _ in range(args.warmup):
         oracle_forward_sample(w, 0.5)
@@ -248,7 +248,7 @@ def run_gdn(args, world, rank, local):
     sampler.start()
 
     # ---- forward, inputs resident in HBM ----
-    w = WORKLOADS[FWD_WORKLOAD]
+    w = WORKLOADS[args.workload]
     es = 2 if w.dtype == "bf16" else 4
     inp = forward_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, seed=w.seed + 1000 * rank, s0_std=w.s0_std,
                          alpha_mu=w.alpha_mu)
@@ -335,7 +335,7 @@ def run_gdn(args, world, rank, local):
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
                        "input_dtype": w.dtype, "state_dtype": "f32", "parallelism": "replicas" if world > 1 else "single",
                        "l2": "inputs larger than L2 (%.2f GB read+written per step)" % (nbytes / 1e9)},
@@ -356,6 +356,9 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["gdn", "reference"], default="gdn")
+    ap.add_argument("--workload", default=FWD_WORKLOAD,
+                    choices=[n for n, w in WORKLOADS.items() if w.kind == "forward"],
+                    help="forward workload timed as the step (default: the 64K-token one)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

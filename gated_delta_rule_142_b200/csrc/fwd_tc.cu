@@ -54,13 +54,16 @@ constexpr uint32_t OFF_P = 98304;         // 8 KB   P      [t][s] K-major
 constexpr uint32_t OFF_TB = 106496;       // 8 KB   T diag(beta)       [t][s] K-major
 constexpr uint32_t OFF_TBG = 114688;      // 8 KB   T diag(beta gamma) [t][s] K-major
 constexpr uint32_t OFF_W = 122880;        // 16 KB  W stored MN-major: row i (key dim), 64 t per row
-constexpr uint32_t OFF_AM = 139264;       // 16 KB  A  fp32 [64][64]
-constexpr uint32_t OFF_TM = 155648;       // 16 KB  T  fp32 [64][64]
-constexpr uint32_t OFF_Y = 172032;        // 3 KB   block-substitution scratch
-constexpr uint32_t OFF_GATES = 175104;    // 1 KB   g, beta, gamma, decay-to-end
-constexpr uint32_t OFF_BARS = 176128;     // mbarriers: full[2], mma
-constexpr uint32_t OFF_MISC = 176192;     // tmem base slot, scan scratch
-constexpr uint32_t SMEM_TC = 176256 + 1024;
+constexpr int LDM = 68;                   // row stride (floats) of the fp32 64x64 tiles: conflict-free rows
+constexpr uint32_t OFF_AM = 139264;       // 17 KB  A  fp32 [64][LDM]
+constexpr uint32_t OFF_TM = 156672;       // 17 KB  T  fp32 [64][LDM]
+constexpr uint32_t OFF_Y = 174080;        // 3 KB   block-substitution scratch
+constexpr uint32_t OFF_GATES = 177152;    // 1.5 KB g, beta, gamma, decay-to-end, e^{g-c}, e^{c-g}
+constexpr uint32_t OFF_BARS = 178688;     // mbarriers: full[2], mma
+constexpr uint32_t OFF_MISC = 178752;     // tmem base slot, scan scratch
+constexpr uint32_t SMEM_TC = 178816 + 1024;
+constexpr uint32_t OFF_OST = OFF_P;       // output staging [64][136] bf16 (reuses P/T/W tiles)
+constexpr int LDO = 136;
 constexpr uint32_t kTxBytes = 3 * 2 * 8192;  // Q, K, V: two 8 KB boxes each
 
 // TMEM column map (512 columns allocated).
@@ -85,6 +88,10 @@ __device__ int g_tc_timeout;  // set when a bounded mbarrier wait gives up
 // W^T 128x64, D 128x128, O^T 128x64, S 128x128, all float32 row-major).
 __device__ float *g_dbg;
 #define DBG_ON (g_dbg != nullptr && blockIdx.x == 0 && c == 0)
+// per-phase clock stamps of CTA 0, chunks 0..7 (int64 at float offset 73728, 16 per chunk)
+#define DBG_CLK(i)                                                                     \
+    if (g_dbg != nullptr && blockIdx.x == 0 && tid == 0 && c < 8)                      \
+        reinterpret_cast<long long *>(g_dbg + 73728)[c * 16 + (i)] = clock64();
 __device__ __forceinline__ void dbg_tmem_rows(uint32_t taddr, int ncols, float *dst) {
     for (int q = 0; q < ncols; q += 32) {
         uint32_t r[32];
@@ -93,6 +100,8 @@ __device__ __forceinline__ void dbg_tmem_rows(uint32_t taddr, int ncols, float *
         for (int i = 0; i < 32; ++i) dst[q + i] = __uint_as_float(r[i]);
     }
 }
+#else
+#define DBG_CLK(i)
 #endif
 
 struct TcArgs {
@@ -136,6 +145,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     float *bet = g + 64;
     float *gam = g + 128;
     float *dl = g + 192;
+    float *ea = g + 256;  // e^{g_t - c}
+    float *eb = g + 320;  // e^{c - g_s}
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + OFF_BARS);
     uint64_t *mma_bar = full + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC);
@@ -210,8 +221,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         uint8_t *qk_ptr = sm + OFF_QK + buf * QK_BYTES;
 
         if (tid == 0 && c + 1 < nchunks) issue_loads(c + 1, buf ^ 1);
+        DBG_CLK(0)
 
         // ---- wait for this chunk's tiles; G = [Q;K] K^T ----
+        DBG_CLK(1)
         bool w = mbar_wait(&full[buf], full_phase[buf]);
         full_phase[buf] ^= 1u;
         if (!__syncthreads_and(w)) { ok = false; break; }
@@ -226,6 +239,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mma_commit(mma_bar);
         }
 
+        DBG_CLK(2)
         // ---- gates: g = cumsum(max(log_alpha, floor)), beta; zero past T ----
         if (tid < 64) {
             const int64_t gi = ((int64_t)b * T + t0 + tid) * H + h;
@@ -243,22 +257,32 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         __syncthreads();
         if (tid >= 32 && tid < 64) g[tid] += scan_tmp[0];
         __syncthreads();
+        // e^{g_t - g_s} = e^{g_t - c} e^{c - g_s} with c = g_31, exact to a few ulp while every
+        // |g_t - c| < 80; a chunk with a wider decay span uses expf(g_t - g_s) per element.
+        bool narrow = true;
         if (tid < 64) {
-            gam[tid] = expf(g[tid]);
-            dl[tid] = expf(g[63] - g[tid]);
+            const float gt = g[tid], cm = g[31];
+            gam[tid] = expf(gt);
+            dl[tid] = expf(g[63] - gt);
+            ea[tid] = expf(gt - cm);
+            eb[tid] = expf(cm - gt);
+            narrow = fabsf(gt - cm) < 80.f;
         }
+        DBG_CLK(3)
         w = mbar_wait(mma_bar, mma_phase);
         mma_phase ^= 1u;
+        narrow = __syncthreads_and(narrow);
         if (!__syncthreads_and(w)) { ok = false; break; }
         tc_fence_after();
 
+        DBG_CLK(4)
 #ifdef GDN_TC_DEBUG
         if (DBG_ON) dbg_tmem_rows(tm + lb + TM_G, 64, g_dbg + tid * 64);
 #endif
         // ---- epilogue of G: P (bf16 tile) from the Q rows, A (fp32) from the K rows; Q <- gamma Q ----
         {
             const int t = tid & 63;
-            const float gt = g[t];
+            const float gt = g[t], at = ea[t];
             if (tid < 64) {
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
@@ -269,8 +293,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
                     for (int i = 0; i < 32; i += 2) {
                         const int s = half * 32 + i;
-                        const float v0 = (s <= t) ? __uint_as_float(r[i]) * expf(gt - g[s]) : 0.f;
-                        const float v1 = (s + 1 <= t) ? __uint_as_float(r[i + 1]) * expf(gt - g[s + 1]) : 0.f;
+                        const float d0 = narrow ? at * eb[s] : expf(gt - g[s]);
+                        const float d1 = narrow ? at * eb[s + 1] : expf(gt - g[s + 1]);
+                        const float v0 = (s <= t) ? __uint_as_float(r[i]) * d0 : 0.f;
+                        const float v1 = (s + 1 <= t) ? __uint_as_float(r[i + 1]) * d1 : 0.f;
                         pk[i >> 1] = pack_bf16x2(v0, v1);
                     }
 #pragma unroll
@@ -290,19 +316,21 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; i += 4) {
-                        float4 v;
-                        const int s = half * 32 + i;
-                        v.x = (s < t) ? bt * expf(gt - g[s]) * __uint_as_float(r[i]) : 0.f;
-                        v.y = (s + 1 < t) ? bt * expf(gt - g[s + 1]) * __uint_as_float(r[i + 1]) : 0.f;
-                        v.z = (s + 2 < t) ? bt * expf(gt - g[s + 2]) * __uint_as_float(r[i + 2]) : 0.f;
-                        v.w = (s + 3 < t) ? bt * expf(gt - g[s + 3]) * __uint_as_float(r[i + 3]) : 0.f;
-                        *reinterpret_cast<float4 *>(Am + t * 64 + s) = v;
+                        float v[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int s = half * 32 + i + e;
+                            const float dd = narrow ? at * eb[s] : expf(gt - g[s]);
+                            v[e] = (s < t) ? bt * dd * __uint_as_float(r[i + e]) : 0.f;
+                        }
+                        *reinterpret_cast<float4 *>(Am + t * LDM + half * 32 + i) = make_float4(v[0], v[1], v[2], v[3]);
                     }
                 }
             }
         }
         __syncthreads();
 
+        DBG_CLK(5)
         // ---- T = (I + A)^{-1}: 16x16 diagonal blocks by substitution (one warp each, a column per lane) ----
         if (lane < 16) {
             const int o = warp * 16;
@@ -311,38 +339,59 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             for (int r = 0; r < 16; ++r) {
                 float acc = (r == lane) ? 1.f : 0.f;
 #pragma unroll
-                for (int s = 0; s < r; ++s) acc -= Am[(o + r) * 64 + o + s] * x[s];
+                for (int s = 0; s < r; ++s) acc -= Am[(o + r) * LDM + o + s] * x[s];
                 x[r] = acc;
             }
 #pragma unroll
-            for (int r = 0; r < 16; ++r) Tm[(o + r) * 64 + o + lane] = x[r];
+            for (int r = 0; r < 16; ++r) Tm[(o + r) * LDM + o + lane] = x[r];
         }
         __syncthreads();
-        // block rows I = 1..3:  T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ
+        DBG_CLK(6)
+        // block rows I = 1..3:  T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ ; one thread per (J, row, 4 columns)
         for (int I = 1; I < 4; ++I) {
-            for (int e = tid; e < I * 256; e += kThreadsTc) {
-                const int J = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-                float acc = 0.f;
-                for (int K = J; K < I; ++K)
+            for (int e = tid; e < I * 64; e += kThreadsTc) {
+                const int J = e >> 6, r = (e >> 2) & 15, c4 = (e & 3) * 4;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int K = J; K < I; ++K) {
+                    const float *arow = Am + (16 * I + r) * LDM + 16 * K;
+                    const float *tcol = Tm + (16 * K) * LDM + 16 * J + c4;
 #pragma unroll
-                    for (int m = 0; m < 16; ++m) acc += Am[(16 * I + r) * 64 + 16 * K + m] * Tm[(16 * K + m) * 64 + 16 * J + cc];
-                Y[e] = acc;
+                    for (int m = 0; m < 16; ++m) {
+                        const float a = arow[m];
+                        const float4 tv = *reinterpret_cast<const float4 *>(tcol + m * LDM);
+                        acc.x = fmaf(a, tv.x, acc.x);
+                        acc.y = fmaf(a, tv.y, acc.y);
+                        acc.z = fmaf(a, tv.z, acc.z);
+                        acc.w = fmaf(a, tv.w, acc.w);
+                    }
+                }
+                *reinterpret_cast<float4 *>(Y + J * 256 + r * 16 + c4) = acc;
             }
             __syncthreads();
-            for (int e = tid; e < I * 256; e += kThreadsTc) {
-                const int J = e >> 8, r = (e >> 4) & 15, cc = e & 15;
-                float acc = 0.f;
+            for (int e = tid; e < I * 64; e += kThreadsTc) {
+                const int J = e >> 6, r = (e >> 2) & 15, c4 = (e & 3) * 4;
+                const float *trow = Tm + (16 * I + r) * LDM + 16 * I;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                for (int m = 0; m < 16; ++m) acc += Tm[(16 * I + r) * 64 + 16 * I + m] * Y[J * 256 + m * 16 + cc];
-                Tm[(16 * I + r) * 64 + 16 * J + cc] = -acc;
+                for (int m = 0; m < 16; ++m) {
+                    const float a = trow[m];
+                    const float4 y = *reinterpret_cast<const float4 *>(Y + J * 256 + m * 16 + c4);
+                    acc.x = fmaf(a, y.x, acc.x);
+                    acc.y = fmaf(a, y.y, acc.y);
+                    acc.z = fmaf(a, y.z, acc.z);
+                    acc.w = fmaf(a, y.w, acc.w);
+                }
+                *reinterpret_cast<float4 *>(Tm + (16 * I + r) * LDM + 16 * J + c4) =
+                    make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
             }
             __syncthreads();
         }
+        DBG_CLK(7)
 #ifdef GDN_TC_DEBUG
         if (DBG_ON)
             for (int e = tid; e < 4096; e += kThreadsTc) {
-                g_dbg[8192 + e] = Am[e];
-                g_dbg[12288 + e] = ((e & 63) <= (e >> 6)) ? Tm[e] : 0.f;
+                g_dbg[8192 + e] = Am[(e >> 6) * LDM + (e & 63)];
+                g_dbg[12288 + e] = ((e & 63) <= (e >> 6)) ? Tm[(e >> 6) * LDM + (e & 63)] : 0.f;
             }
 #endif
         // T diag(beta) (threads 0..63) and T diag(beta gamma) (threads 64..127), bf16, lower triangle
@@ -356,8 +405,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #pragma unroll
                 for (int i = 0; i < 8; i += 2) {
                     const int s = cc * 8 + i;
-                    float v0 = (s <= t) ? Tm[t * 64 + s] * bet[s] : 0.f;
-                    float v1 = (s + 1 <= t) ? Tm[t * 64 + s + 1] * bet[s + 1] : 0.f;
+                    float v0 = (s <= t) ? Tm[t * LDM + s] * bet[s] : 0.f;
+                    float v1 = (s + 1 <= t) ? Tm[t * LDM + s + 1] * bet[s + 1] : 0.f;
                     if (with_gamma) {
                         v0 *= gam[s];
                         v1 *= gam[s + 1];
@@ -371,6 +420,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tc_fence_before();
         __syncthreads();
 
+        DBG_CLK(8)
         // ---- Ut^T = V^T (T beta)^T ;  W^T = K^T (T beta gamma)^T ----
         if (tid == 0) {
             tc_fence_after();
@@ -387,6 +437,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             mma_commit(mma_bar);
         }
 
+        DBG_CLK(9)
         // ---- meanwhile: S -> bf16 operand copy; S <- gamma_C S (float32, in TMEM) ----
         {
             const float gC = gam[63];
@@ -405,6 +456,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             tmem_wait_st();
         }
+        DBG_CLK(10)
         w = mbar_wait(mma_bar, mma_phase);
         mma_phase ^= 1u;
         if (!__syncthreads_and(w)) { ok = false; break; }
@@ -441,6 +493,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tc_fence_before();
         __syncthreads();
 
+        DBG_CLK(11)
         // ---- D = S [W; gamma Q]^T  (A = bf16 S from TMEM) ----
         if (tid == 0) {
             tc_fence_after();
@@ -462,6 +515,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 #ifdef GDN_TC_DEBUG
         if (DBG_ON) dbg_tmem_rows(tm + lb + TM_D1, 128, g_dbg + 32768 + tid * 128);
 #endif
+        DBG_CLK(12)
         // ---- U^T = Ut^T - S W^T  -> bf16 A operand in TMEM ----
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -480,6 +534,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         tc_fence_before();
         __syncthreads();
 
+        DBG_CLK(13)
         // ---- O^T += U^T P^T ;  S += U^T Ktil ----
         if (tid == 0) {
             tc_fence_after();
@@ -504,24 +559,33 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             dbg_tmem_rows(tm + lb + TM_S, 128, g_dbg + 57344 + tid * 128);
         }
 #endif
-        // ---- outputs: thread j holds o[t][j] for the 64 tokens ----
+        DBG_CLK(14)
+        // ---- outputs: thread j holds o[t][j]; stage [t][j] in shared memory, then coalesced rows ----
         {
-            __nv_bfloat16 *ob = p.out + (((int64_t)b * T + t0) * H + h) * kD + tid;
+            __nv_bfloat16 *ost = reinterpret_cast<__nv_bfloat16 *>(sm + OFF_OST);
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t r[32];
                 tmem_ld32(tm + lb + TM_D1 + 64 + half * 32, r);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int t = half * 32 + i;
-                    if (t < n) ob[(int64_t)t * H * kD] = __float2bfloat16_rn(__uint_as_float(r[i]));
-                }
+                for (int i = 0; i < 32; ++i) ost[(half * 32 + i) * LDO + tid] = __float2bfloat16_rn(__uint_as_float(r[i]));
+            }
+            __syncthreads();
+            __nv_bfloat16 *ob = p.out + (((int64_t)b * T + t0) * H + h) * kD;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int q = tid + k * kThreadsTc;  // 16-byte piece: row q / 16, column (q % 16) * 8
+                const int t = q >> 4, c8 = (q & 15) * 8;
+                if (t < n)
+                    *reinterpret_cast<uint4 *>(ob + (int64_t)t * H * kD + c8) =
+                        *reinterpret_cast<const uint4 *>(ost + t * LDO + c8);
             }
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
+        DBG_CLK(15)
     }
 
     if (!ok && tid == 0) atomicExch(&g_tc_timeout, 1);
