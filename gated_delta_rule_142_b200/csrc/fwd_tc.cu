@@ -11,31 +11,41 @@
 //   prep (independent of S):
 //     G    = [Q; K] K^T                                   (tcgen05, M = 128)
 //     A    = strict_lower(beta_t e^{g_t-g_s} (K K^T)_ts),  P = lower(e^{g_t-g_s} (Q K^T)_ts)
-//     T    = (I + A)^{-1}                                  (blocked substitution, fp32)
+//     T    = (I + A)^{-1}   16x16 diagonal blocks by substitution, merged 16->32->64
+//                           with warp-level TF32 MMAs (fp32 accumulation); the final writer
+//                           of each entry also writes T diag(beta) and T diag(beta gamma) in bf16
 //     Ut^T = V^T (T diag(beta))^T,  W^T = K^T (T diag(beta gamma))^T   (tcgen05)
-//     Qg   = diag(gamma) Q
 //   chain (needs S; sequential over chunks):
 //     U^T  = Ut^T - S W^T                      (tcgen05 accumulate, B negated; A = bf16 S in TMEM)
-//     O^T  = S Qg^T + U^T P^T                  (tcgen05; A = bf16 S, then bf16 U^T in TMEM)
 //     S   <- gamma_C S + (U^T diag(dl)) K      (tcgen05 accumulate into the float32 state)
+//   outputs (off the chain), with e^{g_t - g_s} = e^{g_t - c} e^{c - g_s} (c = g_31) when the
+//   chunk's decay span allows it (always exact; otherwise P' = P and f2 = 1):
+//     O1^T = S Q^T,  O2^T = U^T P'^T,  P'_ts = e^{c - g_s} (Q K^T)_ts (s <= t)   (tcgen05)
+//     o_t  = gamma_t O1_t + e^{g_t - c} O2_t, staged in shared memory, written by TMA
 // The state S stays in tensor memory in float32 for the whole sequence; its
 // bf16 operand copy is rewritten from it every chunk.
 //
-// Warp roles (512 threads):
-//   warp 0      control: TMA loads (double-buffered Q/K/V tiles) and every
-//               tcgen05.mma, issued by one thread in dependency order
+// Warp roles (512 threads).  One thread issuing tcgen05.mma sustains about
+// one MMA per ~90 cycles, more than an M128xN64xK16 MMA takes to execute, so
+// the MMAs are issued by three threads, one per independent stream:
+//   warp 0      chain issuer: TMA loads, U^T and S updates (the critical path)
+//   warp 1      output issuer: O1^T = S Q^T, O2^T = U^T P'^T
+//   warp 2      prep issuer: G, Ut^T, W^T
 //   warps 4-11  prep for chunk c+1 (256 threads) while the chain runs chunk c
 //   warps 12-15 chain: state conversion, U^T epilogue, outputs (thread j owns
 //               TMEM lane j, i.e. state row j)
-//   warps 1-3   idle
+//   warp 3      idle
 // Roles hand work to each other through mbarriers (tcgen05.commit for MMA
-// completion, single-thread arrivals after a named barrier otherwise).  Every
-// wait is bounded; a wait that gives up sets an abort flag that makes every
-// other wait return at once, so the CTA always reaches its exit, frees its
-// tensor memory and records the timeout.
+// completion, single-thread arrivals after a named barrier otherwise); every
+// barrier completes once per chunk, and no role can run two completions ahead
+// of a role that waits on it.  Every wait is bounded; a wait that gives up
+// sets an abort flag that releases every other wait, and each role leaves its
+// loop as a whole, so the CTA always frees its tensor memory and exits.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+
+#include <stdlib.h>
 
 #include <atomic>
 
@@ -66,22 +76,25 @@ constexpr uint32_t OFF_W = 131072;       // 16 KB  W stored MN-major: row i (key
 constexpr int LDM = 68;                  // row stride (floats) of the fp32 64x64 tiles
 constexpr uint32_t OFF_AM = 147456;      // 17 KB  A  fp32 [64][LDM]
 constexpr uint32_t OFF_TM = 164864;      // 17 KB  T  fp32 [64][LDM]
-constexpr uint32_t OFF_Y = 182272;       // 3 KB   block-substitution scratch
-constexpr uint32_t OFF_PG = 185344;      // prep gates: g, beta, gamma, e^{g-c}, e^{c-g} (64 each)
-constexpr uint32_t OFF_CG = 186624;      // chain gates: dl (64), scratch
-constexpr uint32_t OFF_BARS = 187136;    // mbarriers
-constexpr uint32_t OFF_MISC = 187264;    // tmem slot, abort flag, scan scratch
-constexpr uint32_t SMEM_TC = 187328 + 1024;
+constexpr uint32_t OFF_XS = 182272;      // 5 KB   merge scratch: 4 x [16][8] (16->32), then [32][LDX2] (32->64)
+constexpr int LDX2 = 40;
+constexpr uint32_t OFF_PG = 187392;      // prep gates: g, beta, gamma, e^{g-c}, e^{c-g} (64 each)
+constexpr uint32_t OFF_CG = 188672;      // chain gates per chunk parity: dl[2][64], f1[2][64], f2[2][64], gamma_C[2]
+constexpr uint32_t OFF_OST = 190464;     // 16 KB  output staging: two [64 t][64 d] bf16 boxes, 128-byte swizzle
+constexpr uint32_t OFF_BARS = 206848;    // mbarriers
+constexpr uint32_t OFF_MISC = 206976;    // tmem slot, abort flag, scan scratch
+constexpr uint32_t SMEM_TC = 207040 + 1024;
 constexpr uint32_t kTxBytes = 3 * 2 * 8192;  // Q, K, V: two 8 KB boxes each
 
 // TMEM column map (512 columns).
 constexpr uint32_t TM_S = 0;     // 128  S float32 (row j in lane j)
 constexpr uint32_t TM_SB = 128;  // 64   bf16 S (A operand, 2 per column)
-constexpr uint32_t TM_O = 192;   // 64   O^T accumulator
+constexpr uint32_t TM_O = 192;   // 64   O1^T = S Q^T
 constexpr uint32_t TM_UB = 256;  // 32   bf16 U^T (A operand)
 constexpr uint32_t TM_UDB = 288; // 32   bf16 U^T diag(dl) (A operand)
-constexpr uint32_t TM_DU = 320;  // 2 x 64  Ut^T, accumulated into U^T (per chunk parity)
-constexpr uint32_t TM_G = 448;   // 64   [Q;K] K^T, later W^T
+constexpr uint32_t TM_DU = 320;  // 64   Ut^T, accumulated into U^T
+constexpr uint32_t TM_G = 384;   // 64   [Q;K] K^T, later W^T
+constexpr uint32_t TM_O2 = 448;  // 64   O2^T = U^T P'^T
 
 constexpr uint32_t IDESC_G = instr_desc_bf16(128, 64, 0, 0);                 // [Q;K] . K^T
 constexpr uint32_t IDESC_MN64 = instr_desc_bf16(128, 64, 1, 0);              // V^T / K^T (MN-major A) . T^T
@@ -89,27 +102,45 @@ constexpr uint32_t IDESC_WNEG = instr_desc_bf16(128, 64, 0, 1) | (1u << 14); // 
 constexpr uint32_t IDESC_Q = instr_desc_bf16(128, 64, 0, 0);                 // S . Qg^T, U^T . P^T
 constexpr uint32_t IDESC_S = instr_desc_bf16(128, 128, 0, 1);                // (U^T dl) . K (MN-major B)
 
-enum Bar { B_FULL0 = 0, B_FULL1, B_GDONE, B_UWDONE, B_M1DONE, B_M2DONE, B_TBREADY, B_PREPREADY, B_SREADY, B_UREADY,
-           B_OFREE, B_COUNT };
+enum Bar {
+    B_FULL0 = 0, B_FULL1,                                 // TMA tiles landed (per buffer)
+    B_GDONE, B_WDONE, B_UTDONE,                           // prep MMAs complete
+    B_M1ADONE, B_M2BDONE,                                 // chain MMAs complete
+    B_M1BDONE, B_M2ADONE,                                 // output MMAs complete
+    B_TBREADY, B_PREPREADY, B_SREADY, B_UREADY, B_OFREE,  // role hand-offs
+    B_COUNT
+};
 
 __device__ int g_tc_timeout;  // set when a bounded mbarrier wait gives up
 
 #ifdef GDN_TC_DEBUG
-// Debug builds only: per-phase clock stamps of CTA 0 for chunks 0..7, three
-// rows of 16 int64 per chunk (control, prep, chain), at float offset 73728.
+// Debug builds only: per-phase clock stamps of CTA 0 for chunks 0..7, five
+// rows of 16 int64 per chunk (chain issuer, output issuer, prep issuer, prep,
+// chain), at float offset 73728.
 __device__ float *g_dbg;
 #define DBG_CLK(row, i)                                                          \
     if (g_dbg != nullptr && blockIdx.x == 0 && c < 8)                            \
-        reinterpret_cast<long long *>(g_dbg + 73728)[(c * 3 + (row)) * 16 + (i)] = clock64();
+        reinterpret_cast<long long *>(g_dbg + 73728)[(c * 5 + (row)) * 16 + (i)] = clock64();
 #else
 #define DBG_CLK(row, i)
 #endif
 
+// One launch covers every (b, h) and, for long sequences with few heads, every
+// segment of the sequence.  mode 0: one CTA per (b, h, segment) computes the
+// outputs of its chunk range from that segment's entry state (S0 for the first
+// segment, else S_entry) and writes S_final from the last segment.  mode 1:
+// two CTAs per (b, h, segment < nseg - 1) compute the segment's affine transfer
+// S_end = S_start M + B: one runs the recurrence from the zero state (-> Bw), the
+// other from the identity with v = 0 (-> Mw; rows of the state evolve
+// independently, so each row of M is a state row with no write term).
 struct TcArgs {
     const float *log_alpha, *beta, *S0;
     __nv_bfloat16 *out;
     float *S_final;
     int64_t T, H;
+    int mode, nseg, seg_len;
+    const float *S_entry;  // [B*H][nseg-1][dv][dk]: entry states of segments 1..nseg-1
+    float *Bw, *Mw;        // [B*H][nseg-1][dv][dk] / [dk][dk]: segment transfers
 };
 
 __device__ __forceinline__ void named_bar(int id, int n) {
@@ -168,6 +199,55 @@ __device__ __forceinline__ void scale_bf16x8(uint4 &u, float f) {
     u = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// ---- warp-level TF32 MMA (m16n8k8, fp32 accumulate) for the 64x64 inverse ----
+// Fragment ownership, g = lane / 4, t = lane % 4:
+//   A 16x8: a0 (g, t), a1 (g+8, t), a2 (g, t+4), a3 (g+8, t+4)
+//   B  8x8: b0 (t, g), b1 (t+4, g)
+//   D 16x8: d0 (g, 2t), d1 (g, 2t+1), d2 (g+8, 2t), d3 (g+8, 2t+1)
+__device__ __forceinline__ uint32_t tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ void mma_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+// A fragment from a row-major fp32 matrix M (row stride ld), rows r0.., columns k0..
+__device__ __forceinline__ void load_a(uint32_t (&a)[4], const float *M, int ld, int r0, int k0, int g, int t) {
+    a[0] = tf32(M[(r0 + g) * ld + k0 + t]);
+    a[1] = tf32(M[(r0 + g + 8) * ld + k0 + t]);
+    a[2] = tf32(M[(r0 + g) * ld + k0 + t + 4]);
+    a[3] = tf32(M[(r0 + g + 8) * ld + k0 + t + 4]);
+}
+// B fragment (K x N) from a row-major fp32 matrix M: element (k, n) = M[k0 + k][n0 + n]
+__device__ __forceinline__ void load_b(uint32_t (&b)[2], const float *M, int ld, int k0, int n0, int g, int t) {
+    b[0] = tf32(M[(k0 + t) * ld + n0 + g]);
+    b[1] = tf32(M[(k0 + t + 4) * ld + n0 + g]);
+}
+// Store -D (16x8 fragment) into a row-major fp32 matrix at (r0, c0).
+__device__ __forceinline__ void store_neg_d(float *M, int ld, int r0, int c0, const float (&d)[4], int g, int t) {
+    *reinterpret_cast<float2 *>(M + (r0 + g) * ld + c0 + 2 * t) = make_float2(-d[0], -d[1]);
+    *reinterpret_cast<float2 *>(M + (r0 + g + 8) * ld + c0 + 2 * t) = make_float2(-d[2], -d[3]);
+}
+__device__ __forceinline__ void store_d(float *M, int ld, int r0, int c0, const float (&d)[4], int g, int t) {
+    *reinterpret_cast<float2 *>(M + (r0 + g) * ld + c0 + 2 * t) = make_float2(d[0], d[1]);
+    *reinterpret_cast<float2 *>(M + (r0 + g + 8) * ld + c0 + 2 * t) = make_float2(d[2], d[3]);
+}
+
+// Writes entries (row, col) and (row, col + 1) (col even) of T diag(beta) and
+// T diag(beta gamma) into their bf16 K-major 128-byte-swizzled tiles.
+__device__ __forceinline__ void store_tb_pair(uint8_t *sm, int row, int col, float v0, float v1, const float *bet,
+                                              const float *gam) {
+    const uint32_t off = sw128(row, col >> 3) + (col & 7) * 2;
+    const float b0 = bet[col], b1 = bet[col + 1];
+    *reinterpret_cast<uint32_t *>(sm + OFF_TB + off) = pack_bf16x2(v0 * b0, v1 * b1);
+    *reinterpret_cast<uint32_t *>(sm + OFF_TBG + off) = pack_bf16x2(v0 * b0 * gam[col], v1 * b1 * gam[col + 1]);
+}
+
 // 64-token inclusive cumsum by two full warps (t = 0..63 across them); `x` is
 // this thread's value, `tmp` a shared slot, (bar_id, n) the role's barrier,
 // which every thread of the role must reach once (callers with t >= 64 call
@@ -187,7 +267,7 @@ __device__ __forceinline__ float chunk_cumsum(float x, int t, float *tmp, int ba
 
 __global__ void __launch_bounds__(kThreadsTc, 1)
 fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-              const __grid_constant__ CUtensorMap tm_v, TcArgs p) {
+              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o, TcArgs p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BARS);
@@ -199,9 +279,24 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t T = p.T, H = p.H;
-    const int64_t bh = blockIdx.x;
+    // work item: (b, h), segment, and kind (0 = outputs, 1 = transfer B, 2 = transfer M)
+    int64_t bh;
+    int seg, kind;
+    if (p.mode == 0) {
+        bh = blockIdx.x / p.nseg;
+        seg = (int)(blockIdx.x % p.nseg);
+        kind = 0;
+    } else {
+        const int64_t q = blockIdx.x >> 1;
+        bh = q / (p.nseg - 1);
+        seg = (int)(q % (p.nseg - 1));
+        kind = 1 + (int)(blockIdx.x & 1);
+    }
+    const bool outputs = (kind == 0);
     const int b = (int)(bh / H), h = (int)(bh % H);
-    const int N = (int)((T + kC - 1) / kC);
+    const int Ntot = (int)((T + kC - 1) / kC);
+    const int c0 = seg * p.seg_len;                                      // first chunk of this CTA
+    const int N = (Ntot - c0 < p.seg_len) ? (Ntot - c0) : p.seg_len;     // chunks of this CTA
     const uint32_t sbase = smem_u32(sm);
 
     if (tid == 0) {
@@ -220,10 +315,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     const uint32_t lb = (uint32_t)((warp & 3) * 32) << 16;  // this warp's TMEM lane quadrant
 
     if (warp == 0) {
-        // ============================== control ==============================
+        // ====================== chain issuer (and TMA) ======================
         if (lane == 0) {
             auto issue_loads = [&](int c) {
-                const int buf = c & 1, t0 = c * kC;
+                const int buf = c & 1, t0 = (c0 + c) * kC;
                 mbar_arrive_expect_tx(&bars[B_FULL0 + buf], kTxBytes);
                 uint8_t *qk = sm + OFF_QK + buf * QK_BYTES;
                 uint8_t *vv = sm + OFF_V + buf * V_BYTES;
@@ -234,8 +329,97 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     tma_load_4d(vv + blk * 8192, &tm_v, &bars[B_FULL0 + buf], blk * 64, h, t0, b);
                 }
             };
-            auto mma_G = [&](int c) {
+            bool ok = true;
+            issue_loads(0);
+            if (N > 1) issue_loads(1);
+            for (int c = 0; c < N && ok; ++c) {
+                const uint32_t par = c & 1;
                 const uint32_t qk = sbase + OFF_QK + (c & 1) * QK_BYTES;
+                DBG_CLK(0, 0)
+                if (!(ok = wait_bar(&bars[B_PREPREADY], par, abort_flag))) break;
+                if (!(ok = wait_bar(&bars[B_SREADY], par, abort_flag))) break;
+                if (!(ok = wait_bar(&bars[B_UTDONE], par, abort_flag))) break;
+                DBG_CLK(0, 1)
+                tc_fence_after();
+                // U^T = Ut^T - S W^T  (transfer-M runs have v = 0, so Ut^T = 0 and U^T starts fresh)
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tm + TM_DU, tm + TM_SB + kk * 8, smem_desc_sw128(sbase + OFF_W + kk * 2048, 8192, 1024),
+                           IDESC_WNEG, (kind != 2 || kk > 0) ? 1u : 0u);
+                mma_commit(&bars[B_M1ADONE]);
+                DBG_CLK(0, 2)
+                if (!(ok = wait_bar(&bars[B_UREADY], par, abort_flag))) break;
+                DBG_CLK(0, 3)
+                tc_fence_after();
+                // S += (U^T diag(dl)) K
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ts(tm + TM_S, tm + TM_UDB + kk * 8, smem_desc_sw128(qk + 8192 + kk * 2048, 16384, 1024),
+                           IDESC_S, 1);
+                mma_commit(&bars[B_M2BDONE]);
+                DBG_CLK(0, 4)
+                if (c + 2 < N) {
+                    // buffer c & 1 is free once both final MMAs of chunk c are done with K and Q
+                    if (!(ok = wait_bar(&bars[B_M2BDONE], par, abort_flag))) break;
+                    if (!(ok = wait_bar(&bars[B_M2ADONE], par, abort_flag))) break;
+                    issue_loads(c + 2);
+                }
+                DBG_CLK(0, 5)
+            }
+            if (ok && N > 0) wait_bar(&bars[B_M2BDONE], (N - 1) & 1, abort_flag);
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ========================= output issuer =========================
+        if (lane == 0) {
+            bool ok = true;
+            for (int c = 0; c < N && ok; ++c) {
+                const uint32_t par = c & 1;
+                const uint32_t qk = sbase + OFF_QK + (c & 1) * QK_BYTES;
+                DBG_CLK(1, 0)
+                if (!(ok = wait_bar(&bars[B_PREPREADY], par, abort_flag))) break;
+                if (!(ok = wait_bar(&bars[B_SREADY], par, abort_flag))) break;
+                if (c > 0 && !(ok = wait_bar(&bars[B_OFREE], (c - 1) & 1, abort_flag))) break;
+                DBG_CLK(1, 1)
+                tc_fence_after();
+                // O1^T = S Q^T  (transfer runs issue no output MMAs; the commits below still arrive)
+                if (outputs) {
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(tm + TM_O, tm + TM_SB + kk * 8,
+                               smem_desc_sw128(qk + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), IDESC_Q, kk > 0);
+                }
+                mma_commit(&bars[B_M1BDONE]);
+                DBG_CLK(1, 2)
+                if (!(ok = wait_bar(&bars[B_UREADY], par, abort_flag))) break;
+                DBG_CLK(1, 3)
+                tc_fence_after();
+                // O2^T = U^T P'^T
+                if (outputs) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts(tm + TM_O2, tm + TM_UB + kk * 8,
+                               smem_desc_sw128(sbase + OFF_P + (c & 1) * 8192 + kk * 32, 16, 1024), IDESC_Q, kk > 0);
+                }
+                mma_commit(&bars[B_M2ADONE]);
+                DBG_CLK(1, 4)
+            }
+            if (ok && N > 0) wait_bar(&bars[B_M2ADONE], (N - 1) & 1, abort_flag);
+        }
+        __syncwarp();
+    } else if (warp == 2) {
+        // ========================== prep issuer ==========================
+        if (lane == 0) {
+            bool ok = true;
+            for (int c = 0; c < N && ok; ++c) {
+                const int buf = c & 1;
+                const uint32_t par = c & 1;
+                const uint32_t qk = sbase + OFF_QK + buf * QK_BYTES, vv = sbase + OFF_V + buf * V_BYTES;
+                DBG_CLK(2, 0)
+                if (!(ok = wait_bar(&bars[B_FULL0 + buf], (c >> 1) & 1, abort_flag))) break;
+                // the G region is free once the prep role has read W^T of the previous chunk
+                if (c > 0 && !(ok = wait_bar(&bars[B_PREPREADY], (c - 1) & 1, abort_flag))) break;
+                DBG_CLK(2, 1)
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
@@ -244,122 +428,68 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                            kk > 0);
                 }
                 mma_commit(&bars[B_GDONE]);
-            };
-            auto mma_UW = [&](int c) {
-                const int buf = c & 1;
-                const uint32_t qk = sbase + OFF_QK + buf * QK_BYTES, vv = sbase + OFF_V + buf * V_BYTES;
+                DBG_CLK(2, 2)
+                if (!(ok = wait_bar(&bars[B_TBREADY], par, abort_flag))) break;
+                DBG_CLK(2, 3)
                 tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ss(tm + TM_DU + buf * 64, smem_desc_sw128(vv + kk * 2048, 8192, 1024),
-                           smem_desc_sw128(sbase + OFF_TB + kk * 32, 16, 1024), IDESC_MN64, kk > 0);
+                // W^T first: the prep role is waiting for it
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_ss(tm + TM_G, smem_desc_sw128(qk + 8192 + kk * 2048, 16384, 1024),
                            smem_desc_sw128(sbase + OFF_TBG + kk * 32, 16, 1024), IDESC_MN64, kk > 0);
-                mma_commit(&bars[B_UWDONE]);
-            };
-            bool ok = true;
-            issue_loads(0);
-            if (N > 1) issue_loads(1);
-            ok = wait_bar(&bars[B_FULL0], 0, abort_flag);
-            if (ok) mma_G(0);
-            if (ok) ok = wait_bar(&bars[B_TBREADY], 0, abort_flag);
-            if (ok) mma_UW(0);
-            for (int c = 0; c < N && ok; ++c) {
-                const int buf = c & 1;
-                const uint32_t par = c & 1;
-                const uint32_t qk = sbase + OFF_QK + buf * QK_BYTES;
-                DBG_CLK(0, 0)
-                if (!(ok = wait_bar(&bars[B_PREPREADY], par, abort_flag))) break;
-                DBG_CLK(0, 1)
-                if (!(ok = wait_bar(&bars[B_SREADY], par, abort_flag))) break;
-                DBG_CLK(0, 2)
+                mma_commit(&bars[B_WDONE]);
+                // the DU region is free once the chain has read U^T of the previous chunk
+                if (c > 0 && !(ok = wait_bar(&bars[B_UREADY], (c - 1) & 1, abort_flag))) break;
                 tc_fence_after();
-                // U^T accumulates -S W^T onto Ut^T
+                if (kind != 2) {
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tm + TM_DU + buf * 64, tm + TM_SB + kk * 8,
-                           smem_desc_sw128(sbase + OFF_W + kk * 2048, 8192, 1024), IDESC_WNEG, 1);
-                DBG_CLK(0, 3)
-                if (c > 0 && !(ok = wait_bar(&bars[B_OFREE], (c - 1) & 1, abort_flag))) break;
-                DBG_CLK(0, 4)
-                tc_fence_after();
-                // O^T = S Qg^T
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tm + TM_O, tm + TM_SB + kk * 8,
-                           smem_desc_sw128(qk + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024), IDESC_Q, kk > 0);
-                mma_commit(&bars[B_M1DONE]);
-                DBG_CLK(0, 5)
-                if (c + 1 < N) {
-                    if (!(ok = wait_bar(&bars[B_FULL0 + ((c + 1) & 1)], ((c + 1) >> 1) & 1, abort_flag))) break;
-                    DBG_CLK(0, 6)
-                    mma_G(c + 1);
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss(tm + TM_DU, smem_desc_sw128(vv + kk * 2048, 8192, 1024),
+                               smem_desc_sw128(sbase + OFF_TB + kk * 32, 16, 1024), IDESC_MN64, kk > 0);
                 }
-                DBG_CLK(0, 7)
-                if (!(ok = wait_bar(&bars[B_UREADY], par, abort_flag))) break;
-                DBG_CLK(0, 8)
-                tc_fence_after();
-                // O^T += U^T P^T ;  S += (U^T diag(dl)) K
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(tm + TM_O, tm + TM_UB + kk * 8,
-                           smem_desc_sw128(sbase + OFF_P + buf * 8192 + kk * 32, 16, 1024), IDESC_Q, 1);
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(tm + TM_S, tm + TM_UDB + kk * 8, smem_desc_sw128(qk + 8192 + kk * 2048, 16384, 1024),
-                           IDESC_S, 1);
-                mma_commit(&bars[B_M2DONE]);
-                DBG_CLK(0, 9)
-                if (c + 2 < N) {
-                    if (!(ok = wait_bar(&bars[B_M2DONE], par, abort_flag))) break;
-                    DBG_CLK(0, 10)
-                    issue_loads(c + 2);
-                }
-                DBG_CLK(0, 11)
-                if (c + 1 < N) {
-                    if (!(ok = wait_bar(&bars[B_TBREADY], (c + 1) & 1, abort_flag))) break;
-                    DBG_CLK(0, 12)
-                    mma_UW(c + 1);
-                }
-                DBG_CLK(0, 13)
+                mma_commit(&bars[B_UTDONE]);
+                DBG_CLK(2, 4)
             }
-            // drain: the last MMAs must be complete before tensor memory is released
-            if (ok && N > 0) wait_bar(&bars[B_M2DONE], (N - 1) & 1, abort_flag);
+            if (ok && N > 0) wait_bar(&bars[B_UTDONE], (N - 1) & 1, abort_flag);
         }
         __syncwarp();
     } else if (warp >= kPrepWarp0 && warp < kChainWarp0) {
         // ============================== prep ==============================
         const int pt = tid - kPrepWarp0 * 32;     // 0..255
-        const int ch = (warp - kPrepWarp0) >> 2;  // column half of the TMEM epilogues
+        const int pw = warp - kPrepWarp0;         // 0..7
+        const int ch = pw >> 2;                   // column half of the TMEM epilogues
+        const int g8 = lane >> 2, t4 = lane & 3;  // MMA fragment coordinates
         float *g = reinterpret_cast<float *>(sm + OFF_PG);
         float *bet = g + 64, *gam = g + 128, *ea = g + 192, *eb = g + 256;
         float *Am = reinterpret_cast<float *>(sm + OFF_AM);
         float *Tm = reinterpret_cast<float *>(sm + OFF_TM);
-        float *Y = reinterpret_cast<float *>(sm + OFF_Y);
+        float *Xs = reinterpret_cast<float *>(sm + OFF_XS);
         bool ok = true;
+        // the upper triangles of the bf16 T tiles are never written below: zero both tiles once
+#pragma unroll
+        for (int it = 0; it < 4; ++it)
+            reinterpret_cast<uint4 *>(sm + OFF_TB)[pt + 256 * it] = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();
         // gates of the chunk being prepared, loaded one chunk ahead (threads pt < 64)
         float la_next = 0.f, be_next = 0.f;
-        if (pt < 64 && pt < T) {
-            const int64_t gi = ((int64_t)b * T + pt) * H + h;
+        if (pt < 64 && (int64_t)c0 * kC + pt < T) {
+            const int64_t gi = ((int64_t)b * T + (int64_t)c0 * kC + pt) * H + h;
             la_next = p.log_alpha[gi];
             be_next = p.beta[gi];
         }
         for (int c = 0; c < N && ok; ++c) {
             const int buf = c & 1;
             const uint32_t par = c & 1;
-            const int t0 = c * kC;
+            const int64_t t0 = (int64_t)(c0 + c) * kC;
             const int n = (T - t0 < kC) ? (int)(T - t0) : kC;
-            uint8_t *qk_ptr = sm + OFF_QK + buf * QK_BYTES;
-            DBG_CLK(1, 0)
+            DBG_CLK(3, 0)
             // ---- gates ----
             if (pt < 64) {
                 const float x = (pt < n) ? fmaxf(la_next, kLogAlphaFloor) : 0.f;
                 bet[pt] = (pt < n) ? be_next : 0.f;
                 const float s = chunk_cumsum(x, pt, prep_tmp, kBarPrep, kNumPrep);
                 g[pt] = s;
-                const int64_t tn = (int64_t)t0 + kC + pt;
+                const int64_t tn = t0 + kC + pt;
                 if (tn < T) {
                     const int64_t gi = ((int64_t)b * T + tn) * H + h;
                     la_next = p.log_alpha[gi];
@@ -374,17 +504,20 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 gam[pt] = expf(gt);
                 ea[pt] = expf(gt - cm);
                 eb[pt] = expf(cm - gt);
-                // e^{g_t - g_s} = e^{g_t - c} e^{c - g_s}, exact to a few ulp while every |g_t - c| < 80
-                const bool nr = __all_sync(0xffffffffu, fabsf(gt - cm) < 80.f);
+                // e^{g_t - g_s} = e^{g_t - c} e^{c - g_s}, exact to a few ulp; used while every
+                // |g_t - c| < 60, so that neither factor nor the output partial sums overflow
+                const bool nr = __all_sync(0xffffffffu, fabsf(gt - cm) < 60.f);
                 if (lane == 0) prep_flags[pt >> 5] = nr ? 1 : 0;
             }
             named_bar(kBarPrep, kNumPrep);
             const bool narrow = prep_flags[0] && prep_flags[1];
-            DBG_CLK(1, 1)
+            DBG_CLK(3, 1)
             if (!(ok = role_wait(&bars[B_GDONE], par, abort_flag, kBarPrep, kNumPrep))) break;
             tc_fence_after();
-            DBG_CLK(1, 2)
-            // ---- epilogue of G: rows 0..63 -> P (bf16), rows 64..127 -> A (fp32); columns split by half ----
+            DBG_CLK(3, 2)
+            // ---- epilogue of G: rows 0..63 -> P' (bf16), rows 64..127 -> A (fp32); columns split by half.
+            //      P'_ts = e^{c - g_s} (q_t . k_s) when the chunk is narrow (the output applies e^{g_t - c}),
+            //      else P_ts = e^{g_t - g_s} (q_t . k_s) ----
             {
                 const int m = (warp & 3) * 32 + lane;  // TMEM lane = row of [Q; K]
                 const int t = m & 63;
@@ -393,10 +526,14 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 tmem_ld32(tm + lb + TM_G + ch * 32, r);
                 tmem_wait_ld();
                 float d[32];
-                DBG_CLK(1, 3)
                 if (narrow) {
+                    if (m < 64) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) d[i] = at * eb[ch * 32 + i];
+                        for (int i = 0; i < 32; ++i) d[i] = eb[ch * 32 + i];
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) d[i] = at * eb[ch * 32 + i];
+                    }
                 } else {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) d[i] = expf(gt - g[ch * 32 + i]);
@@ -427,110 +564,109 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                         *reinterpret_cast<float4 *>(Am + t * LDM + ch * 32 + i) = make_float4(v[0], v[1], v[2], v[3]);
                     }
                 }
-                DBG_CLK(1, 4)
-                // Qg = diag(gamma) Q in place (MMA-G has consumed Q): a quarter row-block per thread
-                {
-                    const int qt = pt & 63, blk = (pt >> 6) & 1, qh = pt >> 7;
-                    uint4 *row = reinterpret_cast<uint4 *>(qk_ptr + blk * 16384 + qt * 128 + qh * 64);
-                    const float gm = gam[qt];
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc) {
-                        uint4 u = row[cc];
-                        scale_bf16x8(u, gm);
-                        row[cc] = u;
-                    }
-                }
             }
             __syncwarp();
             named_bar(kBarPrep, kNumPrep);
-            DBG_CLK(1, 5)
-            // ---- T = (I + A)^{-1}: 16x16 diagonal blocks (warps 4..7, a column per lane) ----
-            if (warp < kPrepWarp0 + 4 && lane < 16) {
-                const int o = (warp - kPrepWarp0) * 16;
+            DBG_CLK(3, 3)
+            // ---- T = (I + A)^{-1} ----
+            // (1) 16x16 diagonal blocks by substitution: role warps 0..3, a column per lane; warps 0 and 2
+            //     also zero the upper 16x16 block inside their 32x32 diagonal block
+            if (pw < 4 && lane < 16) {
+                const int o = pw * 16;
                 float x[16];
 #pragma unroll
                 for (int rr = 0; rr < 16; ++rr) {
-                    float acc = (rr == lane) ? 1.f : 0.f;
+                    float a0 = (rr == lane) ? 1.f : 0.f, a1 = 0.f;
 #pragma unroll
-                    for (int s = 0; s < rr; ++s) acc -= Am[(o + rr) * LDM + o + s] * x[s];
-                    x[rr] = acc;
+                    for (int s = 0; s + 1 < rr; s += 2) {
+                        a0 -= Am[(o + rr) * LDM + o + s] * x[s];
+                        a1 -= Am[(o + rr) * LDM + o + s + 1] * x[s + 1];
+                    }
+                    if (rr & 1) a0 -= Am[(o + rr) * LDM + o + rr - 1] * x[rr - 1];
+                    x[rr] = a0 + a1;
                 }
+                const int col = o + lane;
+                const float bc = bet[col], gbc = bc * gam[col];
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr) Tm[(o + rr) * LDM + o + lane] = x[rr];
+                for (int rr = 0; rr < 16; ++rr) {
+                    Tm[(o + rr) * LDM + col] = x[rr];
+                    const uint32_t off = sw128(o + rr, col >> 3) + (col & 7) * 2;
+                    *reinterpret_cast<__nv_bfloat16 *>(sm + OFF_TB + off) = __float2bfloat16_rn(x[rr] * bc);
+                    *reinterpret_cast<__nv_bfloat16 *>(sm + OFF_TBG + off) = __float2bfloat16_rn(x[rr] * gbc);
+                }
+                if ((pw & 1) == 0) {
+#pragma unroll
+                    for (int rr = 0; rr < 16; ++rr) Tm[(o + rr) * LDM + o + 16 + lane] = 0.f;
+                }
             }
             __syncwarp();
             named_bar(kBarPrep, kNumPrep);
-            DBG_CLK(1, 6)
-            // block rows I = 1..3:  T_IJ = -T_II sum_{K=J}^{I-1} A_IK T_KJ ; a thread per (J, row, 4 columns)
-            for (int I = 1; I < 4; ++I) {
-                if (pt < I * 64) {
-                    const int J = pt >> 6, rr = (pt >> 2) & 15, c4 = (pt & 3) * 4;
-                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                    for (int K = J; K < I; ++K) {
-                        const float *arow = Am + (16 * I + rr) * LDM + 16 * K;
-                        const float *tcol = Tm + (16 * K) * LDM + 16 * J + c4;
+            DBG_CLK(3, 4)
+            // (2) 16 -> 32: T_10 = -T_11 (A_10 T_00) inside each 32x32 diagonal block; one warp per
+            //     (block, 8-column tile); X goes through a per-warp scratch tile
+            if (pw < 4) {
+                const int q0 = (pw >> 1) * 32, n0 = (pw & 1) * 8;
+                float *xs = Xs + pw * 128;  // [16][8]
+                float dacc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                        for (int mm = 0; mm < 16; ++mm) {
-                            const float a = arow[mm];
-                            const float4 tv = *reinterpret_cast<const float4 *>(tcol + mm * LDM);
-                            acc.x = fmaf(a, tv.x, acc.x);
-                            acc.y = fmaf(a, tv.y, acc.y);
-                            acc.z = fmaf(a, tv.z, acc.z);
-                            acc.w = fmaf(a, tv.w, acc.w);
-                        }
-                    }
-                    *reinterpret_cast<float4 *>(Y + J * 256 + rr * 16 + c4) = acc;
+                for (int kk = 0; kk < 2; ++kk) {
+                    uint32_t a[4], bb[2];
+                    load_a(a, Am, LDM, q0 + 16, q0 + 8 * kk, g8, t4);
+                    load_b(bb, Tm, LDM, q0 + 8 * kk, q0 + n0, g8, t4);
+                    mma_tf32(dacc, a, bb);
                 }
-                named_bar(kBarPrep, kNumPrep);
-                if (pt < I * 64) {
-                    const int J = pt >> 6, rr = (pt >> 2) & 15, c4 = (pt & 3) * 4;
-                    const float *trow = Tm + (16 * I + rr) * LDM + 16 * I;
-                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                store_d(xs, 8, 0, 0, dacc, g8, t4);
+                __syncwarp();
+                float e[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int mm = 0; mm < 16; ++mm) {
-                        const float a = trow[mm];
-                        const float4 y = *reinterpret_cast<const float4 *>(Y + J * 256 + mm * 16 + c4);
-                        acc.x = fmaf(a, y.x, acc.x);
-                        acc.y = fmaf(a, y.y, acc.y);
-                        acc.z = fmaf(a, y.z, acc.z);
-                        acc.w = fmaf(a, y.w, acc.w);
-                    }
-                    *reinterpret_cast<float4 *>(Tm + (16 * I + rr) * LDM + 16 * J + c4) =
-                        make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
+                for (int kk = 0; kk < 2; ++kk) {
+                    uint32_t a[4], bb[2];
+                    load_a(a, Tm, LDM, q0 + 16, q0 + 16 + 8 * kk, g8, t4);
+                    load_b(bb, xs, 8, 8 * kk, 0, g8, t4);
+                    mma_tf32(e, a, bb);
                 }
-                named_bar(kBarPrep, kNumPrep);
-                DBG_CLK(1, 6 + I)
+                store_neg_d(Tm, LDM, q0 + 16, q0 + n0, e, g8, t4);
+                store_tb_pair(sm, q0 + 16 + g8, q0 + n0 + 2 * t4, -e[0], -e[1], bet, gam);
+                store_tb_pair(sm, q0 + 24 + g8, q0 + n0 + 2 * t4, -e[2], -e[3], bet, gam);
             }
-            // ---- T diag(beta) and T diag(beta gamma), bf16 K-major: a (tile, row, column half) per thread ----
+            named_bar(kBarPrep, kNumPrep);
+            DBG_CLK(3, 5)
+            // (3) 32 -> 64: X = A[32:64, 0:32] T[0:32, 0:32], then T[32:64, 0:32] = -T[32:64, 32:64] X;
+            //     one warp per (16-row, 8-column) tile; T is lower triangular, so zero k-steps are skipped
             {
-                const int t = pt & 63, with_gamma = (pt >> 6) & 1, hh = pt >> 7;
-                uint8_t *dst = sm + (with_gamma ? OFF_TBG : OFF_TB);
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    uint32_t pk[4];
-#pragma unroll
-                    for (int i = 0; i < 8; i += 2) {
-                        const int s = hh * 32 + cc * 8 + i;
-                        float v0 = (s <= t) ? Tm[t * LDM + s] * bet[s] : 0.f;
-                        float v1 = (s + 1 <= t) ? Tm[t * LDM + s + 1] * bet[s + 1] : 0.f;
-                        if (with_gamma) {
-                            v0 *= gam[s];
-                            v1 *= gam[s + 1];
-                        }
-                        pk[i >> 1] = pack_bf16x2(v0, v1);
-                    }
-                    *reinterpret_cast<uint4 *>(dst + sw128(t, hh * 4 + cc)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                const int mi = pw >> 2, ni = pw & 3;
+                float *x2 = Xs;  // [32][LDX2], reuses the 16->32 scratch (a barrier separates the two)
+                float dacc[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int kk = ni; kk < 4; ++kk) {
+                    uint32_t a[4], bb[2];
+                    load_a(a, Am, LDM, 32 + 16 * mi, 8 * kk, g8, t4);
+                    load_b(bb, Tm, LDM, 8 * kk, 8 * ni, g8, t4);
+                    mma_tf32(dacc, a, bb);
                 }
+                store_d(x2, LDX2, 16 * mi, 8 * ni, dacc, g8, t4);
+                named_bar(kBarPrep, kNumPrep);
+                float e[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int kk = 0; kk <= 2 * mi + 1; ++kk) {
+                    uint32_t a[4], bb[2];
+                    load_a(a, Tm, LDM, 32 + 16 * mi, 32 + 8 * kk, g8, t4);
+                    load_b(bb, x2, LDX2, 8 * kk, 8 * ni, g8, t4);
+                    mma_tf32(e, a, bb);
+                }
+                store_tb_pair(sm, 32 + 16 * mi + g8, 8 * ni + 2 * t4, -e[0], -e[1], bet, gam);
+                store_tb_pair(sm, 40 + 16 * mi + g8, 8 * ni + 2 * t4, -e[2], -e[3], bet, gam);
             }
             fence_proxy_async_smem();
             named_bar(kBarPrep, kNumPrep);
             if (pt == 0) arrive(&bars[B_TBREADY]);
-            DBG_CLK(1, 10)
-            // ---- W (bf16, MN-major rows i) from W^T in TMEM (MMA-1 of the previous chunk is done with W) ----
-            if (!(ok = role_wait(&bars[B_UWDONE], par, abort_flag, kBarPrep, kNumPrep))) break;
-            if (c > 0 && !(ok = role_wait(&bars[B_M1DONE], (c - 1) & 1, abort_flag, kBarPrep, kNumPrep))) break;
+            DBG_CLK(3, 6)
+            DBG_CLK(3, 7)
+            // ---- W (bf16, MN-major rows i) from W^T in TMEM (the MMAs of the previous chunk that read W
+            //      and the bf16 state copy are done) ----
+            if (!(ok = role_wait(&bars[B_WDONE], par, abort_flag, kBarPrep, kNumPrep))) break;
+            if (c > 0 && !(ok = role_wait(&bars[B_M1ADONE], (c - 1) & 1, abort_flag, kBarPrep, kNumPrep))) break;
+            if (c > 0 && !(ok = role_wait(&bars[B_M1BDONE], (c - 1) & 1, abort_flag, kBarPrep, kNumPrep))) break;
             tc_fence_after();
-            DBG_CLK(1, 11)
+            DBG_CLK(3, 8)
             {
                 const int i = (warp & 3) * 32 + lane;
                 uint32_t r[32];
@@ -550,17 +686,24 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             tc_fence_before();
             named_bar(kBarPrep, kNumPrep);
             if (pt == 0) arrive(&bars[B_PREPREADY]);
-            DBG_CLK(1, 12)
+            DBG_CLK(3, 9)
         }
     } else if (warp >= kChainWarp0) {
         // ============================== chain ==============================
         const int j = tid - kChainWarp0 * 32;  // TMEM lane / state row, 0..127
-        float *dl = reinterpret_cast<float *>(sm + OFF_CG);
-        float *gcs = dl + 64;  // [0] = gamma_C of the chunk
+        float *dl = reinterpret_cast<float *>(sm + OFF_CG);  // [2][64] e^{g_C - g_s} per chunk parity
+        float *f1 = dl + 128;                                // [2][64] gamma_t
+        float *f2 = dl + 256;                                // [2][64] e^{g_t - c} (narrow chunk) or 1
+        float *gcs = dl + 384;                               // [2]    gamma_C
+        int *chain_flags = reinterpret_cast<int *>(dl + 388); // [2]
         bool ok = true;
-        // S0 -> TMEM
+        // entry state -> TMEM: S0 (or zero) for the first segment, the prefix-scanned entry state for
+        // later segments, zero for transfer-B runs and the identity for transfer-M runs
         {
-            const float *src = p.S0 ? p.S0 + (bh * kD + j) * (int64_t)kD : nullptr;
+            const float *src = nullptr;
+            if (kind == 0)
+                src = (seg == 0) ? (p.S0 ? p.S0 + (bh * kD + j) * (int64_t)kD : nullptr)
+                                 : p.S_entry + ((bh * (p.nseg - 1) + seg - 1) * kD + j) * (int64_t)kD;
 #pragma unroll
             for (int piece = 0; piece < 4; ++piece) {
                 uint32_t r[32];
@@ -572,56 +715,101 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     r[i + 2] = __float_as_uint(v.z);
                     r[i + 3] = __float_as_uint(v.w);
                 }
+                if (kind == 2) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint((piece * 32 + i == j) ? 1.f : 0.f);
+                }
                 tmem_st32(tm + lb + TM_S + piece * 32, r);
             }
             tmem_wait_st();
         }
+        // chain gates of chunk cg into buffer cg & 1: dl_s = e^{g_C - g_s}, gamma_C and the output
+        // factors; the narrow test repeats the prep role's computation on identical values, so
+        // both roles take the same decision
         float la_next = 0.f;
-        if (j < 64 && j < T) la_next = p.log_alpha[((int64_t)b * T + j) * H + h];
+        if (j < 64 && (int64_t)c0 * kC + j < T) la_next = p.log_alpha[((int64_t)b * T + (int64_t)c0 * kC + j) * H + h];
+        auto chain_gates = [&](int cg) {
+            const int64_t t0g = (int64_t)(c0 + cg) * kC;
+            const int ng = (T - t0g < kC) ? (int)(T - t0g) : kC;
+            float *dlb = dl + (cg & 1) * 64;
+            float s = 0.f;
+            if (j < 64) {
+                const float x = (j < ng) ? fmaxf(la_next, kLogAlphaFloor) : 0.f;
+                s = chunk_cumsum(x, j, chain_tmp, kBarChain, kNumChain);
+                const int64_t tn = t0g + kC + j;
+                if (tn < T) la_next = p.log_alpha[((int64_t)b * T + tn) * H + h];
+                dlb[j] = s;
+            } else {
+                named_bar(kBarChain, kNumChain);  // the barrier inside chunk_cumsum
+            }
+            named_bar(kBarChain, kNumChain);
+            const float g63 = dlb[63], cm = dlb[31];
+            if (j < 64) {
+                const bool nr = __all_sync(0xffffffffu, fabsf(s - cm) < 60.f);
+                if ((j & 31) == 0) chain_flags[j >> 5] = nr ? 1 : 0;
+            }
+            named_bar(kBarChain, kNumChain);
+            const bool narrow = chain_flags[0] && chain_flags[1];
+            if (j < 64) {
+                dlb[j] = expf(g63 - s);
+                f1[(cg & 1) * 64 + j] = expf(s);
+                f2[(cg & 1) * 64 + j] = narrow ? expf(s - cm) : 1.f;
+            }
+            if (j == 0) gcs[cg & 1] = expf(g63);
+            named_bar(kBarChain, kNumChain);
+        };
+        // outputs of chunk cprev: o_t = f1_t O1_t + f2_t O2_t (thread j holds column j of both), staged
+        // as two 64x64 bf16 boxes in the TMA layout and written by two TMA stores
         auto write_out = [&](int cprev) {
-            const int64_t t0p = (int64_t)cprev * kC;
-            const int np = (T - t0p < kC) ? (int)(T - t0p) : kC;
-            __nv_bfloat16 *ob = p.out + (((int64_t)b * T + t0p) * H + h) * kD + j;
+            const float *f1c = f1 + (cprev & 1) * 64, *f2c = f2 + (cprev & 1) * 64;
+            if (j == 0) bulk_wait_read0();  // the previous chunk's stores have read the staging buffer
+            named_bar(kBarChain, kNumChain);
+            const int par = j & 1, colw = j - par;  // this lane writes column pair (colw, colw + 1)
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
-                uint32_t r[32];
-                tmem_ld32(tm + lb + TM_O + half * 32, r);
+                uint32_t r1[32], r2[32];
+                tmem_ld32(tm + lb + TM_O + half * 32, r1);
+                tmem_ld32(tm + lb + TM_O2 + half * 32, r2);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
+                for (int i = 0; i < 32; i += 2) {
                     const int t = half * 32 + i;
-                    if (t < np) ob[(int64_t)t * H * kD] = __float2bfloat16_rn(__uint_as_float(r[i]));
+                    const float o0 = f1c[t] * __uint_as_float(r1[i]) + f2c[t] * __uint_as_float(r2[i]);
+                    const float o1 = f1c[t + 1] * __uint_as_float(r1[i + 1]) + f2c[t + 1] * __uint_as_float(r2[i + 1]);
+                    // even lanes keep row t and take the neighbour's column; odd lanes keep row t+1
+                    const float send = par ? o0 : o1;
+                    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+                    const uint32_t word = par ? pack_bf16x2(recv, o1) : pack_bf16x2(o0, recv);
+                    const int row = t + par;
+                    *reinterpret_cast<uint32_t *>(sm + OFF_OST + (colw >> 6) * 8192 +
+                                                  sw128(row, (colw & 63) >> 3) + (colw & 7) * 2) = word;
                 }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar(kBarChain, kNumChain);
+            if (j == 0) {
+                tma_store_4d(&tm_o, sm + OFF_OST, 0, h, (c0 + cprev) * kC, b);
+                tma_store_4d(&tm_o, sm + OFF_OST + 8192, 64, h, (c0 + cprev) * kC, b);
+                bulk_commit();
             }
         };
+        chain_gates(0);
         for (int c = 0; c < N && ok; ++c) {
-            const int buf = c & 1;
             const uint32_t par = c & 1;
-            const int t0 = c * kC;
-            const int n = (T - t0 < kC) ? (int)(T - t0) : kC;
-            DBG_CLK(2, 0)
-            // ---- chain gates: dl_s = e^{g_C - g_s} and gamma_C ----
-            {
-                float s = 0.f;
-                if (j < 64) {
-                    const float x = (j < n) ? fmaxf(la_next, kLogAlphaFloor) : 0.f;
-                    s = chunk_cumsum(x, j, chain_tmp, kBarChain, kNumChain);
-                    const int64_t tn = (int64_t)t0 + kC + j;
-                    if (tn < T) la_next = p.log_alpha[((int64_t)b * T + tn) * H + h];
-                    dl[j] = s;
-                } else {
-                    named_bar(kBarChain, kNumChain);  // the barrier inside chunk_cumsum
-                }
-                named_bar(kBarChain, kNumChain);
-                const float g63 = dl[63];
-                named_bar(kBarChain, kNumChain);
-                if (j < 64) dl[j] = expf(g63 - s);
-                if (j == 0) gcs[0] = expf(g63);
-                named_bar(kBarChain, kNumChain);
+            const float *dlc = dl + (c & 1) * 64;
+            DBG_CLK(4, 0)
+            if (c > 0) {
+                // the state update of the previous chunk is complete, and its output MMA is done
+                // reading the bf16 state copy
+                if (!(ok = role_wait(&bars[B_M2BDONE], (c - 1) & 1, abort_flag, kBarChain, kNumChain))) break;
+                if (!(ok = role_wait(&bars[B_M1BDONE], (c - 1) & 1, abort_flag, kBarChain, kNumChain))) break;
+                tc_fence_after();
             }
+            DBG_CLK(4, 1)
             // ---- S -> bf16 operand copy; S <- gamma_C S ----
             {
-                const float gC = gcs[0];
+                const float gC = gcs[c & 1];
 #pragma unroll
                 for (int piece = 0; piece < 4; ++piece) {
                     uint32_t r[32];
@@ -641,30 +829,30 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 named_bar(kBarChain, kNumChain);
                 if (j == 0) arrive(&bars[B_SREADY]);
             }
-            DBG_CLK(2, 1)
+            DBG_CLK(4, 2)
             // ---- outputs of the previous chunk (frees the O accumulator) ----
             if (c > 0) {
-                write_out(c - 1);
-                tc_fence_before();
-                named_bar(kBarChain, kNumChain);
+                if (!(ok = role_wait(&bars[B_M2ADONE], (c - 1) & 1, abort_flag, kBarChain, kNumChain))) break;
+                tc_fence_after();
+                if (outputs) write_out(c - 1);  // ends with a chain barrier after the O reads
                 if (j == 0) arrive(&bars[B_OFREE]);
             }
-            DBG_CLK(2, 2)
-            if (!(ok = role_wait(&bars[B_M1DONE], par, abort_flag, kBarChain, kNumChain))) break;
+            DBG_CLK(4, 3)
+            if (!(ok = role_wait(&bars[B_M1ADONE], par, abort_flag, kBarChain, kNumChain))) break;
             tc_fence_after();
-            DBG_CLK(2, 3)
+            DBG_CLK(4, 4)
             // ---- U^T (accumulated in TMEM) -> bf16 U^T and bf16 U^T diag(dl) ----
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t u[32];
-                tmem_ld32(tm + lb + TM_DU + buf * 64 + half * 32, u);
+                tmem_ld32(tm + lb + TM_DU + half * 32, u);
                 tmem_wait_ld();
                 uint32_t pk[16], pd[16];
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
                     const float u0 = __uint_as_float(u[i]), u1 = __uint_as_float(u[i + 1]);
                     pk[i >> 1] = pack_bf16x2(u0, u1);
-                    pd[i >> 1] = pack_bf16x2(u0 * dl[half * 32 + i], u1 * dl[half * 32 + i + 1]);
+                    pd[i >> 1] = pack_bf16x2(u0 * dlc[half * 32 + i], u1 * dlc[half * 32 + i + 1]);
                 }
                 tmem_st16(tm + lb + TM_UB + half * 16, pk);
                 tmem_st16(tm + lb + TM_UDB + half * 16, pd);
@@ -673,14 +861,23 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             tc_fence_before();
             named_bar(kBarChain, kNumChain);
             if (j == 0) arrive(&bars[B_UREADY]);
-            DBG_CLK(2, 4)
-            if (!(ok = role_wait(&bars[B_M2DONE], par, abort_flag, kBarChain, kNumChain))) break;
-            tc_fence_after();
-            DBG_CLK(2, 5)
+            DBG_CLK(4, 5)
+            // gates of the next chunk, while this chunk's last MMAs run
+            if (c + 1 < N) chain_gates(c + 1);
+            DBG_CLK(4, 6)
         }
-        if (ok && N > 0) write_out(N - 1);
-        if (ok && p.S_final) {
-            float *dst = p.S_final + (bh * kD + j) * (int64_t)kD;
+        if (ok && N > 0) {
+            ok = role_wait(&bars[B_M2BDONE], (N - 1) & 1, abort_flag, kBarChain, kNumChain);
+            if (ok) ok = role_wait(&bars[B_M2ADONE], (N - 1) & 1, abort_flag, kBarChain, kNumChain);
+            tc_fence_after();
+            if (ok && outputs) write_out(N - 1);
+        }
+        float *dst = nullptr;
+        if (kind == 0)
+            dst = (seg == p.nseg - 1 && p.S_final) ? p.S_final + (bh * kD + j) * (int64_t)kD : nullptr;
+        else
+            dst = (kind == 1 ? p.Bw : p.Mw) + ((bh * (p.nseg - 1) + seg) * kD + j) * (int64_t)kD;
+        if (ok && dst) {
 #pragma unroll
             for (int piece = 0; piece < 4; ++piece) {
                 uint32_t r[32];
@@ -693,6 +890,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                                     __uint_as_float(r[i + 3]));
             }
         }
+        if (j == 0) bulk_wait0();  // every output store has completed
     }
 
     tc_fence_before();
@@ -701,6 +899,65 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tm, 512);
+    }
+}
+
+// ---------------------------------------------------------------- segment prefix
+// Entry states of segments 1..nseg-1 from the segment transfers, in float32:
+// S_{p+1} = S_p M_p + B_p with S_0 = S0 (or zero).  Rows of the state are
+// independent, so one CTA owns 16 rows of one (b, h) and walks the segments
+// in order; M_p is staged in shared memory for each step.
+constexpr int kPrefixRows = 16;
+constexpr int kPrefixThreads = 256;
+constexpr int kPrefixLd = kD + 4;
+constexpr size_t kPrefixSmem = (size_t)(kD * kPrefixLd + kPrefixRows * kPrefixLd) * sizeof(float);
+
+__global__ void __launch_bounds__(kPrefixThreads)
+seg_prefix_kernel(const float *__restrict__ S0, const float *__restrict__ Bw, const float *__restrict__ Mw,
+                  float *__restrict__ S_entry, int nseg) {
+    extern __shared__ float psm[];
+    float *Ms = psm;                   // [128][kPrefixLd]
+    float *Sr = psm + kD * kPrefixLd;  // [16][kPrefixLd]
+    const int64_t bh = blockIdx.x;
+    const int r0 = blockIdx.y * kPrefixRows;
+    const int tid = threadIdx.x;
+    const int r = tid >> 4, c = (tid & 15) * 8;  // this thread's row and 8 columns
+    for (int i = tid; i < kPrefixRows * (kD / 4); i += kPrefixThreads) {
+        const int rr = i / (kD / 4), cc = (i % (kD / 4)) * 4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (S0) v = *reinterpret_cast<const float4 *>(S0 + (bh * kD + r0 + rr) * (int64_t)kD + cc);
+        *reinterpret_cast<float4 *>(Sr + rr * kPrefixLd + cc) = v;
+    }
+    for (int q = 0; q < nseg - 1; ++q) {
+        const float *M = Mw + (bh * (nseg - 1) + q) * (int64_t)kD * kD;
+        const float *Bq = Bw + ((bh * (nseg - 1) + q) * kD + r0) * (int64_t)kD;
+        __syncthreads();
+        for (int i = tid; i < kD * (kD / 4); i += kPrefixThreads) {
+            const int rr = i / (kD / 4), cc = (i % (kD / 4)) * 4;
+            *reinterpret_cast<float4 *>(Ms + rr * kPrefixLd + cc) = *reinterpret_cast<const float4 *>(M + rr * kD + cc);
+        }
+        __syncthreads();
+        float acc[8];
+        const float4 b0 = *reinterpret_cast<const float4 *>(Bq + r * kD + c);
+        const float4 b1 = *reinterpret_cast<const float4 *>(Bq + r * kD + c + 4);
+        acc[0] = b0.x; acc[1] = b0.y; acc[2] = b0.z; acc[3] = b0.w;
+        acc[4] = b1.x; acc[5] = b1.y; acc[6] = b1.z; acc[7] = b1.w;
+#pragma unroll 4
+        for (int k = 0; k < kD; ++k) {
+            const float a = Sr[r * kPrefixLd + k];
+            const float4 m0 = *reinterpret_cast<const float4 *>(Ms + k * kPrefixLd + c);
+            const float4 m1 = *reinterpret_cast<const float4 *>(Ms + k * kPrefixLd + c + 4);
+            acc[0] = fmaf(a, m0.x, acc[0]); acc[1] = fmaf(a, m0.y, acc[1]);
+            acc[2] = fmaf(a, m0.z, acc[2]); acc[3] = fmaf(a, m0.w, acc[3]);
+            acc[4] = fmaf(a, m1.x, acc[4]); acc[5] = fmaf(a, m1.y, acc[5]);
+            acc[6] = fmaf(a, m1.z, acc[6]); acc[7] = fmaf(a, m1.w, acc[7]);
+        }
+        __syncthreads();  // every thread is done reading this step's rows
+        *reinterpret_cast<float4 *>(Sr + r * kPrefixLd + c) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4 *>(Sr + r * kPrefixLd + c + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        float *dst = S_entry + ((bh * (nseg - 1) + q) * kD + r0 + r) * (int64_t)kD + c;
+        *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4 *>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
 }
 
@@ -752,10 +1009,44 @@ bool fwd_tc_supported(const FwdProblem &p) {
            p.B <= (int64_t)INT32_MAX && p.H <= (int64_t)INT32_MAX;
 }
 
-cudaError_t launch_fwd_tc(const FwdProblem &p, cudaStream_t stream) {
-    CUtensorMap mq, mk, mv;
+// Segments per (b, h): the count minimising a wave model of the two parallel
+// passes (transfers: 2 (nseg - 1) CTAs per head; outputs: nseg CTAs per head,
+// each over ceil(chunks / nseg) chunks).  GDN_SEGMENTS overrides the choice.
+int fwd_tc_segments(const FwdProblem &p, int sm_count) {
+    const int64_t chunks = (p.T + kC - 1) / kC, heads = p.B * p.H;
+    if (chunks <= 0 || heads <= 0) return 1;
+    const char *env = getenv("GDN_SEGMENTS");
+    if (env && atoi(env) >= 1) {
+        int want = atoi(env);
+        if (want > chunks) want = (int)chunks;
+        const int64_t len = (chunks + want - 1) / want;
+        return (int)((chunks + len - 1) / len);
+    }
+    auto waves = [&](int64_t ctas) { return (ctas + sm_count - 1) / sm_count; };
+    int best = 1;
+    int64_t best_cost = waves(heads) * chunks;
+    for (int nseg = 2; nseg <= 64; ++nseg) {
+        const int64_t len = (chunks + nseg - 1) / nseg;
+        if (len < 4) break;
+        const int64_t real = (chunks + len - 1) / len;
+        const int64_t cost = (waves(2 * heads * (real - 1)) + waves(heads * real)) * len;
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = (int)real;
+        }
+    }
+    return best;
+}
+
+size_t fwd_tc_workspace_bytes(const FwdProblem &p, int nseg) {
+    if (nseg <= 1) return 0;
+    return (size_t)3 * (size_t)(p.B * p.H) * (size_t)(nseg - 1) * kD * kD * sizeof(float);
+}
+
+cudaError_t launch_fwd_tc(const FwdProblem &p, int nseg, void *workspace, cudaStream_t stream) {
+    CUtensorMap mq, mk, mv, mo;
     if (!make_map(&mq, p.q, p.B, p.T, p.H) || !make_map(&mk, p.k, p.B, p.T, p.H) ||
-        !make_map(&mv, p.v, p.B, p.T, p.H))
+        !make_map(&mv, p.v, p.B, p.T, p.H) || !make_map(&mo, p.out, p.B, p.T, p.H))
         return cudaErrorInvalidValue;
     static std::atomic<uint64_t> configured{0};
     int dev = 0;
@@ -774,7 +1065,39 @@ cudaError_t launch_fwd_tc(const FwdProblem &p, cudaStream_t stream) {
     a.S_final = p.S_final;
     a.T = p.T;
     a.H = p.H;
-    fwd_tc_kernel<<<(unsigned)(p.B * p.H), kThreadsTc, SMEM_TC, stream>>>(mq, mk, mv, a);
+    const int64_t chunks = (p.T + kC - 1) / kC, heads = p.B * p.H;
+    if (nseg < 1) nseg = 1;
+    a.seg_len = (int)((chunks + nseg - 1) / nseg);
+    a.nseg = (int)((chunks + a.seg_len - 1) / a.seg_len);
+    a.S_entry = nullptr;
+    a.Bw = a.Mw = nullptr;
+    if (a.nseg > 1) {
+        if (!workspace) return cudaErrorInvalidValue;
+        const size_t per = (size_t)heads * (a.nseg - 1) * kD * kD;
+        a.Bw = static_cast<float *>(workspace);
+        a.Mw = a.Bw + per;
+        float *entry = a.Mw + per;
+        a.S_entry = entry;
+        // phase 1: segment transfers of segments 0..nseg-2
+        a.mode = 1;
+        fwd_tc_kernel<<<(unsigned)(heads * (a.nseg - 1) * 2), kThreadsTc, SMEM_TC, stream>>>(mq, mk, mv, mo, a);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        // phase 2: entry states of segments 1..nseg-1
+        static std::atomic<uint64_t> pconf{0};
+        if (!(pconf.load() & bit)) {
+            e = cudaFuncSetAttribute(seg_prefix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPrefixSmem);
+            if (e != cudaSuccess) return e;
+            pconf.fetch_or(bit);
+        }
+        seg_prefix_kernel<<<dim3((unsigned)heads, kD / kPrefixRows), kPrefixThreads, kPrefixSmem, stream>>>(
+            p.S0, a.Bw, a.Mw, entry, a.nseg);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    // outputs of every segment from its entry state
+    a.mode = 0;
+    fwd_tc_kernel<<<(unsigned)(heads * a.nseg), kThreadsTc, SMEM_TC, stream>>>(mq, mk, mv, mo, a);
     return cudaGetLastError();
 }
 

@@ -215,10 +215,19 @@ int gdn_forward(const void *q, const void *k, const void *v, const float *log_al
                      : cudaMemsetAsync(p.S_final, 0, (size_t)nstate, stream);
         }
     } else {
-        if (forced_path() != FwdPath::Simt && gdn::fwd_tc_supported(p))
-            e = gdn::launch_fwd_tc(p, stream);
-        else
+        if (forced_path() != FwdPath::Simt && gdn::fwd_tc_supported(p)) {
+            const int nseg = gdn::fwd_tc_segments(p, info.sm_count);
+            const size_t ws_bytes = gdn::fwd_tc_workspace_bytes(p, nseg);
+            void *ws = nullptr;
+            if (ws_bytes > 0 && cudaMallocAsync(&ws, ws_bytes, stream) != cudaSuccess) {
+                cudaGetLastError();
+                return GDN_ERR_ALLOC;
+            }
+            e = gdn::launch_fwd_tc(p, nseg, ws, stream);
+            if (ws) cudaFreeAsync(ws, stream);
+        } else {
             e = gdn::launch_fwd_simt(p, info.sm_count, stream);
+        }
     }
     if (e != cudaSuccess) {
         cudaGetLastError();

@@ -37,7 +37,12 @@ cudaError_t launch_decode(const DecodeProblem &p, cudaStream_t stream);
 cudaError_t launch_fwd_simt(const FwdProblem &p, int sm_count, cudaStream_t stream);
 
 // fwd_tc.cu -- tcgen05 chunkwise forward: bf16, dk = dv = 128, chunk = 64.
+// Long sequences with few (b, h) are cut into segments: a transfer pass, a
+// float32 prefix over segments and an output pass, with
+// fwd_tc_workspace_bytes() of scratch (device memory, caller-provided).
 bool fwd_tc_supported(const FwdProblem &p);
-cudaError_t launch_fwd_tc(const FwdProblem &p, cudaStream_t stream);
+int fwd_tc_segments(const FwdProblem &p, int sm_count);
+size_t fwd_tc_workspace_bytes(const FwdProblem &p, int nseg);
+cudaError_t launch_fwd_tc(const FwdProblem &p, int nseg, void *workspace, cudaStream_t stream);
 
 }  // namespace gdn

@@ -182,3 +182,21 @@ def test_results_are_deterministic():
     a = run_gpu(inp, 64)
     b = run_gpu(inp, 64)
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("nseg", [2, 3, 5])
+def test_segmented_long_sequence(monkeypatch, nseg):
+    """Sequence cut into segments: transfer pass, float32 prefix over segments, output pass.
+    A ragged last chunk and a non-zero initial state are included."""
+    monkeypatch.setenv("GDN_SEGMENTS", str(nseg))
+    inp = forward_inputs(1, 1000, 2, 128, 128, "bf16", seed=61 + nseg, s0_std=0.1, alpha_mu=-3.0)
+    check(inp, "bf16", 64, label="segments=%d" % nseg)
+
+
+def test_segmented_fast_decay(monkeypatch):
+    """Segments with fast decay (alpha ~ 0.45) and resets inside segments."""
+    monkeypatch.setenv("GDN_SEGMENTS", "4")
+    inp = forward_inputs(2, 777, 2, 128, 128, "bf16", seed=67, s0_std=0.1)
+    inp["log_alpha"][0, 300, 1] = float("-inf")
+    inp["log_alpha"][1, 500:505, 0] = -30.0
+    check(inp, "bf16", 64, label="segments fast decay")
