@@ -32,7 +32,7 @@ GDN_BF16 = 1
 STATUS = {
     0: "GDN_OK", 1: "GDN_ERR_NULL_PTR", 2: "GDN_ERR_INVALID_SIZE", 3: "GDN_ERR_UNSUPPORTED",
     4: "GDN_ERR_MISALIGNED", 5: "GDN_ERR_ALLOC", 6: "GDN_ERR_LAUNCH", 7: "GDN_ERR_DEVICE_TIMEOUT",
-    8: "GDN_ERR_ALIAS", 9: "GDN_ERR_DEVICE",
+    8: "GDN_ERR_ALIAS", 9: "GDN_ERR_DEVICE", 10: "GDN_ERR_SCRATCH_LIMIT",
 }
 
 EXPORTS = ("gdn_forward", "gdn_decode_step", "gdn_status_string", "gdn_version")

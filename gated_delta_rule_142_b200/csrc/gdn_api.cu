@@ -152,6 +152,7 @@ const char *gdn_status_string(int status) {
         case GDN_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
         case GDN_ERR_ALIAS: return "an output buffer overlaps an input it must not overlap";
         case GDN_ERR_DEVICE: return "no usable sm_100 CUDA device is current";
+        case GDN_ERR_SCRATCH_LIMIT: return "problem needs more scratch than GDN_NOALLOC_SCRATCH_BYTES (no-allocation entry point)";
         default: return "unknown gdn status";
     }
 }

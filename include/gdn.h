@@ -70,7 +70,9 @@ typedef enum {
     GDN_ERR_LAUNCH = 6,         /* a kernel launch or an enqueued copy failed          */
     GDN_ERR_DEVICE_TIMEOUT = 7, /* a bounded device-side wait gave up                  */
     GDN_ERR_ALIAS = 8,          /* an output overlaps an input it must not overlap     */
-    GDN_ERR_DEVICE = 9          /* no usable CUDA device / not an sm_100 device        */
+    GDN_ERR_DEVICE = 9,         /* no usable CUDA device / not an sm_100 device        */
+    GDN_ERR_SCRATCH_LIMIT = 10  /* gdn_forward_noalloc: problem needs more scratch than
+                                   GDN_NOALLOC_SCRATCH_BYTES                            */
 } gdn_status;
 
 /*
@@ -125,6 +127,40 @@ int gdn_forward(const void *q, const void *k, const void *v, const float *log_al
 int gdn_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
                     const float *beta, float *S, void *out, int64_t B, int64_t H, int64_t dk,
                     int64_t dv, void *stream, int dtype);
+
+/*
+ * gdn_forward_noalloc -- gdn_forward for callers that cannot allocate device
+ * memory during a call.
+ *
+ * The paper has no counterpart to this entry point; it exists for callers
+ * whose device memory is not theirs to allocate mid-call. Examples: a framework
+ * whose caching allocator already owns the device heap, a serving loop that
+ * must not enter the driver's allocator on its hot path, or code without
+ * permission to grow the process's device footprint.
+ *
+ * Arguments, layouts, results and validation are those of gdn_forward, with
+ * these differences:
+ *   - every pointer must be device (or managed) memory: host buffers, which
+ *     gdn_forward stages through temporary device buffers, are rejected with
+ *     GDN_ERR_UNSUPPORTED;
+ *   - the scratch that long sequences with few heads need (segment transfers
+ *     and entry states) lives in one library-owned device array of
+ *     GDN_NOALLOC_SCRATCH_BYTES, which every GPU that loads the library holds
+ *     until the process exits; a problem that needs more than that returns
+ *     GDN_ERR_SCRATCH_LIMIT before anything is enqueued;
+ *   - no cudaMalloc, cudaMallocAsync, cudaFree or other allocating routine is
+ *     called.
+ * The first call on a device looks up the array's device address on that
+ * device; make that first call before any stream capture. All calls share the
+ * array and it keeps the last call's contents (nothing in it needs to start at
+ * zero); calls whose executions overlap on the GPU race on it, so order them
+ * on one stream or with events.
+ */
+#define GDN_NOALLOC_SCRATCH_BYTES (32 * 1024 * 1024)
+int gdn_forward_noalloc(const void *q, const void *k, const void *v, const float *log_alpha,
+                        const float *beta, const float *S0, void *out, float *S_final, int64_t B,
+                        int64_t T, int64_t H, int64_t dk, int64_t dv, int64_t chunk, void *stream,
+                        int dtype);
 
 /* Static, NUL-terminated description of a gdn_status value. */
 const char *gdn_status_string(int status);
