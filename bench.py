@@ -270,7 +270,7 @@ def run_gdn(args, world, rank, local):
     nbytes = fwd_bytes(w.B, w.T, w.H, w.dk, w.dv, es, w.s0_std is not None, True)
     tflops = flop / (ms_step / 1e3) / 1e12
     gbs = nbytes / (ms_step / 1e3) / 1e9
-    launches_per_fwd = 1
+    scratch_bytes, launches_per_fwd = gdn.forward_plan(w.B, w.T, w.H, w.dk, w.dv, w.chunk, d["q"].dtype)
 
     # ---- decode: 1024 consecutive single-token steps, each its own launch ----
     dec = None
@@ -344,7 +344,8 @@ def run_gdn(args, world, rank, local):
                          "frac": tflops / peaks["bf16_tflops"], "traffic": None, "peak_kind": peak_kind,
                          "flop_per_launch": flop, "hbm_frac": gbs / peaks["hbm_gbs"]},
             "decode": dec, "e2e": e2e, "cpu_baseline": cpu, "clocks": clocks,
-            "gpu_launches": args.steps * launches_per_fwd,
+            "gpu_launches": args.steps * launches_per_fwd, "forward_launches_per_step": launches_per_fwd,
+            "forward_scratch_bytes": scratch_bytes,
         }
         print(json.dumps(line), flush=True)
     return 0

@@ -35,7 +35,8 @@ STATUS = {
     8: "GDN_ERR_ALIAS", 9: "GDN_ERR_DEVICE", 10: "GDN_ERR_SCRATCH_LIMIT",
 }
 
-EXPORTS = ("gdn_forward", "gdn_decode_step", "gdn_status_string", "gdn_version")
+EXPORTS = ("gdn_forward", "gdn_decode_step", "gdn_forward_plan", "gdn_status_string", "gdn_version",
+           "gdn_forward_noalloc")
 
 
 class GdnError(RuntimeError):
@@ -65,6 +66,8 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_version.argtypes = []
     lib.gdn_version.restype = ctypes.c_int
+    lib.gdn_forward_plan.argtypes = [i64] * 6 + [ctypes.c_int, ctypes.POINTER(i64), ctypes.POINTER(ctypes.c_int)]
+    lib.gdn_forward_plan.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -139,6 +142,17 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.
     if st != 0:
         raise GdnError(st, "gdn_forward")
     return out, S_final
+
+
+def forward_plan(B: int, T: int, H: int, dk: int, dv: int, chunk: int = 64, dtype=torch.bfloat16):
+    """(scratch bytes, kernel launches) that gdn_forward takes for these sizes on the current device."""
+    lib = load()
+    code = GDN_BF16 if dtype == torch.bfloat16 else GDN_F32
+    scratch, launches = ctypes.c_int64(0), ctypes.c_int(0)
+    st = lib.gdn_forward_plan(B, T, H, dk, dv, int(chunk), code, ctypes.byref(scratch), ctypes.byref(launches))
+    if st != 0:
+        raise GdnError(st, "gdn_forward_plan")
+    return scratch.value, launches.value
 
 
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,

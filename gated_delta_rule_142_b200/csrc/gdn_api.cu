@@ -239,6 +239,34 @@ int gdn_forward(const void *q, const void *k, const void *v, const float *log_al
     return GDN_OK;
 }
 
+int gdn_forward_plan(int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv, int64_t chunk, int dtype,
+                     int64_t *scratch_bytes, int *launches) {
+    if (scratch_bytes) *scratch_bytes = 0;
+    if (launches) *launches = 0;
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
+    if (B < 0 || T < 0 || H < 0 || dk < 0 || dv < 0 || chunk < 0) return GDN_ERR_INVALID_SIZE;
+    if (!supported_dim(dk) || !supported_dim(dv) || !supported_chunk(chunk)) return GDN_ERR_UNSUPPORTED;
+    int64_t ntok;
+    if (!mul3(B, T, H, &ntok)) return GDN_ERR_INVALID_SIZE;
+    if (B * H == 0 || T == 0) return GDN_OK;
+    DeviceInfo info;
+    if (int st = device_info(&info)) return st;
+    FwdProblem p;
+    p.q = p.k = p.v = nullptr;
+    p.log_alpha = p.beta = p.S0 = nullptr;
+    p.out = nullptr;
+    p.S_final = nullptr;
+    p.B = B; p.T = T; p.H = H; p.dk = dk; p.dv = dv; p.chunk = chunk; p.dtype = dtype;
+    if (forced_path() != FwdPath::Simt && gdn::fwd_tc_supported(p)) {
+        const int nseg = gdn::fwd_tc_segments(p, info.sm_count);
+        if (scratch_bytes) *scratch_bytes = (int64_t)gdn::fwd_tc_workspace_bytes(p, nseg);
+        if (launches) *launches = nseg > 1 ? 3 : 1;
+    } else if (launches) {
+        *launches = 1;
+    }
+    return GDN_OK;
+}
+
 int gdn_decode_step(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                     float *S, void *out, int64_t B, int64_t H, int64_t dk, int64_t dv, void *stream_, int dtype) {
     if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;

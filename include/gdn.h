@@ -111,6 +111,18 @@ int gdn_forward(const void *q, const void *k, const void *v, const float *log_al
                 int dtype);
 
 /*
+ * gdn_forward_plan -- what a gdn_forward call with these sizes will do on the
+ * current device, without doing it: *scratch_bytes receives the device scratch
+ * it takes from the stream-ordered allocator (segment transfers and entry
+ * states; 0 when the sequence is not split into segments, and excluding host
+ * staging), *launches the number of kernels it launches (0 for empty
+ * problems).  Either output pointer may be NULL.  Returns the status the
+ * argument checks of gdn_forward would return, or GDN_ERR_DEVICE.
+ */
+int gdn_forward_plan(int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv, int64_t chunk, int dtype,
+                     int64_t *scratch_bytes, int *launches);
+
+/*
  * gdn_decode_step -- one token for every (b, h), state updated in place.
  *
  * Same equation as gdn_forward with T = 1 (source: the Sec. 3.3 gated-delta

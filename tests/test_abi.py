@@ -138,3 +138,12 @@ def test_binding_validates_shapes_and_dtypes(lib):
         gdn.forward(q.double(), q.double(), q.double(), torch.zeros(1, 4, 2), torch.zeros(1, 4, 2))
     with pytest.raises(ValueError):
         gdn.forward(q.transpose(1, 2), q, q, torch.zeros(1, 4, 2), torch.zeros(1, 4, 2))
+
+
+def test_forward_plan_argument_checks(lib):
+    s, n = ctypes.c_int64(-1), ctypes.c_int(-1)
+    assert lib.gdn_forward_plan(1, 8, 2, 48, 16, 16, 0, ctypes.byref(s), ctypes.byref(n)) == UNSUP
+    assert (s.value, n.value) == (0, 0)
+    assert lib.gdn_forward_plan(-1, 8, 2, 16, 16, 16, 0, None, None) == SIZE
+    assert lib.gdn_forward_plan(0, 8, 2, 16, 16, 16, 1, ctypes.byref(s), ctypes.byref(n)) == OK
+    assert (s.value, n.value) == (0, 0)

@@ -200,3 +200,13 @@ def test_segmented_fast_decay(monkeypatch):
     inp["log_alpha"][0, 300, 1] = float("-inf")
     inp["log_alpha"][1, 500:505, 0] = -30.0
     check(inp, "bf16", 64, label="segments fast decay")
+
+
+def test_forward_plan_reports_scratch_and_launches():
+    """The planning query agrees with what the forward does: one launch and no scratch for many heads,
+    three launches and segment scratch for a long sequence with few heads."""
+    s, n = gdn.forward_plan(8, 2048, 16, 128, 128, 64)
+    assert (s, n) == (0, 1)
+    s, n = gdn.forward_plan(1, 65536, 16, 128, 128, 64)
+    assert n == 3 and s > 0 and s % (3 * 16 * 128 * 128 * 4) == 0
+    assert gdn.forward_plan(1, 100, 2, 64, 64, 32) == (0, 1)  # CUDA-core path
