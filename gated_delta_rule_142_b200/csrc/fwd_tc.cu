@@ -25,15 +25,15 @@
 // The state S stays in tensor memory in float32 for the whole sequence; its
 // bf16 operand copy is rewritten from it every chunk.
 //
-// Warp roles (512 threads).  One thread issuing tcgen05.mma sustains about
+// Warp roles (640 threads).  One thread issuing tcgen05.mma sustains about
 // one MMA per ~90 cycles, more than an M128xN64xK16 MMA takes to execute, so
 // the MMAs are issued by three threads, one per independent stream:
 //   warp 0      chain issuer: TMA loads, U^T and S updates (the critical path)
 //   warp 1      output issuer: O1^T = S Q^T, O2^T = U^T P'^T
 //   warp 2      prep issuer: G, Ut^T, W^T
 //   warps 4-11  prep for chunk c+1 (256 threads) while the chain runs chunk c
-//   warps 12-15 chain: state conversion, U^T epilogue, outputs (thread j owns
-//               TMEM lane j, i.e. state row j)
+//   warps 12-19 chain: state conversion, U^T epilogue, outputs (two warps per
+//               TMEM lane quadrant; a thread owns state row j and a column half)
 //   warp 3      idle
 // Roles hand work to each other through mbarriers (tcgen05.commit for MMA
 // completion, single-thread arrivals after a named barrier otherwise); every
@@ -59,9 +59,9 @@ using namespace sm100;
 
 constexpr int kC = 64;
 constexpr int kD = 128;
-constexpr int kThreadsTc = 512;
+constexpr int kThreadsTc = 640;
 constexpr int kPrepWarp0 = 4, kNumPrep = 256;
-constexpr int kChainWarp0 = 12, kNumChain = 128;
+constexpr int kChainWarp0 = 12, kNumChain = 256;
 constexpr int kBarPrep = 1, kBarChain = 2;  // named barrier ids (0 is __syncthreads)
 
 // Shared memory map (bytes, from a 1024-aligned base).
@@ -78,12 +78,12 @@ constexpr uint32_t OFF_AM = 147456;      // 17 KB  A  fp32 [64][LDM]
 constexpr uint32_t OFF_TM = 164864;      // 17 KB  T  fp32 [64][LDM]
 constexpr uint32_t OFF_XS = 182272;      // 5 KB   merge scratch: 4 x [16][8] (16->32), then [32][LDX2] (32->64)
 constexpr int LDX2 = 40;
-constexpr uint32_t OFF_PG = 187392;      // prep gates: g, beta, gamma, e^{g-c}, e^{c-g} (64 each)
-constexpr uint32_t OFF_CG = 188672;      // chain gates per chunk parity: dl[2][64], f1[2][64], f2[2][64], gamma_C[2]
-constexpr uint32_t OFF_OST = 190464;     // 16 KB  output staging: two [64 t][64 d] bf16 boxes, 128-byte swizzle
-constexpr uint32_t OFF_BARS = 206848;    // mbarriers
-constexpr uint32_t OFF_MISC = 206976;    // tmem slot, abort flag, scan scratch
-constexpr uint32_t SMEM_TC = 207040 + 1024;
+constexpr uint32_t OFF_PG = 187392;      // prep gates per chunk parity: g, beta, gamma, e^{g-c}, e^{c-g} (2 x 5 x 64)
+constexpr uint32_t OFF_CG = 189952;      // chain gates per chunk parity: dl[2][64], f1[2][64], f2[2][64], gamma_C[2]
+constexpr uint32_t OFF_OST = 192512;     // 16 KB  output staging: two [64 t][64 d] bf16 boxes, 128-byte swizzle
+constexpr uint32_t OFF_BARS = 208896;    // mbarriers
+constexpr uint32_t OFF_MISC = 209024;    // tmem slot, abort flag, scan scratch
+constexpr uint32_t SMEM_TC = 209088 + 1024;
 constexpr uint32_t kTxBytes = 3 * 2 * 8192;  // Q, K, V: two 8 KB boxes each
 
 // TMEM column map (512 columns).
@@ -188,17 +188,6 @@ __device__ __forceinline__ void arrive(uint64_t *bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-__device__ __forceinline__ void scale_bf16x8(uint4 &u, float f) {
-    uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        __nv_bfloat162 v = *reinterpret_cast<__nv_bfloat162 *>(&w[i]);
-        float2 x = __bfloat1622float2(v);
-        w[i] = pack_bf16x2(x.x * f, x.y * f);
-    }
-    u = make_uint4(w[0], w[1], w[2], w[3]);
-}
-
 // ---- warp-level TF32 MMA (m16n8k8, fp32 accumulate) for the 64x64 inverse ----
 // Fragment ownership, g = lane / 4, t = lane % 4:
 //   A 16x8: a0 (g, t), a1 (g+8, t), a2 (g, t+4), a3 (g+8, t+4)
@@ -274,8 +263,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + OFF_MISC + 4);
     float *prep_tmp = reinterpret_cast<float *>(sm + OFF_MISC + 8);
-    int *prep_flags = reinterpret_cast<int *>(sm + OFF_MISC + 16);  // [2]
-    float *chain_tmp = reinterpret_cast<float *>(sm + OFF_MISC + 24);
+    int *prep_flags = reinterpret_cast<int *>(sm + OFF_MISC + 16);  // [2 parities][2 warps]
+    float *chain_tmp = reinterpret_cast<float *>(sm + OFF_MISC + 32);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t T = p.T, H = p.H;
@@ -459,8 +448,6 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         const int pw = warp - kPrepWarp0;         // 0..7
         const int ch = pw >> 2;                   // column half of the TMEM epilogues
         const int g8 = lane >> 2, t4 = lane & 3;  // MMA fragment coordinates
-        float *g = reinterpret_cast<float *>(sm + OFF_PG);
-        float *bet = g + 64, *gam = g + 128, *ea = g + 192, *eb = g + 256;
         float *Am = reinterpret_cast<float *>(sm + OFF_AM);
         float *Tm = reinterpret_cast<float *>(sm + OFF_TM);
         float *Xs = reinterpret_cast<float *>(sm + OFF_XS);
@@ -477,19 +464,18 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             la_next = p.log_alpha[gi];
             be_next = p.beta[gi];
         }
-        for (int c = 0; c < N && ok; ++c) {
-            const int buf = c & 1;
-            const uint32_t par = c & 1;
-            const int64_t t0 = (int64_t)(c0 + c) * kC;
-            const int n = (T - t0 < kC) ? (int)(T - t0) : kC;
-            DBG_CLK(3, 0)
-            // ---- gates ----
+        // gates of chunk cg into buffer cg & 1: g (chunk cumsum of log alpha), beta, gamma = e^g,
+        // e^{g_t - c}, e^{c - g_t} with c = g_31, and the narrow-chunk flags
+        auto prep_gates = [&](int cg) {
+            float *gb = reinterpret_cast<float *>(sm + OFF_PG) + (cg & 1) * 320;
+            const int64_t t0g = (int64_t)(c0 + cg) * kC;
+            const int ng = (T - t0g < kC) ? (int)(T - t0g) : kC;
             if (pt < 64) {
-                const float x = (pt < n) ? fmaxf(la_next, kLogAlphaFloor) : 0.f;
-                bet[pt] = (pt < n) ? be_next : 0.f;
+                const float x = (pt < ng) ? fmaxf(la_next, kLogAlphaFloor) : 0.f;
+                gb[64 + pt] = (pt < ng) ? be_next : 0.f;
                 const float s = chunk_cumsum(x, pt, prep_tmp, kBarPrep, kNumPrep);
-                g[pt] = s;
-                const int64_t tn = t0 + kC + pt;
+                gb[pt] = s;
+                const int64_t tn = t0g + kC + pt;
                 if (tn < T) {
                     const int64_t gi = ((int64_t)b * T + tn) * H + h;
                     la_next = p.log_alpha[gi];
@@ -500,17 +486,25 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             }
             named_bar(kBarPrep, kNumPrep);
             if (pt < 64) {
-                const float gt = g[pt], cm = g[31];
-                gam[pt] = expf(gt);
-                ea[pt] = expf(gt - cm);
-                eb[pt] = expf(cm - gt);
+                const float gt = gb[pt], cm = gb[31];
+                gb[128 + pt] = expf(gt);
+                gb[192 + pt] = expf(gt - cm);
+                gb[256 + pt] = expf(cm - gt);
                 // e^{g_t - g_s} = e^{g_t - c} e^{c - g_s}, exact to a few ulp; used while every
                 // |g_t - c| < 60, so that neither factor nor the output partial sums overflow
                 const bool nr = __all_sync(0xffffffffu, fabsf(gt - cm) < 60.f);
-                if (lane == 0) prep_flags[pt >> 5] = nr ? 1 : 0;
+                if (lane == 0) prep_flags[(cg & 1) * 2 + (pt >> 5)] = nr ? 1 : 0;
             }
             named_bar(kBarPrep, kNumPrep);
-            const bool narrow = prep_flags[0] && prep_flags[1];
+        };
+        prep_gates(0);
+        for (int c = 0; c < N && ok; ++c) {
+            const int buf = c & 1;
+            const uint32_t par = c & 1;
+            const float *g = reinterpret_cast<const float *>(sm + OFF_PG) + buf * 320;
+            const float *bet = g + 64, *gam = g + 128, *ea = g + 192, *eb = g + 256;
+            const bool narrow = prep_flags[buf * 2] && prep_flags[buf * 2 + 1];
+            DBG_CLK(3, 0)
             DBG_CLK(3, 1)
             if (!(ok = role_wait(&bars[B_GDONE], par, abort_flag, kBarPrep, kNumPrep))) break;
             tc_fence_after();
@@ -521,47 +515,45 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             {
                 const int m = (warp & 3) * 32 + lane;  // TMEM lane = row of [Q; K]
                 const int t = m & 63;
-                const float gt = g[t], at = ea[t];
-                uint32_t r[32];
-                tmem_ld32(tm + lb + TM_G + ch * 32, r);
-                tmem_wait_ld();
-                float d[32];
-                if (narrow) {
-                    if (m < 64) {
+                const float gt = g[t], at = ea[t], bt = bet[t];
+                const float sc = (m < 64) ? 1.f : at;
+#pragma unroll 1
+                for (int piece = 0; piece < 2; ++piece) {
+                    const int s0 = ch * 32 + piece * 16;  // first column of this piece
+                    uint32_t r[16];
+                    tmem_ld16(tm + lb + TM_G + s0, r);
+                    tmem_wait_ld();
+                    // decay factor of column s: e^{c - g_s} (times e^{g_t - c} for A rows) in a narrow
+                    // chunk, else e^{g_t - g_s}
+                    float d[16];
+                    if (narrow) {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) d[i] = eb[ch * 32 + i];
+                        for (int i = 0; i < 16; ++i) d[i] = sc * eb[s0 + i];
                     } else {
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) d[i] = at * eb[ch * 32 + i];
+                        for (int i = 0; i < 16; ++i) d[i] = expf(gt - g[s0 + i]);
                     }
-                } else {
+                    if (m < 64) {
+                        uint32_t pk[8];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) d[i] = expf(gt - g[ch * 32 + i]);
-                }
-                if (m < 64) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const int s = ch * 32 + i;
-                        const float v0 = (s <= t) ? __uint_as_float(r[i]) * d[i] : 0.f;
-                        const float v1 = (s + 1 <= t) ? __uint_as_float(r[i + 1]) * d[i + 1] : 0.f;
-                        pk[i >> 1] = pack_bf16x2(v0, v1);
-                    }
-#pragma unroll
-                    for (int cc = 0; cc < 4; ++cc)
-                        *reinterpret_cast<uint4 *>(sm + OFF_P + buf * 8192 + sw128(t, ch * 4 + cc)) =
-                            make_uint4(pk[cc * 4], pk[cc * 4 + 1], pk[cc * 4 + 2], pk[cc * 4 + 3]);
-                } else {
-                    const float bt = bet[t];
-#pragma unroll
-                    for (int i = 0; i < 32; i += 4) {
-                        float v[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int s = ch * 32 + i + e;
-                            v[e] = (s < t) ? bt * d[i + e] * __uint_as_float(r[i + e]) : 0.f;
+                        for (int i = 0; i < 16; i += 2) {
+                            const float v0 = (s0 + i <= t) ? __uint_as_float(r[i]) * d[i] : 0.f;
+                            const float v1 = (s0 + i + 1 <= t) ? __uint_as_float(r[i + 1]) * d[i + 1] : 0.f;
+                            pk[i >> 1] = pack_bf16x2(v0, v1);
                         }
-                        *reinterpret_cast<float4 *>(Am + t * LDM + ch * 32 + i) = make_float4(v[0], v[1], v[2], v[3]);
+#pragma unroll
+                        for (int cc = 0; cc < 2; ++cc)
+                            *reinterpret_cast<uint4 *>(sm + OFF_P + buf * 8192 + sw128(t, (s0 >> 3) + cc)) =
+                                make_uint4(pk[cc * 4], pk[cc * 4 + 1], pk[cc * 4 + 2], pk[cc * 4 + 3]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; i += 4) {
+                            float v[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                v[e] = (s0 + i + e < t) ? bt * d[i + e] * __uint_as_float(r[i + e]) : 0.f;
+                            *reinterpret_cast<float4 *>(Am + t * LDM + s0 + i) = make_float4(v[0], v[1], v[2], v[3]);
+                        }
                     }
                 }
             }
@@ -585,15 +577,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                     if (rr & 1) a0 -= Am[(o + rr) * LDM + o + rr - 1] * x[rr - 1];
                     x[rr] = a0 + a1;
                 }
-                const int col = o + lane;
-                const float bc = bet[col], gbc = bc * gam[col];
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr) {
-                    Tm[(o + rr) * LDM + col] = x[rr];
-                    const uint32_t off = sw128(o + rr, col >> 3) + (col & 7) * 2;
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + OFF_TB + off) = __float2bfloat16_rn(x[rr] * bc);
-                    *reinterpret_cast<__nv_bfloat16 *>(sm + OFF_TBG + off) = __float2bfloat16_rn(x[rr] * gbc);
-                }
+                for (int rr = 0; rr < 16; ++rr) Tm[(o + rr) * LDM + o + lane] = x[rr];
                 if ((pw & 1) == 0) {
 #pragma unroll
                     for (int rr = 0; rr < 16; ++rr) Tm[(o + rr) * LDM + o + 16 + lane] = 0.f;
@@ -603,8 +588,25 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             named_bar(kBarPrep, kNumPrep);
             DBG_CLK(3, 4)
             // (2) 16 -> 32: T_10 = -T_11 (A_10 T_00) inside each 32x32 diagonal block; one warp per
-            //     (block, 8-column tile); X goes through a per-warp scratch tile
-            if (pw < 4) {
+            //     (block, 8-column tile); X goes through a per-warp scratch tile. Meanwhile role warps
+            //     4..7 write the four 16x16 diagonal blocks as bf16 T diag(beta) and T diag(beta gamma),
+            //     eight columns (one 16-byte swizzle unit) per thread
+            if (pw >= 4) {
+                const int idx = pt - 128, row = idx >> 1, col = (row & ~15) + (idx & 1) * 8;
+                const float4 x0 = *reinterpret_cast<const float4 *>(Tm + row * LDM + col);
+                const float4 x1 = *reinterpret_cast<const float4 *>(Tm + row * LDM + col + 4);
+                const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                uint32_t wb[4], wg[4];
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    const float b0 = bet[col + e], b1 = bet[col + e + 1];
+                    wb[e >> 1] = pack_bf16x2(xv[e] * b0, xv[e + 1] * b1);
+                    wg[e >> 1] = pack_bf16x2(xv[e] * (b0 * gam[col + e]), xv[e + 1] * (b1 * gam[col + e + 1]));
+                }
+                const uint32_t off = sw128(row, col >> 3);
+                *reinterpret_cast<uint4 *>(sm + OFF_TB + off) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+                *reinterpret_cast<uint4 *>(sm + OFF_TBG + off) = make_uint4(wg[0], wg[1], wg[2], wg[3]);
+            } else {
                 const int q0 = (pw >> 1) * 32, n0 = (pw & 1) * 8;
                 float *xs = Xs + pw * 128;  // [16][8]
                 float dacc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -659,6 +661,8 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             named_bar(kBarPrep, kNumPrep);
             if (pt == 0) arrive(&bars[B_TBREADY]);
             DBG_CLK(3, 6)
+            // gates of the next chunk, while the W MMA of this one runs
+            if (c + 1 < N) prep_gates(c + 1);
             DBG_CLK(3, 7)
             // ---- W (bf16, MN-major rows i) from W^T in TMEM (the MMAs of the previous chunk that read W
             //      and the bf16 state copy are done) ----
@@ -690,7 +694,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         }
     } else if (warp >= kChainWarp0) {
         // ============================== chain ==============================
-        const int j = tid - kChainWarp0 * 32;  // TMEM lane / state row, 0..127
+        // two warps per TMEM lane quadrant: thread (j, ch) owns state row j and column half ch
+        const int ct = tid - kChainWarp0 * 32;       // 0..255
+        const int j = (warp & 3) * 32 + lane;        // TMEM lane / state row, 0..127
+        const int ch = (warp - kChainWarp0) >> 2;    // column half
         float *dl = reinterpret_cast<float *>(sm + OFF_CG);  // [2][64] e^{g_C - g_s} per chunk parity
         float *f1 = dl + 128;                                // [2][64] gamma_t
         float *f2 = dl + 256;                                // [2][64] e^{g_t - c} (narrow chunk) or 1
@@ -704,12 +711,13 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
             if (kind == 0)
                 src = (seg == 0) ? (p.S0 ? p.S0 + (bh * kD + j) * (int64_t)kD : nullptr)
                                  : p.S_entry + ((bh * (p.nseg - 1) + seg - 1) * kD + j) * (int64_t)kD;
-#pragma unroll
-            for (int piece = 0; piece < 4; ++piece) {
+#pragma unroll 1
+            for (int piece = 0; piece < 2; ++piece) {
+                const int col0 = ch * 64 + piece * 32;
                 uint32_t r[32];
 #pragma unroll
                 for (int i = 0; i < 32; i += 4) {
-                    float4 v = src ? *reinterpret_cast<const float4 *>(src + piece * 32 + i) : make_float4(0, 0, 0, 0);
+                    float4 v = src ? *reinterpret_cast<const float4 *>(src + col0 + i) : make_float4(0, 0, 0, 0);
                     r[i] = __float_as_uint(v.x);
                     r[i + 1] = __float_as_uint(v.y);
                     r[i + 2] = __float_as_uint(v.z);
@@ -717,9 +725,9 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 }
                 if (kind == 2) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint((piece * 32 + i == j) ? 1.f : 0.f);
+                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint((col0 + i == j) ? 1.f : 0.f);
                 }
-                tmem_st32(tm + lb + TM_S + piece * 32, r);
+                tmem_st32(tm + lb + TM_S + col0, r);
             }
             tmem_wait_st();
         }
@@ -727,68 +735,70 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         // factors; the narrow test repeats the prep role's computation on identical values, so
         // both roles take the same decision
         float la_next = 0.f;
-        if (j < 64 && (int64_t)c0 * kC + j < T) la_next = p.log_alpha[((int64_t)b * T + (int64_t)c0 * kC + j) * H + h];
+        if (ct < 64 && (int64_t)c0 * kC + ct < T)
+            la_next = p.log_alpha[((int64_t)b * T + (int64_t)c0 * kC + ct) * H + h];
         auto chain_gates = [&](int cg) {
             const int64_t t0g = (int64_t)(c0 + cg) * kC;
             const int ng = (T - t0g < kC) ? (int)(T - t0g) : kC;
             float *dlb = dl + (cg & 1) * 64;
             float s = 0.f;
-            if (j < 64) {
-                const float x = (j < ng) ? fmaxf(la_next, kLogAlphaFloor) : 0.f;
-                s = chunk_cumsum(x, j, chain_tmp, kBarChain, kNumChain);
-                const int64_t tn = t0g + kC + j;
+            if (ct < 64) {
+                const float x = (ct < ng) ? fmaxf(la_next, kLogAlphaFloor) : 0.f;
+                s = chunk_cumsum(x, ct, chain_tmp, kBarChain, kNumChain);
+                const int64_t tn = t0g + kC + ct;
                 if (tn < T) la_next = p.log_alpha[((int64_t)b * T + tn) * H + h];
-                dlb[j] = s;
+                dlb[ct] = s;
             } else {
                 named_bar(kBarChain, kNumChain);  // the barrier inside chunk_cumsum
             }
             named_bar(kBarChain, kNumChain);
             const float g63 = dlb[63], cm = dlb[31];
-            if (j < 64) {
+            if (ct < 64) {
                 const bool nr = __all_sync(0xffffffffu, fabsf(s - cm) < 60.f);
-                if ((j & 31) == 0) chain_flags[j >> 5] = nr ? 1 : 0;
+                if ((ct & 31) == 0) chain_flags[ct >> 5] = nr ? 1 : 0;
             }
             named_bar(kBarChain, kNumChain);
             const bool narrow = chain_flags[0] && chain_flags[1];
-            if (j < 64) {
-                dlb[j] = expf(g63 - s);
-                f1[(cg & 1) * 64 + j] = expf(s);
-                f2[(cg & 1) * 64 + j] = narrow ? expf(s - cm) : 1.f;
+            if (ct < 64) {
+                dlb[ct] = expf(g63 - s);
+                f1[(cg & 1) * 64 + ct] = expf(s);
+                f2[(cg & 1) * 64 + ct] = narrow ? expf(s - cm) : 1.f;
             }
-            if (j == 0) gcs[cg & 1] = expf(g63);
+            if (ct == 0) gcs[cg & 1] = expf(g63);
             named_bar(kBarChain, kNumChain);
         };
-        // outputs of chunk cprev: o_t = f1_t O1_t + f2_t O2_t (thread j holds column j of both), staged
-        // as two 64x64 bf16 boxes in the TMA layout and written by two TMA stores
+        // outputs of chunk cprev: o_t = f1_t O1_t + f2_t O2_t for this thread's column j and tokens
+        // t in its half, staged as two 64x64 bf16 boxes in the TMA layout, written by two TMA stores
         auto write_out = [&](int cprev) {
-            const float *f1c = f1 + (cprev & 1) * 64, *f2c = f2 + (cprev & 1) * 64;
-            if (j == 0) bulk_wait_read0();  // the previous chunk's stores have read the staging buffer
+            const float *f1c = f1 + (cprev & 1) * 64 + ch * 32, *f2c = f2 + (cprev & 1) * 64 + ch * 32;
+            if (ct == 0) bulk_wait_read0();  // the previous chunk's stores have read the staging buffer
             named_bar(kBarChain, kNumChain);
             const int par = j & 1, colw = j - par;  // this lane writes column pair (colw, colw + 1)
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t r1[32], r2[32];
-                tmem_ld32(tm + lb + TM_O + half * 32, r1);
-                tmem_ld32(tm + lb + TM_O2 + half * 32, r2);
+            uint8_t *stage = sm + OFF_OST + (colw >> 6) * 8192;
+            const uint32_t cbyte = (colw & 7) * 2, cchunk = (colw & 63) >> 3;
+#pragma unroll 1
+            for (int piece = 0; piece < 2; ++piece) {
+                uint32_t r1[16], r2[16];
+                tmem_ld16(tm + lb + TM_O + ch * 32 + piece * 16, r1);
+                tmem_ld16(tm + lb + TM_O2 + ch * 32 + piece * 16, r2);
                 tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    const int t = half * 32 + i;
+                for (int i = 0; i < 16; i += 2) {
+                    const int t = piece * 16 + i;
                     const float o0 = f1c[t] * __uint_as_float(r1[i]) + f2c[t] * __uint_as_float(r2[i]);
                     const float o1 = f1c[t + 1] * __uint_as_float(r1[i + 1]) + f2c[t + 1] * __uint_as_float(r2[i + 1]);
                     // even lanes keep row t and take the neighbour's column; odd lanes keep row t+1
                     const float send = par ? o0 : o1;
                     const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
                     const uint32_t word = par ? pack_bf16x2(recv, o1) : pack_bf16x2(o0, recv);
-                    const int row = t + par;
-                    *reinterpret_cast<uint32_t *>(sm + OFF_OST + (colw >> 6) * 8192 +
-                                                  sw128(row, (colw & 63) >> 3) + (colw & 7) * 2) = word;
+                    const int row = ch * 32 + t + par;
+                    *reinterpret_cast<uint32_t *>(stage + sw128(row, cchunk) + cbyte) = word;
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar(kBarChain, kNumChain);
-            if (j == 0) {
+            if (ct == 0) {
                 tma_store_4d(&tm_o, sm + OFF_OST, 0, h, (c0 + cprev) * kC, b);
                 tma_store_4d(&tm_o, sm + OFF_OST + 8192, 64, h, (c0 + cprev) * kC, b);
                 bulk_commit();
@@ -797,7 +807,7 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         chain_gates(0);
         for (int c = 0; c < N && ok; ++c) {
             const uint32_t par = c & 1;
-            const float *dlc = dl + (c & 1) * 64;
+            const float *dlc = dl + (c & 1) * 64 + ch * 32;
             DBG_CLK(4, 0)
             if (c > 0) {
                 // the state update of the previous chunk is complete, and its output MMA is done
@@ -807,60 +817,61 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
                 tc_fence_after();
             }
             DBG_CLK(4, 1)
-            // ---- S -> bf16 operand copy; S <- gamma_C S ----
+            // ---- S -> bf16 operand copy; S <- gamma_C S (this thread: row j, 64 columns) ----
             {
                 const float gC = gcs[c & 1];
-#pragma unroll
-                for (int piece = 0; piece < 4; ++piece) {
+#pragma unroll 1
+                for (int piece = 0; piece < 2; ++piece) {
+                    const int col0 = ch * 64 + piece * 32;
                     uint32_t r[32];
-                    tmem_ld32(tm + lb + TM_S + piece * 32, r);
+                    tmem_ld32(tm + lb + TM_S + col0, r);
                     tmem_wait_ld();
                     uint32_t pk[16];
 #pragma unroll
                     for (int i = 0; i < 32; i += 2)
                         pk[i >> 1] = pack_bf16x2(__uint_as_float(r[i]), __uint_as_float(r[i + 1]));
-                    tmem_st16(tm + lb + TM_SB + piece * 16, pk);
+                    tmem_st16(tm + lb + TM_SB + col0 / 2, pk);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * gC);
-                    tmem_st32(tm + lb + TM_S + piece * 32, r);
+                    tmem_st32(tm + lb + TM_S + col0, r);
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 named_bar(kBarChain, kNumChain);
-                if (j == 0) arrive(&bars[B_SREADY]);
+                if (ct == 0) arrive(&bars[B_SREADY]);
             }
             DBG_CLK(4, 2)
-            // ---- outputs of the previous chunk (frees the O accumulator) ----
+            // ---- outputs of the previous chunk (frees the O accumulators) ----
             if (c > 0) {
                 if (!(ok = role_wait(&bars[B_M2ADONE], (c - 1) & 1, abort_flag, kBarChain, kNumChain))) break;
                 tc_fence_after();
                 if (outputs) write_out(c - 1);  // ends with a chain barrier after the O reads
-                if (j == 0) arrive(&bars[B_OFREE]);
+                if (ct == 0) arrive(&bars[B_OFREE]);
             }
             DBG_CLK(4, 3)
             if (!(ok = role_wait(&bars[B_M1ADONE], par, abort_flag, kBarChain, kNumChain))) break;
             tc_fence_after();
             DBG_CLK(4, 4)
-            // ---- U^T (accumulated in TMEM) -> bf16 U^T and bf16 U^T diag(dl) ----
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t u[32];
-                tmem_ld32(tm + lb + TM_DU + half * 32, u);
+            // ---- U^T (accumulated in TMEM) -> bf16 U^T and bf16 U^T diag(dl) (this thread: 32 tokens) ----
+#pragma unroll 1
+            for (int piece = 0; piece < 2; ++piece) {
+                uint32_t u[16], pk[8];
+                tmem_ld16(tm + lb + TM_DU + ch * 32 + piece * 16, u);
                 tmem_wait_ld();
-                uint32_t pk[16], pd[16];
 #pragma unroll
-                for (int i = 0; i < 32; i += 2) {
-                    const float u0 = __uint_as_float(u[i]), u1 = __uint_as_float(u[i + 1]);
-                    pk[i >> 1] = pack_bf16x2(u0, u1);
-                    pd[i >> 1] = pack_bf16x2(u0 * dlc[half * 32 + i], u1 * dlc[half * 32 + i + 1]);
-                }
-                tmem_st16(tm + lb + TM_UB + half * 16, pk);
-                tmem_st16(tm + lb + TM_UDB + half * 16, pd);
+                for (int i = 0; i < 16; i += 2)
+                    pk[i >> 1] = pack_bf16x2(__uint_as_float(u[i]), __uint_as_float(u[i + 1]));
+                tmem_st8(tm + lb + TM_UB + ch * 16 + piece * 8, pk);
+#pragma unroll
+                for (int i = 0; i < 16; i += 2)
+                    pk[i >> 1] = pack_bf16x2(__uint_as_float(u[i]) * dlc[piece * 16 + i],
+                                             __uint_as_float(u[i + 1]) * dlc[piece * 16 + i + 1]);
+                tmem_st8(tm + lb + TM_UDB + ch * 16 + piece * 8, pk);
             }
             tmem_wait_st();
             tc_fence_before();
             named_bar(kBarChain, kNumChain);
-            if (j == 0) arrive(&bars[B_UREADY]);
+            if (ct == 0) arrive(&bars[B_UREADY]);
             DBG_CLK(4, 5)
             // gates of the next chunk, while this chunk's last MMAs run
             if (c + 1 < N) chain_gates(c + 1);
@@ -878,19 +889,20 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
         else
             dst = (kind == 1 ? p.Bw : p.Mw) + ((bh * (p.nseg - 1) + seg) * kD + j) * (int64_t)kD;
         if (ok && dst) {
-#pragma unroll
-            for (int piece = 0; piece < 4; ++piece) {
+#pragma unroll 1
+            for (int piece = 0; piece < 2; ++piece) {
+                const int col0 = ch * 64 + piece * 32;
                 uint32_t r[32];
-                tmem_ld32(tm + lb + TM_S + piece * 32, r);
+                tmem_ld32(tm + lb + TM_S + col0, r);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; i += 4)
-                    *reinterpret_cast<float4 *>(dst + piece * 32 + i) =
+                    *reinterpret_cast<float4 *>(dst + col0 + i) =
                         make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]), __uint_as_float(r[i + 2]),
                                     __uint_as_float(r[i + 3]));
             }
         }
-        if (j == 0) bulk_wait0();  // every output store has completed
+        if (ct == 0) bulk_wait0();  // every output store has completed
     }
 
     tc_fence_before();
