@@ -36,7 +36,7 @@ STATUS = {
 }
 
 EXPORTS = ("gdn_forward", "gdn_decode_step", "gdn_forward_plan", "gdn_status_string", "gdn_version",
-           "gdn_forward_noalloc")
+           "gdn_forward_noalloc", "gdn_scratch_release")
 
 
 class GdnError(RuntimeError):
@@ -68,6 +68,8 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     lib.gdn_version.restype = ctypes.c_int
     lib.gdn_forward_plan.argtypes = [i64] * 6 + [ctypes.c_int, ctypes.POINTER(i64), ctypes.POINTER(ctypes.c_int)]
     lib.gdn_forward_plan.restype = ctypes.c_int
+    lib.gdn_scratch_release.argtypes = []
+    lib.gdn_scratch_release.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -153,6 +155,13 @@ def forward_plan(B: int, T: int, H: int, dk: int, dv: int, chunk: int = 64, dtyp
     if st != 0:
         raise GdnError(st, "gdn_forward_plan")
     return scratch.value, launches.value
+
+
+def scratch_release() -> None:
+    """Return the library's unused pooled device scratch on the current device to the driver."""
+    st = load().gdn_scratch_release()
+    if st != 0:
+        raise GdnError(st, "gdn_scratch_release")
 
 
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,

@@ -1,0 +1,1048 @@
+// fwd_split.cu -- chunkwise gated-delta forward on the 5th-generation tensor
+// cores in two kernels: a chunk-parallel prep kernel and a chain kernel.
+// bf16 q/k/v, dk = dv = 128, chunk C = 64.
+//
+// Operation: "ATMA: Long-Context Language Modeling via Polar Attention and
+// Gated-Delta Compression Memory", Sec. 3.3 (gated-delta memory equation),
+// computed in the chunkwise UT-transform form of the works that paper cites
+// for the memory ("Gated delta networks"; "Parallelizing linear transformers
+// with the delta rule over sequence length").  Per chunk of 64 tokens with
+// chunk-local log-decay cumsum g_t, gamma_t = e^{g_t}, dl_s = e^{g_C - g_s}:
+//
+//   prep kernel (independent of the state; every chunk of every (b, h) in
+//   parallel, persistent CTAs, two per SM):
+//     G   = [Q; K] K^T                                          (tcgen05, M = 128)
+//     P   = lower(e^{g_t - g_s} (Q K^T)_ts)                     -> workspace, bf16
+//     A   = strict_lower(beta_t e^{g_t - g_s} (K K^T)_ts)
+//     T   = (I + A)^{-1}: 16x16 diagonal blocks by substitution, merged 16 -> 32 -> 64
+//           with warp-level TF32 MMAs (fp32 accumulation)
+//     TB  = T diag(beta)                                        -> workspace, bf16
+//     W^T = K^T (T diag(beta gamma))^T                          (tcgen05) -> workspace, bf16
+//
+//   chain kernel (sequential over the chunks of one (b, h) or segment):
+//     Ut^T = V^T TB^T                               (tcgen05, off the critical path)
+//     U^T  = Ut^T - S W^T                           (accumulated onto Ut^T, B negated)
+//     S   <- gamma_C S + U^T (diag(dl) K)           (float32 state in tensor memory)
+//     O^T  = S (diag(gamma) Q)^T + U^T P^T          (one accumulator, off the critical path)
+//
+// e^{g_t - g_s} is formed as e^{g_t - c} e^{c - g_s} (c = g_31) when every
+// |g_t - c| < 60 in the chunk, else element by element; both are exact to a
+// few ulp.  Workspace: per chunk P (8 KB), TB (8 KB) and W^T (16 KB), each a
+// bf16 tile of 128-byte rows written and read by TMA with 128-byte swizzle,
+// and the chunk's gates gamma_t and dl_s (512 B, float32).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <stdlib.h>
+
+#include <atomic>
+
+#include "gdn_internal.h"
+#include "sm100.cuh"
+#include "tc_util.cuh"
+
+namespace gdn {
+namespace {
+
+using namespace sm100;
+using namespace tcu;
+
+constexpr int kC = 64;
+constexpr int kD = 128;
+constexpr size_t kTileP = 64 * 64 * 2, kTileTB = 64 * 64 * 2, kTileW = 128 * 64 * 2;
+constexpr size_t kGateRec = 128 * 4;  // gamma_t and dl_s of one chunk, float32
+constexpr size_t kWsPerChunk = kTileP + kTileTB + kTileW + kGateRec;  // 32.5 KB
+
+__device__ int g_split_timeout;  // set when a bounded mbarrier wait gives up
+
+#ifdef GDN_TC_DEBUG
+// Debug builds only: per-phase clock stamps of CTA 0 for its first 8 work
+// items, 8 rows of 16 int64 per item.
+__device__ long long *g_split_dbg;
+#define SDBG(row, i)                                                                   \
+    if (g_split_dbg != nullptr && blockIdx.x == 0 && it < 8)                           \
+        g_split_dbg[(it * 8 + (row)) * 16 + (i)] = clock64();
+#else
+#define SDBG(row, i)
+#endif
+
+// ============================================================================
+// prep kernel
+// ============================================================================
+constexpr int kPrepThreads = 288;  // warp 0: TMA + MMA issue; warps 1-8: prep role
+constexpr int kNumPrep = 256;
+constexpr int kBarP = 1;
+constexpr int LDM = 68;   // row stride (floats) of the fp32 64x64 tiles
+constexpr int LDX2 = 40;  // row stride of the 32->64 merge scratch
+
+constexpr uint32_t PO_QK = 0;        // 32 KB: per 64-column block j: [Q 8 KB | K 8 KB]
+constexpr uint32_t PO_TB = 32768;    // 8 KB  T diag(beta)       [t][s], 128-byte swizzle
+constexpr uint32_t PO_TBG = 40960;   // 8 KB  T diag(beta gamma) [t][s]
+constexpr uint32_t PO_P = 49152;     // 8 KB  P [t][s]
+constexpr uint32_t PO_AM = 57344;    // 17 KB A fp32 [64][LDM]; after the inverse: W^T bf16 [128][64] staging
+constexpr uint32_t PO_TM = 74752;    // 17 KB T fp32 [64][LDM]
+constexpr uint32_t PO_XS = 92160;    // 5 KB  merge scratch
+constexpr uint32_t PO_PG = 97280;    // gates per item parity: g, beta, gamma, e^{g-c}, e^{c-g} (2 x 5 x 64)
+constexpr uint32_t PO_BARS = 99840;  // mbarriers
+constexpr uint32_t PO_MISC = 99904;  // tmem slot, abort flag, scan scratch, flags
+constexpr uint32_t SMEM_PREP = 99968 + 1024;
+
+constexpr uint32_t TP_G = 0;   // 64 columns: [Q;K] K^T
+constexpr uint32_t TP_W = 64;  // 64 columns: W^T
+
+constexpr uint32_t IDESC_G = instr_desc_bf16(128, 64, 0, 0);     // [Q;K] . K^T
+constexpr uint32_t IDESC_MN64 = instr_desc_bf16(128, 64, 1, 0);  // K^T / V^T (MN-major A) . T^T
+
+enum PBar { PB_QFULL = 0, PB_KFULL, PB_GDONE, PB_GFREE, PB_TBREADY, PB_WDONE, PB_COUNT };
+
+struct PrepArgs {
+    const float *log_alpha, *beta;
+    float *gate_rec;  // [items][128]: gamma_t, then dl_s = e^{g_63 - g_s}
+    int64_t T, H;
+    int64_t items;  // B * H * chunks
+    int chunks;     // chunks per (b, h)
+};
+
+__global__ void __launch_bounds__(kPrepThreads, 2)
+fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_tb,
+                const __grid_constant__ CUtensorMap tm_w, PrepArgs p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + PO_BARS);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + PO_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + PO_MISC + 4);
+    float *scan_tmp = reinterpret_cast<float *>(sm + PO_MISC + 8);
+    int *nflags = reinterpret_cast<int *>(sm + PO_MISC + 16);  // [2 parities][2 warps]
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t T = p.T, H = p.H;
+    // work items of this CTA: global chunk ids blockIdx.x, blockIdx.x + gridDim.x, ...
+    const int nit = (blockIdx.x < p.items) ? (int)((p.items - 1 - blockIdx.x) / gridDim.x + 1) : 0;
+    auto item = [&](int it) { return (int64_t)blockIdx.x + (int64_t)it * gridDim.x; };
+    const uint32_t sbase = smem_u32(sm);
+
+    if (tid == 0) {
+        for (int i = 0; i < PB_COUNT; ++i) mbar_init(&bars[i], 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tmem_slot;
+    const uint32_t lb = (uint32_t)((warp & 3) * 32) << 16;  // this warp's TMEM lane quadrant
+
+    if (warp == 0) {
+        // ============================ issuer ============================
+        if (lane == 0) {
+            auto coords = [&](int it, int &b, int &h, int &t0) {
+                const int64_t gi = item(it), bh = gi / p.chunks;
+                b = (int)(bh / H);
+                h = (int)(bh % H);
+                t0 = (int)(gi % p.chunks) * kC;
+            };
+            auto load_q = [&](int it) {
+                int b, h, t0;
+                coords(it, b, h, t0);
+                mbar_arrive_expect_tx(&bars[PB_QFULL], 2 * 8192);
+                for (int blk = 0; blk < 2; ++blk)
+                    tma_load_4d(sm + PO_QK + blk * 16384, &tm_q, &bars[PB_QFULL], blk * 64, h, t0, b);
+            };
+            auto load_k = [&](int it) {
+                int b, h, t0;
+                coords(it, b, h, t0);
+                mbar_arrive_expect_tx(&bars[PB_KFULL], 2 * 8192);
+                for (int blk = 0; blk < 2; ++blk)
+                    tma_load_4d(sm + PO_QK + blk * 16384 + 8192, &tm_k, &bars[PB_KFULL], blk * 64, h, t0, b);
+            };
+            bool ok = true;
+            if (nit > 0) {
+                load_q(0);
+                load_k(0);
+            }
+            for (int it = 0; it < nit && ok; ++it) {
+                const uint32_t par = it & 1;
+                SDBG(0, 0)
+                if (!(ok = wait_bar(&bars[PB_QFULL], par, abort_flag))) break;
+                if (!(ok = wait_bar(&bars[PB_KFULL], par, abort_flag))) break;
+                if (it > 0 && !(ok = wait_bar(&bars[PB_GFREE], (it - 1) & 1, abort_flag))) break;
+                SDBG(0, 1)
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint32_t a = sbase + PO_QK + (kk >> 2) * 16384 + (kk & 3) * 32;
+                    mma_ss(tm + TP_G, smem_desc_sw128(a, 16, 1024), smem_desc_sw128(a + 8192, 16, 1024), IDESC_G,
+                           kk > 0);
+                }
+                mma_commit(&bars[PB_GDONE]);
+                // Q is free once G is done
+                if (!(ok = wait_bar(&bars[PB_GDONE], par, abort_flag))) break;
+                if (it + 1 < nit) load_q(it + 1);
+                SDBG(0, 2)
+                if (!(ok = wait_bar(&bars[PB_TBREADY], par, abort_flag))) break;
+                SDBG(0, 3)
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ss(tm + TP_W, smem_desc_sw128(sbase + PO_QK + 8192 + kk * 2048, 16384, 1024),
+                           smem_desc_sw128(sbase + PO_TBG + kk * 32, 16, 1024), IDESC_MN64, kk > 0);
+                mma_commit(&bars[PB_WDONE]);
+                // K is free once W^T is done
+                if (!(ok = wait_bar(&bars[PB_WDONE], par, abort_flag))) break;
+                if (it + 1 < nit) load_k(it + 1);
+                SDBG(0, 4)
+            }
+        }
+        __syncwarp();
+    } else {
+        // ============================== prep ==============================
+        const int pt = tid - 32;          // 0..255
+        const int pw = pt >> 5;           // role warp 0..7
+        const int ch = pw >> 2;           // column half of the TMEM epilogues
+        const int g8 = lane >> 2, t4 = lane & 3;  // MMA fragment coordinates
+        float *Am = reinterpret_cast<float *>(sm + PO_AM);
+        float *Tm = reinterpret_cast<float *>(sm + PO_TM);
+        float *Xs = reinterpret_cast<float *>(sm + PO_XS);
+        bool ok = true;
+        // the upper triangles of the bf16 T tiles are never written below: zero both tiles once
+#pragma unroll
+        for (int i = 0; i < 4; ++i) reinterpret_cast<uint4 *>(sm + PO_TB)[pt + 256 * i] = make_uint4(0u, 0u, 0u, 0u);
+        fence_proxy_async_smem();
+        // gates of work item `it` into buffer it & 1 (threads pt < 64 hold token pt)
+        float la_next = 0.f, be_next = 0.f;
+        auto gate_index = [&](int it, int t) -> int64_t {
+            const int64_t gi = item(it), bh = gi / p.chunks;
+            const int64_t tok = (gi % p.chunks) * kC + t;
+            if (tok >= T) return -1;
+            return ((bh / H) * T + tok) * H + bh % H;
+        };
+        if (nit > 0 && pt < 64) {
+            const int64_t x = gate_index(0, pt);
+            if (x >= 0) {
+                la_next = p.log_alpha[x];
+                be_next = p.beta[x];
+            }
+        }
+        auto prep_gates = [&](int it) {
+            float *gb = reinterpret_cast<float *>(sm + PO_PG) + (it & 1) * 320;
+            if (pt < 64) {
+                const bool valid = gate_index(it, pt) >= 0;
+                const float x = valid ? fmaxf(la_next, kLogAlphaFloor) : 0.f;
+                gb[64 + pt] = valid ? be_next : 0.f;
+                const float s = chunk_cumsum(x, pt, scan_tmp, kBarP, kNumPrep);
+                SDBG(1, 8)
+                gb[pt] = s;
+                if (it + 1 < nit) {
+                    const int64_t xn = gate_index(it + 1, pt);
+                    la_next = xn >= 0 ? p.log_alpha[xn] : 0.f;
+                    be_next = xn >= 0 ? p.beta[xn] : 0.f;
+                }
+            } else {
+                named_bar(kBarP, kNumPrep);  // the barrier inside chunk_cumsum
+            }
+            named_bar(kBarP, kNumPrep);
+            SDBG(1, 9)
+            if (pt < 64) {
+                const float gt = gb[pt], cm = gb[31];
+                const float gm = expf(gt);
+                gb[128 + pt] = gm;
+                gb[192 + pt] = expf(gt - cm);
+                gb[256 + pt] = expf(cm - gt);
+                float *rec = p.gate_rec + item(it) * 128;
+                rec[pt] = gm;
+                rec[64 + pt] = expf(gb[63] - gt);
+                // e^{g_t - g_s} = e^{g_t - c} e^{c - g_s} while every |g_t - c| < 60, so that
+                // neither factor overflows
+                const bool nr = __all_sync(0xffffffffu, fabsf(gt - cm) < 60.f);
+                if (lane == 0) nflags[(it & 1) * 2 + (pt >> 5)] = nr ? 1 : 0;
+            }
+            named_bar(kBarP, kNumPrep);
+        };
+        if (nit > 0) prep_gates(0);
+        for (int it = 0; it < nit && ok; ++it) {
+            const uint32_t par = it & 1;
+            const int64_t gi = item(it);
+            const float *g = reinterpret_cast<const float *>(sm + PO_PG) + par * 320;
+            const float *bet = g + 64, *gam = g + 128, *ea = g + 192, *eb = g + 256;
+            const bool narrow = nflags[par * 2] && nflags[par * 2 + 1];
+            // the stores of the previous item have finished reading P, TB and the W^T staging
+            if (pt == 0) bulk_wait_read0();
+            SDBG(1, 0)
+            if (!(ok = role_wait(&bars[PB_GDONE], par, abort_flag, kBarP, kNumPrep))) break;
+            tc_fence_after();
+            SDBG(1, 1)
+            // ---- epilogue of G: rows 0..63 -> P (bf16), rows 64..127 -> A (fp32); columns by half ----
+            {
+                const int m = (warp & 3) * 32 + lane;  // TMEM lane = row of [Q; K]
+                const int t = m & 63;
+                const float gt = g[t], at = ea[t], bt = bet[t];
+#pragma unroll 1
+                for (int piece = 0; piece < 2; ++piece) {
+                    const int s0 = ch * 32 + piece * 16;
+                    uint32_t r[16];
+                    tmem_ld16(tm + lb + TP_G + s0, r);
+                    tmem_wait_ld();
+                    float d[16];  // e^{g_t - g_s} for the 16 columns s of this piece
+                    if (narrow) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) d[i] = at * eb[s0 + i];
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) d[i] = expf(gt - g[s0 + i]);
+                    }
+                    if (m < 64) {
+                        uint32_t pk[8];
+#pragma unroll
+                        for (int i = 0; i < 16; i += 2) {
+                            const float v0 = (s0 + i <= t) ? __uint_as_float(r[i]) * d[i] : 0.f;
+                            const float v1 = (s0 + i + 1 <= t) ? __uint_as_float(r[i + 1]) * d[i + 1] : 0.f;
+                            pk[i >> 1] = pack_bf16x2(v0, v1);
+                        }
+#pragma unroll
+                        for (int cc = 0; cc < 2; ++cc)
+                            *reinterpret_cast<uint4 *>(sm + PO_P + sw128(t, (s0 >> 3) + cc)) =
+                                make_uint4(pk[cc * 4], pk[cc * 4 + 1], pk[cc * 4 + 2], pk[cc * 4 + 3]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 16; i += 4) {
+                            float v[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                v[e] = (s0 + i + e < t) ? bt * d[i + e] * __uint_as_float(r[i + e]) : 0.f;
+                            *reinterpret_cast<float4 *>(Am + t * LDM + s0 + i) = make_float4(v[0], v[1], v[2], v[3]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            named_bar(kBarP, kNumPrep);
+            if (pt == 0) {
+                arrive(&bars[PB_GFREE]);
+                tma_store_2d(&tm_p, sm + PO_P, 0, (int)(gi * 64));
+                bulk_commit();
+            }
+            SDBG(1, 2)
+            // ---- T = (I + A)^{-1} ----
+            // (1) 16x16 diagonal blocks by substitution: role warps 0..3, a column per lane; warps 0 and 2
+            //     also zero the upper 16x16 block inside their 32x32 diagonal block
+            if (pw < 4 && lane < 16) {
+                const int o = pw * 16;
+                float x[16];
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) {
+                    float a0 = (rr == lane) ? 1.f : 0.f, a1 = 0.f;
+#pragma unroll
+                    for (int s = 0; s + 1 < rr; s += 2) {
+                        a0 -= Am[(o + rr) * LDM + o + s] * x[s];
+                        a1 -= Am[(o + rr) * LDM + o + s + 1] * x[s + 1];
+                    }
+                    if (rr & 1) a0 -= Am[(o + rr) * LDM + o + rr - 1] * x[rr - 1];
+                    x[rr] = a0 + a1;
+                }
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) Tm[(o + rr) * LDM + o + lane] = x[rr];
+                if ((pw & 1) == 0) {
+#pragma unroll
+                    for (int rr = 0; rr < 16; ++rr) Tm[(o + rr) * LDM + o + 16 + lane] = 0.f;
+                }
+            }
+            __syncwarp();
+            named_bar(kBarP, kNumPrep);
+            SDBG(1, 3)
+            // (2) 16 -> 32: T_10 = -T_11 (A_10 T_00) inside each 32x32 diagonal block; one warp per
+            //     (block, 8-column tile).  Meanwhile role warps 4..7 write the four 16x16 diagonal
+            //     blocks as bf16 T diag(beta) and T diag(beta gamma), one 16-byte unit per thread
+            if (pw >= 4) {
+                const int idx = pt - 128, row = idx >> 1, col = (row & ~15) + (idx & 1) * 8;
+                const float4 x0 = *reinterpret_cast<const float4 *>(Tm + row * LDM + col);
+                const float4 x1 = *reinterpret_cast<const float4 *>(Tm + row * LDM + col + 4);
+                const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+                uint32_t wb[4], wg[4];
+#pragma unroll
+                for (int e = 0; e < 8; e += 2) {
+                    const float b0 = bet[col + e], b1 = bet[col + e + 1];
+                    wb[e >> 1] = pack_bf16x2(xv[e] * b0, xv[e + 1] * b1);
+                    wg[e >> 1] = pack_bf16x2(xv[e] * (b0 * gam[col + e]), xv[e + 1] * (b1 * gam[col + e + 1]));
+                }
+                const uint32_t off = sw128(row, col >> 3);
+                *reinterpret_cast<uint4 *>(sm + PO_TB + off) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+                *reinterpret_cast<uint4 *>(sm + PO_TBG + off) = make_uint4(wg[0], wg[1], wg[2], wg[3]);
+            } else {
+                const int q0 = (pw >> 1) * 32, n0 = (pw & 1) * 8;
+                float *xs = Xs + pw * 128;  // [16][8]
+                float dacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int kk = 0; kk < 2; ++kk) {
+                    uint32_t a[4], bb[2];
+                    load_a(a, Am, LDM, q0 + 16, q0 + 8 * kk, g8, t4);
+                    load_b(bb, Tm, LDM, q0 + 8 * kk, q0 + n0, g8, t4);
+                    mma_tf32(dacc, a, bb);
+                }
+                store_d(xs, 8, 0, 0, dacc, g8, t4);
+                __syncwarp();
+                float e[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int kk = 0; kk < 2; ++kk) {
+                    uint32_t a[4], bb[2];
+                    load_a(a, Tm, LDM, q0 + 16, q0 + 16 + 8 * kk, g8, t4);
+                    load_b(bb, xs, 8, 8 * kk, 0, g8, t4);
+                    mma_tf32(e, a, bb);
+                }
+                store_neg_d(Tm, LDM, q0 + 16, q0 + n0, e, g8, t4);
+                store_t_pair(sm + PO_TB, sm + PO_TBG, q0 + 16 + g8, q0 + n0 + 2 * t4, -e[0], -e[1], bet, gam);
+                store_t_pair(sm + PO_TB, sm + PO_TBG, q0 + 24 + g8, q0 + n0 + 2 * t4, -e[2], -e[3], bet, gam);
+            }
+            named_bar(kBarP, kNumPrep);
+            SDBG(1, 4)
+            // (3) 32 -> 64: X = A[32:64, 0:32] T[0:32, 0:32], then T[32:64, 0:32] = -T[32:64, 32:64] X;
+            //     one warp per (16-row, 8-column) tile; T is lower triangular, so zero k-steps are skipped
+            {
+                const int mi = pw >> 2, ni = pw & 3;
+                float *x2 = Xs;  // [32][LDX2], reuses the 16->32 scratch (a barrier separates the two)
+                float dacc[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int kk = ni; kk < 4; ++kk) {
+                    uint32_t a[4], bb[2];
+                    load_a(a, Am, LDM, 32 + 16 * mi, 8 * kk, g8, t4);
+                    load_b(bb, Tm, LDM, 8 * kk, 8 * ni, g8, t4);
+                    mma_tf32(dacc, a, bb);
+                }
+                store_d(x2, LDX2, 16 * mi, 8 * ni, dacc, g8, t4);
+                named_bar(kBarP, kNumPrep);
+                float e[4] = {0.f, 0.f, 0.f, 0.f};
+                for (int kk = 0; kk <= 2 * mi + 1; ++kk) {
+                    uint32_t a[4], bb[2];
+                    load_a(a, Tm, LDM, 32 + 16 * mi, 32 + 8 * kk, g8, t4);
+                    load_b(bb, x2, LDX2, 8 * kk, 8 * ni, g8, t4);
+                    mma_tf32(e, a, bb);
+                }
+                store_t_pair(sm + PO_TB, sm + PO_TBG, 32 + 16 * mi + g8, 8 * ni + 2 * t4, -e[0], -e[1], bet, gam);
+                store_t_pair(sm + PO_TB, sm + PO_TBG, 40 + 16 * mi + g8, 8 * ni + 2 * t4, -e[2], -e[3], bet, gam);
+            }
+            fence_proxy_async_smem();
+            named_bar(kBarP, kNumPrep);
+            if (pt == 0) {
+                arrive(&bars[PB_TBREADY]);
+                tma_store_2d(&tm_tb, sm + PO_TB, 0, (int)(gi * 64));
+                bulk_commit();
+            }
+            SDBG(1, 5)
+            // gates of the next item, while the W^T MMA runs
+            if (it + 1 < nit) prep_gates(it + 1);
+            SDBG(1, 6)
+            // ---- W^T (bf16, rows = key dim i, 64 tokens per row) from TMEM into the staging tile ----
+            if (!(ok = role_wait(&bars[PB_WDONE], par, abort_flag, kBarP, kNumPrep))) break;
+            tc_fence_after();
+            {
+                const int i = (warp & 3) * 32 + lane;
+                uint32_t r[32];
+                tmem_ld32(tm + lb + TP_W + ch * 32, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    uint4 v;
+                    v.x = pack_bf16x2(__uint_as_float(r[cc * 8 + 0]), __uint_as_float(r[cc * 8 + 1]));
+                    v.y = pack_bf16x2(__uint_as_float(r[cc * 8 + 2]), __uint_as_float(r[cc * 8 + 3]));
+                    v.z = pack_bf16x2(__uint_as_float(r[cc * 8 + 4]), __uint_as_float(r[cc * 8 + 5]));
+                    v.w = pack_bf16x2(__uint_as_float(r[cc * 8 + 6]), __uint_as_float(r[cc * 8 + 7]));
+                    *reinterpret_cast<uint4 *>(sm + PO_AM + sw128(i, ch * 4 + cc)) = v;
+                }
+            }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            named_bar(kBarP, kNumPrep);
+            if (pt == 0) {
+                tma_store_2d(&tm_w, sm + PO_AM, 0, (int)(gi * 128));
+                bulk_commit();
+            }
+            SDBG(1, 7)
+        }
+        if (pt == 0) bulk_wait0();  // every workspace store has completed
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && *abort_flag) atomicExch(&g_split_timeout, 1);
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, 128);
+    }
+}
+
+// ============================================================================
+// chain kernel
+// ============================================================================
+constexpr int kChainThreads = 640;
+// warp 0: TMA producer; warp 1: chain MMA issuer; warp 2: output MMA issuer; warp 3: second
+// issuer of U^T (key dims 64..127); warps 4-11: output role; warps 12-19: chain role
+constexpr int kOutWarp0 = 4, kNumOut = 256;
+constexpr int kChnWarp0 = 12, kNumChn = 256;
+constexpr int kBarOut = 1, kBarChn = 2;
+
+// one pipeline stage (per chunk parity)
+constexpr uint32_t ST_Q = 0;        // 16 KB: two [64 t][64 d] boxes
+constexpr uint32_t ST_K = 16384;    // 16 KB
+constexpr uint32_t ST_V = 32768;    // 16 KB
+constexpr uint32_t ST_W = 49152;    // 16 KB: W^T [128 i][64 t]
+constexpr uint32_t ST_P = 65536;    // 8 KB:  P [64 t][64 s]
+constexpr uint32_t ST_TB = 73728;   // 8 KB:  TB [64 t][64 s]
+constexpr uint32_t ST_GATE = 81920; // 512 B: gamma_t [64], dl_s [64]
+constexpr uint32_t ST_BYTES = 82944;
+constexpr uint32_t CO_OST = 2 * ST_BYTES;     // 16 KB output staging: two [64 t][64 d] boxes
+constexpr uint32_t CO_BARS = CO_OST + 16384;
+constexpr uint32_t CO_MISC = CO_BARS + 256;
+constexpr uint32_t SMEM_CHAIN = CO_MISC + 64 + 1024;
+
+constexpr uint32_t TC_S = 0;      // 128  S float32 (row j in lane j)
+constexpr uint32_t TC_SB = 128;   // 2 x 64  bf16 S (A operand), per chunk parity
+constexpr uint32_t TC_DU = 256;   // 64   Ut^T, accumulated into U^T
+constexpr uint32_t TC_UB = 320;   // 2 x 32  bf16 U^T (A operand), per chunk parity
+constexpr uint32_t TC_O = 384;    // 64   O^T
+constexpr uint32_t TC_DU2 = 448;  // 64   -S W^T over key dims 64..127 (second issuer)
+
+constexpr uint32_t IDESC_C64 = instr_desc_bf16(128, 64, 0, 0);               // S . Q^T, U^T . P^T
+constexpr uint32_t IDESC_CMN = instr_desc_bf16(128, 64, 1, 0);               // V^T (MN-major A) . TB^T
+constexpr uint32_t IDESC_CWNEG = instr_desc_bf16(128, 64, 0, 1) | (1u << 14); // S . (-W)^T, W^T MN-major
+constexpr uint32_t IDESC_CS = instr_desc_bf16(128, 128, 0, 1);               // U^T . (dl K), MN-major B
+
+enum CBar {
+    CB_FULL0 = 0, CB_FULL1,        // stage tiles landed
+    CB_EMPTY0, CB_EMPTY1,          // stage consumed by the three issuers (count 3)
+    CB_QK0, CB_QK1,                // stage's Q and K scaled by the output role
+    CB_SREADY0, CB_SREADY1,        // bf16 S copy written (per SB buffer)
+    CB_UREADY0, CB_UREADY1,        // bf16 U^T written (per UB buffer)
+    CB_O1DONE0, CB_O1DONE1,        // S Q^T MMA done (SB buffer free)
+    CB_ODONE0, CB_ODONE1,          // U^T P^T MMA done (O complete, UB buffer free)
+    CB_UDONE, CB_UDONE2,           // U^T MMAs of the two issuers done
+    CB_SDONE, CB_OFREE,            // state update done, O read out
+    CB_COUNT
+};
+
+// mode 0: one CTA per (b, h, segment) computes the outputs of its chunk range
+// from that segment's entry state (S0 for the first segment, else S_entry) and
+// writes S_final from the last segment.  mode 1: two CTAs per (b, h, segment <
+// nseg - 1) compute the segment's affine transfer S_end = S_start M + B: one
+// runs from the zero state (-> Bw), the other from the identity with v = 0
+// (-> Mw; rows of the state evolve independently, so each row of M is a
+// state row with no write term).
+struct ChainArgs {
+    const float *gate_rec;  // [items][128] from the prep kernel
+    const float *S0;
+    float *S_final;
+    int64_t T, H;
+    int chunks;  // chunks per (b, h)
+    int mode, nseg, seg_len;
+    const float *S_entry;  // [B*H][nseg-1][dv][dk]
+    float *Bw, *Mw;        // [B*H][nseg-1][dv][dk] / [dk][dk]
+};
+
+__global__ void __launch_bounds__(kChainThreads, 1)
+fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                 const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_tb,
+                 const __grid_constant__ CUtensorMap tm_w, ChainArgs p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + CO_BARS);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + CO_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + CO_MISC + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t H = p.H;
+    int64_t bh;
+    int seg, kind;  // kind 0 = outputs, 1 = transfer B, 2 = transfer M
+    if (p.mode == 0) {
+        bh = blockIdx.x / p.nseg;
+        seg = (int)(blockIdx.x % p.nseg);
+        kind = 0;
+    } else {
+        const int64_t q = blockIdx.x >> 1;
+        bh = q / (p.nseg - 1);
+        seg = (int)(q % (p.nseg - 1));
+        kind = 1 + (int)(blockIdx.x & 1);
+    }
+    const bool outputs = (kind == 0);
+    const int b = (int)(bh / H), h = (int)(bh % H);
+    const int c0 = seg * p.seg_len;
+    const int N = (p.chunks - c0 < p.seg_len) ? (p.chunks - c0) : p.seg_len;
+    const int64_t item0 = bh * p.chunks + c0;  // workspace tile index of this CTA's first chunk
+    const uint32_t sbase = smem_u32(sm);
+
+    if (tid == 0) {
+        for (int i = 0; i < CB_COUNT; ++i) mbar_init(&bars[i], (i == CB_EMPTY0 || i == CB_EMPTY1) ? 3 : 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tmem_slot;
+    const uint32_t lb = (uint32_t)((warp & 3) * 32) << 16;
+
+    if (warp == 0) {
+        // ============================ producer ============================
+        if (lane == 0) {
+            bool ok = true;
+            const uint32_t bytes =
+                (outputs ? 16384 + 8192 : 0) + 16384 + 16384 + (kind != 2 ? 16384 + 8192 : 0) + (uint32_t)kGateRec;
+            for (int c = 0; c < N && ok; ++c) {
+                const int s = c & 1;
+                if (c >= 2 && !(ok = wait_bar(&bars[CB_EMPTY0 + s], ((c - 2) >> 1) & 1, abort_flag))) break;
+                uint8_t *st = sm + s * ST_BYTES;
+                uint64_t *full = &bars[CB_FULL0 + s];
+                const int t0 = (c0 + c) * kC;
+                const int row = (int)(item0 + c);
+                mbar_arrive_expect_tx(full, bytes);
+                for (int blk = 0; blk < 2; ++blk) {
+                    if (outputs) tma_load_4d(st + ST_Q + blk * 8192, &tm_q, full, blk * 64, h, t0, b);
+                    tma_load_4d(st + ST_K + blk * 8192, &tm_k, full, blk * 64, h, t0, b);
+                    if (kind != 2) tma_load_4d(st + ST_V + blk * 8192, &tm_v, full, blk * 64, h, t0, b);
+                }
+                tma_load_2d(st + ST_W, &tm_w, full, 0, row * 128);
+                if (outputs) tma_load_2d(st + ST_P, &tm_p, full, 0, row * 64);
+                if (kind != 2) tma_load_2d(st + ST_TB, &tm_tb, full, 0, row * 64);
+                bulk_load(st + ST_GATE, p.gate_rec + (int64_t)row * 128, (uint32_t)kGateRec, full);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ========================== chain issuer ==========================
+        if (lane == 0) {
+            bool ok = true;
+            for (int c = 0; c < N && ok; ++c) {
+                const int s = c & 1;
+                const uint32_t sp = (c >> 1) & 1;
+                const uint32_t st = sbase + s * ST_BYTES;
+                const uint32_t sb = TC_SB + (c & 1) * 64, ub = TC_UB + (c & 1) * 32;
+                const int it = c;
+                (void)it;
+                SDBG(2, 0)
+                if (!(ok = wait_bar(&bars[CB_FULL0 + s], sp, abort_flag))) break;
+                tc_fence_after();
+                // Ut^T = V^T TB^T (transfer-M runs have v = 0: U^T starts fresh below)
+                if (kind != 2) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss(tm + TC_DU, smem_desc_sw128(st + ST_V + kk * 2048, 8192, 1024),
+                               smem_desc_sw128(st + ST_TB + kk * 32, 16, 1024), IDESC_CMN, kk > 0);
+                }
+                if (!(ok = wait_bar(&bars[CB_SREADY0 + (c & 1)], sp, abort_flag))) break;
+                SDBG(2, 1)
+                tc_fence_after();
+                // U^T = Ut^T - S W^T over key dims 0..63 (the second issuer takes 64..127)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ts(tm + TC_DU, tm + sb + kk * 8, smem_desc_sw128(st + ST_W + kk * 2048, 8192, 1024),
+                           IDESC_CWNEG, (kind != 2 || kk > 0) ? 1u : 0u);
+                mma_commit(&bars[CB_UDONE]);
+                SDBG(2, 2)
+                if (!(ok = wait_bar(&bars[CB_UREADY0 + (c & 1)], sp, abort_flag))) break;
+                if (!(ok = wait_bar(&bars[CB_QK0 + s], sp, abort_flag))) break;
+                SDBG(2, 3)
+                tc_fence_after();
+                // S += U^T (diag(dl) K)   (S was scaled by gamma_C when its bf16 copy was made)
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ts(tm + TC_S, tm + ub + kk * 8, smem_desc_sw128(st + ST_K + kk * 2048, 8192, 1024), IDESC_CS,
+                           1);
+                mma_commit(&bars[CB_SDONE]);
+                mma_commit(&bars[CB_EMPTY0 + s]);
+                SDBG(2, 4)
+            }
+        }
+        __syncwarp();
+    } else if (warp == 2) {
+        // ========================= output issuer =========================
+        if (lane == 0) {
+            bool ok = true;
+            for (int c = 0; c < N && ok; ++c) {
+                const int s = c & 1;
+                const uint32_t sp = (c >> 1) & 1;
+                const uint32_t st = sbase + s * ST_BYTES;
+                const uint32_t sb = TC_SB + (c & 1) * 64, ub = TC_UB + (c & 1) * 32;
+                const int it = c;
+                (void)it;
+                SDBG(3, 0)
+                if (!(ok = wait_bar(&bars[CB_QK0 + s], sp, abort_flag))) break;
+                if (!(ok = wait_bar(&bars[CB_SREADY0 + (c & 1)], sp, abort_flag))) break;
+                if (c > 0 && !(ok = wait_bar(&bars[CB_OFREE], (c - 1) & 1, abort_flag))) break;
+                SDBG(3, 1)
+                tc_fence_after();
+                // O^T = S (diag(gamma) Q)^T  (transfer runs issue no output MMAs; the commits still arrive)
+                if (outputs) {
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(tm + TC_O, tm + sb + kk * 8,
+                               smem_desc_sw128(st + ST_Q + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), IDESC_C64,
+                               kk > 0);
+                }
+                mma_commit(&bars[CB_O1DONE0 + (c & 1)]);
+                if (!(ok = wait_bar(&bars[CB_UREADY0 + (c & 1)], sp, abort_flag))) break;
+                SDBG(3, 2)
+                tc_fence_after();
+                // O^T += U^T P^T
+                if (outputs) {
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts(tm + TC_O, tm + ub + kk * 8, smem_desc_sw128(st + ST_P + kk * 32, 16, 1024),
+                               IDESC_C64, 1);
+                }
+                mma_commit(&bars[CB_ODONE0 + (c & 1)]);
+                mma_commit(&bars[CB_EMPTY0 + s]);
+                SDBG(3, 3)
+            }
+        }
+        __syncwarp();
+    } else if (warp == 3) {
+        // ====================== second U^T issuer ======================
+        if (lane == 0) {
+            bool ok = true;
+            for (int c = 0; c < N && ok; ++c) {
+                const int s = c & 1;
+                const uint32_t sp = (c >> 1) & 1;
+                const uint32_t st = sbase + s * ST_BYTES;
+                const uint32_t sb = TC_SB + (c & 1) * 64;
+                if (!(ok = wait_bar(&bars[CB_FULL0 + s], sp, abort_flag))) break;
+                // the chain role has read this accumulator for the previous chunk
+                if (c > 0 && !(ok = wait_bar(&bars[CB_UREADY0 + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag)))
+                    break;
+                if (!(ok = wait_bar(&bars[CB_SREADY0 + (c & 1)], sp, abort_flag))) break;
+                tc_fence_after();
+                // -S W^T over key dims 64..127
+#pragma unroll
+                for (int kk = 4; kk < 8; ++kk)
+                    mma_ts(tm + TC_DU2, tm + sb + kk * 8, smem_desc_sw128(st + ST_W + kk * 2048, 8192, 1024),
+                           IDESC_CWNEG, kk > 4 ? 1u : 0u);
+                mma_commit(&bars[CB_UDONE2]);
+                mma_commit(&bars[CB_EMPTY0 + s]);
+            }
+        }
+        __syncwarp();
+    } else if (warp >= kOutWarp0 && warp < kChnWarp0) {
+        // ============================ output role ============================
+        // gates, diag(gamma) Q and diag(dl) K in place, then the outputs of the previous chunk
+        const int ot = tid - kOutWarp0 * 32;         // 0..255
+        const int j = (warp & 3) * 32 + lane;        // TMEM lane = value dim
+        const int ch = (warp - kOutWarp0) >> 2;      // token half of the output tile
+        bool ok = true;
+        auto write_out = [&](int cprev) {
+            if (ot == 0) bulk_wait_read0();  // the previous chunk's stores have read the staging buffer
+            named_bar(kBarOut, kNumOut);
+            const int par = j & 1, colw = j - par;  // this lane writes column pair (colw, colw + 1)
+            uint8_t *stage = sm + CO_OST + (colw >> 6) * 8192;
+            const uint32_t cbyte = (colw & 7) * 2, cchunk = (colw & 63) >> 3;
+#pragma unroll 1
+            for (int piece = 0; piece < 2; ++piece) {
+                uint32_t r[16];
+                tmem_ld16(tm + lb + TC_O + ch * 32 + piece * 16, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; i += 2) {
+                    const float o0 = __uint_as_float(r[i]), o1 = __uint_as_float(r[i + 1]);
+                    // even lanes keep row t and take the neighbour's column; odd lanes keep row t+1
+                    const float send = par ? o0 : o1;
+                    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+                    const uint32_t word = par ? pack_bf16x2(recv, o1) : pack_bf16x2(o0, recv);
+                    const int row = ch * 32 + piece * 16 + i + par;
+                    *reinterpret_cast<uint32_t *>(stage + sw128(row, cchunk) + cbyte) = word;
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar(kBarOut, kNumOut);
+            if (ot == 0) {
+                tma_store_4d(&tm_o, sm + CO_OST, 0, h, (c0 + cprev) * kC, b);
+                tma_store_4d(&tm_o, sm + CO_OST + 8192, 64, h, (c0 + cprev) * kC, b);
+                bulk_commit();
+            }
+        };
+        for (int c = 0; c < N && ok; ++c) {
+            const int s = c & 1;
+            const uint32_t sp = (c >> 1) & 1;
+            uint8_t *st = sm + s * ST_BYTES;
+            const float *gam = reinterpret_cast<const float *>(st + ST_GATE), *dl = gam + 64;
+            const int it = c;
+            (void)it;
+            SDBG(4, 0)
+            if (!(ok = role_wait(&bars[CB_FULL0 + s], sp, abort_flag, kBarOut, kNumOut))) break;
+            SDBG(4, 1)
+            SDBG(4, 2)
+            // ---- scale rows in place: Q row t by gamma_t, K row s by dl_s (16-byte units; a row
+            //      of a 64-column box is one 128-byte line whatever the swizzle) ----
+            {
+                auto scale_tile = [&](uint8_t *tile, const float *f) {
+                    uint4 v[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) v[i] = reinterpret_cast<const uint4 *>(tile)[ot + 256 * i];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float fr = f[((ot + 256 * i) >> 3) & 63];  // unit u covers bytes 16u.. of row (u/8) % 64
+                        uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[e]));
+                            w[e] = pack_bf16x2(x.x * fr, x.y * fr);
+                        }
+                        reinterpret_cast<uint4 *>(tile)[ot + 256 * i] = make_uint4(w[0], w[1], w[2], w[3]);
+                    }
+                };
+                scale_tile(st + ST_K, dl);
+                if (outputs) scale_tile(st + ST_Q, gam);
+            }
+            fence_proxy_async_smem();
+            named_bar(kBarOut, kNumOut);
+            if (ot == 0) arrive(&bars[CB_QK0 + s]);
+            SDBG(4, 3)
+            // ---- outputs of the previous chunk ----
+            if (c > 0) {
+                if (!(ok = role_wait(&bars[CB_ODONE0 + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag, kBarOut,
+                                     kNumOut)))
+                    break;
+                tc_fence_after();
+                if (outputs) write_out(c - 1);  // ends with a role barrier after the O reads
+                if (ot == 0) arrive(&bars[CB_OFREE]);
+            }
+            SDBG(4, 4)
+        }
+        if (ok && N > 0) {
+            ok = role_wait(&bars[CB_ODONE0 + ((N - 1) & 1)], ((N - 1) >> 1) & 1, abort_flag, kBarOut, kNumOut);
+            tc_fence_after();
+            if (ok && outputs) write_out(N - 1);
+        }
+        if (ot == 0) bulk_wait0();  // every output store has completed
+    } else if (warp >= kChnWarp0) {
+        // ============================ chain role ============================
+        // thread (j, ch) owns state row j and column half ch
+        const int ct = tid - kChnWarp0 * 32;       // 0..255
+        const int j = (warp & 3) * 32 + lane;      // TMEM lane / state row
+        const int ch = (warp - kChnWarp0) >> 2;    // column half
+        bool ok = true;
+        // entry state -> TMEM: S0 (or zero) for the first segment, the prefix-scanned entry state for
+        // later segments, zero for transfer-B runs and the identity for transfer-M runs
+        {
+            const float *src = nullptr;
+            if (kind == 0)
+                src = (seg == 0) ? (p.S0 ? p.S0 + (bh * kD + j) * (int64_t)kD : nullptr)
+                                 : p.S_entry + ((bh * (p.nseg - 1) + seg - 1) * kD + j) * (int64_t)kD;
+#pragma unroll 1
+            for (int piece = 0; piece < 2; ++piece) {
+                const int col0 = ch * 64 + piece * 32;
+                uint32_t r[32];
+#pragma unroll
+                for (int i = 0; i < 32; i += 4) {
+                    float4 v = src ? *reinterpret_cast<const float4 *>(src + col0 + i) : make_float4(0, 0, 0, 0);
+                    r[i] = __float_as_uint(v.x);
+                    r[i + 1] = __float_as_uint(v.y);
+                    r[i + 2] = __float_as_uint(v.z);
+                    r[i + 3] = __float_as_uint(v.w);
+                }
+                if (kind == 2) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint((col0 + i == j) ? 1.f : 0.f);
+                }
+                tmem_st32(tm + lb + TC_S + col0, r);
+            }
+            tmem_wait_st();
+        }
+        for (int c = 0; c < N && ok; ++c) {
+            const uint32_t sp = (c >> 1) & 1;
+            const uint32_t sb = TC_SB + (c & 1) * 64, ub = TC_UB + (c & 1) * 32;
+            const int it = c;
+            (void)it;
+            SDBG(5, 0)
+            if (c > 0 && !(ok = role_wait(&bars[CB_SDONE], (c - 1) & 1, abort_flag, kBarChn, kNumChn))) break;
+            // the bf16 copy buffer of this parity was last read by the output MMA of chunk c - 2
+            if (c >= 2 && !(ok = role_wait(&bars[CB_O1DONE0 + (c & 1)], ((c - 2) >> 1) & 1, abort_flag, kBarChn,
+                                           kNumChn)))
+                break;
+            // this chunk's gates have landed with its stage: gamma_C = gamma_63
+            if (!(ok = role_wait(&bars[CB_FULL0 + (c & 1)], sp, abort_flag, kBarChn, kNumChn))) break;
+            const float gC = reinterpret_cast<const float *>(sm + (c & 1) * ST_BYTES + ST_GATE)[63];
+            tc_fence_after();
+            SDBG(5, 1)
+            // ---- bf16 operand copy of S, then S <- gamma_C S (row j, 64 columns) ----
+#pragma unroll 1
+            for (int piece = 0; piece < 2; ++piece) {
+                const int col0 = ch * 64 + piece * 32;
+                uint32_t r[32];
+                tmem_ld32(tm + lb + TC_S + col0, r);
+                tmem_wait_ld();
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 32; i += 2)
+                    pk[i >> 1] = pack_bf16x2(__uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+                tmem_st16(tm + lb + sb + col0 / 2, pk);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * gC);
+                tmem_st32(tm + lb + TC_S + col0, r);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            named_bar(kBarChn, kNumChn);
+            if (ct == 0) arrive(&bars[CB_SREADY0 + (c & 1)]);
+            SDBG(5, 2)
+            if (!(ok = role_wait(&bars[CB_UDONE], c & 1, abort_flag, kBarChn, kNumChn))) break;
+            if (!(ok = role_wait(&bars[CB_UDONE2], c & 1, abort_flag, kBarChn, kNumChn))) break;
+            // the bf16 U^T buffer of this parity was last read by the output MMA of chunk c - 2
+            if (c >= 2 && !(ok = role_wait(&bars[CB_ODONE0 + (c & 1)], ((c - 2) >> 1) & 1, abort_flag, kBarChn,
+                                           kNumChn)))
+                break;
+            tc_fence_after();
+            SDBG(5, 3)
+            // ---- U^T = (Ut^T - S W^T over dims 0..63) + (-S W^T over 64..127) -> bf16 (32 tokens) ----
+#pragma unroll 1
+            for (int piece = 0; piece < 2; ++piece) {
+                uint32_t u[16], u2[16], pk[8];
+                tmem_ld16(tm + lb + TC_DU + ch * 32 + piece * 16, u);
+                tmem_ld16(tm + lb + TC_DU2 + ch * 32 + piece * 16, u2);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; i += 2)
+                    pk[i >> 1] = pack_bf16x2(__uint_as_float(u[i]) + __uint_as_float(u2[i]),
+                                             __uint_as_float(u[i + 1]) + __uint_as_float(u2[i + 1]));
+                tmem_st8(tm + lb + ub + ch * 16 + piece * 8, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            named_bar(kBarChn, kNumChn);
+            if (ct == 0) arrive(&bars[CB_UREADY0 + (c & 1)]);
+            SDBG(5, 4)
+        }
+        if (ok && N > 0) {
+            ok = role_wait(&bars[CB_SDONE], (N - 1) & 1, abort_flag, kBarChn, kNumChn);
+            tc_fence_after();
+        }
+        float *dst = nullptr;
+        if (kind == 0)
+            dst = (seg == p.nseg - 1 && p.S_final) ? p.S_final + (bh * kD + j) * (int64_t)kD : nullptr;
+        else
+            dst = (kind == 1 ? p.Bw : p.Mw) + ((bh * (p.nseg - 1) + seg) * kD + j) * (int64_t)kD;
+        if (ok && dst) {
+#pragma unroll 1
+            for (int piece = 0; piece < 2; ++piece) {
+                const int col0 = ch * 64 + piece * 32;
+                uint32_t r[32];
+                tmem_ld32(tm + lb + TC_S + col0, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; i += 4)
+                    *reinterpret_cast<float4 *>(dst + col0 + i) =
+                        make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]), __uint_as_float(r[i + 2]),
+                                    __uint_as_float(r[i + 3]));
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && *abort_flag) atomicExch(&g_split_timeout, 1);
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, 512);
+    }
+}
+
+bool configure_once(const void *fn, uint32_t smem, std::atomic<uint64_t> &done) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (done.load() & bit) return true;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) return false;
+    done.fetch_or(bit);
+    return true;
+}
+
+}  // namespace
+
+#ifdef GDN_TC_DEBUG
+extern "C" int gdn_debug_set_split_dump(long long *ptr) {
+    return cudaMemcpyToSymbol(g_split_dbg, &ptr, sizeof(ptr)) == cudaSuccess ? 0 : 1;
+}
+#endif
+
+bool fwd_split_supported(const FwdProblem &p) {
+    if (!fwd_tc_supported(p)) return false;
+    const int64_t items = p.B * p.H * ((p.T + kC - 1) / kC);
+    return items * 128 < ((int64_t)1 << 31);  // tile-row coordinates of the workspace maps fit in int32
+}
+
+size_t fwd_split_workspace_bytes(const FwdProblem &p, int nseg) {
+    const size_t items = (size_t)(p.B * p.H) * (size_t)((p.T + kC - 1) / kC);
+    return items * kWsPerChunk + fwd_tc_workspace_bytes(p, nseg);
+}
+
+cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *workspace, cudaStream_t stream) {
+    const int64_t chunks = (p.T + kC - 1) / kC, heads = p.B * p.H, items = heads * chunks;
+    if (items == 0) return cudaSuccess;
+    if (!workspace) return cudaErrorInvalidValue;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint8_t *ws_p = ws, *ws_tb = ws + items * kTileP, *ws_w = ws_tb + items * kTileTB;
+    float *ws_gates = reinterpret_cast<float *>(ws_w + items * kTileW);
+    float *seg_ws = reinterpret_cast<float *>(ws + items * kWsPerChunk);
+    CUtensorMap mq, mk, mv, mo, mp, mtb, mw;
+    if (!make_map_bthd(&mq, p.q, p.B, p.T, p.H) || !make_map_bthd(&mk, p.k, p.B, p.T, p.H) ||
+        !make_map_bthd(&mv, p.v, p.B, p.T, p.H) || !make_map_bthd(&mo, p.out, p.B, p.T, p.H) ||
+        !make_map_tiles(&mp, ws_p, items, 64) || !make_map_tiles(&mtb, ws_tb, items, 64) ||
+        !make_map_tiles(&mw, ws_w, items, 128))
+        return cudaErrorInvalidValue;
+    static std::atomic<uint64_t> conf_prep{0}, conf_chain{0};
+    if (!configure_once((const void *)fwd_prep_kernel, SMEM_PREP, conf_prep) ||
+        !configure_once((const void *)fwd_chain_kernel, SMEM_CHAIN, conf_chain))
+        return cudaErrorInvalidValue;
+
+    PrepArgs pa;
+    pa.log_alpha = p.log_alpha;
+    pa.beta = p.beta;
+    pa.gate_rec = ws_gates;
+    pa.T = p.T;
+    pa.H = p.H;
+    pa.items = items;
+    pa.chunks = (int)chunks;
+    const int64_t pgrid = items < 2 * (int64_t)sm_count ? items : 2 * (int64_t)sm_count;
+    fwd_prep_kernel<<<(unsigned)pgrid, kPrepThreads, SMEM_PREP, stream>>>(mq, mk, mp, mtb, mw, pa);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    ChainArgs a;
+    a.gate_rec = ws_gates;
+    a.S0 = p.S0;
+    a.S_final = p.S_final;
+    a.T = p.T;
+    a.H = p.H;
+    a.chunks = (int)chunks;
+    if (nseg < 1) nseg = 1;
+    a.seg_len = (int)((chunks + nseg - 1) / nseg);
+    a.nseg = (int)((chunks + a.seg_len - 1) / a.seg_len);
+    a.S_entry = nullptr;
+    a.Bw = a.Mw = nullptr;
+    if (a.nseg > 1) {
+        const size_t per = (size_t)heads * (a.nseg - 1) * kD * kD;
+        a.Bw = seg_ws;
+        a.Mw = a.Bw + per;
+        float *entry = a.Mw + per;
+        a.S_entry = entry;
+        a.mode = 1;  // segment transfers of segments 0..nseg-2
+        fwd_chain_kernel<<<(unsigned)(heads * (a.nseg - 1) * 2), kChainThreads, SMEM_CHAIN, stream>>>(
+            mq, mk, mv, mo, mp, mtb, mw, a);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        e = launch_seg_prefix(p.S0, a.Bw, a.Mw, entry, heads, a.nseg, stream);
+        if (e != cudaSuccess) return e;
+    }
+    a.mode = 0;  // outputs of every segment from its entry state
+    fwd_chain_kernel<<<(unsigned)(heads * a.nseg), kChainThreads, SMEM_CHAIN, stream>>>(mq, mk, mv, mo, mp, mtb, mw,
+                                                                                        a);
+    return cudaGetLastError();
+}
+
+}  // namespace gdn

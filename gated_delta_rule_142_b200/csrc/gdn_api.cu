@@ -80,6 +80,46 @@ struct Span {
 };
 bool overlaps(const Span &a, const Span &b) { return !a.empty() && !b.empty() && a.lo < b.hi && b.lo < a.hi; }
 
+// ---------------------------------------------------------------- scratch pool
+// Scratch (the per-chunk workspace, segment transfers, host staging) comes
+// from a library-private stream-ordered pool per device whose release
+// threshold keeps freed memory mapped: a repeated call of the same size takes
+// its scratch back from the pool instead of mapping new memory.
+// gdn_scratch_release() returns what is not in use to the driver.
+std::atomic<cudaMemPool_t> g_pool[kMaxDevices];
+
+cudaMemPool_t scratch_pool(int dev) {
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    cudaMemPool_t pool = g_pool[dev].load(std::memory_order_acquire);
+    if (pool) return pool;
+    cudaMemPoolProps props;
+    memset(&props, 0, sizeof(props));
+    props.allocType = cudaMemAllocationTypePinned;
+    props.handleTypes = cudaMemHandleTypeNone;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    uint64_t keep = UINT64_MAX;
+    cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    cudaMemPool_t expected = nullptr;
+    if (!g_pool[dev].compare_exchange_strong(expected, pool)) {
+        cudaMemPoolDestroy(pool);  // another thread created this device's pool first
+        pool = expected;
+    }
+    return pool;
+}
+
+cudaError_t scratch_alloc(void **p, size_t bytes, cudaStream_t stream) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+    cudaMemPool_t pool = scratch_pool(dev);
+    if (!pool) return cudaErrorMemoryAllocation;
+    return cudaMallocFromPoolAsync(p, bytes, pool, stream);
+}
+
 // ---------------------------------------------------------------- staging
 bool is_device_pointer(const void *p) {
     cudaPointerAttributes attr;
@@ -106,7 +146,7 @@ struct Stager {
             return GDN_OK;
         }
         void *d = nullptr;
-        if (cudaMallocAsync(&d, (size_t)bytes, stream) != cudaSuccess) {
+        if (scratch_alloc(&d, (size_t)bytes, stream) != cudaSuccess) {
             cudaGetLastError();
             return GDN_ERR_ALLOC;
         }
@@ -128,17 +168,35 @@ struct Stager {
     }
 };
 
-enum class FwdPath { Auto, Simt };
+// GDN_FORWARD_PATH=simt forces the float32 CUDA-core forward, =fused the
+// single-kernel tensor-core forward; otherwise the two-kernel tensor-core
+// forward serves every shape it supports.
+enum class FwdPath { Auto, Simt, Fused };
 
 FwdPath forced_path() {
     const char *e = getenv("GDN_FORWARD_PATH");
     if (e && strcmp(e, "simt") == 0) return FwdPath::Simt;
+    if (e && strcmp(e, "fused") == 0) return FwdPath::Fused;
     return FwdPath::Auto;
 }
 
 }  // namespace
 
 extern "C" {
+
+int gdn_scratch_release(void) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+        cudaGetLastError();
+        return GDN_ERR_DEVICE;
+    }
+    cudaMemPool_t pool = dev < kMaxDevices ? g_pool[dev].load(std::memory_order_acquire) : nullptr;
+    if (pool && cudaMemPoolTrimTo(pool, 0) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_DEVICE;
+    }
+    return GDN_OK;
+}
 
 const char *gdn_status_string(int status) {
     switch (status) {
@@ -216,17 +274,31 @@ int gdn_forward(const void *q, const void *k, const void *v, const float *log_al
                      : cudaMemsetAsync(p.S_final, 0, (size_t)nstate, stream);
         }
     } else {
-        if (forced_path() != FwdPath::Simt && gdn::fwd_tc_supported(p)) {
+        const FwdPath path = forced_path();
+        bool done = false;
+        if (path == FwdPath::Auto && gdn::fwd_split_supported(p)) {
+            const int nseg = gdn::fwd_tc_segments(p, info.sm_count);
+            void *ws = nullptr;
+            if (scratch_alloc(&ws, gdn::fwd_split_workspace_bytes(p, nseg), stream) == cudaSuccess) {
+                e = gdn::launch_fwd_split(p, nseg, info.sm_count, ws, stream);
+                cudaFreeAsync(ws, stream);
+                done = true;
+            } else {
+                // too little device memory for the per-chunk workspace: the single-kernel path below
+                cudaGetLastError();
+            }
+        }
+        if (!done && path != FwdPath::Simt && gdn::fwd_tc_supported(p)) {
             const int nseg = gdn::fwd_tc_segments(p, info.sm_count);
             const size_t ws_bytes = gdn::fwd_tc_workspace_bytes(p, nseg);
             void *ws = nullptr;
-            if (ws_bytes > 0 && cudaMallocAsync(&ws, ws_bytes, stream) != cudaSuccess) {
+            if (ws_bytes > 0 && scratch_alloc(&ws, ws_bytes, stream) != cudaSuccess) {
                 cudaGetLastError();
                 return GDN_ERR_ALLOC;
             }
             e = gdn::launch_fwd_tc(p, nseg, ws, stream);
             if (ws) cudaFreeAsync(ws, stream);
-        } else {
+        } else if (!done) {
             e = gdn::launch_fwd_simt(p, info.sm_count, stream);
         }
     }
@@ -257,7 +329,12 @@ int gdn_forward_plan(int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv, in
     p.out = nullptr;
     p.S_final = nullptr;
     p.B = B; p.T = T; p.H = H; p.dk = dk; p.dv = dv; p.chunk = chunk; p.dtype = dtype;
-    if (forced_path() != FwdPath::Simt && gdn::fwd_tc_supported(p)) {
+    const FwdPath path = forced_path();
+    if (path == FwdPath::Auto && gdn::fwd_split_supported(p)) {
+        const int nseg = gdn::fwd_tc_segments(p, info.sm_count);
+        if (scratch_bytes) *scratch_bytes = (int64_t)gdn::fwd_split_workspace_bytes(p, nseg);
+        if (launches) *launches = nseg > 1 ? 4 : 2;
+    } else if (path != FwdPath::Simt && gdn::fwd_tc_supported(p)) {
         const int nseg = gdn::fwd_tc_segments(p, info.sm_count);
         if (scratch_bytes) *scratch_bytes = (int64_t)gdn::fwd_tc_workspace_bytes(p, nseg);
         if (launches) *launches = nseg > 1 ? 3 : 1;

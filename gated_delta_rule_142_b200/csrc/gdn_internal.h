@@ -44,5 +44,17 @@ bool fwd_tc_supported(const FwdProblem &p);
 int fwd_tc_segments(const FwdProblem &p, int sm_count);
 size_t fwd_tc_workspace_bytes(const FwdProblem &p, int nseg);
 cudaError_t launch_fwd_tc(const FwdProblem &p, int nseg, void *workspace, cudaStream_t stream);
+// Entry states of segments 1..nseg-1 from the segment transfers, in float32.
+cudaError_t launch_seg_prefix(const float *S0, const float *Bw, const float *Mw, float *S_entry, int64_t heads,
+                              int nseg, cudaStream_t stream);
+
+// fwd_split.cu -- the same forward as two kernels: a chunk-parallel prep
+// kernel writes P, T diag(beta) and W^T of every chunk to the workspace, and
+// a chain kernel runs the state recurrence and the outputs from them.  The
+// workspace (fwd_split_workspace_bytes) holds 32 KB per chunk plus the
+// segment scratch of fwd_tc_workspace_bytes.
+bool fwd_split_supported(const FwdProblem &p);
+size_t fwd_split_workspace_bytes(const FwdProblem &p, int nseg);
+cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *workspace, cudaStream_t stream);
 
 }  // namespace gdn

@@ -113,8 +113,9 @@ int gdn_forward(const void *q, const void *k, const void *v, const float *log_al
 /*
  * gdn_forward_plan -- what a gdn_forward call with these sizes will do on the
  * current device, without doing it: *scratch_bytes receives the device scratch
- * it takes from the stream-ordered allocator (segment transfers and entry
- * states; 0 when the sequence is not split into segments, and excluding host
+ * it takes from the library's scratch pool (the per-chunk workspace of the
+ * two-kernel tensor-core forward, 32.5 KB per chunk, plus the segment
+ * transfers and entry states of long sequences with few heads; excluding host
  * staging), *launches the number of kernels it launches (0 for empty
  * problems).  Either output pointer may be NULL.  Returns the status the
  * argument checks of gdn_forward would return, or GDN_ERR_DEVICE.
@@ -155,11 +156,14 @@ int gdn_decode_step(const void *q, const void *k, const void *v, const float *lo
  *   - every pointer must be device (or managed) memory: host buffers, which
  *     gdn_forward stages through temporary device buffers, are rejected with
  *     GDN_ERR_UNSUPPORTED;
- *   - the scratch that long sequences with few heads need (segment transfers
- *     and entry states) lives in one library-owned device array of
+ *   - the scratch lives in one library-owned device array of
  *     GDN_NOALLOC_SCRATCH_BYTES, which every GPU that loads the library holds
- *     until the process exits; a problem that needs more than that returns
- *     GDN_ERR_SCRATCH_LIMIT before anything is enqueued;
+ *     until the process exits.  It holds the per-chunk workspace of the
+ *     two-kernel tensor-core forward when that fits (32.5 KB per chunk),
+ *     else the call runs the single-kernel tensor-core forward, whose only
+ *     scratch is the segment transfers and entry states of long sequences
+ *     with few heads; a problem that needs more than the array holds either
+ *     way returns GDN_ERR_SCRATCH_LIMIT before anything is enqueued;
  *   - no cudaMalloc, cudaMallocAsync, cudaFree or other allocating routine is
  *     called.
  * The first call on a device looks up the array's device address on that
@@ -173,6 +177,18 @@ int gdn_forward_noalloc(const void *q, const void *k, const void *v, const float
                         const float *beta, const float *S0, void *out, float *S_final, int64_t B,
                         int64_t T, int64_t H, int64_t dk, int64_t dv, int64_t chunk, void *stream,
                         int dtype);
+
+/*
+ * gdn_scratch_release -- gdn_forward and gdn_decode_step take their device
+ * scratch (the per-chunk workspace, segment transfers, copies of host
+ * buffers) from a stream-ordered memory pool private to the library, one per
+ * device, that keeps freed memory mapped between calls, so that repeated
+ * calls do not map new memory each time.  The paper has no counterpart to
+ * this housekeeping call.  It returns the pool's memory that no call is
+ * using on the current device to the driver; memory of calls still executing
+ * stays with them until they complete.  Returns GDN_OK, or GDN_ERR_DEVICE.
+ */
+int gdn_scratch_release(void);
 
 /* Static, NUL-terminated description of a gdn_status value. */
 const char *gdn_status_string(int status);

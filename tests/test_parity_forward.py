@@ -202,11 +202,28 @@ def test_segmented_fast_decay(monkeypatch):
     check(inp, "bf16", 64, label="segments fast decay")
 
 
-def test_forward_plan_reports_scratch_and_launches():
-    """The planning query agrees with what the forward does: one launch and no scratch for many heads,
-    three launches and segment scratch for a long sequence with few heads."""
+def test_forward_plan_reports_scratch_and_launches(monkeypatch):
+    """The planning query agrees with what the forward does.  Two-kernel path: 32.5 KB of workspace
+    per chunk and two launches, plus segment scratch and two more launches for a long sequence
+    with few heads.  Single-kernel path: no scratch and one launch, or segment scratch and three."""
+    per_chunk, seg_unit = 32768 + 512, 3 * 16 * 128 * 128 * 4
     s, n = gdn.forward_plan(8, 2048, 16, 128, 128, 64)
-    assert (s, n) == (0, 1)
+    assert (s, n) == (8 * 16 * 32 * per_chunk, 2)
     s, n = gdn.forward_plan(1, 65536, 16, 128, 128, 64)
-    assert n == 3 and s > 0 and s % (3 * 16 * 128 * 128 * 4) == 0
+    rest = s - 16 * 1024 * per_chunk
+    assert n == 4 and rest > 0 and rest % seg_unit == 0
     assert gdn.forward_plan(1, 100, 2, 64, 64, 32) == (0, 1)  # CUDA-core path
+    monkeypatch.setenv("GDN_FORWARD_PATH", "fused")
+    assert gdn.forward_plan(8, 2048, 16, 128, 128, 64) == (0, 1)
+    s, n = gdn.forward_plan(1, 65536, 16, 128, 128, 64)
+    assert n == 3 and s > 0 and s % seg_unit == 0
+
+
+@pytest.mark.parametrize("T,nseg", [(130, 1), (1000, 3)])
+def test_single_kernel_path(monkeypatch, T, nseg):
+    """The single-kernel tensor-core forward (used when the two-kernel workspace cannot be had)
+    meets the same bar, with and without segments."""
+    monkeypatch.setenv("GDN_FORWARD_PATH", "fused")
+    monkeypatch.setenv("GDN_SEGMENTS", str(nseg))
+    inp = forward_inputs(2, T, 2, 128, 128, "bf16", seed=73 + T, s0_std=0.1, alpha_mu=-3.0)
+    check(inp, "bf16", 64, label="single kernel T=%d segments=%d" % (T, nseg))
