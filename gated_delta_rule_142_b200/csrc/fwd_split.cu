@@ -10,7 +10,7 @@
 // chunk-local log-decay cumsum g_t, gamma_t = e^{g_t}, dl_s = e^{g_C - g_s}:
 //
 //   prep kernel (independent of the state; every chunk of every (b, h) in
-//   parallel, persistent CTAs, two per SM):
+//   parallel, persistent CTAs, three per SM):
 //     G   = [Q; K] K^T                                          (tcgen05, M = 128)
 //     P   = lower(e^{g_t - g_s} (Q K^T)_ts)                     -> workspace, bf16
 //     A   = strict_lower(beta_t e^{g_t - g_s} (K K^T)_ts)
@@ -60,10 +60,11 @@ __device__ int g_split_timeout;  // set when a bounded mbarrier wait gives up
 // Debug builds only: per-phase clock stamps of CTA 0 for its first 8 work
 // items, 8 rows of 16 int64 per item.
 __device__ long long *g_split_dbg;
-#define SDBG(row, i)                                                                   \
-    if (g_split_dbg != nullptr && blockIdx.x == 0 && it < 8)                           \
-        g_split_dbg[(it * 8 + (row)) * 16 + (i)] = clock64();
+#define SDBG_INIT long long *const dbgp = (blockIdx.x == 0) ? g_split_dbg : nullptr;
+#define SDBG(row, i) \
+    if (dbgp != nullptr && it < 8) dbgp[(it * 8 + (row)) * 16 + (i)] = clock64();
 #else
+#define SDBG_INIT
 #define SDBG(row, i)
 #endif
 
@@ -76,17 +77,20 @@ constexpr int kBarP = 1;
 constexpr int LDM = 68;   // row stride (floats) of the fp32 64x64 tiles
 constexpr int LDX2 = 40;  // row stride of the 32->64 merge scratch
 
+// 73 KB in all, so that three CTAs share an SM.
 constexpr uint32_t PO_QK = 0;        // 32 KB: per 64-column block j: [Q 8 KB | K 8 KB]
+constexpr uint32_t PO_P = 0;         // 8 KB  P [t][s] staging, in the Q block 0 once G is done
 constexpr uint32_t PO_TB = 32768;    // 8 KB  T diag(beta)       [t][s], 128-byte swizzle
 constexpr uint32_t PO_TBG = 40960;   // 8 KB  T diag(beta gamma) [t][s]
-constexpr uint32_t PO_P = 49152;     // 8 KB  P [t][s]
-constexpr uint32_t PO_AM = 57344;    // 17 KB A fp32 [64][LDM]; after the inverse: W^T bf16 [128][64] staging
-constexpr uint32_t PO_TM = 74752;    // 17 KB T fp32 [64][LDM]
-constexpr uint32_t PO_XS = 92160;    // 5 KB  merge scratch
-constexpr uint32_t PO_PG = 97280;    // gates per item parity: g, beta, gamma, e^{g-c}, e^{c-g} (2 x 5 x 64)
-constexpr uint32_t PO_BARS = 99840;  // mbarriers
-constexpr uint32_t PO_MISC = 99904;  // tmem slot, abort flag, scan scratch, flags
-constexpr uint32_t SMEM_PREP = 99968 + 1024;
+constexpr uint32_t PO_AM = 49152;    // 17 KB A fp32 [64][LDM], overwritten by T in place; after the inverse:
+                                     //       W^T bf16 [128][64] staging
+constexpr uint32_t PO_XS = 66560;    // 5 KB  merge scratch
+constexpr uint32_t PO_PG = 71680;    // gates per item parity: g, beta, gamma, e^{g-c}, e^{c-g} (2 x 5 x 64)
+constexpr uint32_t PO_BARS = 74240;  // mbarriers
+constexpr uint32_t PO_MISC = 74304;  // tmem slot, abort flag, scan scratch, flags
+constexpr uint32_t SMEM_PREP = 74368 + 1024;
+constexpr int kPrepCtasPerSm = 3;
+constexpr int kBarMerge = 2;  // named barrier of the four 16->32 merge warps
 
 constexpr uint32_t TP_G = 0;   // 64 columns: [Q;K] K^T
 constexpr uint32_t TP_W = 64;  // 64 columns: W^T
@@ -94,7 +98,7 @@ constexpr uint32_t TP_W = 64;  // 64 columns: W^T
 constexpr uint32_t IDESC_G = instr_desc_bf16(128, 64, 0, 0);     // [Q;K] . K^T
 constexpr uint32_t IDESC_MN64 = instr_desc_bf16(128, 64, 1, 0);  // K^T / V^T (MN-major A) . T^T
 
-enum PBar { PB_QFULL = 0, PB_KFULL, PB_GDONE, PB_GFREE, PB_TBREADY, PB_WDONE, PB_COUNT };
+enum PBar { PB_QFULL = 0, PB_KFULL, PB_GDONE, PB_GFREE, PB_TBREADY, PB_WDONE, PB_QFREE, PB_COUNT };
 
 struct PrepArgs {
     const float *log_alpha, *beta;
@@ -104,7 +108,7 @@ struct PrepArgs {
     int chunks;     // chunks per (b, h)
 };
 
-__global__ void __launch_bounds__(kPrepThreads, 2)
+__global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
 fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_tb,
                 const __grid_constant__ CUtensorMap tm_w, PrepArgs p) {
@@ -118,9 +122,19 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t T = p.T, H = p.H;
+    SDBG_INIT
     // work items of this CTA: global chunk ids blockIdx.x, blockIdx.x + gridDim.x, ...
     const int nit = (blockIdx.x < p.items) ? (int)((p.items - 1 - blockIdx.x) / gridDim.x + 1) : 0;
-    auto item = [&](int it) { return (int64_t)blockIdx.x + (int64_t)it * gridDim.x; };
+    // items < 2^24 (checked on the host), so 32-bit index arithmetic suffices
+    auto item = [&](int it) -> uint32_t { return blockIdx.x + (uint32_t)it * gridDim.x; };
+    // (b, h, first token) of work item `it`
+    auto coords = [&](int it, int &b, int &h, int &t0) {
+        const uint32_t gi = item(it), bh = gi / (uint32_t)p.chunks;
+        const uint32_t hh = (uint32_t)H;
+        b = (int)(bh / hh);
+        h = (int)(bh - (uint32_t)b * hh);
+        t0 = (int)(gi - bh * (uint32_t)p.chunks) * kC;
+    };
     const uint32_t sbase = smem_u32(sm);
 
     if (tid == 0) {
@@ -141,12 +155,6 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     if (warp == 0) {
         // ============================ issuer ============================
         if (lane == 0) {
-            auto coords = [&](int it, int &b, int &h, int &t0) {
-                const int64_t gi = item(it), bh = gi / p.chunks;
-                b = (int)(bh / H);
-                h = (int)(bh % H);
-                t0 = (int)(gi % p.chunks) * kC;
-            };
             auto load_q = [&](int it) {
                 int b, h, t0;
                 coords(it, b, h, t0);
@@ -181,9 +189,6 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                            kk > 0);
                 }
                 mma_commit(&bars[PB_GDONE]);
-                // Q is free once G is done
-                if (!(ok = wait_bar(&bars[PB_GDONE], par, abort_flag))) break;
-                if (it + 1 < nit) load_q(it + 1);
                 SDBG(0, 2)
                 if (!(ok = wait_bar(&bars[PB_TBREADY], par, abort_flag))) break;
                 SDBG(0, 3)
@@ -193,7 +198,9 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     mma_ss(tm + TP_W, smem_desc_sw128(sbase + PO_QK + 8192 + kk * 2048, 16384, 1024),
                            smem_desc_sw128(sbase + PO_TBG + kk * 32, 16, 1024), IDESC_MN64, kk > 0);
                 mma_commit(&bars[PB_WDONE]);
-                // K is free once W^T is done
+                // the Q block is free once the P tile staged in it has been stored, K once W^T is done
+                if (!(ok = wait_bar(&bars[PB_QFREE], par, abort_flag))) break;
+                if (it + 1 < nit) load_q(it + 1);
                 if (!(ok = wait_bar(&bars[PB_WDONE], par, abort_flag))) break;
                 if (it + 1 < nit) load_k(it + 1);
                 SDBG(0, 4)
@@ -207,7 +214,7 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int ch = pw >> 2;           // column half of the TMEM epilogues
         const int g8 = lane >> 2, t4 = lane & 3;  // MMA fragment coordinates
         float *Am = reinterpret_cast<float *>(sm + PO_AM);
-        float *Tm = reinterpret_cast<float *>(sm + PO_TM);
+        float *Tm = Am;  // T overwrites A block by block (see the merge steps)
         float *Xs = reinterpret_cast<float *>(sm + PO_XS);
         bool ok = true;
         // the upper triangles of the bf16 T tiles are never written below: zero both tiles once
@@ -217,10 +224,11 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // gates of work item `it` into buffer it & 1 (threads pt < 64 hold token pt)
         float la_next = 0.f, be_next = 0.f;
         auto gate_index = [&](int it, int t) -> int64_t {
-            const int64_t gi = item(it), bh = gi / p.chunks;
-            const int64_t tok = (gi % p.chunks) * kC + t;
+            int b, h, t0;
+            coords(it, b, h, t0);
+            const int64_t tok = (int64_t)t0 + t;
             if (tok >= T) return -1;
-            return ((bh / H) * T + tok) * H + bh % H;
+            return ((int64_t)b * T + tok) * H + h;
         };
         if (nit > 0 && pt < 64) {
             const int64_t x = gate_index(0, pt);
@@ -254,7 +262,7 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 gb[128 + pt] = gm;
                 gb[192 + pt] = expf(gt - cm);
                 gb[256 + pt] = expf(cm - gt);
-                float *rec = p.gate_rec + item(it) * 128;
+                float *rec = p.gate_rec + (int64_t)item(it) * 128;
                 rec[pt] = gm;
                 rec[64 + pt] = expf(gb[63] - gt);
                 // e^{g_t - g_s} = e^{g_t - c} e^{c - g_s} while every |g_t - c| < 60, so that
@@ -267,12 +275,16 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (nit > 0) prep_gates(0);
         for (int it = 0; it < nit && ok; ++it) {
             const uint32_t par = it & 1;
-            const int64_t gi = item(it);
+            const int gi = (int)item(it);
             const float *g = reinterpret_cast<const float *>(sm + PO_PG) + par * 320;
             const float *bet = g + 64, *gam = g + 128, *ea = g + 192, *eb = g + 256;
             const bool narrow = nflags[par * 2] && nflags[par * 2 + 1];
             // the stores of the previous item have finished reading P, TB and the W^T staging
-            if (pt == 0) bulk_wait_read0();
+            if (pt == 0) {
+                SDBG(1, 14)
+                bulk_wait_read0();
+                SDBG(1, 15)
+            }
             SDBG(1, 0)
             if (!(ok = role_wait(&bars[PB_GDONE], par, abort_flag, kBarP, kNumPrep))) break;
             tc_fence_after();
@@ -325,32 +337,36 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             named_bar(kBarP, kNumPrep);
             if (pt == 0) {
                 arrive(&bars[PB_GFREE]);
+                SDBG(1, 10)
                 tma_store_2d(&tm_p, sm + PO_P, 0, (int)(gi * 64));
                 bulk_commit();
+                SDBG(1, 11)
             }
             SDBG(1, 2)
             // ---- T = (I + A)^{-1} ----
-            // (1) 16x16 diagonal blocks by substitution: role warps 0..3, a column per lane; warps 0 and 2
-            //     also zero the upper 16x16 block inside their 32x32 diagonal block
-            if (pw < 4 && lane < 16) {
+            // (1) 16x16 diagonal blocks by substitution: role warps 0..3, a column per lane, written over
+            //     the block of A once every lane of the warp has read it.  Above the diagonal blocks A
+            //     is zero, as T is.
+            if (pw < 4) {
                 const int o = pw * 16;
                 float x[16];
+                if (lane < 16) {
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr) {
-                    float a0 = (rr == lane) ? 1.f : 0.f, a1 = 0.f;
+                    for (int rr = 0; rr < 16; ++rr) {
+                        float a0 = (rr == lane) ? 1.f : 0.f, a1 = 0.f;
 #pragma unroll
-                    for (int s = 0; s + 1 < rr; s += 2) {
-                        a0 -= Am[(o + rr) * LDM + o + s] * x[s];
-                        a1 -= Am[(o + rr) * LDM + o + s + 1] * x[s + 1];
+                        for (int s = 0; s + 1 < rr; s += 2) {
+                            a0 -= Am[(o + rr) * LDM + o + s] * x[s];
+                            a1 -= Am[(o + rr) * LDM + o + s + 1] * x[s + 1];
+                        }
+                        if (rr & 1) a0 -= Am[(o + rr) * LDM + o + rr - 1] * x[rr - 1];
+                        x[rr] = a0 + a1;
                     }
-                    if (rr & 1) a0 -= Am[(o + rr) * LDM + o + rr - 1] * x[rr - 1];
-                    x[rr] = a0 + a1;
                 }
+                __syncwarp();
+                if (lane < 16) {
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr) Tm[(o + rr) * LDM + o + lane] = x[rr];
-                if ((pw & 1) == 0) {
-#pragma unroll
-                    for (int rr = 0; rr < 16; ++rr) Tm[(o + rr) * LDM + o + 16 + lane] = 0.f;
+                    for (int rr = 0; rr < 16; ++rr) Tm[(o + rr) * LDM + o + lane] = x[rr];
                 }
             }
             __syncwarp();
@@ -386,7 +402,8 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     mma_tf32(dacc, a, bb);
                 }
                 store_d(xs, 8, 0, 0, dacc, g8, t4);
-                __syncwarp();
+                // both warps of a block have read A_10 before either overwrites it with T_10
+                named_bar(kBarMerge, 128);
                 float e[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk) {
@@ -405,7 +422,9 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             //     one warp per (16-row, 8-column) tile; T is lower triangular, so zero k-steps are skipped
             {
                 const int mi = pw >> 2, ni = pw & 3;
-                float *x2 = Xs;  // [32][LDX2], reuses the 16->32 scratch (a barrier separates the two)
+                // [32][LDX2], reuses the 16->32 scratch (a barrier separates the two); the result goes to
+                // the bf16 tiles only, so A[32:64, 0:32] is read in the first half alone
+                float *x2 = Xs;
                 float dacc[4] = {0.f, 0.f, 0.f, 0.f};
                 for (int kk = ni; kk < 4; ++kk) {
                     uint32_t a[4], bb[2];
@@ -429,8 +448,12 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             named_bar(kBarP, kNumPrep);
             if (pt == 0) {
                 arrive(&bars[PB_TBREADY]);
+                bulk_wait_read0();  // the P store has read its staging in the Q block
+                arrive(&bars[PB_QFREE]);
+                SDBG(1, 12)
                 tma_store_2d(&tm_tb, sm + PO_TB, 0, (int)(gi * 64));
                 bulk_commit();
+                SDBG(1, 13)
             }
             SDBG(1, 5)
             // gates of the next item, while the W^T MMA runs
@@ -479,8 +502,10 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 // chain kernel
 // ============================================================================
 constexpr int kChainThreads = 640;
-// warp 0: TMA producer; warp 1: chain MMA issuer; warp 2: output MMA issuer; warp 3: second
-// issuer of U^T (key dims 64..127); warps 4-11: output role; warps 12-19: chain role
+// warp 0: TMA producer; warp 1: Ut^T MMA issuer; warp 2: output MMA issuer; warp 3: idle;
+// warps 4-11: output role; warps 12-19: chain role, whose threads 0 and 32 issue the U^T and
+// state-update MMAs themselves (the chain is latency-bound: a hand-off to another warp costs
+// more than the issue)
 constexpr int kOutWarp0 = 4, kNumOut = 256;
 constexpr int kChnWarp0 = 12, kNumChn = 256;
 constexpr int kBarOut = 1, kBarChn = 2;
@@ -504,7 +529,7 @@ constexpr uint32_t TC_SB = 128;   // 2 x 64  bf16 S (A operand), per chunk parit
 constexpr uint32_t TC_DU = 256;   // 64   Ut^T, accumulated into U^T
 constexpr uint32_t TC_UB = 320;   // 2 x 32  bf16 U^T (A operand), per chunk parity
 constexpr uint32_t TC_O = 384;    // 64   O^T
-constexpr uint32_t TC_DU2 = 448;  // 64   -S W^T over key dims 64..127 (second issuer)
+constexpr uint32_t TC_DU2 = 448;  // 64   -S W^T over key dims 64..127
 
 constexpr uint32_t IDESC_C64 = instr_desc_bf16(128, 64, 0, 0);               // S . Q^T, U^T . P^T
 constexpr uint32_t IDESC_CMN = instr_desc_bf16(128, 64, 1, 0);               // V^T (MN-major A) . TB^T
@@ -515,12 +540,13 @@ enum CBar {
     CB_FULL0 = 0, CB_FULL1,        // stage tiles landed
     CB_EMPTY0, CB_EMPTY1,          // stage consumed by the three issuers (count 3)
     CB_QK0, CB_QK1,                // stage's Q and K scaled by the output role
-    CB_SREADY0, CB_SREADY1,        // bf16 S copy written (per SB buffer)
-    CB_UREADY0, CB_UREADY1,        // bf16 U^T written (per UB buffer)
+    CB_UDONE0, CB_UDONE1,          // first half of the U^T MMA done (so the bf16 S copy is written)
+    CB_SDONE0, CB_SDONE1,          // state update done (so the bf16 U^T is written)
     CB_O1DONE0, CB_O1DONE1,        // S Q^T MMA done (SB buffer free)
     CB_ODONE0, CB_ODONE1,          // U^T P^T MMA done (O complete, UB buffer free)
-    CB_UDONE, CB_UDONE2,           // U^T MMAs of the two issuers done
-    CB_SDONE, CB_OFREE,            // state update done, O read out
+    CB_UTDONE,                     // Ut^T MMA done
+    CB_UDONE2,                     // second half of the U^T MMA done
+    CB_OFREE,                      // O read out
     CB_COUNT
 };
 
@@ -555,6 +581,7 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t H = p.H;
+    SDBG_INIT
     int64_t bh;
     int seg, kind;  // kind 0 = outputs, 1 = transfer B, 2 = transfer M
     if (p.mode == 0) {
@@ -616,48 +643,32 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ========================== chain issuer ==========================
+        // =========================== Ut^T issuer ===========================
         if (lane == 0) {
             bool ok = true;
             for (int c = 0; c < N && ok; ++c) {
                 const int s = c & 1;
                 const uint32_t sp = (c >> 1) & 1;
                 const uint32_t st = sbase + s * ST_BYTES;
-                const uint32_t sb = TC_SB + (c & 1) * 64, ub = TC_UB + (c & 1) * 32;
                 const int it = c;
                 (void)it;
                 SDBG(2, 0)
                 if (!(ok = wait_bar(&bars[CB_FULL0 + s], sp, abort_flag))) break;
+                // the previous chunk's state update is done, so its U^T has been read out of this
+                // accumulator (and the tensor pipe is free while the chain converts the state)
+                if (c > 0 && !(ok = wait_bar(&bars[CB_SDONE0 + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag)))
+                    break;
+                SDBG(2, 1)
                 tc_fence_after();
-                // Ut^T = V^T TB^T (transfer-M runs have v = 0: U^T starts fresh below)
+                // Ut^T = V^T TB^T (transfer-M runs have v = 0: U^T starts fresh in the chain role)
                 if (kind != 2) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_ss(tm + TC_DU, smem_desc_sw128(st + ST_V + kk * 2048, 8192, 1024),
                                smem_desc_sw128(st + ST_TB + kk * 32, 16, 1024), IDESC_CMN, kk > 0);
                 }
-                if (!(ok = wait_bar(&bars[CB_SREADY0 + (c & 1)], sp, abort_flag))) break;
-                SDBG(2, 1)
-                tc_fence_after();
-                // U^T = Ut^T - S W^T over key dims 0..63 (the second issuer takes 64..127)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(tm + TC_DU, tm + sb + kk * 8, smem_desc_sw128(st + ST_W + kk * 2048, 8192, 1024),
-                           IDESC_CWNEG, (kind != 2 || kk > 0) ? 1u : 0u);
-                mma_commit(&bars[CB_UDONE]);
+                mma_commit(&bars[CB_UTDONE]);
                 SDBG(2, 2)
-                if (!(ok = wait_bar(&bars[CB_UREADY0 + (c & 1)], sp, abort_flag))) break;
-                if (!(ok = wait_bar(&bars[CB_QK0 + s], sp, abort_flag))) break;
-                SDBG(2, 3)
-                tc_fence_after();
-                // S += U^T (diag(dl) K)   (S was scaled by gamma_C when its bf16 copy was made)
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ts(tm + TC_S, tm + ub + kk * 8, smem_desc_sw128(st + ST_K + kk * 2048, 8192, 1024), IDESC_CS,
-                           1);
-                mma_commit(&bars[CB_SDONE]);
-                mma_commit(&bars[CB_EMPTY0 + s]);
-                SDBG(2, 4)
             }
         }
         __syncwarp();
@@ -673,8 +684,10 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const int it = c;
                 (void)it;
                 SDBG(3, 0)
+                // O^T is issued once the U^T MMA is done (the bf16 S copy exists, and the tensor pipe
+                // is free while the chain role converts U^T), O2 once the state update is done
                 if (!(ok = wait_bar(&bars[CB_QK0 + s], sp, abort_flag))) break;
-                if (!(ok = wait_bar(&bars[CB_SREADY0 + (c & 1)], sp, abort_flag))) break;
+                if (!(ok = wait_bar(&bars[CB_UDONE0 + (c & 1)], sp, abort_flag))) break;
                 if (c > 0 && !(ok = wait_bar(&bars[CB_OFREE], (c - 1) & 1, abort_flag))) break;
                 SDBG(3, 1)
                 tc_fence_after();
@@ -687,7 +700,7 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                kk > 0);
                 }
                 mma_commit(&bars[CB_O1DONE0 + (c & 1)]);
-                if (!(ok = wait_bar(&bars[CB_UREADY0 + (c & 1)], sp, abort_flag))) break;
+                if (!(ok = wait_bar(&bars[CB_SDONE0 + (c & 1)], sp, abort_flag))) break;
                 SDBG(3, 2)
                 tc_fence_after();
                 // O^T += U^T P^T
@@ -700,31 +713,6 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 mma_commit(&bars[CB_ODONE0 + (c & 1)]);
                 mma_commit(&bars[CB_EMPTY0 + s]);
                 SDBG(3, 3)
-            }
-        }
-        __syncwarp();
-    } else if (warp == 3) {
-        // ====================== second U^T issuer ======================
-        if (lane == 0) {
-            bool ok = true;
-            for (int c = 0; c < N && ok; ++c) {
-                const int s = c & 1;
-                const uint32_t sp = (c >> 1) & 1;
-                const uint32_t st = sbase + s * ST_BYTES;
-                const uint32_t sb = TC_SB + (c & 1) * 64;
-                if (!(ok = wait_bar(&bars[CB_FULL0 + s], sp, abort_flag))) break;
-                // the chain role has read this accumulator for the previous chunk
-                if (c > 0 && !(ok = wait_bar(&bars[CB_UREADY0 + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag)))
-                    break;
-                if (!(ok = wait_bar(&bars[CB_SREADY0 + (c & 1)], sp, abort_flag))) break;
-                tc_fence_after();
-                // -S W^T over key dims 64..127
-#pragma unroll
-                for (int kk = 4; kk < 8; ++kk)
-                    mma_ts(tm + TC_DU2, tm + sb + kk * 8, smem_desc_sw128(st + ST_W + kk * 2048, 8192, 1024),
-                           IDESC_CWNEG, kk > 4 ? 1u : 0u);
-                mma_commit(&bars[CB_UDONE2]);
-                mma_commit(&bars[CB_EMPTY0 + s]);
             }
         }
         __syncwarp();
@@ -855,22 +843,25 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             tmem_wait_st();
         }
         for (int c = 0; c < N && ok; ++c) {
+            const int s = c & 1;
             const uint32_t sp = (c >> 1) & 1;
+            const uint32_t st = sbase + s * ST_BYTES;
             const uint32_t sb = TC_SB + (c & 1) * 64, ub = TC_UB + (c & 1) * 32;
             const int it = c;
             (void)it;
             SDBG(5, 0)
-            if (c > 0 && !(ok = role_wait(&bars[CB_SDONE], (c - 1) & 1, abort_flag, kBarChn, kNumChn))) break;
-            // the bf16 copy buffer of this parity was last read by the output MMA of chunk c - 2
-            if (c >= 2 && !(ok = role_wait(&bars[CB_O1DONE0 + (c & 1)], ((c - 2) >> 1) & 1, abort_flag, kBarChn,
-                                           kNumChn)))
-                break;
-            // this chunk's gates have landed with its stage: gamma_C = gamma_63
-            if (!(ok = role_wait(&bars[CB_FULL0 + (c & 1)], sp, abort_flag, kBarChn, kNumChn))) break;
+            // the previous state update is done; the bf16 copy buffer of this parity was last read by
+            // the output MMA of chunk c - 2; this chunk's stage (with its gates) has landed
+            {
+                bool w = c == 0 || wait_bar(&bars[CB_SDONE0 + ((c - 1) & 1)], ((c - 1) >> 1) & 1, abort_flag);
+                w = w && (c < 2 || wait_bar(&bars[CB_O1DONE0 + (c & 1)], ((c - 2) >> 1) & 1, abort_flag));
+                w = w && wait_bar(&bars[CB_FULL0 + (c & 1)], sp, abort_flag);
+                if (!(ok = bar_and(kBarChn, kNumChn, w))) break;
+            }
             const float gC = reinterpret_cast<const float *>(sm + (c & 1) * ST_BYTES + ST_GATE)[63];
             tc_fence_after();
             SDBG(5, 1)
-            // ---- bf16 operand copy of S, then S <- gamma_C S (row j, 64 columns) ----
+            // ---- bf16 operand copy of S (row j, 64 columns) ----
 #pragma unroll 1
             for (int piece = 0; piece < 2; ++piece) {
                 const int col0 = ch * 64 + piece * 32;
@@ -882,24 +873,59 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 for (int i = 0; i < 32; i += 2)
                     pk[i >> 1] = pack_bf16x2(__uint_as_float(r[i]), __uint_as_float(r[i + 1]));
                 tmem_st16(tm + lb + sb + col0 / 2, pk);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            named_bar(kBarChn, kNumChn);
+            SDBG(5, 2)
+            // ---- U^T = Ut^T - S W^T: key dims 0..63 into DU (onto Ut^T), 64..127 into DU2 ----
+            if (ct == 0) {
+                if (wait_bar(&bars[CB_UTDONE], c & 1, abort_flag)) {
+                    SDBG(5, 5)
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts(tm + TC_DU, tm + sb + kk * 8, smem_desc_sw128(st + ST_W + kk * 2048, 8192, 1024),
+                               IDESC_CWNEG, (kind != 2 || kk > 0) ? 1u : 0u);
+                    mma_commit(&bars[CB_UDONE0 + (c & 1)]);
+                    SDBG(5, 6)
+                }
+            } else if (ct == 32) {
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 4; kk < 8; ++kk)
+                    mma_ts(tm + TC_DU2, tm + sb + kk * 8, smem_desc_sw128(st + ST_W + kk * 2048, 8192, 1024),
+                           IDESC_CWNEG, kk > 4 ? 1u : 0u);
+                mma_commit(&bars[CB_UDONE2]);
+                mma_commit(&bars[CB_EMPTY0 + s]);
+            }
+            // ---- S <- gamma_C S while the U^T MMAs run ----
+#pragma unroll 1
+            for (int piece = 0; piece < 2; ++piece) {
+                const int col0 = ch * 64 + piece * 32;
+                uint32_t r[32];
+                tmem_ld32(tm + lb + TC_S + col0, r);
+                tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * gC);
                 tmem_st32(tm + lb + TC_S + col0, r);
             }
             tmem_wait_st();
-            tc_fence_before();
-            named_bar(kBarChn, kNumChn);
-            if (ct == 0) arrive(&bars[CB_SREADY0 + (c & 1)]);
-            SDBG(5, 2)
-            if (!(ok = role_wait(&bars[CB_UDONE], c & 1, abort_flag, kBarChn, kNumChn))) break;
-            if (!(ok = role_wait(&bars[CB_UDONE2], c & 1, abort_flag, kBarChn, kNumChn))) break;
-            // the bf16 U^T buffer of this parity was last read by the output MMA of chunk c - 2
-            if (c >= 2 && !(ok = role_wait(&bars[CB_ODONE0 + (c & 1)], ((c - 2) >> 1) & 1, abort_flag, kBarChn,
-                                           kNumChn)))
-                break;
+            SDBG(5, 7)
+            // both U^T halves are done; the bf16 U^T buffer of this parity was last read by the
+            // output MMA of chunk c - 2
+            {
+                bool w = wait_bar(&bars[CB_UDONE0 + (c & 1)], sp, abort_flag);
+                SDBG(5, 8)
+                w = w && wait_bar(&bars[CB_UDONE2], c & 1, abort_flag);
+                SDBG(5, 9)
+                w = w && (c < 2 || wait_bar(&bars[CB_ODONE0 + (c & 1)], ((c - 2) >> 1) & 1, abort_flag));
+                if (!(ok = bar_and(kBarChn, kNumChn, w))) break;
+            }
             tc_fence_after();
+            SDBG(5, 10)
             SDBG(5, 3)
-            // ---- U^T = (Ut^T - S W^T over dims 0..63) + (-S W^T over 64..127) -> bf16 (32 tokens) ----
+            // ---- U^T = DU + DU2 -> bf16 (this thread: 32 tokens) ----
 #pragma unroll 1
             for (int piece = 0; piece < 2; ++piece) {
                 uint32_t u[16], u2[16], pk[8];
@@ -915,11 +941,24 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             tmem_wait_st();
             tc_fence_before();
             named_bar(kBarChn, kNumChn);
-            if (ct == 0) arrive(&bars[CB_UREADY0 + (c & 1)]);
+            // ---- S += U^T (diag(dl) K) ----
+            if (ct == 0) {
+                if (wait_bar(&bars[CB_QK0 + s], sp, abort_flag)) {
+                    SDBG(5, 11)
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ts(tm + TC_S, tm + ub + kk * 8, smem_desc_sw128(st + ST_K + kk * 2048, 8192, 1024),
+                               IDESC_CS, 1);
+                    mma_commit(&bars[CB_SDONE0 + (c & 1)]);
+                    mma_commit(&bars[CB_EMPTY0 + s]);
+                    SDBG(5, 12)
+                }
+            }
             SDBG(5, 4)
         }
         if (ok && N > 0) {
-            ok = role_wait(&bars[CB_SDONE], (N - 1) & 1, abort_flag, kBarChn, kNumChn);
+            ok = role_wait(&bars[CB_SDONE0 + ((N - 1) & 1)], ((N - 1) >> 1) & 1, abort_flag, kBarChn, kNumChn);
             tc_fence_after();
         }
         float *dst = nullptr;
@@ -1008,7 +1047,8 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
     pa.H = p.H;
     pa.items = items;
     pa.chunks = (int)chunks;
-    const int64_t pgrid = items < 2 * (int64_t)sm_count ? items : 2 * (int64_t)sm_count;
+    const int64_t pgrid =
+        items < kPrepCtasPerSm * (int64_t)sm_count ? items : kPrepCtasPerSm * (int64_t)sm_count;
     fwd_prep_kernel<<<(unsigned)pgrid, kPrepThreads, SMEM_PREP, stream>>>(mq, mk, mp, mtb, mw, pa);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
