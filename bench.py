@@ -13,9 +13,12 @@ scaling, no collective on the data path); times are device times (CUDA
 events on the launching stream), max over ranks.
 
 The JSON line also carries ``e2e`` (the same metric through the C ABI with
-pinned host buffers, copies inside the timed region), ``roofline`` of the
-forward kernel, ``clocks`` sampled with nvidia-smi during the run, and
-``cpu_baseline`` (the float64 oracle on a bounded sample, host cores).
+pinned host buffers, copies inside the timed region), ``kernels`` (device
+time, share and algorithmic rates of each kernel kind of the forward, from
+CUDA events the library records around each launch inside the timed
+region), ``roofline`` of the dominant one, ``clocks`` sampled with
+nvidia-smi during the run, and ``cpu_baseline`` (the float64 oracle on a
+bounded sample, host cores).
 ``--impl reference`` times the float64 CPU oracle as the reference arm.
 """
 from __future__ import annotations
@@ -58,6 +61,45 @@ def fwd_bytes(B, T, H, dk, dv, es, s0, s_final):
 
 def decode_bytes_per_head_step(dk, dv, es):
     return 2 * dk * dv * 4 + (2 * dk + 2 * dv) * es + 8
+
+
+def kernel_work(kind, w, es, nseg):
+    """Algorithmic (flop, HBM bytes) of ONE launch of a forward kernel kind on workload w.
+
+    Two-kernel tensor-core forward, per token and head (C = chunk, d = dk = dv):
+      prep     G = [Q;K]K^T and W = T diag(beta gamma) K: 6 C d flop (the 64x64 inverse is not
+               counted); reads q, k and two gates, writes P, T diag(beta) (2C bytes each), W^T
+               (2 dk bytes) and the 8-byte gate record.
+      chain    Ut = T diag(beta) V, U = Ut - W S^T, S update, Q S^T, P U: 6 dk dv + 4 C dv flop;
+               reads q, k, v, P, TB, W^T, the gate record, writes out.
+      transfer zero-state run (Ut, U, S: 2 C dv + 4 dk dv; reads k, v, TB, W^T, record) plus
+               identity run (U, S: 4 dk dv; reads k, W^T, record) over the tokens of segments
+               0..nseg-2.
+      prefix   S_{p+1} = S_p M_p + B_p: 2 dv dk^2 flop per segment boundary and head; reads M, B,
+               writes the entry state.
+    """
+    C, dk, dv = w.chunk, w.dk, w.dv
+    nth = w.B * w.T * w.H
+    heads = w.B * w.H
+    chunks = -(-w.T // C)
+    seg_len = -(-chunks // max(nseg, 1))
+    tr_tokens = min(w.T, (nseg - 1) * seg_len * C) * heads if nseg > 1 else 0
+    tile = 2 * C + 2 * C + 2 * dk + 8  # P, TB, W^T, gate record bytes per token
+    if kind == "prep":
+        # reads q, k, gates; writes P, TB, W^T and the gate record
+        return nth * 6 * C * dk, nth * (2 * dk * es + 8 + tile)
+    if kind == "chain":
+        # reads q, k, v, P, TB, W^T, the gate record; writes out
+        return nth * (6 * dk * dv + 4 * C * dv), nth * ((2 * dk + 2 * dv) * es + tile)
+    if kind == "transfer":
+        flop = tr_tokens * ((2 * C * dv + 4 * dk * dv) + 4 * dk * dv)
+        by = tr_tokens * (((dk + dv) * es + 2 * C + 2 * dk + 8) + (dk * es + 2 * dk + 8))
+        return flop, by
+    if kind == "prefix":
+        return heads * (nseg - 1) * 2 * dv * dk * dk, heads * (nseg - 1) * 3 * dv * dk * 4
+    if kind == "fused":
+        return nth * fwd_flop_per_token_head(dk, dv, C), nth * ((2 * dk + 2 * dv) * es + 8)
+    return 0, 0
 
 
 # ---------------------------------------------------------------- helpers
@@ -262,7 +304,11 @@ def run_gdn(args, world, rank, local):
 
     for _ in range(args.warmup):
         fwd_step()
+    # per-kernel device times: every launch inside the timed region is bracketed by CUDA events on
+    # the launching stream (host-side records only)
+    gdn.timing_start()
     ms = time_region(fwd_step, args.steps, stream, world)
+    ktimes = gdn.timing_stop()
     ms_step = max_over_ranks(ms / args.steps, world)
     tokens = w.B * w.T
     value = world * tokens / (ms_step / 1e3)
@@ -271,6 +317,32 @@ def run_gdn(args, world, rank, local):
     tflops = flop / (ms_step / 1e3) / 1e12
     gbs = nbytes / (ms_step / 1e3) / 1e9
     scratch_bytes, launches_per_fwd = gdn.forward_plan(w.B, w.T, w.H, w.dk, w.dv, w.chunk, d["q"].dtype)
+    chunks = -(-w.T // w.chunk)
+    ws_tiles = w.B * w.H * chunks * (32768 + 512)
+    nseg = 1 + max(0, scratch_bytes - ws_tiles) // (3 * w.B * w.H * w.dv * w.dk * 4) if "prep" in ktimes else 1
+    kernels = {}
+    for kind, (kms, n) in ktimes.items():
+        per = kms / n
+        flop, by = kernel_work(kind, w, es, nseg)
+        kernels[kind] = {"launches_per_step": n / args.steps, "ms_per_launch": per, "share": kms / (ms * 1.0),
+                         "tflops": flop / (per / 1e3) / 1e12, "gb_per_s": by / (per / 1e3) / 1e9,
+                         "flop_per_launch": flop, "bytes_per_launch": by}
+    top = max(kernels, key=lambda k: ktimes[k][0]) if kernels else None
+    if top is not None:
+        kt = kernels[top]
+        tf, gb = kt["tflops"] / peaks["bf16_tflops"], kt["gb_per_s"] / peaks["hbm_gbs"]
+        # the nearer roof: the kernel is latency-bound when both fractions are low
+        if tf >= gb:
+            roof = {"bound": "tensor", "achieved": kt["tflops"], "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": tf, "hbm_frac": gb}
+        else:
+            roof = {"bound": "hbm", "achieved": kt["gb_per_s"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": gb, "tensor_frac": tf}
+        roof.update({"kernel": top, "traffic": None, "peak_kind": peak_kind,
+                     "flop_per_launch": kt["flop_per_launch"], "bytes_per_launch": kt["bytes_per_launch"],
+                     "ms_per_launch": kt["ms_per_launch"]})
+    else:
+        roof = None
 
     # ---- decode: 1024 consecutive single-token steps, each its own launch ----
     dec = None
@@ -340,9 +412,7 @@ def run_gdn(args, world, rank, local):
                        "input_dtype": w.dtype, "state_dtype": "f32", "parallelism": "replicas" if world > 1 else "single",
                        "l2": "inputs larger than L2 (%.2f GB read+written per step)" % (nbytes / 1e9)},
             "tflops": tflops, "gb_per_s": gbs,
-            "roofline": {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                         "frac": tflops / peaks["bf16_tflops"], "traffic": None, "peak_kind": peak_kind,
-                         "flop_per_launch": flop, "hbm_frac": gbs / peaks["hbm_gbs"]},
+            "roofline": roof, "kernels": kernels, "segments": nseg,
             "decode": dec, "e2e": e2e, "cpu_baseline": cpu, "clocks": clocks,
             "gpu_launches": args.steps * launches_per_fwd, "forward_launches_per_step": launches_per_fwd,
             "forward_scratch_bytes": scratch_bytes,

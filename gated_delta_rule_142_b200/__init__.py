@@ -36,7 +36,10 @@ STATUS = {
 }
 
 EXPORTS = ("gdn_forward", "gdn_decode_step", "gdn_forward_plan", "gdn_status_string", "gdn_version",
-           "gdn_forward_noalloc", "gdn_scratch_release")
+           "gdn_forward_noalloc", "gdn_scratch_release", "gdn_timing_start", "gdn_timing_stop")
+
+# gdn_kernel_kind names, in enum order
+KERNEL_KINDS = ("prep", "chain", "transfer", "prefix", "fused", "simt", "decode")
 
 
 class GdnError(RuntimeError):
@@ -70,6 +73,10 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     lib.gdn_forward_plan.restype = ctypes.c_int
     lib.gdn_scratch_release.argtypes = []
     lib.gdn_scratch_release.restype = ctypes.c_int
+    lib.gdn_timing_start.argtypes = []
+    lib.gdn_timing_start.restype = ctypes.c_int
+    lib.gdn_timing_stop.argtypes = [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(i64)]
+    lib.gdn_timing_stop.restype = ctypes.c_int
     _lib = lib
     return lib
 
@@ -162,6 +169,24 @@ def scratch_release() -> None:
     st = load().gdn_scratch_release()
     if st != 0:
         raise GdnError(st, "gdn_scratch_release")
+
+
+def timing_start() -> None:
+    """Start recording per-kernel device times of every launch the library makes."""
+    st = load().gdn_timing_start()
+    if st != 0:
+        raise GdnError(st, "gdn_timing_start")
+
+
+def timing_stop() -> dict:
+    """Stop recording; {kernel kind: (total ms, launches)} for the kinds that ran."""
+    n = len(KERNEL_KINDS)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_int64 * n)()
+    st = load().gdn_timing_stop(ms, cnt)
+    if st != 0:
+        raise GdnError(st, "gdn_timing_stop")
+    return {KERNEL_KINDS[i]: (ms[i], cnt[i]) for i in range(n) if cnt[i] > 0}
 
 
 def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,

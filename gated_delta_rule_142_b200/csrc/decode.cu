@@ -16,6 +16,7 @@
 // kUnroll rows in flight, so a CTA of 4 warps owns 4 * (32/(DK/4)) * kUnroll
 // rows of one head (32 rows at dk = 128).  Grid: (B*H) x ceil(dv / rows).
 #include "common.cuh"
+#include "gdn.h"
 #include "gdn_internal.h"
 
 namespace gdn {
@@ -93,9 +94,12 @@ template <typename Tin, int DK>
 cudaError_t launch_decode_t(const DecodeProblem &p, cudaStream_t stream) {
     const int rows = decode_rows_per_cta<DK>();
     dim3 grid((unsigned)(p.B * p.H), (unsigned)((p.dv + rows - 1) / rows));
-    decode_kernel<Tin, DK><<<grid, kDecodeThreads, 0, stream>>>(
-        static_cast<const Tin *>(p.q), static_cast<const Tin *>(p.k), static_cast<const Tin *>(p.v),
-        p.log_alpha, p.beta, p.S, static_cast<Tin *>(p.out), (int)p.dv);
+    {
+        TimedLaunch tl_(GDN_KERNEL_DECODE, stream);
+        decode_kernel<Tin, DK><<<grid, kDecodeThreads, 0, stream>>>(
+            static_cast<const Tin *>(p.q), static_cast<const Tin *>(p.k), static_cast<const Tin *>(p.v),
+            p.log_alpha, p.beta, p.S, static_cast<Tin *>(p.out), (int)p.dv);
+    }
     return cudaGetLastError();
 }
 

@@ -25,6 +25,7 @@
 #include <atomic>
 
 #include "common.cuh"
+#include "gdn.h"
 #include "gdn_internal.h"
 
 namespace gdn {
@@ -318,9 +319,12 @@ cudaError_t launch_t(const FwdProblem &p, int sm_count, cudaStream_t stream) {
         configured.fetch_or(bit);
     }
     const int64_t grid = heads * nslab;
-    fwd_simt_kernel<Tin><<<(unsigned)grid, kThreads, smem, stream>>>(
-        static_cast<const Tin *>(p.q), static_cast<const Tin *>(p.k), static_cast<const Tin *>(p.v), p.log_alpha,
-        p.beta, p.S0, static_cast<Tin *>(p.out), p.S_final, p.T, p.H, d);
+    {
+        TimedLaunch tl_(GDN_KERNEL_SIMT, stream);
+        fwd_simt_kernel<Tin><<<(unsigned)grid, kThreads, smem, stream>>>(
+            static_cast<const Tin *>(p.q), static_cast<const Tin *>(p.k), static_cast<const Tin *>(p.v), p.log_alpha,
+            p.beta, p.S0, static_cast<Tin *>(p.out), p.S_final, p.T, p.H, d);
+    }
     return cudaGetLastError();
 }
 

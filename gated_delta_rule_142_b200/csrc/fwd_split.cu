@@ -38,6 +38,7 @@
 
 #include <atomic>
 
+#include "gdn.h"
 #include "gdn_internal.h"
 #include "sm100.cuh"
 #include "tc_util.cuh"
@@ -99,6 +100,8 @@ constexpr uint32_t IDESC_G = instr_desc_bf16(128, 64, 0, 0);     // [Q;K] . K^T
 constexpr uint32_t IDESC_MN64 = instr_desc_bf16(128, 64, 1, 0);  // K^T / V^T (MN-major A) . T^T
 
 enum PBar { PB_QFULL = 0, PB_KFULL, PB_GDONE, PB_GFREE, PB_TBREADY, PB_WDONE, PB_QFREE, PB_COUNT };
+
+static_assert(PB_COUNT * 8 <= PO_MISC - PO_BARS, "prep-kernel mbarriers overflow their shared-memory slot");
 
 struct PrepArgs {
     const float *log_alpha, *beta;
@@ -557,6 +560,8 @@ enum CBar {
 // runs from the zero state (-> Bw), the other from the identity with v = 0
 // (-> Mw; rows of the state evolve independently, so each row of M is a
 // state row with no write term).
+static_assert(CB_COUNT * 8 <= CO_MISC - CO_BARS, "chain-kernel mbarriers overflow their shared-memory slot");
+
 struct ChainArgs {
     const float *gate_rec;  // [items][128] from the prep kernel
     const float *S0;
@@ -1049,7 +1054,10 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
     pa.chunks = (int)chunks;
     const int64_t pgrid =
         items < kPrepCtasPerSm * (int64_t)sm_count ? items : kPrepCtasPerSm * (int64_t)sm_count;
-    fwd_prep_kernel<<<(unsigned)pgrid, kPrepThreads, SMEM_PREP, stream>>>(mq, mk, mp, mtb, mw, pa);
+    {
+        TimedLaunch tl_(GDN_KERNEL_PREP, stream);
+        fwd_prep_kernel<<<(unsigned)pgrid, kPrepThreads, SMEM_PREP, stream>>>(mq, mk, mp, mtb, mw, pa);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
@@ -1072,16 +1080,22 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
         float *entry = a.Mw + per;
         a.S_entry = entry;
         a.mode = 1;  // segment transfers of segments 0..nseg-2
-        fwd_chain_kernel<<<(unsigned)(heads * (a.nseg - 1) * 2), kChainThreads, SMEM_CHAIN, stream>>>(
-            mq, mk, mv, mo, mp, mtb, mw, a);
+        {
+            TimedLaunch tl_(GDN_KERNEL_TRANSFER, stream);
+            fwd_chain_kernel<<<(unsigned)(heads * (a.nseg - 1) * 2), kChainThreads, SMEM_CHAIN, stream>>>(
+                mq, mk, mv, mo, mp, mtb, mw, a);
+        }
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         e = launch_seg_prefix(p.S0, a.Bw, a.Mw, entry, heads, a.nseg, stream);
         if (e != cudaSuccess) return e;
     }
     a.mode = 0;  // outputs of every segment from its entry state
-    fwd_chain_kernel<<<(unsigned)(heads * a.nseg), kChainThreads, SMEM_CHAIN, stream>>>(mq, mk, mv, mo, mp, mtb, mw,
-                                                                                        a);
+    {
+        TimedLaunch tl_(GDN_KERNEL_CHAIN, stream);
+        fwd_chain_kernel<<<(unsigned)(heads * a.nseg), kChainThreads, SMEM_CHAIN, stream>>>(mq, mk, mv, mo, mp, mtb, mw,
+                                                                                            a);
+    }
     return cudaGetLastError();
 }
 

@@ -49,6 +49,7 @@
 
 #include <atomic>
 
+#include "gdn.h"
 #include "gdn_internal.h"
 #include "sm100.cuh"
 #include "tc_util.cuh"
@@ -112,6 +113,8 @@ enum Bar {
     B_TBREADY, B_PREPREADY, B_SREADY, B_UREADY, B_OFREE,  // role hand-offs
     B_COUNT
 };
+
+static_assert(B_COUNT * 8 <= OFF_MISC - OFF_BARS, "mbarriers overflow their shared-memory slot");
 
 __device__ int g_tc_timeout;  // set when a bounded mbarrier wait gives up
 
@@ -819,56 +822,76 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 // Entry states of segments 1..nseg-1 from the segment transfers, in float32:
 // S_{p+1} = S_p M_p + B_p with S_0 = S0 (or zero).  Rows of the state are
 // independent, so one CTA owns 16 rows of one (b, h) and walks the segments
-// in order; M_p is staged in shared memory for each step.
+// in order.  M_{p+1} is bulk-copied into the second of two shared buffers
+// while step p computes, and B_{p+1} is prefetched into registers.
 constexpr int kPrefixRows = 16;
 constexpr int kPrefixThreads = 256;
 constexpr int kPrefixLd = kD + 4;
-constexpr size_t kPrefixSmem = (size_t)(kD * kPrefixLd + kPrefixRows * kPrefixLd) * sizeof(float);
+constexpr size_t kPrefixSmem = (size_t)(2 * kD * kD + kPrefixRows * kPrefixLd) * sizeof(float) + 16;
 
-__global__ void __launch_bounds__(kPrefixThreads)
+__global__ void __launch_bounds__(kPrefixThreads, 1)
 seg_prefix_kernel(const float *__restrict__ S0, const float *__restrict__ Bw, const float *__restrict__ Mw,
                   float *__restrict__ S_entry, int nseg) {
-    extern __shared__ float psm[];
-    float *Ms = psm;                   // [128][kPrefixLd]
-    float *Sr = psm + kD * kPrefixLd;  // [16][kPrefixLd]
+    extern __shared__ __align__(128) float psm[];
+    float *Ms = psm;                       // [2][128][128]
+    float *Sr = psm + 2 * kD * kD;         // [16][kPrefixLd]
+    uint64_t *full = reinterpret_cast<uint64_t *>(Sr + kPrefixRows * kPrefixLd);  // [2]
     const int64_t bh = blockIdx.x;
     const int r0 = blockIdx.y * kPrefixRows;
     const int tid = threadIdx.x;
     const int r = tid >> 4, c = (tid & 15) * 8;  // this thread's row and 8 columns
+    const int steps = nseg - 1;
+    auto load_m = [&](int q) {
+        const float *M = Mw + (bh * steps + q) * (int64_t)kD * kD;
+        float *dst = Ms + (q & 1) * kD * kD;
+        fence_proxy_async_smem();  // the generic reads of this buffer two steps ago come first
+        mbar_arrive_expect_tx(&full[q & 1], kD * kD * 4);
+        for (int i = 0; i < 4; ++i) bulk_load(dst + i * 4096, M + i * 4096, 16384, &full[q & 1]);
+    };
+    if (tid == 0) {
+        mbar_init(&full[0], 1);
+        mbar_init(&full[1], 1);
+        mbar_fence_init();
+    }
+    __syncthreads();
+    if (tid == 0 && steps > 0) load_m(0);
     for (int i = tid; i < kPrefixRows * (kD / 4); i += kPrefixThreads) {
         const int rr = i / (kD / 4), cc = (i % (kD / 4)) * 4;
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
         if (S0) v = *reinterpret_cast<const float4 *>(S0 + (bh * kD + r0 + rr) * (int64_t)kD + cc);
         *reinterpret_cast<float4 *>(Sr + rr * kPrefixLd + cc) = v;
     }
-    for (int q = 0; q < nseg - 1; ++q) {
-        const float *M = Mw + (bh * (nseg - 1) + q) * (int64_t)kD * kD;
-        const float *Bq = Bw + ((bh * (nseg - 1) + q) * kD + r0) * (int64_t)kD;
-        __syncthreads();
-        for (int i = tid; i < kD * (kD / 4); i += kPrefixThreads) {
-            const int rr = i / (kD / 4), cc = (i % (kD / 4)) * 4;
-            *reinterpret_cast<float4 *>(Ms + rr * kPrefixLd + cc) = *reinterpret_cast<const float4 *>(M + rr * kD + cc);
+    auto b_rows = [&](int q) { return Bw + ((bh * steps + q) * kD + r0 + r) * (int64_t)kD + c; };
+    float4 b0 = make_float4(0.f, 0.f, 0.f, 0.f), b1 = b0;
+    if (steps > 0) {
+        b0 = *reinterpret_cast<const float4 *>(b_rows(0));
+        b1 = *reinterpret_cast<const float4 *>(b_rows(0) + 4);
+    }
+    for (int q = 0; q < steps; ++q) {
+        if (tid == 0 && q + 1 < steps) load_m(q + 1);
+        // bounded wait; a timeout leaves the entry states unwritten rather than hanging
+        const bool landed = mbar_wait(&full[q & 1], (q >> 1) & 1);
+        if (!__syncthreads_and(landed)) break;  // also publishes the previous step's rows of S
+        float acc[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        if (q + 1 < steps) {
+            b0 = *reinterpret_cast<const float4 *>(b_rows(q + 1));
+            b1 = *reinterpret_cast<const float4 *>(b_rows(q + 1) + 4);
         }
-        __syncthreads();
-        float acc[8];
-        const float4 b0 = *reinterpret_cast<const float4 *>(Bq + r * kD + c);
-        const float4 b1 = *reinterpret_cast<const float4 *>(Bq + r * kD + c + 4);
-        acc[0] = b0.x; acc[1] = b0.y; acc[2] = b0.z; acc[3] = b0.w;
-        acc[4] = b1.x; acc[5] = b1.y; acc[6] = b1.z; acc[7] = b1.w;
+        const float *M = Ms + (q & 1) * kD * kD;
 #pragma unroll 4
         for (int k = 0; k < kD; ++k) {
             const float a = Sr[r * kPrefixLd + k];
-            const float4 m0 = *reinterpret_cast<const float4 *>(Ms + k * kPrefixLd + c);
-            const float4 m1 = *reinterpret_cast<const float4 *>(Ms + k * kPrefixLd + c + 4);
+            const float4 m0 = *reinterpret_cast<const float4 *>(M + k * kD + c);
+            const float4 m1 = *reinterpret_cast<const float4 *>(M + k * kD + c + 4);
             acc[0] = fmaf(a, m0.x, acc[0]); acc[1] = fmaf(a, m0.y, acc[1]);
             acc[2] = fmaf(a, m0.z, acc[2]); acc[3] = fmaf(a, m0.w, acc[3]);
             acc[4] = fmaf(a, m1.x, acc[4]); acc[5] = fmaf(a, m1.y, acc[5]);
             acc[6] = fmaf(a, m1.z, acc[6]); acc[7] = fmaf(a, m1.w, acc[7]);
         }
-        __syncthreads();  // every thread is done reading this step's rows
+        __syncthreads();  // every thread is done reading this step's rows and M
         *reinterpret_cast<float4 *>(Sr + r * kPrefixLd + c) = make_float4(acc[0], acc[1], acc[2], acc[3]);
         *reinterpret_cast<float4 *>(Sr + r * kPrefixLd + c + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
-        float *dst = S_entry + ((bh * (nseg - 1) + q) * kD + r0 + r) * (int64_t)kD + c;
+        float *dst = S_entry + ((bh * steps + q) * kD + r0 + r) * (int64_t)kD + c;
         *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
         *reinterpret_cast<float4 *>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
@@ -888,9 +911,11 @@ bool fwd_tc_supported(const FwdProblem &p) {
            p.B <= (int64_t)INT32_MAX && p.H <= (int64_t)INT32_MAX;
 }
 
-// Segments per (b, h): the count minimising a wave model of the two parallel
-// passes (transfers: 2 (nseg - 1) CTAs per head; outputs: nseg CTAs per head,
-// each over ceil(chunks / nseg) chunks).  GDN_SEGMENTS overrides the choice.
+// Segments per (b, h): the count minimising a wave model of the passes, in
+// units of half a chunk step of one CTA: transfers (2 (nseg - 1) CTAs per
+// head) and outputs (nseg CTAs per head), each CTA over ceil(chunks / nseg)
+// chunks, plus the sequential prefix over segments (about half a chunk step
+// per segment).  GDN_SEGMENTS overrides the choice.
 int fwd_tc_segments(const FwdProblem &p, int sm_count) {
     const int64_t chunks = (p.T + kC - 1) / kC, heads = p.B * p.H;
     if (chunks <= 0 || heads <= 0) return 1;
@@ -903,12 +928,12 @@ int fwd_tc_segments(const FwdProblem &p, int sm_count) {
     }
     auto waves = [&](int64_t ctas) { return (ctas + sm_count - 1) / sm_count; };
     int best = 1;
-    int64_t best_cost = waves(heads) * chunks;
+    int64_t best_cost = 2 * waves(heads) * chunks;
     for (int nseg = 2; nseg <= 64; ++nseg) {
         const int64_t len = (chunks + nseg - 1) / nseg;
         if (len < 4) break;
         const int64_t real = (chunks + len - 1) / len;
-        const int64_t cost = (waves(2 * heads * (real - 1)) + waves(heads * real)) * len;
+        const int64_t cost = 2 * (waves(2 * heads * (real - 1)) + waves(heads * real)) * len + (real - 1);
         if (cost < best_cost) {
             best_cost = cost;
             best = (int)real;
@@ -934,8 +959,11 @@ cudaError_t launch_seg_prefix(const float *S0, const float *Bw, const float *Mw,
         if (e != cudaSuccess) return e;
         pconf.fetch_or(bit);
     }
-    seg_prefix_kernel<<<dim3((unsigned)heads, kD / kPrefixRows), kPrefixThreads, kPrefixSmem, stream>>>(
-        S0, Bw, Mw, S_entry, nseg);
+    {
+        TimedLaunch tl_(GDN_KERNEL_PREFIX, stream);
+        seg_prefix_kernel<<<dim3((unsigned)heads, kD / kPrefixRows), kPrefixThreads, kPrefixSmem, stream>>>(
+            S0, Bw, Mw, S_entry, nseg);
+    }
     return cudaGetLastError();
 }
 
@@ -976,7 +1004,10 @@ cudaError_t launch_fwd_tc(const FwdProblem &p, int nseg, void *workspace, cudaSt
         a.S_entry = entry;
         // phase 1: segment transfers of segments 0..nseg-2
         a.mode = 1;
-        fwd_tc_kernel<<<(unsigned)(heads * (a.nseg - 1) * 2), kThreadsTc, SMEM_TC, stream>>>(mq, mk, mv, mo, a);
+        {
+            TimedLaunch tl_(GDN_KERNEL_TRANSFER, stream);
+            fwd_tc_kernel<<<(unsigned)(heads * (a.nseg - 1) * 2), kThreadsTc, SMEM_TC, stream>>>(mq, mk, mv, mo, a);
+        }
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         // phase 2: entry states of segments 1..nseg-1
@@ -985,7 +1016,10 @@ cudaError_t launch_fwd_tc(const FwdProblem &p, int nseg, void *workspace, cudaSt
     }
     // outputs of every segment from its entry state
     a.mode = 0;
-    fwd_tc_kernel<<<(unsigned)(heads * a.nseg), kThreadsTc, SMEM_TC, stream>>>(mq, mk, mv, mo, a);
+    {
+        TimedLaunch tl_(GDN_KERNEL_FUSED, stream);
+        fwd_tc_kernel<<<(unsigned)(heads * a.nseg), kThreadsTc, SMEM_TC, stream>>>(mq, mk, mv, mo, a);
+    }
     return cudaGetLastError();
 }
 

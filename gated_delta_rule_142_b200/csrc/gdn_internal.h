@@ -12,6 +12,22 @@ namespace gdn {
 // log-decay sums stay small enough for float32 differences g_t - g_s.
 constexpr float kLogAlphaFloor = -40.0f;
 
+// Brackets one kernel launch with CUDA events on its stream while
+// gdn_timing_start() recording is on (gdn_timing.cu); a no-op otherwise.
+// Construct it right before the launch, in a scope that ends right after it.
+class TimedLaunch {
+  public:
+    TimedLaunch(int kind, cudaStream_t stream);
+    ~TimedLaunch();
+    TimedLaunch(const TimedLaunch &) = delete;
+    TimedLaunch &operator=(const TimedLaunch &) = delete;
+
+  private:
+    int kind_;
+    cudaStream_t stream_;
+    cudaEvent_t begin_ = nullptr, end_ = nullptr;
+};
+
 struct FwdProblem {
     const void *q, *k, *v;
     const float *log_alpha, *beta, *S0;
@@ -49,10 +65,10 @@ cudaError_t launch_seg_prefix(const float *S0, const float *Bw, const float *Mw,
                               int nseg, cudaStream_t stream);
 
 // fwd_split.cu -- the same forward as two kernels: a chunk-parallel prep
-// kernel writes P, T diag(beta) and W^T of every chunk to the workspace, and
-// a chain kernel runs the state recurrence and the outputs from them.  The
-// workspace (fwd_split_workspace_bytes) holds 32 KB per chunk plus the
-// segment scratch of fwd_tc_workspace_bytes.
+// kernel writes P, T diag(beta), W^T and the gates of every chunk to the
+// workspace, and a chain kernel runs the state recurrence and the outputs
+// from them.  The workspace (fwd_split_workspace_bytes) holds 32.5 KB
+// per chunk plus the segment scratch of fwd_tc_workspace_bytes.
 bool fwd_split_supported(const FwdProblem &p);
 size_t fwd_split_workspace_bytes(const FwdProblem &p, int nseg);
 cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *workspace, cudaStream_t stream);

@@ -190,6 +190,31 @@ int gdn_forward_noalloc(const void *q, const void *k, const void *v, const float
  */
 int gdn_scratch_release(void);
 
+/*
+ * Per-kernel device times, for benchmarking.  The paper has no counterpart to
+ * these two calls.  gdn_timing_start() turns recording on (process-wide) and
+ * discards earlier records: from then on every kernel that gdn_forward,
+ * gdn_forward_noalloc or gdn_decode_step launches is bracketed by a pair of
+ * CUDA events recorded on the caller's stream.  gdn_timing_stop() turns it
+ * off, waits for the recorded events and writes, per kernel kind, the summed
+ * elapsed milliseconds into ms[kind] and the number of launches into
+ * launches[kind] (arrays of GDN_KERNEL_KINDS entries; either may be NULL).
+ * Recording adds host-side event records around each launch and nothing on
+ * the device path.  Returns GDN_OK, or GDN_ERR_LAUNCH if an event failed.
+ */
+typedef enum {
+    GDN_KERNEL_PREP = 0,        /* two-kernel forward: chunk-parallel prep (P, T diag(beta), W)   */
+    GDN_KERNEL_CHAIN = 1,       /* two-kernel forward: state chain and outputs                     */
+    GDN_KERNEL_TRANSFER = 2,    /* segment transfers of long sequences (either forward)            */
+    GDN_KERNEL_PREFIX = 3,      /* entry states of segments from the transfers                     */
+    GDN_KERNEL_FUSED = 4,       /* single-kernel tensor-core forward (outputs)                     */
+    GDN_KERNEL_SIMT = 5,        /* float32 CUDA-core forward                                       */
+    GDN_KERNEL_DECODE = 6,      /* single-token decode step                                        */
+    GDN_KERNEL_KINDS = 7
+} gdn_kernel_kind;
+int gdn_timing_start(void);
+int gdn_timing_stop(double *ms, int64_t *launches);
+
 /* Static, NUL-terminated description of a gdn_status value. */
 const char *gdn_status_string(int status);
 
