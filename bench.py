@@ -24,6 +24,7 @@ bounded sample, host cores).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -61,6 +62,25 @@ def fwd_bytes(B, T, H, dk, dv, es, s0, s_final):
 
 def decode_bytes_per_head_step(dk, dv, es):
     return 2 * dk * dv * 4 + (2 * dk + 2 * dv) * es + 8
+
+
+# DRAM bytes (read + write) per token-head that one ncu capture of each kernel kind measured, from
+# the summaries in profiles/ (fwd_chain_b8h16_t2k_d128.md, fwd_prep_b8h16_t2k_d128.md,
+# fwd_transfer_b1h16_t16k_s4.md).  For the transfer kind the unit is a token-head of the
+# transferred segments (covering both of its runs).  Kept only while those kernels are unchanged.
+NCU_TRAFFIC_PER_TOKEN_HEAD = {"chain": 400.0e6 / 262144, "prep": 225.4e6 / 262144, "transfer": 181.7e6 / 196608}
+
+
+def kernel_units(kind, w, nseg):
+    """Token-heads one launch of a kernel kind processes (the unit of NCU_TRAFFIC_PER_TOKEN_HEAD)."""
+    nth = w.B * w.T * w.H
+    if kind in ("prep", "chain", "fused"):
+        return nth
+    if kind == "transfer":
+        chunks = -(-w.T // w.chunk)
+        seg_len = -(-chunks // max(nseg, 1))
+        return min(w.T, (nseg - 1) * seg_len * w.chunk) * w.B * w.H if nseg > 1 else 0
+    return 0
 
 
 def kernel_work(kind, w, es, nseg):
@@ -291,6 +311,9 @@ def run_gdn(args, world, rank, local):
 
     # ---- forward, inputs resident in HBM ----
     w = WORKLOADS[args.workload]
+    if args.tokens:
+        # a shorter sequence of the same workload, for profiler captures that must stay small
+        w = dataclasses.replace(w, T=args.tokens, name="%s_first%d" % (w.name, args.tokens))
     es = 2 if w.dtype == "bf16" else 4
     inp = forward_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, seed=w.seed + 1000 * rank, s0_std=w.s0_std,
                          alpha_mu=w.alpha_mu)
@@ -338,7 +361,9 @@ def run_gdn(args, world, rank, local):
         else:
             roof = {"bound": "hbm", "achieved": kt["gb_per_s"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": gb, "tensor_frac": tf}
-        roof.update({"kernel": top, "traffic": None, "peak_kind": peak_kind,
+        per_unit = NCU_TRAFFIC_PER_TOKEN_HEAD.get(top)
+        traffic = per_unit * kernel_units(top, w, nseg) if per_unit is not None else None
+        roof.update({"kernel": top, "traffic": traffic, "peak_kind": peak_kind,
                      "flop_per_launch": kt["flop_per_launch"], "bytes_per_launch": kt["bytes_per_launch"],
                      "ms_per_launch": kt["ms_per_launch"]})
     else:
@@ -430,6 +455,8 @@ def main():
     ap.add_argument("--workload", default=FWD_WORKLOAD,
                     choices=[n for n, w in WORKLOADS.items() if w.kind == "forward"],
                     help="forward workload timed as the step (default: the 64K-token one)")
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="time only the first T tokens of the workload (profiler captures); not a bench line")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -839,7 +839,9 @@ seg_prefix_kernel(const float *__restrict__ S0, const float *__restrict__ Bw, co
     const int64_t bh = blockIdx.x;
     const int r0 = blockIdx.y * kPrefixRows;
     const int tid = threadIdx.x;
-    const int r = tid >> 4, c = (tid & 15) * 8;  // this thread's row and 8 columns
+    // this thread's row and columns ca..ca+3, cb..cb+3: consecutive threads read consecutive
+    // 16-byte words of a row of M, without bank conflicts
+    const int r = tid >> 4, ca = (tid & 15) * 4, cb = 64 + ca;
     const int steps = nseg - 1;
     auto load_m = [&](int q) {
         const float *M = Mw + (bh * steps + q) * (int64_t)kD * kD;
@@ -861,11 +863,11 @@ seg_prefix_kernel(const float *__restrict__ S0, const float *__restrict__ Bw, co
         if (S0) v = *reinterpret_cast<const float4 *>(S0 + (bh * kD + r0 + rr) * (int64_t)kD + cc);
         *reinterpret_cast<float4 *>(Sr + rr * kPrefixLd + cc) = v;
     }
-    auto b_rows = [&](int q) { return Bw + ((bh * steps + q) * kD + r0 + r) * (int64_t)kD + c; };
+    auto b_rows = [&](int q) { return Bw + ((bh * steps + q) * kD + r0 + r) * (int64_t)kD; };
     float4 b0 = make_float4(0.f, 0.f, 0.f, 0.f), b1 = b0;
     if (steps > 0) {
-        b0 = *reinterpret_cast<const float4 *>(b_rows(0));
-        b1 = *reinterpret_cast<const float4 *>(b_rows(0) + 4);
+        b0 = *reinterpret_cast<const float4 *>(b_rows(0) + ca);
+        b1 = *reinterpret_cast<const float4 *>(b_rows(0) + cb);
     }
     for (int q = 0; q < steps; ++q) {
         if (tid == 0 && q + 1 < steps) load_m(q + 1);
@@ -874,26 +876,26 @@ seg_prefix_kernel(const float *__restrict__ S0, const float *__restrict__ Bw, co
         if (!__syncthreads_and(landed)) break;  // also publishes the previous step's rows of S
         float acc[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
         if (q + 1 < steps) {
-            b0 = *reinterpret_cast<const float4 *>(b_rows(q + 1));
-            b1 = *reinterpret_cast<const float4 *>(b_rows(q + 1) + 4);
+            b0 = *reinterpret_cast<const float4 *>(b_rows(q + 1) + ca);
+            b1 = *reinterpret_cast<const float4 *>(b_rows(q + 1) + cb);
         }
         const float *M = Ms + (q & 1) * kD * kD;
 #pragma unroll 4
         for (int k = 0; k < kD; ++k) {
             const float a = Sr[r * kPrefixLd + k];
-            const float4 m0 = *reinterpret_cast<const float4 *>(M + k * kD + c);
-            const float4 m1 = *reinterpret_cast<const float4 *>(M + k * kD + c + 4);
+            const float4 m0 = *reinterpret_cast<const float4 *>(M + k * kD + ca);
+            const float4 m1 = *reinterpret_cast<const float4 *>(M + k * kD + cb);
             acc[0] = fmaf(a, m0.x, acc[0]); acc[1] = fmaf(a, m0.y, acc[1]);
             acc[2] = fmaf(a, m0.z, acc[2]); acc[3] = fmaf(a, m0.w, acc[3]);
             acc[4] = fmaf(a, m1.x, acc[4]); acc[5] = fmaf(a, m1.y, acc[5]);
             acc[6] = fmaf(a, m1.z, acc[6]); acc[7] = fmaf(a, m1.w, acc[7]);
         }
         __syncthreads();  // every thread is done reading this step's rows and M
-        *reinterpret_cast<float4 *>(Sr + r * kPrefixLd + c) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        *reinterpret_cast<float4 *>(Sr + r * kPrefixLd + c + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
-        float *dst = S_entry + ((bh * steps + q) * kD + r0 + r) * (int64_t)kD + c;
-        *reinterpret_cast<float4 *>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        *reinterpret_cast<float4 *>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        *reinterpret_cast<float4 *>(Sr + r * kPrefixLd + ca) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4 *>(Sr + r * kPrefixLd + cb) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        float *dst = S_entry + ((bh * steps + q) * kD + r0 + r) * (int64_t)kD;
+        *reinterpret_cast<float4 *>(dst + ca) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4 *>(dst + cb) = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
 }
 
