@@ -19,7 +19,9 @@
 //     TB  = T diag(beta)                                        -> workspace, bf16
 //     W^T = K^T (T diag(beta gamma))^T                          (tcgen05) -> workspace, bf16
 //
-//   chain kernel (sequential over the chunks of one (b, h) or segment):
+//   chain kernel (sequential over the chunks of one (b, h) or segment; for long
+//   sequences with few heads, the transfers of the segments come first from the
+//   paired transfer kernel, and their prefix gives each segment's entry state):
 //     Ut^T = V^T TB^T                               (tcgen05, off the critical path)
 //     U^T  = Ut^T - S W^T                           (accumulated onto Ut^T, B negated)
 //     S   <- gamma_C S + U^T (diag(dl) K)           (float32 state in tensor memory)
@@ -303,13 +305,16 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     uint32_t r[16];
                     tmem_ld16(tm + lb + TP_G + s0, r);
                     tmem_wait_ld();
-                    float d[16];  // e^{g_t - g_s} for the 16 columns s of this piece
+                    // e^{g_t - g_s} for the 16 columns s of this piece; in a wide chunk, __expf's few-ulp
+                    // relative error (larger for large |x|, where the value is far below the bf16
+                    // rounding of P and the TF32 inverse) does not show at the precision of the path
+                    float d[16];
                     if (narrow) {
 #pragma unroll
                         for (int i = 0; i < 16; ++i) d[i] = at * eb[s0 + i];
                     } else {
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) d[i] = expf(gt - g[s0 + i]);
+                        for (int i = 0; i < 16; ++i) d[i] = __expf(gt - g[s0 + i]);
                     }
                     if (m < 64) {
                         uint32_t pk[8];
@@ -553,13 +558,10 @@ enum CBar {
     CB_COUNT
 };
 
-// mode 0: one CTA per (b, h, segment) computes the outputs of its chunk range
-// from that segment's entry state (S0 for the first segment, else S_entry) and
-// writes S_final from the last segment.  mode 1: two CTAs per (b, h, segment <
-// nseg - 1) compute the segment's affine transfer S_end = S_start M + B: one
-// runs from the zero state (-> Bw), the other from the identity with v = 0
-// (-> Mw; rows of the state evolve independently, so each row of M is a
-// state row with no write term).
+// One CTA per (b, h, segment) computes the outputs of its chunk range from that
+// segment's entry state (S0 for the first segment, else S_entry) and writes
+// S_final from the last segment.  The segment transfers are the paired
+// transfer kernel's.
 static_assert(CB_COUNT * 8 <= CO_MISC - CO_BARS, "chain-kernel mbarriers overflow their shared-memory slot");
 
 struct ChainArgs {
@@ -568,7 +570,7 @@ struct ChainArgs {
     float *S_final;
     int64_t T, H;
     int chunks;  // chunks per (b, h)
-    int mode, nseg, seg_len;
+    int nseg, seg_len;
     const float *S_entry;  // [B*H][nseg-1][dv][dk]
     float *Bw, *Mw;        // [B*H][nseg-1][dv][dk] / [dk][dk]
 };
@@ -587,19 +589,8 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t H = p.H;
     SDBG_INIT
-    int64_t bh;
-    int seg, kind;  // kind 0 = outputs, 1 = transfer B, 2 = transfer M
-    if (p.mode == 0) {
-        bh = blockIdx.x / p.nseg;
-        seg = (int)(blockIdx.x % p.nseg);
-        kind = 0;
-    } else {
-        const int64_t q = blockIdx.x >> 1;
-        bh = q / (p.nseg - 1);
-        seg = (int)(q % (p.nseg - 1));
-        kind = 1 + (int)(blockIdx.x & 1);
-    }
-    const bool outputs = (kind == 0);
+    const int64_t bh = blockIdx.x / p.nseg;
+    const int seg = (int)(blockIdx.x % p.nseg);
     const int b = (int)(bh / H), h = (int)(bh % H);
     const int c0 = seg * p.seg_len;
     const int N = (p.chunks - c0 < p.seg_len) ? (p.chunks - c0) : p.seg_len;
@@ -626,7 +617,7 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (lane == 0) {
             bool ok = true;
             const uint32_t bytes =
-                (outputs ? 16384 + 8192 : 0) + 16384 + 16384 + (kind != 2 ? 16384 + 8192 : 0) + (uint32_t)kGateRec;
+                16384 + 8192 + 16384 + 16384 + 16384 + 8192 + (uint32_t)kGateRec;
             for (int c = 0; c < N && ok; ++c) {
                 const int s = c & 1;
                 if (c >= 2 && !(ok = wait_bar(&bars[CB_EMPTY0 + s], ((c - 2) >> 1) & 1, abort_flag))) break;
@@ -636,13 +627,13 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const int row = (int)(item0 + c);
                 mbar_arrive_expect_tx(full, bytes);
                 for (int blk = 0; blk < 2; ++blk) {
-                    if (outputs) tma_load_4d(st + ST_Q + blk * 8192, &tm_q, full, blk * 64, h, t0, b);
+                    tma_load_4d(st + ST_Q + blk * 8192, &tm_q, full, blk * 64, h, t0, b);
                     tma_load_4d(st + ST_K + blk * 8192, &tm_k, full, blk * 64, h, t0, b);
-                    if (kind != 2) tma_load_4d(st + ST_V + blk * 8192, &tm_v, full, blk * 64, h, t0, b);
+                    tma_load_4d(st + ST_V + blk * 8192, &tm_v, full, blk * 64, h, t0, b);
                 }
                 tma_load_2d(st + ST_W, &tm_w, full, 0, row * 128);
-                if (outputs) tma_load_2d(st + ST_P, &tm_p, full, 0, row * 64);
-                if (kind != 2) tma_load_2d(st + ST_TB, &tm_tb, full, 0, row * 64);
+                tma_load_2d(st + ST_P, &tm_p, full, 0, row * 64);
+                tma_load_2d(st + ST_TB, &tm_tb, full, 0, row * 64);
                 bulk_load(st + ST_GATE, p.gate_rec + (int64_t)row * 128, (uint32_t)kGateRec, full);
             }
         }
@@ -665,13 +656,11 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     break;
                 SDBG(2, 1)
                 tc_fence_after();
-                // Ut^T = V^T TB^T (transfer-M runs have v = 0: U^T starts fresh in the chain role)
-                if (kind != 2) {
+                // Ut^T = V^T TB^T
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_ss(tm + TC_DU, smem_desc_sw128(st + ST_V + kk * 2048, 8192, 1024),
-                               smem_desc_sw128(st + ST_TB + kk * 32, 16, 1024), IDESC_CMN, kk > 0);
-                }
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ss(tm + TC_DU, smem_desc_sw128(st + ST_V + kk * 2048, 8192, 1024),
+                           smem_desc_sw128(st + ST_TB + kk * 32, 16, 1024), IDESC_CMN, kk > 0);
                 mma_commit(&bars[CB_UTDONE]);
                 SDBG(2, 2)
             }
@@ -696,25 +685,21 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 if (c > 0 && !(ok = wait_bar(&bars[CB_OFREE], (c - 1) & 1, abort_flag))) break;
                 SDBG(3, 1)
                 tc_fence_after();
-                // O^T = S (diag(gamma) Q)^T  (transfer runs issue no output MMAs; the commits still arrive)
-                if (outputs) {
+                // O^T = S (diag(gamma) Q)^T
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        mma_ts(tm + TC_O, tm + sb + kk * 8,
-                               smem_desc_sw128(st + ST_Q + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), IDESC_C64,
-                               kk > 0);
-                }
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tm + TC_O, tm + sb + kk * 8,
+                           smem_desc_sw128(st + ST_Q + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), IDESC_C64,
+                           kk > 0);
                 mma_commit(&bars[CB_O1DONE0 + (c & 1)]);
                 if (!(ok = wait_bar(&bars[CB_SDONE0 + (c & 1)], sp, abort_flag))) break;
                 SDBG(3, 2)
                 tc_fence_after();
                 // O^T += U^T P^T
-                if (outputs) {
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_ts(tm + TC_O, tm + ub + kk * 8, smem_desc_sw128(st + ST_P + kk * 32, 16, 1024),
-                               IDESC_C64, 1);
-                }
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ts(tm + TC_O, tm + ub + kk * 8, smem_desc_sw128(st + ST_P + kk * 32, 16, 1024), IDESC_C64,
+                           1);
                 mma_commit(&bars[CB_ODONE0 + (c & 1)]);
                 mma_commit(&bars[CB_EMPTY0 + s]);
                 SDBG(3, 3)
@@ -790,7 +775,7 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     }
                 };
                 scale_tile(st + ST_K, dl);
-                if (outputs) scale_tile(st + ST_Q, gam);
+                scale_tile(st + ST_Q, gam);
             }
             fence_proxy_async_smem();
             named_bar(kBarOut, kNumOut);
@@ -802,7 +787,7 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                      kNumOut)))
                     break;
                 tc_fence_after();
-                if (outputs) write_out(c - 1);  // ends with a role barrier after the O reads
+                write_out(c - 1);  // ends with a role barrier after the O reads
                 if (ot == 0) arrive(&bars[CB_OFREE]);
             }
             SDBG(4, 4)
@@ -810,7 +795,7 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (ok && N > 0) {
             ok = role_wait(&bars[CB_ODONE0 + ((N - 1) & 1)], ((N - 1) >> 1) & 1, abort_flag, kBarOut, kNumOut);
             tc_fence_after();
-            if (ok && outputs) write_out(N - 1);
+            if (ok) write_out(N - 1);
         }
         if (ot == 0) bulk_wait0();  // every output store has completed
     } else if (warp >= kChnWarp0) {
@@ -821,12 +806,10 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const int ch = (warp - kChnWarp0) >> 2;    // column half
         bool ok = true;
         // entry state -> TMEM: S0 (or zero) for the first segment, the prefix-scanned entry state for
-        // later segments, zero for transfer-B runs and the identity for transfer-M runs
+        // later segments
         {
-            const float *src = nullptr;
-            if (kind == 0)
-                src = (seg == 0) ? (p.S0 ? p.S0 + (bh * kD + j) * (int64_t)kD : nullptr)
-                                 : p.S_entry + ((bh * (p.nseg - 1) + seg - 1) * kD + j) * (int64_t)kD;
+            const float *src = (seg == 0) ? (p.S0 ? p.S0 + (bh * kD + j) * (int64_t)kD : nullptr)
+                                          : p.S_entry + ((bh * (p.nseg - 1) + seg - 1) * kD + j) * (int64_t)kD;
 #pragma unroll 1
             for (int piece = 0; piece < 2; ++piece) {
                 const int col0 = ch * 64 + piece * 32;
@@ -838,10 +821,6 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     r[i + 1] = __float_as_uint(v.y);
                     r[i + 2] = __float_as_uint(v.z);
                     r[i + 3] = __float_as_uint(v.w);
-                }
-                if (kind == 2) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = __float_as_uint((col0 + i == j) ? 1.f : 0.f);
                 }
                 tmem_st32(tm + lb + TC_S + col0, r);
             }
@@ -891,7 +870,7 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         mma_ts(tm + TC_DU, tm + sb + kk * 8, smem_desc_sw128(st + ST_W + kk * 2048, 8192, 1024),
-                               IDESC_CWNEG, (kind != 2 || kk > 0) ? 1u : 0u);
+                               IDESC_CWNEG, 1u);
                     mma_commit(&bars[CB_UDONE0 + (c & 1)]);
                     SDBG(5, 6)
                 }
@@ -966,17 +945,329 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             ok = role_wait(&bars[CB_SDONE0 + ((N - 1) & 1)], ((N - 1) >> 1) & 1, abort_flag, kBarChn, kNumChn);
             tc_fence_after();
         }
-        float *dst = nullptr;
-        if (kind == 0)
-            dst = (seg == p.nseg - 1 && p.S_final) ? p.S_final + (bh * kD + j) * (int64_t)kD : nullptr;
-        else
-            dst = (kind == 1 ? p.Bw : p.Mw) + ((bh * (p.nseg - 1) + seg) * kD + j) * (int64_t)kD;
+        float *dst = (seg == p.nseg - 1 && p.S_final) ? p.S_final + (bh * kD + j) * (int64_t)kD : nullptr;
         if (ok && dst) {
 #pragma unroll 1
             for (int piece = 0; piece < 2; ++piece) {
                 const int col0 = ch * 64 + piece * 32;
                 uint32_t r[32];
                 tmem_ld32(tm + lb + TC_S + col0, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; i += 4)
+                    *reinterpret_cast<float4 *>(dst + col0 + i) =
+                        make_float4(__uint_as_float(r[i]), __uint_as_float(r[i + 1]), __uint_as_float(r[i + 2]),
+                                    __uint_as_float(r[i + 3]));
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && *abort_flag) atomicExch(&g_split_timeout, 1);
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tm, 512);
+    }
+}
+
+// ============================================================================
+// paired transfer kernel (long sequences with few heads)
+// ============================================================================
+// One CTA per (b, h, segment < nseg - 1) computes the segment's affine transfer
+// S_end = S_start M + B with two chains that share every load: group 0 runs the
+// recurrence from the zero state (-> Bw), group 1 from the identity with v = 0
+// (-> Mw; rows of the state evolve independently, so each row of M is a state
+// row with no write term).  The two chains are independent, so each hides the
+// other's latency.  Each group keeps S, the U^T accumulator and a second half
+// accumulator in 256 TMEM columns; its bf16 operand copies of S and U^T live in
+// shared memory.
+constexpr int kTrThreads = 640;
+// warp 0: TMA producer; warp 1: Ut^T issuer (group 0); warps 2-3: K rows scaled by dl;
+// warps 4-11: group 0; warps 12-19: group 1 (threads 0 and 32 of a group issue its MMAs)
+constexpr int kTrGrpWarp0 = 4, kTrNumGrp = 256, kTrNumScale = 64;
+constexpr int kBarGrp0 = 1, kBarScale = 3;  // group g uses named barrier kBarGrp0 + g
+
+constexpr uint32_t TS_K = 0;         // 16 KB: two [64 t][64 d] boxes
+constexpr uint32_t TS_V = 16384;     // 16 KB
+constexpr uint32_t TS_W = 32768;     // 16 KB: W^T [128 i][64 t]
+constexpr uint32_t TS_TB = 49152;    // 8 KB:  TB [64 t][64 s]
+constexpr uint32_t TS_GATE = 57344;  // 512 B: gamma_t [64], dl_s [64]
+constexpr uint32_t TS_BYTES = 58368;
+constexpr uint32_t TO_SB = 2 * TS_BYTES;        // 2 groups x 32 KB: bf16 S, two [128 j][64 i] boxes
+constexpr uint32_t TO_UB = TO_SB + 2 * 32768;   // 2 groups x 16 KB: bf16 U^T, [128 j][64 t]
+constexpr uint32_t TO_BARS = TO_UB + 2 * 16384;
+constexpr uint32_t TO_MISC = TO_BARS + 256;
+constexpr uint32_t SMEM_TR = TO_MISC + 64 + 1024;
+
+constexpr uint32_t TT_S = 0;      // per group (base 256 g): 128  S float32
+constexpr uint32_t TT_DU = 128;   //                          64   Ut^T - S W^T, key dims 0..63
+constexpr uint32_t TT_DU2 = 192;  //                          64   -S W^T, key dims 64..127
+
+constexpr uint32_t IDESC_TWNEG = instr_desc_bf16(128, 64, 0, 1) | (1u << 14);  // S . (-W)^T, W^T MN-major
+constexpr uint32_t IDESC_TS = instr_desc_bf16(128, 128, 0, 1);                // U^T . (dl K), MN-major B
+
+enum TBar {
+    TB_FULL0 = 0, TB_FULL1,      // stage landed
+    TB_EMPTY0, TB_EMPTY1,        // stage consumed (count 4: the U^T half and state update of each group)
+    TB_KREADY0, TB_KREADY1,      // K scaled by dl
+    TB_UTDONE,                   // Ut^T of group 0 done
+    TB_SISSUED,                  // group 0's state update issued
+    TB_UDONE0, TB_UDONE1,        // per group: first U^T half done
+    TB_UDONE20, TB_UDONE21,      // per group: second U^T half done
+    TB_SDONE0, TB_SDONE1,        // per group: state update done
+    TB_COUNT
+};
+static_assert(TB_COUNT * 8 <= TO_MISC - TO_BARS, "transfer-kernel mbarriers overflow their shared-memory slot");
+static_assert(SMEM_TR <= 232448, "transfer kernel exceeds the shared memory of a CTA");
+
+__global__ void __launch_bounds__(kTrThreads, 1)
+fwd_transfer_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                    const __grid_constant__ CUtensorMap tm_tb, const __grid_constant__ CUtensorMap tm_w,
+                    ChainArgs p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + TO_BARS);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + TO_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + TO_MISC + 4);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t H = p.H;
+    const int64_t bh = blockIdx.x / (p.nseg - 1);
+    const int seg = (int)(blockIdx.x % (p.nseg - 1));
+    const int b = (int)(bh / H), h = (int)(bh % H);
+    const int c0 = seg * p.seg_len;
+    const int N = p.seg_len;  // segments 0..nseg-2 are full
+    const int64_t item0 = bh * p.chunks + c0;
+    const uint32_t sbase = smem_u32(sm);
+
+    if (tid == 0) {
+        for (int i = 0; i < TB_COUNT; ++i) mbar_init(&bars[i], (i == TB_EMPTY0 || i == TB_EMPTY1) ? 4 : 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tmem_slot;
+    const uint32_t lb = (uint32_t)((warp & 3) * 32) << 16;
+
+    if (warp == 0) {
+        // ============================ producer ============================
+        if (lane == 0) {
+            bool ok = true;
+            const uint32_t bytes = 16384 + 16384 + 16384 + 8192 + (uint32_t)kGateRec;
+            for (int c = 0; c < N && ok; ++c) {
+                const int s = c & 1;
+                if (c >= 2 && !(ok = wait_bar(&bars[TB_EMPTY0 + s], ((c - 2) >> 1) & 1, abort_flag))) break;
+                uint8_t *st = sm + s * TS_BYTES;
+                uint64_t *full = &bars[TB_FULL0 + s];
+                const int t0 = (c0 + c) * kC;
+                const int row = (int)(item0 + c);
+                mbar_arrive_expect_tx(full, bytes);
+                for (int blk = 0; blk < 2; ++blk) {
+                    tma_load_4d(st + TS_K + blk * 8192, &tm_k, full, blk * 64, h, t0, b);
+                    tma_load_4d(st + TS_V + blk * 8192, &tm_v, full, blk * 64, h, t0, b);
+                }
+                tma_load_2d(st + TS_W, &tm_w, full, 0, row * 128);
+                tma_load_2d(st + TS_TB, &tm_tb, full, 0, row * 64);
+                bulk_load(st + TS_GATE, p.gate_rec + (int64_t)row * 128, (uint32_t)kGateRec, full);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ===================== Ut^T issuer (group 0) ======================
+        // Ut^T = V^T TB^T of chunk c into group 0's DU2, queued behind that group's state update
+        // of chunk c - 1
+        if (lane == 0) {
+            bool ok = true;
+            for (int c = 0; c < N && ok; ++c) {
+                const int s = c & 1;
+                const uint32_t st = sbase + s * TS_BYTES;
+                if (c > 0 && !(ok = wait_bar(&bars[TB_SISSUED], (c - 1) & 1, abort_flag))) break;
+                if (!(ok = wait_bar(&bars[TB_FULL0 + s], (c >> 1) & 1, abort_flag))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ss(tm + TT_DU2, smem_desc_sw128(st + TS_V + kk * 2048, 8192, 1024),
+                           smem_desc_sw128(st + TS_TB + kk * 32, 16, 1024), IDESC_CMN, kk > 0);
+                mma_commit(&bars[TB_UTDONE]);
+            }
+        }
+        __syncwarp();
+    } else if (warp < kTrGrpWarp0) {
+        // ===================== K rows scaled by dl_s ======================
+        const int kt = tid - 64;  // 0..63
+        bool ok = true;
+        for (int c = 0; c < N && ok; ++c) {
+            const int s = c & 1;
+            uint8_t *st = sm + s * TS_BYTES;
+            if (!(ok = role_wait(&bars[TB_FULL0 + s], (c >> 1) & 1, abort_flag, kBarScale, kTrNumScale))) break;
+            const float *dl = reinterpret_cast<const float *>(st + TS_GATE) + 64;
+            uint4 *ktile = reinterpret_cast<uint4 *>(st + TS_K);
+#pragma unroll 4
+            for (int i = 0; i < 16; ++i) {
+                const int u = kt + 64 * i;  // 16-byte unit u of K covers row (u / 8) % 64
+                const float fr = dl[(u >> 3) & 63];
+                const uint4 v = ktile[u];
+                uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w4[e]));
+                    w4[e] = pack_bf16x2(x.x * fr, x.y * fr);
+                }
+                ktile[u] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            }
+            fence_proxy_async_smem();
+            named_bar(kBarScale, kTrNumScale);
+            if (kt == 0) arrive(&bars[TB_KREADY0 + s]);
+        }
+    } else {
+        // ============================ chain groups ============================
+        const int grp = (warp - kTrGrpWarp0) >> 3;              // 0: from zero (B), 1: from identity (M)
+        const int gt = tid - (kTrGrpWarp0 + 8 * grp) * 32;       // 0..255
+        const int j = (warp & 3) * 32 + lane;                    // TMEM lane / state row
+        const int ch = ((warp - kTrGrpWarp0) >> 2) & 1;           // column half
+        const int barg = kBarGrp0 + grp;
+        const uint32_t tg = tm + (uint32_t)(256 * grp);          // this group's TMEM columns
+        uint8_t *sbs = sm + TO_SB + grp * 32768;                 // bf16 S, [128 j][64 i] x 2 boxes
+        uint8_t *ubs = sm + TO_UB + grp * 16384;                 // bf16 U^T, [128 j][64 t]
+        const uint32_t sbs_a = sbase + TO_SB + grp * 32768, ubs_a = sbase + TO_UB + grp * 16384;
+        bool ok = true;
+        // entry state: zero for group 0, identity for group 1
+#pragma unroll 1
+        for (int piece = 0; piece < 2; ++piece) {
+            const int col0 = ch * 64 + piece * 32;
+            uint32_t r[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint((grp == 1 && col0 + i == j) ? 1.f : 0.f);
+            tmem_st32(tg + lb + TT_S + col0, r);
+        }
+        tmem_wait_st();
+        for (int c = 0; c < N && ok; ++c) {
+            const int s = c & 1;
+            const uint32_t sp = (c >> 1) & 1;
+            const uint32_t st = sbase + s * TS_BYTES;
+            // the previous state update is done (its operands in shared memory are free); this
+            // chunk's stage has landed
+            {
+                bool w = c == 0 || wait_bar(&bars[TB_SDONE0 + grp], (c - 1) & 1, abort_flag);
+                w = w && wait_bar(&bars[TB_FULL0 + s], sp, abort_flag);
+                if (!(ok = bar_and(barg, kTrNumGrp, w))) break;
+            }
+            const float gC = reinterpret_cast<const float *>(sm + s * TS_BYTES + TS_GATE)[63];
+            tc_fence_after();
+            // ---- bf16 copy of S into shared memory (row j, 64 columns = one 128-byte row of a box) ----
+#pragma unroll 1
+            for (int piece = 0; piece < 2; ++piece) {
+                const int col0 = ch * 64 + piece * 32;
+                uint32_t r[32];
+                tmem_ld32(tg + lb + TT_S + col0, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    uint4 v;
+                    v.x = pack_bf16x2(__uint_as_float(r[cc * 8 + 0]), __uint_as_float(r[cc * 8 + 1]));
+                    v.y = pack_bf16x2(__uint_as_float(r[cc * 8 + 2]), __uint_as_float(r[cc * 8 + 3]));
+                    v.z = pack_bf16x2(__uint_as_float(r[cc * 8 + 4]), __uint_as_float(r[cc * 8 + 5]));
+                    v.w = pack_bf16x2(__uint_as_float(r[cc * 8 + 6]), __uint_as_float(r[cc * 8 + 7]));
+                    *reinterpret_cast<uint4 *>(sbs + ch * 16384 + sw128(j, piece * 4 + cc)) = v;
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar(barg, kTrNumGrp);
+            // ---- U^T = Ut^T - S W^T (key dims 0..63 from thread 0, 64..127 from thread 32) ----
+            if (gt == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_ss(tg + TT_DU, smem_desc_sw128(sbs_a + kk * 32, 16, 1024),
+                           smem_desc_sw128(st + TS_W + kk * 2048, 8192, 1024), IDESC_TWNEG, kk > 0);
+                mma_commit(&bars[TB_UDONE0 + grp]);
+            } else if (gt == 32) {
+                // group 0 accumulates onto its Ut^T; group 1 has v = 0 and starts fresh
+                if (grp == 1 || wait_bar(&bars[TB_UTDONE], c & 1, abort_flag)) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 4; kk < 8; ++kk)
+                        mma_ss(tg + TT_DU2, smem_desc_sw128(sbs_a + 16384 + (kk - 4) * 32, 16, 1024),
+                               smem_desc_sw128(st + TS_W + kk * 2048, 8192, 1024), IDESC_TWNEG,
+                               (grp == 0 || kk > 4) ? 1u : 0u);
+                    mma_commit(&bars[TB_UDONE20 + grp]);
+                    mma_commit(&bars[TB_EMPTY0 + s]);
+                }
+            }
+            // ---- S <- gamma_C S while the U^T MMAs run ----
+#pragma unroll 1
+            for (int piece = 0; piece < 2; ++piece) {
+                const int col0 = ch * 64 + piece * 32;
+                uint32_t r[32];
+                tmem_ld32(tg + lb + TT_S + col0, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * gC);
+                tmem_st32(tg + lb + TT_S + col0, r);
+            }
+            tmem_wait_st();
+            {
+                bool w = wait_bar(&bars[TB_UDONE0 + grp], c & 1, abort_flag);
+                w = w && wait_bar(&bars[TB_UDONE20 + grp], c & 1, abort_flag);
+                if (!(ok = bar_and(barg, kTrNumGrp, w))) break;
+            }
+            tc_fence_after();
+            // ---- U^T -> bf16 into shared memory (row j, tokens 32 ch .. 32 ch + 31) ----
+#pragma unroll 1
+            for (int piece = 0; piece < 2; ++piece) {
+                uint32_t u[16], u2[16];
+                tmem_ld16(tg + lb + TT_DU + ch * 32 + piece * 16, u);
+                tmem_ld16(tg + lb + TT_DU2 + ch * 32 + piece * 16, u2);
+                tmem_wait_ld();
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = cc * 8 + 2 * e;
+                        w4[e] = pack_bf16x2(__uint_as_float(u[i]) + __uint_as_float(u2[i]),
+                                            __uint_as_float(u[i + 1]) + __uint_as_float(u2[i + 1]));
+                    }
+                    *reinterpret_cast<uint4 *>(ubs + sw128(j, ch * 4 + piece * 2 + cc)) =
+                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            named_bar(barg, kTrNumGrp);
+            // ---- S += U^T (diag(dl) K) ----
+            if (gt == 0) {
+                if (wait_bar(&bars[TB_KREADY0 + s], sp, abort_flag)) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss(tg + TT_S, smem_desc_sw128(ubs_a + kk * 32, 16, 1024),
+                               smem_desc_sw128(st + TS_K + kk * 2048, 8192, 1024), IDESC_TS, 1);
+                    mma_commit(&bars[TB_SDONE0 + grp]);
+                    mma_commit(&bars[TB_EMPTY0 + s]);
+                }
+                if (grp == 0) arrive(&bars[TB_SISSUED]);
+            }
+        }
+        if (ok && N > 0) {
+            ok = role_wait(&bars[TB_SDONE0 + grp], (N - 1) & 1, abort_flag, barg, kTrNumGrp);
+            tc_fence_after();
+        }
+        float *dst = (grp == 0 ? p.Bw : p.Mw) + ((bh * (p.nseg - 1) + seg) * kD + j) * (int64_t)kD;
+        if (ok) {
+#pragma unroll 1
+            for (int piece = 0; piece < 2; ++piece) {
+                const int col0 = ch * 64 + piece * 32;
+                uint32_t r[32];
+                tmem_ld32(tg + lb + TT_S + col0, r);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; i += 4)
@@ -1039,9 +1330,10 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
         !make_map_tiles(&mp, ws_p, items, 64) || !make_map_tiles(&mtb, ws_tb, items, 64) ||
         !make_map_tiles(&mw, ws_w, items, 128))
         return cudaErrorInvalidValue;
-    static std::atomic<uint64_t> conf_prep{0}, conf_chain{0};
+    static std::atomic<uint64_t> conf_prep{0}, conf_chain{0}, conf_tr{0};
     if (!configure_once((const void *)fwd_prep_kernel, SMEM_PREP, conf_prep) ||
-        !configure_once((const void *)fwd_chain_kernel, SMEM_CHAIN, conf_chain))
+        !configure_once((const void *)fwd_chain_kernel, SMEM_CHAIN, conf_chain) ||
+        !configure_once((const void *)fwd_transfer_kernel, SMEM_TR, conf_tr))
         return cudaErrorInvalidValue;
 
     PrepArgs pa;
@@ -1079,18 +1371,18 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
         a.Mw = a.Bw + per;
         float *entry = a.Mw + per;
         a.S_entry = entry;
-        a.mode = 1;  // segment transfers of segments 0..nseg-2
+        // segment transfers of segments 0..nseg-2, both runs of a segment in one CTA
         {
             TimedLaunch tl_(GDN_KERNEL_TRANSFER, stream);
-            fwd_chain_kernel<<<(unsigned)(heads * (a.nseg - 1) * 2), kChainThreads, SMEM_CHAIN, stream>>>(
-                mq, mk, mv, mo, mp, mtb, mw, a);
+            fwd_transfer_kernel<<<(unsigned)(heads * (a.nseg - 1)), kTrThreads, SMEM_TR, stream>>>(mk, mv, mtb, mw,
+                                                                                                  a);
         }
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         e = launch_seg_prefix(p.S0, a.Bw, a.Mw, entry, heads, a.nseg, stream);
         if (e != cudaSuccess) return e;
     }
-    a.mode = 0;  // outputs of every segment from its entry state
+    // outputs of every segment from its entry state
     {
         TimedLaunch tl_(GDN_KERNEL_CHAIN, stream);
         fwd_chain_kernel<<<(unsigned)(heads * a.nseg), kChainThreads, SMEM_CHAIN, stream>>>(mq, mk, mv, mo, mp, mtb, mw,

@@ -914,11 +914,12 @@ bool fwd_tc_supported(const FwdProblem &p) {
 }
 
 // Segments per (b, h): the count minimising a wave model of the passes, in
-// units of half a chunk step of one CTA: transfers (2 (nseg - 1) CTAs per
-// head) and outputs (nseg CTAs per head), each CTA over ceil(chunks / nseg)
-// chunks, plus the sequential prefix over segments (about half a chunk step
-// per segment).  GDN_SEGMENTS overrides the choice.
-int fwd_tc_segments(const FwdProblem &p, int sm_count) {
+// units of half a chunk step of one CTA: transfers (nseg - 1 CTAs per head
+// when both runs of a segment share a CTA, else 2 (nseg - 1)) and outputs
+// (nseg CTAs per head), each CTA over ceil(chunks / nseg) chunks, plus the
+// sequential prefix over segments (about half a chunk step per segment).
+// GDN_SEGMENTS overrides the choice.
+int fwd_tc_segments(const FwdProblem &p, int sm_count, bool paired_transfers) {
     const int64_t chunks = (p.T + kC - 1) / kC, heads = p.B * p.H;
     if (chunks <= 0 || heads <= 0) return 1;
     const char *env = getenv("GDN_SEGMENTS");
@@ -935,7 +936,8 @@ int fwd_tc_segments(const FwdProblem &p, int sm_count) {
         const int64_t len = (chunks + nseg - 1) / nseg;
         if (len < 4) break;
         const int64_t real = (chunks + len - 1) / len;
-        const int64_t cost = 2 * (waves(2 * heads * (real - 1)) + waves(heads * real)) * len + (real - 1);
+        const int64_t tr = (paired_transfers ? 1 : 2) * heads * (real - 1);
+        const int64_t cost = 2 * (waves(tr) + waves(heads * real)) * len + (real - 1);
         if (cost < best_cost) {
             best_cost = cost;
             best = (int)real;

@@ -277,7 +277,7 @@ int gdn_forward(const void *q, const void *k, const void *v, const float *log_al
         const FwdPath path = forced_path();
         bool done = false;
         if (path == FwdPath::Auto && gdn::fwd_split_supported(p)) {
-            const int nseg = gdn::fwd_tc_segments(p, info.sm_count);
+            const int nseg = gdn::fwd_tc_segments(p, info.sm_count, true);
             void *ws = nullptr;
             if (scratch_alloc(&ws, gdn::fwd_split_workspace_bytes(p, nseg), stream) == cudaSuccess) {
                 e = gdn::launch_fwd_split(p, nseg, info.sm_count, ws, stream);
@@ -289,7 +289,7 @@ int gdn_forward(const void *q, const void *k, const void *v, const float *log_al
             }
         }
         if (!done && path != FwdPath::Simt && gdn::fwd_tc_supported(p)) {
-            const int nseg = gdn::fwd_tc_segments(p, info.sm_count);
+            const int nseg = gdn::fwd_tc_segments(p, info.sm_count, false);
             const size_t ws_bytes = gdn::fwd_tc_workspace_bytes(p, nseg);
             void *ws = nullptr;
             if (ws_bytes > 0 && scratch_alloc(&ws, ws_bytes, stream) != cudaSuccess) {
@@ -331,11 +331,11 @@ int gdn_forward_plan(int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv, in
     p.B = B; p.T = T; p.H = H; p.dk = dk; p.dv = dv; p.chunk = chunk; p.dtype = dtype;
     const FwdPath path = forced_path();
     if (path == FwdPath::Auto && gdn::fwd_split_supported(p)) {
-        const int nseg = gdn::fwd_tc_segments(p, info.sm_count);
+        const int nseg = gdn::fwd_tc_segments(p, info.sm_count, true);
         if (scratch_bytes) *scratch_bytes = (int64_t)gdn::fwd_split_workspace_bytes(p, nseg);
         if (launches) *launches = nseg > 1 ? 4 : 2;
     } else if (path != FwdPath::Simt && gdn::fwd_tc_supported(p)) {
-        const int nseg = gdn::fwd_tc_segments(p, info.sm_count);
+        const int nseg = gdn::fwd_tc_segments(p, info.sm_count, false);
         if (scratch_bytes) *scratch_bytes = (int64_t)gdn::fwd_tc_workspace_bytes(p, nseg);
         if (launches) *launches = nseg > 1 ? 3 : 1;
     } else if (launches) {

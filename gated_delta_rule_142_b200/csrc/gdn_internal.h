@@ -57,7 +57,7 @@ cudaError_t launch_fwd_simt(const FwdProblem &p, int sm_count, cudaStream_t stre
 // float32 prefix over segments and an output pass, with
 // fwd_tc_workspace_bytes() of scratch (device memory, caller-provided).
 bool fwd_tc_supported(const FwdProblem &p);
-int fwd_tc_segments(const FwdProblem &p, int sm_count);
+int fwd_tc_segments(const FwdProblem &p, int sm_count, bool paired_transfers);
 size_t fwd_tc_workspace_bytes(const FwdProblem &p, int nseg);
 cudaError_t launch_fwd_tc(const FwdProblem &p, int nseg, void *workspace, cudaStream_t stream);
 // Entry states of segments 1..nseg-1 from the segment transfers, in float32.

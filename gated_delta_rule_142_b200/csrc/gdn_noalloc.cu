@@ -132,11 +132,12 @@ extern "C" int gdn_forward_noalloc(const void *q, const void *k, const void *v, 
     } else if (gdn::fwd_tc_supported(p)) {
         // the two-kernel forward when its per-chunk workspace fits the array, else the
         // single-kernel forward, which needs scratch only for segments
-        const int nseg = gdn::fwd_tc_segments(p, sms);
+        const int nseg_split = gdn::fwd_tc_segments(p, sms, true);
         if (gdn::fwd_split_supported(p) &&
-            gdn::fwd_split_workspace_bytes(p, nseg) <= (size_t)GDN_NOALLOC_SCRATCH_BYTES) {
-            e = gdn::launch_fwd_split(p, nseg, sms, scratch, stream);
+            gdn::fwd_split_workspace_bytes(p, nseg_split) <= (size_t)GDN_NOALLOC_SCRATCH_BYTES) {
+            e = gdn::launch_fwd_split(p, nseg_split, sms, scratch, stream);
         } else {
+            const int nseg = gdn::fwd_tc_segments(p, sms, false);
             const size_t need = gdn::fwd_tc_workspace_bytes(p, nseg);
             if (need > (size_t)GDN_NOALLOC_SCRATCH_BYTES) return GDN_ERR_SCRATCH_LIMIT;
             e = gdn::launch_fwd_tc(p, nseg, need ? scratch : nullptr, stream);
