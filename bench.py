@@ -67,7 +67,8 @@ def decode_bytes_per_head_step(dk, dv, es):
 # DRAM bytes (read + write) per token-head that one ncu capture of each kernel kind measured, from
 # the summaries in profiles/ (fwd_chain_b8h16_t2k_d128.md, fwd_prep_b8h16_t2k_d128.md,
 # fwd_transfer_b1h16_t16k_s4.md).  For the transfer kind the unit is a token-head of the
-# transferred segments (covering both of its runs).  Kept only while those kernels are unchanged.
+# transferred segments (covering both of its runs, which one CTA runs together).  Kept only while
+# those kernels are unchanged.
 NCU_TRAFFIC_PER_TOKEN_HEAD = {"chain": 400.0e6 / 262144, "prep": 225.4e6 / 262144, "transfer": 181.7e6 / 196608}
 
 
