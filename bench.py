@@ -72,6 +72,12 @@ def decode_bytes_per_head_step(dk, dv, es):
 NCU_TRAFFIC_PER_TOKEN_HEAD = {"chain": 400.0e6 / 262144, "prep": 225.4e6 / 262144, "transfer": 181.7e6 / 196608}
 
 
+# DRAM bytes (read + write) per decode launch from the ncu capture summarised in
+# profiles/decode_bf16_b64h16_d128.md: about half of the 134 MB state stays in the 126 MB L2 from
+# one step to the next, so DRAM moves 0.58x the algorithmic bytes.
+NCU_DECODE_TRAFFIC = {"decode_bf16_b64h16_d128_x1024": 78.2e6}
+
+
 def kernel_units(kind, w, nseg):
     """Token-heads one launch of a kernel kind processes (the unit of NCU_TRAFFIC_PER_TOKEN_HEAD)."""
     nth = w.B * w.T * w.H
@@ -388,15 +394,33 @@ def run_gdn(args, world, rank, local):
 
         for _ in range(max(1, args.warmup // 3)):
             dec_run()
-        dms = time_region(dec_run, 1, stream, world) / dsteps
+        # The 1024 launches (each still one gdn_decode_step call through the C ABI) are captured
+        # once in a CUDA graph and replayed: a Python call costs about as long as one ~20 us decode
+        # kernel, and host overhead must not leave the GPU idle inside the timed region.
+        replay = dec_run
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                cap = torch.cuda.current_stream()
+                for t in range(dsteps):
+                    gdn.decode_step(dd["q"][t], dd["k"][t], dd["v"][t], dd["log_alpha"][t], dd["beta"][t], S,
+                                    out=dout[t], stream=cap)
+            graph.replay()
+            torch.cuda.synchronize()
+            replay = graph.replay
+        except RuntimeError:
+            torch.cuda.synchronize()
+        dms = time_region(replay, 1, stream, world) / dsteps
         dms = max_over_ranks(dms, world)
         des = 2 if wd.dtype == "bf16" else 4
         dbytes = wd.B * wd.H * decode_bytes_per_head_step(wd.dk, wd.dv, des)
         dgbs = dbytes / (dms / 1e3) / 1e9
         dec = {"workload": wd.name, "steps": dsteps, "us_per_step": dms * 1e3,
+               "launch": "cuda_graph" if replay is not dec_run else "eager",
                "tokens_per_s": world * wd.B / (dms / 1e3), "GB_per_s": dgbs,
                "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                            "frac": dgbs / peaks["hbm_gbs"], "traffic": None,
+                            "frac": dgbs / peaks["hbm_gbs"],
+                            "traffic": NCU_DECODE_TRAFFIC.get(wd.name),
                             "peak_kind": peak_kind, "bytes_per_launch": dbytes},
                "launches": dsteps}
         del dd, S, dout

@@ -111,3 +111,25 @@ def test_host_buffers_are_staged():
         del args
     assert rel_err(cpu_f64(torch.stack(outs)).reshape(steps, B * H, d), ref_o) <= TOL["bf16"]
     assert rel_err(cpu_f64(S).reshape(B * H, d, d), ref_S) <= TOL["bf16"]
+
+
+def test_steps_replayed_from_a_cuda_graph():
+    """Device-buffer decode steps can be captured in a CUDA graph (the bench times them that way);
+    a replay gives the oracle's result, like the eager calls."""
+    steps, B, H, d = 5, 4, 2, 128
+    inp = decode_inputs(steps, B, H, d, d, "bf16", seed=59, s0_std=0.1)
+    ref_o, ref_S = oracle_steps(inp, steps)
+    dd = {k: v.cuda() for k, v in inp.items()}
+    S = dd["S"].clone()
+    outs = torch.empty((steps, B, H, d), dtype=dd["q"].dtype, device="cuda")
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        cap = torch.cuda.current_stream()
+        for t in range(steps):
+            gdn.decode_step(dd["q"][t], dd["k"][t], dd["v"][t], dd["log_alpha"][t], dd["beta"][t], S, out=outs[t],
+                            stream=cap)
+    S.copy_(dd["S"])  # capture does not run the kernels; start the replay from the initial state
+    graph.replay()
+    torch.cuda.synchronize()
+    assert rel_err(cpu_f64(outs).reshape(steps, B * H, d), ref_o) <= TOL["bf16"]
+    assert rel_err(cpu_f64(S).reshape(B * H, d, d), ref_S) <= TOL["bf16"]
