@@ -38,7 +38,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from gdn_inputs import WORKLOADS, as_f32_numpy, decode_inputs, forward_inputs  # noqa: E402
+from gdn_inputs import WORKLOADS, as_f32_numpy, decode_inputs, forward_inputs, length_mix, varlen_inputs  # noqa: E402
 
 FWD_WORKLOAD = "fwd_bf16_b1h16_t64k_d128"
 DEC_WORKLOAD = "decode_bf16_b64h16_d128_x1024"
@@ -471,6 +471,67 @@ def run_gdn(args, world, rank, local):
     return 0
 
 
+def run_varlen(args, world, rank):
+    """Packed prefill: args.varlen sequences with lengths drawn log-uniformly from [256, 8192]
+    (seeded), H = 16, d = 128, bf16, one gdn_forward_varlen call per step, inputs in HBM."""
+    import gated_delta_rule_142_b200 as gdn
+    gdn.load()
+    peaks, peak_kind = load_peaks()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    lengths = length_mix(args.varlen, 256, 8192, seed=rank)
+    H, d = 16, 128
+    inp = varlen_inputs(lengths, H, d, d, "bf16", seed=1000 + rank, s0_std=0.02)
+    dd = {n: inp[n].to(dev) for n in ("q", "k", "v", "log_alpha", "beta", "S0")}
+    T = sum(lengths)
+    out = torch.empty((T, H, d), dtype=torch.bfloat16, device=dev)
+    Sf = torch.empty((len(lengths), H, d, d), dtype=torch.float32, device=dev)
+
+    def step():
+        gdn.forward_varlen(dd["q"], dd["k"], dd["v"], dd["log_alpha"], dd["beta"], inp["cu_seqlens"], dd["S0"],
+                           chunk=64, out=out, S_final=Sf, stream=stream)
+
+    sampler = ClockSampler(dev)
+    sampler.start()
+    for _ in range(args.warmup):
+        step()
+    gdn.timing_start()
+    ms = time_region(step, args.steps, stream, world)
+    ktimes = gdn.timing_stop()
+    clocks = sampler.stop()
+    ms_step = max_over_ranks(ms / args.steps, world)
+    nth = T * H
+    work = {"prep": (nth * 6 * 64 * d, nth * (2 * d * 2 + 8 + 2 * 64 + 2 * 64 + 2 * d + 8)),
+            "chain": (nth * (6 * d * d + 4 * 64 * d), nth * (4 * d * 2 + 2 * 64 + 2 * 64 + 2 * d + 8))}
+    kernels = {}
+    for kind, (kms, n) in ktimes.items():
+        per = kms / n
+        flop, by = work.get(kind, (0, 0))
+        kernels[kind] = {"launches_per_step": n / args.steps, "ms_per_launch": per, "share": kms / ms,
+                         "tflops": flop / (per / 1e3) / 1e12, "gb_per_s": by / (per / 1e3) / 1e9}
+    top = max(kernels, key=lambda k: ktimes[k][0]) if kernels else None
+    roof = None
+    if top in work:
+        kt = kernels[top]
+        tf, gb = kt["tflops"] / peaks["bf16_tflops"], kt["gb_per_s"] / peaks["hbm_gbs"]
+        roof = ({"bound": "tensor", "achieved": kt["tflops"], "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                 "frac": tf} if tf >= gb else
+                {"bound": "hbm", "achieved": kt["gb_per_s"], "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gb})
+        roof.update({"kernel": top, "traffic": None, "peak_kind": peak_kind})
+    if rank == 0:
+        line = {"metric": "gated-delta packed prefill tokens/s", "value": world * T / (ms_step / 1e3),
+                "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": "varlen_bf16_n%d_h16_d128" % args.varlen, "sequences": len(lengths),
+                           "tokens": T, "min_len": min(lengths), "max_len": max(lengths), "H": H, "dk": d, "dv": d,
+                           "chunk": 64, "parallelism": "replicas" if world > 1 else "single"},
+                "roofline": roof, "kernels": kernels, "clocks": clocks,
+                "gpu_launches": sum(int(n) for _, n in ktimes.values())}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -482,6 +543,8 @@ def main():
                     help="forward workload timed as the step (default: the 64K-token one)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="time only the first T tokens of the workload (profiler captures); not a bench line")
+    ap.add_argument("--varlen", type=int, default=0,
+                    help="time packed prefill of this many sequences of mixed length instead of the forward step")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -493,6 +556,8 @@ def main():
         return run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
     world, rank, local = dist_setup()
     try:
+        if args.varlen:
+            return run_varlen(args, world, rank)
         return run_gdn(args, world, rank, local)
     finally:
         if world > 1:

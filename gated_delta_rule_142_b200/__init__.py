@@ -36,7 +36,8 @@ STATUS = {
 }
 
 EXPORTS = ("gdn_forward", "gdn_decode_step", "gdn_forward_plan", "gdn_status_string", "gdn_version",
-           "gdn_forward_noalloc", "gdn_scratch_release", "gdn_timing_start", "gdn_timing_stop")
+           "gdn_forward_noalloc", "gdn_scratch_release", "gdn_timing_start", "gdn_timing_stop",
+           "gdn_forward_varlen")
 
 # gdn_kernel_kind names, in enum order
 KERNEL_KINDS = ("prep", "chain", "transfer", "prefix", "fused", "simt", "decode")
@@ -71,6 +72,8 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     lib.gdn_version.restype = ctypes.c_int
     lib.gdn_forward_plan.argtypes = [i64] * 6 + [ctypes.c_int, ctypes.POINTER(i64), ctypes.POINTER(ctypes.c_int)]
     lib.gdn_forward_plan.restype = ctypes.c_int
+    lib.gdn_forward_varlen.argtypes = [vp] * 5 + [ctypes.POINTER(i64), i64] + [vp] * 3 + [i64] * 5 + [vp, ctypes.c_int]
+    lib.gdn_forward_varlen.restype = ctypes.c_int
     lib.gdn_scratch_release.argtypes = []
     lib.gdn_scratch_release.restype = ctypes.c_int
     lib.gdn_timing_start.argtypes = []
@@ -150,6 +153,50 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.
                              _dtype_code(q))
     if st != 0:
         raise GdnError(st, "gdn_forward")
+    return out, S_final
+
+
+def forward_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
+                   beta: torch.Tensor, cu_seqlens, S0: Optional[torch.Tensor] = None, chunk: int = 64,
+                   out: Optional[torch.Tensor] = None, S_final: Optional[torch.Tensor] = None,
+                   output_final_state: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunkwise forward over N packed sequences.  q, k [T_total,H,dk], v [T_total,H,dv];
+    log_alpha, beta [T_total,H] float32; cu_seqlens: N + 1 token offsets (list or CPU int tensor);
+    S0 [N,H,dv,dk] float32 or None.  Returns (out [T_total,H,dv], S_final [N,H,dv,dk] or None)."""
+    lib = load()
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    cu = [int(x) for x in (cu_seqlens.tolist() if torch.is_tensor(cu_seqlens) else cu_seqlens)]
+    N = len(cu) - 1
+    if N < 0:
+        raise ValueError("cu_seqlens needs at least one entry")
+    for name, t, shape in (("k", k, (T, H, dk)), ("v", v, (T, H, dv)), ("log_alpha", log_alpha, (T, H)),
+                           ("beta", beta, (T, H)), ("out", out, (T, H, dv))):
+        if t is not None and tuple(t.shape) != shape:
+            raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), shape))
+    _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype or (out is not None and out.dtype != q.dtype):
+        raise TypeError("q, k, v and out must share one dtype")
+    for name, t in (("log_alpha", log_alpha), ("beta", beta), ("S0", S0), ("S_final", S_final)):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError("%s must be float32" % name)
+    for name, t in (("S0", S0), ("S_final", S_final)):
+        if t is not None and tuple(t.shape) != (N, H, dv, dk):
+            raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), (N, H, dv, dk)))
+    for t in (q, k, v, log_alpha, beta, S0, out, S_final):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    if out is None:
+        out = torch.empty((T, H, dv), dtype=q.dtype, device=q.device, pin_memory=_pinned(q))
+    if S_final is None and output_final_state:
+        S_final = torch.empty((N, H, dv, dk), dtype=torch.float32, device=q.device, pin_memory=_pinned(q))
+    cu_arr = (ctypes.c_int64 * max(len(cu), 1))(*cu)
+    with torch.cuda.device(q.device if q.device.type == "cuda" else torch.cuda.current_device()):
+        st = lib.gdn_forward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), cu_arr, N, _ptr(S0),
+                                    _ptr(out), _ptr(S_final), T, H, dk, dv, int(chunk),
+                                    _stream_handle(q.device, stream), _dtype_code(q))
+    if st != 0:
+        raise GdnError(st, "gdn_forward_varlen")
     return out, S_final
 
 

@@ -39,6 +39,7 @@
 #include <stdlib.h>
 
 #include <atomic>
+#include <vector>
 
 #include "gdn.h"
 #include "gdn_internal.h"
@@ -105,12 +106,16 @@ enum PBar { PB_QFULL = 0, PB_KFULL, PB_GDONE, PB_GFREE, PB_TBREADY, PB_WDONE, PB
 
 static_assert(PB_COUNT * 8 <= PO_MISC - PO_BARS, "prep-kernel mbarriers overflow their shared-memory slot");
 
+// Packed variable-length sequences: chunk i of the packed tensor starts at
+// token ctab[i].x and has ctab[i].y tokens (the last chunk of a sequence may be
+// partial); work item i * H + h is chunk i of head h.
 struct PrepArgs {
     const float *log_alpha, *beta;
     float *gate_rec;  // [items][128]: gamma_t, then dl_s = e^{g_63 - g_s}
     int64_t T, H;
-    int64_t items;  // B * H * chunks
-    int chunks;     // chunks per (b, h)
+    int64_t items;     // B * H * chunks, or (packed chunks) * H
+    int chunks;        // chunks per (b, h) (fixed-length problems)
+    const int2 *ctab;  // packed chunk table, or nullptr for fixed-length problems
 };
 
 __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
@@ -133,12 +138,24 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     // items < 2^24 (checked on the host), so 32-bit index arithmetic suffices
     auto item = [&](int it) -> uint32_t { return blockIdx.x + (uint32_t)it * gridDim.x; };
     // (b, h, first token) of work item `it`
-    auto coords = [&](int it, int &b, int &h, int &t0) {
-        const uint32_t gi = item(it), bh = gi / (uint32_t)p.chunks;
-        const uint32_t hh = (uint32_t)H;
-        b = (int)(bh / hh);
-        h = (int)(bh - (uint32_t)b * hh);
-        t0 = (int)(gi - bh * (uint32_t)p.chunks) * kC;
+    // (b, h, first token, tokens) of work item `it`
+    auto coords = [&](int it, int &b, int &h, int &t0, int &nt) {
+        const uint32_t gi = item(it);
+        if (p.ctab) {
+            const uint32_t cid = gi / (uint32_t)H;
+            const int2 e = p.ctab[cid];
+            b = 0;
+            h = (int)(gi - cid * (uint32_t)H);
+            t0 = e.x;
+            nt = e.y;
+        } else {
+            const uint32_t bh = gi / (uint32_t)p.chunks;
+            const uint32_t hh = (uint32_t)H;
+            b = (int)(bh / hh);
+            h = (int)(bh - (uint32_t)b * hh);
+            t0 = (int)(gi - bh * (uint32_t)p.chunks) * kC;
+            nt = (T - t0 < kC) ? (int)(T - t0) : kC;
+        }
     };
     const uint32_t sbase = smem_u32(sm);
 
@@ -161,15 +178,15 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         // ============================ issuer ============================
         if (lane == 0) {
             auto load_q = [&](int it) {
-                int b, h, t0;
-                coords(it, b, h, t0);
+                int b, h, t0, nt;
+                coords(it, b, h, t0, nt);
                 mbar_arrive_expect_tx(&bars[PB_QFULL], 2 * 8192);
                 for (int blk = 0; blk < 2; ++blk)
                     tma_load_4d(sm + PO_QK + blk * 16384, &tm_q, &bars[PB_QFULL], blk * 64, h, t0, b);
             };
             auto load_k = [&](int it) {
-                int b, h, t0;
-                coords(it, b, h, t0);
+                int b, h, t0, nt;
+                coords(it, b, h, t0, nt);
                 mbar_arrive_expect_tx(&bars[PB_KFULL], 2 * 8192);
                 for (int blk = 0; blk < 2; ++blk)
                     tma_load_4d(sm + PO_QK + blk * 16384 + 8192, &tm_k, &bars[PB_KFULL], blk * 64, h, t0, b);
@@ -228,12 +245,13 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         fence_proxy_async_smem();
         // gates of work item `it` into buffer it & 1 (threads pt < 64 hold token pt)
         float la_next = 0.f, be_next = 0.f;
+        // gates of token t of work item `it`; -1 past the chunk's tokens (they act as alpha = 1,
+        // beta = 0, so they leave the chunk's recurrence unchanged)
         auto gate_index = [&](int it, int t) -> int64_t {
-            int b, h, t0;
-            coords(it, b, h, t0);
-            const int64_t tok = (int64_t)t0 + t;
-            if (tok >= T) return -1;
-            return ((int64_t)b * T + tok) * H + h;
+            int b, h, t0, nt;
+            coords(it, b, h, t0, nt);
+            if (t >= nt) return -1;
+            return ((int64_t)b * T + t0 + t) * H + h;
         };
         if (nit > 0 && pt < 64) {
             const int64_t x = gate_index(0, pt);
@@ -564,15 +582,21 @@ enum CBar {
 // transfer kernel's.
 static_assert(CB_COUNT * 8 <= CO_MISC - CO_BARS, "chain-kernel mbarriers overflow their shared-memory slot");
 
+// Packed variable-length sequences (no segments): CTA i runs sequence
+// ptab[i].x, head ptab[i].y, packed chunks ptab[i].z .. ptab[i].z + ptab[i].w - 1
+// of the chunk table ctab; its states are S0 / S_final [seq * H + head].
 struct ChainArgs {
     const float *gate_rec;  // [items][128] from the prep kernel
     const float *S0;
     float *S_final;
     int64_t T, H;
-    int chunks;  // chunks per (b, h)
+    int chunks;  // chunks per (b, h) (fixed-length problems)
     int nseg, seg_len;
     const float *S_entry;  // [B*H][nseg-1][dv][dk]
     float *Bw, *Mw;        // [B*H][nseg-1][dv][dk] / [dk][dk]
+    const int4 *ptab;      // per-CTA work of packed sequences, or nullptr
+    const int2 *ctab;      // packed chunk table, or nullptr
+    __nv_bfloat16 *out;    // for the plain stores of partial packed chunks
 };
 
 __global__ void __launch_bounds__(kChainThreads, 1)
@@ -589,12 +613,30 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t H = p.H;
     SDBG_INIT
-    const int64_t bh = blockIdx.x / p.nseg;
-    const int seg = (int)(blockIdx.x % p.nseg);
-    const int b = (int)(bh / H), h = (int)(bh % H);
-    const int c0 = seg * p.seg_len;
-    const int N = (p.chunks - c0 < p.seg_len) ? (p.chunks - c0) : p.seg_len;
-    const int64_t item0 = bh * p.chunks + c0;  // workspace tile index of this CTA's first chunk
+    // work of this CTA: state index bh (S0 / S_final row block), segment, head and chunks; chunk c
+    // starts at token tok0(c) of batch row b and is workspace item witem(c)
+    int64_t bh;
+    int seg, b, h, c0, N;
+    const bool packed = p.ptab != nullptr;
+    if (packed) {
+        const int4 w = p.ptab[blockIdx.x];
+        bh = (int64_t)w.x * H + w.y;
+        seg = 0;
+        b = 0;
+        h = w.y;
+        c0 = w.z;
+        N = w.w;
+    } else {
+        bh = blockIdx.x / p.nseg;
+        seg = (int)(blockIdx.x % p.nseg);
+        b = (int)(bh / H);
+        h = (int)(bh % H);
+        c0 = seg * p.seg_len;
+        N = (p.chunks - c0 < p.seg_len) ? (p.chunks - c0) : p.seg_len;
+    }
+    auto tok0 = [&](int c) -> int { return packed ? p.ctab[c0 + c].x : (c0 + c) * kC; };
+    auto ntok = [&](int c) -> int { return packed ? p.ctab[c0 + c].y : kC; };  // TMA clips at T otherwise
+    auto witem = [&](int c) -> int64_t { return packed ? (int64_t)(c0 + c) * H + h : bh * p.chunks + c0 + c; };
     const uint32_t sbase = smem_u32(sm);
 
     if (tid == 0) {
@@ -623,8 +665,8 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 if (c >= 2 && !(ok = wait_bar(&bars[CB_EMPTY0 + s], ((c - 2) >> 1) & 1, abort_flag))) break;
                 uint8_t *st = sm + s * ST_BYTES;
                 uint64_t *full = &bars[CB_FULL0 + s];
-                const int t0 = (c0 + c) * kC;
-                const int row = (int)(item0 + c);
+                const int t0 = tok0(c);
+                const int row = (int)witem(c);
                 mbar_arrive_expect_tx(full, bytes);
                 for (int blk = 0; blk < 2; ++blk) {
                     tma_load_4d(st + ST_Q + blk * 8192, &tm_q, full, blk * 64, h, t0, b);
@@ -738,10 +780,27 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             fence_proxy_async_smem();
             tc_fence_before();
             named_bar(kBarOut, kNumOut);
-            if (ot == 0) {
-                tma_store_4d(&tm_o, sm + CO_OST, 0, h, (c0 + cprev) * kC, b);
-                tma_store_4d(&tm_o, sm + CO_OST + 8192, 64, h, (c0 + cprev) * kC, b);
-                bulk_commit();
+            const int t0 = tok0(cprev), nt = ntok(cprev);
+            if (nt == kC) {
+                if (ot == 0) {
+                    tma_store_4d(&tm_o, sm + CO_OST, 0, h, t0, b);
+                    tma_store_4d(&tm_o, sm + CO_OST + 8192, 64, h, t0, b);
+                    bulk_commit();
+                }
+            } else {
+                // a partial chunk of a packed sequence: a 64-row box would write the next sequence's
+                // rows, so its nt rows leave by plain 16-byte stores (unit u: box u >> 9, row
+                // (u >> 3) & 63, 16-byte column chunk u & 7)
+                __nv_bfloat16 *o = p.out;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int u = ot + 256 * i, box = u >> 9, row = (u >> 3) & 63, cc = u & 7;
+                    if (row < nt) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(sm + CO_OST + box * 8192 + sw128(row, cc));
+                        *reinterpret_cast<uint4 *>(o + ((int64_t)(t0 + row) * H + h) * kD + box * 64 + cc * 8) = v;
+                    }
+                }
+                named_bar(kBarOut, kNumOut);  // the staging buffer is read before the next chunk writes it
             }
         };
         for (int c = 0; c < N && ok; ++c) {
@@ -1344,6 +1403,7 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
     pa.H = p.H;
     pa.items = items;
     pa.chunks = (int)chunks;
+    pa.ctab = nullptr;
     const int64_t pgrid =
         items < kPrepCtasPerSm * (int64_t)sm_count ? items : kPrepCtasPerSm * (int64_t)sm_count;
     {
@@ -1365,6 +1425,9 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
     a.nseg = (int)((chunks + a.seg_len - 1) / a.seg_len);
     a.S_entry = nullptr;
     a.Bw = a.Mw = nullptr;
+    a.ptab = nullptr;
+    a.ctab = nullptr;
+    a.out = static_cast<__nv_bfloat16 *>(p.out);
     if (a.nseg > 1) {
         const size_t per = (size_t)heads * (a.nseg - 1) * kD * kD;
         a.Bw = seg_ws;
@@ -1387,6 +1450,95 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
         TimedLaunch tl_(GDN_KERNEL_CHAIN, stream);
         fwd_chain_kernel<<<(unsigned)(heads * a.nseg), kChainThreads, SMEM_CHAIN, stream>>>(mq, mk, mv, mo, mp, mtb, mw,
                                                                                             a);
+    }
+    return cudaGetLastError();
+}
+
+// Tables after the per-chunk tiles: the chunk table (int2 entries), then, from the next 256-byte
+// boundary, the per-CTA table (int4 entries, read with 16-byte loads).
+size_t packed_ctab_bytes(int64_t total_chunks) {
+    return ((size_t)total_chunks * sizeof(int2) + 255) & ~(size_t)255;
+}
+
+size_t fwd_split_packed_workspace_bytes(int64_t total_chunks, int64_t H, int64_t N) {
+    const size_t items = (size_t)total_chunks * (size_t)H;
+    return items * kWsPerChunk + packed_ctab_bytes(total_chunks) + (size_t)(N * H) * sizeof(int4);
+}
+
+cudaError_t launch_fwd_split_packed(const FwdProblem &p, const int64_t *cu_seqlens, int64_t N, int sm_count,
+                                    void *workspace, cudaStream_t stream) {
+    const int64_t H = p.H;
+    // chunk table over the packed tokens and one work entry per (sequence, head)
+    std::vector<int2> ctab;
+    std::vector<int4> ptab;
+    ptab.reserve((size_t)(N * H));
+    for (int64_t i = 0; i < N; ++i) {
+        const int64_t t0 = cu_seqlens[i], len = cu_seqlens[i + 1] - t0;
+        const int first = (int)ctab.size(), n = (int)((len + kC - 1) / kC);
+        for (int c = 0; c < n; ++c) {
+            const int64_t tc = t0 + (int64_t)c * kC;
+            ctab.push_back(make_int2((int)tc, (int)((len - (int64_t)c * kC) < kC ? (len - (int64_t)c * kC) : kC)));
+        }
+        for (int64_t h = 0; h < H; ++h) ptab.push_back(make_int4((int)i, (int)h, first, n));
+    }
+    const int64_t chunks = (int64_t)ctab.size(), items = chunks * H;
+    if (N * H == 0) return cudaSuccess;
+    if (!workspace) return cudaErrorInvalidValue;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    uint8_t *ws_p = ws, *ws_tb = ws + items * kTileP, *ws_w = ws_tb + items * kTileTB;
+    float *ws_gates = reinterpret_cast<float *>(ws_w + items * kTileW);
+    int2 *d_ctab = reinterpret_cast<int2 *>(ws + items * kWsPerChunk);
+    int4 *d_ptab = reinterpret_cast<int4 *>(ws + items * kWsPerChunk + packed_ctab_bytes(chunks));
+    cudaError_t e = cudaSuccess;
+    if (chunks > 0) e = cudaMemcpyAsync(d_ctab, ctab.data(), ctab.size() * sizeof(int2), cudaMemcpyHostToDevice, stream);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(d_ptab, ptab.data(), ptab.size() * sizeof(int4), cudaMemcpyHostToDevice, stream);
+    if (e != cudaSuccess) return e;
+    const int64_t rows = items > 0 ? items : 1;  // tile maps need a non-empty extent
+    CUtensorMap mq, mk, mv, mo, mp, mtb, mw;
+    if (!make_map_bthd(&mq, p.q, 1, p.T, p.H) || !make_map_bthd(&mk, p.k, 1, p.T, p.H) ||
+        !make_map_bthd(&mv, p.v, 1, p.T, p.H) || !make_map_bthd(&mo, p.out, 1, p.T, p.H) ||
+        !make_map_tiles(&mp, ws_p, rows, 64) || !make_map_tiles(&mtb, ws_tb, rows, 64) ||
+        !make_map_tiles(&mw, ws_w, rows, 128))
+        return cudaErrorInvalidValue;
+    static std::atomic<uint64_t> conf_prep{0}, conf_chain{0};
+    if (!configure_once((const void *)fwd_prep_kernel, SMEM_PREP, conf_prep) ||
+        !configure_once((const void *)fwd_chain_kernel, SMEM_CHAIN, conf_chain))
+        return cudaErrorInvalidValue;
+    if (items > 0) {
+        PrepArgs pa;
+        pa.log_alpha = p.log_alpha;
+        pa.beta = p.beta;
+        pa.gate_rec = ws_gates;
+        pa.T = p.T;
+        pa.H = p.H;
+        pa.items = items;
+        pa.chunks = 0;
+        pa.ctab = d_ctab;
+        const int64_t pgrid =
+            items < kPrepCtasPerSm * (int64_t)sm_count ? items : kPrepCtasPerSm * (int64_t)sm_count;
+        TimedLaunch tl_(GDN_KERNEL_PREP, stream);
+        fwd_prep_kernel<<<(unsigned)pgrid, kPrepThreads, SMEM_PREP, stream>>>(mq, mk, mp, mtb, mw, pa);
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    ChainArgs a;
+    a.gate_rec = ws_gates;
+    a.S0 = p.S0;
+    a.S_final = p.S_final;
+    a.T = p.T;
+    a.H = p.H;
+    a.chunks = 0;
+    a.nseg = 1;
+    a.seg_len = 0;
+    a.S_entry = nullptr;
+    a.Bw = a.Mw = nullptr;
+    a.ptab = d_ptab;
+    a.ctab = d_ctab;
+    a.out = static_cast<__nv_bfloat16 *>(p.out);
+    {
+        TimedLaunch tl_(GDN_KERNEL_CHAIN, stream);
+        fwd_chain_kernel<<<(unsigned)(N * H), kChainThreads, SMEM_CHAIN, stream>>>(mq, mk, mv, mo, mp, mtb, mw, a);
     }
     return cudaGetLastError();
 }

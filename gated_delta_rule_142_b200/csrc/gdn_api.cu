@@ -311,6 +311,121 @@ int gdn_forward(const void *q, const void *k, const void *v, const float *log_al
     return GDN_OK;
 }
 
+int gdn_forward_varlen(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                       const int64_t *cu_seqlens, int64_t N, const float *S0, void *out, float *S_final,
+                       int64_t T_total, int64_t H, int64_t dk, int64_t dv, int64_t chunk, void *stream_,
+                       int dtype) {
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
+    if (N < 0 || T_total < 0 || H < 0 || dk < 0 || dv < 0 || chunk < 0) return GDN_ERR_INVALID_SIZE;
+    if (!supported_dim(dk) || !supported_dim(dv) || !supported_chunk(chunk)) return GDN_ERR_UNSUPPORTED;
+    if (N > 0 && !cu_seqlens) return GDN_ERR_INVALID_SIZE;
+    if (N > 0) {
+        if (cu_seqlens[0] != 0 || cu_seqlens[N] != T_total) return GDN_ERR_INVALID_SIZE;
+        for (int64_t i = 0; i < N; ++i)
+            if (cu_seqlens[i + 1] < cu_seqlens[i]) return GDN_ERR_INVALID_SIZE;
+    } else if (T_total != 0) {
+        return GDN_ERR_INVALID_SIZE;
+    }
+    const int64_t es = (dtype == GDN_F32) ? 4 : 2;
+    if (N > (int64_t)INT32_MAX / (H > 0 ? H : 1) || T_total > (int64_t)INT32_MAX / 2) return GDN_ERR_INVALID_SIZE;
+    int64_t ntok, nqk, nv, nstate;
+    if (!mul3(1, T_total, H, &ntok) || !mul3(ntok, dk, es, &nqk) || !mul3(ntok, dv, es, &nv) ||
+        !mul3(N * H, dv, dk * 4, &nstate) || ntok > (INT64_MAX / 8))
+        return GDN_ERR_INVALID_SIZE;
+    if (N * H == 0) return GDN_OK;
+    if (ntok > 0 && (!q || !k || !v || !log_alpha || !beta || !out)) return GDN_ERR_NULL_PTR;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(log_alpha) || !aligned4(beta) ||
+        !aligned16(S0) || !aligned16(out) || !aligned16(S_final))
+        return GDN_ERR_MISALIGNED;
+    const Span sq(q, nqk), sk(k, nqk), sv(v, nv), sla(log_alpha, ntok * 4), sbe(beta, ntok * 4);
+    const Span s0(S0, nstate), sf(S_final, nstate), so(out, nv);
+    const Span inputs[] = {sq, sk, sv, sla, sbe, s0, sf};
+    for (const Span &x : inputs)
+        if (overlaps(so, x)) return GDN_ERR_ALIAS;
+    if (overlaps(sf, s0) && !(sf.lo == s0.lo)) return GDN_ERR_ALIAS;
+    for (const Span &x : {sq, sk, sv, sla, sbe})
+        if (overlaps(sf, x)) return GDN_ERR_ALIAS;
+
+    DeviceInfo info;
+    if (int st = device_info(&info)) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    Stager stg(stream);
+    FwdProblem p;
+    int st = GDN_OK;
+    const void *dS0 = nullptr;
+    if ((st = stg.in(q, nqk, true, &p.q)) || (st = stg.in(k, nqk, true, &p.k)) || (st = stg.in(v, nv, true, &p.v)) ||
+        (st = stg.in(log_alpha, ntok * 4, true, reinterpret_cast<const void **>(&p.log_alpha))) ||
+        (st = stg.in(beta, ntok * 4, true, reinterpret_cast<const void **>(&p.beta))) ||
+        (st = stg.in(S0, nstate, true, &dS0)))
+        return st;
+    p.S0 = static_cast<const float *>(dS0);
+    const void *dout = nullptr, *dSf = nullptr;
+    if ((st = stg.in(out, nv, false, &dout))) return st;
+    if (S_final && S_final == S0) {
+        dSf = dS0;
+    } else if ((st = stg.in(S_final, nstate, false, &dSf))) {
+        return st;
+    }
+    p.out = const_cast<void *>(dout);
+    p.S_final = static_cast<float *>(const_cast<void *>(dSf));
+    p.B = 1; p.T = T_total; p.H = H; p.dk = dk; p.dv = dv; p.chunk = chunk; p.dtype = dtype;
+
+    cudaError_t e = cudaSuccess;
+    const FwdPath path = forced_path();
+    bool done = false;
+    if (T_total == 0) {  // every sequence is empty: S_final receives S0 (or zeros)
+        if (p.S_final && p.S_final != p.S0)
+            e = p.S0 ? cudaMemcpyAsync(p.S_final, p.S0, (size_t)nstate, cudaMemcpyDeviceToDevice, stream)
+                     : cudaMemsetAsync(p.S_final, 0, (size_t)nstate, stream);
+        done = true;
+    }
+    int64_t chunks = 0;
+    for (int64_t i = 0; i < N; ++i) chunks += (cu_seqlens[i + 1] - cu_seqlens[i] + 63) / 64;
+    if (!done && path == FwdPath::Auto && gdn::fwd_tc_supported(p) && chunks * H * 128 < ((int64_t)1 << 31)) {
+        // every sequence at once on the two-kernel tensor-core forward
+        void *ws = nullptr;
+        if (scratch_alloc(&ws, gdn::fwd_split_packed_workspace_bytes(chunks, H, N), stream) == cudaSuccess) {
+            e = gdn::launch_fwd_split_packed(p, cu_seqlens, N, info.sm_count, ws, stream);
+            cudaFreeAsync(ws, stream);
+            done = true;
+        } else {
+            cudaGetLastError();
+        }
+    }
+    // otherwise one fixed-length launch per sequence: the single-kernel tensor-core forward (no
+    // segments, so no scratch) or the CUDA-core forward
+    const int64_t state = H * dv * dk;
+    for (int64_t i = 0; i < N && !done && e == cudaSuccess; ++i) {
+        const int64_t t0 = cu_seqlens[i], len = cu_seqlens[i + 1] - t0;
+        FwdProblem pi = p;
+        pi.q = static_cast<const uint8_t *>(p.q) + t0 * H * dk * es;
+        pi.k = static_cast<const uint8_t *>(p.k) + t0 * H * dk * es;
+        pi.v = static_cast<const uint8_t *>(p.v) + t0 * H * dv * es;
+        pi.log_alpha = p.log_alpha + t0 * H;
+        pi.beta = p.beta + t0 * H;
+        pi.out = static_cast<uint8_t *>(p.out) + t0 * H * dv * es;
+        pi.S0 = p.S0 ? p.S0 + i * state : nullptr;
+        pi.S_final = p.S_final ? p.S_final + i * state : nullptr;
+        pi.T = len;
+        if (len == 0) {
+            if (pi.S_final && pi.S_final != pi.S0)
+                e = pi.S0 ? cudaMemcpyAsync(pi.S_final, pi.S0, (size_t)(state * 4), cudaMemcpyDeviceToDevice, stream)
+                          : cudaMemsetAsync(pi.S_final, 0, (size_t)(state * 4), stream);
+        } else if (path != FwdPath::Simt && gdn::fwd_tc_supported(pi)) {
+            e = gdn::launch_fwd_tc(pi, 1, nullptr, stream);
+        } else {
+            e = gdn::launch_fwd_simt(pi, info.sm_count, stream);
+        }
+    }
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_LAUNCH;
+    }
+    if ((st = stg.out_back(out, p.out, nv))) return st;
+    if ((st = stg.out_back(S_final, p.S_final, nstate))) return st;
+    return GDN_OK;
+}
+
 int gdn_forward_plan(int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv, int64_t chunk, int dtype,
                      int64_t *scratch_bytes, int *launches) {
     if (scratch_bytes) *scratch_bytes = 0;

@@ -72,5 +72,10 @@ cudaError_t launch_seg_prefix(const float *S0, const float *Bw, const float *Mw,
 bool fwd_split_supported(const FwdProblem &p);
 size_t fwd_split_workspace_bytes(const FwdProblem &p, int nseg);
 cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *workspace, cudaStream_t stream);
+// Packed variable-length sequences (p.B = 1, p.T = total tokens; cu_seqlens on the
+// host, N + 1 entries): one chain per (sequence, head), no segments.
+size_t fwd_split_packed_workspace_bytes(int64_t total_chunks, int64_t H, int64_t N);
+cudaError_t launch_fwd_split_packed(const FwdProblem &p, const int64_t *cu_seqlens, int64_t N, int sm_count,
+                                    void *workspace, cudaStream_t stream);
 
 }  // namespace gdn

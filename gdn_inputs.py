@@ -105,6 +105,35 @@ def decode_inputs(steps: int, B: int, H: int, dk: int, dv: int, dtype: str = "bf
     return {"S": S, "q": q, "k": k, "v": v, "log_alpha": log_alpha, "beta": beta}
 
 
+def varlen_inputs(lengths, H: int, dk: int, dv: int, dtype: str = "bf16", seed: int = 0,
+                  s0_std: Optional[float] = None, alpha_mu: float = 0.0) -> Dict[str, object]:
+    """Packed sequences of the given lengths: CPU tensors q, k [T,H,dk], v [T,H,dv] (dtype),
+    log_alpha, beta [T,H] fp32 (drawn as one forward_inputs sequence of T = sum(lengths)
+    tokens), S0 [N,H,dv,dk] fp32 or None, and cu_seqlens, a list of N + 1 offsets."""
+    lengths = [int(x) for x in lengths]
+    T = sum(lengths)
+    d = forward_inputs(1, T, H, dk, dv, dtype, seed, None, alpha_mu)
+    out: Dict[str, object] = {n: d[n][0] for n in ("q", "k", "v", "log_alpha", "beta")}
+    out["S0"] = None
+    if s0_std is not None:
+        g = torch.Generator(device="cpu")
+        g.manual_seed(seed + 1)
+        out["S0"] = torch.randn((len(lengths), H, dv, dk), generator=g, dtype=torch.float32) * s0_std
+    cu = [0]
+    for n in lengths:
+        cu.append(cu[-1] + n)
+    out["cu_seqlens"] = cu
+    return out
+
+
+def length_mix(n: int, lo: int, hi: int, seed: int = 0):
+    """n sequence lengths drawn log-uniformly from [lo, hi] (a prefill batch of mixed requests)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    u = torch.rand((n,), generator=g, dtype=torch.float64)
+    return [int(round(lo * (hi / lo) ** float(x))) for x in u]
+
+
 def workload_inputs(w: Workload, steps: Optional[int] = None) -> Dict[str, torch.Tensor]:
     if w.kind == "forward":
         return forward_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, w.seed, w.s0_std, w.alpha_mu)

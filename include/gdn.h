@@ -111,6 +111,40 @@ int gdn_forward(const void *q, const void *k, const void *v, const float *log_al
                 int dtype);
 
 /*
+ * gdn_forward_varlen -- gdn_forward over N sequences of different lengths
+ * packed along the token axis (prefill of a batch of requests).
+ *
+ * Same recurrence as gdn_forward (source: the Sec. 3.3 gated-delta memory
+ * equation), run independently on each sequence i, which is tokens
+ * cu_seqlens[i] .. cu_seqlens[i+1]-1 of the packed tensors; no state flows
+ * from one sequence to the next.
+ *
+ * Arguments:
+ *   q, k           [T_total, H, dk]    (packed; dtype given by `dtype`)
+ *   v, out         [T_total, H, dv]
+ *   log_alpha, beta [T_total, H] float32
+ *   cu_seqlens     HOST array of N + 1 int64 offsets: cu_seqlens[0] = 0,
+ *                  non-decreasing, cu_seqlens[N] = T_total.  Read during the
+ *                  call only.  Empty sequences are allowed.
+ *   S0, S_final    [N, H, dv, dk] float32, one state per sequence and head, or
+ *                  NULL (zero initial state / not written).  S0 == S_final is
+ *                  allowed.
+ *   H, dk, dv, chunk, stream, dtype   as for gdn_forward
+ *
+ * Layout, alignment, aliasing and host-buffer staging rules are those of
+ * gdn_forward with B = 1 and T = T_total.  Errors: GDN_ERR_INVALID_SIZE when
+ * cu_seqlens is not a valid offset array (NULL with N > 0, cu_seqlens[0] !=
+ * 0, decreasing, or cu_seqlens[N] != T_total); the rest as for gdn_forward.
+ * bf16 with dk = dv = 128 and chunk = 64 runs the two-kernel tensor-core
+ * forward over all sequences at once (one chain per sequence and head, no
+ * segments); other shapes run the CUDA-core forward once per sequence.
+ */
+int gdn_forward_varlen(const void *q, const void *k, const void *v, const float *log_alpha,
+                       const float *beta, const int64_t *cu_seqlens, int64_t N, const float *S0,
+                       void *out, float *S_final, int64_t T_total, int64_t H, int64_t dk, int64_t dv,
+                       int64_t chunk, void *stream, int dtype);
+
+/*
  * gdn_forward_plan -- what a gdn_forward call with these sizes will do on the
  * current device, without doing it: *scratch_bytes receives the device scratch
  * it takes from the library's scratch pool (the per-chunk workspace of the

@@ -173,5 +173,31 @@ def decode_step(*args, **kw):
     return get().decode_step(*args, **kw)
 
 
+def forward_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, nthreads: int = 0):
+    """Packed sequences: the recurrence run on each sequence i (tokens cu_seqlens[i] ..
+    cu_seqlens[i+1]-1) from its own initial state S0[i] (zero when S0 is None), with no state
+    passed from one sequence to the next.  q, k [T,H,dk], v [T,H,dv], gates [T,H],
+    S0 [N,H,dv,dk].  Returns (out [T,H,dv] float64, S_final [N,H,dv,dk] float64)."""
+    o = get()
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    cu = [int(x) for x in cu_seqlens]
+    N = len(cu) - 1
+    out = np.zeros((T, H, dv), np.float64)
+    Sf = np.zeros((N, H, dv, dk), np.float64)
+    for i in range(N):
+        a, b = cu[i], cu[i + 1]
+        s0 = None if S0 is None else np.asarray(S0[i:i + 1], np.float64)
+        if b == a:
+            if s0 is not None:
+                Sf[i] = s0[0]
+            continue
+        oi, si = o.forward(q[None, a:b], k[None, a:b], v[None, a:b], log_alpha[None, a:b], beta[None, a:b], s0,
+                           nthreads=nthreads)
+        out[a:b] = oi[0]
+        Sf[i] = si[0]
+    return out, Sf
+
+
 def forward_chunked(*args, **kw):
     return get().forward_chunked(*args, **kw)

@@ -94,6 +94,29 @@ def test_forward_rejects_bad_arguments(lib):
     assert fwd(lib, Sf=A + 0x1000000) == ALIAS
 
 
+def fwd_varlen(lib, cu=(0, 3, 8), q=A, k=A + 0x1000000, v=A + 0x2000000, la=A + 0x3000000, be=A + 0x4000000,
+               S0=None, out=A + 0x5000000, Sf=None, T=8, H=2, dk=16, dv=16, chunk=16, dtype=0):
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    arr = (ctypes.c_int64 * len(cu))(*cu) if cu is not None else None
+    n = len(cu) - 1 if cu is not None else 1
+    return lib.gdn_forward_varlen(P(q), P(k), P(v), P(la), P(be), arr, n, P(S0), P(out), P(Sf), T, H, dk, dv,
+                                  chunk, None, dtype)
+
+
+def test_forward_varlen_rejects_bad_offsets(lib):
+    lib.gdn_forward_varlen.argtypes = [ctypes.c_void_p] * 5 + [ctypes.POINTER(ctypes.c_int64), ctypes.c_int64] + \
+        [ctypes.c_void_p] * 3 + [ctypes.c_int64] * 5 + [ctypes.c_void_p, ctypes.c_int]
+    assert fwd_varlen(lib, cu=(1, 3, 8)) == SIZE   # must start at 0
+    assert fwd_varlen(lib, cu=(0, 5, 3)) == SIZE   # decreasing
+    assert fwd_varlen(lib, cu=(0, 3, 7)) == SIZE   # must end at T
+    assert fwd_varlen(lib, cu=None) == SIZE        # NULL offsets with N > 0
+    assert fwd_varlen(lib, dk=24) == UNSUP
+    assert fwd_varlen(lib, q=A + 8) == MISAL
+    assert fwd_varlen(lib, out=A + 0x2000000) == ALIAS
+    assert fwd_varlen(lib, cu=(0,), T=0) == OK      # no sequences
+    assert fwd_varlen(lib, H=0) == OK
+
+
 def test_forward_empty_problems_are_noops(lib):
     assert fwd(lib, B=0) == OK
     assert fwd(lib, H=0, q=None, k=None, v=None, la=None, be=None, out=None) == OK
