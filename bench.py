@@ -38,7 +38,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from gdn_inputs import WORKLOADS, as_f32_numpy, decode_inputs, forward_inputs, length_mix, varlen_inputs  # noqa: E402
+from gdn_inputs import (WORKLOADS, as_f32_numpy, decode_inputs, forward_inputs, length_mix, raw_inputs,  # noqa: E402
+                        varlen_inputs)
 
 FWD_WORKLOAD = "fwd_bf16_b1h16_t64k_d128"
 DEC_WORKLOAD = "decode_bf16_b64h16_d128_x1024"
@@ -111,7 +112,7 @@ def kernel_work(kind, w, es, nseg):
     chunks = -(-w.T // C)
     seg_len = -(-chunks // max(nseg, 1))
     tr_tokens = min(w.T, (nseg - 1) * seg_len * C) * heads if nseg > 1 else 0
-    tile = 2 * C + 2 * C + 2 * dk + 8  # P, TB, W^T, gate record bytes per token
+    tile = 2 * C + 2 * C + 2 * dk + 8.25  # P, TB, W^T, gate record (528 B per chunk) bytes per token
     if kind == "prep":
         # reads q, k, gates; writes P, TB, W^T and the gate record
         return nth * 6 * C * dk, nth * (2 * dk * es + 8 + tile)
@@ -322,14 +323,23 @@ def run_gdn(args, world, rank, local):
         # a shorter sequence of the same workload, for profiler captures that must stay small
         w = dataclasses.replace(w, T=args.tokens, name="%s_first%d" % (w.name, args.tokens))
     es = 2 if w.dtype == "bf16" else 4
-    inp = forward_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, seed=w.seed + 1000 * rank, s0_std=w.s0_std,
-                         alpha_mu=w.alpha_mu)
+    if args.raw:
+        # the layer's raw projections: q, k unnormalised, gate logits in place of the gates; the
+        # step then includes the input stage
+        r = raw_inputs((w.B, w.T, w.H), w.dk, w.dv, w.dtype, seed=w.seed + 1000 * rank,
+                       s0_shape=(w.B, w.H, w.dv, w.dk), s0_std=w.s0_std, alpha_mu=w.alpha_mu)
+        inp = {"q": r["q"], "k": r["k"], "v": r["v"], "log_alpha": r["x_alpha"], "beta": r["x_beta"], "S0": r["S0"]}
+        w = dataclasses.replace(w, name=w.name + "_raw")
+    else:
+        inp = forward_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, seed=w.seed + 1000 * rank, s0_std=w.s0_std,
+                             alpha_mu=w.alpha_mu)
+    fwd = gdn.forward_raw if args.raw else gdn.forward
     d = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}
     out = torch.empty((w.B, w.T, w.H, w.dv), dtype=d["q"].dtype, device=dev)
     Sf = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=dev)
 
     def fwd_step():
-        gdn.forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"], chunk=w.chunk, out=out,
+        fwd(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"], chunk=w.chunk, out=out,
                     S_final=Sf, stream=stream)
 
     for _ in range(args.warmup):
@@ -348,7 +358,7 @@ def run_gdn(args, world, rank, local):
     gbs = nbytes / (ms_step / 1e3) / 1e9
     scratch_bytes, launches_per_fwd = gdn.forward_plan(w.B, w.T, w.H, w.dk, w.dv, w.chunk, d["q"].dtype)
     chunks = -(-w.T // w.chunk)
-    ws_tiles = w.B * w.H * chunks * (32768 + 512)
+    ws_tiles = w.B * w.H * chunks * (32768 + 528)
     nseg = 1 + max(0, scratch_bytes - ws_tiles) // (3 * w.B * w.H * w.dv * w.dk * 4) if "prep" in ktimes else 1
     kernels = {}
     for kind, (kms, n) in ktimes.items():
@@ -434,7 +444,7 @@ def run_gdn(args, world, rank, local):
         hSf = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32).pin_memory()
 
         def e2e_step():
-            gdn.forward(h["q"], h["k"], h["v"], h["log_alpha"], h["beta"], h["S0"], chunk=w.chunk, out=hout,
+            fwd(h["q"], h["k"], h["v"], h["log_alpha"], h["beta"], h["S0"], chunk=w.chunk, out=hout,
                         S_final=hSf, stream=stream)
 
         e2e_step()
@@ -459,7 +469,8 @@ def run_gdn(args, world, rank, local):
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
-                       "input_dtype": w.dtype, "state_dtype": "f32", "parallelism": "replicas" if world > 1 else "single",
+                       "input_dtype": w.dtype, "state_dtype": "f32",
+                       "input_stage": "fused (raw q, k and gate logits)" if args.raw else "none (unit q, k; gates)", "parallelism": "replicas" if world > 1 else "single",
                        "l2": "inputs larger than L2 (%.2f GB read+written per step)" % (nbytes / 1e9)},
             "tflops": tflops, "gb_per_s": gbs,
             "roofline": roof, "kernels": kernels, "segments": nseg,
@@ -543,6 +554,8 @@ def main():
                     help="forward workload timed as the step (default: the 64K-token one)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="time only the first T tokens of the workload (profiler captures); not a bench line")
+    ap.add_argument("--raw", action="store_true",
+                    help="time gdn_forward_raw (input stage fused: raw q, k and gate logits) instead")
     ap.add_argument("--varlen", type=int, default=0,
                     help="time packed prefill of this many sequences of mixed length instead of the forward step")
     ap.add_argument("--no-decode", action="store_true")

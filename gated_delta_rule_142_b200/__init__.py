@@ -37,10 +37,10 @@ STATUS = {
 
 EXPORTS = ("gdn_forward", "gdn_decode_step", "gdn_forward_plan", "gdn_status_string", "gdn_version",
            "gdn_forward_noalloc", "gdn_scratch_release", "gdn_timing_start", "gdn_timing_stop",
-           "gdn_forward_varlen")
+           "gdn_forward_varlen", "gdn_forward_raw", "gdn_forward_varlen_raw", "gdn_decode_step_raw")
 
 # gdn_kernel_kind names, in enum order
-KERNEL_KINDS = ("prep", "chain", "transfer", "prefix", "fused", "simt", "decode")
+KERNEL_KINDS = ("prep", "chain", "transfer", "prefix", "fused", "simt", "decode", "input")
 
 
 class GdnError(RuntimeError):
@@ -62,18 +62,21 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
                            "`python -m gated_delta_rule_142_b200.build`" % path)
     lib = ctypes.CDLL(path)
     vp, i64 = ctypes.c_void_p, ctypes.c_int64
-    lib.gdn_forward.argtypes = [vp] * 8 + [i64] * 6 + [vp, ctypes.c_int]
-    lib.gdn_forward.restype = ctypes.c_int
-    lib.gdn_decode_step.argtypes = [vp] * 7 + [i64] * 4 + [vp, ctypes.c_int]
-    lib.gdn_decode_step.restype = ctypes.c_int
+    for fn in (lib.gdn_forward, lib.gdn_forward_raw):
+        fn.argtypes = [vp] * 8 + [i64] * 6 + [vp, ctypes.c_int]
+        fn.restype = ctypes.c_int
+    for fn in (lib.gdn_decode_step, lib.gdn_decode_step_raw):
+        fn.argtypes = [vp] * 7 + [i64] * 4 + [vp, ctypes.c_int]
+        fn.restype = ctypes.c_int
     lib.gdn_status_string.argtypes = [ctypes.c_int]
     lib.gdn_status_string.restype = ctypes.c_char_p
     lib.gdn_version.argtypes = []
     lib.gdn_version.restype = ctypes.c_int
     lib.gdn_forward_plan.argtypes = [i64] * 6 + [ctypes.c_int, ctypes.POINTER(i64), ctypes.POINTER(ctypes.c_int)]
     lib.gdn_forward_plan.restype = ctypes.c_int
-    lib.gdn_forward_varlen.argtypes = [vp] * 5 + [ctypes.POINTER(i64), i64] + [vp] * 3 + [i64] * 5 + [vp, ctypes.c_int]
-    lib.gdn_forward_varlen.restype = ctypes.c_int
+    for fn in (lib.gdn_forward_varlen, lib.gdn_forward_varlen_raw):
+        fn.argtypes = [vp] * 5 + [ctypes.POINTER(i64), i64] + [vp] * 3 + [i64] * 5 + [vp, ctypes.c_int]
+        fn.restype = ctypes.c_int
     lib.gdn_scratch_release.argtypes = []
     lib.gdn_scratch_release.restype = ctypes.c_int
     lib.gdn_timing_start.argtypes = []
@@ -124,6 +127,21 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.
     """Chunkwise forward.  q, k [B,T,H,dk], v [B,T,H,dv] (float32 or bfloat16, same dtype);
     log_alpha, beta [B,T,H] float32; S0 [B,H,dv,dk] float32 or None.
     Returns (out [B,T,H,dv] in the input dtype, S_final [B,H,dv,dk] float32 or None)."""
+    return _forward("gdn_forward", q, k, v, log_alpha, beta, S0, chunk, out, S_final, output_final_state, stream)
+
+
+def forward_raw(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, x_alpha: torch.Tensor,
+                x_beta: torch.Tensor, S0: Optional[torch.Tensor] = None, chunk: int = 64,
+                out: Optional[torch.Tensor] = None, S_final: Optional[torch.Tensor] = None,
+                output_final_state: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """forward() with the input stage in the kernels: q, k in any scale (L2-normalised inside),
+    x_alpha, x_beta [B,T,H] float32 gate logits (log alpha = -softplus(x_alpha),
+    beta = sigmoid(x_beta))."""
+    return _forward("gdn_forward_raw", q, k, v, x_alpha, x_beta, S0, chunk, out, S_final, output_final_state,
+                    stream)
+
+
+def _forward(entry, q, k, v, log_alpha, beta, S0, chunk, out, S_final, output_final_state, stream):
     lib = load()
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -148,11 +166,11 @@ def forward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.
     if S_final is None and output_final_state:
         S_final = torch.empty((B, H, dv, dk), dtype=torch.float32, device=q.device, pin_memory=_pinned(q))
     with torch.cuda.device(q.device if q.device.type == "cuda" else torch.cuda.current_device()):
-        st = lib.gdn_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(out),
-                             _ptr(S_final), B, T, H, dk, dv, int(chunk), _stream_handle(q.device, stream),
-                             _dtype_code(q))
+        st = getattr(lib, entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(out),
+                                 _ptr(S_final), B, T, H, dk, dv, int(chunk), _stream_handle(q.device, stream),
+                                 _dtype_code(q))
     if st != 0:
-        raise GdnError(st, "gdn_forward")
+        raise GdnError(st, entry)
     return out, S_final
 
 
@@ -163,6 +181,21 @@ def forward_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha:
     """Chunkwise forward over N packed sequences.  q, k [T_total,H,dk], v [T_total,H,dv];
     log_alpha, beta [T_total,H] float32; cu_seqlens: N + 1 token offsets (list or CPU int tensor);
     S0 [N,H,dv,dk] float32 or None.  Returns (out [T_total,H,dv], S_final [N,H,dv,dk] or None)."""
+    return _forward_varlen("gdn_forward_varlen", q, k, v, log_alpha, beta, cu_seqlens, S0, chunk, out, S_final,
+                           output_final_state, stream)
+
+
+def forward_varlen_raw(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, x_alpha: torch.Tensor,
+                       x_beta: torch.Tensor, cu_seqlens, S0: Optional[torch.Tensor] = None, chunk: int = 64,
+                       out: Optional[torch.Tensor] = None, S_final: Optional[torch.Tensor] = None,
+                       output_final_state: bool = True, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """forward_varlen() with the input stage in the kernels (see forward_raw)."""
+    return _forward_varlen("gdn_forward_varlen_raw", q, k, v, x_alpha, x_beta, cu_seqlens, S0, chunk, out,
+                           S_final, output_final_state, stream)
+
+
+def _forward_varlen(entry, q, k, v, log_alpha, beta, cu_seqlens, S0, chunk, out, S_final, output_final_state,
+                    stream):
     lib = load()
     T, H, dk = q.shape
     dv = v.shape[-1]
@@ -192,11 +225,11 @@ def forward_varlen(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha:
         S_final = torch.empty((N, H, dv, dk), dtype=torch.float32, device=q.device, pin_memory=_pinned(q))
     cu_arr = (ctypes.c_int64 * max(len(cu), 1))(*cu)
     with torch.cuda.device(q.device if q.device.type == "cuda" else torch.cuda.current_device()):
-        st = lib.gdn_forward_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), cu_arr, N, _ptr(S0),
-                                    _ptr(out), _ptr(S_final), T, H, dk, dv, int(chunk),
-                                    _stream_handle(q.device, stream), _dtype_code(q))
+        st = getattr(lib, entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), cu_arr, N, _ptr(S0),
+                                 _ptr(out), _ptr(S_final), T, H, dk, dv, int(chunk),
+                                 _stream_handle(q.device, stream), _dtype_code(q))
     if st != 0:
-        raise GdnError(st, "gdn_forward_varlen")
+        raise GdnError(st, entry)
     return out, S_final
 
 
@@ -241,6 +274,17 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: to
                 stream=None) -> torch.Tensor:
     """One token for every (b, h).  q, k [B,H,dk]; v [B,H,dv]; log_alpha, beta [B,H] float32;
     S [B,H,dv,dk] float32 is updated in place.  Returns out [B,H,dv]."""
+    return _decode("gdn_decode_step", q, k, v, log_alpha, beta, S, out, stream)
+
+
+def decode_step_raw(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, x_alpha: torch.Tensor,
+                    x_beta: torch.Tensor, S: torch.Tensor, out: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """decode_step() with the input stage in the kernel (see forward_raw)."""
+    return _decode("gdn_decode_step_raw", q, k, v, x_alpha, x_beta, S, out, stream)
+
+
+def _decode(entry, q, k, v, log_alpha, beta, S, out, stream):
     lib = load()
     B, H, dk = q.shape
     dv = v.shape[-1]
@@ -259,8 +303,8 @@ def decode_step(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: to
     if out is None:
         out = torch.empty((B, H, dv), dtype=q.dtype, device=q.device, pin_memory=_pinned(q))
     with torch.cuda.device(q.device if q.device.type == "cuda" else torch.cuda.current_device()):
-        st = lib.gdn_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S), _ptr(out),
+        st = getattr(lib, entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S), _ptr(out),
                                  B, H, dk, dv, _stream_handle(q.device, stream), _dtype_code(q))
     if st != 0:
-        raise GdnError(st, "gdn_decode_step")
+        raise GdnError(st, entry)
     return out

@@ -15,6 +15,12 @@
 // (one float4).  A warp covers 32/(DK/4) rows per step and each thread keeps
 // kUnroll rows in flight, so a CTA of 4 warps owns 4 * (32/(DK/4)) * kUnroll
 // rows of one head (32 rows at dk = 128).  Grid: (B*H) x ceil(dv / rows).
+//
+// With the input stage fused (RAW), q and k arrive unnormalised and the gates
+// as logits: the kernel scales its q, k registers by 1 / sqrt(|.|^2 + eps)
+// (the squared norms come from the same lane-group sums as k . q) and maps
+// log alpha = -softplus(x_alpha), beta = sigmoid(x_beta); nothing extra is
+// read or written.
 #include "common.cuh"
 #include "gdn.h"
 #include "gdn_internal.h"
@@ -30,7 +36,7 @@ constexpr int decode_rows_per_cta() {
     return (kDecodeThreads / 32) * (32 / (DK / 4)) * kUnroll;
 }
 
-template <typename Tin, int DK>
+template <typename Tin, int DK, bool RAW>
 __global__ void __launch_bounds__(kDecodeThreads)
 decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
               const float *__restrict__ log_alpha, const float *__restrict__ beta,
@@ -43,10 +49,21 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     const int grp = lane / LPR, gl = lane % LPR;
     const int row_base = blockIdx.y * decode_rows_per_cta<DK>() + warp * RPW + grp;
 
-    const float4 kf = load4(k + head * DK + 4 * gl);
-    const float4 qf = load4(q + head * DK + 4 * gl);
-    const float alpha = expf(log_alpha[head]);
-    const float bt = beta[head];
+    float4 kf = load4(k + head * DK + 4 * gl);
+    float4 qf = load4(q + head * DK + 4 * gl);
+    float alpha, bt;
+    if (RAW) {
+        const float rk = rsqrtf(group_sum<LPR>(dot4(kf, kf)) + kNormEps);
+        const float rq = rsqrtf(group_sum<LPR>(dot4(qf, qf)) + kNormEps);
+        kf = make_float4(kf.x * rk, kf.y * rk, kf.z * rk, kf.w * rk);
+        qf = make_float4(qf.x * rq, qf.y * rq, qf.z * rq, qf.w * rq);
+        const float xa = log_alpha[head], xb = beta[head];
+        alpha = expf(-(fmaxf(xa, 0.f) + log1pf(expf(-fabsf(xa)))));
+        bt = 1.f / (1.f + expf(-xb));
+    } else {
+        alpha = expf(log_alpha[head]);
+        bt = beta[head];
+    }
     const float kq = group_sum<LPR>(dot4(kf, qf));
 
     float *Sh = S + head * (int64_t)dv * DK;
@@ -96,9 +113,10 @@ cudaError_t launch_decode_t(const DecodeProblem &p, cudaStream_t stream) {
     dim3 grid((unsigned)(p.B * p.H), (unsigned)((p.dv + rows - 1) / rows));
     {
         TimedLaunch tl_(GDN_KERNEL_DECODE, stream);
-        decode_kernel<Tin, DK><<<grid, kDecodeThreads, 0, stream>>>(
-            static_cast<const Tin *>(p.q), static_cast<const Tin *>(p.k), static_cast<const Tin *>(p.v),
-            p.log_alpha, p.beta, p.S, static_cast<Tin *>(p.out), (int)p.dv);
+        auto kern = p.raw_inputs ? decode_kernel<Tin, DK, true> : decode_kernel<Tin, DK, false>;
+        kern<<<grid, kDecodeThreads, 0, stream>>>(static_cast<const Tin *>(p.q), static_cast<const Tin *>(p.k),
+                                                  static_cast<const Tin *>(p.v), p.log_alpha, p.beta, p.S,
+                                                  static_cast<Tin *>(p.out), (int)p.dv);
     }
     return cudaGetLastError();
 }

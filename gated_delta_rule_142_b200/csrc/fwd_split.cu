@@ -55,7 +55,11 @@ using namespace tcu;
 constexpr int kC = 64;
 constexpr int kD = 128;
 constexpr size_t kTileP = 64 * 64 * 2, kTileTB = 64 * 64 * 2, kTileW = 128 * 64 * 2;
-constexpr size_t kGateRec = 128 * 4;  // gamma_t and dl_s of one chunk, float32
+// Gate record of one chunk, float32: [0, 64) gamma_t, [64, 128) dl_s = e^{g_63 - g_s}, [128] gamma_C,
+// [129, 132) zero.  With the input stage fused, gamma_t carries 1 / |q_t| and dl_s 1 / |k_s|, the
+// scales of diag(gamma) Q and diag(dl) K in the chain.
+constexpr int kRecFloats = 132;
+constexpr size_t kGateRec = kRecFloats * 4;
 constexpr size_t kWsPerChunk = kTileP + kTileTB + kTileW + kGateRec;  // 32.5 KB
 
 __device__ int g_split_timeout;  // set when a bounded mbarrier wait gives up
@@ -89,11 +93,17 @@ constexpr uint32_t PO_TBG = 40960;   // 8 KB  T diag(beta gamma) [t][s]
 constexpr uint32_t PO_AM = 49152;    // 17 KB A fp32 [64][LDM], overwritten by T in place; after the inverse:
                                      //       W^T bf16 [128][64] staging
 constexpr uint32_t PO_XS = 66560;    // 5 KB  merge scratch
-constexpr uint32_t PO_PG = 71680;    // gates per item parity: g, beta, gamma, e^{g-c}, e^{c-g} (2 x 5 x 64)
-constexpr uint32_t PO_BARS = 74240;  // mbarriers
-constexpr uint32_t PO_MISC = 74304;  // tmem slot, abort flag, scan scratch, flags
-constexpr uint32_t SMEM_PREP = 74368 + 1024;
+constexpr uint32_t PO_PG = 71680;    // gates per item parity: g, beta, gamma, e^{g-c}, e^{c-g}, beta gamma
+                                     // (2 x 6 x 64)
+constexpr int kPG = 384;             // floats per parity
+constexpr uint32_t PO_NRM = 74752;   // input stage: 1 / |q_t|, 1 / |k_s|, g_s - ln(1 / |k_s|) (3 x 64)
+constexpr uint32_t PO_BARS = 75520;  // mbarriers
+constexpr uint32_t PO_MISC = 75584;  // tmem slot, abort flag, scan scratch, flags
+constexpr uint32_t SMEM_PREP = 75648 + 1024;
 constexpr int kPrepCtasPerSm = 3;
+static_assert(PO_PG + 2 * kPG * 4 <= PO_NRM && PO_NRM + 3 * 64 * 4 <= PO_BARS,
+              "prep-kernel gate buffers overflow their slot");
+static_assert(kPrepCtasPerSm * (SMEM_PREP + 1024) <= 233472, "three prep CTAs no longer fit an SM");
 constexpr int kBarMerge = 2;  // named barrier of the four 16->32 merge warps
 
 constexpr uint32_t TP_G = 0;   // 64 columns: [Q;K] K^T
@@ -111,12 +121,22 @@ static_assert(PB_COUNT * 8 <= PO_MISC - PO_BARS, "prep-kernel mbarriers overflow
 // partial); work item i * H + h is chunk i of head h.
 struct PrepArgs {
     const float *log_alpha, *beta;
-    float *gate_rec;  // [items][128]: gamma_t, then dl_s = e^{g_63 - g_s}
+    float *gate_rec;  // [items][kRecFloats]
     int64_t T, H;
     int64_t items;     // B * H * chunks, or (packed chunks) * H
     int chunks;        // chunks per (b, h) (fixed-length problems)
     const int2 *ctab;  // packed chunk table, or nullptr for fixed-length problems
+    int raw_inputs;    // q, k not yet L2-normalised; log_alpha, beta hold the gate logits
 };
+
+// Writes entries (row, col) and (row, col + 1) (col even) of T diag(beta) and T diag(bgk) into
+// their bf16 K-major 128-byte-swizzled tiles.
+__device__ __forceinline__ void store_tb_tbg(uint8_t *tb, uint8_t *tbg, int row, int col, float v0, float v1,
+                                             const float *bet, const float *bgk) {
+    const uint32_t off = sw128(row, col >> 3) + (col & 7) * 2;
+    *reinterpret_cast<uint32_t *>(tb + off) = pack_bf16x2(v0 * bet[col], v1 * bet[col + 1]);
+    *reinterpret_cast<uint32_t *>(tbg + off) = pack_bf16x2(v0 * bgk[col], v1 * bgk[col + 1]);
+}
 
 __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
 fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -261,11 +281,17 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         }
         auto prep_gates = [&](int it) {
-            float *gb = reinterpret_cast<float *>(sm + PO_PG) + (it & 1) * 320;
+            float *gb = reinterpret_cast<float *>(sm + PO_PG) + (it & 1) * kPG;
             if (pt < 64) {
                 const bool valid = gate_index(it, pt) >= 0;
-                const float x = valid ? fmaxf(la_next, kLogAlphaFloor) : 0.f;
-                gb[64 + pt] = valid ? be_next : 0.f;
+                float la = la_next, be = be_next;
+                if (p.raw_inputs) {
+                    // the input stage: log alpha = -softplus(x_alpha), beta = sigmoid(x_beta)
+                    la = -(fmaxf(la, 0.f) + log1pf(expf(-fabsf(la))));
+                    be = 1.f / (1.f + expf(-be));
+                }
+                const float x = valid ? fmaxf(la, kLogAlphaFloor) : 0.f;
+                gb[64 + pt] = valid ? be : 0.f;
                 const float s = chunk_cumsum(x, pt, scan_tmp, kBarP, kNumPrep);
                 SDBG(1, 8)
                 gb[pt] = s;
@@ -285,9 +311,15 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 gb[128 + pt] = gm;
                 gb[192 + pt] = expf(gt - cm);
                 gb[256 + pt] = expf(cm - gt);
-                float *rec = p.gate_rec + (int64_t)item(it) * 128;
-                rec[pt] = gm;
-                rec[64 + pt] = expf(gb[63] - gt);
+                gb[320 + pt] = gb[64 + pt] * gm;
+                if (!p.raw_inputs) {
+                    // the chunk's gate record: gamma_t, dl_s, gamma_C (with the input stage fused it is
+                    // written once the norms are known)
+                    float *rec = p.gate_rec + (int64_t)item(it) * kRecFloats;
+                    rec[pt] = gm;
+                    rec[64 + pt] = expf(gb[63] - gt);
+                    if (pt >= 60) rec[128 + 63 - pt] = (pt == 63) ? gb[63 + 128] : 0.f;  // [128] gamma_C
+                }
                 // e^{g_t - g_s} = e^{g_t - c} e^{c - g_s} while every |g_t - c| < 60, so that
                 // neither factor overflows
                 const bool nr = __all_sync(0xffffffffu, fabsf(gt - cm) < 60.f);
@@ -299,8 +331,10 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int it = 0; it < nit && ok; ++it) {
             const uint32_t par = it & 1;
             const int gi = (int)item(it);
-            const float *g = reinterpret_cast<const float *>(sm + PO_PG) + par * 320;
-            const float *bet = g + 64, *gam = g + 128, *ea = g + 192, *eb = g + 256;
+            float *g = reinterpret_cast<float *>(sm + PO_PG) + par * kPG;
+            // beta, gamma, e^{g - c}, e^{c - g}, beta gamma (the last two carry 1 / |k_s| once the input
+            // stage below has run)
+            const float *bet = g + 64, *gam = g + 128, *ea = g + 192, *eb = g + 256, *bgm = g + 320;
             const bool narrow = nflags[par * 2] && nflags[par * 2 + 1];
             // the stores of the previous item have finished reading P, TB and the W^T staging
             if (pt == 0) {
@@ -309,14 +343,67 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 SDBG(1, 15)
             }
             SDBG(1, 0)
-            if (!(ok = role_wait(&bars[PB_GDONE], par, abort_flag, kBarP, kNumPrep))) break;
+            // with the input stage fused these threads read the Q and K rows too: they also observe the
+            // loads' own barriers (whose phases of this item completed before the G MMA was issued)
+            {
+                bool w = wait_bar(&bars[PB_GDONE], par, abort_flag);
+                if (p.raw_inputs)
+                    w = w && wait_bar(&bars[PB_QFULL], par, abort_flag) && wait_bar(&bars[PB_KFULL], par, abort_flag);
+                if (!(ok = bar_and(kBarP, kNumPrep, w))) break;
+            }
             tc_fence_after();
             SDBG(1, 1)
+            // ---- with the input stage fused: 1 / |q_t| and 1 / |k_s| (the thread pair of a row of
+            //      [Q; K] reads its two 64-column boxes), folded into this item's gate buffers in place:
+            //      e^{c - g_s} and beta_s gamma_s take 1 / |k_s|; the record's gamma_t takes 1 / |q_t|
+            //      and dl_s 1 / |k_s|; the rows' factor enters the G epilogue below ----
+            float *rq = reinterpret_cast<float *>(sm + PO_NRM), *rk = rq + 64, *gkn = rq + 128;
+            const float *gk = p.raw_inputs ? gkn : g;
+            if (p.raw_inputs) {
+                const int r = pt >> 1, box = pt & 1;
+                const uint4 *rowp =
+                    reinterpret_cast<const uint4 *>(sm + PO_QK + box * 16384 + (r >> 6) * 8192 + (r & 63) * 128);
+                // the 16-byte chunks in an order rotated by row and box, so that the eight lanes of
+                // each quarter warp read eight different bank groups
+                float ss = 0.f;
+#pragma unroll 1
+                for (int u = 0; u < 8; ++u) {
+                    const uint4 w4 = rowp[(u + r + 4 * box) & 7];
+                    const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ws[e]));
+                        ss = fmaf(x.x, x.x, fmaf(x.y, x.y, ss));
+                    }
+                }
+                ss += __shfl_xor_sync(0xffffffffu, ss, 1);
+                const float inv = rsqrtf(ss + kNormEps);
+                float *rec = p.gate_rec + (int64_t)gi * kRecFloats;
+                if (box == 0) {
+                    if (r < 64) {
+                        rq[r] = inv;
+                        rec[r] = g[128 + r] * inv;  // gamma_t / |q_t|
+                    } else {
+                        const int c = r - 64;
+                        rk[c] = inv;
+                        gkn[c] = g[c] - logf(inv);
+                        rec[64 + c] = expf(g[63] - g[c]) * inv;  // dl_s / |k_s|
+                        g[256 + c] *= inv;
+                        g[320 + c] *= inv;
+                    }
+                } else if (pt < 8) {
+                    rec[128 + (pt >> 1)] = (pt == 1) ? g[128 + 63] : 0.f;  // [128] gamma_C, [129, 132) 0
+                }
+                named_bar(kBarP, kNumPrep);
+            }
             // ---- epilogue of G: rows 0..63 -> P (bf16), rows 64..127 -> A (fp32); columns by half ----
             {
                 const int m = (warp & 3) * 32 + lane;  // TMEM lane = row of [Q; K]
                 const int t = m & 63;
-                const float gt = g[t], at = ea[t], bt = bet[t];
+                // with the input stage fused, the factors 1 / |q_t| (rows of P) or 1 / |k_t| (rows of A)
+                // and 1 / |k_s| enter through the decays: e^{g_t - g_s} -> e^{(g_t + ln rf_t) - (g_s - ln rk_s)}
+                const float rf = p.raw_inputs ? ((m < 64) ? rq[t] : rk[t]) : 1.f;
+                const float gt = p.raw_inputs ? g[t] + logf(rf) : g[t], at = ea[t] * rf, bt = bet[t];
 #pragma unroll 1
                 for (int piece = 0; piece < 2; ++piece) {
                     const int s0 = ch * 32 + piece * 16;
@@ -332,7 +419,7 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         for (int i = 0; i < 16; ++i) d[i] = at * eb[s0 + i];
                     } else {
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) d[i] = __expf(gt - g[s0 + i]);
+                        for (int i = 0; i < 16; ++i) d[i] = __expf(gt - gk[s0 + i]);
                     }
                     if (m < 64) {
                         uint32_t pk[8];
@@ -409,9 +496,8 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 uint32_t wb[4], wg[4];
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
-                    const float b0 = bet[col + e], b1 = bet[col + e + 1];
-                    wb[e >> 1] = pack_bf16x2(xv[e] * b0, xv[e + 1] * b1);
-                    wg[e >> 1] = pack_bf16x2(xv[e] * (b0 * gam[col + e]), xv[e + 1] * (b1 * gam[col + e + 1]));
+                    wb[e >> 1] = pack_bf16x2(xv[e] * bet[col + e], xv[e + 1] * bet[col + e + 1]);
+                    wg[e >> 1] = pack_bf16x2(xv[e] * bgm[col + e], xv[e + 1] * bgm[col + e + 1]);
                 }
                 const uint32_t off = sw128(row, col >> 3);
                 *reinterpret_cast<uint4 *>(sm + PO_TB + off) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
@@ -439,8 +525,8 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     mma_tf32(e, a, bb);
                 }
                 store_neg_d(Tm, LDM, q0 + 16, q0 + n0, e, g8, t4);
-                store_t_pair(sm + PO_TB, sm + PO_TBG, q0 + 16 + g8, q0 + n0 + 2 * t4, -e[0], -e[1], bet, gam);
-                store_t_pair(sm + PO_TB, sm + PO_TBG, q0 + 24 + g8, q0 + n0 + 2 * t4, -e[2], -e[3], bet, gam);
+                store_tb_tbg(sm + PO_TB, sm + PO_TBG, q0 + 16 + g8, q0 + n0 + 2 * t4, -e[0], -e[1], bet, bgm);
+                store_tb_tbg(sm + PO_TB, sm + PO_TBG, q0 + 24 + g8, q0 + n0 + 2 * t4, -e[2], -e[3], bet, bgm);
             }
             named_bar(kBarP, kNumPrep);
             SDBG(1, 4)
@@ -467,8 +553,8 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     load_b(bb, x2, LDX2, 8 * kk, 8 * ni, g8, t4);
                     mma_tf32(e, a, bb);
                 }
-                store_t_pair(sm + PO_TB, sm + PO_TBG, 32 + 16 * mi + g8, 8 * ni + 2 * t4, -e[0], -e[1], bet, gam);
-                store_t_pair(sm + PO_TB, sm + PO_TBG, 40 + 16 * mi + g8, 8 * ni + 2 * t4, -e[2], -e[3], bet, gam);
+                store_tb_tbg(sm + PO_TB, sm + PO_TBG, 32 + 16 * mi + g8, 8 * ni + 2 * t4, -e[0], -e[1], bet, bgm);
+                store_tb_tbg(sm + PO_TB, sm + PO_TBG, 40 + 16 * mi + g8, 8 * ni + 2 * t4, -e[2], -e[3], bet, bgm);
             }
             fence_proxy_async_smem();
             named_bar(kBarP, kNumPrep);
@@ -543,7 +629,7 @@ constexpr uint32_t ST_V = 32768;    // 16 KB
 constexpr uint32_t ST_W = 49152;    // 16 KB: W^T [128 i][64 t]
 constexpr uint32_t ST_P = 65536;    // 8 KB:  P [64 t][64 s]
 constexpr uint32_t ST_TB = 73728;   // 8 KB:  TB [64 t][64 s]
-constexpr uint32_t ST_GATE = 81920; // 512 B: gamma_t [64], dl_s [64]
+constexpr uint32_t ST_GATE = 81920; // 528 B: the chunk's gate record
 constexpr uint32_t ST_BYTES = 82944;
 constexpr uint32_t CO_OST = 2 * ST_BYTES;     // 16 KB output staging: two [64 t][64 d] boxes
 constexpr uint32_t CO_BARS = CO_OST + 16384;
@@ -586,7 +672,7 @@ static_assert(CB_COUNT * 8 <= CO_MISC - CO_BARS, "chain-kernel mbarriers overflo
 // ptab[i].x, head ptab[i].y, packed chunks ptab[i].z .. ptab[i].z + ptab[i].w - 1
 // of the chunk table ctab; its states are S0 / S_final [seq * H + head].
 struct ChainArgs {
-    const float *gate_rec;  // [items][128] from the prep kernel
+    const float *gate_rec;  // [items][kRecFloats] from the prep kernel
     const float *S0;
     float *S_final;
     int64_t T, H;
@@ -676,7 +762,7 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 tma_load_2d(st + ST_W, &tm_w, full, 0, row * 128);
                 tma_load_2d(st + ST_P, &tm_p, full, 0, row * 64);
                 tma_load_2d(st + ST_TB, &tm_tb, full, 0, row * 64);
-                bulk_load(st + ST_GATE, p.gate_rec + (int64_t)row * 128, (uint32_t)kGateRec, full);
+                bulk_load(st + ST_GATE, p.gate_rec + (int64_t)row * kRecFloats, (uint32_t)kGateRec, full);
             }
         }
         __syncwarp();
@@ -901,7 +987,7 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 w = w && wait_bar(&bars[CB_FULL0 + (c & 1)], sp, abort_flag);
                 if (!(ok = bar_and(kBarChn, kNumChn, w))) break;
             }
-            const float gC = reinterpret_cast<const float *>(sm + (c & 1) * ST_BYTES + ST_GATE)[63];
+            const float gC = reinterpret_cast<const float *>(sm + (c & 1) * ST_BYTES + ST_GATE)[128];
             tc_fence_after();
             SDBG(5, 1)
             // ---- bf16 operand copy of S (row j, 64 columns) ----
@@ -1051,7 +1137,7 @@ constexpr uint32_t TS_K = 0;         // 16 KB: two [64 t][64 d] boxes
 constexpr uint32_t TS_V = 16384;     // 16 KB
 constexpr uint32_t TS_W = 32768;     // 16 KB: W^T [128 i][64 t]
 constexpr uint32_t TS_TB = 49152;    // 8 KB:  TB [64 t][64 s]
-constexpr uint32_t TS_GATE = 57344;  // 512 B: gamma_t [64], dl_s [64]
+constexpr uint32_t TS_GATE = 57344;  // 528 B: the chunk's gate record
 constexpr uint32_t TS_BYTES = 58368;
 constexpr uint32_t TO_SB = 2 * TS_BYTES;        // 2 groups x 32 KB: bf16 S, two [128 j][64 i] boxes
 constexpr uint32_t TO_UB = TO_SB + 2 * 32768;   // 2 groups x 16 KB: bf16 U^T, [128 j][64 t]
@@ -1134,7 +1220,7 @@ fwd_transfer_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 }
                 tma_load_2d(st + TS_W, &tm_w, full, 0, row * 128);
                 tma_load_2d(st + TS_TB, &tm_tb, full, 0, row * 64);
-                bulk_load(st + TS_GATE, p.gate_rec + (int64_t)row * 128, (uint32_t)kGateRec, full);
+                bulk_load(st + TS_GATE, p.gate_rec + (int64_t)row * kRecFloats, (uint32_t)kGateRec, full);
             }
         }
         __syncwarp();
@@ -1218,7 +1304,7 @@ fwd_transfer_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 w = w && wait_bar(&bars[TB_FULL0 + s], sp, abort_flag);
                 if (!(ok = bar_and(barg, kTrNumGrp, w))) break;
             }
-            const float gC = reinterpret_cast<const float *>(sm + s * TS_BYTES + TS_GATE)[63];
+            const float gC = reinterpret_cast<const float *>(sm + s * TS_BYTES + TS_GATE)[128];
             tc_fence_after();
             // ---- bf16 copy of S into shared memory (row j, 64 columns = one 128-byte row of a box) ----
 #pragma unroll 1
@@ -1404,6 +1490,7 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
     pa.items = items;
     pa.chunks = (int)chunks;
     pa.ctab = nullptr;
+    pa.raw_inputs = p.raw_inputs;
     const int64_t pgrid =
         items < kPrepCtasPerSm * (int64_t)sm_count ? items : kPrepCtasPerSm * (int64_t)sm_count;
     {
@@ -1515,6 +1602,7 @@ cudaError_t launch_fwd_split_packed(const FwdProblem &p, const int64_t *cu_seqle
         pa.items = items;
         pa.chunks = 0;
         pa.ctab = d_ctab;
+        pa.raw_inputs = p.raw_inputs;
         const int64_t pgrid =
             items < kPrepCtasPerSm * (int64_t)sm_count ? items : kPrepCtasPerSm * (int64_t)sm_count;
         TimedLaunch tl_(GDN_KERNEL_PREP, stream);

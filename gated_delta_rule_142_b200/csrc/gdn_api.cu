@@ -180,6 +180,43 @@ FwdPath forced_path() {
     return FwdPath::Auto;
 }
 
+int64_t round256(int64_t x) { return (x + 255) & ~int64_t(255); }
+
+// For the forwards that read normalised inputs: runs the input stage over the `rows` (token,
+// head) rows of p into scratch taken on `stream` and points p at the results.  *scratch
+// receives the allocation (released by the caller once the forward is enqueued).
+int stage_inputs(FwdProblem &p, int64_t rows, void **scratch, cudaStream_t stream) {
+    const int64_t es = (p.dtype == GDN_F32) ? 4 : 2;
+    const int64_t nqk = round256(rows * p.dk * es), ng = round256(rows * 4);
+    if (scratch_alloc(scratch, (size_t)(2 * nqk + 2 * ng), stream) != cudaSuccess) {
+        cudaGetLastError();
+        *scratch = nullptr;
+        return GDN_ERR_ALLOC;
+    }
+    uint8_t *base = static_cast<uint8_t *>(*scratch);
+    float *la = reinterpret_cast<float *>(base + 2 * nqk), *be = reinterpret_cast<float *>(base + 2 * nqk + ng);
+    if (gdn::launch_input_stage(p.q, p.k, p.log_alpha, p.beta, base, base + nqk, la, be, rows, p.dk, p.dtype,
+                                stream) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_LAUNCH;
+    }
+    p.q = base;
+    p.k = base + nqk;
+    p.log_alpha = la;
+    p.beta = be;
+    p.raw_inputs = 0;
+    return GDN_OK;
+}
+
+int forward_impl(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                 const float *S0, void *out, float *S_final, int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
+                 int64_t chunk, void *stream_, int dtype, bool raw);
+int varlen_impl(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                const int64_t *cu_seqlens, int64_t N, const float *S0, void *out, float *S_final, int64_t T_total,
+                int64_t H, int64_t dk, int64_t dv, int64_t chunk, void *stream_, int dtype, bool raw);
+int decode_impl(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta, float *S,
+                void *out, int64_t B, int64_t H, int64_t dk, int64_t dv, void *stream_, int dtype, bool raw);
+
 }  // namespace
 
 extern "C" {
@@ -219,7 +256,48 @@ int gdn_version(void) { return 100; }  // 0.1.0
 
 int gdn_forward(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                 const float *S0, void *out, float *S_final, int64_t B, int64_t T, int64_t H, int64_t dk,
-                int64_t dv, int64_t chunk, void *stream_, int dtype) {
+                int64_t dv, int64_t chunk, void *stream, int dtype) {
+    return forward_impl(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv, chunk, stream, dtype, false);
+}
+
+int gdn_forward_raw(const void *q, const void *k, const void *v, const float *x_alpha, const float *x_beta,
+                    const float *S0, void *out, float *S_final, int64_t B, int64_t T, int64_t H, int64_t dk,
+                    int64_t dv, int64_t chunk, void *stream, int dtype) {
+    return forward_impl(q, k, v, x_alpha, x_beta, S0, out, S_final, B, T, H, dk, dv, chunk, stream, dtype, true);
+}
+
+int gdn_forward_varlen(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                       const int64_t *cu_seqlens, int64_t N, const float *S0, void *out, float *S_final,
+                       int64_t T_total, int64_t H, int64_t dk, int64_t dv, int64_t chunk, void *stream, int dtype) {
+    return varlen_impl(q, k, v, log_alpha, beta, cu_seqlens, N, S0, out, S_final, T_total, H, dk, dv, chunk, stream,
+                       dtype, false);
+}
+
+int gdn_forward_varlen_raw(const void *q, const void *k, const void *v, const float *x_alpha, const float *x_beta,
+                           const int64_t *cu_seqlens, int64_t N, const float *S0, void *out, float *S_final,
+                           int64_t T_total, int64_t H, int64_t dk, int64_t dv, int64_t chunk, void *stream,
+                           int dtype) {
+    return varlen_impl(q, k, v, x_alpha, x_beta, cu_seqlens, N, S0, out, S_final, T_total, H, dk, dv, chunk, stream,
+                       dtype, true);
+}
+
+int gdn_decode_step(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                    float *S, void *out, int64_t B, int64_t H, int64_t dk, int64_t dv, void *stream, int dtype) {
+    return decode_impl(q, k, v, log_alpha, beta, S, out, B, H, dk, dv, stream, dtype, false);
+}
+
+int gdn_decode_step_raw(const void *q, const void *k, const void *v, const float *x_alpha, const float *x_beta,
+                        float *S, void *out, int64_t B, int64_t H, int64_t dk, int64_t dv, void *stream, int dtype) {
+    return decode_impl(q, k, v, x_alpha, x_beta, S, out, B, H, dk, dv, stream, dtype, true);
+}
+
+}  // extern "C"
+
+namespace {
+
+int forward_impl(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                 const float *S0, void *out, float *S_final, int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
+                 int64_t chunk, void *stream_, int dtype, bool raw) {
     if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
     if (B < 0 || T < 0 || H < 0 || dk < 0 || dv < 0 || chunk < 0) return GDN_ERR_INVALID_SIZE;
     if (!supported_dim(dk) || !supported_dim(dv) || !supported_chunk(chunk)) return GDN_ERR_UNSUPPORTED;
@@ -280,6 +358,7 @@ int gdn_forward(const void *q, const void *k, const void *v, const float *log_al
             const int nseg = gdn::fwd_tc_segments(p, info.sm_count, true);
             void *ws = nullptr;
             if (scratch_alloc(&ws, gdn::fwd_split_workspace_bytes(p, nseg), stream) == cudaSuccess) {
+                p.raw_inputs = raw ? 1 : 0;  // the prep kernel runs the input stage on its own loads
                 e = gdn::launch_fwd_split(p, nseg, info.sm_count, ws, stream);
                 cudaFreeAsync(ws, stream);
                 done = true;
@@ -288,12 +367,20 @@ int gdn_forward(const void *q, const void *k, const void *v, const float *log_al
                 cudaGetLastError();
             }
         }
+        void *staged = nullptr;
+        if (!done && raw) {
+            if ((st = stage_inputs(p, ntok, &staged, stream))) {
+                if (staged) cudaFreeAsync(staged, stream);
+                return st;
+            }
+        }
         if (!done && path != FwdPath::Simt && gdn::fwd_tc_supported(p)) {
             const int nseg = gdn::fwd_tc_segments(p, info.sm_count, false);
             const size_t ws_bytes = gdn::fwd_tc_workspace_bytes(p, nseg);
             void *ws = nullptr;
             if (ws_bytes > 0 && scratch_alloc(&ws, ws_bytes, stream) != cudaSuccess) {
                 cudaGetLastError();
+                if (staged) cudaFreeAsync(staged, stream);
                 return GDN_ERR_ALLOC;
             }
             e = gdn::launch_fwd_tc(p, nseg, ws, stream);
@@ -301,6 +388,7 @@ int gdn_forward(const void *q, const void *k, const void *v, const float *log_al
         } else if (!done) {
             e = gdn::launch_fwd_simt(p, info.sm_count, stream);
         }
+        if (staged) cudaFreeAsync(staged, stream);
     }
     if (e != cudaSuccess) {
         cudaGetLastError();
@@ -311,10 +399,9 @@ int gdn_forward(const void *q, const void *k, const void *v, const float *log_al
     return GDN_OK;
 }
 
-int gdn_forward_varlen(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
-                       const int64_t *cu_seqlens, int64_t N, const float *S0, void *out, float *S_final,
-                       int64_t T_total, int64_t H, int64_t dk, int64_t dv, int64_t chunk, void *stream_,
-                       int dtype) {
+int varlen_impl(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                const int64_t *cu_seqlens, int64_t N, const float *S0, void *out, float *S_final, int64_t T_total,
+                int64_t H, int64_t dk, int64_t dv, int64_t chunk, void *stream_, int dtype, bool raw) {
     if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
     if (N < 0 || T_total < 0 || H < 0 || dk < 0 || dv < 0 || chunk < 0) return GDN_ERR_INVALID_SIZE;
     if (!supported_dim(dk) || !supported_dim(dv) || !supported_chunk(chunk)) return GDN_ERR_UNSUPPORTED;
@@ -385,6 +472,7 @@ int gdn_forward_varlen(const void *q, const void *k, const void *v, const float 
         // every sequence at once on the two-kernel tensor-core forward
         void *ws = nullptr;
         if (scratch_alloc(&ws, gdn::fwd_split_packed_workspace_bytes(chunks, H, N), stream) == cudaSuccess) {
+            p.raw_inputs = raw ? 1 : 0;  // the prep kernel runs the input stage on its own loads
             e = gdn::launch_fwd_split_packed(p, cu_seqlens, N, info.sm_count, ws, stream);
             cudaFreeAsync(ws, stream);
             done = true;
@@ -394,6 +482,13 @@ int gdn_forward_varlen(const void *q, const void *k, const void *v, const float 
     }
     // otherwise one fixed-length launch per sequence: the single-kernel tensor-core forward (no
     // segments, so no scratch) or the CUDA-core forward
+    void *staged = nullptr;
+    if (!done && raw) {
+        if ((st = stage_inputs(p, ntok, &staged, stream))) {
+            if (staged) cudaFreeAsync(staged, stream);
+            return st;
+        }
+    }
     const int64_t state = H * dv * dk;
     for (int64_t i = 0; i < N && !done && e == cudaSuccess; ++i) {
         const int64_t t0 = cu_seqlens[i], len = cu_seqlens[i + 1] - t0;
@@ -417,6 +512,7 @@ int gdn_forward_varlen(const void *q, const void *k, const void *v, const float 
             e = gdn::launch_fwd_simt(pi, info.sm_count, stream);
         }
     }
+    if (staged) cudaFreeAsync(staged, stream);
     if (e != cudaSuccess) {
         cudaGetLastError();
         return GDN_ERR_LAUNCH;
@@ -425,6 +521,10 @@ int gdn_forward_varlen(const void *q, const void *k, const void *v, const float 
     if ((st = stg.out_back(S_final, p.S_final, nstate))) return st;
     return GDN_OK;
 }
+
+}  // namespace
+
+extern "C" {
 
 int gdn_forward_plan(int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv, int64_t chunk, int dtype,
                      int64_t *scratch_bytes, int *launches) {
@@ -459,8 +559,12 @@ int gdn_forward_plan(int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv, in
     return GDN_OK;
 }
 
-int gdn_decode_step(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
-                    float *S, void *out, int64_t B, int64_t H, int64_t dk, int64_t dv, void *stream_, int dtype) {
+}  // extern "C"
+
+namespace {
+
+int decode_impl(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta, float *S,
+                void *out, int64_t B, int64_t H, int64_t dk, int64_t dv, void *stream_, int dtype, bool raw) {
     if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
     if (B < 0 || H < 0 || dk < 0 || dv < 0) return GDN_ERR_INVALID_SIZE;
     if (!supported_dim(dk) || !supported_dim(dv)) return GDN_ERR_UNSUPPORTED;
@@ -496,6 +600,7 @@ int gdn_decode_step(const void *q, const void *k, const void *v, const float *lo
     p.S = static_cast<float *>(const_cast<void *>(dS));
     p.out = const_cast<void *>(dout);
     p.B = B; p.H = H; p.dk = dk; p.dv = dv; p.dtype = dtype;
+    p.raw_inputs = raw ? 1 : 0;
     if (gdn::launch_decode(p, stream) != cudaSuccess) {
         cudaGetLastError();
         return GDN_ERR_LAUNCH;
@@ -505,4 +610,4 @@ int gdn_decode_step(const void *q, const void *k, const void *v, const float *lo
     return GDN_OK;
 }
 
-}  // extern "C"
+}  // namespace

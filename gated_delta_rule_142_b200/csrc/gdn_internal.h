@@ -35,6 +35,10 @@ struct FwdProblem {
     float *S_final;
     int64_t B, T, H, dk, dv, chunk;
     int dtype;  // gdn_dtype
+    // 1: q, k are not yet L2-normalised and log_alpha, beta hold the gate logits x_alpha,
+    // x_beta (log alpha = -softplus(x_alpha), beta = sigmoid(x_beta)); only the two-kernel
+    // forward takes this form, the others get the output of launch_input_stage()
+    int raw_inputs = 0;
 };
 
 struct DecodeProblem {
@@ -44,10 +48,21 @@ struct DecodeProblem {
     void *out;
     int64_t B, H, dk, dv;
     int dtype;
+    int raw_inputs = 0;  // as FwdProblem::raw_inputs
 };
+
+// Input stage epsilon: x / sqrt(sum x^2 + kNormEps), so that a zero vector stays zero.
+constexpr float kNormEps = 1e-12f;
 
 // decode.cu
 cudaError_t launch_decode(const DecodeProblem &p, cudaStream_t stream);
+
+// input_stage.cu -- the input stage as a pass of its own, for the forwards that do not fuse
+// it: L2-normalised q, k (dtype of the problem) and log alpha, beta from the gate logits, for
+// `rows` (token, head) rows of dk elements; outputs may not alias inputs.
+cudaError_t launch_input_stage(const void *q, const void *k, const float *x_alpha, const float *x_beta, void *qn,
+                               void *kn, float *log_alpha, float *beta, int64_t rows, int64_t dk, int dtype,
+                               cudaStream_t stream);
 
 // fwd_simt.cu -- float32 SIMT chunkwise forward, any supported (dk, dv, chunk).
 cudaError_t launch_fwd_simt(const FwdProblem &p, int sm_count, cudaStream_t stream);

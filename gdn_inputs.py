@@ -15,6 +15,12 @@ Draw order for a forward workload (one ``torch.Generator('cpu')`` seeded with
   * S0 ~ N(0, s0_std) (float32, standard deviation s0_std) or absent.
 The decode workload draws, per step in step order, q, k, v, x_beta, x_alpha
 the same way (stacked over steps), after the initial state S.
+
+Raw inputs (for the entry points that run the input stage themselves) draw
+q, k, v, x_beta, x_alpha, a row scale for q and one for k, then S0:
+  * q, k ~ N(0, 1) times a per-row scale log-uniform in [1/20, 20], with a
+    fraction ``zero_rows`` of the rows set to zero; cast to the dtype;
+  * v ~ N(0, 1); x_beta ~ N(0, 2); x_alpha ~ N(alpha_mu, 2) (float32 logits).
 """
 from __future__ import annotations
 
@@ -124,6 +130,31 @@ def varlen_inputs(lengths, H: int, dk: int, dv: int, dtype: str = "bf16", seed: 
         cu.append(cu[-1] + n)
     out["cu_seqlens"] = cu
     return out
+
+
+def raw_inputs(shape, dk: int, dv: int, dtype: str = "bf16", seed: int = 0, s0_shape=None,
+               s0_std: Optional[float] = None, alpha_mu: float = 0.0, zero_rows: float = 0.0) -> Dict[str, object]:
+    """CPU tensors for the raw-input entry points, `shape` the (token, head) grid ([B,T,H],
+    [T,H] or [B,H]): q, k [*shape, dk] and v [*shape, dv] (dtype, q and k not normalised),
+    x_alpha, x_beta [*shape] float32 gate logits, S0 of `s0_shape` (N(0, s0_std)) or None."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    td = torch_dtype(dtype)
+    shape = tuple(int(x) for x in shape)
+    q = torch.randn(shape + (dk,), generator=g, dtype=torch.float32)
+    k = torch.randn(shape + (dk,), generator=g, dtype=torch.float32)
+    v = torch.randn(shape + (dv,), generator=g, dtype=torch.float32).to(td)
+    x_beta = torch.randn(shape, generator=g, dtype=torch.float32) * 2.0
+    x_alpha = torch.randn(shape, generator=g, dtype=torch.float32) * 2.0 + alpha_mu
+    for x in (q, k):
+        u = torch.rand(shape + (1,), generator=g, dtype=torch.float32)
+        x.mul_(torch.exp((u * 2.0 - 1.0) * 2.9957323))  # 20 ** (2u - 1)
+        if zero_rows > 0:
+            x.mul_((torch.rand(shape + (1,), generator=g, dtype=torch.float32) >= zero_rows).to(torch.float32))
+    S0 = None
+    if s0_std is not None and s0_shape is not None:
+        S0 = torch.randn(tuple(s0_shape), generator=g, dtype=torch.float32) * s0_std
+    return {"q": q.to(td), "k": k.to(td), "v": v, "x_alpha": x_alpha, "x_beta": x_beta, "S0": S0}
 
 
 def length_mix(n: int, lo: int, hi: int, seed: int = 0):

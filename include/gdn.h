@@ -13,7 +13,8 @@
  *
  * No scale is applied to q, and q, k are used as given: callers that want
  * the paper's unit-norm keys and queries (its App. A.2 assumes
- * ||q_t|| = ||k_t|| = 1) normalise them before the call.
+ * ||q_t|| = ||k_t|| = 1) normalise them before the call, or call the *_raw
+ * entry points below, which normalise them (and map gate logits) in-kernel.
  *
  * Layouts (row-major, contiguous, 64-bit indexing):
  *     q, k            [B, T, H, dk]   dtype (GDN_F32 or GDN_BF16)
@@ -176,6 +177,43 @@ int gdn_decode_step(const void *q, const void *k, const void *v, const float *lo
                     int64_t dv, void *stream, int dtype);
 
 /*
+ * The input stage fused: gdn_forward_raw, gdn_forward_varlen_raw and
+ * gdn_decode_step_raw take the memory's inputs as the layer produces them
+ * and form what the recurrence reads inside the kernels.  The paper's memory
+ * reads unit-norm queries and keys (App. A.2 takes ||q_t|| = ||k_t|| = 1), a
+ * decay alpha_t in (0, 1) and a write strength beta_t in (0, 1); these calls
+ * compute, per (token, head),
+ *
+ *     q_t <- q_t / sqrt(|q_t|^2 + 1e-12),   k_t <- k_t / sqrt(|k_t|^2 + 1e-12)
+ *     log alpha_t = -softplus(x_alpha_t) = -log(1 + exp(x_alpha_t))
+ *     beta_t      = sigmoid(x_beta_t)    = 1 / (1 + exp(-x_beta_t))
+ *
+ * and then run the recurrence of gdn_forward / gdn_forward_varlen /
+ * gdn_decode_step on them (the 1e-12 keeps a zero vector at zero).  The
+ * normalised q, k are not rounded to dtype: the norms are applied in float32
+ * to the products that use q and k.
+ *
+ * Arguments, layouts, validation, aliasing and staging are those of the
+ * matching call, with x_alpha, x_beta (float32 gate logits, the layout of
+ * log_alpha, beta) in place of log_alpha, beta, and q, k in any scale.
+ * bf16 with dk = dv = 128 and chunk = 64 (and every decode step) runs the
+ * stage inside the kernels that already load q, k and the gates, with no pass
+ * of its own; other shapes run it as one extra pass (GDN_KERNEL_INPUT) into
+ * scratch before the forward.
+ */
+int gdn_forward_raw(const void *q, const void *k, const void *v, const float *x_alpha,
+                    const float *x_beta, const float *S0, void *out, float *S_final, int64_t B,
+                    int64_t T, int64_t H, int64_t dk, int64_t dv, int64_t chunk, void *stream,
+                    int dtype);
+int gdn_forward_varlen_raw(const void *q, const void *k, const void *v, const float *x_alpha,
+                           const float *x_beta, const int64_t *cu_seqlens, int64_t N,
+                           const float *S0, void *out, float *S_final, int64_t T_total, int64_t H,
+                           int64_t dk, int64_t dv, int64_t chunk, void *stream, int dtype);
+int gdn_decode_step_raw(const void *q, const void *k, const void *v, const float *x_alpha,
+                        const float *x_beta, float *S, void *out, int64_t B, int64_t H, int64_t dk,
+                        int64_t dv, void *stream, int dtype);
+
+/*
  * gdn_forward_noalloc -- gdn_forward for callers that cannot allocate device
  * memory during a call.
  *
@@ -244,7 +282,8 @@ typedef enum {
     GDN_KERNEL_FUSED = 4,       /* single-kernel tensor-core forward (outputs)                     */
     GDN_KERNEL_SIMT = 5,        /* float32 CUDA-core forward                                       */
     GDN_KERNEL_DECODE = 6,      /* single-token decode step                                        */
-    GDN_KERNEL_KINDS = 7
+    GDN_KERNEL_INPUT = 7,       /* input stage as a pass of its own (the *_raw forwards' fallbacks) */
+    GDN_KERNEL_KINDS = 8
 } gdn_kernel_kind;
 int gdn_timing_start(void);
 int gdn_timing_stop(double *ms, int64_t *launches);

@@ -68,13 +68,20 @@ class Oracle:
         L.gdn_oracle_decode_step.argtypes = [_ptr] * 7 + [_i64] * 4 + [ctypes.c_int]
         L.gdn_oracle_segment_transfer.argtypes = [_ptr] * 6 + [_i64] * 4
         L.gdn_oracle_dense_product.argtypes = [_ptr] * 8 + [_i64] * 3
+        L.gdn_oracle_input_stage.argtypes = [_ptr] * 8 + [_i64] * 2
+        L.gdn_oracle_forward_raw.argtypes = [_ptr] * 8 + [_i64] * 5 + [ctypes.c_int]
+        L.gdn_oracle_decode_step_raw.argtypes = [_ptr] * 7 + [_i64] * 4 + [ctypes.c_int]
         for f in ("gdn_oracle_forward", "gdn_oracle_forward_chunked", "gdn_oracle_decode_step",
-                  "gdn_oracle_segment_transfer", "gdn_oracle_dense_product"):
+                  "gdn_oracle_segment_transfer", "gdn_oracle_dense_product", "gdn_oracle_input_stage",
+                  "gdn_oracle_forward_raw", "gdn_oracle_decode_step_raw"):
             getattr(L, f).restype = ctypes.c_int
 
     # -- the definition: token-by-token recurrence ---------------------------------
-    def forward(self, q, k, v, log_alpha, beta, S0=None, nthreads: int = 0, want_out: bool = True):
-        """Sequential recurrence.  Returns (out [B,T,H,dv] float64 or None, S_final float64)."""
+    def forward(self, q, k, v, log_alpha, beta, S0=None, nthreads: int = 0, want_out: bool = True,
+                raw: bool = False):
+        """Sequential recurrence.  Returns (out [B,T,H,dv] float64 or None, S_final float64).
+        raw=True: q, k in any scale and log_alpha, beta holding the gate logits x_alpha, x_beta;
+        the input stage (see input_stage) runs first, in float64."""
         q, k, v, la, be = _f32(q), _f32(k), _f32(v), _f32(log_alpha), _f32(beta)
         B, T, H, dk = q.shape
         dv = v.shape[-1]
@@ -84,23 +91,38 @@ class Oracle:
             assert S0.shape == (B, H, dv, dk)
         out = np.empty((B, T, H, dv), np.float64) if want_out else None
         Sf = np.empty((B, H, dv, dk), np.float64)
-        rc = self.lib.gdn_oracle_forward(_p(q), _p(k), _p(v), _p(la), _p(be), _p(S0), _p(out), _p(Sf),
-                                         B, T, H, dk, dv, nthreads)
+        fn = self.lib.gdn_oracle_forward_raw if raw else self.lib.gdn_oracle_forward
+        rc = fn(_p(q), _p(k), _p(v), _p(la), _p(be), _p(S0), _p(out), _p(Sf), B, T, H, dk, dv, nthreads)
         if rc != 0:
             raise RuntimeError("gdn_oracle_forward failed (%d)" % rc)
         return out, Sf
 
-    def decode_step(self, q, k, v, log_alpha, beta, S, nthreads: int = 0):
+    def input_stage(self, q, k, x_alpha, x_beta):
+        """Unit-norm q, k (x / sqrt(|x|^2 + 1e-12) over the last axis), log alpha = -softplus(x_alpha),
+        beta = sigmoid(x_beta), all float64, shapes as given."""
+        q, k, xa, xb = _f32(q), _f32(k), _f32(x_alpha), _f32(x_beta)
+        d = q.shape[-1]
+        rows = q.size // d
+        assert k.shape == q.shape and xa.size == rows and xb.size == rows
+        qn, kn = np.empty(q.shape, np.float64), np.empty(k.shape, np.float64)
+        la, be = np.empty(xa.shape, np.float64), np.empty(xb.shape, np.float64)
+        rc = self.lib.gdn_oracle_input_stage(_p(q), _p(k), _p(xa), _p(xb), _p(qn), _p(kn), _p(la), _p(be), rows, d)
+        if rc != 0:
+            raise RuntimeError("gdn_oracle_input_stage failed (%d)" % rc)
+        return qn, kn, la, be
+
+    def decode_step(self, q, k, v, log_alpha, beta, S, nthreads: int = 0, raw: bool = False):
         """One token for every (b, h); S [B,H,dv,dk] float64 is updated in place.
-        q, k [B,H,dk]; v [B,H,dv]; gates [B,H].  Returns out [B,H,dv] float64."""
+        q, k [B,H,dk]; v [B,H,dv]; gates [B,H].  Returns out [B,H,dv] float64.
+        raw=True: the input stage first, as in forward()."""
         q, k, v, la, be = _f32(q), _f32(k), _f32(v), _f32(log_alpha), _f32(beta)
         B, H, dk = q.shape
         dv = v.shape[-1]
         assert S.dtype == np.float64 and S.flags.c_contiguous and S.shape == (B, H, dv, dk)
         assert k.shape == (B, H, dk) and v.shape == (B, H, dv) and la.shape == (B, H) and be.shape == (B, H)
         out = np.empty((B, H, dv), np.float64)
-        rc = self.lib.gdn_oracle_decode_step(_p(q), _p(k), _p(v), _p(la), _p(be), _p(S), _p(out),
-                                             B, H, dk, dv, nthreads)
+        fn = self.lib.gdn_oracle_decode_step_raw if raw else self.lib.gdn_oracle_decode_step
+        rc = fn(_p(q), _p(k), _p(v), _p(la), _p(be), _p(S), _p(out), B, H, dk, dv, nthreads)
         if rc != 0:
             raise RuntimeError("gdn_oracle_decode_step failed (%d)" % rc)
         return out
@@ -173,7 +195,25 @@ def decode_step(*args, **kw):
     return get().decode_step(*args, **kw)
 
 
-def forward_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, nthreads: int = 0):
+def input_stage(*args, **kw):
+    return get().input_stage(*args, **kw)
+
+
+def forward_raw(q, k, v, x_alpha, x_beta, S0=None, nthreads: int = 0):
+    """The input stage, then the recurrence (float64 throughout)."""
+    return get().forward(q, k, v, x_alpha, x_beta, S0, nthreads=nthreads, raw=True)
+
+
+def decode_step_raw(q, k, v, x_alpha, x_beta, S, nthreads: int = 0):
+    return get().decode_step(q, k, v, x_alpha, x_beta, S, nthreads=nthreads, raw=True)
+
+
+def forward_varlen_raw(q, k, v, x_alpha, x_beta, cu_seqlens, S0=None, nthreads: int = 0):
+    """forward_varlen with the input stage first."""
+    return forward_varlen(q, k, v, x_alpha, x_beta, cu_seqlens, S0, nthreads, raw=True)
+
+
+def forward_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, nthreads: int = 0, raw: bool = False):
     """Packed sequences: the recurrence run on each sequence i (tokens cu_seqlens[i] ..
     cu_seqlens[i+1]-1) from its own initial state S0[i] (zero when S0 is None), with no state
     passed from one sequence to the next.  q, k [T,H,dk], v [T,H,dv], gates [T,H],
@@ -193,7 +233,7 @@ def forward_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, nthreads: int 
                 Sf[i] = s0[0]
             continue
         oi, si = o.forward(q[None, a:b], k[None, a:b], v[None, a:b], log_alpha[None, a:b], beta[None, a:b], s0,
-                           nthreads=nthreads)
+                           nthreads=nthreads, raw=raw)
         out[a:b] = oi[0]
         Sf[i] = si[0]
     return out, Sf

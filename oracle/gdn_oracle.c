@@ -42,6 +42,9 @@
  *                               run of tokens, built chunk by chunk
  *   gdn_oracle_dense_product    brute force: explicit d_k x d_k factors
  *                               alpha_t (I - beta_t k_t k_t^T), tiny T only
+ *   gdn_oracle_input_stage      unit-norm q, k and the gate maps from logits
+ *   gdn_oracle_forward_raw,     the input stage followed by the recurrence
+ *   gdn_oracle_decode_step_raw
  */
 #include <math.h>
 #include <stdint.h>
@@ -444,4 +447,127 @@ int gdn_oracle_dense_product(const float *q, const float *k, const float *v,
     }
     free(F); free(P); free(tmp); free(St);
     return 0;
+}
+
+/* ------------------------------------------------------------------------
+ * The input stage.  The memory of Sec. 3.3 reads unit-norm queries and keys
+ * (App. A.2 takes ||q_t|| = ||k_t|| = 1), a decay alpha_t in (0, 1) and a write
+ * strength beta_t in (0, 1).  From raw projections q, k and gate logits
+ * x_alpha, x_beta this stage forms, in double,
+ *     q_t / sqrt(|q_t|^2 + eps),  k_t / sqrt(|k_t|^2 + eps)   (eps = 1e-12)
+ *     log alpha_t = -softplus(x_alpha) = -log(1 + exp(x_alpha))
+ *     beta_t      = sigmoid(x_beta)    = 1 / (1 + exp(-x_beta))
+ * The eps only keeps a zero vector at zero.  The *_raw functions run this
+ * stage and then the same recurrence as gdn_oracle_forward / _decode_step,
+ * on the double results (nothing is rounded back to float).
+ */
+#define GDN_ORACLE_NORM_EPS 1e-12
+
+static void unit_row(const float *x, double *y, int64_t d) {
+    double ss = 0.0;
+    for (int64_t i = 0; i < d; ++i) ss += (double)x[i] * (double)x[i];
+    const double inv = 1.0 / sqrt(ss + GDN_ORACLE_NORM_EPS);
+    for (int64_t i = 0; i < d; ++i) y[i] = (double)x[i] * inv;
+}
+
+static double neg_softplus(double x) { return -log1p(exp(x)); }
+static double sigmoid(double x) { return 1.0 / (1.0 + exp(-x)); }
+
+/* Input stage alone over `rows` (token, head) rows of d elements. */
+int gdn_oracle_input_stage(const float *q, const float *k, const float *x_alpha, const float *x_beta,
+                           double *qn, double *kn, double *log_alpha, double *beta, int64_t rows,
+                           int64_t d) {
+    if (rows < 0 || d < 1) return 1;
+    for (int64_t r = 0; r < rows; ++r) {
+        unit_row(q + r * d, qn + r * d, d);
+        unit_row(k + r * d, kn + r * d, d);
+        log_alpha[r] = neg_softplus((double)x_alpha[r]);
+        beta[r] = sigmoid((double)x_beta[r]);
+    }
+    return 0;
+}
+
+/* One token of the Sec. 3.3 recurrence with double q, k and gates (the
+ * counterpart of recurrence_step above for the input stage's outputs). */
+static void recurrence_step_d(double *S, const double *q, const double *k, const float *v, double a,
+                              double bt, double *o, double *x, int64_t dk, int64_t dv) {
+    for (int64_t r = 0; r < dv; ++r) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < dk; ++c) acc += S[r * dk + c] * k[c];
+        x[r] = acc;
+    }
+    for (int64_t r = 0; r < dv; ++r)
+        for (int64_t c = 0; c < dk; ++c) {
+            const double sk = S[r * dk + c] - bt * x[r] * k[c];
+            S[r * dk + c] = a * sk + bt * (double)v[r] * k[c];
+        }
+    for (int64_t r = 0; r < dv; ++r) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < dk; ++c) acc += S[r * dk + c] * q[c];
+        o[r] = acc;
+    }
+}
+
+/* gdn_oracle_forward with the input stage first: q, k raw, x_alpha, x_beta the
+ * gate logits (layouts as gdn_oracle_forward). */
+int gdn_oracle_forward_raw(const float *q, const float *k, const float *v, const float *x_alpha,
+                           const float *x_beta, const double *S0, double *out, double *S_final,
+                           int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv, int nthreads) {
+    if (B < 0 || T < 0 || H < 0 || dk < 1 || dv < 1) return 1;
+    set_threads(nthreads);
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        const int64_t b = bh / H, h = bh % H;
+        double *S = (double *)malloc(sizeof(double) * dv * dk);
+        double *x = (double *)malloc(sizeof(double) * dv);
+        double *o = (double *)malloc(sizeof(double) * dv);
+        double *qk = (double *)malloc(sizeof(double) * 2 * dk);
+        if (!S || !x || !o || !qk) {
+            free(S); free(x); free(o); free(qk);
+#pragma omp atomic write
+            failed = 1;
+            continue;
+        }
+        if (S0) memcpy(S, S0 + IDX_STATE(b, h, H, dv, dk), sizeof(double) * dv * dk);
+        else memset(S, 0, sizeof(double) * dv * dk);
+        for (int64_t t = 0; t < T; ++t) {
+            const int64_t gi = IDX_GATE(b, t, h, T, H);
+            unit_row(q + IDX_TOK(b, t, h, 0, T, H, dk), qk, dk);
+            unit_row(k + IDX_TOK(b, t, h, 0, T, H, dk), qk + dk, dk);
+            recurrence_step_d(S, qk, qk + dk, v + IDX_TOK(b, t, h, 0, T, H, dv),
+                              exp(neg_softplus((double)x_alpha[gi])), sigmoid((double)x_beta[gi]), o, x, dk,
+                              dv);
+            if (out) memcpy(out + IDX_TOK(b, t, h, 0, T, H, dv), o, sizeof(double) * dv);
+        }
+        if (S_final) memcpy(S_final + IDX_STATE(b, h, H, dv, dk), S, sizeof(double) * dv * dk);
+        free(S); free(x); free(o); free(qk);
+    }
+    return failed ? 2 : 0;
+}
+
+/* gdn_oracle_decode_step with the input stage first. */
+int gdn_oracle_decode_step_raw(const float *q, const float *k, const float *v, const float *x_alpha,
+                               const float *x_beta, double *S, double *out, int64_t B, int64_t H,
+                               int64_t dk, int64_t dv, int nthreads) {
+    if (B < 0 || H < 0 || dk < 1 || dv < 1) return 1;
+    set_threads(nthreads);
+    int failed = 0;
+#pragma omp parallel for schedule(static)
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        double *x = (double *)malloc(sizeof(double) * dv);
+        double *qk = (double *)malloc(sizeof(double) * 2 * dk);
+        if (!x || !qk) {
+            free(x); free(qk);
+#pragma omp atomic write
+            failed = 1;
+            continue;
+        }
+        unit_row(q + bh * dk, qk, dk);
+        unit_row(k + bh * dk, qk + dk, dk);
+        recurrence_step_d(S + bh * dv * dk, qk, qk + dk, v + bh * dv, exp(neg_softplus((double)x_alpha[bh])),
+                          sigmoid((double)x_beta[bh]), out + bh * dv, x, dk, dv);
+        free(x); free(qk);
+    }
+    return failed ? 2 : 0;
 }

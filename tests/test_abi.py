@@ -134,6 +134,38 @@ def test_decode_rejects_bad_arguments(lib):
     assert dec(lib, B=0) == OK
 
 
+def test_raw_entry_points_validate_like_the_plain_ones(lib):
+    """gdn_forward_raw, gdn_forward_varlen_raw and gdn_decode_step_raw take the same arguments (gate
+    logits in place of the gates) and reject the same calls with the same status."""
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    vp, i64 = ctypes.c_void_p, ctypes.c_int64
+    lib.gdn_forward_raw.argtypes = [vp] * 8 + [i64] * 6 + [vp, ctypes.c_int]
+    lib.gdn_decode_step_raw.argtypes = [vp] * 7 + [i64] * 4 + [vp, ctypes.c_int]
+    lib.gdn_forward_varlen_raw.argtypes = [vp] * 5 + [ctypes.POINTER(i64), i64] + [vp] * 3 + [i64] * 5 + \
+        [vp, ctypes.c_int]
+    cases = [dict(dtype=7), dict(B=-1), dict(dk=48), dict(q=None), dict(q=A + 8), dict(la=A + 0x3000002),
+             dict(out=A + 0x2000000), dict(Sf=A + 0x1000000), dict(B=0)]
+    for kw in cases:
+        a = dict(q=A, k=A + 0x1000000, v=A + 0x2000000, la=A + 0x3000000, be=A + 0x4000000, S0=None,
+                 out=A + 0x5000000, Sf=None, B=1, T=8, H=2, dk=16, dv=16, chunk=16, dtype=0)
+        a.update(kw)
+        raw = lib.gdn_forward_raw(P(a["q"]), P(a["k"]), P(a["v"]), P(a["la"]), P(a["be"]), P(a["S0"]), P(a["out"]),
+                                  P(a["Sf"]), a["B"], a["T"], a["H"], a["dk"], a["dv"], a["chunk"], None, a["dtype"])
+        assert raw == fwd(lib, **a) and raw != OK or kw == dict(B=0), kw
+    for kw in (dict(dk=8), dict(S=None), dict(out=A + 0x6000000), dict(B=0)):
+        a = dict(q=A, k=A + 0x1000000, v=A + 0x2000000, la=A + 0x3000000, be=A + 0x4000000, S=A + 0x6000000,
+                 out=A + 0x5000000, B=2, H=2, dk=16, dv=16, dtype=1)
+        a.update(kw)
+        raw = lib.gdn_decode_step_raw(P(a["q"]), P(a["k"]), P(a["v"]), P(a["la"]), P(a["be"]), P(a["S"]),
+                                      P(a["out"]), a["B"], a["H"], a["dk"], a["dv"], None, a["dtype"])
+        assert raw == dec(lib, **a), kw
+    for cu in ((1, 3, 8), (0, 5, 3), (0, 3, 7)):
+        arr = (ctypes.c_int64 * 3)(*cu)
+        assert lib.gdn_forward_varlen_raw(P(A), P(A + 0x1000000), P(A + 0x2000000), P(A + 0x3000000),
+                                          P(A + 0x4000000), arr, 2, None, P(A + 0x5000000), None, 8, 2, 16, 16, 16,
+                                          None, 0) == SIZE
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
 def test_valid_call_without_device_reports_device_error(lib):
     # S0 == S_final (in place) is allowed; with no CUDA device the call stops at the device check.

@@ -12,6 +12,7 @@ import pytest
 
 import oracle as oracle_pkg
 from test_oracle import PINS
+from test_oracle_input_stage import RAW_PINS
 
 
 def _swap_output_before_update(src: str) -> str:
@@ -54,6 +55,20 @@ MUTANTS = {
     "chunk_inverse_sign": ("x -= A[t * n + s] * Tinv[s * n + j];", "x += A[t * n + s] * Tinv[s * n + j];"),
     "chunk_inter_without_gamma": ("o[t * dv + r] = gamma[t] * inter + intra;", "o[t * dv + r] = inter + intra;"),
     "dense_factor_sign": ("a * (((i == j) ? 1.0 : 0.0) - bt *", "a * (((i == j) ? 1.0 : 0.0) + bt *"),
+    "norm_without_sqrt": ("const double inv = 1.0 / sqrt(ss + GDN_ORACLE_NORM_EPS);",
+                          "const double inv = 1.0 / (ss + GDN_ORACLE_NORM_EPS);"),
+    "norm_without_eps": ("const double inv = 1.0 / sqrt(ss + GDN_ORACLE_NORM_EPS);",
+                         "const double inv = 1.0 / sqrt(ss);"),
+    "softplus_sign": ("return -log1p(exp(x));", "return -log1p(exp(-x));"),
+    "softplus_drops_one": ("return -log1p(exp(x));", "return -log(exp(x));"),
+    "sigmoid_sign": ("return 1.0 / (1.0 + exp(-x));", "return 1.0 / (1.0 + exp(x));"),
+    "raw_gate_not_exponentiated": ("exp(neg_softplus((double)x_alpha[gi]))", "(1.0 + neg_softplus((double)x_alpha[gi]))"),
+    "raw_prediction_uses_q": ("for (int64_t c = 0; c < dk; ++c) acc += S[r * dk + c] * k[c];",
+                              "for (int64_t c = 0; c < dk; ++c) acc += S[r * dk + c] * q[c];"),
+    "raw_write_without_beta": ("S[r * dk + c] = a * sk + bt * (double)v[r] * k[c];",
+                               "S[r * dk + c] = a * sk + (double)v[r] * k[c];"),
+    "raw_decode_swaps_q_k": ("unit_row(q + bh * dk, qk, dk);\n        unit_row(k + bh * dk, qk + dk, dk);",
+                             "unit_row(k + bh * dk, qk, dk);\n        unit_row(q + bh * dk, qk + dk, dk);"),
 }
 
 
@@ -74,7 +89,7 @@ def test_planted_mistake_is_caught(tmp_path, name):
     lib = oracle_pkg.build(src=c_path, out=os.path.join(str(tmp_path), "libmutant.so"), force=True)
     mutant = oracle_pkg.Oracle(lib)
     caught = []
-    for pin in PINS:
+    for pin in PINS + RAW_PINS:
         try:
             pin(mutant)
         except (AssertionError, RuntimeError, FloatingPointError, ValueError):

@@ -133,3 +133,20 @@ def test_steps_replayed_from_a_cuda_graph():
     torch.cuda.synchronize()
     assert rel_err(cpu_f64(outs).reshape(steps, B * H, d), ref_o) <= TOL["bf16"]
     assert rel_err(cpu_f64(S).reshape(B * H, d, d), ref_S) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("B", [128, 512])
+def test_serving_batch(B):
+    """Decode at serving batch sizes (128 to 512 sequences), bf16, d = 128; every head checked at
+    B = 128, a sample of heads at B = 512."""
+    steps, H, d = 3, 4, 128
+    inp = decode_inputs(steps, B, H, d, d, "bf16", seed=61 + B, s0_std=0.05)
+    outs, S = run_steps(inp, steps)
+    heads = None if B == 128 else list(range(0, B * H, 37))
+    ref_o, ref_S = oracle_steps(inp, steps, heads=heads)
+    o = cpu_f64(outs).reshape(steps, B * H, d)
+    Sn = cpu_f64(S).reshape(B * H, d, d)
+    if heads is not None:
+        o, Sn = o[:, heads], Sn[heads]
+    assert rel_err(o, ref_o.reshape(o.shape)) <= TOL["bf16"]
+    assert rel_err(Sn, ref_S.reshape(Sn.shape)) <= TOL["bf16"]

@@ -206,7 +206,7 @@ def test_forward_plan_reports_scratch_and_launches(monkeypatch):
     """The planning query agrees with what the forward does.  Two-kernel path: 32.5 KB of workspace
     per chunk and two launches, plus segment scratch and two more launches for a long sequence
     with few heads.  Single-kernel path: no scratch and one launch, or segment scratch and three."""
-    per_chunk, seg_unit = 32768 + 512, 3 * 16 * 128 * 128 * 4
+    per_chunk, seg_unit = 32768 + 528, 3 * 16 * 128 * 128 * 4
     s, n = gdn.forward_plan(8, 2048, 16, 128, 128, 64)
     assert (s, n) == (8 * 16 * 32 * per_chunk, 2)
     s, n = gdn.forward_plan(1, 65536, 16, 128, 128, 64)
