@@ -45,6 +45,7 @@
  *   gdn_oracle_input_stage      unit-norm q, k and the gate maps from logits
  *   gdn_oracle_forward_raw,     the input stage followed by the recurrence
  *   gdn_oracle_decode_step_raw
+ *   gdn_oracle_backward         reverse mode of the recurrence, token by token
  */
 #include <math.h>
 #include <stdint.h>
@@ -568,6 +569,112 @@ int gdn_oracle_decode_step_raw(const float *q, const float *k, const float *v, c
         recurrence_step_d(S + bh * dv * dk, qk, qk + dk, v + bh * dv, exp(neg_softplus((double)x_alpha[bh])),
                           sigmoid((double)x_beta[bh]), out + bh * dv, x, dk, dv);
         free(x); free(qk);
+    }
+    return failed ? 2 : 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Backward (reverse mode) of the Sec. 3.3 recurrence, token by token.
+ *
+ * Given dL/do_t (d_out) and dL/dS_T (dS_final, NULL = 0) for the loss L of
+ * the forward outputs, the adjoint G_t = dL/dS_t runs backwards:
+ *     G_T = dS_final;   for t = T .. 1:
+ *       G_t   += do_t q_t^T                       (o_t = S_t q_t)
+ *       dq_t   = S_t^T do_t
+ *       with x = S_{t-1} k_t and Gk = G_t k_t, from
+ *       S_t = alpha_t S_{t-1} - alpha_t beta_t x k_t^T + beta_t v_t k_t^T:
+ *       dv_t         = beta_t Gk
+ *       dbeta_t      = (v_t - alpha_t x) . Gk
+ *       dlog_alpha_t = alpha_t (<G_t, S_{t-1}> - beta_t x . Gk)
+ *       dk_t         = -alpha_t beta_t (S_{t-1}^T Gk + G_t^T x) + beta_t G_t^T v_t
+ *       G_{t-1}      = alpha_t G_t (I - beta_t k_t k_t^T)
+ *     dS0 = G_0.
+ * The forward states S_0 .. S_T are recomputed and kept (T + 1 states per
+ * (b, h)), so this is for test sizes only.  All outputs are double.
+ */
+int gdn_oracle_backward(const float *q, const float *k, const float *v, const float *log_alpha,
+                        const float *beta, const double *S0, const double *d_out,
+                        const double *dS_final, double *dq, double *dk_out, double *dv_out,
+                        double *dlog_alpha, double *dbeta, double *dS0, int64_t B, int64_t T,
+                        int64_t H, int64_t dk, int64_t dv, int nthreads) {
+    if (B < 0 || T < 0 || H < 0 || dk < 1 || dv < 1) return 1;
+    set_threads(nthreads);
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        const int64_t b = bh / H, h = bh % H;
+        const int64_t ns = dv * dk;
+        double *St = (double *)malloc(sizeof(double) * ns * (T + 1));
+        double *G = (double *)malloc(sizeof(double) * ns);
+        double *x = (double *)malloc(sizeof(double) * dv);
+        double *Gk = (double *)malloc(sizeof(double) * dv);
+        double *o = (double *)malloc(sizeof(double) * dv);
+        if (!St || !G || !x || !Gk || !o) {
+            free(St); free(G); free(x); free(Gk); free(o);
+#pragma omp atomic write
+            failed = 1;
+            continue;
+        }
+        /* forward, keeping every state */
+        if (S0) memcpy(St, S0 + IDX_STATE(b, h, H, dv, dk), sizeof(double) * ns);
+        else memset(St, 0, sizeof(double) * ns);
+        for (int64_t t = 0; t < T; ++t) {
+            memcpy(St + (t + 1) * ns, St + t * ns, sizeof(double) * ns);
+            recurrence_step(St + (t + 1) * ns, q + IDX_TOK(b, t, h, 0, T, H, dk), k + IDX_TOK(b, t, h, 0, T, H, dk),
+                            v + IDX_TOK(b, t, h, 0, T, H, dv), log_alpha[IDX_GATE(b, t, h, T, H)],
+                            beta[IDX_GATE(b, t, h, T, H)], o, x, dk, dv);
+        }
+        /* reverse sweep */
+        if (dS_final) memcpy(G, dS_final + IDX_STATE(b, h, H, dv, dk), sizeof(double) * ns);
+        else memset(G, 0, sizeof(double) * ns);
+        for (int64_t t = T - 1; t >= 0; --t) {
+            const float *qt = q + IDX_TOK(b, t, h, 0, T, H, dk), *kt = k + IDX_TOK(b, t, h, 0, T, H, dk);
+            const float *vt = v + IDX_TOK(b, t, h, 0, T, H, dv);
+            const double *dot = d_out + IDX_TOK(b, t, h, 0, T, H, dv);
+            const double *Sn = St + (t + 1) * ns, *Sp = St + t * ns;   /* S_t and S_{t-1} */
+            const int64_t gi = IDX_GATE(b, t, h, T, H);
+            const double a = exp((double)log_alpha[gi]), bt = (double)beta[gi];
+            for (int64_t r = 0; r < dv; ++r)
+                for (int64_t c = 0; c < dk; ++c) G[r * dk + c] += dot[r] * (double)qt[c];
+            double *dqt = dq + IDX_TOK(b, t, h, 0, T, H, dk);
+            for (int64_t c = 0; c < dk; ++c) {
+                double acc = 0.0;
+                for (int64_t r = 0; r < dv; ++r) acc += Sn[r * dk + c] * dot[r];
+                dqt[c] = acc;
+            }
+            double gs = 0.0, xgk = 0.0, vgk = 0.0;
+            for (int64_t r = 0; r < dv; ++r) {
+                double ax = 0.0, ag = 0.0;
+                for (int64_t c = 0; c < dk; ++c) {
+                    ax += Sp[r * dk + c] * (double)kt[c];
+                    ag += G[r * dk + c] * (double)kt[c];
+                    gs += G[r * dk + c] * Sp[r * dk + c];
+                }
+                x[r] = ax;
+                Gk[r] = ag;
+                xgk += ax * ag;
+                vgk += (double)vt[r] * ag;
+            }
+            double *dvt = dv_out + IDX_TOK(b, t, h, 0, T, H, dv);
+            for (int64_t r = 0; r < dv; ++r) dvt[r] = bt * Gk[r];
+            dbeta[gi] = vgk - a * xgk;
+            dlog_alpha[gi] = a * (gs - bt * xgk);
+            double *dkt = dk_out + IDX_TOK(b, t, h, 0, T, H, dk);
+            for (int64_t c = 0; c < dk; ++c) {
+                double sgk = 0.0, gx = 0.0, gv = 0.0;
+                for (int64_t r = 0; r < dv; ++r) {
+                    sgk += Sp[r * dk + c] * Gk[r];
+                    gx += G[r * dk + c] * x[r];
+                    gv += G[r * dk + c] * (double)vt[r];
+                }
+                dkt[c] = -a * bt * (sgk + gx) + bt * gv;
+            }
+            for (int64_t r = 0; r < dv; ++r)
+                for (int64_t c = 0; c < dk; ++c)
+                    G[r * dk + c] = a * (G[r * dk + c] - bt * Gk[r] * (double)kt[c]);
+        }
+        if (dS0) memcpy(dS0 + IDX_STATE(b, h, H, dv, dk), G, sizeof(double) * ns);
+        free(St); free(G); free(x); free(Gk); free(o);
     }
     return failed ? 2 : 0;
 }

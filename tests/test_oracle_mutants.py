@@ -12,6 +12,7 @@ import pytest
 
 import oracle as oracle_pkg
 from test_oracle import PINS
+from test_oracle_backward import BWD_PINS
 from test_oracle_input_stage import RAW_PINS
 
 
@@ -67,6 +68,15 @@ MUTANTS = {
                               "for (int64_t c = 0; c < dk; ++c) acc += S[r * dk + c] * q[c];"),
     "raw_write_without_beta": ("S[r * dk + c] = a * sk + bt * (double)v[r] * k[c];",
                                "S[r * dk + c] = a * sk + (double)v[r] * k[c];"),
+    "bwd_dk_sign": ("dkt[c] = -a * bt * (sgk + gx) + bt * gv;", "dkt[c] = a * bt * (sgk + gx) + bt * gv;"),
+    "bwd_dk_drops_transpose_term": ("dkt[c] = -a * bt * (sgk + gx) + bt * gv;", "dkt[c] = -a * bt * sgk + bt * gv;"),
+    "bwd_adjoint_without_alpha": ("G[r * dk + c] = a * (G[r * dk + c] - bt * Gk[r] * (double)kt[c]);",
+                                  "G[r * dk + c] = (G[r * dk + c] - bt * Gk[r] * (double)kt[c]);"),
+    "bwd_dbeta_sign": ("dbeta[gi] = vgk - a * xgk;", "dbeta[gi] = vgk + a * xgk;"),
+    "bwd_dlogalpha_without_alpha": ("dlog_alpha[gi] = a * (gs - bt * xgk);", "dlog_alpha[gi] = (gs - bt * xgk);"),
+    "bwd_dq_uses_previous_state": ("for (int64_t r = 0; r < dv; ++r) acc += Sn[r * dk + c] * dot[r];",
+                                   "for (int64_t r = 0; r < dv; ++r) acc += Sp[r * dk + c] * dot[r];"),
+    "bwd_output_grad_uses_k": ("G[r * dk + c] += dot[r] * (double)qt[c];", "G[r * dk + c] += dot[r] * (double)kt[c];"),
     "raw_decode_swaps_q_k": ("unit_row(q + bh * dk, qk, dk);\n        unit_row(k + bh * dk, qk + dk, dk);",
                              "unit_row(k + bh * dk, qk, dk);\n        unit_row(q + bh * dk, qk + dk, dk);"),
 }
@@ -89,7 +99,7 @@ def test_planted_mistake_is_caught(tmp_path, name):
     lib = oracle_pkg.build(src=c_path, out=os.path.join(str(tmp_path), "libmutant.so"), force=True)
     mutant = oracle_pkg.Oracle(lib)
     caught = []
-    for pin in PINS + RAW_PINS:
+    for pin in PINS + RAW_PINS + BWD_PINS:
         try:
             pin(mutant)
         except (AssertionError, RuntimeError, FloatingPointError, ValueError):
