@@ -37,10 +37,11 @@ STATUS = {
 
 EXPORTS = ("gdn_forward", "gdn_decode_step", "gdn_forward_plan", "gdn_status_string", "gdn_version",
            "gdn_forward_noalloc", "gdn_scratch_release", "gdn_timing_start", "gdn_timing_stop",
-           "gdn_forward_varlen", "gdn_forward_raw", "gdn_forward_varlen_raw", "gdn_decode_step_raw")
+           "gdn_forward_varlen", "gdn_forward_raw", "gdn_forward_varlen_raw", "gdn_decode_step_raw",
+           "gdn_backward")
 
 # gdn_kernel_kind names, in enum order
-KERNEL_KINDS = ("prep", "chain", "transfer", "prefix", "fused", "simt", "decode", "input")
+KERNEL_KINDS = ("prep", "chain", "transfer", "prefix", "fused", "simt", "decode", "input", "backward")
 
 
 class GdnError(RuntimeError):
@@ -77,6 +78,8 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     for fn in (lib.gdn_forward_varlen, lib.gdn_forward_varlen_raw):
         fn.argtypes = [vp] * 5 + [ctypes.POINTER(i64), i64] + [vp] * 3 + [i64] * 5 + [vp, ctypes.c_int]
         fn.restype = ctypes.c_int
+    lib.gdn_backward.argtypes = [vp] * 14 + [i64] * 6 + [vp, ctypes.c_int]
+    lib.gdn_backward.restype = ctypes.c_int
     lib.gdn_scratch_release.argtypes = []
     lib.gdn_scratch_release.restype = ctypes.c_int
     lib.gdn_timing_start.argtypes = []
@@ -231,6 +234,45 @@ def _forward_varlen(entry, q, k, v, log_alpha, beta, cu_seqlens, S0, chunk, out,
     if st != 0:
         raise GdnError(st, entry)
     return out, S_final
+
+
+def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor, beta: torch.Tensor,
+             S0: Optional[torch.Tensor], grad_out: torch.Tensor, grad_S_final: Optional[torch.Tensor] = None,
+             chunk: int = 64, want_grad_S0: bool = True, stream=None):
+    """Reverse mode of forward().  grad_out [B,T,H,dv] (dtype of q); grad_S_final [B,H,dv,dk] float32 or
+    None.  Returns (dq, dk, dv in the input dtype; dlog_alpha, dbeta [B,T,H] float32; dS0 or None)."""
+    lib = load()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for name, t, shape in (("k", k, (B, T, H, dk)), ("v", v, (B, T, H, dv)), ("log_alpha", log_alpha, (B, T, H)),
+                           ("beta", beta, (B, T, H)), ("grad_out", grad_out, (B, T, H, dv)),
+                           ("S0", S0, (B, H, dv, dk)), ("grad_S_final", grad_S_final, (B, H, dv, dk))):
+        if t is not None and tuple(t.shape) != shape:
+            raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), shape))
+    _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype or grad_out.dtype != q.dtype:
+        raise TypeError("q, k, v and grad_out must share one dtype")
+    for name, t in (("log_alpha", log_alpha), ("beta", beta), ("S0", S0), ("grad_S_final", grad_S_final)):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError("%s must be float32" % name)
+    for t in (q, k, v, log_alpha, beta, S0, grad_out, grad_S_final):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    pin = _pinned(q)
+    dq = torch.empty_like(q, pin_memory=pin) if q.device.type == "cpu" else torch.empty_like(q)
+    dk_ = torch.empty_like(k, pin_memory=pin) if k.device.type == "cpu" else torch.empty_like(k)
+    dv_ = torch.empty_like(v, pin_memory=pin) if v.device.type == "cpu" else torch.empty_like(v)
+    dla = torch.empty((B, T, H), dtype=torch.float32, device=q.device, pin_memory=pin)
+    dbe = torch.empty((B, T, H), dtype=torch.float32, device=q.device, pin_memory=pin)
+    dS0 = (torch.empty((B, H, dv, dk), dtype=torch.float32, device=q.device, pin_memory=pin)
+           if want_grad_S0 else None)
+    with torch.cuda.device(q.device if q.device.type == "cuda" else torch.cuda.current_device()):
+        st = lib.gdn_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(grad_out),
+                              _ptr(grad_S_final), _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dla), _ptr(dbe), _ptr(dS0),
+                              B, T, H, dk, dv, int(chunk), _stream_handle(q.device, stream), _dtype_code(q))
+    if st != 0:
+        raise GdnError(st, "gdn_backward")
+    return dq, dk_, dv_, dla, dbe, dS0
 
 
 def forward_plan(B: int, T: int, H: int, dk: int, dv: int, chunk: int = 64, dtype=torch.bfloat16):

@@ -22,6 +22,10 @@
 // one head run in parallel (each recomputes the slab-independent A and P).
 // Tail chunks are zero-padded with log_alpha = 0, beta = 0, which leaves the
 // recurrence unchanged.
+//
+// For the backward pass the same kernel recomputes the forward with outputs
+// off (out == nullptr) and writes the state at the start of every chunk to a
+// checkpoint array [B*H][chunks][dv][dk].
 #include <atomic>
 
 #include "common.cuh"
@@ -77,7 +81,7 @@ __global__ void __launch_bounds__(kThreads)
 fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
                 const float *__restrict__ log_alpha, const float *__restrict__ beta,
                 const float *__restrict__ S0, Tin *__restrict__ out, float *__restrict__ S_final,
-                int64_t T, int64_t H, SimtDims d) {
+                float *__restrict__ ckpt, int64_t T, int64_t H, SimtDims d) {
     extern __shared__ __align__(16) float sm[];
     const int dk = d.dk, dv = d.dv, C = d.C, rows = d.rows;
     const int LDK = d.ldk, LDR = d.ldr, LDC = d.ldc;
@@ -114,9 +118,19 @@ fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
     }
 
     const int tpc = kThreads / rows;  // threads per column in the substitution
+    const bool want_out = out != nullptr;
+    const int64_t nchunks = (T + C - 1) / C;
     for (int64_t t0 = 0; t0 < T; t0 += C) {
         const int n = (int)((T - t0 < C) ? (T - t0) : C);
         __syncthreads();  // previous chunk fully consumed
+        if (ckpt) {  // the state entering this chunk
+            float *dst = ckpt + ((bh * nchunks + t0 / C) * dv + r0) * (int64_t)dk;
+            for (int i = tid; i < rows * (dk / 4); i += kThreads) {
+                const int j = i / (dk / 4), c4 = i % (dk / 4);
+                *reinterpret_cast<float4 *>(dst + (int64_t)j * dk + 4 * c4) =
+                    *reinterpret_cast<const float4 *>(Ss + j * LDK + 4 * c4);
+            }
+        }
         // ---- load chunk (zero-padded tail) ----
         for (int i = tid; i < C * (dk / 4); i += kThreads) {
             const int t = i / (dk / 4), c4 = i % (dk / 4);
@@ -197,7 +211,7 @@ fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
         }
 
         // ---- P = mask_{s<=t}(Q K^T o e^{g_t-g_s}) ;  Xs <- diag(gamma) Q S^T ----
-        {
+        if (want_out) {
             const int nx = (C / 4) * (rows / 4), na = (C / 4) * (C / 4);
             for (int w = tid; w < nx + na; w += kThreads) {
                 float acc[4][4] = {};
@@ -226,7 +240,7 @@ fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
 
         // ---- O = Xs + P U  (to global) ;  S <- gamma_last S + U^T diag(dl) K ----
         {
-            const int no = (C / 4) * (rows / 4), ns = (rows / 4) * (dk / 4);
+            const int no = want_out ? (C / 4) * (rows / 4) : 0, ns = (rows / 4) * (dk / 4);
             const float gl = gam[C - 1];
             for (int w = tid; w < no + ns; w += kThreads) {
                 float acc[4][4] = {};
@@ -323,7 +337,7 @@ cudaError_t launch_t(const FwdProblem &p, int sm_count, cudaStream_t stream) {
         TimedLaunch tl_(GDN_KERNEL_SIMT, stream);
         fwd_simt_kernel<Tin><<<(unsigned)grid, kThreads, smem, stream>>>(
             static_cast<const Tin *>(p.q), static_cast<const Tin *>(p.k), static_cast<const Tin *>(p.v), p.log_alpha,
-            p.beta, p.S0, static_cast<Tin *>(p.out), p.S_final, p.T, p.H, d);
+            p.beta, p.S0, static_cast<Tin *>(p.out), p.S_final, p.ckpt, p.T, p.H, d);
     }
     return cudaGetLastError();
 }

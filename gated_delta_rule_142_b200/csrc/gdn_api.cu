@@ -133,7 +133,7 @@ bool is_device_pointer(const void *p) {
 // Stream-ordered device copies of host buffers, released on the same stream.
 struct Stager {
     cudaStream_t stream;
-    void *bufs[10];
+    void *bufs[16];
     int n = 0;
     explicit Stager(cudaStream_t s) : stream(s) {}
     ~Stager() {
@@ -611,3 +611,93 @@ int decode_impl(const void *q, const void *k, const void *v, const float *log_al
 }
 
 }  // namespace
+
+extern "C" int gdn_backward(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                            const float *S0, const void *grad_out, const float *grad_S_final, void *grad_q,
+                            void *grad_k, void *grad_v, float *grad_log_alpha, float *grad_beta, float *grad_S0,
+                            int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv, int64_t chunk, void *stream_,
+                            int dtype) {
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
+    if (B < 0 || T < 0 || H < 0 || dk < 0 || dv < 0 || chunk < 0) return GDN_ERR_INVALID_SIZE;
+    if (!supported_dim(dk) || !supported_dim(dv) || !supported_chunk(chunk)) return GDN_ERR_UNSUPPORTED;
+    const int64_t es = (dtype == GDN_F32) ? 4 : 2;
+    int64_t ntok, nqk, nv, nstate;
+    if (!mul3(B, T, H, &ntok) || !mul3(ntok, dk, es, &nqk) || !mul3(ntok, dv, es, &nv) ||
+        !mul3(B * H, dv, dk * 4, &nstate) || ntok > (INT64_MAX / 8))
+        return GDN_ERR_INVALID_SIZE;
+    if (B * H == 0) return GDN_OK;
+    if (ntok > 0 && (!q || !k || !v || !log_alpha || !beta || !grad_out || !grad_q || !grad_k || !grad_v ||
+                     !grad_log_alpha || !grad_beta))
+        return GDN_ERR_NULL_PTR;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(log_alpha) || !aligned4(beta) ||
+        !aligned16(S0) || !aligned16(grad_out) || !aligned16(grad_S_final) || !aligned16(grad_q) ||
+        !aligned16(grad_k) || !aligned16(grad_v) || !aligned4(grad_log_alpha) || !aligned4(grad_beta) ||
+        !aligned16(grad_S0))
+        return GDN_ERR_MISALIGNED;
+    const Span inputs[] = {Span(q, nqk), Span(k, nqk), Span(v, nv), Span(log_alpha, ntok * 4), Span(beta, ntok * 4),
+                           Span(S0, nstate), Span(grad_out, nv), Span(grad_S_final, nstate)};
+    const Span outputs[] = {Span(grad_q, nqk), Span(grad_k, nqk), Span(grad_v, nv), Span(grad_log_alpha, ntok * 4),
+                            Span(grad_beta, ntok * 4), Span(grad_S0, nstate)};
+    for (const Span &o : outputs) {
+        for (const Span &x : inputs)
+            if (overlaps(o, x)) return GDN_ERR_ALIAS;
+        for (const Span &x : outputs)
+            if (&x != &o && overlaps(o, x)) return GDN_ERR_ALIAS;
+    }
+
+    DeviceInfo info;
+    if (int st = device_info(&info)) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    Stager stg(stream);
+    gdn::BwdProblem p;
+    int st = GDN_OK;
+    const void *dS0in = nullptr, *dgo = nullptr, *dgSf = nullptr;
+    if ((st = stg.in(q, nqk, true, &p.f.q)) || (st = stg.in(k, nqk, true, &p.f.k)) ||
+        (st = stg.in(v, nv, true, &p.f.v)) ||
+        (st = stg.in(log_alpha, ntok * 4, true, reinterpret_cast<const void **>(&p.f.log_alpha))) ||
+        (st = stg.in(beta, ntok * 4, true, reinterpret_cast<const void **>(&p.f.beta))) ||
+        (st = stg.in(S0, nstate, true, &dS0in)) || (st = stg.in(grad_out, nv, true, &dgo)) ||
+        (st = stg.in(grad_S_final, nstate, true, &dgSf)))
+        return st;
+    p.f.S0 = static_cast<const float *>(dS0in);
+    p.d_out = dgo;
+    p.dS_final = static_cast<const float *>(dgSf);
+    const void *oq = nullptr, *ok = nullptr, *ov = nullptr, *ola = nullptr, *obe = nullptr, *oS0 = nullptr;
+    if ((st = stg.in(grad_q, nqk, false, &oq)) || (st = stg.in(grad_k, nqk, false, &ok)) ||
+        (st = stg.in(grad_v, nv, false, &ov)) || (st = stg.in(grad_log_alpha, ntok * 4, false, &ola)) ||
+        (st = stg.in(grad_beta, ntok * 4, false, &obe)) || (st = stg.in(grad_S0, nstate, false, &oS0)))
+        return st;
+    p.dq = const_cast<void *>(oq);
+    p.dk = const_cast<void *>(ok);
+    p.dv = const_cast<void *>(ov);
+    p.dlog_alpha = static_cast<float *>(const_cast<void *>(ola));
+    p.dbeta = static_cast<float *>(const_cast<void *>(obe));
+    p.dS0 = static_cast<float *>(const_cast<void *>(oS0));
+    p.f.out = nullptr;
+    p.f.S_final = nullptr;
+    p.f.B = B; p.f.T = T; p.f.H = H; p.f.dk = dk; p.f.dv = dv; p.f.chunk = chunk; p.f.dtype = dtype;
+
+    cudaError_t e = cudaSuccess;
+    if (T == 0) {  // nothing flows but dS_final -> dS0
+        if (p.dS0)
+            e = p.dS_final ? cudaMemcpyAsync(p.dS0, p.dS_final, (size_t)nstate, cudaMemcpyDeviceToDevice, stream)
+                           : cudaMemsetAsync(p.dS0, 0, (size_t)nstate, stream);
+    } else {
+        void *ws = nullptr;
+        if (scratch_alloc(&ws, gdn::bwd_simt_workspace_bytes(p), stream) != cudaSuccess) {
+            cudaGetLastError();
+            return GDN_ERR_ALLOC;
+        }
+        e = gdn::launch_bwd_simt(p, info.sm_count, ws, stream);
+        cudaFreeAsync(ws, stream);
+    }
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_LAUNCH;
+    }
+    if ((st = stg.out_back(grad_q, p.dq, nqk)) || (st = stg.out_back(grad_k, p.dk, nqk)) ||
+        (st = stg.out_back(grad_v, p.dv, nv)) || (st = stg.out_back(grad_log_alpha, p.dlog_alpha, ntok * 4)) ||
+        (st = stg.out_back(grad_beta, p.dbeta, ntok * 4)) || (st = stg.out_back(grad_S0, p.dS0, nstate)))
+        return st;
+    return GDN_OK;
+}

@@ -39,6 +39,9 @@ struct FwdProblem {
     // x_beta (log alpha = -softplus(x_alpha), beta = sigmoid(x_beta)); only the two-kernel
     // forward takes this form, the others get the output of launch_input_stage()
     int raw_inputs = 0;
+    // CUDA-core forward only: when set, the state entering every chunk is written here,
+    // [B*H][chunks][dv][dk] float32 (the backward's checkpoints); out may then be nullptr
+    float *ckpt = nullptr;
 };
 
 struct DecodeProblem {
@@ -66,6 +69,18 @@ cudaError_t launch_input_stage(const void *q, const void *k, const float *x_alph
 
 // fwd_simt.cu -- float32 SIMT chunkwise forward, any supported (dk, dv, chunk).
 cudaError_t launch_fwd_simt(const FwdProblem &p, int sm_count, cudaStream_t stream);
+
+// bwd_simt.cu -- reverse mode of the forward (float32 CUDA cores, any supported shape).
+struct BwdProblem {
+    FwdProblem f;             // inputs and sizes (f.out, f.S_final unused)
+    const void *d_out;        // [B, T, H, dv] dtype
+    const float *dS_final;    // [B, H, dv, dk] or nullptr (zero)
+    void *dq, *dk, *dv;       // [B, T, H, dk|dv] dtype
+    float *dlog_alpha, *dbeta;  // [B, T, H]
+    float *dS0;               // [B, H, dv, dk] or nullptr (not written)
+};
+size_t bwd_simt_workspace_bytes(const BwdProblem &p);
+cudaError_t launch_bwd_simt(const BwdProblem &p, int sm_count, void *workspace, cudaStream_t stream);
 
 // fwd_tc.cu -- tcgen05 chunkwise forward: bf16, dk = dv = 128, chunk = 64.
 // Long sequences with few (b, h) are cut into segments: a transfer pass, a

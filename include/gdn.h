@@ -214,6 +214,32 @@ int gdn_decode_step_raw(const void *q, const void *k, const void *v, const float
                         int64_t dv, void *stream, int dtype);
 
 /*
+ * gdn_backward -- reverse mode of gdn_forward (the training backward).
+ *
+ * For a loss L whose gradients with respect to the forward's outputs are
+ * grad_out = dL/dout [B, T, H, dv] (dtype) and grad_S_final = dL/dS_final
+ * [B, H, dv, dk] (float32, NULL = zero), writes dL/dq, dL/dk [B, T, H, dk]
+ * and dL/dv [B, T, H, dv] in dtype, dL/dlog_alpha and dL/dbeta [B, T, H]
+ * float32, and dL/dS0 [B, H, dv, dk] float32 (grad_S0 NULL = not written).
+ * q, k, v, log_alpha, beta, S0 (NULL = zero), B, T, H, dk, dv, chunk,
+ * stream and dtype are exactly the forward's arguments.  The recurrence is
+ * the one of gdn_forward (source: the Sec. 3.3 gated-delta memory equation);
+ * the gradient of log_alpha below the forward's floor of -40 is zero.
+ *
+ * The forward is recomputed (the state entering every chunk is kept in
+ * scratch, dv * dk * 4 bytes per chunk and head), then the chunks are walked
+ * backwards with the chunkwise adjoint, in float32 on the CUDA cores.
+ * Scratch also holds float32 accumulators of dq and dk for bf16.
+ * Alignment and staging as for gdn_forward; no output may overlap an input
+ * or another output (GDN_ERR_ALIAS).
+ */
+int gdn_backward(const void *q, const void *k, const void *v, const float *log_alpha,
+                 const float *beta, const float *S0, const void *grad_out,
+                 const float *grad_S_final, void *grad_q, void *grad_k, void *grad_v,
+                 float *grad_log_alpha, float *grad_beta, float *grad_S0, int64_t B, int64_t T,
+                 int64_t H, int64_t dk, int64_t dv, int64_t chunk, void *stream, int dtype);
+
+/*
  * gdn_forward_noalloc -- gdn_forward for callers that cannot allocate device
  * memory during a call.
  *
@@ -283,7 +309,8 @@ typedef enum {
     GDN_KERNEL_SIMT = 5,        /* float32 CUDA-core forward                                       */
     GDN_KERNEL_DECODE = 6,      /* single-token decode step                                        */
     GDN_KERNEL_INPUT = 7,       /* input stage as a pass of its own (the *_raw forwards' fallbacks) */
-    GDN_KERNEL_KINDS = 8
+    GDN_KERNEL_BACKWARD = 8,    /* backward pass (its forward recompute counts as SIMT)            */
+    GDN_KERNEL_KINDS = 9
 } gdn_kernel_kind;
 int gdn_timing_start(void);
 int gdn_timing_stop(double *ms, int64_t *launches);

@@ -166,6 +166,35 @@ def test_raw_entry_points_validate_like_the_plain_ones(lib):
                                           None, 0) == SIZE
 
 
+def bwd(lib, **kw):
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    vp, i64 = ctypes.c_void_p, ctypes.c_int64
+    lib.gdn_backward.argtypes = [vp] * 14 + [i64] * 6 + [vp, ctypes.c_int]
+    a = dict(q=A, k=A + 0x1000000, v=A + 0x2000000, la=A + 0x3000000, be=A + 0x4000000, S0=None,
+             go=A + 0x5000000, gSf=None, gq=A + 0x8000000, gk=A + 0x9000000, gv=A + 0xA000000,
+             gla=A + 0xB000000, gbe=A + 0xC000000, gS0=None, B=1, T=8, H=2, dk=16, dv=16, chunk=16, dtype=0)
+    a.update(kw)
+    return lib.gdn_backward(*[P(a[n]) for n in ("q", "k", "v", "la", "be", "S0", "go", "gSf", "gq", "gk", "gv",
+                                                 "gla", "gbe", "gS0")],
+                            a["B"], a["T"], a["H"], a["dk"], a["dv"], a["chunk"], None, a["dtype"])
+
+
+def test_backward_rejects_bad_arguments(lib):
+    assert bwd(lib, dtype=5) == UNSUP
+    assert bwd(lib, dk=24) == UNSUP
+    assert bwd(lib, chunk=128) == UNSUP
+    assert bwd(lib, T=-1) == SIZE
+    assert bwd(lib, go=None) == NULL
+    assert bwd(lib, gq=None) == NULL
+    assert bwd(lib, gbe=None) == NULL
+    assert bwd(lib, gk=A + 0x9000008) == MISAL
+    assert bwd(lib, gla=A + 0xB000002) == MISAL
+    assert bwd(lib, gq=A) == ALIAS                  # an output over an input
+    assert bwd(lib, gk=A + 0x8000000) == ALIAS      # two outputs over each other
+    assert bwd(lib, gS0=A + 0x5000000) == ALIAS     # dS0 over grad_out
+    assert bwd(lib, B=0) == OK
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
 def test_valid_call_without_device_reports_device_error(lib):
     # S0 == S_final (in place) is allowed; with no CUDA device the call stops at the device check.

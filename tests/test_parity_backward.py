@@ -1,0 +1,102 @@
+"""GPU parity of gdn_backward (reverse mode of the forward) against the float64 oracle's reverse
+mode on the same inputs (needs a B200).  Same bar as the forward, per gradient tensor:
+max |gpu - ref| / max |ref| <= 1e-4 for float32 inputs, <= 2e-2 for bfloat16 inputs."""
+import numpy as np
+import pytest
+import torch
+
+import gated_delta_rule_142_b200 as gdn
+import oracle
+from gdn_inputs import as_f32_numpy, forward_inputs
+from parity_util import TOL, cpu_f64, oracle_threads, rel_err
+
+pytestmark = pytest.mark.gpu
+
+NAMES = ("dq", "dk", "dv", "dlog_alpha", "dbeta", "dS0")
+
+
+def grads_in(B, T, H, dv, dk, dtype, seed, final=True):
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    td = torch.float32 if dtype == "f32" else torch.bfloat16
+    d_out = torch.randn((B, T, H, dv), generator=g, dtype=torch.float32).to(td)
+    dSf = torch.randn((B, H, dv, dk), generator=g, dtype=torch.float32) if final else None
+    return d_out, dSf
+
+
+def check(inp, d_out, dSf, dtype, chunk, host=False, label=""):
+    dev = lambda t: None if t is None else (t.pin_memory() if host else t.cuda())  # noqa: E731
+    got = gdn.backward(dev(inp["q"]), dev(inp["k"]), dev(inp["v"]), dev(inp["log_alpha"]), dev(inp["beta"]),
+                       dev(inp["S0"]), dev(d_out), dev(dSf), chunk=chunk)
+    torch.cuda.synchronize()
+    S0 = None if inp["S0"] is None else as_f32_numpy(inp["S0"]).astype(np.float64)
+    ref = oracle.backward(*[as_f32_numpy(inp[n]) for n in ("q", "k", "v", "log_alpha", "beta")], S0,
+                          as_f32_numpy(d_out).astype(np.float64),
+                          None if dSf is None else dSf.numpy().astype(np.float64), nthreads=oracle_threads())
+    for name, gt, rf in zip(NAMES, got, ref):
+        e = rel_err(cpu_f64(gt), rf)
+        assert e <= TOL[dtype], "%s %s err %.3e" % (label, name, e)
+    return got
+
+
+@pytest.mark.parametrize("dtype,B,T,H,dk,dv,chunk,s0", [
+    ("f32", 1, 64, 2, 16, 16, 16, False),
+    ("f32", 2, 100, 3, 32, 64, 32, True),
+    ("f32", 1, 130, 2, 128, 128, 64, True),
+    ("f32", 1, 47, 2, 64, 16, 16, True),
+    ("bf16", 2, 150, 2, 128, 128, 64, True),
+    ("bf16", 1, 1, 2, 128, 128, 64, True),
+    ("bf16", 2, 77, 3, 64, 128, 32, False),
+])
+def test_backward_matches_oracle(dtype, B, T, H, dk, dv, chunk, s0):
+    inp = forward_inputs(B, T, H, dk, dv, dtype, seed=300 + T + dk + dv, s0_std=0.5 if s0 else None)
+    d_out, dSf = grads_in(B, T, H, dv, dk, dtype, seed=400 + T)
+    check(inp, d_out, dSf, dtype, chunk, label="%s B%d T%d H%d dk%d dv%d C%d" % (dtype, B, T, H, dk, dv, chunk))
+
+
+def test_backward_training_shape_sampled_heads():
+    """The 2K training shape (B8 H16 d128 C64, bf16): the whole batch on the GPU, the oracle on two
+    (b, h) problems cut out of it (heads and batch rows are independent)."""
+    B, T, H, d = 8, 2048, 16, 128
+    inp = forward_inputs(B, T, H, d, d, "bf16", seed=1, s0_std=0.02)
+    d_out, dSf = grads_in(B, T, H, d, d, "bf16", seed=11)
+    got = gdn.backward(*[inp[n].cuda() for n in ("q", "k", "v", "log_alpha", "beta", "S0")], d_out.cuda(),
+                       dSf.cuda(), chunk=64)
+    torch.cuda.synchronize()
+    for (b, h) in ((0, 0), (5, 11)):
+        sl = lambda t: as_f32_numpy(t[b:b + 1, :, h:h + 1].contiguous())  # noqa: E731
+        ref = oracle.backward(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["log_alpha"]), sl(inp["beta"]),
+                              inp["S0"][b:b + 1, h:h + 1].numpy().astype(np.float64),
+                              sl(d_out).astype(np.float64), dSf[b:b + 1, h:h + 1].numpy().astype(np.float64),
+                              nthreads=oracle_threads())
+        for i, name in enumerate(NAMES[:5]):
+            gt = cpu_f64(got[i])[b:b + 1, :, h:h + 1]
+            assert rel_err(gt, ref[i]) <= TOL["bf16"], (b, h, name)
+        assert rel_err(cpu_f64(got[5])[b:b + 1, h:h + 1], ref[5]) <= TOL["bf16"], (b, h, "dS0")
+
+
+def test_chunk_size_does_not_change_the_gradients():
+    inp = forward_inputs(1, 100, 2, 32, 32, "f32", seed=501, s0_std=0.3)
+    d_out, dSf = grads_in(1, 100, 2, 32, 32, "f32", seed=502)
+    a = gdn.backward(*[inp[n].cuda() for n in ("q", "k", "v", "log_alpha", "beta", "S0")], d_out.cuda(),
+                     dSf.cuda(), chunk=16)
+    b = gdn.backward(*[inp[n].cuda() for n in ("q", "k", "v", "log_alpha", "beta", "S0")], d_out.cuda(),
+                     dSf.cuda(), chunk=64)
+    torch.cuda.synchronize()
+    for x, y in zip(a, b):
+        assert rel_err(cpu_f64(x), cpu_f64(y)) <= 1e-5
+
+
+def test_host_buffers_and_no_final_gradient():
+    inp = forward_inputs(1, 70, 2, 64, 64, "f32", seed=503, s0_std=0.2)
+    d_out, _ = grads_in(1, 70, 2, 64, 64, "f32", seed=504, final=False)
+    check(inp, d_out, None, "f32", 32, host=True, label="host buffers")
+
+
+def test_empty_sequence_passes_the_final_gradient_through():
+    inp = forward_inputs(1, 0, 2, 16, 16, "f32", seed=505, s0_std=0.2)
+    d_out, dSf = grads_in(1, 0, 2, 16, 16, "f32", seed=506)
+    got = gdn.backward(*[inp[n].cuda() for n in ("q", "k", "v", "log_alpha", "beta", "S0")], d_out.cuda(),
+                       dSf.cuda(), chunk=16)
+    torch.cuda.synchronize()
+    assert torch.equal(got[5].cpu(), dSf)
