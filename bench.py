@@ -543,19 +543,81 @@ def run_varlen(args, world, rank):
     return 0
 
 
+# float32 FMA peak of the CUDA cores, derived from unit counts and the clock: 148 SMs x 128 FP32
+# lanes x 2 FLOP per FMA x 1.965 GHz (the backward runs on the CUDA cores in float32)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def run_backward(args, world, rank):
+    """gdn_backward over the chosen forward workload (inputs, grad_out and grad_S_final in HBM); one
+    call per step.  Counted work: twice the forward's counted FLOP per token-head (the usual
+    backward-to-forward ratio of the dense contractions), against the float32 CUDA-core peak."""
+    import gated_delta_rule_142_b200 as gdn
+    gdn.load()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    w = WORKLOADS[args.workload]
+    if args.tokens:
+        w = dataclasses.replace(w, T=args.tokens, name="%s_first%d" % (w.name, args.tokens))
+    inp = forward_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, seed=w.seed + 1000 * rank, s0_std=w.s0_std,
+                         alpha_mu=w.alpha_mu)
+    d = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed + 77)
+    g_out = torch.randn((w.B, w.T, w.H, w.dv), generator=g).to(d["q"].dtype).to(dev)
+    g_Sf = torch.randn((w.B, w.H, w.dv, w.dk), generator=g).to(dev)
+
+    def step():
+        gdn.backward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"], g_out, g_Sf, chunk=w.chunk,
+                     stream=stream)
+
+    sampler = ClockSampler(dev)
+    sampler.start()
+    for _ in range(args.warmup):
+        step()
+    gdn.timing_start()
+    ms = time_region(step, args.steps, stream, world)
+    ktimes = gdn.timing_stop()
+    clocks = sampler.stop()
+    ms_step = max_over_ranks(ms / args.steps, world)
+    flop = 2 * w.B * w.T * w.H * fwd_flop_per_token_head(w.dk, w.dv, w.chunk)
+    tflops = flop / (ms_step / 1e3) / 1e12
+    kernels = {kind: {"launches_per_step": n / args.steps, "ms_per_launch": kms / n, "share": kms / ms}
+               for kind, (kms, n) in ktimes.items()}
+    if rank == 0:
+        line = {"metric": "gated-delta backward tokens/s", "value": world * w.B * w.T / (ms_step / 1e3),
+                "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f32", "data": "synthetic",
+                "config": {"workload": w.name + "_backward", "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
+                           "chunk": w.chunk, "input_dtype": w.dtype,
+                           "parallelism": "replicas" if world > 1 else "single"},
+                "tflops": tflops,
+                "roofline": {"bound": "alu", "achieved": tflops, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+                             "frac": tflops / FP32_ALU_TFLOPS, "traffic": None,
+                             "peak_kind": "derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz",
+                             "flop_per_step": flop},
+                "kernels": kernels, "clocks": clocks,
+                "gpu_launches": sum(int(n) for _, n in ktimes.values())}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["gdn", "reference"], default="gdn")
-    ap.add_argument("--workload", default=FWD_WORKLOAD,
+    ap.add_argument("--workload", default=None,
                     choices=[n for n, w in WORKLOADS.items() if w.kind == "forward"],
                     help="forward workload timed as the step (default: the 64K-token one)")
     ap.add_argument("--tokens", type=int, default=0,
                     help="time only the first T tokens of the workload (profiler captures); not a bench line")
     ap.add_argument("--raw", action="store_true",
                     help="time gdn_forward_raw (input stage fused: raw q, k and gate logits) instead")
+    ap.add_argument("--backward", action="store_true",
+                    help="time gdn_backward on the workload (default workload then: the 2K training shape)")
     ap.add_argument("--varlen", type=int, default=0,
                     help="time packed prefill of this many sequences of mixed length instead of the forward step")
     ap.add_argument("--no-decode", action="store_true")
@@ -564,6 +626,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-step-seconds", type=float, default=8.0)
     args = ap.parse_args()
+    if args.workload is None:
+        args.workload = "fwd_bf16_b8h16_t2k_d128" if args.backward else FWD_WORKLOAD
     if args.impl == "reference":
         # CPU oracle arm: rank 0 alone runs and prints; other ranks exit without work.
         return run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
@@ -571,6 +635,8 @@ def main():
     try:
         if args.varlen:
             return run_varlen(args, world, rank)
+        if args.backward:
+            return run_backward(args, world, rank)
         return run_gdn(args, world, rank, local)
     finally:
         if world > 1:

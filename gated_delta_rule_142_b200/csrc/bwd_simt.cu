@@ -38,7 +38,7 @@
 namespace gdn {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 
 struct BwdDims {
     int dk, dv, C, rows, nslab, nchunks;
