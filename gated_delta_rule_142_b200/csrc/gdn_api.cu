@@ -295,6 +295,197 @@ int gdn_decode_step_raw(const void *q, const void *k, const void *v, const float
 
 namespace {
 
+// One forward on device buffers (T > 0): the two-kernel tensor-core forward where it applies and its
+// workspace can be had, else the single-kernel tensor-core forward, else the CUDA-core forward.
+int run_device(FwdProblem p, const DeviceInfo &info, bool raw, cudaStream_t stream) {
+    const int64_t ntok = p.B * p.T * p.H;
+    int st = GDN_OK;
+    cudaError_t e = cudaSuccess;
+    const FwdPath path = forced_path();
+    bool done = false;
+    if (path == FwdPath::Auto && gdn::fwd_split_supported(p)) {
+        const int nseg = gdn::fwd_tc_segments(p, info.sm_count, true);
+        void *ws = nullptr;
+        if (scratch_alloc(&ws, gdn::fwd_split_workspace_bytes(p, nseg), stream) == cudaSuccess) {
+            p.raw_inputs = raw ? 1 : 0;  // the prep kernel runs the input stage on its own loads
+            e = gdn::launch_fwd_split(p, nseg, info.sm_count, ws, stream);
+            cudaFreeAsync(ws, stream);
+            done = true;
+        } else {
+            // too little device memory for the per-chunk workspace: the single-kernel path below
+            cudaGetLastError();
+        }
+    }
+    void *staged = nullptr;
+    if (!done && raw) {
+        if ((st = stage_inputs(p, ntok, &staged, stream))) {
+            if (staged) cudaFreeAsync(staged, stream);
+            return st;
+        }
+    }
+    if (!done && path != FwdPath::Simt && gdn::fwd_tc_supported(p)) {
+        const int nseg = gdn::fwd_tc_segments(p, info.sm_count, false);
+        const size_t ws_bytes = gdn::fwd_tc_workspace_bytes(p, nseg);
+        void *ws = nullptr;
+        if (ws_bytes > 0 && scratch_alloc(&ws, ws_bytes, stream) != cudaSuccess) {
+            cudaGetLastError();
+            if (staged) cudaFreeAsync(staged, stream);
+            return GDN_ERR_ALLOC;
+        }
+        e = gdn::launch_fwd_tc(p, nseg, ws, stream);
+        if (ws) cudaFreeAsync(ws, stream);
+    } else if (!done) {
+        e = gdn::launch_fwd_simt(p, info.sm_count, stream);
+    }
+    if (staged) cudaFreeAsync(staged, stream);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_LAUNCH;
+    }
+    return GDN_OK;
+}
+
+// ---------------------------------------------------------------- host pipeline
+bool is_pinned_host(const void *p) {
+    cudaPointerAttributes attr;
+    if (!p || cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return attr.type == cudaMemoryTypeHost;
+}
+
+// B rows of `width` bytes between buffers with row pitches dpitch and spitch: one strided copy
+// where the pitches allow it, else one copy per row.
+bool copy_rows(void *dst, int64_t dpitch, const void *src, int64_t spitch, int64_t width, int64_t B,
+               cudaMemcpyKind kind, cudaStream_t s) {
+    if (B == 1) return cudaMemcpyAsync(dst, src, (size_t)width, kind, s) == cudaSuccess;
+    if (dpitch < ((int64_t)1 << 31) && spitch < ((int64_t)1 << 31))
+        return cudaMemcpy2DAsync(dst, (size_t)dpitch, src, (size_t)spitch, (size_t)width, (size_t)B, kind, s) ==
+               cudaSuccess;
+    for (int64_t b = 0; b < B; ++b)
+        if (cudaMemcpyAsync(static_cast<uint8_t *>(dst) + b * dpitch, static_cast<const uint8_t *>(src) + b * spitch,
+                            (size_t)width, kind, s) != cudaSuccess)
+            return false;
+    return true;
+}
+
+// Two library-owned copy streams per device (host-to-device, device-to-host), created on first use.
+std::atomic<cudaStream_t> g_copy_streams[kMaxDevices][2];
+
+cudaStream_t copy_stream(int dev, int which) {
+    cudaStream_t s = g_copy_streams[dev][which].load(std::memory_order_acquire);
+    if (s) return s;
+    if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    cudaStream_t expected = nullptr;
+    if (!g_copy_streams[dev][which].compare_exchange_strong(expected, s)) {
+        cudaStreamDestroy(s);
+        s = expected;
+    }
+    return s;
+}
+
+// gdn_forward with q, k, v, gates and out in pinned host memory, cut along T into pieces of whole
+// chunks: while piece p runs on the caller's stream, piece p + 1 is copied in on one copy stream
+// and piece p - 1 copied out on the other, so that the two directions of the host link and the
+// kernels overlap.  The state passes from piece to piece on the device in float32 (the forward
+// over T1 then T2 tokens from the state at T1 is the forward over T1 + T2 tokens).  Device
+// buffers: two piece slots and two states.  Returns GDN_OK, or a status when nothing could be
+// set up (the caller then takes the staged path), or GDN_ERR_LAUNCH after a failed enqueue.
+int forward_pipelined(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                      const float *S0, void *out, float *S_final, int64_t B, int64_t T, int64_t H, int64_t dk,
+                      int64_t dv, int64_t chunk, int dtype, bool raw, int npieces, const DeviceInfo &info,
+                      cudaStream_t cs) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return GDN_ERR_DEVICE;
+    }
+    cudaStream_t hs = copy_stream(dev, 0), ds = copy_stream(dev, 1);
+    if (!hs || !ds) return GDN_ERR_ALLOC;
+    const int64_t es = (dtype == GDN_F32) ? 4 : 2;
+    const int64_t L = ((T + npieces - 1) / npieces + chunk - 1) / chunk * chunk;  // tokens per piece
+    const int64_t P = (T + L - 1) / L;
+    const int64_t nstate = B * H * dv * dk * 4;
+    // slot layout: q, k, v, out, log_alpha, beta of one piece, [B, L, H, .] each
+    const int64_t bq = B * L * H * dk * es, bv = B * L * H * dv * es, bg = B * L * H * 4;
+    const int64_t slot = 2 * bq + 2 * bv + 2 * bg;
+    void *mem = nullptr;
+    if (scratch_alloc(&mem, (size_t)(2 * slot + 3 * nstate), cs) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_ALLOC;
+    }
+    uint8_t *base = static_cast<uint8_t *>(mem);
+    float *st[2] = {reinterpret_cast<float *>(base + 2 * slot), reinterpret_cast<float *>(base + 2 * slot + nstate)};
+    float *s0dev = reinterpret_cast<float *>(base + 2 * slot + 2 * nstate);
+    cudaEvent_t ev[7] = {};
+    bool ok = true;
+    for (cudaEvent_t &x : ev) ok = ok && cudaEventCreateWithFlags(&x, cudaEventDisableTiming) == cudaSuccess;
+    // ev[0]: the allocation (and S0) on the caller's stream; ev[1 + s]: inputs of slot s landed;
+    // ev[3 + s]: slot s computed; ev[5 + s]: outputs of slot s copied out
+    const float *s_in = nullptr;
+    if (ok && S0) {
+        ok = cudaMemcpyAsync(s0dev, S0, (size_t)nstate, cudaMemcpyDefault, cs) == cudaSuccess;
+        s_in = s0dev;
+    }
+    ok = ok && cudaEventRecord(ev[0], cs) == cudaSuccess && cudaStreamWaitEvent(hs, ev[0], 0) == cudaSuccess &&
+         cudaStreamWaitEvent(ds, ev[0], 0) == cudaSuccess;
+    int st_status = GDN_OK;
+    for (int64_t pc = 0; pc < P && ok; ++pc) {
+        const int sl = (int)(pc & 1);
+        const int64_t t0 = pc * L, len = (T - t0 < L) ? (T - t0) : L;
+        uint8_t *sb = base + sl * slot;
+        uint8_t *dq = sb, *dkk = sb + bq, *dvv = sb + 2 * bq, *dout = sb + 2 * bq + bv;
+        float *dla = reinterpret_cast<float *>(sb + 2 * bq + 2 * bv), *dbe = reinterpret_cast<float *>(sb + 2 * bq + 2 * bv + bg);
+        // inputs of this piece: one strided copy per tensor (B rows of len * H * d elements)
+        if (pc >= 2) ok = ok && cudaStreamWaitEvent(hs, ev[3 + sl], 0) == cudaSuccess;
+        auto in2d = [&](void *dst, const void *src, int64_t tok_bytes) {
+            return copy_rows(dst, len * tok_bytes, static_cast<const uint8_t *>(src) + t0 * tok_bytes, T * tok_bytes,
+                             len * tok_bytes, B, cudaMemcpyHostToDevice, hs);
+        };
+        ok = ok && in2d(dq, q, H * dk * es) && in2d(dkk, k, H * dk * es) && in2d(dvv, v, H * dv * es) &&
+             in2d(dla, log_alpha, H * 4) && in2d(dbe, beta, H * 4);
+        ok = ok && cudaEventRecord(ev[1 + sl], hs) == cudaSuccess;
+        // the piece's forward on the caller's stream
+        ok = ok && cudaStreamWaitEvent(cs, ev[1 + sl], 0) == cudaSuccess;
+        if (pc >= 2) ok = ok && cudaStreamWaitEvent(cs, ev[5 + sl], 0) == cudaSuccess;
+        if (!ok) break;
+        FwdProblem p;
+        p.q = dq; p.k = dkk; p.v = dvv; p.log_alpha = dla; p.beta = dbe;
+        p.S0 = s_in;
+        p.out = dout;
+        p.S_final = st[sl];
+        p.B = B; p.T = len; p.H = H; p.dk = dk; p.dv = dv; p.chunk = chunk; p.dtype = dtype;
+        if ((st_status = run_device(p, info, raw, cs))) {
+            ok = false;
+            break;
+        }
+        s_in = st[sl];
+        ok = ok && cudaEventRecord(ev[3 + sl], cs) == cudaSuccess;
+        // outputs of this piece
+        ok = ok && cudaStreamWaitEvent(ds, ev[3 + sl], 0) == cudaSuccess &&
+             copy_rows(static_cast<uint8_t *>(out) + t0 * H * dv * es, T * H * dv * es, dout, len * H * dv * es,
+                       len * H * dv * es, B, cudaMemcpyDeviceToHost, ds) &&
+             cudaEventRecord(ev[5 + sl], ds) == cudaSuccess;
+    }
+    // the caller's stream orders after everything enqueued on the copy streams (also after a
+    // failure part-way); then the final state and the frees
+    ok = cudaEventRecord(ev[1], hs) == cudaSuccess && cudaEventRecord(ev[5], ds) == cudaSuccess &&
+         cudaStreamWaitEvent(cs, ev[1], 0) == cudaSuccess && cudaStreamWaitEvent(cs, ev[5], 0) == cudaSuccess && ok;
+    if (ok && S_final && s_in) ok = cudaMemcpyAsync(S_final, s_in, (size_t)nstate, cudaMemcpyDefault, cs) == cudaSuccess;
+    for (cudaEvent_t &x : ev)
+        if (x) cudaEventDestroy(x);
+    cudaFreeAsync(mem, cs);
+    if (!ok) {
+        cudaGetLastError();
+        return st_status ? st_status : GDN_ERR_LAUNCH;
+    }
+    return GDN_OK;
+}
+
 int forward_impl(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                  const float *S0, void *out, float *S_final, int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
                  int64_t chunk, void *stream_, int dtype, bool raw) {
@@ -324,6 +515,22 @@ int forward_impl(const void *q, const void *k, const void *v, const float *log_a
     if (int st = device_info(&info)) return st;
     cudaStream_t stream = static_cast<cudaStream_t>(stream_);
 
+    // Large problems whose token-major tensors are all in pinned host memory: pipelined over
+    // pieces of T (copies in both directions overlap the kernels), unless GDN_HOST_PIPELINE=0.
+    const int64_t host_bytes = 2 * nqk + 2 * nv + 2 * ntok * 4;
+    const char *pipe_env = getenv("GDN_HOST_PIPELINE");
+    if (T >= 2 * chunk && host_bytes >= ((int64_t)64 << 20) && !(pipe_env && strcmp(pipe_env, "0") == 0) &&
+        is_pinned_host(q) && is_pinned_host(k) && is_pinned_host(v) && is_pinned_host(log_alpha) &&
+        is_pinned_host(beta) && is_pinned_host(out)) {
+        int64_t pieces = host_bytes / ((int64_t)64 << 20);
+        pieces = pieces < 2 ? 2 : (pieces > 16 ? 16 : pieces);
+        if (pieces > T / chunk) pieces = T / chunk;
+        const int st = forward_pipelined(q, k, v, log_alpha, beta, S0, out, S_final, B, T, H, dk, dv, chunk,
+                                         dtype, raw, (int)pieces, info, stream);
+        if (st != GDN_ERR_ALLOC && st != GDN_ERR_DEVICE) return st;
+        // no room for the pipeline's buffers: the staged path below
+    }
+
     Stager stg(stream);
     FwdProblem p;
     int st = GDN_OK;
@@ -351,44 +558,8 @@ int forward_impl(const void *q, const void *k, const void *v, const float *log_a
             e = p.S0 ? cudaMemcpyAsync(p.S_final, p.S0, (size_t)nstate, cudaMemcpyDeviceToDevice, stream)
                      : cudaMemsetAsync(p.S_final, 0, (size_t)nstate, stream);
         }
-    } else {
-        const FwdPath path = forced_path();
-        bool done = false;
-        if (path == FwdPath::Auto && gdn::fwd_split_supported(p)) {
-            const int nseg = gdn::fwd_tc_segments(p, info.sm_count, true);
-            void *ws = nullptr;
-            if (scratch_alloc(&ws, gdn::fwd_split_workspace_bytes(p, nseg), stream) == cudaSuccess) {
-                p.raw_inputs = raw ? 1 : 0;  // the prep kernel runs the input stage on its own loads
-                e = gdn::launch_fwd_split(p, nseg, info.sm_count, ws, stream);
-                cudaFreeAsync(ws, stream);
-                done = true;
-            } else {
-                // too little device memory for the per-chunk workspace: the single-kernel path below
-                cudaGetLastError();
-            }
-        }
-        void *staged = nullptr;
-        if (!done && raw) {
-            if ((st = stage_inputs(p, ntok, &staged, stream))) {
-                if (staged) cudaFreeAsync(staged, stream);
-                return st;
-            }
-        }
-        if (!done && path != FwdPath::Simt && gdn::fwd_tc_supported(p)) {
-            const int nseg = gdn::fwd_tc_segments(p, info.sm_count, false);
-            const size_t ws_bytes = gdn::fwd_tc_workspace_bytes(p, nseg);
-            void *ws = nullptr;
-            if (ws_bytes > 0 && scratch_alloc(&ws, ws_bytes, stream) != cudaSuccess) {
-                cudaGetLastError();
-                if (staged) cudaFreeAsync(staged, stream);
-                return GDN_ERR_ALLOC;
-            }
-            e = gdn::launch_fwd_tc(p, nseg, ws, stream);
-            if (ws) cudaFreeAsync(ws, stream);
-        } else if (!done) {
-            e = gdn::launch_fwd_simt(p, info.sm_count, stream);
-        }
-        if (staged) cudaFreeAsync(staged, stream);
+    } else if ((st = run_device(p, info, raw, stream))) {
+        return st;
     }
     if (e != cudaSuccess) {
         cudaGetLastError();

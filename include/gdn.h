@@ -32,13 +32,23 @@
  * device-to-host copies of the results after them; with pinned host output
  * memory the results are valid after the stream has been synchronised,
  * with pageable host output memory they are valid when the call returns.
+ * One exception for throughput: a gdn_forward / gdn_forward_raw whose q, k,
+ * v, gates and out are all pinned host memory (64 MB or more of them) is cut
+ * along T into pieces of whole chunks.  The copies of one piece in, the
+ * kernels of the next and the copy of another piece out overlap on the
+ * library's two copy streams and on `stream`.  The state passes between
+ * pieces in float32 on the device.  `stream` still orders after every copy,
+ * so results are valid once it has been synchronised.  Set the environment
+ * variable GDN_HOST_PIPELINE=0 to stage the whole problem instead.
  * The library keeps no pointer after a call returns and owns no buffer.
  *
  * Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
- * stream).  All device work of a call is enqueued on it; calls are
- * asynchronous unless host staging forces a synchronous copy.  The library
- * holds no global mutable state, so calls on different streams may run
- * concurrently provided their buffers do not overlap.
+ * stream).  All device work of a call is enqueued on it, apart from the
+ * pipelined host copies above; calls are asynchronous unless host staging
+ * forces a synchronous copy.  The library's only global state is immutable
+ * per-device data: device properties, the scratch pool and the two copy
+ * streams.  Calls on different streams may therefore run concurrently,
+ * provided their buffers do not overlap.
  *
  * Errors: every entry point returns a gdn_status.  Arguments are validated
  * on the host before anything is enqueued; a rejected call enqueues nothing
