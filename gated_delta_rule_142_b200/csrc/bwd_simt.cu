@@ -25,10 +25,15 @@
 // adjoint of the chunk-local cumsum.
 //
 // The states entering the chunks come from a forward recompute that writes
-// them as checkpoints (fwd_simt.cu).  One CTA owns one (b, h) and a slab of
+// them as checkpoints: the two-kernel tensor-core forward (its chain kernel
+// stores the float32 state it holds in tensor memory at every chunk start)
+// where that forward applies, else the CUDA-core forward with outputs off.  One CTA owns one (b, h) and a slab of
 // `rows` value dimensions.  dU, dR, dV and the slab of dS depend only on the
 // slab's value dimensions; dQ, dK, dbeta and dlog_alpha are sums over value
 // dimensions, so each slab adds its share with float32 atomics.
+#include <stdlib.h>
+#include <string.h>
+
 #include <atomic>
 
 #include "common.cuh"
@@ -516,19 +521,51 @@ BwdDims plan(const BwdProblem &p, int sm_count) {
     return d;
 }
 
+// The tensor-core recompute serves the shapes of the two-kernel forward unless
+// GDN_BWD_RECOMPUTE=simt.
+bool tc_recompute(const FwdProblem &f) {
+    const char *e = getenv("GDN_BWD_RECOMPUTE");
+    return fwd_split_supported(f) && !(e && strcmp(e, "simt") == 0);
+}
+
+// workspace: checkpoints | (bf16) float32 dq, dk accumulators | (tensor-core recompute) its
+// per-chunk workspace and an output buffer
+struct BwdLayout {
+    size_t ckpt, acc, fwd_ws, fwd_out, total;
+    int nseg;
+};
+
+BwdLayout layout(const BwdProblem &p, int sm_count) {
+    const FwdProblem &f = p.f;
+    BwdLayout l;
+    const int64_t nchunks = (f.T + f.chunk - 1) / f.chunk, ntok = f.B * f.T * f.H;
+    auto round = [](size_t x) { return (x + 255) & ~size_t(255); };
+    l.ckpt = round((size_t)(f.B * f.H) * nchunks * f.dv * f.dk * 4);
+    l.acc = f.dtype != GDN_F32 ? round(2 * (size_t)ntok * f.dk * 4) : 0;
+    l.nseg = 1;
+    l.fwd_ws = l.fwd_out = 0;
+    if (tc_recompute(f)) {
+        l.nseg = fwd_tc_segments(f, sm_count, true);
+        l.fwd_ws = round(fwd_split_workspace_bytes(f, l.nseg));
+        l.fwd_out = round((size_t)ntok * f.dv * 2);
+    }
+    l.total = l.ckpt + l.acc + l.fwd_ws + l.fwd_out;
+    return l;
+}
+
 template <typename Tin>
 cudaError_t launch_t(const BwdProblem &p, int sm_count, void *workspace, cudaStream_t stream) {
     const FwdProblem &f = p.f;
     const BwdDims d = plan(p, sm_count);
+    const BwdLayout l = layout(p, sm_count);
     const size_t smem = d.smem_floats() * sizeof(float);
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
     const int64_t ntok = f.B * f.T * f.H;
-    // workspace: checkpoints, then (bf16) float32 accumulators of dq and dk
-    float *ckpt = static_cast<float *>(workspace);
-    const size_t nck = (size_t)(f.B * f.H) * d.nchunks * f.dv * f.dk;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    float *ckpt = reinterpret_cast<float *>(ws);
     const bool f32 = f.dtype == GDN_F32;
-    float *dq_acc = f32 ? static_cast<float *>(p.dq) : ckpt + nck;
-    float *dk_acc = f32 ? static_cast<float *>(p.dk) : ckpt + nck + ntok * f.dk;
+    float *dq_acc = f32 ? static_cast<float *>(p.dq) : reinterpret_cast<float *>(ws + l.ckpt);
+    float *dk_acc = f32 ? static_cast<float *>(p.dk) : dq_acc + ntok * f.dk;
     cudaError_t e;
     // forward recompute: the state entering every chunk
     FwdProblem fc = f;
@@ -536,7 +573,12 @@ cudaError_t launch_t(const BwdProblem &p, int sm_count, void *workspace, cudaStr
     fc.S_final = nullptr;
     fc.ckpt = ckpt;
     fc.raw_inputs = 0;
-    if ((e = launch_fwd_simt(fc, sm_count, stream)) != cudaSuccess) return e;
+    if (l.fwd_ws) {
+        fc.out = ws + l.ckpt + l.acc + l.fwd_ws;
+        if ((e = launch_fwd_split(fc, l.nseg, sm_count, ws + l.ckpt + l.acc, stream)) != cudaSuccess) return e;
+    } else if ((e = launch_fwd_simt(fc, sm_count, stream)) != cudaSuccess) {
+        return e;
+    }
     if ((e = cudaMemsetAsync(dq_acc, 0, (size_t)ntok * f.dk * 4, stream)) != cudaSuccess ||
         (e = cudaMemsetAsync(dk_acc, 0, (size_t)ntok * f.dk * 4, stream)) != cudaSuccess ||
         (e = cudaMemsetAsync(p.dlog_alpha, 0, (size_t)ntok * 4, stream)) != cudaSuccess ||
@@ -573,13 +615,7 @@ cudaError_t launch_t(const BwdProblem &p, int sm_count, void *workspace, cudaStr
 
 }  // namespace
 
-size_t bwd_simt_workspace_bytes(const BwdProblem &p) {
-    const FwdProblem &f = p.f;
-    const int64_t nchunks = (f.T + f.chunk - 1) / f.chunk;
-    size_t bytes = (size_t)(f.B * f.H) * nchunks * f.dv * f.dk * 4;
-    if (f.dtype != GDN_F32) bytes += 2 * (size_t)(f.B * f.T * f.H) * f.dk * 4;
-    return bytes;
-}
+size_t bwd_simt_workspace_bytes(const BwdProblem &p, int sm_count) { return layout(p, sm_count).total; }
 
 cudaError_t launch_bwd_simt(const BwdProblem &p, int sm_count, void *workspace, cudaStream_t stream) {
     if (p.f.B * p.f.H == 0 || p.f.T == 0) return cudaSuccess;

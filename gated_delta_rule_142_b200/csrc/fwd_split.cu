@@ -683,6 +683,8 @@ struct ChainArgs {
     const int4 *ptab;      // per-CTA work of packed sequences, or nullptr
     const int2 *ctab;      // packed chunk table, or nullptr
     __nv_bfloat16 *out;    // for the plain stores of partial packed chunks
+    float *ckpt;           // fixed-length only, or nullptr: the state entering every chunk,
+                           // [B*H][chunks][dv][dk] float32 (the backward's checkpoints)
 };
 
 __global__ void __launch_bounds__(kChainThreads, 1)
@@ -997,6 +999,13 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 uint32_t r[32];
                 tmem_ld32(tm + lb + TC_S + col0, r);
                 tmem_wait_ld();
+                if (p.ckpt) {  // the state entering chunk c, as a checkpoint
+                    float4 *dst = reinterpret_cast<float4 *>(p.ckpt + (witem(c) * kD + j) * kD + col0);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
+                                             __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
+                }
                 uint32_t pk[16];
 #pragma unroll
                 for (int i = 0; i < 32; i += 2)
@@ -1515,6 +1524,7 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
     a.ptab = nullptr;
     a.ctab = nullptr;
     a.out = static_cast<__nv_bfloat16 *>(p.out);
+    a.ckpt = p.ckpt;
     if (a.nseg > 1) {
         const size_t per = (size_t)heads * (a.nseg - 1) * kD * kD;
         a.Bw = seg_ws;
@@ -1624,6 +1634,7 @@ cudaError_t launch_fwd_split_packed(const FwdProblem &p, const int64_t *cu_seqle
     a.ptab = d_ptab;
     a.ctab = d_ctab;
     a.out = static_cast<__nv_bfloat16 *>(p.out);
+    a.ckpt = nullptr;
     {
         TimedLaunch tl_(GDN_KERNEL_CHAIN, stream);
         fwd_chain_kernel<<<(unsigned)(N * H), kChainThreads, SMEM_CHAIN, stream>>>(mq, mk, mv, mo, mp, mtb, mw, a);

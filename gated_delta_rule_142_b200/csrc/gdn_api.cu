@@ -855,7 +855,7 @@ extern "C" int gdn_backward(const void *q, const void *k, const void *v, const f
                            : cudaMemsetAsync(p.dS0, 0, (size_t)nstate, stream);
     } else {
         void *ws = nullptr;
-        if (scratch_alloc(&ws, gdn::bwd_simt_workspace_bytes(p), stream) != cudaSuccess) {
+        if (scratch_alloc(&ws, gdn::bwd_simt_workspace_bytes(p, info.sm_count), stream) != cudaSuccess) {
             cudaGetLastError();
             return GDN_ERR_ALLOC;
         }

@@ -39,8 +39,9 @@ struct FwdProblem {
     // x_beta (log alpha = -softplus(x_alpha), beta = sigmoid(x_beta)); only the two-kernel
     // forward takes this form, the others get the output of launch_input_stage()
     int raw_inputs = 0;
-    // CUDA-core forward only: when set, the state entering every chunk is written here,
-    // [B*H][chunks][dv][dk] float32 (the backward's checkpoints); out may then be nullptr
+    // CUDA-core and two-kernel forwards: when set, the state entering every chunk is written
+    // here, [B*H][chunks][dv][dk] float32 (the backward's checkpoints); the CUDA-core forward
+    // then also accepts out == nullptr
     float *ckpt = nullptr;
 };
 
@@ -79,7 +80,7 @@ struct BwdProblem {
     float *dlog_alpha, *dbeta;  // [B, T, H]
     float *dS0;               // [B, H, dv, dk] or nullptr (not written)
 };
-size_t bwd_simt_workspace_bytes(const BwdProblem &p);
+size_t bwd_simt_workspace_bytes(const BwdProblem &p, int sm_count);
 cudaError_t launch_bwd_simt(const BwdProblem &p, int sm_count, void *workspace, cudaStream_t stream);
 
 // fwd_tc.cu -- tcgen05 chunkwise forward: bf16, dk = dv = 128, chunk = 64.

@@ -75,6 +75,15 @@ def test_backward_training_shape_sampled_heads():
         assert rel_err(cpu_f64(got[5])[b:b + 1, h:h + 1], ref[5]) <= TOL["bf16"], (b, h, "dS0")
 
 
+def test_simt_recompute_matches(monkeypatch):
+    """bf16, d = 128, chunk 64 recomputes the forward on the tensor cores by default; the CUDA-core
+    recompute (GDN_BWD_RECOMPUTE=simt) meets the same bar."""
+    monkeypatch.setenv("GDN_BWD_RECOMPUTE", "simt")
+    inp = forward_inputs(2, 150, 2, 128, 128, "bf16", seed=511, s0_std=0.5)
+    d_out, dSf = grads_in(2, 150, 2, 128, 128, "bf16", seed=512)
+    check(inp, d_out, dSf, "bf16", 64, label="simt recompute")
+
+
 def test_chunk_size_does_not_change_the_gradients():
     inp = forward_inputs(1, 100, 2, 32, 32, "f32", seed=501, s0_std=0.3)
     d_out, dSf = grads_in(1, 100, 2, 32, 32, "f32", seed=502)
