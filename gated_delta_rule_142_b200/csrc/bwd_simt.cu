@@ -54,15 +54,18 @@ struct BwdDims {
     }
 };
 
-// acc[a][b] += sum_c X[(i0+a)*ldx + c] * Y[(j0+b)*ldy + c],  c in [0, K)
-__device__ __forceinline__ void tile_nt(const float *X, int ldx, const float *Y, int ldy, int i0, int j0, int K,
-                                        float acc[4][4]) {
+// acc[a][b] += sum_c X[(i0+a)*ldx + c] * Y[(jb+G*b)*ldy + c],  c in [0, K).  The Y rows of a thread
+// are G apart, so that neighbouring threads (consecutive jb, one i0) read neighbouring rows: the eight
+// 16-byte loads of a quarter warp then fall in eight different bank groups (rows 4 apart would share
+// two, with a row pitch of an odd number of 16-byte units).
+__device__ __forceinline__ void tile_nt(const float *X, int ldx, const float *Y, int ldy, int i0, int jb, int G,
+                                        int K, float acc[4][4]) {
     for (int c = 0; c < K; c += 4) {
         float4 x[4], y[4];
 #pragma unroll
         for (int a = 0; a < 4; ++a) x[a] = *reinterpret_cast<const float4 *>(X + (i0 + a) * ldx + c);
 #pragma unroll
-        for (int b = 0; b < 4; ++b) y[b] = *reinterpret_cast<const float4 *>(Y + (j0 + b) * ldy + c);
+        for (int b = 0; b < 4; ++b) y[b] = *reinterpret_cast<const float4 *>(Y + (jb + G * b) * ldy + c);
 #pragma unroll
         for (int a = 0; a < 4; ++a)
 #pragma unroll
@@ -120,7 +123,7 @@ bwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
     float *dRs = Us + C * LDR;      // C x LDR  diag(dl) K dS^T, then dU, then dR
     float *MA = dRs + C * LDR;      // C x LDC  e^{g_t-g_s} (k_t . k_s) (s < t), then F
     float *MP = MA + C * LDC;       // C x LDC  P
-    float *MD = MP + C * LDC;       // C x LDC  dP o E
+    float *MD = MP + C * LDC;       // C x LDC  MA transposed (for the back substitution), then dP o E
     float *g = MD + C * LDC;        // C
     float *bet = g + C;             // C
     float *gam = bet + C;           // C
@@ -136,7 +139,6 @@ bwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
     const int r0 = slab * rows;
     const int64_t tsk = H * dk, tsv = H * dv;  // token strides
     const int64_t base_k = (b * T * H + h) * dk, base_v = (b * T * H + h) * dv, base_g = b * T * H + h;
-    const int tpc = kThreads / rows;  // threads per column in the substitutions
 
     // dS slab <- dS_final (or zero)
     for (int i = tid; i < rows * (dk / 4); i += kThreads) {
@@ -211,51 +213,70 @@ bwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
             for (int w = tid; w < 2 * nx + 2 * nc; w += kThreads) {
                 float acc[4][4] = {};
                 if (w < 2 * nx) {
-                    const int ww = w % nx;
-                    const int i0 = (ww / (rows / 4)) * 4, j0 = (ww % (rows / 4)) * 4;
+                    const int ww = w % nx, G = rows / 4;
+                    const int i0 = (ww / G) * 4, jb = ww % G;
                     const bool isx = w < nx;
-                    tile_nt(Ks, LDK, isx ? Ss : dSs, LDK, i0, j0, dk, acc);
+                    tile_nt(Ks, LDK, isx ? Ss : dSs, LDK, i0, jb, G, dk, acc);
                     float *dst = isx ? Xs : dRs;
                     const float *f = isx ? gam : dl;
 #pragma unroll
                     for (int a = 0; a < 4; ++a)
 #pragma unroll
-                        for (int bb = 0; bb < 4; ++bb) dst[(i0 + a) * LDR + j0 + bb] = f[i0 + a] * acc[a][bb];
+                        for (int bb = 0; bb < 4; ++bb) dst[(i0 + a) * LDR + jb + G * bb] = f[i0 + a] * acc[a][bb];
                 } else {
-                    const int ww = (w - 2 * nx) % nc;
+                    const int ww = (w - 2 * nx) % nc, G = C / 4;
                     const bool isa = (w - 2 * nx) < nc;
-                    const int i0 = (ww / (C / 4)) * 4, j0 = (ww % (C / 4)) * 4;
-                    if (j0 <= i0 + 3) tile_nt(isa ? Ks : Qs, LDK, Ks, LDK, i0, j0, dk, acc);
+                    const int i0 = (ww / G) * 4, jb = ww % G;
+                    if (jb <= i0 + 3) tile_nt(isa ? Ks : Qs, LDK, Ks, LDK, i0, jb, G, dk, acc);
                     float *dst = isa ? MA : MP;
 #pragma unroll
                     for (int a = 0; a < 4; ++a)
 #pragma unroll
                         for (int bb = 0; bb < 4; ++bb) {
-                            const int t = i0 + a, s = j0 + bb;
+                            const int t = i0 + a, s = jb + G * bb;
                             const bool keep = isa ? (s < t) : (s <= t);
-                            dst[t * LDC + s] = keep ? expf(g[t] - g[s]) * acc[a][bb] : 0.f;
+                            const float x = keep ? expf(g[t] - g[s]) * acc[a][bb] : 0.f;
+                            dst[t * LDC + s] = x;
+                            if (isa) MD[s * LDC + t] = x;
                         }
                 }
             }
         }
         __syncthreads();
 
-        // ---- pass 2: U by forward substitution, U_t = beta_t (v_t - X_t) - sum_{s<t} beta_t MA_ts U_s ----
+        // ---- pass 2: U by forward substitution, U_t = beta_t (v_t - X_t) - sum_{s<t} beta_t MA_ts U_s.
+        //      A warp owns value columns two at a time and keeps them in registers (lane l holds
+        //      tokens l and l + 32); each step is a shuffle reduction, with no block barrier ----
         {
-            const int j = tid / tpc, part = tid % tpc;
-            for (int t = 0; t < C; ++t) {
-                float acc = 0.f;
-                for (int s = part; s < t; s += tpc) acc += MA[t * LDC + s] * Us[s * LDR + j];
-                for (int off = tpc / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-                if (part == 0) Us[t * LDR + j] = bet[t] * (Vs[t * LDR + j] - Xs[t * LDR + j] - acc);
-                __syncthreads();
+            const int lane = tid & 31, warp = tid >> 5, nw = kThreads / 32;
+            for (int j0 = 2 * warp; j0 < rows; j0 += 2 * nw) {
+                const int j1 = (j0 + 1 < rows) ? j0 + 1 : j0;
+                float ua0 = 0.f, ua1 = 0.f, ub0 = 0.f, ub1 = 0.f;  // column j0 / j1, tokens lane / lane + 32
+                for (int t = 0; t < C; ++t) {
+                    const float m0 = (lane < t) ? MA[t * LDC + lane] : 0.f;
+                    const float m1 = (lane + 32 < t) ? MA[t * LDC + lane + 32] : 0.f;
+                    float sa = fmaf(m0, ua0, m1 * ua1), sb = fmaf(m0, ub0, m1 * ub1);
+#pragma unroll
+                    for (int off = 16; off >= 1; off >>= 1) {
+                        sa += __shfl_xor_sync(0xffffffffu, sa, off);
+                        sb += __shfl_xor_sync(0xffffffffu, sb, off);
+                    }
+                    const float va = bet[t] * (Vs[t * LDR + j0] - Xs[t * LDR + j0] - sa);
+                    const float vb = bet[t] * (Vs[t * LDR + j1] - Xs[t * LDR + j1] - sb);
+                    if (lane == t) { ua0 = va; ub0 = vb; }
+                    if (lane + 32 == t) { ua1 = va; ub1 = vb; }
+                }
+                if (lane < C) { Us[lane * LDR + j0] = ua0; Us[lane * LDR + j1] = ub0; }
+                if (lane + 32 < C) { Us[(lane + 32) * LDR + j0] = ua1; Us[(lane + 32) * LDR + j1] = ub1; }
             }
         }
+        __syncthreads();
 
         // ---- pass 3: dU = P^T dO + diag(dl) K dS^T (with d g from dl: w_s = U_s . dl_s (K dS^T)_s);
         //      d g_t from the outputs' gamma_t Q S^T term;  d g_C from gamma_C <dS, S> ----
         {
             const int nu = (C / 4) * (rows / 4), ny = nu, ns = rows * (dk / 4);
+            float dgc_part = 0.f;  // this thread's share of d g_C, summed over its warp at the end
             for (int w = tid; w < nu + ny + ns; w += kThreads) {
                 if (w < nu) {
                     const int s0 = (w / (rows / 4)) * 4, j0 = (w % (rows / 4)) * 4;
@@ -279,41 +300,61 @@ bwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
 #pragma unroll
                     for (int a = 0; a < 4; ++a) {
                         atomicAdd(&dg[s0 + a], -wsum[a]);
-                        atomicAdd(dgC, wsum[a]);
+                        dgc_part += wsum[a];
                     }
                 } else if (w < nu + ny) {
-                    const int ww = w - nu;
-                    const int i0 = (ww / (rows / 4)) * 4, j0 = (ww % (rows / 4)) * 4;
+                    const int ww = w - nu, G = rows / 4;
+                    const int i0 = (ww / G) * 4, jb = ww % G;
                     float acc[4][4] = {};
-                    tile_nt(Qs, LDK, Ss, LDK, i0, j0, dk, acc);
+                    tile_nt(Qs, LDK, Ss, LDK, i0, jb, G, dk, acc);
 #pragma unroll
                     for (int a = 0; a < 4; ++a) {
                         float x = 0.f;
 #pragma unroll
-                        for (int bb = 0; bb < 4; ++bb) x = fmaf(acc[a][bb], dOs[(i0 + a) * LDR + j0 + bb], x);
+                        for (int bb = 0; bb < 4; ++bb) x = fmaf(acc[a][bb], dOs[(i0 + a) * LDR + jb + G * bb], x);
                         atomicAdd(&dg[i0 + a], gam[i0 + a] * x);
                     }
                 } else {
                     const int ww = w - nu - ny;
                     const int j = ww / (dk / 4), c4 = ww % (dk / 4);
                     const float4 a4 = ld4(dSs + j * LDK + 4 * c4), s4 = ld4(Ss + j * LDK + 4 * c4);
-                    atomicAdd(dgC, gam[C - 1] * dot4(a4, s4));
+                    dgc_part = fmaf(gam[C - 1], dot4(a4, s4), dgc_part);
                 }
             }
+#pragma unroll
+            for (int off = 16; off >= 1; off >>= 1) dgc_part += __shfl_xor_sync(0xffffffffu, dgc_part, off);
+            if ((tid & 31) == 0) atomicAdd(dgC, dgc_part);
         }
         __syncthreads();
 
-        // ---- pass 4: dR by back substitution, dR_s = dU_s - sum_{t>s} beta_t MA_ts dR_t ----
+        // ---- pass 4: dR by back substitution, dR_s = dU_s - sum_{t>s} beta_t MA_ts dR_t, the same way
+        //      (MA read through its transposed copy in MD, so a warp's loads are contiguous) ----
         {
-            const int j = tid / tpc, part = tid % tpc;
-            for (int s = C - 1; s >= 0; --s) {
-                float acc = 0.f;
-                for (int t = s + 1 + part; t < C; t += tpc) acc += bet[t] * MA[t * LDC + s] * dRs[t * LDR + j];
-                for (int off = tpc / 2; off >= 1; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-                if (part == 0) dRs[s * LDR + j] -= acc;
-                __syncthreads();
+            const int lane = tid & 31, warp = tid >> 5, nw = kThreads / 32;
+            const float b0 = (lane < C) ? bet[lane] : 0.f, b1 = (lane + 32 < C) ? bet[lane + 32] : 0.f;
+            for (int j0 = 2 * warp; j0 < rows; j0 += 2 * nw) {
+                const int j1 = (j0 + 1 < rows) ? j0 + 1 : j0;
+                float ra0 = (lane < C) ? dRs[lane * LDR + j0] : 0.f, rb0 = (lane < C) ? dRs[lane * LDR + j1] : 0.f;
+                float ra1 = (lane + 32 < C) ? dRs[(lane + 32) * LDR + j0] : 0.f;
+                float rb1 = (lane + 32 < C) ? dRs[(lane + 32) * LDR + j1] : 0.f;
+                for (int sidx = C - 1; sidx >= 0; --sidx) {
+                    const float m0 = (lane > sidx && lane < C) ? b0 * MD[sidx * LDC + lane] : 0.f;
+                    const float m1 = (lane + 32 > sidx && lane + 32 < C) ? b1 * MD[sidx * LDC + lane + 32] : 0.f;
+                    float sa = fmaf(m0, ra0, m1 * ra1), sb = fmaf(m0, rb0, m1 * rb1);
+#pragma unroll
+                    for (int off = 16; off >= 1; off >>= 1) {
+                        sa += __shfl_xor_sync(0xffffffffu, sa, off);
+                        sb += __shfl_xor_sync(0xffffffffu, sb, off);
+                    }
+                    if (lane == sidx) { ra0 -= sa; rb0 -= sb; }
+                    if (lane + 32 == sidx) { ra1 -= sa; rb1 -= sb; }
+                }
+                __syncwarp();
+                if (lane < C) { dRs[lane * LDR + j0] = ra0; dRs[lane * LDR + j1] = rb0; }
+                if (lane + 32 < C) { dRs[(lane + 32) * LDR + j0] = ra1; dRs[(lane + 32) * LDR + j1] = rb1; }
             }
         }
+        __syncthreads();
 
         // ---- pass 5: dV = diag(beta) dR (stored);  dbeta, d g from R;  MD = dP o E (d g from P);
         //      MA <- F = dA beta_t E (dbeta, d g from A) ----
@@ -335,18 +376,18 @@ bwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
                                         bet[t] * r4.z, bet[t] * r4.w);
                     }
                 } else {
-                    const int ww = (w - nv) % nc;
+                    const int ww = (w - nv) % nc, G = C / 4;
                     const bool isp = (w - nv) < nc;
-                    const int i0 = (ww / (C / 4)) * 4, j0 = (ww % (C / 4)) * 4;
+                    const int i0 = (ww / G) * 4, jb = ww % G;
                     // dP = dO U^T, or -dA = dR U^T
                     float acc[4][4] = {};
-                    if (j0 <= i0 + 3) tile_nt(isp ? dOs : dRs, LDR, Us, LDR, i0, j0, rows, acc);
+                    if (jb <= i0 + 3) tile_nt(isp ? dOs : dRs, LDR, Us, LDR, i0, jb, G, rows, acc);
                     float rs[4] = {0.f, 0.f, 0.f, 0.f}, cs[4] = {0.f, 0.f, 0.f, 0.f}, bs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int a = 0; a < 4; ++a)
 #pragma unroll
                         for (int bb = 0; bb < 4; ++bb) {
-                            const int t = i0 + a, s = j0 + bb;
+                            const int t = i0 + a, s = jb + G * bb;
                             if (isp) {
                                 float dd = 0.f;
                                 if (s <= t) {
@@ -375,7 +416,7 @@ bwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
 #pragma unroll
                     for (int a = 0; a < 4; ++a) {
                         if (rs[a] != 0.f) atomicAdd(&dg[i0 + a], rs[a]);
-                        if (cs[a] != 0.f) atomicAdd(&dg[j0 + a], -cs[a]);
+                        if (cs[a] != 0.f) atomicAdd(&dg[jb + G * a], -cs[a]);
                         if (!isp && bs[a] != 0.f) atomicAdd(&db[i0 + a], bs[a]);
                     }
                 }
