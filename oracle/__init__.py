@@ -72,9 +72,11 @@ class Oracle:
         L.gdn_oracle_forward_raw.argtypes = [_ptr] * 8 + [_i64] * 5 + [ctypes.c_int]
         L.gdn_oracle_decode_step_raw.argtypes = [_ptr] * 7 + [_i64] * 4 + [ctypes.c_int]
         L.gdn_oracle_backward.argtypes = [_ptr] * 14 + [_i64] * 5 + [ctypes.c_int]
+        L.gdn_oracle_forward_grouped.argtypes = [_ptr] * 8 + [_i64] * 6 + [ctypes.c_int]
         for f in ("gdn_oracle_forward", "gdn_oracle_forward_chunked", "gdn_oracle_decode_step",
                   "gdn_oracle_segment_transfer", "gdn_oracle_dense_product", "gdn_oracle_input_stage",
-                  "gdn_oracle_forward_raw", "gdn_oracle_decode_step_raw", "gdn_oracle_backward"):
+                  "gdn_oracle_forward_raw", "gdn_oracle_decode_step_raw", "gdn_oracle_backward",
+                  "gdn_oracle_forward_grouped"):
             getattr(L, f).restype = ctypes.c_int
 
     # -- the definition: token-by-token recurrence ---------------------------------
@@ -150,6 +152,24 @@ class Oracle:
         if rc != 0:
             raise RuntimeError("gdn_oracle_backward failed (%d)" % rc)
         return gq, gk, gv, gla, gbe, gS0
+
+    def forward_grouped(self, q, k, v, log_alpha, beta, S0=None, nthreads: int = 0):
+        """Grouped heads: q [B,T,Hq,dk]; k [B,T,Hkv,dk], v [B,T,Hkv,dv], gates [B,T,Hkv];
+        S0 [B,Hkv,dv,dk].  Query head h reads the memory of key-value head h // (Hq // Hkv).
+        Returns (out [B,T,Hq,dv], S_final [B,Hkv,dv,dk]) float64."""
+        q, k, v, la, be = _f32(q), _f32(k), _f32(v), _f32(log_alpha), _f32(beta)
+        B, T, Hq, dk = q.shape
+        Hkv, dv = k.shape[2], v.shape[-1]
+        assert k.shape == (B, T, Hkv, dk) and v.shape == (B, T, Hkv, dv)
+        assert la.shape == (B, T, Hkv) and be.shape == (B, T, Hkv) and Hq % Hkv == 0
+        S0 = None if S0 is None else _f64(S0)
+        out = np.empty((B, T, Hq, dv), np.float64)
+        Sf = np.empty((B, Hkv, dv, dk), np.float64)
+        rc = self.lib.gdn_oracle_forward_grouped(_p(q), _p(k), _p(v), _p(la), _p(be), _p(S0), _p(out), _p(Sf),
+                                                 B, T, Hq, Hkv, dk, dv, nthreads)
+        if rc != 0:
+            raise RuntimeError("gdn_oracle_forward_grouped failed (%d)" % rc)
+        return out, Sf
 
     # -- test-only alternative forms ----------------------------------------------
     def forward_chunked(self, q, k, v, log_alpha, beta, S0=None, chunk: int = 64, nthreads: int = 0):
@@ -261,6 +281,19 @@ def forward_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, nthreads: int 
         out[a:b] = oi[0]
         Sf[i] = si[0]
     return out, Sf
+
+
+def forward_grouped(*args, **kw):
+    return get().forward_grouped(*args, **kw)
+
+
+def decode_step_grouped(q, k, v, log_alpha, beta, S, nthreads: int = 0):
+    """Grouped-heads decode step: the forward over one token.  q [B,Hq,dk], k [B,Hkv,dk],
+    v [B,Hkv,dv], gates [B,Hkv]; S [B,Hkv,dv,dk] float64 updated in place.  Returns out [B,Hq,dv]."""
+    o, Sf = get().forward_grouped(q[:, None], k[:, None], v[:, None], log_alpha[:, None], beta[:, None], S,
+                                  nthreads=nthreads)
+    S[...] = Sf
+    return o[:, 0]
 
 
 def backward(*args, **kw):

@@ -46,6 +46,8 @@
  *   gdn_oracle_forward_raw,     the input stage followed by the recurrence
  *   gdn_oracle_decode_step_raw
  *   gdn_oracle_backward         reverse mode of the recurrence, token by token
+ *   gdn_oracle_forward_grouped  grouped heads: query heads reading the memory of
+ *                               their key-value head
  */
 #include <math.h>
 #include <stdint.h>
@@ -675,6 +677,59 @@ int gdn_oracle_backward(const float *q, const float *k, const float *v, const fl
         }
         if (dS0) memcpy(dS0 + IDX_STATE(b, h, H, dv, dk), G, sizeof(double) * ns);
         free(St); free(G); free(x); free(Gk); free(o);
+    }
+    return failed ? 2 : 0;
+}
+
+/* ------------------------------------------------------------------------
+ * Grouped heads.  H_q query heads read the memories of H_kv = H_q / G
+ * key-value heads: the memory of key-value head hk is written by its k, v
+ * and gates (layouts [B, T, H_kv, .]) by the Sec. 3.3 recurrence, and query
+ * head h = hk * G + g (g < G) reads it: o_t^(h) = S_t^(hk) q_t^(h).
+ * q, out are [B, T, H_q, .]; S0, S_final are [B, H_kv, dv, dk].  (Reading:
+ * the pages give the attention layers 8 query and 2 key-value heads but say
+ * nothing of how the memory's heads map; this is the grouped-query mapping.)
+ */
+int gdn_oracle_forward_grouped(const float *q, const float *k, const float *v, const float *log_alpha,
+                               const float *beta, const double *S0, double *out, double *S_final,
+                               int64_t B, int64_t T, int64_t Hq, int64_t Hkv, int64_t dk, int64_t dv,
+                               int nthreads) {
+    if (B < 0 || T < 0 || Hq < 0 || Hkv < 1 || dk < 1 || dv < 1 || Hq % Hkv) return 1;
+    const int64_t G = Hq / Hkv;
+    set_threads(nthreads);
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < B * Hkv; ++bh) {
+        const int64_t b = bh / Hkv, hk = bh % Hkv;
+        double *S = (double *)malloc(sizeof(double) * dv * dk);
+        double *x = (double *)malloc(sizeof(double) * dv);
+        double *o = (double *)malloc(sizeof(double) * dv);
+        if (!S || !x || !o) {
+            free(S); free(x); free(o);
+#pragma omp atomic write
+            failed = 1;
+            continue;
+        }
+        if (S0) memcpy(S, S0 + IDX_STATE(b, hk, Hkv, dv, dk), sizeof(double) * dv * dk);
+        else memset(S, 0, sizeof(double) * dv * dk);
+        for (int64_t t = 0; t < T; ++t) {
+            /* the memory's step (its output for the first query head of the group is discarded
+               and recomputed below with the others) */
+            recurrence_step(S, q + IDX_TOK(b, t, hk * G, 0, T, Hq, dk), k + IDX_TOK(b, t, hk, 0, T, Hkv, dk),
+                            v + IDX_TOK(b, t, hk, 0, T, Hkv, dv), log_alpha[IDX_GATE(b, t, hk, T, Hkv)],
+                            beta[IDX_GATE(b, t, hk, T, Hkv)], o, x, dk, dv);
+            for (int64_t g = 0; g < G; ++g) {
+                const float *qh = q + IDX_TOK(b, t, hk * G + g, 0, T, Hq, dk);
+                double *oh = out + IDX_TOK(b, t, hk * G + g, 0, T, Hq, dv);
+                for (int64_t r = 0; r < dv; ++r) {
+                    double acc = 0.0;
+                    for (int64_t c = 0; c < dk; ++c) acc += S[r * dk + c] * (double)qh[c];
+                    oh[r] = acc;
+                }
+            }
+        }
+        if (S_final) memcpy(S_final + IDX_STATE(b, hk, Hkv, dv, dk), S, sizeof(double) * dv * dk);
+        free(S); free(x); free(o);
     }
     return failed ? 2 : 0;
 }

@@ -13,6 +13,7 @@ import pytest
 import oracle as oracle_pkg
 from test_oracle import PINS
 from test_oracle_backward import BWD_PINS
+from test_oracle_grouped import GROUPED_PINS
 from test_oracle_input_stage import RAW_PINS
 
 
@@ -77,6 +78,10 @@ MUTANTS = {
     "bwd_dq_uses_previous_state": ("for (int64_t r = 0; r < dv; ++r) acc += Sn[r * dk + c] * dot[r];",
                                    "for (int64_t r = 0; r < dv; ++r) acc += Sp[r * dk + c] * dot[r];"),
     "bwd_output_grad_uses_k": ("G[r * dk + c] += dot[r] * (double)qt[c];", "G[r * dk + c] += dot[r] * (double)kt[c];"),
+    "grouped_wrong_kv_head": ("k + IDX_TOK(b, t, hk, 0, T, Hkv, dk),\n                            v + IDX_TOK(b, t, hk, 0, T, Hkv, dv)",
+                              "k + IDX_TOK(b, t, (hk + 1) % Hkv, 0, T, Hkv, dk),\n                            v + IDX_TOK(b, t, hk, 0, T, Hkv, dv)"),
+    "grouped_reads_first_query_only": ("const float *qh = q + IDX_TOK(b, t, hk * G + g, 0, T, Hq, dk);",
+                                       "const float *qh = q + IDX_TOK(b, t, hk * G, 0, T, Hq, dk);"),
     "raw_decode_swaps_q_k": ("unit_row(q + bh * dk, qk, dk);\n        unit_row(k + bh * dk, qk + dk, dk);",
                              "unit_row(k + bh * dk, qk, dk);\n        unit_row(q + bh * dk, qk + dk, dk);"),
 }
@@ -99,7 +104,7 @@ def test_planted_mistake_is_caught(tmp_path, name):
     lib = oracle_pkg.build(src=c_path, out=os.path.join(str(tmp_path), "libmutant.so"), force=True)
     mutant = oracle_pkg.Oracle(lib)
     caught = []
-    for pin in PINS + RAW_PINS + BWD_PINS:
+    for pin in PINS + RAW_PINS + BWD_PINS + GROUPED_PINS:
         try:
             pin(mutant)
         except (AssertionError, RuntimeError, FloatingPointError, ValueError):
