@@ -38,7 +38,7 @@ STATUS = {
 EXPORTS = ("gdn_forward", "gdn_decode_step", "gdn_forward_plan", "gdn_status_string", "gdn_version",
            "gdn_forward_noalloc", "gdn_scratch_release", "gdn_timing_start", "gdn_timing_stop",
            "gdn_forward_varlen", "gdn_forward_raw", "gdn_forward_varlen_raw", "gdn_decode_step_raw",
-           "gdn_backward")
+           "gdn_backward", "gdn_forward_grouped", "gdn_decode_step_grouped")
 
 # gdn_kernel_kind names, in enum order
 KERNEL_KINDS = ("prep", "chain", "transfer", "prefix", "fused", "simt", "decode", "input", "backward")
@@ -79,6 +79,10 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
         fn.argtypes = [vp] * 5 + [ctypes.POINTER(i64), i64] + [vp] * 3 + [i64] * 5 + [vp, ctypes.c_int]
         fn.restype = ctypes.c_int
     lib.gdn_backward.argtypes = [vp] * 14 + [i64] * 6 + [vp, ctypes.c_int]
+    lib.gdn_forward_grouped.argtypes = [vp] * 8 + [i64] * 7 + [vp, ctypes.c_int]
+    lib.gdn_forward_grouped.restype = ctypes.c_int
+    lib.gdn_decode_step_grouped.argtypes = [vp] * 7 + [i64] * 5 + [vp, ctypes.c_int]
+    lib.gdn_decode_step_grouped.restype = ctypes.c_int
     lib.gdn_backward.restype = ctypes.c_int
     lib.gdn_scratch_release.argtypes = []
     lib.gdn_scratch_release.restype = ctypes.c_int
@@ -273,6 +277,67 @@ def backward(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch
     if st != 0:
         raise GdnError(st, "gdn_backward")
     return dq, dk_, dv_, dla, dbe, dS0
+
+
+def forward_grouped(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
+                    beta: torch.Tensor, S0: Optional[torch.Tensor] = None, chunk: int = 64,
+                    out: Optional[torch.Tensor] = None, S_final: Optional[torch.Tensor] = None,
+                    output_final_state: bool = True, stream=None):
+    """Grouped heads: q [B,T,Hq,dk]; k [B,T,Hkv,dk], v [B,T,Hkv,dv], log_alpha, beta [B,T,Hkv];
+    S0 [B,Hkv,dv,dk] or None.  Query head h reads the memory of key-value head h // (Hq // Hkv).
+    Returns (out [B,T,Hq,dv], S_final [B,Hkv,dv,dk] or None)."""
+    lib = load()
+    B, T, Hq, dk = q.shape
+    Hkv, dv = k.shape[2], v.shape[-1]
+    for name, t, shape in (("k", k, (B, T, Hkv, dk)), ("v", v, (B, T, Hkv, dv)),
+                           ("log_alpha", log_alpha, (B, T, Hkv)), ("beta", beta, (B, T, Hkv)),
+                           ("out", out, (B, T, Hq, dv)), ("S0", S0, (B, Hkv, dv, dk)),
+                           ("S_final", S_final, (B, Hkv, dv, dk))):
+        if t is not None and tuple(t.shape) != shape:
+            raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), shape))
+    _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype or (out is not None and out.dtype != q.dtype):
+        raise TypeError("q, k, v and out must share one dtype")
+    for t in (q, k, v, log_alpha, beta, S0, out, S_final):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    if out is None:
+        out = torch.empty((B, T, Hq, dv), dtype=q.dtype, device=q.device, pin_memory=_pinned(q))
+    if S_final is None and output_final_state:
+        S_final = torch.empty((B, Hkv, dv, dk), dtype=torch.float32, device=q.device, pin_memory=_pinned(q))
+    with torch.cuda.device(q.device if q.device.type == "cuda" else torch.cuda.current_device()):
+        st = lib.gdn_forward_grouped(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S0), _ptr(out),
+                                     _ptr(S_final), B, T, Hq, Hkv, dk, dv, int(chunk),
+                                     _stream_handle(q.device, stream), _dtype_code(q))
+    if st != 0:
+        raise GdnError(st, "gdn_forward_grouped")
+    return out, S_final
+
+
+def decode_step_grouped(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_alpha: torch.Tensor,
+                        beta: torch.Tensor, S: torch.Tensor, out: Optional[torch.Tensor] = None,
+                        stream=None) -> torch.Tensor:
+    """Grouped-heads decode step: q [B,Hq,dk]; k [B,Hkv,dk], v [B,Hkv,dv], gates [B,Hkv];
+    S [B,Hkv,dv,dk] float32 updated in place.  Returns out [B,Hq,dv]."""
+    lib = load()
+    B, Hq, dk = q.shape
+    Hkv, dv = k.shape[1], v.shape[-1]
+    for name, t, shape in (("k", k, (B, Hkv, dk)), ("v", v, (B, Hkv, dv)), ("log_alpha", log_alpha, (B, Hkv)),
+                           ("beta", beta, (B, Hkv)), ("S", S, (B, Hkv, dv, dk)), ("out", out, (B, Hq, dv))):
+        if t is not None and tuple(t.shape) != shape:
+            raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), shape))
+    _dtype_code(q)
+    for t in (q, k, v, log_alpha, beta, S, out):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    if out is None:
+        out = torch.empty((B, Hq, dv), dtype=q.dtype, device=q.device, pin_memory=_pinned(q))
+    with torch.cuda.device(q.device if q.device.type == "cuda" else torch.cuda.current_device()):
+        st = lib.gdn_decode_step_grouped(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S), _ptr(out),
+                                         B, Hq, Hkv, dk, dv, _stream_handle(q.device, stream), _dtype_code(q))
+    if st != 0:
+        raise GdnError(st, "gdn_decode_step_grouped")
+    return out
 
 
 def forward_plan(B: int, T: int, H: int, dk: int, dv: int, chunk: int = 64, dtype=torch.bfloat16):

@@ -107,9 +107,71 @@ decode_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *_
     }
 }
 
+// Grouped heads: the memory of key-value head hk (its k, v, gates and state) is
+// updated once, then read by its `group` query heads hk * group .. hk * group +
+// group - 1: o_{r,g} = S'_r . q_g, from the updated rows still in registers.
+template <typename Tin, int DK>
+__global__ void __launch_bounds__(kDecodeThreads)
+decode_grouped_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
+                      const float *__restrict__ log_alpha, const float *__restrict__ beta, float *__restrict__ S,
+                      Tin *__restrict__ out, int dv, int group) {
+    constexpr int LPR = DK / 4;
+    constexpr int RPW = 32 / LPR;
+    constexpr int STRIDE = (kDecodeThreads / 32) * RPW;
+    const int64_t head = blockIdx.x;  // b * Hkv + hk
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int grp = lane / LPR, gl = lane % LPR;
+    const int row_base = blockIdx.y * decode_rows_per_cta<DK>() + warp * RPW + grp;
+
+    const float4 kf = load4(k + head * DK + 4 * gl);
+    const float alpha = expf(log_alpha[head]);
+    const float bt = beta[head];
+    float *Sh = S + head * (int64_t)dv * DK;
+    float4 s[kUnroll];
+    float vr[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const int r = row_base + u * STRIDE;
+        if (r < dv) {
+            s[u] = *reinterpret_cast<const float4 *>(Sh + (int64_t)r * DK + 4 * gl);
+            vr[u] = to_f32(v[head * dv + r]);
+        } else {
+            s[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            vr[u] = 0.f;
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+        const float a = group_sum<LPR>(dot4(s[u], kf));
+        const float ur = bt * (vr[u] - alpha * a);
+        s[u] = make_float4(fmaf(alpha, s[u].x, ur * kf.x), fmaf(alpha, s[u].y, ur * kf.y),
+                           fmaf(alpha, s[u].z, ur * kf.z), fmaf(alpha, s[u].w, ur * kf.w));
+        const int r = row_base + u * STRIDE;
+        if (r < dv) *reinterpret_cast<float4 *>(Sh + (int64_t)r * DK + 4 * gl) = s[u];
+    }
+    for (int g = 0; g < group; ++g) {
+        const int64_t qh = head * group + g;  // (b * Hkv + hk) * group + g = b * Hq + hk * group + g
+        const float4 qf = load4(q + qh * DK + 4 * gl);
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const float o = group_sum<LPR>(dot4(s[u], qf));
+            const int r = row_base + u * STRIDE;
+            if (r < dv && gl == 0) out[qh * dv + r] = from_f32<Tin>(o);
+        }
+    }
+}
+
 template <typename Tin, int DK>
 cudaError_t launch_decode_t(const DecodeProblem &p, cudaStream_t stream) {
     const int rows = decode_rows_per_cta<DK>();
+    if (p.group > 1) {
+        dim3 grid((unsigned)(p.B * (p.H / p.group)), (unsigned)((p.dv + rows - 1) / rows));
+        TimedLaunch tl_(GDN_KERNEL_DECODE, stream);
+        decode_grouped_kernel<Tin, DK><<<grid, kDecodeThreads, 0, stream>>>(
+            static_cast<const Tin *>(p.q), static_cast<const Tin *>(p.k), static_cast<const Tin *>(p.v),
+            p.log_alpha, p.beta, p.S, static_cast<Tin *>(p.out), (int)p.dv, p.group);
+        return cudaGetLastError();
+    }
     dim3 grid((unsigned)(p.B * p.H), (unsigned)((p.dv + rows - 1) / rows));
     {
         TimedLaunch tl_(GDN_KERNEL_DECODE, stream);

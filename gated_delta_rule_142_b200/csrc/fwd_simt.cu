@@ -23,6 +23,11 @@
 // Tail chunks are zero-padded with log_alpha = 0, beta = 0, which leaves the
 // recurrence unchanged.
 //
+// Grouped heads (group > 1): q and out have H heads, k, v and the gates H / group;
+// query head h reads the memory of key-value head h / group, which each of the
+// group's CTAs recomputes (S0 / S_final are per query head here; the caller
+// expands and picks them).
+//
 // For the backward pass the same kernel recomputes the forward with outputs
 // off (out == nullptr) and writes the state at the start of every chunk to a
 // checkpoint array [B*H][chunks][dv][dk].
@@ -81,7 +86,7 @@ __global__ void __launch_bounds__(kThreads)
 fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
                 const float *__restrict__ log_alpha, const float *__restrict__ beta,
                 const float *__restrict__ S0, Tin *__restrict__ out, float *__restrict__ S_final,
-                float *__restrict__ ckpt, int64_t T, int64_t H, SimtDims d) {
+                float *__restrict__ ckpt, int64_t T, int64_t H, int group, SimtDims d) {
     extern __shared__ __align__(16) float sm[];
     const int dk = d.dk, dv = d.dv, C = d.C, rows = d.rows;
     const int LDK = d.ldk, LDR = d.ldr, LDC = d.ldc;
@@ -101,13 +106,14 @@ fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
     const int slab = blockIdx.x % d.nslab;
     const int64_t b = bh / H, h = bh % H;
     const int r0 = slab * rows;
-    const int64_t tok_stride_k = H * dk, tok_stride_v = H * dv;
+    const int64_t Hkv = H / group, hk = h / group;  // key-value heads; this query head's
+    const int64_t tok_stride_q = H * dk, tok_stride_k = Hkv * dk, tok_stride_v = Hkv * dv, tok_stride_o = H * dv;
     const Tin *qb = q + (b * T * H + h) * dk;
-    const Tin *kb = k + (b * T * H + h) * dk;
-    const Tin *vb = v + (b * T * H + h) * dv + r0;
+    const Tin *kb = k + (b * T * Hkv + hk) * dk;
+    const Tin *vb = v + (b * T * Hkv + hk) * dv + r0;
     Tin *ob = out + (b * T * H + h) * dv + r0;
-    const float *lab = log_alpha + b * T * H + h;
-    const float *beb = beta + b * T * H + h;
+    const float *lab = log_alpha + b * T * Hkv + hk;
+    const float *beb = beta + b * T * Hkv + hk;
 
     // state slab <- S0 (or zero)
     for (int i = tid; i < rows * (dk / 4); i += kThreads) {
@@ -136,7 +142,7 @@ fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
             const int t = i / (dk / 4), c4 = i % (dk / 4);
             float4 qa = make_float4(0.f, 0.f, 0.f, 0.f), ka = qa;
             if (t < n) {
-                qa = load4(qb + (t0 + t) * tok_stride_k + 4 * c4);
+                qa = load4(qb + (t0 + t) * tok_stride_q + 4 * c4);
                 ka = load4(kb + (t0 + t) * tok_stride_k + 4 * c4);
             }
             *reinterpret_cast<float4 *>(Qs + t * LDK + 4 * c4) = qa;
@@ -151,8 +157,8 @@ fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
         if (tid < 32) {  // chunk-local inclusive cumsum of clamped log_alpha (C <= 64)
             float x0 = 0.f, x1 = 0.f;
             const int e0 = 2 * tid, e1 = 2 * tid + 1;
-            if (e0 < n) x0 = fmaxf(lab[(t0 + e0) * H], kLogAlphaFloor);
-            if (e1 < n) x1 = fmaxf(lab[(t0 + e1) * H], kLogAlphaFloor);
+            if (e0 < n) x0 = fmaxf(lab[(t0 + e0) * Hkv], kLogAlphaFloor);
+            if (e1 < n) x1 = fmaxf(lab[(t0 + e1) * Hkv], kLogAlphaFloor);
             float s = x0 + x1;
 #pragma unroll
             for (int off = 1; off < 32; off <<= 1) {
@@ -162,7 +168,7 @@ fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
             if (e0 < C) g[e0] = s - x1;
             if (e1 < C) g[e1] = s;
         }
-        for (int t = tid; t < C; t += kThreads) bet[t] = (t < n) ? beb[(t0 + t) * H] : 0.f;
+        for (int t = tid; t < C; t += kThreads) bet[t] = (t < n) ? beb[(t0 + t) * Hkv] : 0.f;
         __syncthreads();
         for (int t = tid; t < C; t += kThreads) {
             gam[t] = expf(g[t]);
@@ -262,7 +268,7 @@ fwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
                         const int t = i0 + a;
                         if (t < n) {
                             const float *x = Xs + t * LDR + j0;
-                            store4<Tin>(ob + (t0 + t) * tok_stride_v + j0, x[0] + acc[a][0], x[1] + acc[a][1],
+                            store4<Tin>(ob + (t0 + t) * tok_stride_o + j0, x[0] + acc[a][0], x[1] + acc[a][1],
                                         x[2] + acc[a][2], x[3] + acc[a][3]);
                         }
                     }
@@ -337,7 +343,7 @@ cudaError_t launch_t(const FwdProblem &p, int sm_count, cudaStream_t stream) {
         TimedLaunch tl_(GDN_KERNEL_SIMT, stream);
         fwd_simt_kernel<Tin><<<(unsigned)grid, kThreads, smem, stream>>>(
             static_cast<const Tin *>(p.q), static_cast<const Tin *>(p.k), static_cast<const Tin *>(p.v), p.log_alpha,
-            p.beta, p.S0, static_cast<Tin *>(p.out), p.S_final, p.ckpt, p.T, p.H, d);
+            p.beta, p.S0, static_cast<Tin *>(p.out), p.S_final, p.ckpt, p.T, p.H, p.group, d);
     }
     return cudaGetLastError();
 }

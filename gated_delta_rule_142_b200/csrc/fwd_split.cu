@@ -127,6 +127,7 @@ struct PrepArgs {
     int chunks;        // chunks per (b, h) (fixed-length problems)
     const int2 *ctab;  // packed chunk table, or nullptr for fixed-length problems
     int raw_inputs;    // q, k not yet L2-normalised; log_alpha, beta hold the gate logits
+    int group;         // grouped heads: k and the gates have H / group heads (head h / group)
 };
 
 // Writes entries (row, col) and (row, col + 1) (col even) of T diag(beta) and T diag(bgk) into
@@ -152,6 +153,7 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t T = p.T, H = p.H;
+    const int Hkv = (int)H / p.group;  // key-value heads (grouped heads), H otherwise
     SDBG_INIT
     // work items of this CTA: global chunk ids blockIdx.x, blockIdx.x + gridDim.x, ...
     const int nit = (blockIdx.x < p.items) ? (int)((p.items - 1 - blockIdx.x) / gridDim.x + 1) : 0;
@@ -209,7 +211,8 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 coords(it, b, h, t0, nt);
                 mbar_arrive_expect_tx(&bars[PB_KFULL], 2 * 8192);
                 for (int blk = 0; blk < 2; ++blk)
-                    tma_load_4d(sm + PO_QK + blk * 16384 + 8192, &tm_k, &bars[PB_KFULL], blk * 64, h, t0, b);
+                    tma_load_4d(sm + PO_QK + blk * 16384 + 8192, &tm_k, &bars[PB_KFULL], blk * 64, h / p.group, t0,
+                                b);
             };
             bool ok = true;
             if (nit > 0) {
@@ -271,7 +274,7 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             int b, h, t0, nt;
             coords(it, b, h, t0, nt);
             if (t >= nt) return -1;
-            return ((int64_t)b * T + t0 + t) * H + h;
+            return ((int64_t)b * T + t0 + t) * Hkv + (p.group == 1 ? h : h / p.group);
         };
         if (nit > 0 && pt < 64) {
             const int64_t x = gate_index(0, pt);
@@ -685,6 +688,7 @@ struct ChainArgs {
     __nv_bfloat16 *out;    // for the plain stores of partial packed chunks
     float *ckpt;           // fixed-length only, or nullptr: the state entering every chunk,
                            // [B*H][chunks][dv][dk] float32 (the backward's checkpoints)
+    int group;             // grouped heads: k and v have H / group heads (head h / group)
 };
 
 __global__ void __launch_bounds__(kChainThreads, 1)
@@ -758,8 +762,8 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 mbar_arrive_expect_tx(full, bytes);
                 for (int blk = 0; blk < 2; ++blk) {
                     tma_load_4d(st + ST_Q + blk * 8192, &tm_q, full, blk * 64, h, t0, b);
-                    tma_load_4d(st + ST_K + blk * 8192, &tm_k, full, blk * 64, h, t0, b);
-                    tma_load_4d(st + ST_V + blk * 8192, &tm_v, full, blk * 64, h, t0, b);
+                    tma_load_4d(st + ST_K + blk * 8192, &tm_k, full, blk * 64, h / p.group, t0, b);
+                    tma_load_4d(st + ST_V + blk * 8192, &tm_v, full, blk * 64, h / p.group, t0, b);
                 }
                 tma_load_2d(st + ST_W, &tm_w, full, 0, row * 128);
                 tma_load_2d(st + ST_P, &tm_p, full, 0, row * 64);
@@ -1224,8 +1228,8 @@ fwd_transfer_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 const int row = (int)(item0 + c);
                 mbar_arrive_expect_tx(full, bytes);
                 for (int blk = 0; blk < 2; ++blk) {
-                    tma_load_4d(st + TS_K + blk * 8192, &tm_k, full, blk * 64, h, t0, b);
-                    tma_load_4d(st + TS_V + blk * 8192, &tm_v, full, blk * 64, h, t0, b);
+                    tma_load_4d(st + TS_K + blk * 8192, &tm_k, full, blk * 64, h / p.group, t0, b);
+                    tma_load_4d(st + TS_V + blk * 8192, &tm_v, full, blk * 64, h / p.group, t0, b);
                 }
                 tma_load_2d(st + TS_W, &tm_w, full, 0, row * 128);
                 tma_load_2d(st + TS_TB, &tm_tb, full, 0, row * 64);
@@ -1479,8 +1483,9 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
     float *ws_gates = reinterpret_cast<float *>(ws_w + items * kTileW);
     float *seg_ws = reinterpret_cast<float *>(ws + items * kWsPerChunk);
     CUtensorMap mq, mk, mv, mo, mp, mtb, mw;
-    if (!make_map_bthd(&mq, p.q, p.B, p.T, p.H) || !make_map_bthd(&mk, p.k, p.B, p.T, p.H) ||
-        !make_map_bthd(&mv, p.v, p.B, p.T, p.H) || !make_map_bthd(&mo, p.out, p.B, p.T, p.H) ||
+    if (p.group < 1 || p.H % p.group) return cudaErrorInvalidValue;
+    if (!make_map_bthd(&mq, p.q, p.B, p.T, p.H) || !make_map_bthd(&mk, p.k, p.B, p.T, p.H / p.group) ||
+        !make_map_bthd(&mv, p.v, p.B, p.T, p.H / p.group) || !make_map_bthd(&mo, p.out, p.B, p.T, p.H) ||
         !make_map_tiles(&mp, ws_p, items, 64) || !make_map_tiles(&mtb, ws_tb, items, 64) ||
         !make_map_tiles(&mw, ws_w, items, 128))
         return cudaErrorInvalidValue;
@@ -1500,6 +1505,7 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
     pa.chunks = (int)chunks;
     pa.ctab = nullptr;
     pa.raw_inputs = p.raw_inputs;
+    pa.group = p.group;
     const int64_t pgrid =
         items < kPrepCtasPerSm * (int64_t)sm_count ? items : kPrepCtasPerSm * (int64_t)sm_count;
     {
@@ -1525,6 +1531,7 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
     a.ctab = nullptr;
     a.out = static_cast<__nv_bfloat16 *>(p.out);
     a.ckpt = p.ckpt;
+    a.group = p.group;
     if (a.nseg > 1) {
         const size_t per = (size_t)heads * (a.nseg - 1) * kD * kD;
         a.Bw = seg_ws;
@@ -1613,6 +1620,7 @@ cudaError_t launch_fwd_split_packed(const FwdProblem &p, const int64_t *cu_seqle
         pa.chunks = 0;
         pa.ctab = d_ctab;
         pa.raw_inputs = p.raw_inputs;
+        pa.group = 1;
         const int64_t pgrid =
             items < kPrepCtasPerSm * (int64_t)sm_count ? items : kPrepCtasPerSm * (int64_t)sm_count;
         TimedLaunch tl_(GDN_KERNEL_PREP, stream);
@@ -1635,6 +1643,7 @@ cudaError_t launch_fwd_split_packed(const FwdProblem &p, const int64_t *cu_seqle
     a.ctab = d_ctab;
     a.out = static_cast<__nv_bfloat16 *>(p.out);
     a.ckpt = nullptr;
+    a.group = 1;
     {
         TimedLaunch tl_(GDN_KERNEL_CHAIN, stream);
         fwd_chain_kernel<<<(unsigned)(N * H), kChainThreads, SMEM_CHAIN, stream>>>(mq, mk, mv, mo, mp, mtb, mw, a);

@@ -323,7 +323,7 @@ int run_device(FwdProblem p, const DeviceInfo &info, bool raw, cudaStream_t stre
             return st;
         }
     }
-    if (!done && path != FwdPath::Simt && gdn::fwd_tc_supported(p)) {
+    if (!done && path != FwdPath::Simt && p.group == 1 && gdn::fwd_tc_supported(p)) {
         const int nseg = gdn::fwd_tc_segments(p, info.sm_count, false);
         const size_t ws_bytes = gdn::fwd_tc_workspace_bytes(p, nseg);
         void *ws = nullptr;
@@ -870,5 +870,139 @@ extern "C" int gdn_backward(const void *q, const void *k, const void *v, const f
         (st = stg.out_back(grad_v, p.dv, nv)) || (st = stg.out_back(grad_log_alpha, p.dlog_alpha, ntok * 4)) ||
         (st = stg.out_back(grad_beta, p.dbeta, ntok * 4)) || (st = stg.out_back(grad_S0, p.dS0, nstate)))
         return st;
+    return GDN_OK;
+}
+
+extern "C" int gdn_forward_grouped(const void *q, const void *k, const void *v, const float *log_alpha,
+                                   const float *beta, const float *S0, void *out, float *S_final, int64_t B,
+                                   int64_t T, int64_t Hq, int64_t Hkv, int64_t dk, int64_t dv, int64_t chunk,
+                                   void *stream_, int dtype) {
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
+    if (B < 0 || T < 0 || Hq < 0 || Hkv < 0 || dk < 0 || dv < 0 || chunk < 0) return GDN_ERR_INVALID_SIZE;
+    if (!supported_dim(dk) || !supported_dim(dv) || !supported_chunk(chunk)) return GDN_ERR_UNSUPPORTED;
+    if ((Hq > 0) != (Hkv > 0) || (Hkv > 0 && (Hq % Hkv != 0 || Hq / Hkv > INT32_MAX))) return GDN_ERR_INVALID_SIZE;
+    const int64_t es = (dtype == GDN_F32) ? 4 : 2;
+    int64_t nq, nkv, nqk, nk, nv, nout, nstate, nxstate;
+    if (!mul3(B, T, Hq, &nq) || !mul3(B, T, Hkv, &nkv) || !mul3(nq, dk, es, &nqk) || !mul3(nkv, dk, es, &nk) ||
+        !mul3(nkv, dv, es, &nv) || !mul3(nq, dv, es, &nout) || !mul3(B * Hkv, dv, dk * 4, &nstate) ||
+        !mul3(B * Hq, dv, dk * 4, &nxstate) || nq > (INT64_MAX / 8))
+        return GDN_ERR_INVALID_SIZE;
+    if (B * Hq == 0) return GDN_OK;
+    if (nq > 0 && (!q || !k || !v || !log_alpha || !beta || !out)) return GDN_ERR_NULL_PTR;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(log_alpha) || !aligned4(beta) ||
+        !aligned16(S0) || !aligned16(out) || !aligned16(S_final))
+        return GDN_ERR_MISALIGNED;
+    const Span sq(q, nqk), sk(k, nk), sv(v, nv), sla(log_alpha, nkv * 4), sbe(beta, nkv * 4);
+    const Span s0(S0, nstate), sf(S_final, nstate), so(out, nout);
+    for (const Span &x : {sq, sk, sv, sla, sbe, s0, sf})
+        if (overlaps(so, x)) return GDN_ERR_ALIAS;
+    if (overlaps(sf, s0) && !(sf.lo == s0.lo)) return GDN_ERR_ALIAS;
+    for (const Span &x : {sq, sk, sv, sla, sbe})
+        if (overlaps(sf, x)) return GDN_ERR_ALIAS;
+    const int group = (int)(Hq / Hkv);
+    if (group == 1)
+        return gdn_forward(q, k, v, log_alpha, beta, S0, out, S_final, B, T, Hq, dk, dv, chunk, stream_, dtype);
+
+    DeviceInfo info;
+    if (int st = device_info(&info)) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    Stager stg(stream);
+    FwdProblem p;
+    int st = GDN_OK;
+    const void *dS0 = nullptr, *dout = nullptr, *dSf = nullptr;
+    if ((st = stg.in(q, nqk, true, &p.q)) || (st = stg.in(k, nk, true, &p.k)) || (st = stg.in(v, nv, true, &p.v)) ||
+        (st = stg.in(log_alpha, nkv * 4, true, reinterpret_cast<const void **>(&p.log_alpha))) ||
+        (st = stg.in(beta, nkv * 4, true, reinterpret_cast<const void **>(&p.beta))) ||
+        (st = stg.in(S0, nstate, true, &dS0)) || (st = stg.in(out, nout, false, &dout)))
+        return st;
+    if (S_final && S_final == S0) {
+        dSf = dS0;
+    } else if ((st = stg.in(S_final, nstate, false, &dSf))) {
+        return st;
+    }
+    // per-query-head copies of the states (each query head of a group recomputes its memory)
+    void *xs = nullptr;
+    if (scratch_alloc(&xs, (size_t)(2 * nxstate), stream) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_ALLOC;
+    }
+    float *S0x = static_cast<float *>(xs), *Sfx = S0x + nxstate / 4;
+    cudaError_t e = cudaSuccess;
+    if (dS0) e = gdn::launch_expand_states(static_cast<const float *>(dS0), S0x, B, Hq, group, dv * dk, stream);
+    p.S0 = dS0 ? S0x : nullptr;
+    p.out = const_cast<void *>(dout);
+    p.S_final = dSf ? Sfx : nullptr;
+    p.B = B; p.T = T; p.H = Hq; p.dk = dk; p.dv = dv; p.chunk = chunk; p.dtype = dtype;
+    p.group = group;
+    if (e == cudaSuccess) {
+        if (T == 0) {
+            if (p.S_final)
+                e = p.S0 ? cudaMemcpyAsync(Sfx, S0x, (size_t)nxstate, cudaMemcpyDeviceToDevice, stream)
+                         : cudaMemsetAsync(Sfx, 0, (size_t)nxstate, stream);
+        } else if ((st = run_device(p, info, false, stream))) {
+            cudaFreeAsync(xs, stream);
+            return st;
+        }
+    }
+    if (e == cudaSuccess && dSf)
+        e = gdn::launch_pick_states(Sfx, static_cast<float *>(const_cast<void *>(dSf)), B, Hq, group, dv * dk,
+                                    stream);
+    cudaFreeAsync(xs, stream);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_LAUNCH;
+    }
+    if ((st = stg.out_back(out, dout, nout))) return st;
+    if ((st = stg.out_back(S_final, dSf, nstate))) return st;
+    return GDN_OK;
+}
+
+extern "C" int gdn_decode_step_grouped(const void *q, const void *k, const void *v, const float *log_alpha,
+                                       const float *beta, float *S, void *out, int64_t B, int64_t Hq, int64_t Hkv,
+                                       int64_t dk, int64_t dv, void *stream_, int dtype) {
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
+    if (B < 0 || Hq < 0 || Hkv < 0 || dk < 0 || dv < 0) return GDN_ERR_INVALID_SIZE;
+    if (!supported_dim(dk) || !supported_dim(dv)) return GDN_ERR_UNSUPPORTED;
+    if ((Hq > 0) != (Hkv > 0) || (Hkv > 0 && (Hq % Hkv != 0 || Hq / Hkv > 64))) return GDN_ERR_INVALID_SIZE;
+    const int64_t es = (dtype == GDN_F32) ? 4 : 2;
+    int64_t nhq, nhk, nq, nk, nv, nout, nstate;
+    if (__builtin_mul_overflow(B, Hq, &nhq) || __builtin_mul_overflow(B, Hkv, &nhk) || !mul3(nhq, dk, es, &nq) ||
+        !mul3(nhk, dk, es, &nk) || !mul3(nhk, dv, es, &nv) || !mul3(nhq, dv, es, &nout) ||
+        !mul3(nhk, dv, dk * 4, &nstate) || nhq > (int64_t)INT32_MAX)
+        return GDN_ERR_INVALID_SIZE;
+    if (nhq == 0) return GDN_OK;
+    if (!q || !k || !v || !log_alpha || !beta || !S || !out) return GDN_ERR_NULL_PTR;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(log_alpha) || !aligned4(beta) ||
+        !aligned16(S) || !aligned16(out))
+        return GDN_ERR_MISALIGNED;
+    const Span sq(q, nq), sk(k, nk), sv(v, nv), sla(log_alpha, nhk * 4), sbe(beta, nhk * 4);
+    const Span ss(S, nstate), so(out, nout);
+    for (const Span &x : {sq, sk, sv, sla, sbe, ss})
+        if (overlaps(so, x)) return GDN_ERR_ALIAS;
+    for (const Span &x : {sq, sk, sv, sla, sbe})
+        if (overlaps(ss, x)) return GDN_ERR_ALIAS;
+
+    DeviceInfo info;
+    if (int st = device_info(&info)) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    Stager stg(stream);
+    DecodeProblem p;
+    int st = GDN_OK;
+    const void *dS = nullptr, *dout = nullptr;
+    if ((st = stg.in(q, nq, true, &p.q)) || (st = stg.in(k, nk, true, &p.k)) || (st = stg.in(v, nv, true, &p.v)) ||
+        (st = stg.in(log_alpha, nhk * 4, true, reinterpret_cast<const void **>(&p.log_alpha))) ||
+        (st = stg.in(beta, nhk * 4, true, reinterpret_cast<const void **>(&p.beta))) ||
+        (st = stg.in(S, nstate, true, &dS)) || (st = stg.in(out, nout, false, &dout)))
+        return st;
+    p.S = static_cast<float *>(const_cast<void *>(dS));
+    p.out = const_cast<void *>(dout);
+    p.B = B; p.H = Hq; p.dk = dk; p.dv = dv; p.dtype = dtype;
+    p.group = (int)(Hq / Hkv);
+    if (gdn::launch_decode(p, stream) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_LAUNCH;
+    }
+    if ((st = stg.out_back(out, p.out, nout))) return st;
+    if ((st = stg.out_back(S, p.S, nstate))) return st;
     return GDN_OK;
 }

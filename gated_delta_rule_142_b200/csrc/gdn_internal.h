@@ -43,6 +43,10 @@ struct FwdProblem {
     // here, [B*H][chunks][dv][dk] float32 (the backward's checkpoints); the CUDA-core forward
     // then also accepts out == nullptr
     float *ckpt = nullptr;
+    // grouped heads: H query heads share the memories of H / group key-value heads (k, v and the
+    // gates have H / group heads; S0 / S_final stay per query head, expanded by the caller).
+    // The two-kernel and the CUDA-core forwards take it.
+    int group = 1;
 };
 
 struct DecodeProblem {
@@ -53,6 +57,7 @@ struct DecodeProblem {
     int64_t B, H, dk, dv;
     int dtype;
     int raw_inputs = 0;  // as FwdProblem::raw_inputs
+    int group = 1;       // grouped heads: H query heads, H / group key-value heads (and states)
 };
 
 // Input stage epsilon: x / sqrt(sum x^2 + kNormEps), so that a zero vector stays zero.
@@ -60,6 +65,13 @@ constexpr float kNormEps = 1e-12f;
 
 // decode.cu
 cudaError_t launch_decode(const DecodeProblem &p, cudaStream_t stream);
+
+// grouped.cu -- per-key-value-head states <-> per-query-head copies (grouped heads):
+// dst[b, h] = src[b, h / group] for h < H, and dst[b, hk] = src[b, hk * group].
+cudaError_t launch_expand_states(const float *src, float *dst, int64_t B, int64_t H, int group, int64_t n,
+                                 cudaStream_t stream);
+cudaError_t launch_pick_states(const float *src, float *dst, int64_t B, int64_t H, int group, int64_t n,
+                               cudaStream_t stream);
 
 // input_stage.cu -- the input stage as a pass of its own, for the forwards that do not fuse
 // it: L2-normalised q, k (dtype of the problem) and log alpha, beta from the gate logits, for

@@ -250,6 +250,38 @@ int gdn_backward(const void *q, const void *k, const void *v, const float *log_a
                  int64_t H, int64_t dk, int64_t dv, int64_t chunk, void *stream, int dtype);
 
 /*
+ * Grouped heads: gdn_forward_grouped and gdn_decode_step_grouped.
+ *
+ * Hq query heads read the memories of Hkv key-value heads, G = Hq / Hkv
+ * query heads per memory.  The memory of key-value head hk is written by
+ * its own k, v, log_alpha and beta with the gdn_forward recurrence (source:
+ * the Sec. 3.3 gated-delta memory equation).  Query head h = hk * G + g
+ * (g < G) reads it: o_t^(h) = S_t^(hk) q_t^(h).  The paper's attention
+ * layers have 8 query and 2 key-value heads (Sec. 3) but it does not say how
+ * the memory's heads map; this grouped-query mapping is the reading taken.
+ *
+ * Layouts: q, out [B, T, Hq, .]; k, v [B, T, Hkv, .]; log_alpha, beta
+ * [B, T, Hkv]; S0, S_final [B, Hkv, dv, dk].  For the decode step the T
+ * axis is absent and S [B, Hkv, dv, dk] is updated in place, once per memory.
+ * Hq must be a multiple of Hkv (GDN_ERR_INVALID_SIZE otherwise); for decode
+ * G <= 64.  G = 1 is gdn_forward / gdn_decode_step.  Validation, alignment,
+ * aliasing and staging are otherwise those of the ungrouped calls.
+ *
+ * The decode kernel updates each memory once and forms the G outputs from
+ * the updated rows.  The forward runs the two-kernel tensor-core forward
+ * (bf16, dk = dv = 128, chunk = 64) or the CUDA-core forward with per-query-
+ * head work items: each query head of a group recomputes its memory.  This
+ * costs G times the memory's work, but no kernel reads another's state.
+ */
+int gdn_forward_grouped(const void *q, const void *k, const void *v, const float *log_alpha,
+                        const float *beta, const float *S0, void *out, float *S_final, int64_t B,
+                        int64_t T, int64_t Hq, int64_t Hkv, int64_t dk, int64_t dv, int64_t chunk,
+                        void *stream, int dtype);
+int gdn_decode_step_grouped(const void *q, const void *k, const void *v, const float *log_alpha,
+                            const float *beta, float *S, void *out, int64_t B, int64_t Hq,
+                            int64_t Hkv, int64_t dk, int64_t dv, void *stream, int dtype);
+
+/*
  * gdn_forward_noalloc -- gdn_forward for callers that cannot allocate device
  * memory during a call.
  *

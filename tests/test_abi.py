@@ -195,6 +195,36 @@ def test_backward_rejects_bad_arguments(lib):
     assert bwd(lib, B=0) == OK
 
 
+def test_grouped_entry_points_reject_bad_head_counts(lib):
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    vp, i64 = ctypes.c_void_p, ctypes.c_int64
+    lib.gdn_forward_grouped.argtypes = [vp] * 8 + [i64] * 7 + [vp, ctypes.c_int]
+    lib.gdn_decode_step_grouped.argtypes = [vp] * 7 + [i64] * 5 + [vp, ctypes.c_int]
+
+    def fg(Hq, Hkv, **kw):
+        a = dict(q=A, k=A + 0x1000000, v=A + 0x2000000, la=A + 0x3000000, be=A + 0x4000000, out=A + 0x5000000,
+                 dk=16, dtype=0)
+        a.update(kw)
+        return lib.gdn_forward_grouped(P(a["q"]), P(a["k"]), P(a["v"]), P(a["la"]), P(a["be"]), None, P(a["out"]),
+                                       None, 1, 8, Hq, Hkv, a["dk"], 16, 16, None, a["dtype"])
+
+    def dg(Hq, Hkv):
+        return lib.gdn_decode_step_grouped(P(A), P(A + 0x1000000), P(A + 0x2000000), P(A + 0x3000000),
+                                           P(A + 0x4000000), P(A + 0x6000000), P(A + 0x5000000), 2, Hq, Hkv, 16, 16,
+                                           None, 1)
+
+    assert fg(6, 4) == SIZE      # not a multiple
+    assert fg(4, 0) == SIZE      # no key-value heads
+    assert fg(-8, 2) == SIZE
+    assert fg(8, 2, dk=24) == UNSUP
+    assert fg(8, 2, q=None) == NULL
+    assert fg(8, 2, out=A + 0x1000000) == ALIAS
+    assert fg(0, 0) == OK
+    assert dg(6, 4) == SIZE
+    assert dg(130, 2) == SIZE    # more than 64 query heads per memory
+    assert dg(0, 0) == OK
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
 def test_valid_call_without_device_reports_device_error(lib):
     # S0 == S_final (in place) is allowed; with no CUDA device the call stops at the device check.
