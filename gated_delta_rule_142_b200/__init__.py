@@ -38,7 +38,7 @@ STATUS = {
 EXPORTS = ("gdn_forward", "gdn_decode_step", "gdn_forward_plan", "gdn_status_string", "gdn_version",
            "gdn_forward_noalloc", "gdn_scratch_release", "gdn_timing_start", "gdn_timing_stop",
            "gdn_forward_varlen", "gdn_forward_raw", "gdn_forward_varlen_raw", "gdn_decode_step_raw",
-           "gdn_backward", "gdn_forward_grouped", "gdn_decode_step_grouped")
+           "gdn_backward", "gdn_forward_grouped", "gdn_decode_step_grouped", "gdn_causal_conv")
 
 # gdn_kernel_kind names, in enum order
 KERNEL_KINDS = ("prep", "chain", "transfer", "prefix", "fused", "simt", "decode", "input", "backward")
@@ -79,6 +79,8 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
         fn.argtypes = [vp] * 5 + [ctypes.POINTER(i64), i64] + [vp] * 3 + [i64] * 5 + [vp, ctypes.c_int]
         fn.restype = ctypes.c_int
     lib.gdn_backward.argtypes = [vp] * 14 + [i64] * 6 + [vp, ctypes.c_int]
+    lib.gdn_causal_conv.argtypes = [vp] * 5 + [i64] * 4 + [vp, ctypes.c_int]
+    lib.gdn_causal_conv.restype = ctypes.c_int
     lib.gdn_forward_grouped.argtypes = [vp] * 8 + [i64] * 7 + [vp, ctypes.c_int]
     lib.gdn_forward_grouped.restype = ctypes.c_int
     lib.gdn_decode_step_grouped.argtypes = [vp] * 7 + [i64] * 5 + [vp, ctypes.c_int]
@@ -338,6 +340,38 @@ def decode_step_grouped(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, log_a
     if st != 0:
         raise GdnError(st, "gdn_decode_step_grouped")
     return out
+
+
+def causal_conv(x: torch.Tensor, weight: torch.Tensor, state_in: Optional[torch.Tensor] = None,
+                out: Optional[torch.Tensor] = None, state_out: Optional[torch.Tensor] = None,
+                want_state: bool = True, stream=None):
+    """Depthwise causal convolution: x [B,T,C] (or [B,T,H,d], flattened), weight [C,W] float32,
+    state_in [B,W-1,C] float32 or None.  Returns (y like x, state_out [B,W-1,C] or None)."""
+    lib = load()
+    B, T = x.shape[0], x.shape[1]
+    C = 1
+    for s_ in x.shape[2:]:
+        C *= s_
+    W = weight.shape[-1]
+    if tuple(weight.shape) != (C, W) or weight.dtype != torch.float32:
+        raise ValueError("weight must be float32 [C, W] with C = %d" % C)
+    for name, t in (("state_in", state_in), ("state_out", state_out)):
+        if t is not None and (tuple(t.shape) != (B, W - 1, C) or t.dtype != torch.float32):
+            raise ValueError("%s must be float32 [B, W-1, C]" % name)
+    _dtype_code(x)
+    for t in (x, weight, state_in, out, state_out):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    if out is None:
+        out = torch.empty_like(x, pin_memory=_pinned(x)) if x.device.type == "cpu" else torch.empty_like(x)
+    if state_out is None and want_state:
+        state_out = torch.empty((B, W - 1, C), dtype=torch.float32, device=x.device, pin_memory=_pinned(x))
+    with torch.cuda.device(x.device if x.device.type == "cuda" else torch.cuda.current_device()):
+        st = lib.gdn_causal_conv(_ptr(x), _ptr(weight), _ptr(state_in), _ptr(out), _ptr(state_out), B, T, C, W,
+                                 _stream_handle(x.device, stream), _dtype_code(x))
+    if st != 0:
+        raise GdnError(st, "gdn_causal_conv")
+    return out, state_out
 
 
 def forward_plan(B: int, T: int, H: int, dk: int, dv: int, chunk: int = 64, dtype=torch.bfloat16):

@@ -1006,3 +1006,62 @@ extern "C" int gdn_decode_step_grouped(const void *q, const void *k, const void 
     if ((st = stg.out_back(S, p.S, nstate))) return st;
     return GDN_OK;
 }
+
+extern "C" int gdn_causal_conv(const void *x, const float *weight, const float *state_in, void *y,
+                               float *state_out, int64_t B, int64_t T, int64_t C, int64_t W, void *stream_,
+                               int dtype) {
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
+    if (B < 0 || T < 0 || C < 0) return GDN_ERR_INVALID_SIZE;
+    if (W < 1 || W > 4) return GDN_ERR_UNSUPPORTED;
+    const int64_t es = (dtype == GDN_F32) ? 4 : 2;
+    int64_t nx, nst;
+    if (!mul3(B, T, C * es, &nx) || !mul3(B, W - 1, C * 4, &nst) || C > (INT64_MAX / 16)) return GDN_ERR_INVALID_SIZE;
+    if (B * C == 0) return GDN_OK;
+    if ((T > 0 && (!x || !y)) || !weight) return GDN_ERR_NULL_PTR;
+    if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & (uintptr_t)(es - 1)) return GDN_ERR_MISALIGNED;
+    if (!aligned4(weight) || !aligned4(state_in) || !aligned4(state_out)) return GDN_ERR_MISALIGNED;
+    const Span sx(x, nx), sy(y, nx), sw(weight, C * W * 4), si(state_in, nst), so(state_out, nst);
+    for (const Span &o : {sy, so})
+        for (const Span &i : {sx, sw})
+            if (overlaps(o, i)) return GDN_ERR_ALIAS;
+    if (overlaps(sy, si) || overlaps(sy, so)) return GDN_ERR_ALIAS;
+    if (overlaps(si, so) && si.lo != so.lo) return GDN_ERR_ALIAS;
+
+    DeviceInfo info;
+    if (int st = device_info(&info)) return st;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    Stager stg(stream);
+    int st = GDN_OK;
+    const void *dx = nullptr, *dw = nullptr, *dsi = nullptr, *dy = nullptr, *dso = nullptr;
+    if ((st = stg.in(x, nx, true, &dx)) || (st = stg.in(weight, C * W * 4, true, &dw)) ||
+        (st = stg.in(state_in, nst, true, &dsi)) || (st = stg.in(y, nx, false, &dy)))
+        return st;
+    if (state_out && state_out == state_in) {
+        dso = dsi;
+    } else if ((st = stg.in(state_out, nst, false, &dso))) {
+        return st;
+    }
+    // an in-place state update with several token tiles reads the old state from a copy
+    void *copy = nullptr;
+    cudaError_t e = cudaSuccess;
+    if (dso && dso == dsi && T > 128 && nst > 0) {
+        if (scratch_alloc(&copy, (size_t)nst, stream) != cudaSuccess) {
+            cudaGetLastError();
+            return GDN_ERR_ALLOC;
+        }
+        e = cudaMemcpyAsync(copy, dsi, (size_t)nst, cudaMemcpyDeviceToDevice, stream);
+        dsi = copy;
+    }
+    if (e == cudaSuccess)
+        e = gdn::launch_causal_conv(dx, static_cast<const float *>(dw), static_cast<const float *>(dsi),
+                                    const_cast<void *>(dy), static_cast<float *>(const_cast<void *>(dso)), B, T, C,
+                                    (int)W, dtype, stream);
+    if (copy) cudaFreeAsync(copy, stream);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_LAUNCH;
+    }
+    if ((st = stg.out_back(y, dy, nx))) return st;
+    if ((st = stg.out_back(state_out, dso, nst))) return st;
+    return GDN_OK;
+}

@@ -73,6 +73,12 @@ cudaError_t launch_expand_states(const float *src, float *dst, int64_t B, int64_
 cudaError_t launch_pick_states(const float *src, float *dst, int64_t B, int64_t H, int group, int64_t n,
                                cudaStream_t stream);
 
+// causal_conv.cu -- depthwise causal convolution over [B, T, C] (dtype), weights [C, W] float32,
+// carried states [B, W - 1, C] float32 (either may be nullptr); W in 1..4.  state_out must not
+// alias state_in when T > 128 (the host copies first).
+cudaError_t launch_causal_conv(const void *x, const float *w, const float *state_in, void *y, float *state_out,
+                               int64_t B, int64_t T, int64_t C, int W, int dtype, cudaStream_t stream);
+
 // input_stage.cu -- the input stage as a pass of its own, for the forwards that do not fuse
 // it: L2-normalised q, k (dtype of the problem) and log alpha, beta from the gate logits, for
 // `rows` (token, head) rows of dk elements; outputs may not alias inputs.

@@ -282,6 +282,30 @@ int gdn_decode_step_grouped(const void *q, const void *k, const void *v, const f
                             int64_t Hkv, int64_t dk, int64_t dv, void *stream, int dtype);
 
 /*
+ * gdn_causal_conv -- the short depthwise causal convolution applied to q, k
+ * and v before the memory (source: Sec. 3, "Canon depthwise causal
+ * convolutions are applied to q, k and v"; the paper fixes neither width,
+ * weights nor placement, so this is the plain reading).  Per batch row, channel
+ * c (C = heads x head dim) and token t:
+ *
+ *     y_t[c] = sum_{j < W} weight[c][j] * x_{t-j}[c]
+ *
+ * x_{-1} .. x_{-(W-1)} come from state_in (NULL = zeros).  No activation is
+ * applied; a residual connection is weight[c][0] + 1.
+ *
+ * Arguments: x, y [B, T, C] dtype; weight [C, W] float32 (W in 1..4);
+ * state_in, state_out [B, W-1, C] float32, the last W - 1 inputs, oldest
+ * first (NULL = zero history / not written; state_out == state_in updates in
+ * place, which is how decode (T = 1) carries it).  y may not overlap any
+ * input or state.  T = 0 only passes the state through.
+ *
+ * It is a pass of its own, bound by HBM: one read of x and one write of y.
+ */
+int gdn_causal_conv(const void *x, const float *weight, const float *state_in, void *y,
+                    float *state_out, int64_t B, int64_t T, int64_t C, int64_t W, void *stream,
+                    int dtype);
+
+/*
  * gdn_forward_noalloc -- gdn_forward for callers that cannot allocate device
  * memory during a call.
  *

@@ -283,6 +283,23 @@ def forward_varlen(q, k, v, log_alpha, beta, cu_seqlens, S0=None, nthreads: int 
     return out, Sf
 
 
+def causal_conv(x, weight, state=None):
+    """Depthwise causal convolution, float64 (the short convolution of ATMA Sec. 3 in its plain
+    reading): y_t[c] = sum_{j<W} weight[c, j] x_{t-j}[c] over x [B,T,C], the W-1 inputs before
+    t = 0 taken from state [B,W-1,C] (oldest first) or zero.  Returns (y, state after: the last
+    W-1 inputs)."""
+    x = np.asarray(x, np.float64)
+    w = np.asarray(weight, np.float64)
+    B, T, C = x.shape
+    W = w.shape[1]
+    hist = np.zeros((B, W - 1, C)) if state is None else np.asarray(state, np.float64)
+    xx = np.concatenate([hist, x], axis=1)          # token t of x is xx[:, t + W - 1]
+    y = np.zeros((B, T, C))
+    for j in range(W):
+        y += w[:, j] * xx[:, W - 1 - j: W - 1 - j + T]
+    return y, xx[:, T:T + W - 1].copy()
+
+
 def forward_grouped(*args, **kw):
     return get().forward_grouped(*args, **kw)
 
