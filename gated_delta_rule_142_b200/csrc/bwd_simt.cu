@@ -123,7 +123,7 @@ bwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
     float *dRs = Us + C * LDR;      // C x LDR  diag(dl) K dS^T, then dU, then dR
     float *MA = dRs + C * LDR;      // C x LDC  e^{g_t-g_s} (k_t . k_s) (s < t), then F
     float *MP = MA + C * LDC;       // C x LDC  P
-    float *MD = MP + C * LDC;       // C x LDC  MA transposed (for the back substitution), then dP o E
+    float *MD = MP + C * LDC;       // C x LDC  T = (I + A)^{-1}, then dP o E
     float *g = MD + C * LDC;        // C
     float *bet = g + C;             // C
     float *gam = bet + C;           // C
@@ -237,37 +237,75 @@ bwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
                             const bool keep = isa ? (s < t) : (s <= t);
                             const float x = keep ? expf(g[t] - g[s]) * acc[a][bb] : 0.f;
                             dst[t * LDC + s] = x;
-                            if (isa) MD[s * LDC + t] = x;
                         }
                 }
             }
         }
         __syncthreads();
 
-        // ---- pass 2: U by forward substitution, U_t = beta_t (v_t - X_t) - sum_{s<t} beta_t MA_ts U_s.
-        //      A warp owns value columns two at a time and keeps them in registers (lane l holds
-        //      tokens l and l + 32); each step is a shuffle reduction, with no block barrier ----
+        // ---- pass 2: T = (I + A)^{-1} into MD, A_ts = beta_t MA_ts (unit lower triangular), blocked:
+        //      16 x 16 diagonal blocks by substitution in registers (a thread per block column), then
+        //      T_10 = -T_11 (A_10 T_00) for the 16 -> 32 and 32 -> 64 merges, with Us as scratch ----
         {
-            const int lane = tid & 31, warp = tid >> 5, nw = kThreads / 32;
-            for (int j0 = 2 * warp; j0 < rows; j0 += 2 * nw) {
-                const int j1 = (j0 + 1 < rows) ? j0 + 1 : j0;
-                float ua0 = 0.f, ua1 = 0.f, ub0 = 0.f, ub1 = 0.f;  // column j0 / j1, tokens lane / lane + 32
-                for (int t = 0; t < C; ++t) {
-                    const float m0 = (lane < t) ? MA[t * LDC + lane] : 0.f;
-                    const float m1 = (lane + 32 < t) ? MA[t * LDC + lane + 32] : 0.f;
-                    float sa = fmaf(m0, ua0, m1 * ua1), sb = fmaf(m0, ub0, m1 * ub1);
+            for (int i = tid; i < C * C; i += kThreads) MD[(i / C) * LDC + (i % C)] = 0.f;
+            __syncthreads();
+            if (tid < C) {
+                const int o = (tid / 16) * 16, col = tid % 16;
+                float x[16];
 #pragma unroll
-                    for (int off = 16; off >= 1; off >>= 1) {
-                        sa += __shfl_xor_sync(0xffffffffu, sa, off);
-                        sb += __shfl_xor_sync(0xffffffffu, sb, off);
-                    }
-                    const float va = bet[t] * (Vs[t * LDR + j0] - Xs[t * LDR + j0] - sa);
-                    const float vb = bet[t] * (Vs[t * LDR + j1] - Xs[t * LDR + j1] - sb);
-                    if (lane == t) { ua0 = va; ub0 = vb; }
-                    if (lane + 32 == t) { ua1 = va; ub1 = vb; }
+                for (int r = 0; r < 16; ++r) {
+                    float acc = (r == col) ? 1.f : 0.f;
+                    const float br = bet[o + r];
+#pragma unroll
+                    for (int s2 = 0; s2 < r; ++s2) acc = fmaf(-br * MA[(o + r) * LDC + o + s2], x[s2], acc);
+                    x[r] = acc;
                 }
-                if (lane < C) { Us[lane * LDR + j0] = ua0; Us[lane * LDR + j1] = ub0; }
-                if (lane + 32 < C) { Us[(lane + 32) * LDR + j0] = ua1; Us[(lane + 32) * LDR + j1] = ub1; }
+#pragma unroll
+                for (int r = 0; r < 16; ++r) MD[(o + r) * LDC + o + col] = x[r];
+            }
+            __syncthreads();
+            float *Y = Us;  // [32][32] scratch, row stride 32
+            for (int h = 16; h < C; h *= 2) {
+                // each 2h block: Y = A_10 T_00 (h x h), then T_10 = -T_11 Y
+                const int nb = C / (2 * h), per = h * h;
+                for (int i = tid; i < nb * per; i += kThreads) {
+                    const int blk = i / per, r = (i % per) / h, cc = i % h, o = blk * 2 * h;
+                    float acc = 0.f;
+                    const float br = bet[o + h + r];
+                    for (int kk = cc; kk < h; ++kk)  // T_00 is lower triangular: rows kk >= cc
+                        acc = fmaf(br * MA[(o + h + r) * LDC + o + kk], MD[(o + kk) * LDC + o + cc], acc);
+                    Y[(blk * h + r) * 32 + cc] = acc;
+                }
+                __syncthreads();
+                for (int i = tid; i < nb * per; i += kThreads) {
+                    const int blk = i / per, r = (i % per) / h, cc = i % h, o = blk * 2 * h;
+                    float acc = 0.f;
+                    for (int kk = 0; kk <= r; ++kk)  // T_11 is lower triangular: columns kk <= r
+                        acc = fmaf(MD[(o + h + r) * LDC + o + h + kk], Y[(blk * h + kk) * 32 + cc], acc);
+                    MD[(o + h + r) * LDC + o + cc] = -acc;
+                }
+                __syncthreads();
+            }
+        }
+
+        // ---- pass 2b: U = T R, R_s = beta_s (v_s - X_s), R formed on the fly ----
+        {
+            const int nu = (C / 4) * (rows / 4);
+            for (int w = tid; w < nu; w += kThreads) {
+                const int t0l = (w / (rows / 4)) * 4, j0 = (w % (rows / 4)) * 4;
+                float acc[4][4] = {};
+                for (int s2 = 0; s2 <= t0l + 3 && s2 < C; ++s2) {
+                    const float x[4] = {MD[t0l * LDC + s2], MD[(t0l + 1) * LDC + s2], MD[(t0l + 2) * LDC + s2],
+                                        MD[(t0l + 3) * LDC + s2]};
+                    const float4 v4 = ld4(Vs + s2 * LDR + j0), x4 = ld4(Xs + s2 * LDR + j0);
+                    const float bs = bet[s2];
+                    outer4(acc, x, make_float4(bs * (v4.x - x4.x), bs * (v4.y - x4.y), bs * (v4.z - x4.z),
+                                               bs * (v4.w - x4.w)));
+                }
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+                    *reinterpret_cast<float4 *>(Us + (t0l + a) * LDR + j0) =
+                        make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
             }
         }
         __syncthreads();
@@ -327,31 +365,26 @@ bwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
         }
         __syncthreads();
 
-        // ---- pass 4: dR by back substitution, dR_s = dU_s - sum_{t>s} beta_t MA_ts dR_t, the same way
-        //      (MA read through its transposed copy in MD, so a warp's loads are contiguous) ----
+        // ---- pass 4: dR = T^T dU (in place: every tile is read before any is written) ----
         {
-            const int lane = tid & 31, warp = tid >> 5, nw = kThreads / 32;
-            const float b0 = (lane < C) ? bet[lane] : 0.f, b1 = (lane + 32 < C) ? bet[lane + 32] : 0.f;
-            for (int j0 = 2 * warp; j0 < rows; j0 += 2 * nw) {
-                const int j1 = (j0 + 1 < rows) ? j0 + 1 : j0;
-                float ra0 = (lane < C) ? dRs[lane * LDR + j0] : 0.f, rb0 = (lane < C) ? dRs[lane * LDR + j1] : 0.f;
-                float ra1 = (lane + 32 < C) ? dRs[(lane + 32) * LDR + j0] : 0.f;
-                float rb1 = (lane + 32 < C) ? dRs[(lane + 32) * LDR + j1] : 0.f;
-                for (int sidx = C - 1; sidx >= 0; --sidx) {
-                    const float m0 = (lane > sidx && lane < C) ? b0 * MD[sidx * LDC + lane] : 0.f;
-                    const float m1 = (lane + 32 > sidx && lane + 32 < C) ? b1 * MD[sidx * LDC + lane + 32] : 0.f;
-                    float sa = fmaf(m0, ra0, m1 * ra1), sb = fmaf(m0, rb0, m1 * rb1);
-#pragma unroll
-                    for (int off = 16; off >= 1; off >>= 1) {
-                        sa += __shfl_xor_sync(0xffffffffu, sa, off);
-                        sb += __shfl_xor_sync(0xffffffffu, sb, off);
-                    }
-                    if (lane == sidx) { ra0 -= sa; rb0 -= sb; }
-                    if (lane + 32 == sidx) { ra1 -= sa; rb1 -= sb; }
+            const int nr = (C / 4) * (rows / 4);
+            float acc[4][4] = {};
+            int s0l = -1, j0 = 0;
+            if (tid < nr) {  // nr <= kThreads: one tile per thread
+                s0l = (tid / (rows / 4)) * 4;
+                j0 = (tid % (rows / 4)) * 4;
+                for (int t = s0l; t < C; ++t) {
+                    const float4 m4 = ld4(MD + t * LDC + s0l);
+                    const float x[4] = {m4.x, m4.y, m4.z, m4.w};
+                    outer4(acc, x, ld4(dRs + t * LDR + j0));
                 }
-                __syncwarp();
-                if (lane < C) { dRs[lane * LDR + j0] = ra0; dRs[lane * LDR + j1] = rb0; }
-                if (lane + 32 < C) { dRs[(lane + 32) * LDR + j0] = ra1; dRs[(lane + 32) * LDR + j1] = rb1; }
+            }
+            __syncthreads();
+            if (s0l >= 0) {
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+                    *reinterpret_cast<float4 *>(dRs + (s0l + a) * LDR + j0) =
+                        make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
             }
         }
         __syncthreads();
