@@ -288,24 +288,22 @@ bwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
             }
         }
 
-        // ---- pass 2b: U = T R, R_s = beta_s (v_s - X_s), R formed on the fly ----
+        // ---- pass 2b: U = T R, R_s = beta_s (v_s - X_s), R formed on the fly; one row and four
+        //      columns per thread, so that every thread has work ----
         {
-            const int nu = (C / 4) * (rows / 4);
+            const int nu = C * (rows / 4);
             for (int w = tid; w < nu; w += kThreads) {
-                const int t0l = (w / (rows / 4)) * 4, j0 = (w % (rows / 4)) * 4;
-                float acc[4][4] = {};
-                for (int s2 = 0; s2 <= t0l + 3 && s2 < C; ++s2) {
-                    const float x[4] = {MD[t0l * LDC + s2], MD[(t0l + 1) * LDC + s2], MD[(t0l + 2) * LDC + s2],
-                                        MD[(t0l + 3) * LDC + s2]};
+                const int t = w / (rows / 4), j0 = (w % (rows / 4)) * 4;
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int s2 = 0; s2 <= t; ++s2) {
+                    const float m = MD[t * LDC + s2] * bet[s2];
                     const float4 v4 = ld4(Vs + s2 * LDR + j0), x4 = ld4(Xs + s2 * LDR + j0);
-                    const float bs = bet[s2];
-                    outer4(acc, x, make_float4(bs * (v4.x - x4.x), bs * (v4.y - x4.y), bs * (v4.z - x4.z),
-                                               bs * (v4.w - x4.w)));
+                    acc.x = fmaf(m, v4.x - x4.x, acc.x);
+                    acc.y = fmaf(m, v4.y - x4.y, acc.y);
+                    acc.z = fmaf(m, v4.z - x4.z, acc.z);
+                    acc.w = fmaf(m, v4.w - x4.w, acc.w);
                 }
-#pragma unroll
-                for (int a = 0; a < 4; ++a)
-                    *reinterpret_cast<float4 *>(Us + (t0l + a) * LDR + j0) =
-                        make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+                *reinterpret_cast<float4 *>(Us + t * LDR + j0) = acc;
             }
         }
         __syncthreads();
