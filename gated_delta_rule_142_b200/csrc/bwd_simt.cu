@@ -463,16 +463,27 @@ bwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
                 const int i0 = (ww / (dk / 4)) * 4, c0 = (ww % (dk / 4)) * 4;
                 float acc[4][4] = {};
                 if (w < nq) {
-                    // dQ = diag(gamma) dO S + (dP o E) K
-                    for (int j = 0; j < rows; ++j) {
-                        const float x[4] = {dOs[i0 * LDR + j] * gam[i0], dOs[(i0 + 1) * LDR + j] * gam[i0 + 1],
-                                            dOs[(i0 + 2) * LDR + j] * gam[i0 + 2], dOs[(i0 + 3) * LDR + j] * gam[i0 + 3]};
-                        outer4(acc, x, ld4(Ss + j * LDK + c0));
+                    // dQ = diag(gamma) dO S + (dP o E) K; the row operands are read four columns at a time
+                    for (int j = 0; j < rows; j += 4) {
+                        float xo[4][4];
+#pragma unroll
+                        for (int a = 0; a < 4; ++a) {
+                            const float4 o4 = ld4(dOs + (i0 + a) * LDR + j);
+                            const float ga = gam[i0 + a];
+                            xo[0][a] = o4.x * ga; xo[1][a] = o4.y * ga; xo[2][a] = o4.z * ga; xo[3][a] = o4.w * ga;
+                        }
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) outer4(acc, xo[jj], ld4(Ss + (j + jj) * LDK + c0));
                     }
-                    for (int s = 0; s <= i0 + 3 && s < C; ++s) {
-                        const float x[4] = {MD[i0 * LDC + s], MD[(i0 + 1) * LDC + s], MD[(i0 + 2) * LDC + s],
-                                            MD[(i0 + 3) * LDC + s]};
-                        outer4(acc, x, ld4(Ks + s * LDK + c0));
+                    for (int s = 0; s <= i0; s += 4) {  // columns s .. s + 3; D is zero above the diagonal
+                        float xd[4][4];
+#pragma unroll
+                        for (int a = 0; a < 4; ++a) {
+                            const float4 d4 = ld4(MD + (i0 + a) * LDC + s);
+                            xd[0][a] = d4.x; xd[1][a] = d4.y; xd[2][a] = d4.z; xd[3][a] = d4.w;
+                        }
+#pragma unroll
+                        for (int ss = 0; ss < 4; ++ss) outer4(acc, xd[ss], ld4(Ks + (s + ss) * LDK + c0));
                     }
                 } else {
                     // dK = (dP o E)^T Q + F^T K + F K - diag(beta gamma) dR S + diag(dl) U dS
@@ -482,10 +493,15 @@ bwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
                         outer4(acc, xd, ld4(Qs + t * LDK + c0));
                         outer4(acc, xf, ld4(Ks + t * LDK + c0));
                     }
-                    for (int s = 0; s < i0 + 3 && s < C; ++s) {
-                        const float x[4] = {MA[i0 * LDC + s], MA[(i0 + 1) * LDC + s], MA[(i0 + 2) * LDC + s],
-                                            MA[(i0 + 3) * LDC + s]};
-                        outer4(acc, x, ld4(Ks + s * LDK + c0));
+                    for (int s = 0; s <= i0; s += 4) {  // F K; F is zero on and above the diagonal
+                        float xf[4][4];
+#pragma unroll
+                        for (int a = 0; a < 4; ++a) {
+                            const float4 f4 = ld4(MA + (i0 + a) * LDC + s);
+                            xf[0][a] = f4.x; xf[1][a] = f4.y; xf[2][a] = f4.z; xf[3][a] = f4.w;
+                        }
+#pragma unroll
+                        for (int ss = 0; ss < 4; ++ss) outer4(acc, xf[ss], ld4(Ks + (s + ss) * LDK + c0));
                     }
                     float fr[4], fu[4];
 #pragma unroll
@@ -493,13 +509,21 @@ bwd_simt_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin 
                         fr[a] = -bet[i0 + a] * gam[i0 + a];
                         fu[a] = dl[i0 + a];
                     }
-                    for (int j = 0; j < rows; ++j) {
-                        const float xr[4] = {dRs[i0 * LDR + j] * fr[0], dRs[(i0 + 1) * LDR + j] * fr[1],
-                                             dRs[(i0 + 2) * LDR + j] * fr[2], dRs[(i0 + 3) * LDR + j] * fr[3]};
-                        const float xu[4] = {Us[i0 * LDR + j] * fu[0], Us[(i0 + 1) * LDR + j] * fu[1],
-                                             Us[(i0 + 2) * LDR + j] * fu[2], Us[(i0 + 3) * LDR + j] * fu[3]};
-                        outer4(acc, xr, ld4(Ss + j * LDK + c0));
-                        outer4(acc, xu, ld4(dSs + j * LDK + c0));
+                    for (int j = 0; j < rows; j += 4) {
+                        float xr[4][4], xu[4][4];
+#pragma unroll
+                        for (int a = 0; a < 4; ++a) {
+                            const float4 r4 = ld4(dRs + (i0 + a) * LDR + j), u4 = ld4(Us + (i0 + a) * LDR + j);
+                            xr[0][a] = r4.x * fr[a]; xr[1][a] = r4.y * fr[a]; xr[2][a] = r4.z * fr[a];
+                            xr[3][a] = r4.w * fr[a];
+                            xu[0][a] = u4.x * fu[a]; xu[1][a] = u4.y * fu[a]; xu[2][a] = u4.z * fu[a];
+                            xu[3][a] = u4.w * fu[a];
+                        }
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            outer4(acc, xr[jj], ld4(Ss + (j + jj) * LDK + c0));
+                            outer4(acc, xu[jj], ld4(dSs + (j + jj) * LDK + c0));
+                        }
                     }
                 }
                 float *dst = (w < nq) ? dq_acc : dk_acc;
