@@ -38,7 +38,8 @@ STATUS = {
 EXPORTS = ("gdn_forward", "gdn_decode_step", "gdn_forward_plan", "gdn_status_string", "gdn_version",
            "gdn_forward_noalloc", "gdn_scratch_release", "gdn_timing_start", "gdn_timing_stop",
            "gdn_forward_varlen", "gdn_forward_raw", "gdn_forward_varlen_raw", "gdn_decode_step_raw",
-           "gdn_backward", "gdn_forward_grouped", "gdn_decode_step_grouped", "gdn_causal_conv")
+           "gdn_backward", "gdn_forward_grouped", "gdn_decode_step_grouped", "gdn_causal_conv",
+           "gdn_device_status", "gdn_selftest_device_timeout")
 
 # gdn_kernel_kind names, in enum order
 KERNEL_KINDS = ("prep", "chain", "transfer", "prefix", "fused", "simt", "decode", "input", "backward")
@@ -79,6 +80,10 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
         fn.argtypes = [vp] * 5 + [ctypes.POINTER(i64), i64] + [vp] * 3 + [i64] * 5 + [vp, ctypes.c_int]
         fn.restype = ctypes.c_int
     lib.gdn_backward.argtypes = [vp] * 14 + [i64] * 6 + [vp, ctypes.c_int]
+    lib.gdn_device_status.argtypes = [vp]
+    lib.gdn_device_status.restype = ctypes.c_int
+    lib.gdn_selftest_device_timeout.argtypes = [vp]
+    lib.gdn_selftest_device_timeout.restype = ctypes.c_int
     lib.gdn_causal_conv.argtypes = [vp] * 5 + [i64] * 4 + [vp, ctypes.c_int]
     lib.gdn_causal_conv.restype = ctypes.c_int
     lib.gdn_forward_grouped.argtypes = [vp] * 8 + [i64] * 7 + [vp, ctypes.c_int]
@@ -383,6 +388,21 @@ def forward_plan(B: int, T: int, H: int, dk: int, dv: int, chunk: int = 64, dtyp
     if st != 0:
         raise GdnError(st, "gdn_forward_plan")
     return scratch.value, launches.value
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and return GDN_OK (0), or the status of a bounded device-side wait that
+    gave up since the last call (GDN_ERR_DEVICE_TIMEOUT = 7)."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    return int(load().gdn_device_status(_stream_handle(dev, stream)))
+
+
+def selftest_device_timeout(stream=None) -> None:
+    """Enqueue a kernel whose bounded wait gives up by design (see gdn_selftest_device_timeout)."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    st = load().gdn_selftest_device_timeout(_stream_handle(dev, stream))
+    if st != 0:
+        raise GdnError(st, "gdn_selftest_device_timeout")
 
 
 def scratch_release() -> None:

@@ -1457,6 +1457,21 @@ bool configure_once(const void *fn, uint32_t smem, std::atomic<uint64_t> &done) 
 
 }  // namespace
 
+// Reads and clears the word the kernels of this file set when a bounded wait gave up
+// (synchronous: it follows the work already enqueued on the legacy default stream's device).
+bool take_split_timeout() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_split_timeout, sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    if (v) {
+        const int zero = 0;
+        cudaMemcpyToSymbol(g_split_timeout, &zero, sizeof(int));
+    }
+    return v != 0;
+}
+
 #ifdef GDN_TC_DEBUG
 extern "C" int gdn_debug_set_split_dump(long long *ptr) {
     return cudaMemcpyToSymbol(g_split_dbg, &ptr, sizeof(ptr)) == cudaSuccess ? 0 : 1;

@@ -902,6 +902,21 @@ seg_prefix_kernel(const float *__restrict__ S0, const float *__restrict__ Bw, co
 // ---------------------------------------------------------------- host side
 }  // namespace
 
+// Reads and clears the word the kernels of this file set when a bounded wait gave up
+// (synchronous: it follows the work already enqueued on the legacy default stream's device).
+bool take_tc_timeout() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_tc_timeout, sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    if (v) {
+        const int zero = 0;
+        cudaMemcpyToSymbol(g_tc_timeout, &zero, sizeof(int));
+    }
+    return v != 0;
+}
+
 #ifdef GDN_TC_DEBUG
 extern "C" int gdn_debug_set_dump(float *ptr) {
     return cudaMemcpyToSymbol(g_dbg, &ptr, sizeof(ptr)) == cudaSuccess ? 0 : 1;

@@ -112,7 +112,15 @@ cudaMemPool_t scratch_pool(int dev) {
     return pool;
 }
 
+// GDN_TEST_FAIL_ALLOC=1 makes every scratch allocation fail: a test hook for the allocation-failure
+// paths (fallbacks and GDN_ERR_ALLOC); no kernel is involved.
+bool alloc_fails_for_test() {
+    const char *e = getenv("GDN_TEST_FAIL_ALLOC");
+    return e && strcmp(e, "1") == 0;
+}
+
 cudaError_t scratch_alloc(void **p, size_t bytes, cudaStream_t stream) {
+    if (alloc_fails_for_test()) return cudaErrorMemoryAllocation;
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
     cudaMemPool_t pool = scratch_pool(dev);
@@ -1063,5 +1071,27 @@ extern "C" int gdn_causal_conv(const void *x, const float *weight, const float *
     }
     if ((st = stg.out_back(y, dy, nx))) return st;
     if ((st = stg.out_back(state_out, dso, nst))) return st;
+    return GDN_OK;
+}
+
+extern "C" int gdn_device_status(void *stream_) {
+    DeviceInfo info;
+    if (int st = device_info(&info)) return st;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream_)) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_LAUNCH;
+    }
+    // take every word (each read clears it), then report
+    const bool a = gdn::take_split_timeout(), b = gdn::take_tc_timeout(), c = gdn::take_selftest_timeout();
+    return (a || b || c) ? GDN_ERR_DEVICE_TIMEOUT : GDN_OK;
+}
+
+extern "C" int gdn_selftest_device_timeout(void *stream_) {
+    DeviceInfo info;
+    if (int st = device_info(&info)) return st;
+    if (gdn::launch_selftest_timeout(static_cast<cudaStream_t>(stream_)) != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_LAUNCH;
+    }
     return GDN_OK;
 }

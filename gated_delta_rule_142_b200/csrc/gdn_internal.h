@@ -66,6 +66,13 @@ constexpr float kNormEps = 1e-12f;
 // decode.cu
 cudaError_t launch_decode(const DecodeProblem &p, cudaStream_t stream);
 
+// Device error words: set by a kernel whose bounded wait gave up (the kernel then aborts and
+// returns); take_* reads and clears one.  status.cu holds the self-test's word and the wait.
+bool take_split_timeout();
+bool take_tc_timeout();
+bool take_selftest_timeout();
+cudaError_t launch_selftest_timeout(cudaStream_t stream);
+
 // grouped.cu -- per-key-value-head states <-> per-query-head copies (grouped heads):
 // dst[b, h] = src[b, h / group] for h < H, and dst[b, hk] = src[b, hk * group].
 cudaError_t launch_expand_states(const float *src, float *dst, int64_t B, int64_t H, int group, int64_t n,

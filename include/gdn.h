@@ -381,6 +381,25 @@ typedef enum {
 int gdn_timing_start(void);
 int gdn_timing_stop(double *ms, int64_t *launches);
 
+/*
+ * gdn_device_status -- failure detection for waits inside the kernels.  The
+ * paper has no counterpart.  Every wait inside the library's kernels is
+ * bounded.  A kernel whose wait gives up aborts its other waits, frees its
+ * tensor memory, sets a device error word and returns; its results are
+ * wrong, but nothing hangs and the context stays usable.  This call
+ * synchronises `stream`, reads and clears the words of every kernel, and
+ * returns GDN_ERR_DEVICE_TIMEOUT if any was set since the last call, else
+ * GDN_OK (or GDN_ERR_DEVICE / GDN_ERR_LAUNCH).
+ *
+ * gdn_selftest_device_timeout -- enqueues a one-thread kernel whose bounded
+ * wait on an mbarrier phase that nothing completes gives up by design and
+ * sets its word, so that the next gdn_device_status(stream) returns
+ * GDN_ERR_DEVICE_TIMEOUT.  It exercises the reporting path without any
+ * fault; it enqueues no other work.
+ */
+int gdn_device_status(void *stream);
+int gdn_selftest_device_timeout(void *stream);
+
 /* Static, NUL-terminated description of a gdn_status value. */
 const char *gdn_status_string(int status);
 
