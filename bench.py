@@ -603,6 +603,99 @@ def run_backward(args, world, rank):
     return 0
 
 
+def run_conv(args, world, rank):
+    """gdn_causal_conv over one q/k/v-shaped tensor of the forward workload (B, T, H x d channels,
+    bf16), width 4, state carried in place; HBM-bound: x read once, y written once."""
+    import gated_delta_rule_142_b200 as gdn
+    gdn.load()
+    peaks, peak_kind = load_peaks()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    w = WORKLOADS[args.workload]
+    C, W = w.H * w.dk, 4
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed + 1000 * rank + 5)
+    x = torch.randn((w.B, w.T, C), generator=g).to(torch.bfloat16).to(dev)
+    wt = torch.randn((C, W), generator=g).to(dev)
+    st = torch.zeros((w.B, W - 1, C), device=dev)
+    y = torch.empty_like(x)
+
+    def step():
+        gdn.causal_conv(x, wt, st, out=y, state_out=st, stream=stream)
+
+    sampler = ClockSampler(dev)
+    sampler.start()
+    for _ in range(args.warmup):
+        step()
+    gdn.timing_start()
+    ms = time_region(step, args.steps, stream, world)
+    ktimes = gdn.timing_stop()
+    clocks = sampler.stop()
+    ms_step = max_over_ranks(ms / args.steps, world)
+    nbytes = 2 * w.B * w.T * C * 2 + C * W * 4 + 2 * w.B * (W - 1) * C * 4
+    gbs = nbytes / (ms_step / 1e3) / 1e9
+    if rank == 0:
+        line = {"metric": "short causal convolution GB/s vs HBM", "value": world * w.B * w.T / (ms_step / 1e3),
+                "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": "conv_w4_" + w.name, "B": w.B, "T": w.T, "channels": C, "width": W,
+                           "l2": "inputs larger than L2"},
+                "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": gbs / peaks["hbm_gbs"], "traffic": None, "peak_kind": peak_kind,
+                             "bytes_per_launch": nbytes},
+                "kernels": {k: {"ms_per_launch": v[0] / v[1], "launches_per_step": v[1] / args.steps}
+                            for k, v in ktimes.items()},
+                "clocks": clocks, "gpu_launches": sum(int(n) for _, n in ktimes.values())}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_grouped(args, world, rank):
+    """gdn_forward_grouped on the ATMA head shape: 8 query heads reading 2 key-value memories,
+    d = 128, over the forward workload's B and T (bf16, inputs in HBM)."""
+    import gated_delta_rule_142_b200 as gdn
+    gdn.load()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    w = WORKLOADS[args.workload]
+    Hq, Hkv = 8, 2
+    a = forward_inputs(w.B, w.T, Hq, w.dk, w.dv, w.dtype, seed=w.seed + 1000 * rank, alpha_mu=w.alpha_mu)
+    b = forward_inputs(w.B, w.T, Hkv, w.dk, w.dv, w.dtype, seed=w.seed + 1000 * rank + 1, s0_std=w.s0_std,
+                       alpha_mu=w.alpha_mu)
+    d = {"q": a["q"].to(dev), "k": b["k"].to(dev), "v": b["v"].to(dev), "la": b["log_alpha"].to(dev),
+         "be": b["beta"].to(dev), "S0": None if b["S0"] is None else b["S0"].to(dev)}
+    out = torch.empty((w.B, w.T, Hq, w.dv), dtype=d["q"].dtype, device=dev)
+    Sf = torch.empty((w.B, Hkv, w.dv, w.dk), dtype=torch.float32, device=dev)
+
+    def step():
+        gdn.forward_grouped(d["q"], d["k"], d["v"], d["la"], d["be"], d["S0"], chunk=w.chunk, out=out, S_final=Sf,
+                            stream=stream)
+
+    sampler = ClockSampler(dev)
+    sampler.start()
+    for _ in range(args.warmup):
+        step()
+    gdn.timing_start()
+    ms = time_region(step, args.steps, stream, world)
+    ktimes = gdn.timing_stop()
+    clocks = sampler.stop()
+    ms_step = max_over_ranks(ms / args.steps, world)
+    if rank == 0:
+        line = {"metric": "gated-delta grouped-heads forward tokens/s", "value": world * w.B * w.T / (ms_step / 1e3),
+                "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": w.dtype, "data": "synthetic",
+                "config": {"workload": "grouped_q8_kv2_" + w.name, "B": w.B, "T": w.T, "Hq": Hq, "Hkv": Hkv,
+                           "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
+                           "note": "each query head recomputes its group's memory"},
+                "kernels": {k: {"ms_per_launch": v[0] / v[1], "launches_per_step": v[1] / args.steps}
+                            for k, v in ktimes.items()},
+                "clocks": clocks, "gpu_launches": sum(int(n) for _, n in ktimes.values())}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -618,6 +711,9 @@ def main():
                     help="time gdn_forward_raw (input stage fused: raw q, k and gate logits) instead")
     ap.add_argument("--backward", action="store_true",
                     help="time gdn_backward on the workload (default workload then: the 2K training shape)")
+    ap.add_argument("--conv", action="store_true", help="time gdn_causal_conv on a q-shaped tensor instead")
+    ap.add_argument("--grouped", action="store_true",
+                    help="time gdn_forward_grouped with 8 query / 2 key-value heads instead")
     ap.add_argument("--varlen", type=int, default=0,
                     help="time packed prefill of this many sequences of mixed length instead of the forward step")
     ap.add_argument("--no-decode", action="store_true")
@@ -637,6 +733,10 @@ def main():
             return run_varlen(args, world, rank)
         if args.backward:
             return run_backward(args, world, rank)
+        if args.conv:
+            return run_conv(args, world, rank)
+        if args.grouped:
+            return run_grouped(args, world, rank)
         return run_gdn(args, world, rank, local)
     finally:
         if world > 1:
