@@ -254,6 +254,29 @@ def test_binding_validates_shapes_and_dtypes(lib):
         gdn.forward(q.transpose(1, 2), q, q, torch.zeros(1, 4, 2), torch.zeros(1, 4, 2))
 
 
+def test_bindings_of_the_wider_entry_points_validate_before_calling(lib):
+    """Shape and dtype errors in the raw, grouped, backward and convolution bindings are raised on the
+    host, before any library call (so they need no device)."""
+    z = torch.zeros
+    q = z(1, 4, 8, 16)
+    with pytest.raises(ValueError):  # gates with the query-head count instead of the key-value one
+        gdn.forward_grouped(q, z(1, 4, 2, 16), z(1, 4, 2, 16), z(1, 4, 8), z(1, 4, 8))
+    with pytest.raises(ValueError):  # S0 per query head
+        gdn.forward_grouped(q, z(1, 4, 2, 16), z(1, 4, 2, 16), z(1, 4, 2), z(1, 4, 2), S0=z(1, 8, 16, 16))
+    with pytest.raises(ValueError):
+        gdn.decode_step_grouped(z(2, 8, 16), z(2, 2, 16), z(2, 2, 16), z(2, 2), z(2, 2), z(2, 8, 16, 16))
+    with pytest.raises(ValueError):
+        gdn.forward_raw(q, z(1, 4, 8, 8), z(1, 4, 8, 16), z(1, 4, 8), z(1, 4, 8))
+    with pytest.raises(ValueError):  # grad_out shape
+        gdn.backward(q, q, q, z(1, 4, 8), z(1, 4, 8), None, z(1, 4, 8, 8))
+    with pytest.raises(TypeError):  # grad_out dtype differs from q
+        gdn.backward(q, q, q, z(1, 4, 8), z(1, 4, 8), None, q.double())
+    with pytest.raises(ValueError):  # weight [C, W] with the wrong C
+        gdn.causal_conv(z(1, 4, 32), z(16, 4))
+    with pytest.raises(ValueError):  # state [B, W-1, C]
+        gdn.causal_conv(z(1, 4, 32), z(32, 4), state_in=z(1, 4, 32))
+
+
 def test_forward_plan_argument_checks(lib):
     s, n = ctypes.c_int64(-1), ctypes.c_int(-1)
     assert lib.gdn_forward_plan(1, 8, 2, 48, 16, 16, 0, ctypes.byref(s), ctypes.byref(n)) == UNSUP
