@@ -73,10 +73,11 @@ class Oracle:
         L.gdn_oracle_decode_step_raw.argtypes = [_ptr] * 7 + [_i64] * 4 + [ctypes.c_int]
         L.gdn_oracle_backward.argtypes = [_ptr] * 14 + [_i64] * 5 + [ctypes.c_int]
         L.gdn_oracle_forward_grouped.argtypes = [_ptr] * 8 + [_i64] * 6 + [ctypes.c_int]
+        L.gdn_oracle_backward_chunked.argtypes = [_ptr] * 14 + [_i64] * 6
         for f in ("gdn_oracle_forward", "gdn_oracle_forward_chunked", "gdn_oracle_decode_step",
                   "gdn_oracle_segment_transfer", "gdn_oracle_dense_product", "gdn_oracle_input_stage",
                   "gdn_oracle_forward_raw", "gdn_oracle_decode_step_raw", "gdn_oracle_backward",
-                  "gdn_oracle_forward_grouped"):
+                  "gdn_oracle_forward_grouped", "gdn_oracle_backward_chunked"):
             getattr(L, f).restype = ctypes.c_int
 
     # -- the definition: token-by-token recurrence ---------------------------------
@@ -151,6 +152,27 @@ class Oracle:
                                           nthreads)
         if rc != 0:
             raise RuntimeError("gdn_oracle_backward failed (%d)" % rc)
+        return gq, gk, gv, gla, gbe, gS0
+
+    def backward_chunked(self, q, k, v, log_alpha, beta, S0, d_out, dS_final=None, chunk: int = 64):
+        """The reverse mode in chunkwise form (the adjoint of each line of the chunk algebra), float64;
+        same arguments and results as backward()."""
+        q, k, v, la, be = _f32(q), _f32(k), _f32(v), _f32(log_alpha), _f32(beta)
+        B, T, H, dk = q.shape
+        dv = v.shape[-1]
+        _check_shapes(q, k, v, la, be, B, T, H, dk, dv)
+        S0 = None if S0 is None else _f64(S0)
+        d_out = _f64(d_out)
+        dS_final = None if dS_final is None else _f64(dS_final)
+        gq, gk = np.empty((B, T, H, dk)), np.empty((B, T, H, dk))
+        gv = np.empty((B, T, H, dv))
+        gla, gbe = np.empty((B, T, H)), np.empty((B, T, H))
+        gS0 = np.empty((B, H, dv, dk))
+        rc = self.lib.gdn_oracle_backward_chunked(_p(q), _p(k), _p(v), _p(la), _p(be), _p(S0), _p(d_out),
+                                                  _p(dS_final), _p(gq), _p(gk), _p(gv), _p(gla), _p(gbe), _p(gS0),
+                                                  B, T, H, dk, dv, chunk)
+        if rc != 0:
+            raise RuntimeError("gdn_oracle_backward_chunked failed (%d)" % rc)
         return gq, gk, gv, gla, gbe, gS0
 
     def forward_grouped(self, q, k, v, log_alpha, beta, S0=None, nthreads: int = 0):

@@ -733,3 +733,215 @@ int gdn_oracle_forward_grouped(const float *q, const float *k, const float *v, c
     }
     return failed ? 2 : 0;
 }
+
+/* ------------------------------------------------------------------------
+ * The reverse mode in chunkwise form (test-only alternative form, float64).
+ * For a chunk of n <= C tokens with entry state S (from the forward),
+ * chunk-local g_t = sum_{r<=t} log alpha_r, gamma_t = e^{g_t}, dl_s =
+ * e^{g_last - g_s}, A_ts = beta_t e^{g_t - g_s} (k_t . k_s) (s < t),
+ * T = (I + A)^{-1}, R_t = beta_t (v_t - gamma_t S k_t), U = T R,
+ * P_ts = e^{g_t - g_s} (q_t . k_s) (s <= t), O = diag(gamma) Q S^T + P U and
+ * S' = gamma_last S + U^T diag(dl) K.  Given dO and dS' the adjoint of each
+ * line, in reverse order:
+ *   dU  = P^T dO + diag(dl) K dS'^T;   dR = T^T dU;   dV = diag(beta) dR
+ *   dP_ts = dO_t . U_s (s <= t);       dA_ts = -dR_t . U_s (s < t)
+ *   dQ  = diag(gamma) dO S + (dP o E) K,   E_ts = e^{g_t - g_s}
+ *   dK  = (dP o E)^T Q + F K + F^T K - diag(beta gamma) dR S + diag(dl) U dS',
+ *         F_ts = dA_ts beta_t E_ts
+ *   dbeta_t = dR_t . (v_t - gamma_t S k_t) + sum_s dA_ts E_ts (k_t . k_s)
+ *   dg: from gamma_t in O and R, from E in P and A, from dl and gamma_last;
+ *       dlog_alpha_r = sum_{t >= r} dg_t + dg_last
+ *   dS  = gamma_last dS' + dO^T diag(gamma) Q - dR^T diag(beta gamma) K
+ * The chunk states come from the token recurrence.  Layouts as
+ * gdn_oracle_backward.
+ */
+int gdn_oracle_backward_chunked(const float *q, const float *k, const float *v, const float *log_alpha,
+                                const float *beta, const double *S0, const double *d_out,
+                                const double *dS_final, double *dq, double *dk_out, double *dv_out,
+                                double *dlog_alpha, double *dbeta, double *dS0, int64_t B, int64_t T,
+                                int64_t H, int64_t dk, int64_t dv, int64_t C) {
+    if (B < 0 || T < 0 || H < 0 || dk < 1 || dv < 1 || C < 1) return 1;
+    const int64_t nc = (T + C - 1) / C, ns = dv * dk;
+    for (int64_t bh = 0; bh < B * H; ++bh) {
+        const int64_t b = bh / H, h = bh % H;
+        double *Sc = (double *)malloc(sizeof(double) * ns * (nc + 1));
+        double *S = (double *)malloc(sizeof(double) * ns);
+        double *dS = (double *)malloc(sizeof(double) * ns), *dSn = (double *)malloc(sizeof(double) * ns);
+        double *tmpx = (double *)malloc(sizeof(double) * dv), *tmpo = (double *)malloc(sizeof(double) * dv);
+        double *g = (double *)malloc(sizeof(double) * C * 8);
+        double *Am = (double *)malloc(sizeof(double) * C * C * 6);
+        double *Mv = (double *)malloc(sizeof(double) * C * dv * 6);
+        double *Mk = (double *)malloc(sizeof(double) * C * dk * 2);
+        if (!Sc || !S || !dS || !dSn || !tmpx || !tmpo || !g || !Am || !Mv || !Mk) {
+            free(Sc); free(S); free(dS); free(dSn); free(tmpx); free(tmpo); free(g); free(Am); free(Mv); free(Mk);
+            return 2;
+        }
+        double *gam = g + C, *dl = g + 2 * C, *bet = g + 3 * C, *dg = g + 4 * C, *db = g + 5 * C;
+        double *A = Am, *Tm = Am + C * C, *P = Am + 2 * C * C, *E = Am + 3 * C * C, *D = Am + 4 * C * C,
+               *F = Am + 5 * C * C;
+        double *X = Mv, *R = Mv + C * dv, *U = Mv + 2 * C * dv, *dO = Mv + 3 * C * dv, *dU = Mv + 4 * C * dv,
+               *dR = Mv + 5 * C * dv;
+        double *Q = Mk, *K = Mk + C * dk;
+        /* chunk-start states by the token recurrence */
+        if (S0) memcpy(S, S0 + IDX_STATE(b, h, H, dv, dk), sizeof(double) * ns);
+        else memset(S, 0, sizeof(double) * ns);
+        for (int64_t c = 0; c < nc; ++c) {
+            memcpy(Sc + c * ns, S, sizeof(double) * ns);
+            for (int64_t t = c * C; t < T && t < (c + 1) * C; ++t)
+                recurrence_step(S, q + IDX_TOK(b, t, h, 0, T, H, dk), k + IDX_TOK(b, t, h, 0, T, H, dk),
+                                v + IDX_TOK(b, t, h, 0, T, H, dv), log_alpha[IDX_GATE(b, t, h, T, H)],
+                                beta[IDX_GATE(b, t, h, T, H)], tmpo, tmpx, dk, dv);
+        }
+        if (dS_final) memcpy(dS, dS_final + IDX_STATE(b, h, H, dv, dk), sizeof(double) * ns);
+        else memset(dS, 0, sizeof(double) * ns);
+        for (int64_t c = nc - 1; c >= 0; --c) {
+            const int64_t t0 = c * C, n = (T - t0 < C) ? T - t0 : C;
+            const double *Se = Sc + c * ns;
+            double acc = 0.0;
+            for (int64_t t = 0; t < n; ++t) {
+                const int64_t gi = IDX_GATE(b, t0 + t, h, T, H);
+                acc += (double)log_alpha[gi];
+                g[t] = acc;
+                gam[t] = exp(acc);
+                bet[t] = (double)beta[gi];
+                dg[t] = 0.0;
+                db[t] = 0.0;
+                for (int64_t i = 0; i < dk; ++i) {
+                    Q[t * dk + i] = (double)q[IDX_TOK(b, t0 + t, h, i, T, H, dk)];
+                    K[t * dk + i] = (double)k[IDX_TOK(b, t0 + t, h, i, T, H, dk)];
+                }
+                for (int64_t j = 0; j < dv; ++j) dO[t * dv + j] = d_out[IDX_TOK(b, t0 + t, h, j, T, H, dv)];
+            }
+            const double gl = g[n - 1], gaml = gam[n - 1];
+            for (int64_t t = 0; t < n; ++t) dl[t] = exp(gl - g[t]);
+            for (int64_t t = 0; t < n; ++t)
+                for (int64_t s2 = 0; s2 < n; ++s2) {
+                    double kk = 0.0, qk = 0.0;
+                    for (int64_t i = 0; i < dk; ++i) {
+                        kk += K[t * dk + i] * K[s2 * dk + i];
+                        qk += Q[t * dk + i] * K[s2 * dk + i];
+                    }
+                    E[t * C + s2] = (s2 <= t) ? exp(g[t] - g[s2]) : 0.0;
+                    A[t * C + s2] = (s2 < t) ? bet[t] * E[t * C + s2] * kk : 0.0;
+                    P[t * C + s2] = (s2 <= t) ? E[t * C + s2] * qk : 0.0;
+                }
+            /* T = (I + A)^{-1} by forward substitution, column by column */
+            for (int64_t j = 0; j < n; ++j)
+                for (int64_t t = 0; t < n; ++t) {
+                    double x = (t == j) ? 1.0 : 0.0;
+                    for (int64_t s2 = 0; s2 < t; ++s2) x -= A[t * C + s2] * Tm[s2 * C + j];
+                    Tm[t * C + j] = x;
+                }
+            /* X = gamma_t S k_t, R = beta (v - X), U = T R */
+            for (int64_t t = 0; t < n; ++t)
+                for (int64_t j = 0; j < dv; ++j) {
+                    double a = 0.0;
+                    for (int64_t i = 0; i < dk; ++i) a += Se[j * dk + i] * K[t * dk + i];
+                    X[t * dv + j] = gam[t] * a;
+                    R[t * dv + j] = bet[t] * ((double)v[IDX_TOK(b, t0 + t, h, j, T, H, dv)] - X[t * dv + j]);
+                }
+            for (int64_t t = 0; t < n; ++t)
+                for (int64_t j = 0; j < dv; ++j) {
+                    double a = 0.0;
+                    for (int64_t s2 = 0; s2 <= t; ++s2) a += Tm[t * C + s2] * R[s2 * dv + j];
+                    U[t * dv + j] = a;
+                }
+            /* dU = P^T dO + diag(dl) K dS^T, with d g from dl */
+            double dgl = 0.0;
+            for (int64_t s2 = 0; s2 < n; ++s2) {
+                double w = 0.0;
+                for (int64_t j = 0; j < dv; ++j) {
+                    double a = 0.0, kd = 0.0;
+                    for (int64_t t = s2; t < n; ++t) a += P[t * C + s2] * dO[t * dv + j];
+                    for (int64_t i = 0; i < dk; ++i) kd += K[s2 * dk + i] * dS[j * dk + i];
+                    dU[s2 * dv + j] = a + dl[s2] * kd;
+                    w += U[s2 * dv + j] * dl[s2] * kd;
+                }
+                dg[s2] -= w;
+                dgl += w;
+            }
+            /* d g from the outputs' gamma_t Q S^T term and from gamma_last S in S' */
+            for (int64_t t = 0; t < n; ++t)
+                for (int64_t j = 0; j < dv; ++j) {
+                    double a = 0.0;
+                    for (int64_t i = 0; i < dk; ++i) a += Se[j * dk + i] * Q[t * dk + i];
+                    dg[t] += gam[t] * a * dO[t * dv + j];
+                }
+            for (int64_t e = 0; e < ns; ++e) dgl += gaml * dS[e] * Se[e];
+            /* dR = T^T dU */
+            for (int64_t s2 = 0; s2 < n; ++s2)
+                for (int64_t j = 0; j < dv; ++j) {
+                    double a = 0.0;
+                    for (int64_t t = s2; t < n; ++t) a += Tm[t * C + s2] * dU[t * dv + j];
+                    dR[s2 * dv + j] = a;
+                }
+            /* dV, dbeta and d g from R */
+            for (int64_t t = 0; t < n; ++t) {
+                double rb = 0.0, rg = 0.0;
+                for (int64_t j = 0; j < dv; ++j) {
+                    dv_out[IDX_TOK(b, t0 + t, h, j, T, H, dv)] = bet[t] * dR[t * dv + j];
+                    rb += dR[t * dv + j] * ((double)v[IDX_TOK(b, t0 + t, h, j, T, H, dv)] - X[t * dv + j]);
+                    rg += dR[t * dv + j] * X[t * dv + j];
+                }
+                db[t] += rb;
+                dg[t] -= bet[t] * rg;
+            }
+            /* dP o E (= D), F from dA; dbeta and d g from P and A */
+            for (int64_t t = 0; t < n; ++t)
+                for (int64_t s2 = 0; s2 < n; ++s2) {
+                    double dp = 0.0, da = 0.0;
+                    for (int64_t j = 0; j < dv; ++j) {
+                        dp += dO[t * dv + j] * U[s2 * dv + j];
+                        da -= dR[t * dv + j] * U[s2 * dv + j];
+                    }
+                    D[t * C + s2] = (s2 <= t) ? dp * E[t * C + s2] : 0.0;
+                    F[t * C + s2] = (s2 < t) ? da * bet[t] * E[t * C + s2] : 0.0;
+                    if (s2 <= t) {
+                        dg[t] += dp * P[t * C + s2];
+                        dg[s2] -= dp * P[t * C + s2];
+                    }
+                    if (s2 < t) {
+                        double kk = 0.0;
+                        for (int64_t i = 0; i < dk; ++i) kk += K[t * dk + i] * K[s2 * dk + i];
+                        db[t] += da * E[t * C + s2] * kk;
+                        dg[t] += da * A[t * C + s2];
+                        dg[s2] -= da * A[t * C + s2];
+                    }
+                }
+            /* dQ, dK */
+            for (int64_t t = 0; t < n; ++t)
+                for (int64_t i = 0; i < dk; ++i) {
+                    double aq = 0.0, ak = 0.0;
+                    for (int64_t j = 0; j < dv; ++j) {
+                        aq += gam[t] * dO[t * dv + j] * Se[j * dk + i];
+                        ak += -bet[t] * gam[t] * dR[t * dv + j] * Se[j * dk + i] + dl[t] * U[t * dv + j] * dS[j * dk + i];
+                    }
+                    for (int64_t s2 = 0; s2 < n; ++s2) {
+                        aq += D[t * C + s2] * K[s2 * dk + i];
+                        ak += D[s2 * C + t] * Q[s2 * dk + i] + F[t * C + s2] * K[s2 * dk + i] + F[s2 * C + t] * K[s2 * dk + i];
+                    }
+                    dq[IDX_TOK(b, t0 + t, h, i, T, H, dk)] = aq;
+                    dk_out[IDX_TOK(b, t0 + t, h, i, T, H, dk)] = ak;
+                }
+            /* d log alpha and dbeta */
+            for (int64_t r = 0; r < n; ++r) {
+                double sum = dgl;
+                for (int64_t t = r; t < n; ++t) sum += dg[t];
+                dlog_alpha[IDX_GATE(b, t0 + r, h, T, H)] = sum;
+                dbeta[IDX_GATE(b, t0 + r, h, T, H)] = db[r];
+            }
+            /* dS for the previous chunk */
+            for (int64_t j = 0; j < dv; ++j)
+                for (int64_t i = 0; i < dk; ++i) {
+                    double a = gaml * dS[j * dk + i];
+                    for (int64_t t = 0; t < n; ++t)
+                        a += gam[t] * dO[t * dv + j] * Q[t * dk + i] - bet[t] * gam[t] * dR[t * dv + j] * K[t * dk + i];
+                    dSn[j * dk + i] = a;
+                }
+            memcpy(dS, dSn, sizeof(double) * ns);
+        }
+        if (dS0) memcpy(dS0 + IDX_STATE(b, h, H, dv, dk), dS, sizeof(double) * ns);
+        free(Sc); free(S); free(dS); free(dSn); free(tmpx); free(tmpo); free(g); free(Am); free(Mv); free(Mk);
+    }
+    return 0;
+}

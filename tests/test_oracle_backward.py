@@ -111,8 +111,23 @@ def pin_backward_split(orc):
     assert rel_err(first[5], full[5]) < 1e-12
 
 
+def pin_backward_chunked(orc):
+    """The chunkwise adjoint (the algebra the CUDA kernel uses) equals the token-by-token reverse mode for
+    chunk lengths 1 .. 64, with a ragged last chunk."""
+    rng = np.random.default_rng(36)
+    B, T, H, dk, dv = 1, 23, 2, 8, 5
+    q, k, v, la, be, S0 = rand_inputs(rng, B, T, H, dk, dv)
+    dO = rng.standard_normal((B, T, H, dv))
+    dSf = rng.standard_normal((B, H, dv, dk))
+    ref = orc.backward(q, k, v, la, be, S0, dO, dSf)
+    for C in (1, 2, 3, 7, 16, 64):
+        got = orc.backward_chunked(q, k, v, la, be, S0, dO, dSf, chunk=C)
+        for a, b in zip(got, ref):
+            assert rel_err(a, b) < 1e-10, C
+
+
 BWD_PINS = [pin_backward_finite_differences, pin_backward_frozen_state, pin_backward_linearity,
-            pin_backward_split]
+            pin_backward_split, pin_backward_chunked]
 
 
 @pytest.fixture(scope="module")

@@ -82,6 +82,11 @@ MUTANTS = {
                               "k + IDX_TOK(b, t, (hk + 1) % Hkv, 0, T, Hkv, dk),\n                            v + IDX_TOK(b, t, hk, 0, T, Hkv, dv)"),
     "grouped_reads_first_query_only": ("const float *qh = q + IDX_TOK(b, t, hk * G + g, 0, T, Hq, dk);",
                                        "const float *qh = q + IDX_TOK(b, t, hk * G, 0, T, Hq, dk);"),
+    "bwdc_dR_without_transpose": ("for (int64_t t = s2; t < n; ++t) a += Tm[t * C + s2] * dU[t * dv + j];",
+                                  "for (int64_t t = s2; t < n; ++t) a += Tm[s2 * C + t] * dU[t * dv + j];"),
+    "bwdc_dl_gradient_sign": ("dg[s2] -= w;\n                dgl += w;", "dg[s2] += w;\n                dgl += w;"),
+    "bwdc_F_without_beta": ("F[t * C + s2] = (s2 < t) ? da * bet[t] * E[t * C + s2] : 0.0;",
+                            "F[t * C + s2] = (s2 < t) ? da * E[t * C + s2] : 0.0;"),
     "raw_decode_swaps_q_k": ("unit_row(q + bh * dk, qk, dk);\n        unit_row(k + bh * dk, qk + dk, dk);",
                              "unit_row(k + bh * dk, qk, dk);\n        unit_row(q + bh * dk, qk + dk, dk);"),
 }
