@@ -27,6 +27,7 @@ import argparse
 import dataclasses
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -42,7 +43,10 @@ from gdn_inputs import (WORKLOADS, as_f32_numpy, decode_inputs, forward_inputs, 
                         varlen_inputs)
 
 FWD_WORKLOAD = "fwd_bf16_b1h16_t64k_d128"
-DEC_WORKLOAD = "decode_bf16_b64h16_d128_x1024"
+# the decode workload of the survey (state 67 MB, 134 MB read and written per step, partly served by the
+# 126 MB L2) and one whose state (268 MB, 537 MB per step) is twice L2, so that its HBM fraction is not
+# helped by the cache
+DEC_WORKLOADS = ("decode_bf16_b64h16_d128_x1024", "decode_bf16_b256h16_d128_x256")
 METRIC = "gated-delta forward tokens/s & TFLOP/s vs BF16 roofline; decode GB/s vs HBM peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -65,22 +69,53 @@ def decode_bytes_per_head_step(dk, dv, es):
     return 2 * dk * dv * 4 + (2 * dk + 2 * dv) * es + 8
 
 
-# DRAM bytes (read + write) per token-head that one ncu capture of each kernel kind measured, from
-# the summaries in profiles/ (fwd_chain_b8h16_t2k_d128.md, fwd_prep_b8h16_t2k_d128.md,
-# fwd_transfer_b1h16_t16k_s4.md).  For the transfer kind the unit is a token-head of the
-# transferred segments (covering both of its runs, which one CTA runs together).  Kept only while
-# those kernels are unchanged.
-NCU_TRAFFIC_PER_TOKEN_HEAD = {"chain": 400.0e6 / 262144, "prep": 225.4e6 / 262144, "transfer": 181.7e6 / 196608}
+# Counted FLOP of each kernel kind per token-head: the method's contractions assigned to the kernel
+# that performs them.  The prep kernel forms K K^T, Q K^T (one [Q;K] K^T product) and W = T diag(beta
+# gamma) K; the chain kernel forms Ut = T diag(beta) V, P U, W S^T, Q S^T and U^T Ktil.  They sum to
+# fwd_flop_per_token_head.  The transfer and prefix kernels exist only to cut long sequences into
+# segments: their arithmetic is overhead and earns no count.
+def counted_flop_per_token_head(kind, dk, dv, C):
+    if kind == "prep":
+        return 6 * C * dk
+    if kind == "chain":
+        return 4 * C * dv + 6 * dk * dv
+    if kind == "fused":
+        return fwd_flop_per_token_head(dk, dv, C)
+    return 0
 
 
-# DRAM bytes (read + write) per decode launch from the ncu capture summarised in
-# profiles/decode_bf16_b64h16_d128.md: about half of the 134 MB state stays in the 126 MB L2 from
-# one step to the next, so DRAM moves 0.58x the algorithmic bytes.
-NCU_DECODE_TRAFFIC = {"decode_bf16_b64h16_d128_x1024": 78.2e6}
+def source_sha(relpath):
+    """First 16 hex digits of the sha256 of a source file of the repository."""
+    import hashlib
+    with open(os.path.join(ROOT, relpath), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def measured_traffic(profile):
+    """DRAM bytes (read + write) per unit that an ncu capture recorded for each kernel kind, from the
+    machine-readable lines of a summary under profiles/:
+        traffic <kind> <source file> <sha256[:16] of that file at capture time> <bytes per unit>
+    A kind whose source has changed since the capture is left out (its traffic is unknown)."""
+    path = os.path.join(ROOT, "profiles", profile)
+    out = {}
+    if not os.path.exists(path):
+        return out
+    with open(path) as f:
+        for line in f:
+            m = re.match(r"\s*traffic\s+(\S+)\s+(\S+)\s+([0-9a-f]{16})\s+([0-9.eE+]+)\s*$", line)
+            if m and os.path.exists(os.path.join(ROOT, m.group(2))) and source_sha(m.group(2)) == m.group(3):
+                out[m.group(1)] = float(m.group(4))
+    return out
+
+
+FWD_TRAFFIC_PROFILE = "fwd_traffic_b1h16_t16k_d128.md"
+DECODE_TRAFFIC_PROFILE = "decode_traffic_d128.md"
 
 
 def kernel_units(kind, w, nseg):
-    """Token-heads one launch of a kernel kind processes (the unit of NCU_TRAFFIC_PER_TOKEN_HEAD)."""
+    """Units one launch of a kernel kind processes, the unit its measured traffic is quoted per:
+    token-heads (prep, chain, fused), token-heads of the transferred segments (transfer), segment
+    boundaries times heads (prefix)."""
     nth = w.B * w.T * w.H
     if kind in ("prep", "chain", "fused"):
         return nth
@@ -88,46 +123,30 @@ def kernel_units(kind, w, nseg):
         chunks = -(-w.T // w.chunk)
         seg_len = -(-chunks // max(nseg, 1))
         return min(w.T, (nseg - 1) * seg_len * w.chunk) * w.B * w.H if nseg > 1 else 0
+    if kind == "prefix":
+        return w.B * w.H * max(nseg - 1, 0)
     return 0
 
 
-def kernel_work(kind, w, es, nseg):
-    """Algorithmic (flop, HBM bytes) of ONE launch of a forward kernel kind on workload w.
-
-    Two-kernel tensor-core forward, per token and head (C = chunk, d = dk = dv):
-      prep     G = [Q;K]K^T and W = T diag(beta gamma) K: 6 C d flop (the 64x64 inverse is not
-               counted); reads q, k and two gates, writes P, T diag(beta) (2C bytes each), W^T
-               (2 dk bytes) and the 8-byte gate record.
-      chain    Ut = T diag(beta) V, U = Ut - W S^T, S update, Q S^T, P U: 6 dk dv + 4 C dv flop;
-               reads q, k, v, P, TB, W^T, the gate record, writes out.
-      transfer zero-state run (Ut, U, S: 2 C dv + 4 dk dv; reads k, v, TB, W^T, record) plus
-               identity run (U, S: 4 dk dv; reads k, W^T, record) over the tokens of segments
-               0..nseg-2.
-      prefix   S_{p+1} = S_p M_p + B_p: 2 dv dk^2 flop per segment boundary and head; reads M, B,
-               writes the entry state.
-    """
+def kernel_design_bytes(kind, w, es, nseg):
+    """HBM bytes ONE launch of a kernel kind moves by this design (inputs, outputs and the two-kernel
+    forward's per-chunk workspace: P and T diag(beta) at 2C bytes per token each, W^T at 2 dk, the
+    gate record at 528 B per chunk).  This is the design's own traffic, not the algorithmic bytes:
+    the compulsory bytes of the step are fwd_bytes."""
     C, dk, dv = w.chunk, w.dk, w.dv
     nth = w.B * w.T * w.H
-    heads = w.B * w.H
-    chunks = -(-w.T // C)
-    seg_len = -(-chunks // max(nseg, 1))
-    tr_tokens = min(w.T, (nseg - 1) * seg_len * C) * heads if nseg > 1 else 0
-    tile = 2 * C + 2 * C + 2 * dk + 8.25  # P, TB, W^T, gate record (528 B per chunk) bytes per token
+    tile = 2 * C + 2 * C + 2 * dk + 528.0 / C
     if kind == "prep":
-        # reads q, k, gates; writes P, TB, W^T and the gate record
-        return nth * 6 * C * dk, nth * (2 * dk * es + 8 + tile)
+        return nth * (2 * dk * es + 8 + tile)
     if kind == "chain":
-        # reads q, k, v, P, TB, W^T, the gate record; writes out
-        return nth * (6 * dk * dv + 4 * C * dv), nth * ((2 * dk + 2 * dv) * es + tile)
+        return nth * ((2 * dk + 2 * dv) * es + tile)
     if kind == "transfer":
-        flop = tr_tokens * ((2 * C * dv + 4 * dk * dv) + 4 * dk * dv)
-        by = tr_tokens * (((dk + dv) * es + 2 * C + 2 * dk + 8) + (dk * es + 2 * dk + 8))
-        return flop, by
+        return kernel_units(kind, w, nseg) * ((dk + dv) * es + tile - 2 * C)
     if kind == "prefix":
-        return heads * (nseg - 1) * 2 * dv * dk * dk, heads * (nseg - 1) * 3 * dv * dk * 4
+        return kernel_units(kind, w, nseg) * 3 * dv * dk * 4
     if kind == "fused":
-        return nth * fwd_flop_per_token_head(dk, dv, C), nth * ((2 * dk + 2 * dv) * es + 8)
-    return 0, 0
+        return nth * ((2 * dk + 2 * dv) * es + 8)
+    return 0
 
 
 # ---------------------------------------------------------------- helpers
@@ -237,6 +256,18 @@ def cpu_info():
     return model, len(os.sched_getaffinity(0))
 
 
+def fwd_config(w, raw, world):
+    """The `config` object of the forward line, shared by the GPU arm and the reference arm so that
+    both describe the same workload in the same words."""
+    es = 2 if w.dtype == "bf16" else 4
+    nbytes = fwd_bytes(w.B, w.T, w.H, w.dk, w.dv, es, w.s0_std is not None, True)
+    return {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
+            "input_dtype": w.dtype, "state_dtype": "f32",
+            "input_stage": "fused (raw q, k and gate logits)" if raw else "none (unit q, k; gates)",
+            "parallelism": "replicas" if world > 1 else "single",
+            "l2": "inputs larger than L2 (%.2f GB read+written per step)" % (nbytes / 1e9)}
+
+
 # ---------------------------------------------------------------- oracle timing
 def oracle_forward_sample(w, budget_s: float):
     """Float64 oracle on a bounded prefix of the forward workload (all heads of batch row 0,
@@ -244,7 +275,7 @@ def oracle_forward_sample(w, budget_s: float):
     Returns (tokens/s, cores, description)."""
     import oracle
     _, cores = cpu_info()
-    threads = min(cores, w.B * w.H)
+    threads = min(cores, w.B * w.H)  # the oracle parallelises over (b, h) only
 
     def run(Tp):
         inp = forward_inputs(1, Tp, w.H, w.dk, w.dv, w.dtype, seed=w.seed, alpha_mu=w.alpha_mu)
@@ -275,14 +306,14 @@ def run_reference(args, world, rank):
         times.append(dt)
         toks.append(Tp)
     value = sum(toks) / sum(times)
+    sample = desc + "; CPU: " + model
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * statistics.mean(times),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
-                   "input_dtype": w.dtype, "parallelism": "replicas"},
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                         "sample": desc + "; CPU: " + model},
+        "config": fwd_config(w, False, int(os.environ.get("WORLD_SIZE", "1"))),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "host_cores": cores,
+                         "oracle_threads": threads, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "gpu_launches": 0,
     }
@@ -303,6 +334,74 @@ def time_region(fn, steps, stream, world):
     torch.cuda.synchronize()
     barrier(world)
     return start.elapsed_time(end)  # ms
+
+
+def time_decode(gdn, wd, dev, stream, world, rank, warmup, peaks, peak_kind):
+    """Times wd.steps consecutive gdn_decode_step launches (replayed from a CUDA graph) on a decode
+    workload whose inputs are all resident in HBM; returns its object of the JSON line."""
+    dsteps = wd.steps
+    di = decode_inputs(dsteps, wd.B, wd.H, wd.dk, wd.dv, wd.dtype, seed=wd.seed + 1000 * rank, s0_std=wd.s0_std)
+    dd = {k: v.to(dev) for k, v in di.items()}
+    del di
+    S = dd["S"].clone()
+    dout = torch.empty((dsteps, wd.B, wd.H, wd.dv), dtype=dd["q"].dtype, device=dev)
+
+    def dec_run():
+        for t in range(dsteps):
+            gdn.decode_step(dd["q"][t], dd["k"][t], dd["v"][t], dd["log_alpha"][t], dd["beta"][t], S,
+                            out=dout[t], stream=stream)
+
+    for _ in range(max(1, warmup // 3)):
+        dec_run()
+    # The launches (each still one gdn_decode_step call through the C ABI) are captured once in a CUDA
+    # graph and replayed: a Python call costs about as long as one decode kernel, and host overhead
+    # must not leave the GPU idle inside the timed region.
+    replay = dec_run
+    graph = None
+    try:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            cap = torch.cuda.current_stream()
+            for t in range(dsteps):
+                gdn.decode_step(dd["q"][t], dd["k"][t], dd["v"][t], dd["log_alpha"][t], dd["beta"][t], S,
+                                out=dout[t], stream=cap)
+        graph.replay()
+        torch.cuda.synchronize()
+        replay = graph.replay
+    except RuntimeError:
+        torch.cuda.synchronize()
+    dms = time_region(replay, 1, stream, world) / dsteps
+    dms = max_over_ranks(dms, world)
+    des = 2 if wd.dtype == "bf16" else 4
+    dbytes = wd.B * wd.H * decode_bytes_per_head_step(wd.dk, wd.dv, des)
+    dgbs = dbytes / (dms / 1e3) / 1e9
+    tr_unit = measured_traffic(DECODE_TRAFFIC_PROFILE).get("decode_b%d" % wd.B)
+    res = {"workload": wd.name, "steps": dsteps, "us_per_step": dms * 1e3,
+           "state_bytes": wd.B * wd.H * wd.dv * wd.dk * 4,
+           "launch": "cuda_graph" if replay is not dec_run else "eager",
+           "tokens_per_s": world * wd.B / (dms / 1e3), "GB_per_s": dgbs,
+           "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                        "frac": dgbs / peaks["hbm_gbs"],
+                        "traffic": None if tr_unit is None else tr_unit * wd.B * wd.H,
+                        "traffic_source": "profiles/" + DECODE_TRAFFIC_PROFILE,
+                        "peak_kind": peak_kind, "bytes_per_launch": dbytes},
+           "launches": dsteps}
+    del dd, S, dout, graph, replay
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_decode_only(args, world, rank):
+    """One decode workload alone (for profiler captures of the decode kernel)."""
+    import gated_delta_rule_142_b200 as gdn
+    gdn.load()
+    peaks, peak_kind = load_peaks()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    res = time_decode(gdn, WORKLOADS[args.decode_only], dev, torch.cuda.current_stream(dev), world, rank,
+                      args.warmup, peaks, peak_kind)
+    if rank == 0:
+        print(json.dumps({"decode": res}), flush=True)
+    return 0
 
 
 def run_gdn(args, world, rank, local):
@@ -329,10 +428,10 @@ def run_gdn(args, world, rank, local):
         r = raw_inputs((w.B, w.T, w.H), w.dk, w.dv, w.dtype, seed=w.seed + 1000 * rank,
                        s0_shape=(w.B, w.H, w.dv, w.dk), s0_std=w.s0_std, alpha_mu=w.alpha_mu)
         inp = {"q": r["q"], "k": r["k"], "v": r["v"], "log_alpha": r["x_alpha"], "beta": r["x_beta"], "S0": r["S0"]}
-        w = dataclasses.replace(w, name=w.name + "_raw")
     else:
         inp = forward_inputs(w.B, w.T, w.H, w.dk, w.dv, w.dtype, seed=w.seed + 1000 * rank, s0_std=w.s0_std,
                              alpha_mu=w.alpha_mu)
+    w_cfg = w  # the workload as the reference arm names it (the raw flag goes into the config)
     fwd = gdn.forward_raw if args.raw else gdn.forward
     d = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}
     out = torch.empty((w.B, w.T, w.H, w.dv), dtype=d["q"].dtype, device=dev)
@@ -360,80 +459,41 @@ def run_gdn(args, world, rank, local):
     chunks = -(-w.T // w.chunk)
     ws_tiles = w.B * w.H * chunks * (32768 + 528)
     nseg = 1 + max(0, scratch_bytes - ws_tiles) // (3 * w.B * w.H * w.dv * w.dk * 4) if "prep" in ktimes else 1
+    traffic_unit = measured_traffic(FWD_TRAFFIC_PROFILE)
     kernels = {}
+    step_traffic = 0.0
     for kind, (kms, n) in ktimes.items():
         per = kms / n
-        flop, by = kernel_work(kind, w, es, nseg)
+        cf = counted_flop_per_token_head(kind, w.dk, w.dv, w.chunk)
+        kflop = w.B * w.T * w.H * cf
+        by = kernel_design_bytes(kind, w, es, nseg)
+        units = kernel_units(kind, w, nseg)
+        tr = traffic_unit[kind] * units if kind in traffic_unit else None
         kernels[kind] = {"launches_per_step": n / args.steps, "ms_per_launch": per, "share": kms / (ms * 1.0),
-                         "tflops": flop / (per / 1e3) / 1e12, "gb_per_s": by / (per / 1e3) / 1e9,
-                         "flop_per_launch": flop, "bytes_per_launch": by}
+                         "counted_flop_per_token_head": cf, "counted_flop_per_launch": kflop,
+                         "counted_tflops": kflop / (per / 1e3) / 1e12,
+                         "design_bytes_per_launch": by, "design_gb_per_s": by / (per / 1e3) / 1e9,
+                         "traffic_per_launch": tr}
+        step_traffic = None if (step_traffic is None or tr is None) else step_traffic + tr * n / args.steps
     top = max(kernels, key=lambda k: ktimes[k][0]) if kernels else None
-    if top is not None:
-        kt = kernels[top]
-        tf, gb = kt["tflops"] / peaks["bf16_tflops"], kt["gb_per_s"] / peaks["hbm_gbs"]
-        # the nearer roof: the kernel is latency-bound when both fractions are low
-        if tf >= gb:
-            roof = {"bound": "tensor", "achieved": kt["tflops"], "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                    "frac": tf, "hbm_frac": gb}
-        else:
-            roof = {"bound": "hbm", "achieved": kt["gb_per_s"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": gb, "tensor_frac": tf}
-        per_unit = NCU_TRAFFIC_PER_TOKEN_HEAD.get(top)
-        traffic = per_unit * kernel_units(top, w, nseg) if per_unit is not None else None
-        roof.update({"kernel": top, "traffic": traffic, "peak_kind": peak_kind,
-                     "flop_per_launch": kt["flop_per_launch"], "bytes_per_launch": kt["bytes_per_launch"],
-                     "ms_per_launch": kt["ms_per_launch"]})
-    else:
-        roof = None
+    # SURVEY-style roofline of the whole step: the counted FLOP of the chunkwise method over the step's
+    # device time against the measured dense bf16 peak (burst: the step is timed as a short burst of
+    # launches), and the compulsory bytes against the measured copy bandwidth beside it.
+    roof = {"bound": "tensor", "kernel": "forward step (%d launches)" % launches_per_fwd,
+            "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": tflops / peaks["bf16_tflops"], "peak_kind": peak_kind + " bf16 burst",
+            "flop_per_step": flop, "flop_per_token_head": fwd_flop_per_token_head(w.dk, w.dv, w.chunk),
+            "hbm": {"achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                    "compulsory_bytes_per_step": nbytes},
+            "traffic": step_traffic,
+            "traffic_over_compulsory": None if step_traffic is None else step_traffic / nbytes,
+            "traffic_source": "profiles/" + FWD_TRAFFIC_PROFILE,
+            "dominant_kernel": top}
 
-    # ---- decode: 1024 consecutive single-token steps, each its own launch ----
-    dec = None
-    if not args.no_decode:
-        wd = WORKLOADS[DEC_WORKLOAD]
-        dsteps = wd.steps
-        di = decode_inputs(dsteps, wd.B, wd.H, wd.dk, wd.dv, wd.dtype, seed=wd.seed + 1000 * rank,
-                           s0_std=wd.s0_std)
-        dd = {k: v.to(dev) for k, v in di.items()}
-        S = dd["S"].clone()
-        dout = torch.empty((dsteps, wd.B, wd.H, wd.dv), dtype=dd["q"].dtype, device=dev)
-
-        def dec_run():
-            for t in range(dsteps):
-                gdn.decode_step(dd["q"][t], dd["k"][t], dd["v"][t], dd["log_alpha"][t], dd["beta"][t], S,
-                                out=dout[t], stream=stream)
-
-        for _ in range(max(1, args.warmup // 3)):
-            dec_run()
-        # The 1024 launches (each still one gdn_decode_step call through the C ABI) are captured
-        # once in a CUDA graph and replayed: a Python call costs about as long as one ~20 us decode
-        # kernel, and host overhead must not leave the GPU idle inside the timed region.
-        replay = dec_run
-        try:
-            graph = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(graph):
-                cap = torch.cuda.current_stream()
-                for t in range(dsteps):
-                    gdn.decode_step(dd["q"][t], dd["k"][t], dd["v"][t], dd["log_alpha"][t], dd["beta"][t], S,
-                                    out=dout[t], stream=cap)
-            graph.replay()
-            torch.cuda.synchronize()
-            replay = graph.replay
-        except RuntimeError:
-            torch.cuda.synchronize()
-        dms = time_region(replay, 1, stream, world) / dsteps
-        dms = max_over_ranks(dms, world)
-        des = 2 if wd.dtype == "bf16" else 4
-        dbytes = wd.B * wd.H * decode_bytes_per_head_step(wd.dk, wd.dv, des)
-        dgbs = dbytes / (dms / 1e3) / 1e9
-        dec = {"workload": wd.name, "steps": dsteps, "us_per_step": dms * 1e3,
-               "launch": "cuda_graph" if replay is not dec_run else "eager",
-               "tokens_per_s": world * wd.B / (dms / 1e3), "GB_per_s": dgbs,
-               "roofline": {"bound": "hbm", "achieved": dgbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                            "frac": dgbs / peaks["hbm_gbs"],
-                            "traffic": NCU_DECODE_TRAFFIC.get(wd.name),
-                            "peak_kind": peak_kind, "bytes_per_launch": dbytes},
-               "launches": dsteps}
-        del dd, S, dout
+    # ---- decode: consecutive single-token steps, each its own launch ----
+    decs = [time_decode(gdn, WORKLOADS[n], dev, stream, world, rank, args.warmup, peaks, peak_kind)
+            for n in ([] if args.no_decode else DEC_WORKLOADS)]
+    dec = decs[0] if decs else None
     clocks = sampler.stop()
 
     # ---- e2e: same forward through the C ABI with pinned host buffers ----
@@ -454,27 +514,27 @@ def run_gdn(args, world, rank, local):
         h2d = sum(t.numel() * t.element_size() for k, t in h.items() if t is not None)
         d2h = hout.numel() * hout.element_size() + hSf.numel() * hSf.element_size()
         e2e = {"value": world * tokens / (ems / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": ke}
+               "d2h_bytes_per_step": d2h, "ms_per_step": ems, "steps": ke,
+               "host_link_gb_per_s": (h2d + d2h) / (ems / 1e3) / 1e9,
+               "bound": "host link: every step moves its inputs in and its outputs out over PCIe"}
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N = 1 only) ----
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        model, _ = cpu_info()
+        model, host_cores = cpu_info()
         tps, threads, desc, _, _ = oracle_forward_sample(w, args.cpu_seconds)
-        cpu = {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc + "; CPU: " + model}
+        cpu = {"value": tps, "unit": "tokens/s", "cores": threads, "host_cores": host_cores,
+               "oracle_threads": threads, "kind": "oracle", "sample": desc + "; CPU: " + model}
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv, "chunk": w.chunk,
-                       "input_dtype": w.dtype, "state_dtype": "f32",
-                       "input_stage": "fused (raw q, k and gate logits)" if args.raw else "none (unit q, k; gates)", "parallelism": "replicas" if world > 1 else "single",
-                       "l2": "inputs larger than L2 (%.2f GB read+written per step)" % (nbytes / 1e9)},
+            "config": fwd_config(w_cfg, args.raw, world),
             "tflops": tflops, "gb_per_s": gbs,
             "roofline": roof, "kernels": kernels, "segments": nseg,
-            "decode": dec, "e2e": e2e, "cpu_baseline": cpu, "clocks": clocks,
+            "decode": dec, "decode_large_state": decs[1] if len(decs) > 1 else None, "e2e": e2e, "cpu_baseline": cpu, "clocks": clocks,
             "gpu_launches": args.steps * launches_per_fwd, "forward_launches_per_step": launches_per_fwd,
             "forward_scratch_bytes": scratch_bytes,
         }
@@ -717,6 +777,8 @@ def main():
     ap.add_argument("--varlen", type=int, default=0,
                     help="time packed prefill of this many sequences of mixed length instead of the forward step")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-only", default=None, choices=[n for n, w in WORKLOADS.items() if w.kind == "decode"],
+                    help="time only this decode workload (profiler captures of the decode kernel); not a bench line")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
@@ -737,6 +799,8 @@ def main():
             return run_conv(args, world, rank)
         if args.grouped:
             return run_grouped(args, world, rank)
+        if args.decode_only:
+            return run_decode_only(args, world, rank)
         return run_gdn(args, world, rank, local)
     finally:
         if world > 1:

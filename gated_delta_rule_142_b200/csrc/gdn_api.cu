@@ -62,6 +62,11 @@ bool supported_chunk(int64_t c) { return c == 16 || c == 32 || c == 64; }
 bool aligned16(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
+bool mul2ok(int64_t a, int64_t b) {
+    int64_t t;
+    return !__builtin_mul_overflow(a, b, &t);
+}
+
 bool mul3(int64_t a, int64_t b, int64_t c, int64_t *r) {
     int64_t t;
     return !__builtin_mul_overflow(a, b, &t) && !__builtin_mul_overflow(t, c, r);
@@ -503,7 +508,7 @@ int forward_impl(const void *q, const void *k, const void *v, const float *log_a
     const int64_t es = (dtype == GDN_F32) ? 4 : 2;
     int64_t ntok, nqk, nv, nstate;
     if (!mul3(B, T, H, &ntok) || !mul3(ntok, dk, es, &nqk) || !mul3(ntok, dv, es, &nv) ||
-        !mul3(B * H, dv, dk * 4, &nstate) || ntok > (INT64_MAX / 8))
+        !mul2ok(B, H) || !mul3(B * H, dv, dk * 4, &nstate) || ntok > (INT64_MAX / 8))
         return GDN_ERR_INVALID_SIZE;
     if (B * H == 0) return GDN_OK;
     if (ntok > 0 && (!q || !k || !v || !log_alpha || !beta || !out)) return GDN_ERR_NULL_PTR;
@@ -596,7 +601,7 @@ int varlen_impl(const void *q, const void *k, const void *v, const float *log_al
     if (N > (int64_t)INT32_MAX / (H > 0 ? H : 1) || T_total > (int64_t)INT32_MAX / 2) return GDN_ERR_INVALID_SIZE;
     int64_t ntok, nqk, nv, nstate;
     if (!mul3(1, T_total, H, &ntok) || !mul3(ntok, dk, es, &nqk) || !mul3(ntok, dv, es, &nv) ||
-        !mul3(N * H, dv, dk * 4, &nstate) || ntok > (INT64_MAX / 8))
+        !mul2ok(N, H) || !mul3(N * H, dv, dk * 4, &nstate) || ntok > (INT64_MAX / 8))
         return GDN_ERR_INVALID_SIZE;
     if (N * H == 0) return GDN_OK;
     if (ntok > 0 && (!q || !k || !v || !log_alpha || !beta || !out)) return GDN_ERR_NULL_PTR;
@@ -802,7 +807,7 @@ extern "C" int gdn_backward(const void *q, const void *k, const void *v, const f
     const int64_t es = (dtype == GDN_F32) ? 4 : 2;
     int64_t ntok, nqk, nv, nstate;
     if (!mul3(B, T, H, &ntok) || !mul3(ntok, dk, es, &nqk) || !mul3(ntok, dv, es, &nv) ||
-        !mul3(B * H, dv, dk * 4, &nstate) || ntok > (INT64_MAX / 8))
+        !mul2ok(B, H) || !mul3(B * H, dv, dk * 4, &nstate) || ntok > (INT64_MAX / 8))
         return GDN_ERR_INVALID_SIZE;
     if (B * H == 0) return GDN_OK;
     if (ntok > 0 && (!q || !k || !v || !log_alpha || !beta || !grad_out || !grad_q || !grad_k || !grad_v ||
@@ -893,7 +898,7 @@ extern "C" int gdn_forward_grouped(const void *q, const void *k, const void *v, 
     int64_t nq, nkv, nqk, nk, nv, nout, nstate, nxstate;
     if (!mul3(B, T, Hq, &nq) || !mul3(B, T, Hkv, &nkv) || !mul3(nq, dk, es, &nqk) || !mul3(nkv, dk, es, &nk) ||
         !mul3(nkv, dv, es, &nv) || !mul3(nq, dv, es, &nout) || !mul3(B * Hkv, dv, dk * 4, &nstate) ||
-        !mul3(B * Hq, dv, dk * 4, &nxstate) || nq > (INT64_MAX / 8))
+        !mul2ok(B, Hq) || !mul3(B * Hq, dv, dk * 4, &nxstate) || nq > (INT64_MAX / 8))
         return GDN_ERR_INVALID_SIZE;
     if (B * Hq == 0) return GDN_OK;
     if (nq > 0 && (!q || !k || !v || !log_alpha || !beta || !out)) return GDN_ERR_NULL_PTR;

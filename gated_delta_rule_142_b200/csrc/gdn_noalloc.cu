@@ -17,11 +17,13 @@
 // not use the symbol itself as a device address). That first call on a device
 // should therefore come before any stream capture. Every call shares the array
 // and leaves its last contents there. Nothing in it needs to start at zero,
-// because each launch writes every scratch element before reading it. Calls
+// because each launch writes every scratch element before reading it (the
+// test runs an unrelated problem between two checked calls to show it). Calls
 // whose executions overlap on the GPU (different streams, no ordering) race
 // on the array.
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 #include <atomic>
 
@@ -81,12 +83,13 @@ extern "C" int gdn_forward_noalloc(const void *q, const void *k, const void *v, 
     if (B < 0 || T < 0 || H < 0 || dk < 0 || dv < 0 || chunk < 0) return GDN_ERR_INVALID_SIZE;
     if (!dim_ok(dk) || !dim_ok(dv) || !(chunk == 16 || chunk == 32 || chunk == 64)) return GDN_ERR_UNSUPPORTED;
     const int64_t es = (dtype == GDN_F32) ? 4 : 2;
-    int64_t ntok, nqk, nv, nst;
-    if (__builtin_mul_overflow(B, T, &ntok) || __builtin_mul_overflow(ntok, H, &ntok) ||
+    // the same size checks as gdn_forward: B * H first, since with T == 0 the token count says nothing
+    int64_t nh, ntok, nqk, nv, nst;
+    if (__builtin_mul_overflow(B, H, &nh) || __builtin_mul_overflow(nh, T, &ntok) ||
         __builtin_mul_overflow(ntok, dk * es, &nqk) || __builtin_mul_overflow(ntok, dv * es, &nv) ||
-        __builtin_mul_overflow(B * H, dv * dk * 4, &nst))
+        __builtin_mul_overflow(nh, dv * dk * 4, &nst) || ntok > (INT64_MAX / 8))
         return GDN_ERR_INVALID_SIZE;
-    if (B * H == 0) return GDN_OK;
+    if (nh == 0) return GDN_OK;
     if (ntok > 0 && (!q || !k || !v || !log_alpha || !beta || !out)) return GDN_ERR_NULL_PTR;
     if (!al(q, 15) || !al(k, 15) || !al(v, 15) || !al(log_alpha, 3) || !al(beta, 3) || !al(S0, 15) ||
         !al(out, 15) || !al(S_final, 15))
@@ -137,9 +140,16 @@ extern "C" int gdn_forward_noalloc(const void *q, const void *k, const void *v, 
             gdn::fwd_split_workspace_bytes(p, nseg_split) <= (size_t)GDN_NOALLOC_SCRATCH_BYTES) {
             e = gdn::launch_fwd_split(p, nseg_split, sms, scratch, stream);
         } else {
-            const int nseg = gdn::fwd_tc_segments(p, sms, false);
+            int nseg = gdn::fwd_tc_segments(p, sms, false);
+            if (gdn::fwd_tc_workspace_bytes(p, nseg) > (size_t)GDN_NOALLOC_SCRATCH_BYTES) {
+                // a segment count the caller forced through GDN_SEGMENTS is honoured or refused;
+                // otherwise the forward runs with the most segments whose scratch fits (one
+                // segment needs none), trading chunk-level parallelism for the fixed array
+                const char *env = getenv("GDN_SEGMENTS");
+                if (env && atoi(env) >= 1) return GDN_ERR_SCRATCH_LIMIT;
+                while (nseg > 1 && gdn::fwd_tc_workspace_bytes(p, nseg) > (size_t)GDN_NOALLOC_SCRATCH_BYTES) --nseg;
+            }
             const size_t need = gdn::fwd_tc_workspace_bytes(p, nseg);
-            if (need > (size_t)GDN_NOALLOC_SCRATCH_BYTES) return GDN_ERR_SCRATCH_LIMIT;
             e = gdn::launch_fwd_tc(p, nseg, need ? scratch : nullptr, stream);
         }
     } else {

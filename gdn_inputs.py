@@ -61,6 +61,8 @@ WORKLOADS: Dict[str, Workload] = {
                  alpha_mu=-3.0, seed=3, describe="bf16, B=1 H=16 T=262144 d=128 chunk=64, slow decay, S_T"),
         Workload("decode_bf16_b64h16_d128_x1024", "decode", "bf16", B=64, H=16, dk=128, dv=128, steps=1024,
                  s0_std=0.02, seed=4, describe="decode, B=64 H=16 d=128, 1024 steps, S~N(0,0.02)"),
+        Workload("decode_bf16_b256h16_d128_x256", "decode", "bf16", B=256, H=16, dk=128, dv=128, steps=256,
+                 s0_std=0.02, seed=5, describe="decode, B=256 H=16 d=128 (state 268 MB, twice L2), 256 steps"),
     ]
 }
 

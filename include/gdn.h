@@ -82,8 +82,8 @@ typedef enum {
     GDN_ERR_DEVICE_TIMEOUT = 7, /* a bounded device-side wait gave up                  */
     GDN_ERR_ALIAS = 8,          /* an output overlaps an input it must not overlap     */
     GDN_ERR_DEVICE = 9,         /* no usable CUDA device / not an sm_100 device        */
-    GDN_ERR_SCRATCH_LIMIT = 10  /* gdn_forward_noalloc: problem needs more scratch than
-                                   GDN_NOALLOC_SCRATCH_BYTES                            */
+    GDN_ERR_SCRATCH_LIMIT = 10  /* gdn_forward_noalloc: a forced segment count needs more
+                                   scratch than GDN_NOALLOC_SCRATCH_BYTES               */
 } gdn_status;
 
 /*
@@ -326,8 +326,13 @@ int gdn_causal_conv(const void *x, const float *weight, const float *state_in, v
  *     two-kernel tensor-core forward when that fits (32.5 KB per chunk),
  *     else the call runs the single-kernel tensor-core forward, whose only
  *     scratch is the segment transfers and entry states of long sequences
- *     with few heads; a problem that needs more than the array holds either
- *     way returns GDN_ERR_SCRATCH_LIMIT before anything is enqueued;
+ *     with few heads (3 x 64 KiB per head and segment boundary).  When the
+ *     planned segment count needs more than the array holds, the call runs
+ *     with the most segments that fit (one segment needs none), so every
+ *     supported problem runs, with less chunk-level parallelism; only a
+ *     segment count forced through the environment variable GDN_SEGMENTS
+ *     that does not fit returns GDN_ERR_SCRATCH_LIMIT, before anything is
+ *     enqueued;
  *   - no cudaMalloc, cudaMallocAsync, cudaFree or other allocating routine is
  *     called.
  * The first call on a device looks up the array's device address on that

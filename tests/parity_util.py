@@ -13,6 +13,10 @@ from gdn_inputs import as_f32_numpy
 # and float32 state), applied to the outputs and the final state separately.
 TOL = {"f32": 1e-4, "bf16": 2e-2}
 
+# Every error the GPU tests compute, with the test that computed it: printed in the terminal summary
+# (tests/conftest.py) and, when GDN_PARITY_LOG names a file, appended to it as JSON lines.
+ACHIEVED = []
+
 
 def rel_err(gpu, ref) -> float:
     gpu = np.asarray(gpu, dtype=np.float64)
@@ -22,7 +26,10 @@ def rel_err(gpu, ref) -> float:
         return 0.0
     scale = np.abs(ref).max()
     assert np.isfinite(gpu).all(), "non-finite GPU values"
-    return float(np.abs(gpu - ref).max() / max(scale, 1e-30))
+    e = float(np.abs(gpu - ref).max() / max(scale, 1e-30))
+    test = os.environ.get("PYTEST_CURRENT_TEST", "?").split(" ")[0]
+    ACHIEVED.append((test, e))
+    return e
 
 
 def oracle_threads() -> int:

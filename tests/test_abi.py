@@ -284,3 +284,20 @@ def test_forward_plan_argument_checks(lib):
     assert lib.gdn_forward_plan(-1, 8, 2, 16, 16, 16, 0, None, None) == SIZE
     assert lib.gdn_forward_plan(0, 8, 2, 16, 16, 16, 1, ctypes.byref(s), ctypes.byref(n)) == OK
     assert (s.value, n.value) == (0, 0)
+
+
+def test_head_count_overflow_is_rejected_even_with_no_tokens(lib):
+    """B * H overflows int64 while T == 0: both forward entry points refuse the sizes before
+    anything else (the token count is zero and would not reveal it)."""
+    big = 1 << 40
+    assert fwd(lib, B=big, H=big, T=0) == SIZE
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    na = lib.gdn_forward_noalloc
+    na.argtypes = [ctypes.c_void_p] * 8 + [ctypes.c_int64] * 6 + [ctypes.c_void_p, ctypes.c_int]
+    na.restype = ctypes.c_int
+    args = [P(A), P(A + 0x1000000), P(A + 0x2000000), P(A + 0x3000000), P(A + 0x4000000), None, P(A + 0x5000000),
+            None]
+    assert na(*args, big, 0, big, 16, 16, 16, None, 0) == SIZE
+    # a token count beyond INT64_MAX / 8 is refused by both, as gdn_forward documents
+    assert fwd(lib, B=1 << 31, T=1 << 31, H=2) == SIZE
+    assert na(*args, 1 << 31, 1 << 31, 2, 16, 16, 16, None, 0) == SIZE

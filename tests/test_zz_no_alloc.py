@@ -4,15 +4,21 @@ Some callers cannot allocate device memory in the middle of a call. Examples:
 a framework whose caching allocator already owns the whole device heap, or a
 serving loop that must not enter the driver's allocator on its hot path. For
 them the library provides gdn_forward_noalloc. Its scratch is a fixed,
-library-owned device array of GDN_NOALLOC_SCRATCH_BYTES instead of
+library-owned device array of GDN_NOALLOC_SCRATCH_BYTES (32 MiB) instead of
 stream-ordered allocations.
 
-Checked here, through the C ABI:
-- two consecutive calls give the same outputs and final state as gdn_forward,
-  within the bf16 tolerance the other parity tests use, on a problem that goes
-  through the segmented path (the path that needs scratch);
-- a problem that needs more scratch than the array holds is refused before
-  anything is enqueued.
+Checked here, through the C ABI, against the float64 oracle (not against
+gdn_forward, so that an error the two entry points shared would still show):
+- the two-kernel path (its per-chunk workspace and the segment scratch in the
+  array): two checked calls on the same problem, with a call on an unrelated
+  problem (another seed, another segment count) between them, so that the
+  second checked call starts from array contents it did not write itself;
+- the single-kernel path that problems whose per-chunk workspace exceeds the
+  array take, with its segment transfers, prefix and entry states in the
+  array;
+- a long sequence whose planned segment scratch exceeds the array runs with
+  fewer segments instead, and a segment count forced beyond the array is
+  refused before anything is enqueued.
 
 The file name makes pytest collect it last. A run that stops at the first
 failure has then already run every other test. It also passes when run alone
@@ -25,12 +31,13 @@ import torch
 
 import gated_delta_rule_142_b200 as gdn
 from gdn_inputs import forward_inputs
-from parity_util import TOL, cpu_f64, rel_err, to_device
+from parity_util import TOL, cpu_f64, oracle_forward, rel_err, to_device
 
 pytestmark = pytest.mark.gpu
 
 GDN_BF16 = 1
 GDN_ERR_SCRATCH_LIMIT = 10
+SCRATCH_BYTES = 32 << 20
 
 
 def noalloc_fn():
@@ -53,24 +60,68 @@ def call_noalloc(fn, d, out, Sf, chunk=64):
               ptr(Sf), B, T, H, dk, dv, chunk, stream, GDN_BF16)
 
 
-def test_noalloc_matches_forward_on_two_consecutive_calls(monkeypatch):
-    # four segments: the transfer pass, the prefix and the output pass all use the scratch array
-    monkeypatch.setenv("GDN_SEGMENTS", "4")
+def run_noalloc(fn, d):
+    B, T, H, _ = d["q"].shape
+    out = torch.full((B, T, H, d["v"].shape[-1]), float("nan"), dtype=d["q"].dtype, device="cuda")
+    Sf = torch.full((B, H, d["v"].shape[-1], d["q"].shape[-1]), float("nan"), device="cuda")
+    assert call_noalloc(fn, d, out, Sf) == 0
+    torch.cuda.synchronize()
+    return out, Sf
+
+
+def check_against_oracle(inp, out, Sf, heads=None):
+    ref_o, ref_S = oracle_forward(inp, heads=heads)
+    o, S = cpu_f64(out), cpu_f64(Sf)
+    if heads is not None:
+        o, S = o[:, :, list(heads)], S[:, list(heads)]
+    assert rel_err(o, ref_o) <= TOL["bf16"]
+    assert rel_err(S, ref_S) <= TOL["bf16"]
+
+
+def test_noalloc_two_kernel_path_with_unrelated_call_between(monkeypatch):
     fn = noalloc_fn()
     inp = forward_inputs(1, 2048, 4, 128, 128, "bf16", seed=71, s0_std=0.1, alpha_mu=-3.0)
+    other = forward_inputs(2, 1500, 3, 128, 128, "bf16", seed=72, s0_std=0.3)
+    d, d_other = to_device(inp), to_device(other)
+    # four segments: the per-chunk workspace, the transfers, the prefix and the entry states all sit in
+    # the array (about 4.2 MB of workspace and 2.3 MB of segment scratch)
+    monkeypatch.setenv("GDN_SEGMENTS", "4")
+    out, Sf = run_noalloc(fn, d)
+    check_against_oracle(inp, out, Sf)
+    # an unrelated problem with another segment count overwrites the array with its own data
+    monkeypatch.setenv("GDN_SEGMENTS", "3")
+    o2, S2 = run_noalloc(fn, d_other)
+    check_against_oracle(other, o2, S2)
+    monkeypatch.setenv("GDN_SEGMENTS", "4")
+    out, Sf = run_noalloc(fn, d)
+    check_against_oracle(inp, out, Sf)
+
+
+def test_noalloc_single_kernel_path_when_the_workspace_does_not_fit(monkeypatch):
+    # 4 heads x 512 chunks of 32.5 KB workspace = 68 MB > 32 MiB: the single-kernel forward runs, with
+    # its 4-segment transfers, prefix and entry states (2.4 MB) in the array
+    B, T, H = 1, 32768, 4
+    assert H * (T // 64) * (32768 + 528) > SCRATCH_BYTES
+    monkeypatch.setenv("GDN_SEGMENTS", "4")
+    fn = noalloc_fn()
+    inp = forward_inputs(B, T, H, 128, 128, "bf16", seed=74, s0_std=0.05, alpha_mu=-3.0)
     d = to_device(inp)
-    ref_out, ref_S = gdn.forward(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], d["S0"], chunk=64)
-    torch.cuda.synchronize()
-    for _ in range(2):
-        out = torch.full_like(ref_out, float("nan"))
-        Sf = torch.full_like(ref_S, float("nan"))
-        assert call_noalloc(fn, d, out, Sf) == 0
-        torch.cuda.synchronize()
-        assert rel_err(cpu_f64(out), cpu_f64(ref_out)) <= TOL["bf16"]
-        assert rel_err(cpu_f64(Sf), cpu_f64(ref_S)) <= TOL["bf16"]
+    out, Sf = run_noalloc(fn, d)
+    check_against_oracle(inp, out, Sf, heads=[0, 3])
 
 
-def test_noalloc_refuses_problems_beyond_its_scratch(monkeypatch):
+def test_noalloc_lowers_the_segment_count_to_fit(monkeypatch):
+    # 8 heads over 256K tokens: the planner's segment scratch (about 37 segments, 57 MB) exceeds the
+    # array, so the call runs with the most segments that fit (22) instead of being refused
+    monkeypatch.delenv("GDN_SEGMENTS", raising=False)
+    fn = noalloc_fn()
+    inp = forward_inputs(1, 262144, 8, 128, 128, "bf16", seed=75, alpha_mu=-3.0)
+    d = to_device(inp)
+    out, Sf = run_noalloc(fn, d)
+    check_against_oracle(inp, out, Sf, heads=[6])
+
+
+def test_noalloc_refuses_a_forced_segment_count_beyond_its_scratch(monkeypatch):
     # 64 heads cut into 64 segments would need 3 * 64 * 63 * 64 KiB of scratch, far above the array
     monkeypatch.setenv("GDN_SEGMENTS", "64")
     fn = noalloc_fn()
