@@ -56,8 +56,10 @@ constexpr int kC = 64;
 constexpr int kD = 128;
 constexpr size_t kTileP = 64 * 64 * 2, kTileTB = 64 * 64 * 2, kTileW = 128 * 64 * 2;
 // Gate record of one chunk, float32: [0, 64) gamma_t, [64, 128) dl_s = e^{g_63 - g_s}, [128] gamma_C,
-// [129, 132) zero.  With the input stage fused, gamma_t carries 1 / |q_t| and dl_s 1 / |k_s|, the
-// scales of diag(gamma) Q and diag(dl) K in the chain.
+// [129] rho_C, the chunk's transfer bound gamma_C prod_t max(1, |1 - beta_t |k_t|^2|) (see
+// kNegligibleTransfer), [130, 132) zero.  With the input stage fused, gamma_t carries 1 / |q_t| and
+// dl_s 1 / |k_s|, the scales of diag(gamma) Q and diag(dl) K in the chain, and |k_t| is the
+// normalised key's.
 constexpr int kRecFloats = 132;
 constexpr size_t kGateRec = kRecFloats * 4;
 constexpr size_t kWsPerChunk = kTileP + kTileTB + kTileW + kGateRec;  // 32.5 KB
@@ -321,7 +323,8 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     float *rec = p.gate_rec + (int64_t)item(it) * kRecFloats;
                     rec[pt] = gm;
                     rec[64 + pt] = expf(gb[63] - gt);
-                    if (pt >= 60) rec[128 + 63 - pt] = (pt == 63) ? gb[63 + 128] : 0.f;  // [128] gamma_C
+                    // [128] gamma_C, [130, 132) zero; [129] is written after the G epilogue
+                    if (pt >= 60 && pt != 62) rec[128 + 63 - pt] = (pt == 63) ? gb[63 + 128] : 0.f;
                 }
                 // e^{g_t - g_s} = e^{g_t - c} e^{c - g_s} while every |g_t - c| < 60, so that
                 // neither factor overflows
@@ -394,8 +397,8 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         g[256 + c] *= inv;
                         g[320 + c] *= inv;
                     }
-                } else if (pt < 8) {
-                    rec[128 + (pt >> 1)] = (pt == 1) ? g[128 + 63] : 0.f;  // [128] gamma_C, [129, 132) 0
+                } else if (pt < 8 && (pt >> 1) != 1) {
+                    rec[128 + (pt >> 1)] = (pt == 1) ? g[128 + 63] : 0.f;  // [128] gamma_C, [130, 132) 0
                 }
                 named_bar(kBarP, kNumPrep);
             }
@@ -437,14 +440,21 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                             *reinterpret_cast<uint4 *>(sm + PO_P + sw128(t, (s0 >> 3) + cc)) =
                                 make_uint4(pk[cc * 4], pk[cc * 4 + 1], pk[cc * 4 + 2], pk[cc * 4 + 3]);
                     } else {
+                        // the diagonal beta_t |k_t|^2 (normalised key with the input stage fused) gives the
+                        // token's transfer factor max(1, |1 - beta_t |k_t|^2|), reduced into rho_C below
+                        float diag = 0.f;
 #pragma unroll
                         for (int i = 0; i < 16; i += 4) {
                             float v[4];
 #pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                v[e] = (s0 + i + e < t) ? bt * d[i + e] * __uint_as_float(r[i + e]) : 0.f;
+                            for (int e = 0; e < 4; ++e) {
+                                const float x = bt * d[i + e] * __uint_as_float(r[i + e]);
+                                v[e] = (s0 + i + e < t) ? x : 0.f;
+                                diag = (s0 + i + e == t) ? x : diag;
+                            }
                             *reinterpret_cast<float4 *>(Am + t * LDM + s0 + i) = make_float4(v[0], v[1], v[2], v[3]);
                         }
+                        if (t >= s0 && t < s0 + 16) Xs[t] = fmaxf(1.f, fabsf(1.f - diag));
                     }
                 }
             }
@@ -484,6 +494,12 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
                     for (int rr = 0; rr < 16; ++rr) Tm[(o + rr) * LDM + o + lane] = x[rr];
                 }
+            } else if (pw == 4) {
+                // rho_C = gamma_C prod_t max(1, |1 - beta_t |k_t|^2|) into the gate record
+                float pr = Xs[lane] * Xs[lane + 32];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) pr *= __shfl_xor_sync(0xffffffffu, pr, o);
+                if (lane == 0) p.gate_rec[(int64_t)gi * kRecFloats + 129] = g[128 + 63] * pr;
             }
             __syncwarp();
             named_bar(kBarP, kNumPrep);
@@ -683,6 +699,7 @@ struct ChainArgs {
     int nseg, seg_len;
     const float *S_entry;  // [B*H][nseg-1][dv][dk]
     float *Bw, *Mw;        // [B*H][nseg-1][dv][dk] / [dk][dk]
+    int *Mflag;            // [B*H][nseg-1]: 1 where the segment's transfer matrix is negligible (not written)
     const int4 *ptab;      // per-CTA work of packed sequences, or nullptr
     const int2 *ctab;      // packed chunk table, or nullptr
     __nv_bfloat16 *out;    // for the plain stores of partial packed chunks
@@ -1140,6 +1157,13 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 // other's latency.  Each group keeps S, the U^T accumulator and a second half
 // accumulator in 256 TMEM columns; its bf16 operand copies of S and U^T live in
 // shared memory.
+//
+// A segment whose chunks' transfer bounds rho_C multiply to at most e^-40 over
+// its last m chunks (kNegligibleTransfer) needs neither run in full: the
+// state entering the segment, and whatever the zero-state run gathered before
+// those m chunks, reach the segment's end scaled by at most e^-40.  Such a CTA
+// runs the zero-state run over the last m chunks only, skips the identity run
+// and flags M as negligible for the prefix.
 constexpr int kTrThreads = 640;
 // warp 0: TMA producer; warp 1: Ut^T issuer (group 0); warps 2-3: K rows scaled by dl;
 // warps 4-11: group 0; warps 12-19: group 1 (threads 0 and 32 of a group issue its MMAs)
@@ -1194,13 +1218,44 @@ fwd_transfer_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     const int64_t bh = blockIdx.x / (p.nseg - 1);
     const int seg = (int)(blockIdx.x % (p.nseg - 1));
     const int b = (int)(bh / H), h = (int)(bh % H);
-    const int c0 = seg * p.seg_len;
-    const int N = p.seg_len;  // segments 0..nseg-2 are full
-    const int64_t item0 = bh * p.chunks + c0;
+    const int64_t seg_item0 = bh * p.chunks + (int64_t)seg * p.seg_len;  // segments 0..nseg-2 are full
     const uint32_t sbase = smem_u32(sm);
+    volatile int *span = reinterpret_cast<volatile int *>(sm + TO_MISC + 8);  // chunks run, M negligible
 
+    if (warp == 0) {
+        // the shortest tail of the segment whose transfer bounds multiply to at most e^-40: warp-wide
+        // suffix products over blocks of 32 chunk records, from the segment's end backwards
+        int m = p.seg_len, negl = 0;
+        float run = 1.f;
+        for (int base = 0; base < p.seg_len; base += 32) {
+            const int i = base + lane;  // i-th chunk from the end
+            float x = (i < p.seg_len) ? p.gate_rec[(seg_item0 + p.seg_len - 1 - i) * kRecFloats + 129] : 1.f;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x *= y;
+            }
+            x *= run;
+            const uint32_t hit = __ballot_sync(0xffffffffu, i < p.seg_len && x <= kNegligibleTransfer);
+            if (hit) {
+                m = base + __ffs(hit);
+                negl = 1;
+                break;
+            }
+            run = __shfl_sync(0xffffffffu, x, 31);
+        }
+        if (lane == 0) {
+            span[0] = negl ? m : p.seg_len;
+            span[1] = negl;
+            p.Mflag[bh * (p.nseg - 1) + seg] = negl;
+        }
+        __syncwarp();
+    }
     if (tid == 0) {
-        for (int i = 0; i < TB_COUNT; ++i) mbar_init(&bars[i], (i == TB_EMPTY0 || i == TB_EMPTY1) ? 4 : 1);
+        __threadfence_block();
+        // each group's U^T and state-update MMAs release a stage: two commits per running group
+        const int cnt = span[1] ? 2 : 4;
+        for (int i = 0; i < TB_COUNT; ++i) mbar_init(&bars[i], (i == TB_EMPTY0 || i == TB_EMPTY1) ? cnt : 1);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -1213,6 +1268,11 @@ fwd_transfer_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     tc_fence_after();
     const uint32_t tm = *tmem_slot;
     const uint32_t lb = (uint32_t)((warp & 3) * 32) << 16;
+    // the chunks run: the whole segment, or its last N chunks when its transfer matrix is negligible
+    const int N = span[0];
+    const bool negligible = span[1] != 0;
+    const int c0 = seg * p.seg_len + (p.seg_len - N);
+    const int64_t item0 = bh * p.chunks + c0;
 
     if (warp == 0) {
         // ============================ producer ============================
@@ -1284,7 +1344,7 @@ fwd_transfer_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             named_bar(kBarScale, kTrNumScale);
             if (kt == 0) arrive(&bars[TB_KREADY0 + s]);
         }
-    } else {
+    } else if (!negligible || warp < kTrGrpWarp0 + 8) {
         // ============================ chain groups ============================
         const int grp = (warp - kTrGrpWarp0) >> 3;              // 0: from zero (B), 1: from identity (M)
         const int gt = tid - (kTrGrpWarp0 + 8 * grp) * 32;       // 0..255
@@ -1484,9 +1544,14 @@ bool fwd_split_supported(const FwdProblem &p) {
     return items * 128 < ((int64_t)1 << 31);  // tile-row coordinates of the workspace maps fit in int32
 }
 
+// Flags of the segment transfers (one int per head and segment boundary), after the segment scratch.
+size_t seg_flag_bytes(const FwdProblem &p, int nseg) {
+    return nseg > 1 ? (((size_t)(p.B * p.H) * (size_t)(nseg - 1) * sizeof(int) + 255) & ~(size_t)255) : 0;
+}
+
 size_t fwd_split_workspace_bytes(const FwdProblem &p, int nseg) {
     const size_t items = (size_t)(p.B * p.H) * (size_t)((p.T + kC - 1) / kC);
-    return items * kWsPerChunk + fwd_tc_workspace_bytes(p, nseg);
+    return items * kWsPerChunk + fwd_tc_workspace_bytes(p, nseg) + seg_flag_bytes(p, nseg);
 }
 
 cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *workspace, cudaStream_t stream) {
@@ -1542,6 +1607,7 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
     a.nseg = (int)((chunks + a.seg_len - 1) / a.seg_len);
     a.S_entry = nullptr;
     a.Bw = a.Mw = nullptr;
+    a.Mflag = nullptr;
     a.ptab = nullptr;
     a.ctab = nullptr;
     a.out = static_cast<__nv_bfloat16 *>(p.out);
@@ -1553,6 +1619,7 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
         a.Mw = a.Bw + per;
         float *entry = a.Mw + per;
         a.S_entry = entry;
+        a.Mflag = reinterpret_cast<int *>(entry + per);
         // segment transfers of segments 0..nseg-2, both runs of a segment in one CTA
         {
             TimedLaunch tl_(GDN_KERNEL_TRANSFER, stream);
@@ -1561,7 +1628,7 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
         }
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        e = launch_seg_prefix(p.S0, a.Bw, a.Mw, entry, heads, a.nseg, stream);
+        e = launch_seg_prefix(p.S0, a.Bw, a.Mw, a.Mflag, entry, heads, a.nseg, stream);
         if (e != cudaSuccess) return e;
     }
     // outputs of every segment from its entry state
@@ -1654,6 +1721,7 @@ cudaError_t launch_fwd_split_packed(const FwdProblem &p, const int64_t *cu_seqle
     a.seg_len = 0;
     a.S_entry = nullptr;
     a.Bw = a.Mw = nullptr;
+    a.Mflag = nullptr;
     a.ptab = d_ptab;
     a.ctab = d_ctab;
     a.out = static_cast<__nv_bfloat16 *>(p.out);

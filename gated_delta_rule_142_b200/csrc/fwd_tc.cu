@@ -822,8 +822,11 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 // Entry states of segments 1..nseg-1 from the segment transfers, in float32:
 // S_{p+1} = S_p M_p + B_p with S_0 = S0 (or zero).  Rows of the state are
 // independent, so one CTA owns 16 rows of one (b, h) and walks the segments
-// in order.  M_{p+1} is bulk-copied into the second of two shared buffers
-// while step p computes, and B_{p+1} is prefetched into registers.
+// in order.  The next needed M is bulk-copied into the second of two shared
+// buffers while a step computes, and B_{p+1} is prefetched into registers.
+// Where Mflag marks a transfer matrix as negligible (its bound is at most
+// e^-40, see kNegligibleTransfer) the step is S_{p+1} = B_p and M_p is neither
+// read nor multiplied.
 constexpr int kPrefixRows = 16;
 constexpr int kPrefixThreads = 256;
 constexpr int kPrefixLd = kD + 4;
@@ -831,7 +834,7 @@ constexpr size_t kPrefixSmem = (size_t)(2 * kD * kD + kPrefixRows * kPrefixLd) *
 
 __global__ void __launch_bounds__(kPrefixThreads, 1)
 seg_prefix_kernel(const float *__restrict__ S0, const float *__restrict__ Bw, const float *__restrict__ Mw,
-                  float *__restrict__ S_entry, int nseg) {
+                  const int *__restrict__ Mflag, float *__restrict__ S_entry, int nseg) {
     extern __shared__ __align__(128) float psm[];
     float *Ms = psm;                       // [2][128][128]
     float *Sr = psm + 2 * kD * kD;         // [16][kPrefixLd]
@@ -843,12 +846,19 @@ seg_prefix_kernel(const float *__restrict__ S0, const float *__restrict__ Bw, co
     // 16-byte words of a row of M, without bank conflicts
     const int r = tid >> 4, ca = (tid & 15) * 4, cb = 64 + ca;
     const int steps = nseg - 1;
-    auto load_m = [&](int q) {
+    auto needs_m = [&](int q) { return Mflag == nullptr || Mflag[bh * steps + q] == 0; };
+    // the n-th matrix loaded goes to buffer n & 1 and completes phase (n >> 1) & 1 of full[n & 1]
+    auto load_m = [&](int q, int n) {
         const float *M = Mw + (bh * steps + q) * (int64_t)kD * kD;
-        float *dst = Ms + (q & 1) * kD * kD;
-        fence_proxy_async_smem();  // the generic reads of this buffer two steps ago come first
-        mbar_arrive_expect_tx(&full[q & 1], kD * kD * 4);
-        for (int i = 0; i < 4; ++i) bulk_load(dst + i * 4096, M + i * 4096, 16384, &full[q & 1]);
+        float *dst = Ms + (n & 1) * kD * kD;
+        fence_proxy_async_smem();  // the generic reads of this buffer two loads ago come first
+        mbar_arrive_expect_tx(&full[n & 1], kD * kD * 4);
+        for (int i = 0; i < 4; ++i) bulk_load(dst + i * 4096, M + i * 4096, 16384, &full[n & 1]);
+    };
+    // the first step at or after q that needs its M, or steps
+    auto next_needed = [&](int q) {
+        while (q < steps && !needs_m(q)) ++q;
+        return q;
     };
     if (tid == 0) {
         mbar_init(&full[0], 1);
@@ -856,7 +866,9 @@ seg_prefix_kernel(const float *__restrict__ S0, const float *__restrict__ Bw, co
         mbar_fence_init();
     }
     __syncthreads();
-    if (tid == 0 && steps > 0) load_m(0);
+    int loaded = 0;  // matrices consumed so far
+    int pending = next_needed(0);  // the step whose M is in flight (steps: none)
+    if (tid == 0 && pending < steps) load_m(pending, 0);
     for (int i = tid; i < kPrefixRows * (kD / 4); i += kPrefixThreads) {
         const int rr = i / (kD / 4), cc = (i % (kD / 4)) * 4;
         float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -870,25 +882,34 @@ seg_prefix_kernel(const float *__restrict__ S0, const float *__restrict__ Bw, co
         b1 = *reinterpret_cast<const float4 *>(b_rows(0) + cb);
     }
     for (int q = 0; q < steps; ++q) {
-        if (tid == 0 && q + 1 < steps) load_m(q + 1);
-        // bounded wait; a timeout leaves the entry states unwritten rather than hanging
-        const bool landed = mbar_wait(&full[q & 1], (q >> 1) & 1);
-        if (!__syncthreads_and(landed)) break;  // also publishes the previous step's rows of S
         float acc[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-        if (q + 1 < steps) {
+        if (q == pending) {
+            // the next needed M goes into the other buffer, free since the step that read it ended
+            const int nxt = next_needed(q + 1);
+            if (tid == 0 && nxt < steps) load_m(nxt, loaded + 1);
+            // bounded wait; a timeout leaves the entry states unwritten rather than hanging
+            const bool landed = mbar_wait(&full[loaded & 1], (loaded >> 1) & 1);
+            if (!__syncthreads_and(landed)) break;  // also publishes the previous step's rows of S
+            if (q + 1 < steps) {
+                b0 = *reinterpret_cast<const float4 *>(b_rows(q + 1) + ca);
+                b1 = *reinterpret_cast<const float4 *>(b_rows(q + 1) + cb);
+            }
+            const float *M = Ms + (loaded & 1) * kD * kD;
+#pragma unroll 4
+            for (int k = 0; k < kD; ++k) {
+                const float a = Sr[r * kPrefixLd + k];
+                const float4 m0 = *reinterpret_cast<const float4 *>(M + k * kD + ca);
+                const float4 m1 = *reinterpret_cast<const float4 *>(M + k * kD + cb);
+                acc[0] = fmaf(a, m0.x, acc[0]); acc[1] = fmaf(a, m0.y, acc[1]);
+                acc[2] = fmaf(a, m0.z, acc[2]); acc[3] = fmaf(a, m0.w, acc[3]);
+                acc[4] = fmaf(a, m1.x, acc[4]); acc[5] = fmaf(a, m1.y, acc[5]);
+                acc[6] = fmaf(a, m1.z, acc[6]); acc[7] = fmaf(a, m1.w, acc[7]);
+            }
+            ++loaded;
+            pending = nxt;
+        } else if (q + 1 < steps) {
             b0 = *reinterpret_cast<const float4 *>(b_rows(q + 1) + ca);
             b1 = *reinterpret_cast<const float4 *>(b_rows(q + 1) + cb);
-        }
-        const float *M = Ms + (q & 1) * kD * kD;
-#pragma unroll 4
-        for (int k = 0; k < kD; ++k) {
-            const float a = Sr[r * kPrefixLd + k];
-            const float4 m0 = *reinterpret_cast<const float4 *>(M + k * kD + ca);
-            const float4 m1 = *reinterpret_cast<const float4 *>(M + k * kD + cb);
-            acc[0] = fmaf(a, m0.x, acc[0]); acc[1] = fmaf(a, m0.y, acc[1]);
-            acc[2] = fmaf(a, m0.z, acc[2]); acc[3] = fmaf(a, m0.w, acc[3]);
-            acc[4] = fmaf(a, m1.x, acc[4]); acc[5] = fmaf(a, m1.y, acc[5]);
-            acc[6] = fmaf(a, m1.z, acc[6]); acc[7] = fmaf(a, m1.w, acc[7]);
         }
         __syncthreads();  // every thread is done reading this step's rows and M
         *reinterpret_cast<float4 *>(Sr + r * kPrefixLd + ca) = make_float4(acc[0], acc[1], acc[2], acc[3]);
@@ -966,8 +987,8 @@ size_t fwd_tc_workspace_bytes(const FwdProblem &p, int nseg) {
     return (size_t)3 * (size_t)(p.B * p.H) * (size_t)(nseg - 1) * kD * kD * sizeof(float);
 }
 
-cudaError_t launch_seg_prefix(const float *S0, const float *Bw, const float *Mw, float *S_entry, int64_t heads,
-                              int nseg, cudaStream_t stream) {
+cudaError_t launch_seg_prefix(const float *S0, const float *Bw, const float *Mw, const int *Mflag, float *S_entry,
+                              int64_t heads, int nseg, cudaStream_t stream) {
     static std::atomic<uint64_t> pconf{0};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -981,7 +1002,7 @@ cudaError_t launch_seg_prefix(const float *S0, const float *Bw, const float *Mw,
     {
         TimedLaunch tl_(GDN_KERNEL_PREFIX, stream);
         seg_prefix_kernel<<<dim3((unsigned)heads, kD / kPrefixRows), kPrefixThreads, kPrefixSmem, stream>>>(
-            S0, Bw, Mw, S_entry, nseg);
+            S0, Bw, Mw, Mflag, S_entry, nseg);
     }
     return cudaGetLastError();
 }
@@ -1030,7 +1051,7 @@ cudaError_t launch_fwd_tc(const FwdProblem &p, int nseg, void *workspace, cudaSt
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         // phase 2: entry states of segments 1..nseg-1
-        e = launch_seg_prefix(p.S0, a.Bw, a.Mw, entry, heads, a.nseg, stream);
+        e = launch_seg_prefix(p.S0, a.Bw, a.Mw, nullptr, entry, heads, a.nseg, stream);
         if (e != cudaSuccess) return e;
     }
     // outputs of every segment from its entry state

@@ -12,6 +12,20 @@ namespace gdn {
 // log-decay sums stay small enough for float32 differences g_t - g_s.
 constexpr float kLogAlphaFloor = -40.0f;
 
+// Segment transfers of long sequences (the chunk-level parallelism of the
+// forward) use a bound on how much a state entering a span of chunks can still
+// matter at its end.  Over one token the state is multiplied on the right by
+// alpha_t (I - beta_t k_t k_t^T), whose spectral norm is
+// alpha_t max(1, |1 - beta_t |k_t|^2|) (the matrix is symmetric, with
+// eigenvalue 1 - beta_t |k_t|^2 along k_t and 1 across it).  The product of
+// these factors over a chunk, rho_C = gamma_C prod_t max(1, |1 - beta_t |k_t|^2|),
+// bounds the chunk's transfer, and the product of rho_C over a span bounds the
+// span's.  When that product is at most kNegligibleTransfer (e^-40), a state
+// entering the span contributes at most e^-40 of its own norm (bounded by the
+// paper's App. A.2 estimate) at the span's end: far below float32 resolution
+// of the result.  Such spans need no exact transfer matrix.
+constexpr float kNegligibleTransfer = 4.248354e-18f;  // e^-40
+
 // Brackets one kernel launch with CUDA events on its stream while
 // gdn_timing_start() recording is on (gdn_timing.cu); a no-op otherwise.
 // Construct it right before the launch, in a scope that ends right after it.
@@ -116,9 +130,10 @@ bool fwd_tc_supported(const FwdProblem &p);
 int fwd_tc_segments(const FwdProblem &p, int sm_count, bool paired_transfers);
 size_t fwd_tc_workspace_bytes(const FwdProblem &p, int nseg);
 cudaError_t launch_fwd_tc(const FwdProblem &p, int nseg, void *workspace, cudaStream_t stream);
-// Entry states of segments 1..nseg-1 from the segment transfers, in float32.
-cudaError_t launch_seg_prefix(const float *S0, const float *Bw, const float *Mw, float *S_entry, int64_t heads,
-                              int nseg, cudaStream_t stream);
+// Entry states of segments 1..nseg-1 from the segment transfers, in float32.  Mflag (or nullptr)
+// marks the transfer matrices that are negligible and were not written.
+cudaError_t launch_seg_prefix(const float *S0, const float *Bw, const float *Mw, const int *Mflag, float *S_entry,
+                              int64_t heads, int nseg, cudaStream_t stream);
 
 // fwd_split.cu -- the same forward as two kernels: a chunk-parallel prep
 // kernel writes P, T diag(beta), W^T and the gates of every chunk to the

@@ -211,7 +211,8 @@ def test_forward_plan_reports_scratch_and_launches(monkeypatch):
     assert (s, n) == (8 * 16 * 32 * per_chunk, 2)
     s, n = gdn.forward_plan(1, 65536, 16, 128, 128, 64)
     rest = s - 16 * 1024 * per_chunk
-    assert n == 4 and rest > 0 and rest % seg_unit == 0
+    boundaries = rest // seg_unit  # segments - 1, then one int flag per head and boundary (256-byte rounded)
+    assert n == 4 and boundaries > 0 and rest - boundaries * seg_unit == -(-16 * boundaries * 4 // 256) * 256
     assert gdn.forward_plan(1, 100, 2, 64, 64, 32) == (0, 1)  # CUDA-core path
     monkeypatch.setenv("GDN_FORWARD_PATH", "fused")
     assert gdn.forward_plan(8, 2048, 16, 128, 128, 64) == (0, 1)
@@ -227,3 +228,16 @@ def test_single_kernel_path(monkeypatch, T, nseg):
     monkeypatch.setenv("GDN_SEGMENTS", str(nseg))
     inp = forward_inputs(2, T, 2, 128, 128, "bf16", seed=73 + T, s0_std=0.1, alpha_mu=-3.0)
     check(inp, "bf16", 64, label="single kernel T=%d segments=%d" % (T, nseg))
+
+
+@pytest.mark.parametrize("alpha_mu", [-1.75, -3.0])
+def test_segmented_transfers_negligible_and_exact_mixed(monkeypatch, alpha_mu):
+    """Segment transfers whose decay makes the entering state negligible (the product of the chunks'
+    transfer bounds reaches e^-40 inside the segment: only the segment's tail is run, the identity run
+    and the prefix product are skipped) next to heads whose gates barely decay (the exact transfer
+    runs), in one launch: heads 0 and 2 decay, heads 1 and 3 keep alpha close to 1."""
+    monkeypatch.setenv("GDN_SEGMENTS", "4")
+    inp = forward_inputs(1, 64 * 40 + 17, 4, 128, 128, "bf16", seed=81, s0_std=0.1, alpha_mu=alpha_mu)
+    inp["log_alpha"][:, :, 1::2] = -1e-3 * torch.rand(inp["log_alpha"][:, :, 1::2].shape,
+                                                       generator=torch.Generator().manual_seed(5))
+    check(inp, "bf16", 64, label="mixed transfers alpha_mu=%g" % alpha_mu)
