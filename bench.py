@@ -114,16 +114,13 @@ DECODE_TRAFFIC_PROFILE = "decode_traffic_d128.md"
 
 def kernel_units(kind, w, nseg):
     """Units one launch of a kernel kind processes, the unit its measured traffic is quoted per:
-    token-heads (prep, chain, fused), token-heads of the transferred segments (transfer), segment
-    boundaries times heads (prefix)."""
+    token-heads (prep, chain, fused), segment boundaries times heads (transfer, prefix)."""
     nth = w.B * w.T * w.H
     if kind in ("prep", "chain", "fused"):
         return nth
-    if kind == "transfer":
-        chunks = -(-w.T // w.chunk)
-        seg_len = -(-chunks // max(nseg, 1))
-        return min(w.T, (nseg - 1) * seg_len * w.chunk) * w.B * w.H if nseg > 1 else 0
-    if kind == "prefix":
+    if kind in ("transfer", "prefix"):
+        # a transfer CTA runs only as many chunks as its segment's decay makes necessary (the whole
+        # segment when the gates barely decay), so its work is counted per segment boundary
         return w.B * w.H * max(nseg - 1, 0)
     return 0
 
@@ -141,7 +138,7 @@ def kernel_design_bytes(kind, w, es, nseg):
     if kind == "chain":
         return nth * ((2 * dk + 2 * dv) * es + tile)
     if kind == "transfer":
-        return kernel_units(kind, w, nseg) * ((dk + dv) * es + tile - 2 * C)
+        return None  # data-dependent: the chunks a segment's decay requires (its measured traffic is reported)
     if kind == "prefix":
         return kernel_units(kind, w, nseg) * 3 * dv * dk * 4
     if kind == "fused":
@@ -472,7 +469,8 @@ def run_gdn(args, world, rank, local):
         kernels[kind] = {"launches_per_step": n / args.steps, "ms_per_launch": per, "share": kms / (ms * 1.0),
                          "counted_flop_per_token_head": cf, "counted_flop_per_launch": kflop,
                          "counted_tflops": kflop / (per / 1e3) / 1e12,
-                         "design_bytes_per_launch": by, "design_gb_per_s": by / (per / 1e3) / 1e9,
+                         "design_bytes_per_launch": by,
+                         "design_gb_per_s": None if by is None else by / (per / 1e3) / 1e9,
                          "traffic_per_launch": tr}
         step_traffic = None if (step_traffic is None or tr is None) else step_traffic + tr * n / args.steps
     top = max(kernels, key=lambda k: ktimes[k][0]) if kernels else None
