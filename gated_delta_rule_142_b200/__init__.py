@@ -39,7 +39,7 @@ EXPORTS = ("gdn_forward", "gdn_decode_step", "gdn_forward_plan", "gdn_status_str
            "gdn_forward_noalloc", "gdn_scratch_release", "gdn_timing_start", "gdn_timing_stop",
            "gdn_forward_varlen", "gdn_forward_raw", "gdn_forward_varlen_raw", "gdn_decode_step_raw",
            "gdn_backward", "gdn_forward_grouped", "gdn_decode_step_grouped", "gdn_causal_conv",
-           "gdn_device_status", "gdn_selftest_device_timeout")
+           "gdn_device_status", "gdn_selftest_device_timeout", "gdn_forward_conv")
 
 # gdn_kernel_kind names, in enum order
 KERNEL_KINDS = ("prep", "chain", "transfer", "prefix", "fused", "simt", "decode", "input", "backward")
@@ -86,6 +86,8 @@ def load(path: str = LIBRARY) -> ctypes.CDLL:
     lib.gdn_selftest_device_timeout.restype = ctypes.c_int
     lib.gdn_causal_conv.argtypes = [vp] * 5 + [i64] * 4 + [vp, ctypes.c_int]
     lib.gdn_causal_conv.restype = ctypes.c_int
+    lib.gdn_forward_conv.argtypes = [vp] * 11 + [i64] * 7 + [vp, ctypes.c_int]
+    lib.gdn_forward_conv.restype = ctypes.c_int
     lib.gdn_forward_grouped.argtypes = [vp] * 8 + [i64] * 7 + [vp, ctypes.c_int]
     lib.gdn_forward_grouped.restype = ctypes.c_int
     lib.gdn_decode_step_grouped.argtypes = [vp] * 7 + [i64] * 5 + [vp, ctypes.c_int]
@@ -377,6 +379,47 @@ def causal_conv(x: torch.Tensor, weight: torch.Tensor, state_in: Optional[torch.
     if st != 0:
         raise GdnError(st, "gdn_causal_conv")
     return out, state_out
+
+
+def forward_conv(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, x_alpha: torch.Tensor, x_beta: torch.Tensor,
+                 conv_weight: torch.Tensor, conv_state: Optional[torch.Tensor] = None, S0: Optional[torch.Tensor] = None,
+                 chunk: int = 64, out: Optional[torch.Tensor] = None, S_final: Optional[torch.Tensor] = None,
+                 conv_state_out: Optional[torch.Tensor] = None, stream=None):
+    """The short causal convolution of q, k, v, then the raw forward (gdn_forward_conv).
+    conv_weight float32 [3, H*d, W] (q, k, v blocks; dk == dv), conv_state float32 [3, B, W-1, H*d] or
+    None.  Device tensors only.  Returns (out, S_final, conv_state_out)."""
+    lib = load()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if dk != dv:
+        raise ValueError("this binding takes dk == dv (the C entry point takes separate block sizes)")
+    W = conv_weight.shape[-1]
+    if tuple(conv_weight.shape) != (3, H * dk, W) or conv_weight.dtype != torch.float32:
+        raise ValueError("conv_weight must be float32 [3, H*d, W]")
+    for name, t in (("conv_state", conv_state), ("conv_state_out", conv_state_out)):
+        if t is not None and (tuple(t.shape) != (3, B, W - 1, H * dk) or t.dtype != torch.float32):
+            raise ValueError("%s must be float32 [3, B, W-1, H*d]" % name)
+    for name, t, shape in (("k", k, (B, T, H, dk)), ("v", v, (B, T, H, dv)), ("x_alpha", x_alpha, (B, T, H)),
+                           ("x_beta", x_beta, (B, T, H)), ("S0", S0, (B, H, dv, dk))):
+        if t is not None and tuple(t.shape) != shape:
+            raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), shape))
+    _dtype_code(q)
+    for t in (q, k, v, x_alpha, x_beta, conv_weight, conv_state, S0, out, S_final, conv_state_out):
+        if t is not None and (not t.is_contiguous() or t.device.type != "cuda"):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if S_final is None:
+        S_final = torch.empty((B, H, dv, dk), dtype=torch.float32, device=q.device)
+    if conv_state_out is None and W > 1:
+        conv_state_out = torch.empty((3, B, W - 1, H * dk), dtype=torch.float32, device=q.device)
+    with torch.cuda.device(q.device):
+        st = lib.gdn_forward_conv(_ptr(q), _ptr(k), _ptr(v), _ptr(x_alpha), _ptr(x_beta), _ptr(conv_weight),
+                                  _ptr(conv_state), _ptr(conv_state_out), _ptr(S0), _ptr(out), _ptr(S_final), B, T,
+                                  H, dk, dv, W, chunk, _stream_handle(q.device, stream), _dtype_code(q))
+    if st != 0:
+        raise GdnError(st, "gdn_forward_conv")
+    return out, S_final, conv_state_out
 
 
 def forward_plan(B: int, T: int, H: int, dk: int, dv: int, chunk: int = 64, dtype=torch.bfloat16):

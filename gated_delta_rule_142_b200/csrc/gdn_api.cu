@@ -1100,3 +1100,86 @@ extern "C" int gdn_selftest_device_timeout(void *stream_) {
     }
     return GDN_OK;
 }
+
+// ---------------------------------------------------------------- forward with the short convolution
+extern "C" int gdn_forward_conv(const void *q, const void *k, const void *v, const float *x_alpha, const float *x_beta,
+                                const float *conv_weight, const float *conv_state, float *conv_state_out,
+                                const float *S0, void *out, float *S_final, int64_t B, int64_t T, int64_t H,
+                                int64_t dk, int64_t dv, int64_t W, int64_t chunk, void *stream_, int dtype) {
+    if (dtype != GDN_F32 && dtype != GDN_BF16) return GDN_ERR_UNSUPPORTED;
+    if (B < 0 || T < 0 || H < 0 || dk < 0 || dv < 0 || chunk < 0 || W < 0) return GDN_ERR_INVALID_SIZE;
+    if (!supported_dim(dk) || !supported_dim(dv) || !supported_chunk(chunk) || W < 1 || W > 4)
+        return GDN_ERR_UNSUPPORTED;
+    const int64_t es = (dtype == GDN_F32) ? 4 : 2;
+    int64_t ntok, nqk, nv, nstate, cq = 0, cv = 0, nw = 0, ncs = 0;
+    if (!mul3(B, T, H, &ntok) || !mul3(ntok, dk, es, &nqk) || !mul3(ntok, dv, es, &nv) || !mul2ok(B, H) ||
+        !mul3(B * H, dv, dk * 4, &nstate) || ntok > (INT64_MAX / 8) || __builtin_mul_overflow(H, dk, &cq) ||
+        __builtin_mul_overflow(H, dv, &cv) || !mul3(2 * cq + cv, W, 4, &nw) || !mul3(B, (W - 1) * 4, 2 * cq + cv, &ncs))
+        return GDN_ERR_INVALID_SIZE;
+    if (B * H == 0) return GDN_OK;
+    if (ntok > 0 && (!q || !k || !v || !x_alpha || !x_beta || !out || !conv_weight)) return GDN_ERR_NULL_PTR;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned4(x_alpha) || !aligned4(x_beta) ||
+        !aligned16(S0) || !aligned16(out) || !aligned16(S_final) || !aligned4(conv_weight) || !aligned4(conv_state) ||
+        !aligned4(conv_state_out))
+        return GDN_ERR_MISALIGNED;
+    const Span sq(q, nqk), sk(k, nqk), sv(v, nv), sla(x_alpha, ntok * 4), sbe(x_beta, ntok * 4);
+    const Span s0(S0, nstate), sf(S_final, nstate), so(out, nv), swt(conv_weight, nw), scs(conv_state, ncs),
+        sco(conv_state_out, ncs);
+    for (const Span &x : {sq, sk, sv, sla, sbe, s0, sf, swt, scs, sco})
+        if (overlaps(so, x)) return GDN_ERR_ALIAS;
+    if (overlaps(sf, s0) && !(sf.lo == s0.lo)) return GDN_ERR_ALIAS;
+    for (const Span &x : {sq, sk, sv, sla, sbe, swt, scs, sco})
+        if (overlaps(sf, x)) return GDN_ERR_ALIAS;
+    if (overlaps(sco, scs) && !(sco.lo == scs.lo)) return GDN_ERR_ALIAS;
+    for (const Span &x : {sq, sk, sv, sla, sbe, swt, s0})
+        if (overlaps(sco, x)) return GDN_ERR_ALIAS;
+    DeviceInfo info;
+    if (int st = device_info(&info)) return st;
+    // device memory only
+    const void *ptrs[] = {q, k, v, x_alpha, x_beta, conv_weight, conv_state, conv_state_out, S0, out, S_final};
+    for (const void *ptr : ptrs)
+        if (ptr && !is_device_pointer(ptr)) return GDN_ERR_UNSUPPORTED;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    const float *st_q = conv_state, *st_k = conv_state ? conv_state + B * (W - 1) * cq : nullptr,
+                *st_v = conv_state ? conv_state + 2 * B * (W - 1) * cq : nullptr;
+    cudaError_t e = cudaSuccess;
+    int st = GDN_OK;
+    if (T == 0) {
+        if (S_final && S_final != S0)
+            e = S0 ? cudaMemcpyAsync(S_final, S0, (size_t)nstate, cudaMemcpyDeviceToDevice, stream)
+                   : cudaMemsetAsync(S_final, 0, (size_t)nstate, stream);
+    } else {
+        // the convolution of q, k and v into scratch (one launch), then the raw forward on its outputs
+        void *y = nullptr;
+        if (scratch_alloc(&y, (size_t)(2 * nqk + nv), stream) != cudaSuccess) {
+            cudaGetLastError();
+            return GDN_ERR_ALLOC;
+        }
+        uint8_t *yb = static_cast<uint8_t *>(y);
+        const void *xs[3] = {q, k, v};
+        const float *wts[3] = {conv_weight, conv_weight + cq * W, conv_weight + 2 * cq * W};
+        const float *sts[3] = {st_q, st_k, st_v};
+        void *ys[3] = {yb, yb + nqk, yb + 2 * nqk};
+        const int64_t Cs[3] = {cq, cq, cv};
+        e = gdn::launch_causal_conv3(xs, wts, sts, ys, Cs, 3, B, T, (int)W, dtype, stream);
+        if (e == cudaSuccess)
+            st = forward_impl(yb, yb + nqk, yb + 2 * nqk, x_alpha, x_beta, S0, out, S_final, B, T, H, dk, dv, chunk,
+                              stream_, dtype, true);
+        cudaFreeAsync(y, stream);
+        if (st) return st;
+    }
+    // the carried state after the call (after every read of the old one on this stream)
+    if (e == cudaSuccess && conv_state_out) {
+        float *o = conv_state_out;
+        e = gdn::launch_conv_state_update(q, st_q, o, B, T, cq, (int)W, dtype, stream);
+        if (e == cudaSuccess)
+            e = gdn::launch_conv_state_update(k, st_k, o + B * (W - 1) * cq, B, T, cq, (int)W, dtype, stream);
+        if (e == cudaSuccess)
+            e = gdn::launch_conv_state_update(v, st_v, o + 2 * B * (W - 1) * cq, B, T, cv, (int)W, dtype, stream);
+    }
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return GDN_ERR_LAUNCH;
+    }
+    return GDN_OK;
+}

@@ -99,6 +99,16 @@ cudaError_t launch_pick_states(const float *src, float *dst, int64_t B, int64_t 
 // alias state_in when T > 128 (the host copies first).
 cudaError_t launch_causal_conv(const void *x, const float *w, const float *state_in, void *y, float *state_out,
                                int64_t B, int64_t T, int64_t C, int W, int dtype, cudaStream_t stream);
+// Up to three convolutions over the same (B, T) in one launch (the state is not written): tensor i is
+// x[i] [B, T, C[i]] with weights w[i] [C[i], W] and carried inputs state_in[i] [B, W - 1, C[i]] (or
+// nullptr), into y[i].  One launch when every tensor allows 16-byte words, else one per tensor.
+cudaError_t launch_causal_conv3(const void *const x[3], const float *const w[3], const float *const state_in[3],
+                                void *const y[3], const int64_t C[3], int njobs, int64_t B, int64_t T, int W, int dtype,
+                                cudaStream_t stream);
+// The carried state of the short convolution after a call of T tokens (the last W - 1 inputs, oldest
+// first); state_out may equal state_in.
+cudaError_t launch_conv_state_update(const void *x, const float *state_in, float *state_out, int64_t B, int64_t T,
+                                     int64_t C, int W, int dtype, cudaStream_t stream);
 
 // input_stage.cu -- the input stage as a pass of its own, for the forwards that do not fuse
 // it: L2-normalised q, k (dtype of the problem) and log alpha, beta from the gate logits, for

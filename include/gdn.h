@@ -306,6 +306,39 @@ int gdn_causal_conv(const void *x, const float *weight, const float *state_in, v
                     int dtype);
 
 /*
+ * gdn_forward_conv -- the layer's memory input in one call: the short causal
+ * convolution of q, k and v (gdn_causal_conv, source: Sec. 3, "Canon"
+ * depthwise causal convolutions in front of the memory), then gdn_forward_raw
+ * on its outputs:
+ *
+ *     q' = conv(q), k' = conv(k), v' = conv(v)      (each with its own weights)
+ *     out, S_final = gdn_forward_raw(q', k', v', x_alpha, x_beta, S0)
+ *
+ * The convolution of all three tensors runs as one launch into library
+ * scratch (3 x B x T x H x d elements of the input dtype), then the raw
+ * forward reads it.  The rounding is gdn_causal_conv's: the convolution in
+ * float32 (w0 x_t first, then the older inputs), rounded to the input dtype;
+ * the call gives the same bits as gdn_causal_conv on each tensor followed by
+ * gdn_forward_raw.
+ *
+ * Arguments: those of gdn_forward_raw, and
+ *   conv_weight     float32 [3][H*d][W]: the q block [H*dk][W], then the k
+ *                   block [H*dk][W], then the v block [H*dv][W]
+ *   conv_state      float32 [3][B][W-1][H*d], the last W - 1 inputs of each
+ *                   tensor before this call, oldest first (blocks q, k, v as
+ *                   for the weights), or NULL for a zero history
+ *   conv_state_out  the same layout, or NULL (not written); may equal
+ *                   conv_state (updated in place)
+ *   W               1..4
+ * Device memory only (GDN_ERR_UNSUPPORTED for host buffers).  With T == 0
+ * S_final receives S0 and conv_state_out receives conv_state (or zeros).
+ */
+int gdn_forward_conv(const void *q, const void *k, const void *v, const float *x_alpha, const float *x_beta,
+                     const float *conv_weight, const float *conv_state, float *conv_state_out, const float *S0,
+                     void *out, float *S_final, int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv, int64_t W,
+                     int64_t chunk, void *stream, int dtype);
+
+/*
  * gdn_forward_noalloc -- gdn_forward for callers that cannot allocate device
  * memory during a call.
  *

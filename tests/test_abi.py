@@ -301,3 +301,21 @@ def test_head_count_overflow_is_rejected_even_with_no_tokens(lib):
     # a token count beyond INT64_MAX / 8 is refused by both, as gdn_forward documents
     assert fwd(lib, B=1 << 31, T=1 << 31, H=2) == SIZE
     assert na(*args, 1 << 31, 1 << 31, 2, 16, 16, 16, None, 0) == SIZE
+
+
+def test_forward_conv_validates_before_any_device_work(lib):
+    """gdn_forward_conv: the convolution width and the usual sizes are checked on the host."""
+    P = lambda x: None if x is None else ctypes.c_void_p(x)  # noqa: E731
+    fc = lib.gdn_forward_conv
+
+    def call(W=4, B=1, T=8, H=2, d=16, chunk=16, dtype=0, weight=A + 0x7000000):
+        return fc(P(A), P(A + 0x1000000), P(A + 0x2000000), P(A + 0x3000000), P(A + 0x4000000), P(weight), None,
+                  None, None, P(A + 0x5000000), None, B, T, H, d, d, W, chunk, None, dtype)
+
+    assert call(W=5) == UNSUP
+    assert call(W=0) == UNSUP
+    assert call(W=-1) == SIZE
+    assert call(dtype=7) == UNSUP
+    assert call(weight=None) == NULL
+    assert call(B=0) == OK
+    assert call(weight=A + 0x7000001) == MISAL

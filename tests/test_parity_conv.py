@@ -66,3 +66,37 @@ def test_empty_sequence_passes_the_state_through():
     y, so = gdn.causal_conv(x.cuda(), w.cuda(), s.cuda())
     torch.cuda.synchronize()
     assert y.shape == (2, 0, 64) and torch.equal(so.cpu(), s)
+
+
+@pytest.mark.parametrize("dtype,C", [("bf16", 100), ("f32", 66), ("bf16", 2056)])
+def test_channel_counts_of_either_kernel(dtype, C):
+    """Channel counts that are not a whole number of 16-byte words take the one-channel kernel; the
+    others take the wide one (2056 bf16 channels: 257 words).  Tokens 130 = two 64-token tiles and a
+    ragged third."""
+    B, T, W = 2, 130, 4
+    x, w, s = draw(B, T, C, W, dtype, seed=870 + C)
+    y, so = gdn.causal_conv(x.cuda(), w.cuda(), s.cuda())
+    torch.cuda.synchronize()
+    ry, rs = oracle.causal_conv(as_f32_numpy(x), w.numpy(), s.numpy())
+    assert rel_err(cpu_f64(y), ry) <= TOL[dtype]
+    assert rel_err(cpu_f64(so), rs) <= 1e-7
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_wide_and_one_channel_kernels_give_identical_bits(dtype):
+    """The same input at a 16-byte aligned address (wide kernel) and one element past it (one-channel
+    kernel): both compute w0 x_t first and then the older inputs, so the outputs are bit-identical."""
+    B, T, C, W = 2, 257, 1024, 4
+    x, w, s = draw(B, T, C, W, dtype, seed=880)
+    xa = x.cuda()
+    buf = torch.empty(x.numel() + 8, dtype=x.dtype, device="cuda")
+    xm = buf[1:1 + x.numel()].view(B, T, C)
+    xm.copy_(xa)
+    ybuf = torch.empty_like(buf)
+    ym = ybuf[1:1 + x.numel()].view(B, T, C)
+    assert xm.data_ptr() % 16 != 0 and ym.data_ptr() % 16 != 0
+    y1, s1 = gdn.causal_conv(xa, w.cuda(), s.cuda())
+    _, s2 = gdn.causal_conv(xm, w.cuda(), s.cuda(), out=ym)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, ym)
+    assert torch.equal(s1, s2)
