@@ -542,15 +542,21 @@ def run_gdn(args, world, rank, local):
 
 def run_varlen(args, world, rank):
     """Packed prefill: args.varlen sequences with lengths drawn log-uniformly from [256, 8192]
-    (seeded), H = 16, d = 128, bf16, one gdn_forward_varlen call per step, inputs in HBM."""
+    (seeded), H = 16, d = 128, bf16, one gdn_forward_varlen call per step, inputs in HBM.  With
+    --varlen-long L the first sequence has L tokens instead (one long sequence among short ones,
+    gates of the long-context workloads: x_alpha ~ N(-3, 1))."""
     import gated_delta_rule_142_b200 as gdn
     gdn.load()
     peaks, peak_kind = load_peaks()
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream(dev)
     lengths = length_mix(args.varlen, 256, 8192, seed=rank)
+    alpha_mu = 0.0
+    if args.varlen_long:
+        lengths = [args.varlen_long] + lengths[1:]
+        alpha_mu = -3.0
     H, d = 16, 128
-    inp = varlen_inputs(lengths, H, d, d, "bf16", seed=1000 + rank, s0_std=0.02)
+    inp = varlen_inputs(lengths, H, d, d, "bf16", seed=1000 + rank, s0_std=0.02, alpha_mu=alpha_mu)
     dd = {n: inp[n].to(dev) for n in ("q", "k", "v", "log_alpha", "beta", "S0")}
     T = sum(lengths)
     out = torch.empty((T, H, d), dtype=torch.bfloat16, device=dev)
@@ -592,7 +598,9 @@ def run_varlen(args, world, rank):
                 "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": "varlen_bf16_n%d_h16_d128" % args.varlen, "sequences": len(lengths),
+                "config": {"workload": "varlen_bf16_n%d%s_h16_d128" % (
+                               args.varlen, "_long%d" % args.varlen_long if args.varlen_long else ""),
+                           "sequences": len(lengths), "alpha_mu": alpha_mu,
                            "tokens": T, "min_len": min(lengths), "max_len": max(lengths), "H": H, "dk": d, "dv": d,
                            "chunk": 64, "parallelism": "replicas" if world > 1 else "single"},
                 "roofline": roof, "kernels": kernels, "clocks": clocks,
@@ -709,6 +717,72 @@ def run_conv(args, world, rank):
     return 0
 
 
+def run_forward_conv(args, world, rank):
+    """gdn_forward_conv on the forward workload: raw q, k, v and gate logits, the short convolution
+    (width 4, carried state) of all three in one launch, then the raw forward, one call per step
+    (bf16, inputs in HBM).  The same step composed of the public calls (three gdn_causal_conv
+    passes, then gdn_forward_raw) is timed beside it."""
+    import gated_delta_rule_142_b200 as gdn
+    gdn.load()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream(dev)
+    w = WORKLOADS[args.workload]
+    if args.tokens:
+        w = dataclasses.replace(w, T=args.tokens, name="%s_first%d" % (w.name, args.tokens))
+    W = 4
+    r = raw_inputs((w.B, w.T, w.H), w.dk, w.dv, w.dtype, seed=w.seed + 1000 * rank, s0_shape=(w.B, w.H, w.dv, w.dk),
+                   s0_std=w.s0_std, alpha_mu=w.alpha_mu)
+    g = torch.Generator(device="cpu")
+    g.manual_seed(w.seed + 1000 * rank + 9)
+    C = w.H * w.dk
+    d = {n: (None if r[n] is None else r[n].to(dev)) for n in ("q", "k", "v", "x_alpha", "x_beta", "S0")}
+    cw = (torch.randn((3, C, W), generator=g) * 0.5).to(dev)
+    cs = torch.randn((3, w.B, W - 1, C), generator=g).to(dev)
+    out = torch.empty((w.B, w.T, w.H, w.dv), dtype=d["q"].dtype, device=dev)
+    Sf = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=dev)
+    cso = torch.empty_like(cs)
+    ys = [torch.empty_like(d[n]) for n in ("q", "k", "v")]
+
+    def call():
+        gdn.forward_conv(d["q"], d["k"], d["v"], d["x_alpha"], d["x_beta"], cw, cs, d["S0"], chunk=w.chunk, out=out,
+                         S_final=Sf, conv_state_out=cso, stream=stream)
+
+    def composed():
+        for i, n in enumerate(("q", "k", "v")):
+            gdn.causal_conv(d[n], cw[i], cs[i], out=ys[i], state_out=cso[i], stream=stream)
+        gdn.forward_raw(ys[0], ys[1], ys[2], d["x_alpha"], d["x_beta"], d["S0"], chunk=w.chunk, out=out, S_final=Sf,
+                        stream=stream)
+
+    sampler = ClockSampler(dev)
+    sampler.start()
+    for _ in range(args.warmup):
+        call()
+        composed()
+    gdn.timing_start()
+    ms = time_region(call, args.steps, stream, world)
+    ktimes = gdn.timing_stop()
+    ms_c = time_region(composed, args.steps, stream, world)
+    clocks = sampler.stop()
+    ms_step = max_over_ranks(ms / args.steps, world)
+    ms_comp = max_over_ranks(ms_c / args.steps, world)
+    nbytes = fwd_bytes(w.B, w.T, w.H, w.dk, w.dv, 2 if w.dtype == "bf16" else 4, w.s0_std is not None, True)
+    if rank == 0:
+        line = {"metric": "gated-delta forward with the short convolution, tokens/s",
+                "value": world * w.B * w.T / (ms_step / 1e3), "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+                "config": {"workload": "conv4_raw_" + w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
+                           "chunk": w.chunk, "conv_width": W, "l2": "inputs larger than L2"},
+                "compulsory_gb_per_s": nbytes / (ms_step / 1e3) / 1e9,
+                "composed_ms_per_step": ms_comp,
+                "composed": "gdn_causal_conv on q, k, v (three passes), then gdn_forward_raw",
+                "kernels": {k: {"ms_per_launch": v[0] / v[1], "launches_per_step": v[1] / args.steps}
+                            for k, v in ktimes.items()},
+                "clocks": clocks, "gpu_launches": sum(int(n) for _, n in ktimes.values())}
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def run_grouped(args, world, rank):
     """gdn_forward_grouped on the ATMA head shape: 8 query heads reading 2 key-value memories,
     d = 128, over the forward workload's B and T (bf16, inputs in HBM)."""
@@ -770,8 +844,12 @@ def main():
     ap.add_argument("--backward", action="store_true",
                     help="time gdn_backward on the workload (default workload then: the 2K training shape)")
     ap.add_argument("--conv", action="store_true", help="time gdn_causal_conv on a q-shaped tensor instead")
+    ap.add_argument("--forward-conv", action="store_true",
+                    help="time gdn_forward_conv (the short convolution of q, k, v, then the raw forward) instead")
     ap.add_argument("--grouped", action="store_true",
                     help="time gdn_forward_grouped with 8 query / 2 key-value heads instead")
+    ap.add_argument("--varlen-long", type=int, default=0,
+                    help="with --varlen: the first sequence has this many tokens")
     ap.add_argument("--varlen", type=int, default=0,
                     help="time packed prefill of this many sequences of mixed length instead of the forward step")
     ap.add_argument("--no-decode", action="store_true")
@@ -797,6 +875,8 @@ def main():
             return run_conv(args, world, rank)
         if args.grouped:
             return run_grouped(args, world, rank)
+        if args.forward_conv:
+            return run_forward_conv(args, world, rank)
         if args.decode_only:
             return run_decode_only(args, world, rank)
         return run_gdn(args, world, rank, local)

@@ -38,7 +38,12 @@
 
 #include <stdlib.h>
 
+#include <string.h>
+
+#include <algorithm>
 #include <atomic>
+#include <functional>
+#include <queue>
 #include <vector>
 
 #include "gdn.h"
@@ -687,9 +692,14 @@ enum CBar {
 // transfer kernel's.
 static_assert(CB_COUNT * 8 <= CO_MISC - CO_BARS, "chain-kernel mbarriers overflow their shared-memory slot");
 
-// Packed variable-length sequences (no segments): CTA i runs sequence
-// ptab[i].x, head ptab[i].y, packed chunks ptab[i].z .. ptab[i].z + ptab[i].w - 1
-// of the chunk table ctab; its states are S0 / S_final [seq * H + head].
+// Packed variable-length sequences: CTA i runs sequence ptab[i].x, head
+// ptab[i].y, packed chunks ptab[i].z .. ptab[i].z + ptab[i].w - 1 of the chunk
+// table ctab.  Sequences longer than the segment length run as segments:
+// pseg[i] = {slot of S_entry holding the state entering the CTA's chunks, or -1
+// for S0 [seq * H + head]; 1 if the chunks end the sequence (S_final [seq * H +
+// head])}.  Transfer CTA i runs the full segment of seg_len chunks from packed
+// chunk trtab[i].z of sequence trtab[i].x, head trtab[i].y, into slot
+// trtab[i].w of Bw / Mw / Mflag.
 struct ChainArgs {
     const float *gate_rec;  // [items][kRecFloats] from the prep kernel
     const float *S0;
@@ -701,6 +711,8 @@ struct ChainArgs {
     float *Bw, *Mw;        // [B*H][nseg-1][dv][dk] / [dk][dk]
     int *Mflag;            // [B*H][nseg-1]: 1 where the segment's transfer matrix is negligible (not written)
     const int4 *ptab;      // per-CTA work of packed sequences, or nullptr
+    const int2 *pseg;      // packed: per-CTA entry slot and last flag, or nullptr (one CTA per sequence)
+    const int4 *trtab;     // packed: per-CTA work of the segment transfers
     const int2 *ctab;      // packed chunk table, or nullptr
     __nv_bfloat16 *out;    // for the plain stores of partial packed chunks
     float *ckpt;           // fixed-length only, or nullptr: the state entering every chunk,
@@ -725,23 +737,29 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // work of this CTA: state index bh (S0 / S_final row block), segment, head and chunks; chunk c
     // starts at token tok0(c) of batch row b and is workspace item witem(c)
     int64_t bh;
-    int seg, b, h, c0, N;
+    int b, h, c0, N;
+    int64_t entry_slot;  // slot of S_entry holding the state entering the chunks, or -1 for S0
+    bool last;           // the chunks end the sequence: S_final is written
     const bool packed = p.ptab != nullptr;
     if (packed) {
         const int4 w = p.ptab[blockIdx.x];
         bh = (int64_t)w.x * H + w.y;
-        seg = 0;
         b = 0;
         h = w.y;
         c0 = w.z;
         N = w.w;
+        const int2 sg = p.pseg ? p.pseg[blockIdx.x] : make_int2(-1, 1);
+        entry_slot = sg.x;
+        last = sg.y != 0;
     } else {
         bh = blockIdx.x / p.nseg;
-        seg = (int)(blockIdx.x % p.nseg);
+        const int seg = (int)(blockIdx.x % p.nseg);
         b = (int)(bh / H);
         h = (int)(bh % H);
         c0 = seg * p.seg_len;
         N = (p.chunks - c0 < p.seg_len) ? (p.chunks - c0) : p.seg_len;
+        entry_slot = seg == 0 ? -1 : bh * (p.nseg - 1) + seg - 1;
+        last = seg == p.nseg - 1;
     }
     auto tok0 = [&](int c) -> int { return packed ? p.ctab[c0 + c].x : (c0 + c) * kC; };
     auto ntok = [&](int c) -> int { return packed ? p.ctab[c0 + c].y : kC; };  // TMA clips at T otherwise
@@ -976,8 +994,8 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // entry state -> TMEM: S0 (or zero) for the first segment, the prefix-scanned entry state for
         // later segments
         {
-            const float *src = (seg == 0) ? (p.S0 ? p.S0 + (bh * kD + j) * (int64_t)kD : nullptr)
-                                          : p.S_entry + ((bh * (p.nseg - 1) + seg - 1) * kD + j) * (int64_t)kD;
+            const float *src = (entry_slot < 0) ? (p.S0 ? p.S0 + (bh * kD + j) * (int64_t)kD : nullptr)
+                                                : p.S_entry + (entry_slot * kD + j) * (int64_t)kD;
 #pragma unroll 1
             for (int piece = 0; piece < 2; ++piece) {
                 const int col0 = ch * 64 + piece * 32;
@@ -1120,7 +1138,7 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             ok = role_wait(&bars[CB_SDONE0 + ((N - 1) & 1)], ((N - 1) >> 1) & 1, abort_flag, kBarChn, kNumChn);
             tc_fence_after();
         }
-        float *dst = (seg == p.nseg - 1 && p.S_final) ? p.S_final + (bh * kD + j) * (int64_t)kD : nullptr;
+        float *dst = (last && p.S_final) ? p.S_final + (bh * kD + j) * (int64_t)kD : nullptr;
         if (ok && dst) {
 #pragma unroll 1
             for (int piece = 0; piece < 2; ++piece) {
@@ -1215,10 +1233,30 @@ fwd_transfer_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t H = p.H;
-    const int64_t bh = blockIdx.x / (p.nseg - 1);
-    const int seg = (int)(blockIdx.x % (p.nseg - 1));
-    const int b = (int)(bh / H), h = (int)(bh % H);
-    const int64_t seg_item0 = bh * p.chunks + (int64_t)seg * p.seg_len;  // segments 0..nseg-2 are full
+    // the segment: its first chunk cseg, its slot of Bw / Mw / Mflag, and the workspace item of chunk c
+    // (a (b, h)'s chunk index for fixed-length problems, a packed chunk index for packed sequences)
+    int b, h, cseg;
+    int64_t slot, ibase, istride;
+    if (p.trtab) {
+        const int4 w = p.trtab[blockIdx.x];
+        b = 0;
+        h = w.y;
+        cseg = w.z;
+        slot = w.w;
+        ibase = h;
+        istride = H;
+    } else {
+        const int64_t bh = blockIdx.x / (p.nseg - 1);
+        const int seg = (int)(blockIdx.x % (p.nseg - 1));
+        b = (int)(bh / H);
+        h = (int)(bh % H);
+        cseg = seg * p.seg_len;  // segments 0..nseg-2 are full
+        slot = bh * (p.nseg - 1) + seg;
+        ibase = bh * p.chunks;
+        istride = 1;
+    }
+    auto item = [&](int c) -> int64_t { return ibase + (int64_t)c * istride; };
+    auto tok0 = [&](int c) -> int { return p.trtab ? p.ctab[c].x : c * kC; };  // transfer chunks are full
     const uint32_t sbase = smem_u32(sm);
     volatile int *span = reinterpret_cast<volatile int *>(sm + TO_MISC + 8);  // chunks run, M negligible
 
@@ -1229,7 +1267,7 @@ fwd_transfer_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         float run = 1.f;
         for (int base = 0; base < p.seg_len; base += 32) {
             const int i = base + lane;  // i-th chunk from the end
-            float x = (i < p.seg_len) ? p.gate_rec[(seg_item0 + p.seg_len - 1 - i) * kRecFloats + 129] : 1.f;
+            float x = (i < p.seg_len) ? p.gate_rec[item(cseg + p.seg_len - 1 - i) * kRecFloats + 129] : 1.f;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const float y = __shfl_up_sync(0xffffffffu, x, o);
@@ -1247,7 +1285,7 @@ fwd_transfer_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
         if (lane == 0) {
             span[0] = negl ? m : p.seg_len;
             span[1] = negl;
-            p.Mflag[bh * (p.nseg - 1) + seg] = negl;
+            p.Mflag[slot] = negl;
         }
         __syncwarp();
     }
@@ -1271,8 +1309,7 @@ fwd_transfer_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     // the chunks run: the whole segment, or its last N chunks when its transfer matrix is negligible
     const int N = span[0];
     const bool negligible = span[1] != 0;
-    const int c0 = seg * p.seg_len + (p.seg_len - N);
-    const int64_t item0 = bh * p.chunks + c0;
+    const int c0 = cseg + (p.seg_len - N);
 
     if (warp == 0) {
         // ============================ producer ============================
@@ -1284,8 +1321,8 @@ fwd_transfer_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
                 if (c >= 2 && !(ok = wait_bar(&bars[TB_EMPTY0 + s], ((c - 2) >> 1) & 1, abort_flag))) break;
                 uint8_t *st = sm + s * TS_BYTES;
                 uint64_t *full = &bars[TB_FULL0 + s];
-                const int t0 = (c0 + c) * kC;
-                const int row = (int)(item0 + c);
+                const int t0 = tok0(c0 + c);
+                const int row = (int)item(c0 + c);
                 mbar_arrive_expect_tx(full, bytes);
                 for (int blk = 0; blk < 2; ++blk) {
                     tma_load_4d(st + TS_K + blk * 8192, &tm_k, full, blk * 64, h / p.group, t0, b);
@@ -1479,7 +1516,7 @@ fwd_transfer_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
             ok = role_wait(&bars[TB_SDONE0 + grp], (N - 1) & 1, abort_flag, barg, kTrNumGrp);
             tc_fence_after();
         }
-        float *dst = (grp == 0 ? p.Bw : p.Mw) + ((bh * (p.nseg - 1) + seg) * kD + j) * (int64_t)kD;
+        float *dst = (grp == 0 ? p.Bw : p.Mw) + (slot * kD + j) * (int64_t)kD;
         if (ok) {
 #pragma unroll 1
             for (int piece = 0; piece < 2; ++piece) {
@@ -1609,6 +1646,8 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
     a.Bw = a.Mw = nullptr;
     a.Mflag = nullptr;
     a.ptab = nullptr;
+    a.pseg = nullptr;
+    a.trtab = nullptr;
     a.ctab = nullptr;
     a.out = static_cast<__nv_bfloat16 *>(p.out);
     a.ckpt = p.ckpt;
@@ -1642,43 +1681,155 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
 
 // Tables after the per-chunk tiles: the chunk table (int2 entries), then, from the next 256-byte
 // boundary, the per-CTA table (int4 entries, read with 16-byte loads).
-size_t packed_ctab_bytes(int64_t total_chunks) {
-    return ((size_t)total_chunks * sizeof(int2) + 255) & ~(size_t)255;
-}
+namespace {
 
-size_t fwd_split_packed_workspace_bytes(int64_t total_chunks, int64_t H, int64_t N) {
-    const size_t items = (size_t)total_chunks * (size_t)H;
-    return items * kWsPerChunk + packed_ctab_bytes(total_chunks) + (size_t)(N * H) * sizeof(int4);
-}
+size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-cudaError_t launch_fwd_split_packed(const FwdProblem &p, const int64_t *cu_seqlens, int64_t N, int sm_count,
-                                    void *workspace, cudaStream_t stream) {
-    const int64_t H = p.H;
-    // chunk table over the packed tokens and one work entry per (sequence, head)
-    std::vector<int2> ctab;
-    std::vector<int4> ptab;
-    ptab.reserve((size_t)(N * H));
-    for (int64_t i = 0; i < N; ++i) {
-        const int64_t t0 = cu_seqlens[i], len = cu_seqlens[i + 1] - t0;
-        const int first = (int)ctab.size(), n = (int)((len + kC - 1) / kC);
-        for (int c = 0; c < n; ++c) {
-            const int64_t tc = t0 + (int64_t)c * kC;
-            ctab.push_back(make_int2((int)tc, (int)((len - (int64_t)c * kC) < kC ? (len - (int64_t)c * kC) : kC)));
-        }
-        for (int64_t h = 0; h < H; ++h) ptab.push_back(make_int4((int)i, (int)h, first, n));
+// Makespan of CTAs of the given lengths on sm_count SMs, one CTA per SM at a time, launched
+// longest first onto the SM that frees first.
+int64_t list_makespan(std::vector<int64_t> &len, int sm_count) {
+    std::sort(len.begin(), len.end(), std::greater<int64_t>());
+    std::priority_queue<int64_t, std::vector<int64_t>, std::greater<int64_t>> free_at;
+    for (int i = 0; i < sm_count; ++i) free_at.push(0);
+    int64_t end = 0;
+    for (int64_t l : len) {
+        const int64_t t = free_at.top() + l;
+        free_at.pop();
+        free_at.push(t);
+        end = t > end ? t : end;
     }
-    const int64_t chunks = (int64_t)ctab.size(), items = chunks * H;
-    if (N * H == 0) return cudaSuccess;
-    if (!workspace) return cudaErrorInvalidValue;
+    return end;
+}
+
+}  // namespace
+
+// The segment length of packed sequences: the one minimising a model of the three passes, in
+// units of half a chunk step of one CTA: the transfer pass (segments but the last of each cut
+// sequence, L chunks each) and the output pass (every segment), each as a list schedule over the
+// SMs, plus the sequential prefix (about half a chunk step per segment of the most-cut
+// sequence).  Candidates cut the longest sequence into 2..64 segments of at least 4 chunks.
+bool plan_packed(const int64_t *cu_seqlens, int64_t N, int64_t H, int sm_count, PackedPlan *pl) {
+    pl->H = H;
+    pl->sm_count = sm_count;
+    std::vector<int> first((size_t)N), n((size_t)N);
+    int64_t chunks = 0, nmax = 0;
+    for (int64_t i = 0; i < N; ++i) {
+        const int64_t len = cu_seqlens[i + 1] - cu_seqlens[i];
+        if (len < 0) return false;
+        const int64_t ni = (len + kC - 1) / kC;
+        first[(size_t)i] = (int)chunks;
+        n[(size_t)i] = (int)ni;
+        chunks += ni;
+        nmax = ni > nmax ? ni : nmax;
+    }
+    if (chunks * H * 128 >= ((int64_t)1 << 31)) return false;  // workspace tile rows stay in int32
+    pl->chunks = chunks;
+    // chunk lengths of the output CTAs of one head when sequences above L chunks are cut
+    auto segments_of = [&](int64_t ni, int64_t L) -> int64_t { return (L > 0 && ni > L) ? (ni + L - 1) / L : 1; };
+    int64_t L = 0;
+    const char *env = getenv("GDN_SEGMENTS");
+    if (env && atoi(env) >= 1) {
+        const int64_t k = atoi(env);
+        if (k > 1 && nmax > 1) L = (nmax + k - 1) / k;
+    } else if (nmax * sm_count > H * chunks && N * H * 64 <= ((int64_t)1 << 20)) {
+        // the longest sequence outlasts the average load of an SM: try cutting it
+        auto cost = [&](int64_t Lc) {
+            std::vector<int64_t> out_len;
+            int64_t ntr = 0, steps = 0;
+            for (int64_t i = 0; i < N; ++i) {
+                const int64_t m = segments_of(n[(size_t)i], Lc);
+                for (int64_t q = 0; q < m; ++q) {
+                    const int64_t cl = (q + 1 < m) ? Lc : n[(size_t)i] - (m - 1) * Lc;
+                    for (int64_t h = 0; h < H; ++h) out_len.push_back(cl);
+                }
+                ntr += m - 1;
+                steps = (m - 1) > steps ? (m - 1) : steps;
+            }
+            const int64_t waves = (ntr * H + sm_count - 1) / sm_count;
+            return 2 * (waves * Lc + list_makespan(out_len, sm_count)) + steps;
+        };
+        int64_t best = cost(0);
+        for (int64_t m = 2; m <= 64; ++m) {
+            const int64_t Lc = (nmax + m - 1) / m;
+            if (Lc < 4) break;
+            const int64_t c = cost(Lc);
+            if (c < best) {
+                best = c;
+                L = Lc;
+            }
+        }
+    }
+    pl->seg_len = (int)L;
+    // tables: chunk table; output CTAs (longest first) with their entry slot and last flag; transfer
+    // CTAs; prefix rows.  The transfers and entry states of a (sequence, head) take consecutive slots.
+    std::vector<int2> ctab;
+    ctab.reserve((size_t)chunks);
+    struct OutCta { int4 w; int2 sg; };
+    std::vector<OutCta> outs;
+    std::vector<int4> trs, pfs;
+    int64_t slot0 = 0;
+    for (int64_t i = 0; i < N; ++i) {
+        const int64_t t0 = cu_seqlens[i], len = cu_seqlens[i + 1] - t0, ni = n[(size_t)i];
+        for (int64_t c = 0; c < ni; ++c) {
+            const int64_t rest = len - c * kC;
+            ctab.push_back(make_int2((int)(t0 + c * kC), (int)(rest < kC ? rest : kC)));
+        }
+        const int64_t m = segments_of(ni, L);
+        for (int64_t h = 0; h < H; ++h) {
+            const int64_t base = slot0 + h * (m - 1);
+            for (int64_t q = 0; q < m; ++q) {
+                const int64_t c0 = first[(size_t)i] + q * L, cl = (q + 1 < m) ? L : ni - q * L;
+                outs.push_back({make_int4((int)i, (int)h, (int)c0, (int)cl),
+                                make_int2(q == 0 ? -1 : (int)(base + q - 1), q == m - 1 ? 1 : 0)});
+                if (q + 1 < m) trs.push_back(make_int4((int)i, (int)h, (int)c0, (int)(base + q)));
+            }
+            if (m > 1) pfs.push_back(make_int4((int)(i * H + h), (int)base, (int)(m - 1), 0));
+        }
+        slot0 += H * (m - 1);
+    }
+    std::stable_sort(outs.begin(), outs.end(), [](const OutCta &x, const OutCta &y) { return x.w.w > y.w.w; });
+    pl->slots = slot0;
+    pl->n_chain = (int64_t)outs.size();
+    pl->n_transfer = (int64_t)trs.size();
+    pl->n_prefix = (int64_t)pfs.size();
+    pl->off_chain = round256(ctab.size() * sizeof(int2));
+    pl->off_seg = pl->off_chain + round256(outs.size() * sizeof(int4));
+    pl->off_transfer = pl->off_seg + round256(outs.size() * sizeof(int2));
+    pl->off_prefix = pl->off_transfer + round256(trs.size() * sizeof(int4));
+    pl->tables.assign(pl->off_prefix + round256(pfs.size() * sizeof(int4)), 0);
+    uint8_t *t = pl->tables.data();
+    if (!ctab.empty()) memcpy(t, ctab.data(), ctab.size() * sizeof(int2));
+    for (size_t x = 0; x < outs.size(); ++x) {
+        memcpy(t + pl->off_chain + x * sizeof(int4), &outs[x].w, sizeof(int4));
+        memcpy(t + pl->off_seg + x * sizeof(int2), &outs[x].sg, sizeof(int2));
+    }
+    if (!trs.empty()) memcpy(t + pl->off_transfer, trs.data(), trs.size() * sizeof(int4));
+    if (!pfs.empty()) memcpy(t + pl->off_prefix, pfs.data(), pfs.size() * sizeof(int4));
+    return true;
+}
+
+// Workspace of a packed launch: the per-chunk tiles, the segment scratch (transfers, entry states;
+// 3 x 64 KiB per slot), the flags of the transfers, then the tables.
+size_t packed_workspace_bytes(const PackedPlan &pl) {
+    const size_t items = (size_t)pl.chunks * (size_t)pl.H;
+    return items * kWsPerChunk + (size_t)3 * (size_t)pl.slots * kD * kD * sizeof(float) +
+           round256((size_t)pl.slots * sizeof(int)) + pl.tables.size();
+}
+
+cudaError_t launch_fwd_split_packed(const FwdProblem &p, const PackedPlan &pl, void *workspace,
+                                    cudaStream_t stream) {
+    const int64_t H = p.H, chunks = pl.chunks, items = chunks * H;
+    if (pl.n_chain == 0) return cudaSuccess;
+    if (!workspace || pl.H != H) return cudaErrorInvalidValue;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     uint8_t *ws_p = ws, *ws_tb = ws + items * kTileP, *ws_w = ws_tb + items * kTileTB;
     float *ws_gates = reinterpret_cast<float *>(ws_w + items * kTileW);
-    int2 *d_ctab = reinterpret_cast<int2 *>(ws + items * kWsPerChunk);
-    int4 *d_ptab = reinterpret_cast<int4 *>(ws + items * kWsPerChunk + packed_ctab_bytes(chunks));
-    cudaError_t e = cudaSuccess;
-    if (chunks > 0) e = cudaMemcpyAsync(d_ctab, ctab.data(), ctab.size() * sizeof(int2), cudaMemcpyHostToDevice, stream);
-    if (e == cudaSuccess)
-        e = cudaMemcpyAsync(d_ptab, ptab.data(), ptab.size() * sizeof(int4), cudaMemcpyHostToDevice, stream);
+    const size_t per = (size_t)pl.slots * kD * kD;
+    float *Bw = reinterpret_cast<float *>(ws + items * kWsPerChunk), *Mw = Bw + per, *S_entry = Mw + per;
+    int *Mflag = reinterpret_cast<int *>(S_entry + per);
+    uint8_t *dtab = reinterpret_cast<uint8_t *>(Mflag) + round256((size_t)pl.slots * sizeof(int));
+    const int2 *d_ctab = reinterpret_cast<const int2 *>(dtab);
+    cudaError_t e = cudaMemcpyAsync(dtab, pl.tables.data(), pl.tables.size(), cudaMemcpyHostToDevice, stream);
     if (e != cudaSuccess) return e;
     const int64_t rows = items > 0 ? items : 1;  // tile maps need a non-empty extent
     CUtensorMap mq, mk, mv, mo, mp, mtb, mw;
@@ -1687,10 +1838,12 @@ cudaError_t launch_fwd_split_packed(const FwdProblem &p, const int64_t *cu_seqle
         !make_map_tiles(&mp, ws_p, rows, 64) || !make_map_tiles(&mtb, ws_tb, rows, 64) ||
         !make_map_tiles(&mw, ws_w, rows, 128))
         return cudaErrorInvalidValue;
-    static std::atomic<uint64_t> conf_prep{0}, conf_chain{0};
+    static std::atomic<uint64_t> conf_prep{0}, conf_chain{0}, conf_tr{0};
     if (!configure_once((const void *)fwd_prep_kernel, SMEM_PREP, conf_prep) ||
-        !configure_once((const void *)fwd_chain_kernel, SMEM_CHAIN, conf_chain))
+        !configure_once((const void *)fwd_chain_kernel, SMEM_CHAIN, conf_chain) ||
+        !configure_once((const void *)fwd_transfer_kernel, SMEM_TR, conf_tr))
         return cudaErrorInvalidValue;
+    const int64_t sm_count = pl.sm_count;
     if (items > 0) {
         PrepArgs pa;
         pa.log_alpha = p.log_alpha;
@@ -1718,18 +1871,34 @@ cudaError_t launch_fwd_split_packed(const FwdProblem &p, const int64_t *cu_seqle
     a.H = p.H;
     a.chunks = 0;
     a.nseg = 1;
-    a.seg_len = 0;
-    a.S_entry = nullptr;
-    a.Bw = a.Mw = nullptr;
-    a.Mflag = nullptr;
-    a.ptab = d_ptab;
+    a.seg_len = pl.seg_len;
+    a.S_entry = S_entry;
+    a.Bw = Bw;
+    a.Mw = Mw;
+    a.Mflag = Mflag;
+    a.ptab = reinterpret_cast<const int4 *>(dtab + pl.off_chain);
+    a.pseg = reinterpret_cast<const int2 *>(dtab + pl.off_seg);
+    a.trtab = reinterpret_cast<const int4 *>(dtab + pl.off_transfer);
     a.ctab = d_ctab;
     a.out = static_cast<__nv_bfloat16 *>(p.out);
     a.ckpt = nullptr;
     a.group = 1;
+    if (pl.n_transfer > 0) {
+        // transfers of every segment but the last of each cut sequence, then the entry states
+        {
+            TimedLaunch tl_(GDN_KERNEL_TRANSFER, stream);
+            fwd_transfer_kernel<<<(unsigned)pl.n_transfer, kTrThreads, SMEM_TR, stream>>>(mk, mv, mtb, mw, a);
+        }
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        e = launch_seg_prefix(p.S0, Bw, Mw, Mflag, S_entry, pl.n_prefix, 0, stream,
+                              reinterpret_cast<const int4 *>(dtab + pl.off_prefix));
+        if (e != cudaSuccess) return e;
+    }
     {
         TimedLaunch tl_(GDN_KERNEL_CHAIN, stream);
-        fwd_chain_kernel<<<(unsigned)(N * H), kChainThreads, SMEM_CHAIN, stream>>>(mq, mk, mv, mo, mp, mtb, mw, a);
+        fwd_chain_kernel<<<(unsigned)pl.n_chain, kChainThreads, SMEM_CHAIN, stream>>>(mq, mk, mv, mo, mp, mtb, mw,
+                                                                                     a);
     }
     return cudaGetLastError();
 }

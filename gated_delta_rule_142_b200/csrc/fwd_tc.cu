@@ -822,7 +822,10 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 // Entry states of segments 1..nseg-1 from the segment transfers, in float32:
 // S_{p+1} = S_p M_p + B_p with S_0 = S0 (or zero).  Rows of the state are
 // independent, so one CTA owns 16 rows of one (b, h) and walks the segments
-// in order.  The next needed M is bulk-copied into the second of two shared
+// in order.  A (b, h)'s transfers and entry states sit in consecutive slots;
+// with a table (packed sequences, whose segment counts differ), CTA row x
+// takes S0 [tab[x].x], slots tab[x].y .. tab[x].y + tab[x].z - 1; without
+// one, (b, h) = x takes S0 [x] and slots x (nseg - 1) onwards.  The next needed M is bulk-copied into the second of two shared
 // buffers while a step computes, and B_{p+1} is prefetched into registers.
 // Where Mflag marks a transfer matrix as negligible (its bound is at most
 // e^-40, see kNegligibleTransfer) the step is S_{p+1} = B_p and M_p is neither
@@ -834,22 +837,33 @@ constexpr size_t kPrefixSmem = (size_t)(2 * kD * kD + kPrefixRows * kPrefixLd) *
 
 __global__ void __launch_bounds__(kPrefixThreads, 1)
 seg_prefix_kernel(const float *__restrict__ S0, const float *__restrict__ Bw, const float *__restrict__ Mw,
-                  const int *__restrict__ Mflag, float *__restrict__ S_entry, int nseg) {
+                  const int *__restrict__ Mflag, float *__restrict__ S_entry, int nseg,
+                  const int4 *__restrict__ tab) {
     extern __shared__ __align__(128) float psm[];
     float *Ms = psm;                       // [2][128][128]
     float *Sr = psm + 2 * kD * kD;         // [16][kPrefixLd]
     uint64_t *full = reinterpret_cast<uint64_t *>(Sr + kPrefixRows * kPrefixLd);  // [2]
-    const int64_t bh = blockIdx.x;
+    int64_t bh, base;  // S0 row block and first slot
+    int steps;
+    if (tab) {
+        const int4 w = tab[blockIdx.x];
+        bh = w.x;
+        base = w.y;
+        steps = w.z;
+    } else {
+        bh = blockIdx.x;
+        steps = nseg - 1;
+        base = bh * steps;
+    }
     const int r0 = blockIdx.y * kPrefixRows;
     const int tid = threadIdx.x;
     // this thread's row and columns ca..ca+3, cb..cb+3: consecutive threads read consecutive
     // 16-byte words of a row of M, without bank conflicts
     const int r = tid >> 4, ca = (tid & 15) * 4, cb = 64 + ca;
-    const int steps = nseg - 1;
-    auto needs_m = [&](int q) { return Mflag == nullptr || Mflag[bh * steps + q] == 0; };
+    auto needs_m = [&](int q) { return Mflag == nullptr || Mflag[base + q] == 0; };
     // the n-th matrix loaded goes to buffer n & 1 and completes phase (n >> 1) & 1 of full[n & 1]
     auto load_m = [&](int q, int n) {
-        const float *M = Mw + (bh * steps + q) * (int64_t)kD * kD;
+        const float *M = Mw + (base + q) * (int64_t)kD * kD;
         float *dst = Ms + (n & 1) * kD * kD;
         fence_proxy_async_smem();  // the generic reads of this buffer two loads ago come first
         mbar_arrive_expect_tx(&full[n & 1], kD * kD * 4);
@@ -875,7 +889,7 @@ seg_prefix_kernel(const float *__restrict__ S0, const float *__restrict__ Bw, co
         if (S0) v = *reinterpret_cast<const float4 *>(S0 + (bh * kD + r0 + rr) * (int64_t)kD + cc);
         *reinterpret_cast<float4 *>(Sr + rr * kPrefixLd + cc) = v;
     }
-    auto b_rows = [&](int q) { return Bw + ((bh * steps + q) * kD + r0 + r) * (int64_t)kD; };
+    auto b_rows = [&](int q) { return Bw + ((base + q) * kD + r0 + r) * (int64_t)kD; };
     float4 b0 = make_float4(0.f, 0.f, 0.f, 0.f), b1 = b0;
     if (steps > 0) {
         b0 = *reinterpret_cast<const float4 *>(b_rows(0) + ca);
@@ -914,7 +928,7 @@ seg_prefix_kernel(const float *__restrict__ S0, const float *__restrict__ Bw, co
         __syncthreads();  // every thread is done reading this step's rows and M
         *reinterpret_cast<float4 *>(Sr + r * kPrefixLd + ca) = make_float4(acc[0], acc[1], acc[2], acc[3]);
         *reinterpret_cast<float4 *>(Sr + r * kPrefixLd + cb) = make_float4(acc[4], acc[5], acc[6], acc[7]);
-        float *dst = S_entry + ((bh * steps + q) * kD + r0 + r) * (int64_t)kD;
+        float *dst = S_entry + ((base + q) * kD + r0 + r) * (int64_t)kD;
         *reinterpret_cast<float4 *>(dst + ca) = make_float4(acc[0], acc[1], acc[2], acc[3]);
         *reinterpret_cast<float4 *>(dst + cb) = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
@@ -988,7 +1002,7 @@ size_t fwd_tc_workspace_bytes(const FwdProblem &p, int nseg) {
 }
 
 cudaError_t launch_seg_prefix(const float *S0, const float *Bw, const float *Mw, const int *Mflag, float *S_entry,
-                              int64_t heads, int nseg, cudaStream_t stream) {
+                              int64_t heads, int nseg, cudaStream_t stream, const int4 *tab) {
     static std::atomic<uint64_t> pconf{0};
     int dev = 0;
     cudaGetDevice(&dev);
@@ -1002,7 +1016,7 @@ cudaError_t launch_seg_prefix(const float *S0, const float *Bw, const float *Mw,
     {
         TimedLaunch tl_(GDN_KERNEL_PREFIX, stream);
         seg_prefix_kernel<<<dim3((unsigned)heads, kD / kPrefixRows), kPrefixThreads, kPrefixSmem, stream>>>(
-            S0, Bw, Mw, Mflag, S_entry, nseg);
+            S0, Bw, Mw, Mflag, S_entry, nseg, tab);
     }
     return cudaGetLastError();
 }

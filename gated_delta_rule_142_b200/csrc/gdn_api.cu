@@ -650,14 +650,14 @@ int varlen_impl(const void *q, const void *k, const void *v, const float *log_al
                      : cudaMemsetAsync(p.S_final, 0, (size_t)nstate, stream);
         done = true;
     }
-    int64_t chunks = 0;
-    for (int64_t i = 0; i < N; ++i) chunks += (cu_seqlens[i + 1] - cu_seqlens[i] + 63) / 64;
-    if (!done && path == FwdPath::Auto && gdn::fwd_tc_supported(p) && chunks * H * 128 < ((int64_t)1 << 31)) {
+    gdn::PackedPlan plan;
+    if (!done && path == FwdPath::Auto && gdn::fwd_tc_supported(p) &&
+        gdn::plan_packed(cu_seqlens, N, H, info.sm_count, &plan)) {
         // every sequence at once on the two-kernel tensor-core forward
         void *ws = nullptr;
-        if (scratch_alloc(&ws, gdn::fwd_split_packed_workspace_bytes(chunks, H, N), stream) == cudaSuccess) {
+        if (scratch_alloc(&ws, gdn::packed_workspace_bytes(plan), stream) == cudaSuccess) {
             p.raw_inputs = raw ? 1 : 0;  // the prep kernel runs the input stage on its own loads
-            e = gdn::launch_fwd_split_packed(p, cu_seqlens, N, info.sm_count, ws, stream);
+            e = gdn::launch_fwd_split_packed(p, plan, ws, stream);
             cudaFreeAsync(ws, stream);
             done = true;
         } else {

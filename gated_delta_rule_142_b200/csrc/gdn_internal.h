@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <vector>
+
 namespace gdn {
 
 // Floor applied to log_alpha inside the chunkwise forward: exp(-40) < 5e-18,
@@ -141,9 +143,11 @@ int fwd_tc_segments(const FwdProblem &p, int sm_count, bool paired_transfers);
 size_t fwd_tc_workspace_bytes(const FwdProblem &p, int nseg);
 cudaError_t launch_fwd_tc(const FwdProblem &p, int nseg, void *workspace, cudaStream_t stream);
 // Entry states of segments 1..nseg-1 from the segment transfers, in float32.  Mflag (or nullptr)
-// marks the transfer matrices that are negligible and were not written.
+// marks the transfer matrices that are negligible and were not written.  Without a table, heads
+// (b, h) of nseg segments each; with one (device memory), `heads` rows {S0 index, first slot,
+// steps, unused}.
 cudaError_t launch_seg_prefix(const float *S0, const float *Bw, const float *Mw, const int *Mflag, float *S_entry,
-                              int64_t heads, int nseg, cudaStream_t stream);
+                              int64_t heads, int nseg, cudaStream_t stream, const int4 *tab = nullptr);
 
 // fwd_split.cu -- the same forward as two kernels: a chunk-parallel prep
 // kernel writes P, T diag(beta), W^T and the gates of every chunk to the
@@ -153,10 +157,23 @@ cudaError_t launch_seg_prefix(const float *S0, const float *Bw, const float *Mw,
 bool fwd_split_supported(const FwdProblem &p);
 size_t fwd_split_workspace_bytes(const FwdProblem &p, int nseg);
 cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *workspace, cudaStream_t stream);
-// Packed variable-length sequences (p.B = 1, p.T = total tokens; cu_seqlens on the
-// host, N + 1 entries): one chain per (sequence, head), no segments.
-size_t fwd_split_packed_workspace_bytes(int64_t total_chunks, int64_t H, int64_t N);
-cudaError_t launch_fwd_split_packed(const FwdProblem &p, const int64_t *cu_seqlens, int64_t N, int sm_count,
-                                    void *workspace, cudaStream_t stream);
+// Packed variable-length sequences (p.B = 1, p.T = total tokens; cu_seqlens on the host, N + 1
+// entries).  plan_packed builds the host tables: the chunk table over the packed tokens and the
+// per-CTA work.  A sequence longer than the plan's segment length runs as segments, with segment
+// transfers and a prefix as for fixed-length problems, so that one long sequence among short ones
+// still spreads over the SMs.  GDN_SEGMENTS=k cuts the longest sequence into k segments (1: none).
+struct PackedPlan {
+    int64_t H = 0, chunks = 0;  // heads, packed chunks over all sequences
+    int sm_count = 148;
+    int seg_len = 0;            // chunks per segment (0: no sequence is cut)
+    int64_t slots = 0;          // segment boundaries over all (sequence, head)
+    int64_t n_chain = 0, n_transfer = 0, n_prefix = 0;  // CTAs of the three passes
+    std::vector<uint8_t> tables;  // chunk table | chain | chain segments | transfers | prefix rows
+    size_t off_chain = 0, off_seg = 0, off_transfer = 0, off_prefix = 0;
+};
+bool plan_packed(const int64_t *cu_seqlens, int64_t N, int64_t H, int sm_count, PackedPlan *plan);
+size_t packed_workspace_bytes(const PackedPlan &plan);
+cudaError_t launch_fwd_split_packed(const FwdProblem &p, const PackedPlan &plan, void *workspace,
+                                    cudaStream_t stream);
 
 }  // namespace gdn

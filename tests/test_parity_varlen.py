@@ -85,3 +85,32 @@ def test_rejects_bad_offsets():
     for cu in ([0, 20, 10], [1, 10, 30], [0, 10, 29]):
         with pytest.raises(gdn.GdnError):
             gdn.forward_varlen(d["q"], d["k"], d["v"], d["log_alpha"], d["beta"], cu, chunk=64)
+
+
+@pytest.mark.parametrize("lengths,nseg,alpha_mu", [
+    ([1000, 65, 0, 300, 1], "3", 0.0),      # the 16-chunk sequence cut 6 + 6 + 4, its last chunk partial
+    ([768, 768, 64], "4", 0.0),             # whole-chunk sequences cut 3 + 3 + 3 + 3
+    ([64 * 40 + 17, 130, 2000], "5", -1.75),  # decay that makes some transfers negligible, not all
+    ([64 * 40 + 17, 130, 2000], "5", -3.0),
+])
+def test_long_sequences_cut_into_segments(monkeypatch, lengths, nseg, alpha_mu):
+    """Sequences longer than the segment length run as segments: transfers of every segment but
+    the last, a prefix over them from the sequence's S0, and outputs from each segment's entry
+    state.  Shorter sequences in the same batch run whole.  GDN_SEGMENTS cuts the longest
+    sequence into that many segments."""
+    monkeypatch.setenv("GDN_SEGMENTS", nseg)
+    inp = varlen_inputs(lengths, 3, 128, 128, "bf16", seed=sum(lengths) + int(nseg), s0_std=0.1, alpha_mu=alpha_mu)
+    check(inp, "bf16", 64, label="%s cut %s" % (lengths, nseg))
+
+
+def test_one_long_sequence_among_short_ones_is_cut_by_the_planner(monkeypatch):
+    """Without an override the planner cuts a sequence that would outlast every other SM's work:
+    one 16K-token sequence beside three short ones, 4 heads."""
+    monkeypatch.delenv("GDN_SEGMENTS", raising=False)
+    inp = varlen_inputs([16384 + 33, 100, 2000, 64], 4, 128, 128, "bf16", seed=91, s0_std=0.05, alpha_mu=-3.0)
+    gdn.timing_start()
+    try:
+        check(inp, "bf16", 64, label="planner cut")
+    finally:
+        kinds = gdn.timing_stop()
+    assert {"prep", "transfer", "prefix", "chain"} <= set(kinds), kinds
