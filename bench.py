@@ -617,7 +617,9 @@ FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 def run_backward(args, world, rank):
     """gdn_backward over the chosen forward workload (inputs, grad_out and grad_S_final in HBM); one
     call per step.  Counted work: twice the forward's counted FLOP per token-head (the usual
-    backward-to-forward ratio of the dense contractions), against the float32 CUDA-core peak."""
+    backward-to-forward ratio of the dense contractions).  The tensor-core reverse mode (two backward
+    launches per call) is reported against the measured bf16 tensor peak, the CUDA-core one against
+    the float32 CUDA-core peak."""
     import gated_delta_rule_142_b200 as gdn
     gdn.load()
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -650,19 +652,30 @@ def run_backward(args, world, rank):
     tflops = flop / (ms_step / 1e3) / 1e12
     kernels = {kind: {"launches_per_step": n / args.steps, "ms_per_launch": kms / n, "share": kms / ms}
                for kind, (kms, n) in ktimes.items()}
+    # the library's choice: bf16, d = 128, chunk 64 on the tensor cores unless the environment asks for
+    # the CUDA-core reverse mode (whose bf16 form also launches two casts: three backward launches)
+    tensor_cores = ("backward" in ktimes and ktimes["backward"][1] == 2 * args.steps and w.dtype == "bf16"
+                    and os.environ.get("GDN_BWD_PATH") != "simt" and os.environ.get("GDN_BWD_RECOMPUTE") != "simt")
+    if tensor_cores:
+        peaks, peak_kind = load_peaks()
+        roof = {"bound": "tensor", "achieved": tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": tflops / peaks["bf16_tflops"], "traffic": None, "peak_kind": peak_kind + " bf16 burst",
+                "flop_per_step": flop}
+    else:
+        roof = {"bound": "alu", "achieved": tflops, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+                "frac": tflops / FP32_ALU_TFLOPS, "traffic": None,
+                "peak_kind": "derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz", "flop_per_step": flop}
     if rank == 0:
         line = {"metric": "gated-delta backward tokens/s", "value": world * w.B * w.T / (ms_step / 1e3),
                 "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "f32", "data": "synthetic",
+                "dtype": "bf16" if tensor_cores else "f32", "data": "synthetic",
+                "path": "tensor cores (tcgen05)" if tensor_cores else "CUDA cores",
                 "config": {"workload": w.name + "_backward", "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
                            "chunk": w.chunk, "input_dtype": w.dtype,
                            "parallelism": "replicas" if world > 1 else "single"},
                 "tflops": tflops,
-                "roofline": {"bound": "alu", "achieved": tflops, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
-                             "frac": tflops / FP32_ALU_TFLOPS, "traffic": None,
-                             "peak_kind": "derived: 148 SMs x 128 FP32 lanes x 2 x 1.965 GHz",
-                             "flop_per_step": flop},
+                "roofline": roof,
                 "kernels": kernels, "clocks": clocks,
                 "gpu_launches": sum(int(n) for _, n in ktimes.values())}
         print(json.dumps(line), flush=True)

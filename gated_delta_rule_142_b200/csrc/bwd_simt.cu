@@ -701,9 +701,14 @@ cudaError_t launch_t(const BwdProblem &p, int sm_count, void *workspace, cudaStr
     if (!f32) {
         const int64_t n4 = ntok * f.dk / 4;
         const unsigned grid = (unsigned)(n4 / 256 + 1 < (int64_t)sm_count * 8 ? n4 / 256 + 1 : (int64_t)sm_count * 8);
-        TimedLaunch tl_(GDN_KERNEL_BACKWARD, stream);
-        cast_bf16_kernel<<<grid, 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16 *>(p.dq), n4);
-        cast_bf16_kernel<<<grid, 256, 0, stream>>>(dk_acc, static_cast<__nv_bfloat16 *>(p.dk), n4);
+        {
+            TimedLaunch tl_(GDN_KERNEL_BACKWARD, stream);
+            cast_bf16_kernel<<<grid, 256, 0, stream>>>(dq_acc, static_cast<__nv_bfloat16 *>(p.dq), n4);
+        }
+        {
+            TimedLaunch tl_(GDN_KERNEL_BACKWARD, stream);
+            cast_bf16_kernel<<<grid, 256, 0, stream>>>(dk_acc, static_cast<__nv_bfloat16 *>(p.dk), n4);
+        }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;

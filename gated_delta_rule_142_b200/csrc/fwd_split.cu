@@ -135,15 +135,19 @@ struct PrepArgs {
     const int2 *ctab;  // packed chunk table, or nullptr for fixed-length problems
     int raw_inputs;    // q, k not yet L2-normalised; log_alpha, beta hold the gate logits
     int group;         // grouped heads: k and the gates have H / group heads (head h / group)
+    // or nullptr: T = (I + A)^{-1} of every item, bf16 [items][64][64] row-major (the backward's
+    // recompute); only the lower triangle is written, the caller zeroes the rest
+    __nv_bfloat16 *t_out;
 };
 
 // Writes entries (row, col) and (row, col + 1) (col even) of T diag(beta) and T diag(bgk) into
-// their bf16 K-major 128-byte-swizzled tiles.
+// their bf16 K-major 128-byte-swizzled tiles, and of T itself into `tout` (row-major, or nullptr).
 __device__ __forceinline__ void store_tb_tbg(uint8_t *tb, uint8_t *tbg, int row, int col, float v0, float v1,
-                                             const float *bet, const float *bgk) {
+                                             const float *bet, const float *bgk, __nv_bfloat16 *tout) {
     const uint32_t off = sw128(row, col >> 3) + (col & 7) * 2;
     *reinterpret_cast<uint32_t *>(tb + off) = pack_bf16x2(v0 * bet[col], v1 * bet[col + 1]);
     *reinterpret_cast<uint32_t *>(tbg + off) = pack_bf16x2(v0 * bgk[col], v1 * bgk[col + 1]);
+    if (tout) *reinterpret_cast<uint32_t *>(tout + row * 64 + col) = pack_bf16x2(v0, v1);
 }
 
 __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
@@ -342,6 +346,7 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int it = 0; it < nit && ok; ++it) {
             const uint32_t par = it & 1;
             const int gi = (int)item(it);
+            __nv_bfloat16 *const tout = p.t_out ? p.t_out + (int64_t)gi * 4096 : nullptr;
             float *g = reinterpret_cast<float *>(sm + PO_PG) + par * kPG;
             // beta, gamma, e^{g - c}, e^{c - g}, beta gamma (the last two carry 1 / |k_s| once the input
             // stage below has run)
@@ -526,6 +531,10 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const uint32_t off = sw128(row, col >> 3);
                 *reinterpret_cast<uint4 *>(sm + PO_TB + off) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
                 *reinterpret_cast<uint4 *>(sm + PO_TBG + off) = make_uint4(wg[0], wg[1], wg[2], wg[3]);
+                if (tout)
+                    *reinterpret_cast<uint4 *>(tout + row * 64 + col) =
+                        make_uint4(pack_bf16x2(xv[0], xv[1]), pack_bf16x2(xv[2], xv[3]), pack_bf16x2(xv[4], xv[5]),
+                                   pack_bf16x2(xv[6], xv[7]));
             } else {
                 const int q0 = (pw >> 1) * 32, n0 = (pw & 1) * 8;
                 float *xs = Xs + pw * 128;  // [16][8]
@@ -549,8 +558,8 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     mma_tf32(e, a, bb);
                 }
                 store_neg_d(Tm, LDM, q0 + 16, q0 + n0, e, g8, t4);
-                store_tb_tbg(sm + PO_TB, sm + PO_TBG, q0 + 16 + g8, q0 + n0 + 2 * t4, -e[0], -e[1], bet, bgm);
-                store_tb_tbg(sm + PO_TB, sm + PO_TBG, q0 + 24 + g8, q0 + n0 + 2 * t4, -e[2], -e[3], bet, bgm);
+                store_tb_tbg(sm + PO_TB, sm + PO_TBG, q0 + 16 + g8, q0 + n0 + 2 * t4, -e[0], -e[1], bet, bgm, tout);
+                store_tb_tbg(sm + PO_TB, sm + PO_TBG, q0 + 24 + g8, q0 + n0 + 2 * t4, -e[2], -e[3], bet, bgm, tout);
             }
             named_bar(kBarP, kNumPrep);
             SDBG(1, 4)
@@ -577,8 +586,8 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     load_b(bb, x2, LDX2, 8 * kk, 8 * ni, g8, t4);
                     mma_tf32(e, a, bb);
                 }
-                store_tb_tbg(sm + PO_TB, sm + PO_TBG, 32 + 16 * mi + g8, 8 * ni + 2 * t4, -e[0], -e[1], bet, bgm);
-                store_tb_tbg(sm + PO_TB, sm + PO_TBG, 40 + 16 * mi + g8, 8 * ni + 2 * t4, -e[2], -e[3], bet, bgm);
+                store_tb_tbg(sm + PO_TB, sm + PO_TBG, 32 + 16 * mi + g8, 8 * ni + 2 * t4, -e[0], -e[1], bet, bgm, tout);
+                store_tb_tbg(sm + PO_TB, sm + PO_TBG, 40 + 16 * mi + g8, 8 * ni + 2 * t4, -e[2], -e[3], bet, bgm, tout);
             }
             fence_proxy_async_smem();
             named_bar(kBarP, kNumPrep);
@@ -717,6 +726,7 @@ struct ChainArgs {
     __nv_bfloat16 *out;    // for the plain stores of partial packed chunks
     float *ckpt;           // fixed-length only, or nullptr: the state entering every chunk,
                            // [B*H][chunks][dv][dk] float32 (the backward's checkpoints)
+    int ckpt_bf16;         // the checkpoints in bf16 instead (same layout)
     int group;             // grouped heads: k and v have H / group heads (head h / group)
 };
 
@@ -1038,17 +1048,22 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 uint32_t r[32];
                 tmem_ld32(tm + lb + TC_S + col0, r);
                 tmem_wait_ld();
-                if (p.ckpt) {  // the state entering chunk c, as a checkpoint
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 32; i += 2)
+                    pk[i >> 1] = pack_bf16x2(__uint_as_float(r[i]), __uint_as_float(r[i + 1]));
+                if (p.ckpt && p.ckpt_bf16) {  // the state entering chunk c, as a bf16 checkpoint
+                    uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.ckpt) +
+                                                           (witem(c) * kD + j) * kD + col0);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                } else if (p.ckpt) {  // the state entering chunk c, as a checkpoint
                     float4 *dst = reinterpret_cast<float4 *>(p.ckpt + (witem(c) * kD + j) * kD + col0);
 #pragma unroll
                     for (int i = 0; i < 8; ++i)
                         dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
                                              __uint_as_float(r[4 * i + 2]), __uint_as_float(r[4 * i + 3]));
                 }
-                uint32_t pk[16];
-#pragma unroll
-                for (int i = 0; i < 32; i += 2)
-                    pk[i >> 1] = pack_bf16x2(__uint_as_float(r[i]), __uint_as_float(r[i + 1]));
                 tmem_st16(tm + lb + sb + col0 / 2, pk);
             }
             tmem_wait_st();
@@ -1586,6 +1601,12 @@ size_t seg_flag_bytes(const FwdProblem &p, int nseg) {
     return nseg > 1 ? (((size_t)(p.B * p.H) * (size_t)(nseg - 1) * sizeof(int) + 255) & ~(size_t)255) : 0;
 }
 
+void fwd_split_ws_tiles(void *workspace, int64_t items, void **p_tiles, void **tb_tiles) {
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    *p_tiles = ws;
+    *tb_tiles = ws + items * kTileP;
+}
+
 size_t fwd_split_workspace_bytes(const FwdProblem &p, int nseg) {
     const size_t items = (size_t)(p.B * p.H) * (size_t)((p.T + kC - 1) / kC);
     return items * kWsPerChunk + fwd_tc_workspace_bytes(p, nseg) + seg_flag_bytes(p, nseg);
@@ -1623,6 +1644,7 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
     pa.ctab = nullptr;
     pa.raw_inputs = p.raw_inputs;
     pa.group = p.group;
+    pa.t_out = static_cast<__nv_bfloat16 *>(p.t_out);
     const int64_t pgrid =
         items < kPrepCtasPerSm * (int64_t)sm_count ? items : kPrepCtasPerSm * (int64_t)sm_count;
     {
@@ -1651,6 +1673,7 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
     a.ctab = nullptr;
     a.out = static_cast<__nv_bfloat16 *>(p.out);
     a.ckpt = p.ckpt;
+    a.ckpt_bf16 = p.ckpt_bf16;
     a.group = p.group;
     if (a.nseg > 1) {
         const size_t per = (size_t)heads * (a.nseg - 1) * kD * kD;
@@ -1856,6 +1879,7 @@ cudaError_t launch_fwd_split_packed(const FwdProblem &p, const PackedPlan &pl, v
         pa.ctab = d_ctab;
         pa.raw_inputs = p.raw_inputs;
         pa.group = 1;
+        pa.t_out = nullptr;
         const int64_t pgrid =
             items < kPrepCtasPerSm * (int64_t)sm_count ? items : kPrepCtasPerSm * (int64_t)sm_count;
         TimedLaunch tl_(GDN_KERNEL_PREP, stream);
@@ -1882,6 +1906,7 @@ cudaError_t launch_fwd_split_packed(const FwdProblem &p, const PackedPlan &pl, v
     a.ctab = d_ctab;
     a.out = static_cast<__nv_bfloat16 *>(p.out);
     a.ckpt = nullptr;
+    a.ckpt_bf16 = 0;
     a.group = 1;
     if (pl.n_transfer > 0) {
         // transfers of every segment but the last of each cut sequence, then the entry states

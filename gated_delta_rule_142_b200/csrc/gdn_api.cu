@@ -868,12 +868,25 @@ extern "C" int gdn_backward(const void *q, const void *k, const void *v, const f
                            : cudaMemsetAsync(p.dS0, 0, (size_t)nstate, stream);
     } else {
         void *ws = nullptr;
-        if (scratch_alloc(&ws, gdn::bwd_simt_workspace_bytes(p, info.sm_count), stream) != cudaSuccess) {
-            cudaGetLastError();
-            return GDN_ERR_ALLOC;
+        bool done = false;
+        if (gdn::bwd_tc_supported(p)) {
+            // the tensor-core reverse mode; without room for its workspace, the CUDA-core one below
+            if (scratch_alloc(&ws, gdn::bwd_tc_workspace_bytes(p, info.sm_count), stream) == cudaSuccess) {
+                e = gdn::launch_bwd_tc(p, info.sm_count, ws, stream);
+                cudaFreeAsync(ws, stream);
+                done = true;
+            } else {
+                cudaGetLastError();
+            }
         }
-        e = gdn::launch_bwd_simt(p, info.sm_count, ws, stream);
-        cudaFreeAsync(ws, stream);
+        if (!done) {
+            if (scratch_alloc(&ws, gdn::bwd_simt_workspace_bytes(p, info.sm_count), stream) != cudaSuccess) {
+                cudaGetLastError();
+                return GDN_ERR_ALLOC;
+            }
+            e = gdn::launch_bwd_simt(p, info.sm_count, ws, stream);
+            cudaFreeAsync(ws, stream);
+        }
     }
     if (e != cudaSuccess) {
         cudaGetLastError();
@@ -1087,8 +1100,9 @@ extern "C" int gdn_device_status(void *stream_) {
         return GDN_ERR_LAUNCH;
     }
     // take every word (each read clears it), then report
-    const bool a = gdn::take_split_timeout(), b = gdn::take_tc_timeout(), c = gdn::take_selftest_timeout();
-    return (a || b || c) ? GDN_ERR_DEVICE_TIMEOUT : GDN_OK;
+    const bool a = gdn::take_split_timeout(), b = gdn::take_tc_timeout(), c = gdn::take_selftest_timeout(),
+               d = gdn::take_bwd_timeout();
+    return (a || b || c || d) ? GDN_ERR_DEVICE_TIMEOUT : GDN_OK;
 }
 
 extern "C" int gdn_selftest_device_timeout(void *stream_) {

@@ -63,6 +63,11 @@ struct FwdProblem {
     // gates have H / group heads; S0 / S_final stay per query head, expanded by the caller).
     // The two-kernel and the CUDA-core forwards take it.
     int group = 1;
+    // two-kernel forward, for the tensor-core backward's recompute: checkpoints in bf16 instead of
+    // float32, and T = (I + A)^{-1} of every chunk into t_out (bf16 [B*H*chunks][64][64], lower
+    // triangle written; the caller zeroes the rest), or nullptr
+    int ckpt_bf16 = 0;
+    void *t_out = nullptr;
 };
 
 struct DecodeProblem {
@@ -133,6 +138,13 @@ struct BwdProblem {
 };
 size_t bwd_simt_workspace_bytes(const BwdProblem &p, int sm_count);
 cudaError_t launch_bwd_simt(const BwdProblem &p, int sm_count, void *workspace, cudaStream_t stream);
+// bwd_tc.cu -- the same reverse mode on the tensor cores (bf16, dk = dv = 128, chunk = 64, one head
+// per memory): a forward recompute, a reverse chain over the chunks of each (b, h) and a
+// chunk-parallel gradient pass.
+bool bwd_tc_supported(const BwdProblem &p);
+size_t bwd_tc_workspace_bytes(const BwdProblem &p, int sm_count);
+cudaError_t launch_bwd_tc(const BwdProblem &p, int sm_count, void *workspace, cudaStream_t stream);
+bool take_bwd_timeout();
 
 // fwd_tc.cu -- tcgen05 chunkwise forward: bf16, dk = dv = 128, chunk = 64.
 // Long sequences with few (b, h) are cut into segments: a transfer pass, a
@@ -156,6 +168,8 @@ cudaError_t launch_seg_prefix(const float *S0, const float *Bw, const float *Mw,
 // per chunk plus the segment scratch of fwd_tc_workspace_bytes.
 bool fwd_split_supported(const FwdProblem &p);
 size_t fwd_split_workspace_bytes(const FwdProblem &p, int nseg);
+// The P and T diag(beta) tiles (bf16 [items][64][64] each) inside a two-kernel workspace.
+void fwd_split_ws_tiles(void *workspace, int64_t items, void **p_tiles, void **tb_tiles);
 cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *workspace, cudaStream_t stream);
 // Packed variable-length sequences (p.B = 1, p.T = total tokens; cu_seqlens on the host, N + 1
 // entries).  plan_packed builds the host tables: the chunk table over the packed tokens and the

@@ -109,3 +109,39 @@ def test_empty_sequence_passes_the_final_gradient_through():
                        dSf.cuda(), chunk=16)
     torch.cuda.synchronize()
     assert torch.equal(got[5].cpu(), dSf)
+
+
+@pytest.mark.parametrize("B,T,H,s0,final", [(1, 64, 1, True, True), (2, 300, 3, True, False), (1, 1000, 2, False, True),
+                                            (3, 128, 4, False, False)])
+def test_tensor_core_backward(monkeypatch, B, T, H, s0, final):
+    """bf16, d = 128, chunk 64 runs the tensor-core reverse mode (a reverse chain and a
+    chunk-parallel gradient pass: two backward launches, where the CUDA-core one takes three with its
+    two bf16 casts); whole chunks, ragged last chunks, with and without S0 and dS_final."""
+    monkeypatch.delenv("GDN_BWD_PATH", raising=False)
+    monkeypatch.delenv("GDN_BWD_RECOMPUTE", raising=False)
+    inp = forward_inputs(B, T, H, 128, 128, "bf16", seed=600 + T + H, s0_std=0.5 if s0 else None)
+    d_out, dSf = grads_in(B, T, H, 128, 128, "bf16", seed=700 + T, final=final)
+    gdn.timing_start()
+    try:
+        check(inp, d_out, dSf, "bf16", 64, label="tc B%d T%d H%d" % (B, T, H))
+    finally:
+        kinds = gdn.timing_stop()
+    assert kinds["backward"][1] == 2, kinds
+
+
+def test_tensor_core_and_cuda_core_backward_agree(monkeypatch):
+    """The two reverse modes on the same inputs: each meets the bar against the oracle, and they
+    agree with each other within it."""
+    inp = forward_inputs(2, 200, 2, 128, 128, "bf16", seed=811, s0_std=0.3)
+    d_out, dSf = grads_in(2, 200, 2, 128, 128, "bf16", seed=812)
+    monkeypatch.delenv("GDN_BWD_PATH", raising=False)
+    a = check(inp, d_out, dSf, "bf16", 64, label="tensor cores")
+    monkeypatch.setenv("GDN_BWD_PATH", "simt")
+    gdn.timing_start()
+    try:
+        b = check(inp, d_out, dSf, "bf16", 64, label="cuda cores")
+    finally:
+        kinds = gdn.timing_stop()
+    assert kinds["backward"][1] == 3, kinds
+    for x, y in zip(a, b):
+        assert rel_err(cpu_f64(x), cpu_f64(y)) <= TOL["bf16"]
