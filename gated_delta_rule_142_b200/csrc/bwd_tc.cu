@@ -144,8 +144,9 @@ constexpr uint32_t IDESC_128_KK = instr_desc_bf16(128, 128, 0, 0);
 // ============================================================================
 // pass 1: reverse chain
 // ============================================================================
-constexpr int kP1Threads = 160;  // warps 0-3: the chain (thread j = TMEM lane = value dim j); warp 4: TMA
-constexpr int kP1Compute = 128;
+constexpr int kP1Threads = 288;  // warps 0-7: the chain, two per TMEM lane quadrant (value dim j = lane
+                                 // 32 (w & 3) + lane, column half w >> 2); warp 8: TMA
+constexpr int kP1Compute = 256;
 constexpr int kBarP1 = 1;
 
 constexpr uint32_t S1_DO = 0;       // 16 KB: dO, two [64 t][64 j] boxes
@@ -217,7 +218,7 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
     tc_fence_after();
     const uint32_t tm = *tmem_slot;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ============================ producer ============================
         if (lane == 0) {
             bool ok = true;
@@ -241,13 +242,14 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
         __syncwarp();
     } else {
         // ============================ the chain ============================
-        const int j = tid;  // value dim = TMEM lane
-        const uint32_t lb = (uint32_t)(warp * 32) << 16;
+        const int j = (warp & 3) * 32 + lane;  // value dim = TMEM lane
+        const int ch = warp >> 2;             // column half
+        const uint32_t lb = (uint32_t)((warp & 3) * 32) << 16;
         bool ok = true;
         uint32_t mph = 0;  // phase of the next wait on B1_MMA
         // dS <- dS_final (or zero)
 #pragma unroll 1
-        for (int pc = 0; pc < 4; ++pc) {
+        for (int pc = 2 * ch; pc < 2 * ch + 2; ++pc) {
             uint32_t r[32];
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
@@ -295,8 +297,8 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             }
             // ---- Q rows scaled by gamma_t in place (16-byte unit u: box u >> 9, row (u >> 3) & 63) ----
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int u = tid + 128 * i;
+            for (int i = 0; i < 4; ++i) {
+                const int u = tid + 256 * i;
                 uint4 *ptr = reinterpret_cast<uint4 *>(st + S1_Q) + u;
                 float f[8];
                 unpack8(*ptr, f);
@@ -310,7 +312,7 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             {
                 __nv_bfloat16 *dsg = p.ds_ws + (item * kD + j) * kD;
 #pragma unroll 1
-                for (int pc = 0; pc < 4; ++pc) {
+                for (int pc = 2 * ch; pc < 2 * ch + 2; ++pc) {
                     uint32_t r[32];
                     tmem_ld32(tm + lb + T1_DS + 32 * pc, r);
                     tmem_wait_ld();
@@ -345,8 +347,8 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             mma_round();
             if (!ok) break;
             // ---- dU^T = dO^T P + (dS K^T) diag(dl), in bf16 ----
-#pragma unroll 1
-            for (int pc = 0; pc < 2; ++pc) {
+            {
+                const int pc = ch;
                 uint32_t a[32], d2[32];
                 tmem_ld32(tm + lb + T1_DU + 32 * pc, a);
                 tmem_ld32(tm + lb + T1_D2 + 32 * pc, d2);
@@ -375,20 +377,24 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             {
                 __nv_bfloat16 *drg = p.dr_ws + item * kC * kD + j;
                 __nv_bfloat16 *dvg = p.dv + (((int64_t)b * T + t0) * H + h) * kD + j;
-#pragma unroll 1
-                for (int pc = 0; pc < 2; ++pc) {
+                {
+                    const int pc = ch;
                     uint32_t r[32];
                     tmem_ld32(tm + lb + T1_DR + 32 * pc, r);
                     tmem_wait_ld();
                     uint32_t pk[16];
+                    const int64_t vstr = H * kD;  // token stride of dV
+                    __nv_bfloat16 *dr_row = drg + (int64_t)(32 * pc) * kD, *dv_row = dvg + (int64_t)(32 * pc) * vstr;
 #pragma unroll
                     for (int i = 0; i < 32; i += 2) {
                         const int t = 32 * pc + i;
                         const float x0 = __uint_as_float(r[i]), x1 = __uint_as_float(r[i + 1]);
-                        drg[(int64_t)t * kD] = __float2bfloat16_rn(x0);
-                        drg[(int64_t)(t + 1) * kD] = __float2bfloat16_rn(x1);
-                        if (t < n) dvg[(int64_t)t * H * kD] = __float2bfloat16_rn(bet[t] * x0);
-                        if (t + 1 < n) dvg[(int64_t)(t + 1) * H * kD] = __float2bfloat16_rn(bet[t + 1] * x1);
+                        dr_row[i * kD] = __float2bfloat16_rn(x0);
+                        dr_row[(i + 1) * kD] = __float2bfloat16_rn(x1);
+                        if (t < n) *dv_row = __float2bfloat16_rn(bet[t] * x0);
+                        dv_row += vstr;
+                        if (t + 1 < n) *dv_row = __float2bfloat16_rn(bet[t + 1] * x1);
+                        dv_row += vstr;
                         pk[i >> 1] = pack_bf16x2(-bet[t] * gam[t] * x0, -bet[t + 1] * gam[t + 1] * x1);
                     }
                     tmem_st16(tm + lb + T1_DRB + 16 * pc, pk);
@@ -413,7 +419,7 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
         // dS0: the adjoint of the state entering chunk 0
         if (ok && p.dS0) {
 #pragma unroll 1
-            for (int pc = 0; pc < 4; ++pc) {
+            for (int pc = 2 * ch; pc < 2 * ch + 2; ++pc) {
                 uint32_t r[32];
                 tmem_ld32(tm + lb + T1_DS + 32 * pc, r);
                 tmem_wait_ld();
@@ -438,7 +444,7 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
 // ============================================================================
 // pass 2: chunk-parallel gradients
 // ============================================================================
-constexpr int kP2Threads = 128;  // thread m = TMEM lane m
+constexpr int kP2Threads = 256;  // two threads per TMEM lane: row m = 32 (w & 3) + lane, column half w >> 2
 
 constexpr uint32_t R_QK = 0;        // 32 KB: box b = [Q rows 0-63 | K rows 64-127] x columns 64b..64b+63
 constexpr uint32_t R_DOR = 32768;   // 32 KB: box b = [dO rows 0-63 | dR rows 64-127]
@@ -479,11 +485,13 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float *g = reinterpret_cast<float *>(sm + R_F), *bet = g + 64, *gam = g + 128, *dl = g + 192, *dg = g + 256,
           *db = g + 320, *colsum = g + 384, *misc = g + 448;  // misc: scan scratch, <dS', S>, sum of w
 
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t H = p.H, T = p.T;
     const int nch = p.chunks;
     const uint32_t sbase = smem_u32(sm);
-    const uint32_t lb = (uint32_t)(warp * 32) << 16;
+    const int m = (warp & 3) * 32 + lane;  // TMEM lane / row of the 128-row tiles
+    const int ch = warp >> 2;              // column half
+    const uint32_t lb = (uint32_t)((warp & 3) * 32) << 16;
 
     if (tid == 0) {
         for (int i = 0; i < B2_COUNT; ++i) mbar_init(&bars[i], 1);
@@ -573,12 +581,13 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             mma_commit(&bars[B2_MMA]);
         }
-        // <dS'_j, S_j> for d g_C, while round 1 runs (row j = tid of both bf16 tiles)
+        // <dS'_j, S_j> for d g_C, while round 1 runs (row j = m of both bf16 tiles, this thread's
+        // 64-column box)
         {
             float acc = 0.f;
 #pragma unroll
-            for (int q = 0; q < 16; ++q) {
-                const uint32_t off = (q >> 3) * 16384 + sw128(tid, q & 7);
+            for (int q = 0; q < 8; ++q) {
+                const uint32_t off = ch * 16384 + sw128(m, q);
                 float x[8], y[8];
                 unpack8(*reinterpret_cast<const uint4 *>(sm + R_DS + off), x);
                 unpack8(*reinterpret_cast<const uint4 *>(sm + R_S + off), y);
@@ -592,11 +601,11 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mma_round();
         if (!ok) break;
         // ---- epilogue 1: rows t: d g_t from the outputs' gamma_t Q S^T term; rows 64 + t: X, Y ----
-        if (tid < 64) {
-            const int t = tid;
+        if (m < 64) {
+            const int t = m;
             float acc = 0.f;
 #pragma unroll 1
-            for (int pc = 0; pc < 4; ++pc) {
+            for (int pc = 2 * ch; pc < 2 * ch + 2; ++pc) {
                 uint32_t z[32];
                 tmem_ld32(tm + lb + T2_Z + 32 * pc, z);
                 tmem_wait_ld();
@@ -611,11 +620,11 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             atomicAdd(&dg[t], gam[t] * acc);
         } else {
-            const int t = tid - 64;
+            const int t = m - 64;
             const float gt = gam[t], bt = bet[t];
             float ry = 0.f, rx = 0.f;
 #pragma unroll 1
-            for (int pc = 0; pc < 4; ++pc) {
+            for (int pc = 2 * ch; pc < 2 * ch + 2; ++pc) {
                 uint32_t z[32];
                 tmem_ld32(tm + lb + T2_Z + 32 * pc, z);
                 tmem_wait_ld();
@@ -653,9 +662,9 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (!ok) break;
         // ---- epilogue 2 (row j = tid): U^T into shared memory in bf16; w_s = dl_s sum_j U^T_js D2_js ----
         {
-            const int j = tid;
-#pragma unroll 1
-            for (int pc = 0; pc < 2; ++pc) {
+            const int j = m;
+            {
+                const int pc = ch;
                 uint32_t u[32], d2[32];
                 tmem_ld32(tm + lb + T2_U + 32 * pc, u);
                 tmem_ld32(tm + lb + T2_D2 + 32 * pc, d2);
@@ -670,7 +679,7 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 float v[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(u[i]) * __uint_as_float(d2[i]);
-                atomicAdd(&colsum[32 * pc + (tid & 31)], warp_colsum32(v));
+                atomicAdd(&colsum[32 * pc + lane], warp_colsum32(v));
             }
         }
         publish_smem();  // also publishes colsum
@@ -694,15 +703,16 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mma_round();
         if (!ok) break;
         // ---- epilogue 3: dP o E, F, their d g and dbeta terms; the A1 operand of round 4 ----
-        if (tid < 64) {
-            const int t = tid;
+        if (m < 64) {
+            const int t = m;
             const float gt = g[t];
             float rs = 0.f;
-            // A1 row t, columns 0..63: zero
+            // A1 row t, columns 0..63: zero (each thread of the row half of them)
 #pragma unroll
-            for (int q = 0; q < 8; ++q) *reinterpret_cast<uint4 *>(sm + R_A1 + sw128(t, q)) = make_uint4(0, 0, 0, 0);
-#pragma unroll 1
-            for (int pc = 0; pc < 2; ++pc) {
+            for (int q = 4 * ch; q < 4 * ch + 4; ++q)
+                *reinterpret_cast<uint4 *>(sm + R_A1 + sw128(t, q)) = make_uint4(0, 0, 0, 0);
+            {
+                const int pc = ch;
                 uint32_t a[32], qk[32];
                 tmem_ld32(tm + lb + T2_DG + 32 * pc, a);
                 tmem_ld32(tm + lb + T2_G + 32 * pc, qk);
@@ -726,15 +736,15 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     *reinterpret_cast<uint4 *>(sm + R_A1 + 16384 + sw128(t, 4 * pc + q)) =
                         make_uint4(pack_bf16x2(pe[8 * q], pe[8 * q + 1]), pack_bf16x2(pe[8 * q + 2], pe[8 * q + 3]),
                                    pack_bf16x2(pe[8 * q + 4], pe[8 * q + 5]), pack_bf16x2(pe[8 * q + 6], pe[8 * q + 7]));
-                atomicAdd(&colsum[32 * pc + (tid & 31)], warp_colsum32(cv));
+                atomicAdd(&colsum[32 * pc + lane], warp_colsum32(cv));
             }
             atomicAdd(&dg[t], rs);
         } else {
-            const int t = tid - 64;
+            const int t = m - 64;
             const float gt = g[t], bt = bet[t];
             float rs = 0.f, bs = 0.f;
-#pragma unroll 1
-            for (int pc = 0; pc < 2; ++pc) {
+            {
+                const int pc = ch;
                 uint32_t a[32], kk2[32];
                 tmem_ld32(tm + lb + T2_DG + 32 * pc, a);
                 tmem_ld32(tm + lb + T2_G + 32 * pc, kk2);
@@ -762,7 +772,7 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                         *reinterpret_cast<uint16_t *>(sm + R_A1 + 16384 + sw128(64 + t, s >> 3) + (s & 7) * 2) =
                             bf16_bits(f);
                 }
-                atomicAdd(&colsum[32 * pc + (tid & 31)], warp_colsum32(cv));
+                atomicAdd(&colsum[32 * pc + lane], warp_colsum32(cv));
             }
             atomicAdd(&dg[t], rs);
             atomicAdd(&db[t], bs);
@@ -790,12 +800,12 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (tid == 0 && item + gridDim.x < p.items) issue_loads(item + gridDim.x);
         // ---- epilogue 4: dQ (rows t), dK (rows 64 + s) ----
         {
-            const int r = tid & 63;
-            const bool isq = tid < 64;
+            const int r = m & 63;
+            const bool isq = m < 64;
             const float f2 = isq ? gam[r] : -bet[r] * gam[r], f3 = dl[r];
             __nv_bfloat16 *dst = (isq ? p.dq : p.dk) + (((int64_t)b * T + t0 + r) * H + h) * kD;
 #pragma unroll 1
-            for (int pc = 0; pc < 4; ++pc) {
+            for (int pc = 2 * ch; pc < 2 * ch + 2; ++pc) {
                 uint32_t x1[32], x2[32], x3[32];
                 tmem_ld32(tm + lb + T2_H1 + 32 * pc, x1);
                 tmem_ld32(tm + lb + T2_H2 + 32 * pc, x2);
