@@ -42,7 +42,8 @@ EXPORTS = ("gdn_forward", "gdn_decode_step", "gdn_forward_plan", "gdn_status_str
            "gdn_device_status", "gdn_selftest_device_timeout", "gdn_forward_conv")
 
 # gdn_kernel_kind names, in enum order
-KERNEL_KINDS = ("prep", "chain", "transfer", "prefix", "fused", "simt", "decode", "input", "backward")
+KERNEL_KINDS = ("prep", "chain", "transfer", "prefix", "fused", "simt", "decode", "input", "backward",
+                "group_out")
 
 
 class GdnError(RuntimeError):

@@ -727,6 +727,11 @@ struct ChainArgs {
     float *ckpt;           // fixed-length only, or nullptr: the state entering every chunk,
                            // [B*H][chunks][dv][dk] float32 (the backward's checkpoints)
     int ckpt_bf16;         // the checkpoints in bf16 instead (same layout)
+    // one memory per key-value head (fixed-length problems): lead = group runs the transfers and the
+    // chain for query heads hk * group only (the CTA's state index bh then counts (b, hk); S0,
+    // S_final, the segment slots, the checkpoints and u_out follow it), 1 runs every head
+    int lead;
+    __nv_bfloat16 *u_out;  // or nullptr: U^T of every chunk, bf16 [bh][chunks][128][64]
     int group;             // grouped heads: k and v have H / group heads (head h / group)
 };
 
@@ -764,8 +769,9 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     } else {
         bh = blockIdx.x / p.nseg;
         const int seg = (int)(blockIdx.x % p.nseg);
-        b = (int)(bh / H);
-        h = (int)(bh % H);
+        const int64_t Hc = H / p.lead;  // memories per batch row
+        b = (int)(bh / Hc);
+        h = (int)(bh % Hc) * p.lead;
         c0 = seg * p.seg_len;
         N = (p.chunks - c0 < p.seg_len) ? (p.chunks - c0) : p.seg_len;
         entry_slot = seg == 0 ? -1 : bh * (p.nseg - 1) + seg - 1;
@@ -773,7 +779,10 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     auto tok0 = [&](int c) -> int { return packed ? p.ctab[c0 + c].x : (c0 + c) * kC; };
     auto ntok = [&](int c) -> int { return packed ? p.ctab[c0 + c].y : kC; };  // TMA clips at T otherwise
-    auto witem = [&](int c) -> int64_t { return packed ? (int64_t)(c0 + c) * H + h : bh * p.chunks + c0 + c; };
+    auto witem = [&](int c) -> int64_t {
+        return packed ? (int64_t)(c0 + c) * H + h : ((int64_t)b * H + h) * p.chunks + c0 + c;
+    };
+    auto citem = [&](int c) -> int64_t { return bh * p.chunks + c0 + c; };  // checkpoints and u_out
     const uint32_t sbase = smem_u32(sm);
 
     if (tid == 0) {
@@ -1054,11 +1063,11 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     pk[i >> 1] = pack_bf16x2(__uint_as_float(r[i]), __uint_as_float(r[i + 1]));
                 if (p.ckpt && p.ckpt_bf16) {  // the state entering chunk c, as a bf16 checkpoint
                     uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(p.ckpt) +
-                                                           (witem(c) * kD + j) * kD + col0);
+                                                           (citem(c) * kD + j) * kD + col0);
 #pragma unroll
                     for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
                 } else if (p.ckpt) {  // the state entering chunk c, as a checkpoint
-                    float4 *dst = reinterpret_cast<float4 *>(p.ckpt + (witem(c) * kD + j) * kD + col0);
+                    float4 *dst = reinterpret_cast<float4 *>(p.ckpt + (citem(c) * kD + j) * kD + col0);
 #pragma unroll
                     for (int i = 0; i < 8; ++i)
                         dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
@@ -1129,6 +1138,11 @@ fwd_chain_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     pk[i >> 1] = pack_bf16x2(__uint_as_float(u[i]) + __uint_as_float(u2[i]),
                                              __uint_as_float(u[i + 1]) + __uint_as_float(u2[i + 1]));
                 tmem_st8(tm + lb + ub + ch * 16 + piece * 8, pk);
+                if (p.u_out) {  // U^T row j, tokens 32 ch + 16 piece .. + 15
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.u_out + (citem(c) * kD + j) * kC + ch * 32 + piece * 16);
+                    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                }
             }
             tmem_wait_st();
             tc_fence_before();
@@ -1263,11 +1277,12 @@ fwd_transfer_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_const
     } else {
         const int64_t bh = blockIdx.x / (p.nseg - 1);
         const int seg = (int)(blockIdx.x % (p.nseg - 1));
-        b = (int)(bh / H);
-        h = (int)(bh % H);
+        const int64_t Hc = H / p.lead;
+        b = (int)(bh / Hc);
+        h = (int)(bh % Hc) * p.lead;
         cseg = seg * p.seg_len;  // segments 0..nseg-2 are full
         slot = bh * (p.nseg - 1) + seg;
-        ibase = bh * p.chunks;
+        ibase = ((int64_t)b * H + h) * p.chunks;
         istride = 1;
     }
     auto item = [&](int c) -> int64_t { return ibase + (int64_t)c * istride; };
@@ -1598,7 +1613,12 @@ bool fwd_split_supported(const FwdProblem &p) {
 
 // Flags of the segment transfers (one int per head and segment boundary), after the segment scratch.
 size_t seg_flag_bytes(const FwdProblem &p, int nseg) {
-    return nseg > 1 ? (((size_t)(p.B * p.H) * (size_t)(nseg - 1) * sizeof(int) + 255) & ~(size_t)255) : 0;
+    return nseg > 1 ? (((size_t)(p.B * p.H / p.lead) * (size_t)(nseg - 1) * sizeof(int) + 255) & ~(size_t)255) : 0;
+}
+
+const float *fwd_split_ws_gates(const void *workspace, int64_t items) {
+    return reinterpret_cast<const float *>(static_cast<const uint8_t *>(workspace) +
+                                           items * (kTileP + kTileTB + kTileW));
 }
 
 void fwd_split_ws_tiles(void *workspace, int64_t items, void **p_tiles, void **tb_tiles) {
@@ -1613,7 +1633,9 @@ size_t fwd_split_workspace_bytes(const FwdProblem &p, int nseg) {
 }
 
 cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *workspace, cudaStream_t stream) {
-    const int64_t chunks = (p.T + kC - 1) / kC, heads = p.B * p.H, items = heads * chunks;
+    const int64_t chunks = (p.T + kC - 1) / kC, items = p.B * p.H * chunks;
+    if (p.lead < 1 || p.H % p.lead || (p.lead > 1 && p.lead != p.group)) return cudaErrorInvalidValue;
+    const int64_t heads = p.B * p.H / p.lead;  // memories: the transfer, prefix and chain CTAs' (b, h)
     if (items == 0) return cudaSuccess;
     if (!workspace) return cudaErrorInvalidValue;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -1674,6 +1696,8 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
     a.out = static_cast<__nv_bfloat16 *>(p.out);
     a.ckpt = p.ckpt;
     a.ckpt_bf16 = p.ckpt_bf16;
+    a.lead = p.lead;
+    a.u_out = static_cast<__nv_bfloat16 *>(p.u_out);
     a.group = p.group;
     if (a.nseg > 1) {
         const size_t per = (size_t)heads * (a.nseg - 1) * kD * kD;
@@ -1907,6 +1931,8 @@ cudaError_t launch_fwd_split_packed(const FwdProblem &p, const PackedPlan &pl, v
     a.out = static_cast<__nv_bfloat16 *>(p.out);
     a.ckpt = nullptr;
     a.ckpt_bf16 = 0;
+    a.lead = 1;
+    a.u_out = nullptr;
     a.group = 1;
     if (pl.n_transfer > 0) {
         // transfers of every segment but the last of each cut sequence, then the entry states

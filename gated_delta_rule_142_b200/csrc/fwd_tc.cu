@@ -998,7 +998,7 @@ int fwd_tc_segments(const FwdProblem &p, int sm_count, bool paired_transfers) {
 
 size_t fwd_tc_workspace_bytes(const FwdProblem &p, int nseg) {
     if (nseg <= 1) return 0;
-    return (size_t)3 * (size_t)(p.B * p.H) * (size_t)(nseg - 1) * kD * kD * sizeof(float);
+    return (size_t)3 * (size_t)(p.B * p.H / p.lead) * (size_t)(nseg - 1) * kD * kD * sizeof(float);
 }
 
 cudaError_t launch_seg_prefix(const float *S0, const float *Bw, const float *Mw, const int *Mflag, float *S_entry,

@@ -946,6 +946,50 @@ extern "C" int gdn_forward_grouped(const void *q, const void *k, const void *v, 
     } else if ((st = stg.in(S_final, nstate, false, &dSf))) {
         return st;
     }
+    p.out = const_cast<void *>(dout);
+    p.B = B; p.T = T; p.H = Hq; p.dk = dk; p.dv = dv; p.chunk = chunk; p.dtype = dtype;
+    p.group = group;
+    if (T > 0 && forced_path() == FwdPath::Auto && gdn::fwd_split_supported(p)) {
+        // one memory per key-value head: the two-kernel forward in lead mode (prep over every query
+        // head, transfers, prefix and chain over the key-value heads, checkpoints and U^T kept), then
+        // the other query heads' outputs from them
+        FwdProblem pl = p;
+        pl.lead = group;
+        pl.S0 = static_cast<const float *>(dS0);
+        pl.S_final = static_cast<float *>(const_cast<void *>(dSf));
+        pl.ckpt_bf16 = 1;
+        FwdProblem plan = pl;  // the planner counts memories
+        plan.H = Hkv;
+        plan.group = 1;
+        plan.lead = 1;
+        const int nseg = gdn::fwd_tc_segments(plan, info.sm_count, true);
+        const int64_t nch = (T + 63) / 64, mems = B * Hkv * nch;
+        auto round256 = [](size_t x) { return (x + 255) & ~(size_t)255; };
+        const size_t wsb = round256(gdn::fwd_split_workspace_bytes(pl, nseg)), ckb = (size_t)mems * 128 * 128 * 2,
+                     ub = (size_t)mems * 128 * 64 * 2;
+        void *ws = nullptr;
+        if (scratch_alloc(&ws, wsb + ckb + ub, stream) == cudaSuccess) {
+            uint8_t *w8 = static_cast<uint8_t *>(ws);
+            pl.ckpt = reinterpret_cast<float *>(w8 + wsb);
+            pl.u_out = w8 + wsb + ckb;
+            cudaError_t e = gdn::launch_fwd_split(pl, nseg, info.sm_count, ws, stream);
+            if (e == cudaSuccess) {
+                void *pt = nullptr, *tbt = nullptr;
+                gdn::fwd_split_ws_tiles(ws, B * Hq * nch, &pt, &tbt);
+                e = gdn::launch_grouped_outputs(pl, pl.ckpt, pl.u_out, pt, gdn::fwd_split_ws_gates(ws, B * Hq * nch),
+                                                info.sm_count, stream);
+            }
+            cudaFreeAsync(ws, stream);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                return GDN_ERR_LAUNCH;
+            }
+            if ((st = stg.out_back(out, dout, nout))) return st;
+            if ((st = stg.out_back(S_final, dSf, nstate))) return st;
+            return GDN_OK;
+        }
+        cudaGetLastError();
+    }
     // per-query-head copies of the states (each query head of a group recomputes its memory)
     void *xs = nullptr;
     if (scratch_alloc(&xs, (size_t)(2 * nxstate), stream) != cudaSuccess) {
@@ -1101,8 +1145,8 @@ extern "C" int gdn_device_status(void *stream_) {
     }
     // take every word (each read clears it), then report
     const bool a = gdn::take_split_timeout(), b = gdn::take_tc_timeout(), c = gdn::take_selftest_timeout(),
-               d = gdn::take_bwd_timeout();
-    return (a || b || c || d) ? GDN_ERR_DEVICE_TIMEOUT : GDN_OK;
+               d = gdn::take_bwd_timeout(), g = gdn::take_grouped_timeout();
+    return (a || b || c || d || g) ? GDN_ERR_DEVICE_TIMEOUT : GDN_OK;
 }
 
 extern "C" int gdn_selftest_device_timeout(void *stream_) {

@@ -68,6 +68,13 @@ struct FwdProblem {
     // triangle written; the caller zeroes the rest), or nullptr
     int ckpt_bf16 = 0;
     void *t_out = nullptr;
+    // two-kernel forward with grouped heads: lead = group runs one memory per key-value head (the
+    // transfers, prefix and chain of query heads hk * group only, with S0 / S_final, the segment
+    // scratch and the checkpoints per key-value head) and writes U^T of every chunk into u_out
+    // (bf16 [B * H / group][chunks][128][64]); the other query heads' outputs come from
+    // launch_grouped_outputs.  1: every head runs its own chain.
+    int lead = 1;
+    void *u_out = nullptr;
 };
 
 struct DecodeProblem {
@@ -170,6 +177,16 @@ bool fwd_split_supported(const FwdProblem &p);
 size_t fwd_split_workspace_bytes(const FwdProblem &p, int nseg);
 // The P and T diag(beta) tiles (bf16 [items][64][64] each) inside a two-kernel workspace.
 void fwd_split_ws_tiles(void *workspace, int64_t items, void **p_tiles, void **tb_tiles);
+// The gate records (float32 [items][132]) inside a two-kernel workspace.
+const float *fwd_split_ws_gates(const void *workspace, int64_t items);
+// grouped_out.cu -- outputs of the query heads hk * group + r (r = 1 .. group - 1) from the memory
+// of key-value head hk that a lead = group two-kernel forward left behind: its bf16 checkpoints
+// (ckpt, [B * Hkv][chunks][128][128]) and U^T (u, [B * Hkv][chunks][128][64]), with each query
+// head's P tiles and gate records from that forward's workspace (p_tiles, gates):
+// O^T = S (diag(gamma) Q)^T + U^T P^T.
+cudaError_t launch_grouped_outputs(const FwdProblem &p, const void *ckpt, const void *u, const void *p_tiles,
+                                   const float *gates, int sm_count, cudaStream_t stream);
+bool take_grouped_timeout();
 cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *workspace, cudaStream_t stream);
 // Packed variable-length sequences (p.B = 1, p.T = total tokens; cu_seqlens on the host, N + 1
 // entries).  plan_packed builds the host tables: the chunk table over the packed tokens and the

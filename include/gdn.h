@@ -413,8 +413,9 @@ typedef enum {
     GDN_KERNEL_SIMT = 5,        /* float32 CUDA-core forward                                       */
     GDN_KERNEL_DECODE = 6,      /* single-token decode step                                        */
     GDN_KERNEL_INPUT = 7,       /* input stage as a pass of its own (the *_raw forwards' fallbacks) */
-    GDN_KERNEL_BACKWARD = 8,    /* backward pass (its forward recompute counts as SIMT)            */
-    GDN_KERNEL_KINDS = 9
+    GDN_KERNEL_BACKWARD = 8,    /* backward pass (its forward recompute counts as PREP and CHAIN)  */
+    GDN_KERNEL_GROUP_OUT = 9,   /* grouped heads: outputs of the query heads sharing a memory       */
+    GDN_KERNEL_KINDS = 10
 } gdn_kernel_kind;
 int gdn_timing_start(void);
 int gdn_timing_stop(double *ms, int64_t *launches);

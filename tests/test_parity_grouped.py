@@ -33,15 +33,37 @@ def check(inp, dtype, chunk, host=False, label=""):
     assert eo <= TOL[dtype] and es <= TOL[dtype], (label, eo, es)
 
 
-@pytest.mark.parametrize("B,T,Hq,Hkv", [(1, 300, 8, 2), (2, 130, 4, 1), (1, 64, 6, 3)])
+@pytest.mark.parametrize("B,T,Hq,Hkv", [(1, 300, 8, 2), (2, 130, 4, 1), (1, 64, 6, 3), (2, 257, 16, 2)])
 def test_two_kernel_forward(B, T, Hq, Hkv):
-    """bf16, d = 128, chunk 64: the ATMA shape (8 query / 2 key-value heads) and others."""
-    check(grouped(B, T, Hq, Hkv, 128, "bf16", seed=700 + T), "bf16", 64, label="%d/%d" % (Hq, Hkv))
+    """bf16, d = 128, chunk 64: the ATMA shape (8 query / 2 key-value heads) and others.  One chain
+    per key-value head (its query head hk * G), and the other query heads' outputs from that
+    memory's checkpoints and U^T by the grouped-output kernel."""
+    gdn.timing_start()
+    try:
+        check(grouped(B, T, Hq, Hkv, 128, "bf16", seed=700 + T), "bf16", 64, label="%d/%d" % (Hq, Hkv))
+    finally:
+        kinds = gdn.timing_stop()
+    assert kinds["group_out"][1] == 1 and kinds["chain"][1] == 1, kinds
 
 
-def test_two_kernel_forward_with_segments(monkeypatch):
-    monkeypatch.setenv("GDN_SEGMENTS", "3")
-    check(grouped(1, 1000, 8, 2, 128, "bf16", seed=711, alpha_mu=-3.0), "bf16", 64, label="segments")
+@pytest.mark.parametrize("nseg", ["3", "7"])
+def test_two_kernel_forward_with_segments(monkeypatch, nseg):
+    """Segments of the key-value heads' chains: transfers, prefix and entry states per memory."""
+    monkeypatch.setenv("GDN_SEGMENTS", nseg)
+    check(grouped(1, 1000, 8, 2, 128, "bf16", seed=711, alpha_mu=-3.0), "bf16", 64, label="segments " + nseg)
+    check(grouped(2, 700, 4, 2, 128, "bf16", seed=712, alpha_mu=0.0), "bf16", 64, label="fast decay " + nseg)
+
+
+def test_other_paths_recompute_per_query_head(monkeypatch):
+    """With the two-kernel forward switched off (GDN_FORWARD_PATH=fused) grouped heads take the
+    CUDA-core forward, where each query head recomputes its memory; same bar at d = 128."""
+    monkeypatch.setenv("GDN_FORWARD_PATH", "fused")
+    gdn.timing_start()
+    try:
+        check(grouped(1, 200, 8, 2, 128, "bf16", seed=713), "bf16", 64, label="recompute")
+    finally:
+        kinds = gdn.timing_stop()
+    assert "group_out" not in kinds, kinds
 
 
 @pytest.mark.parametrize("dtype,d,chunk", [("f32", 64, 32), ("f32", 16, 16), ("bf16", 64, 64)])
