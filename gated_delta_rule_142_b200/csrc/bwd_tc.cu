@@ -266,7 +266,8 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
         auto mma_round = [&]() {  // every compute thread: wait for the MMAs committed to B1_MMA
             const bool w = wait_bar(&bars[B1_MMA], mph, abort_flag);
             mph ^= 1u;
-            ok = bar_and(kBarP1, kP1Compute, w);
+            const bool r = bar_and(kBarP1, kP1Compute, w);
+            ok = ok && r;
             tc_fence_after();
         };
         auto sync_after_tmem_st = [&]() {
@@ -275,38 +276,47 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             named_bar(kBarP1, kP1Compute);
             tc_fence_after();
         };
-#pragma unroll 1
-        for (int idx = 0; idx < nch && ok; ++idx) {
+        // the gates of chunk number idx (counted from the last) into the gate buffers, its stage
+        // landed, its Q rows scaled by gamma_t in place (16-byte unit u: box u >> 9, row (u >> 3) & 63);
+        // returns gamma_C
+        auto prepare = [&](int idx) -> float {
             const int c = nch - 1 - idx, s = idx & 1;
             const int t0 = c * kC;
             const int n = (T - t0 < kC) ? (int)(T - t0) : kC;
-            const int64_t item = bh * nch + c;
-            uint8_t *st = sm + s * S1_BYTES;
-            const uint32_t sta = sbase + s * S1_BYTES;
-            // ---- gates of the chunk ----
             chunk_gates(p.log_alpha, p.beta, (int64_t)b * T * H + h, H, t0, n, tid, g, bet, scratch, kBarP1,
                         kP1Compute);
             if (tid < 64) {
                 gam[tid] = expf(g[tid]);
                 dl[tid] = expf(g[63] - g[tid]);
             }
-            const float gC = expf(g[63]);
-            {
-                const bool w = wait_bar(&bars[B1_FULL0 + s], (idx >> 1) & 1, abort_flag);
-                if (!(ok = bar_and(kBarP1, kP1Compute, w))) break;  // also publishes gam, dl
-            }
-            // ---- Q rows scaled by gamma_t in place (16-byte unit u: box u >> 9, row (u >> 3) & 63) ----
+            const float gc = expf(g[63]);
+            const bool w = wait_bar(&bars[B1_FULL0 + s], (idx >> 1) & 1, abort_flag);
+            const bool r = bar_and(kBarP1, kP1Compute, w);  // also publishes gam, dl
+            ok = ok && r;
+            if (r) {
+                uint8_t *st = sm + s * S1_BYTES;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int u = tid + 256 * i;
-                uint4 *ptr = reinterpret_cast<uint4 *>(st + S1_Q) + u;
-                float f[8];
-                unpack8(*ptr, f);
-                const float x = gam[(u >> 3) & 63];
-                *ptr = make_uint4(pack_bf16x2(f[0] * x, f[1] * x), pack_bf16x2(f[2] * x, f[3] * x),
-                                  pack_bf16x2(f[4] * x, f[5] * x), pack_bf16x2(f[6] * x, f[7] * x));
+                for (int i = 0; i < 4; ++i) {
+                    const int u = tid + 256 * i;
+                    uint4 *ptr = reinterpret_cast<uint4 *>(st + S1_Q) + u;
+                    float f[8];
+                    unpack8(*ptr, f);
+                    const float x = gam[(u >> 3) & 63];
+                    *ptr = make_uint4(pack_bf16x2(f[0] * x, f[1] * x), pack_bf16x2(f[2] * x, f[3] * x),
+                                      pack_bf16x2(f[4] * x, f[5] * x), pack_bf16x2(f[6] * x, f[7] * x));
+                }
+                fence_proxy_async_smem();
             }
-            fence_proxy_async_smem();
+            return gc;
+        };
+        float gC = (nch > 0) ? prepare(0) : 0.f;
+#pragma unroll 1
+        for (int idx = 0; idx < nch && ok; ++idx) {
+            const int c = nch - 1 - idx, s = idx & 1;
+            const int t0 = c * kC;
+            const int n = (T - t0 < kC) ? (int)(T - t0) : kC;
+            const int64_t item = bh * nch + c;
+            const uint32_t sta = sbase + s * S1_BYTES;
             // ---- dS (the adjoint of the state leaving chunk c): bf16 copy into TMEM and to the
             //      workspace, then dS <- gamma_C dS ----
             {
@@ -414,6 +424,9 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
                 mma_commit(&bars[B1_EMPTY0 + s]);
                 mma_commit(&bars[B1_MMA]);
             }
+            // the next chunk's gates and Q while the state update runs (this chunk's epilogues are
+            // done with the gate buffers, and its Q is in the other stage)
+            if (idx + 1 < nch) gC = prepare(idx + 1);
             mma_round();
         }
         // dS0: the adjoint of the state entering chunk 0
