@@ -804,6 +804,8 @@ def run_grouped(args, world, rank):
     dev = torch.device("cuda", torch.cuda.current_device())
     stream = torch.cuda.current_stream(dev)
     w = WORKLOADS[args.workload]
+    if args.tokens:
+        w = dataclasses.replace(w, T=args.tokens, name="%s_first%d" % (w.name, args.tokens))
     Hq, Hkv = 8, 2
     a = forward_inputs(w.B, w.T, Hq, w.dk, w.dv, w.dtype, seed=w.seed + 1000 * rank, alpha_mu=w.alpha_mu)
     b = forward_inputs(w.B, w.T, Hkv, w.dk, w.dv, w.dtype, seed=w.seed + 1000 * rank + 1, s0_std=w.s0_std,
