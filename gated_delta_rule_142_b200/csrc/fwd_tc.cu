@@ -825,11 +825,12 @@ fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ 
 // in order.  A (b, h)'s transfers and entry states sit in consecutive slots;
 // with a table (packed sequences, whose segment counts differ), CTA row x
 // takes S0 [tab[x].x], slots tab[x].y .. tab[x].y + tab[x].z - 1; without
-// one, (b, h) = x takes S0 [x] and slots x (nseg - 1) onwards.  The next needed M is bulk-copied into the second of two shared
-// buffers while a step computes, and B_{p+1} is prefetched into registers.
-// Where Mflag marks a transfer matrix as negligible (its bound is at most
-// e^-40, see kNegligibleTransfer) the step is S_{p+1} = B_p and M_p is neither
-// read nor multiplied.
+// one, (b, h) = x takes S0 [x] and slots x (nseg - 1) onwards.  The next
+// needed M is bulk-copied into the second of two shared buffers while a step
+// computes.  Where Mflag marks a transfer matrix as negligible (its bound is at
+// most e^-40, see kNegligibleTransfer) the step is S_{p+1} = B_p: M_p is
+// neither read nor multiplied, and all such steps are copied at once before
+// the others run in order.
 constexpr int kPrefixRows = 16;
 constexpr int kPrefixThreads = 256;
 constexpr int kPrefixLd = kD + 4;
@@ -881,7 +882,8 @@ seg_prefix_kernel(const float *__restrict__ S0, const float *__restrict__ Bw, co
     }
     __syncthreads();
     int loaded = 0;  // matrices consumed so far
-    int pending = next_needed(0);  // the step whose M is in flight (steps: none)
+    // blocks with blockIdx.z > 0 only copy their share of the negligible steps (pass 1 below)
+    int pending = blockIdx.z == 0 ? next_needed(0) : steps;  // the step whose M is in flight (steps: none)
     if (tid == 0 && pending < steps) load_m(pending, 0);
     for (int i = tid; i < kPrefixRows * (kD / 4); i += kPrefixThreads) {
         const int rr = i / (kD / 4), cc = (i % (kD / 4)) * 4;
@@ -890,47 +892,73 @@ seg_prefix_kernel(const float *__restrict__ S0, const float *__restrict__ Bw, co
         *reinterpret_cast<float4 *>(Sr + rr * kPrefixLd + cc) = v;
     }
     auto b_rows = [&](int q) { return Bw + ((base + q) * kD + r0 + r) * (int64_t)kD; };
-    float4 b0 = make_float4(0.f, 0.f, 0.f, 0.f), b1 = b0;
-    if (steps > 0) {
-        b0 = *reinterpret_cast<const float4 *>(b_rows(0) + ca);
-        b1 = *reinterpret_cast<const float4 *>(b_rows(0) + cb);
-    }
-    for (int q = 0; q < steps; ++q) {
-        float acc[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-        if (q == pending) {
-            // the next needed M goes into the other buffer, free since the step that read it ended
-            const int nxt = next_needed(q + 1);
-            if (tid == 0 && nxt < steps) load_m(nxt, loaded + 1);
-            // bounded wait; a timeout leaves the entry states unwritten rather than hanging
-            const bool landed = mbar_wait(&full[loaded & 1], (loaded >> 1) & 1);
-            if (!__syncthreads_and(landed)) break;  // also publishes the previous step's rows of S
-            if (q + 1 < steps) {
-                b0 = *reinterpret_cast<const float4 *>(b_rows(q + 1) + ca);
-                b1 = *reinterpret_cast<const float4 *>(b_rows(q + 1) + cb);
+    // pass 1: a step whose transfer matrix is negligible needs no state, S_{q+1} = B_q: all such
+    // steps at once, spread over the gridDim.z blocks of these rows (steps z, z + gridDim.z, ...),
+    // eight 16-byte loads in flight per thread
+    if (Mflag) {
+        constexpr int kUnits = kPrefixRows * (kD / 4);  // 16-byte units of this CTA's rows, per step
+        const int zs = (int)gridDim.z, mine = (steps - (int)blockIdx.z + zs - 1) / zs;  // this block's steps
+        const int total = mine * kUnits;
+        for (int i0 = tid; i0 < total; i0 += 8 * kPrefixThreads) {
+            float4 v[8];
+            int64_t off[8];
+            bool copy[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int i = i0 + u * kPrefixThreads;
+                const int q = (int)blockIdx.z + (i / kUnits) * zs, rr = (i % kUnits) / (kD / 4),
+                          cc = (i % (kD / 4)) * 4;
+                copy[u] = i < total && !needs_m(q);
+                off[u] = ((base + q) * kD + r0 + rr) * (int64_t)kD + cc;
+                if (copy[u]) v[u] = *reinterpret_cast<const float4 *>(Bw + off[u]);
             }
-            const float *M = Ms + (loaded & 1) * kD * kD;
-#pragma unroll 4
-            for (int k = 0; k < kD; ++k) {
-                const float a = Sr[r * kPrefixLd + k];
-                const float4 m0 = *reinterpret_cast<const float4 *>(M + k * kD + ca);
-                const float4 m1 = *reinterpret_cast<const float4 *>(M + k * kD + cb);
-                acc[0] = fmaf(a, m0.x, acc[0]); acc[1] = fmaf(a, m0.y, acc[1]);
-                acc[2] = fmaf(a, m0.z, acc[2]); acc[3] = fmaf(a, m0.w, acc[3]);
-                acc[4] = fmaf(a, m1.x, acc[4]); acc[5] = fmaf(a, m1.y, acc[5]);
-                acc[6] = fmaf(a, m1.z, acc[6]); acc[7] = fmaf(a, m1.w, acc[7]);
-            }
-            ++loaded;
-            pending = nxt;
-        } else if (q + 1 < steps) {
-            b0 = *reinterpret_cast<const float4 *>(b_rows(q + 1) + ca);
-            b1 = *reinterpret_cast<const float4 *>(b_rows(q + 1) + cb);
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (copy[u]) *reinterpret_cast<float4 *>(S_entry + off[u]) = v[u];
         }
+    }
+    // pass 2: the steps that need their M, in order.  The state entering step q is S0 (q = 0), the
+    // previous step's result still in Sr, or B_{q-1} when step q - 1 was negligible.
+    int prev = -1;  // the step whose result Sr holds (-1: S0)
+    while (pending < steps) {
+        const int q = pending;
+        // the next needed M goes into the other buffer, free since the step that read it ended
+        const int nxt = next_needed(q + 1);
+        if (tid == 0 && nxt < steps) load_m(nxt, loaded + 1);
+        if (q > 0 && prev != q - 1) {
+            __syncthreads();  // every thread is done with Sr
+            for (int i = tid; i < kPrefixRows * (kD / 4); i += kPrefixThreads) {
+                const int rr = i / (kD / 4), cc = (i % (kD / 4)) * 4;
+                *reinterpret_cast<float4 *>(Sr + rr * kPrefixLd + cc) =
+                    *reinterpret_cast<const float4 *>(Bw + ((base + q - 1) * kD + r0 + rr) * (int64_t)kD + cc);
+            }
+        }
+        const float4 b0 = *reinterpret_cast<const float4 *>(b_rows(q) + ca);
+        const float4 b1 = *reinterpret_cast<const float4 *>(b_rows(q) + cb);
+        float acc[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        // bounded wait; a timeout leaves the entry states unwritten rather than hanging
+        const bool landed = mbar_wait(&full[loaded & 1], (loaded >> 1) & 1);
+        if (!__syncthreads_and(landed)) break;  // also publishes the rows of Sr
+        const float *M = Ms + (loaded & 1) * kD * kD;
+#pragma unroll 4
+        for (int k = 0; k < kD; ++k) {
+            const float a = Sr[r * kPrefixLd + k];
+            const float4 m0 = *reinterpret_cast<const float4 *>(M + k * kD + ca);
+            const float4 m1 = *reinterpret_cast<const float4 *>(M + k * kD + cb);
+            acc[0] = fmaf(a, m0.x, acc[0]); acc[1] = fmaf(a, m0.y, acc[1]);
+            acc[2] = fmaf(a, m0.z, acc[2]); acc[3] = fmaf(a, m0.w, acc[3]);
+            acc[4] = fmaf(a, m1.x, acc[4]); acc[5] = fmaf(a, m1.y, acc[5]);
+            acc[6] = fmaf(a, m1.z, acc[6]); acc[7] = fmaf(a, m1.w, acc[7]);
+        }
+        ++loaded;
         __syncthreads();  // every thread is done reading this step's rows and M
         *reinterpret_cast<float4 *>(Sr + r * kPrefixLd + ca) = make_float4(acc[0], acc[1], acc[2], acc[3]);
         *reinterpret_cast<float4 *>(Sr + r * kPrefixLd + cb) = make_float4(acc[4], acc[5], acc[6], acc[7]);
         float *dst = S_entry + ((base + q) * kD + r0 + r) * (int64_t)kD;
         *reinterpret_cast<float4 *>(dst + ca) = make_float4(acc[0], acc[1], acc[2], acc[3]);
         *reinterpret_cast<float4 *>(dst + cb) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+        prev = q;
+        pending = nxt;
     }
 }
 
@@ -1015,7 +1043,11 @@ cudaError_t launch_seg_prefix(const float *S0, const float *Bw, const float *Mw,
     }
     {
         TimedLaunch tl_(GDN_KERNEL_PREFIX, stream);
-        seg_prefix_kernel<<<dim3((unsigned)heads, kD / kPrefixRows), kPrefixThreads, kPrefixSmem, stream>>>(
+        // with flags and many steps, up to three more blocks per row block share the copies of the
+        // negligible steps
+        const int zsi = Mflag ? (nseg - 1) / 8 : 1;
+        const unsigned zs = zsi < 1 ? 1u : (zsi > 4 ? 4u : (unsigned)zsi);
+        seg_prefix_kernel<<<dim3((unsigned)heads, kD / kPrefixRows, zs), kPrefixThreads, kPrefixSmem, stream>>>(
             S0, Bw, Mw, Mflag, S_entry, nseg, tab);
     }
     return cudaGetLastError();

@@ -147,8 +147,11 @@ int gdn_forward(const void *q, const void *k, const void *v, const float *log_al
  * cu_seqlens is not a valid offset array (NULL with N > 0, cu_seqlens[0] !=
  * 0, decreasing, or cu_seqlens[N] != T_total); the rest as for gdn_forward.
  * bf16 with dk = dv = 128 and chunk = 64 runs the two-kernel tensor-core
- * forward over all sequences at once (one chain per sequence and head, no
- * segments); other shapes run the CUDA-core forward once per sequence.
+ * forward over all sequences at once: one chain per sequence and head, except
+ * that a sequence long enough to outlast the others is cut into segments
+ * (transfers, a prefix from its S0, and one chain per segment), as a long
+ * gdn_forward is; GDN_SEGMENTS=k cuts the longest sequence into k segments.
+ * Other shapes run the CUDA-core forward once per sequence.
  */
 int gdn_forward_varlen(const void *q, const void *k, const void *v, const float *log_alpha,
                        const float *beta, const int64_t *cu_seqlens, int64_t N, const float *S0,
@@ -236,10 +239,16 @@ int gdn_decode_step_raw(const void *q, const void *k, const void *v, const float
  * the one of gdn_forward (source: the Sec. 3.3 gated-delta memory equation);
  * the gradient of log_alpha below the forward's floor of -40 is zero.
  *
- * The forward is recomputed (the state entering every chunk is kept in
- * scratch, dv * dk * 4 bytes per chunk and head), then the chunks are walked
- * backwards with the chunkwise adjoint, in float32 on the CUDA cores.
- * Scratch also holds float32 accumulators of dq and dk for bf16.
+ * The forward is recomputed, keeping the state entering every chunk in
+ * scratch.  For bf16 with dk = dv = 128 and chunk = 64 the reverse mode then
+ * runs on the tensor cores: a reverse chain over each (b, h)'s chunks (the
+ * adjoint of the state in tensor memory) and a chunk-parallel pass forming
+ * every chunk's gradients (scratch about 136 KB per chunk and head: the
+ * recompute's workspace, bf16 checkpoints, T of every chunk, and the
+ * adjoints passed between the two).  Every other shape, or
+ * GDN_BWD_PATH=simt, walks the chunks backwards with the chunkwise adjoint in
+ * float32 on the CUDA cores (checkpoints of dv * dk * 4 bytes per chunk and
+ * head, and float32 accumulators of dq and dk for bf16).
  * Alignment and staging as for gdn_forward; no output may overlap an input
  * or another output (GDN_ERR_ALIAS).
  */
@@ -268,10 +277,13 @@ int gdn_backward(const void *q, const void *k, const void *v, const float *log_a
  * aliasing and staging are otherwise those of the ungrouped calls.
  *
  * The decode kernel updates each memory once and forms the G outputs from
- * the updated rows.  The forward runs the two-kernel tensor-core forward
- * (bf16, dk = dv = 128, chunk = 64) or the CUDA-core forward with per-query-
- * head work items: each query head of a group recomputes its memory.  This
- * costs G times the memory's work, but no kernel reads another's state.
+ * the updated rows.  The forward, for bf16 with dk = dv = 128 and chunk = 64,
+ * runs each memory once as well: the two-kernel tensor-core forward runs the
+ * memory of key-value head hk on query head hk * G's chunk items (writing
+ * that head's outputs, and per chunk the bf16 state entering it and U^T, in
+ * scratch), then one chunk-parallel kernel forms the other query heads'
+ * outputs from them.  Other shapes run the CUDA-core forward with
+ * per-query-head work items, where each query head recomputes its memory.
  */
 int gdn_forward_grouped(const void *q, const void *k, const void *v, const float *log_alpha,
                         const float *beta, const float *S0, void *out, float *S_final, int64_t B,
