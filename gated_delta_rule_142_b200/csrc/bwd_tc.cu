@@ -53,6 +53,7 @@ using namespace tcu;
 
 constexpr int kC = 64;
 constexpr int kD = 128;
+constexpr int kRecFloats = 132;  // the forward prep kernel's gate record per chunk; [129] is rho_C
 
 __device__ int g_bwd_timeout;  // set when a bounded mbarrier wait gives up
 
@@ -183,6 +184,19 @@ struct BwdArgs {
     __nv_bfloat16 *dr_ws;    // [items][64][128]:  dR of every chunk
     int64_t T, H, items;
     int chunks;
+    // Segments: chunks [p seg_len, (p + 1) seg_len) of each (b, h) form segment p (nseg = 1: one
+    // segment).  The adjoint leaving a segment maps to the one entering it by dS -> dS X_p + B'_p,
+    // X_p = M_p^T the transpose of the segment's forward transfer (S -> S M_p + B_p).
+    int nseg, seg_len;
+    // 0: one CTA per (b, h) and segment walks its chunks backwards from the adjoint leaving the segment
+    //    (dS_final for the last one, else `entry`) and writes every output (dS0 for segment 0);
+    // 1: transfers, a CTA pair per (b, h) and segment p >= 1 writing only the adjoint it reaches at the
+    //    segment's start: run 0 from zero with dO (B'_p), run 1 from the identity without dO (X_p).
+    int mode;
+    const float *gate_rec;  // the forward's gate records: rho_C at [129] bounds the chunks' transfers
+    const float *entry;     // [B*H][nseg - 1][128][128]: the prefix's result, slot q for segment nseg - 2 - q
+    float *xb, *xm;         // [B*H][nseg - 1][128][128]: B'_p and X_p in slot q = nseg - 1 - p
+    int *xflag;             // [B*H][nseg - 1]: X_p negligible (slot q)
 };
 
 __global__ void __launch_bounds__(kP1Threads, 1)
@@ -199,11 +213,56 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t H = p.H, T = p.T;
-    const int64_t bh = blockIdx.x;
+    int64_t bh;
+    int seg, run = 0;
+    if (p.mode == 0) {
+        bh = blockIdx.x / p.nseg;
+        seg = (int)(blockIdx.x % p.nseg);
+    } else {
+        bh = (blockIdx.x >> 1) / (p.nseg - 1);
+        seg = 1 + (int)((blockIdx.x >> 1) % (p.nseg - 1));
+        run = (int)(blockIdx.x & 1);
+    }
     const int b = (int)(bh / H), h = (int)(bh % H);
     const int nch = p.chunks;
+    const int c_lo = seg * p.seg_len, c_hi = (c_lo + p.seg_len < nch) ? c_lo + p.seg_len : nch;
+    const bool idrun = p.mode == 1 && run == 1;  // the identity run: no dO
+    const int64_t slot = bh * (p.nseg - 1) + (p.nseg - 1 - seg);
+    volatile int *span = reinterpret_cast<volatile int *>(sm + O1_MISC + 8);  // chunks walked
     const uint32_t sbase = smem_u32(sm);
 
+    if (warp == 0) {
+        int nrun = c_hi - c_lo;
+        if (p.mode == 1) {
+            // the shortest head of the segment whose transfer bounds multiply to at most e^-40: the
+            // chunks after it reach the segment's start scaled by at most that, so the zero run walks
+            // the head alone and X_p is negligible (warp-wide prefix products over blocks of 32 records)
+            const int len = c_hi - c_lo;
+            int m = len, negl = 0;
+            float acc = 1.f;
+            for (int base = 0; base < len; base += 32) {
+                const int i = base + lane;
+                float x = (i < len) ? p.gate_rec[(bh * nch + c_lo + i) * kRecFloats + 129] : 1.f;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float y = __shfl_up_sync(0xffffffffu, x, o);
+                    if (lane >= o) x *= y;
+                }
+                x *= acc;
+                const uint32_t hit = __ballot_sync(0xffffffffu, i < len && x <= kNegligibleTransfer);
+                if (hit) {
+                    m = base + __ffs(hit);
+                    negl = 1;
+                    break;
+                }
+                acc = __shfl_sync(0xffffffffu, x, 31);
+            }
+            nrun = idrun ? (negl ? 0 : len) : m;
+            if (idrun && lane == 0) p.xflag[slot] = negl;
+        }
+        if (lane == 0) span[0] = nrun;
+        __syncwarp();
+    }
     if (tid == 0) {
         for (int i = 0; i < B1_COUNT; ++i) mbar_init(&bars[i], 1);
         *abort_flag = 0;
@@ -217,25 +276,30 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = *tmem_slot;
+    const int nrun = span[0];
+    const int c_top = c_lo + nrun - 1;  // the walk's first chunk
 
     if (warp == 8) {
         // ============================ producer ============================
         if (lane == 0) {
             bool ok = true;
-            for (int idx = 0; idx < nch && ok; ++idx) {
-                const int c = nch - 1 - idx, s = idx & 1;
+            for (int idx = 0; idx < nrun && ok; ++idx) {
+                const int c = c_top - idx, s = idx & 1;
                 if (idx >= 2 && !(ok = wait_bar(&bars[B1_EMPTY0 + s], ((idx - 2) >> 1) & 1, abort_flag))) break;
                 uint8_t *st = sm + s * S1_BYTES;
                 uint64_t *full = &bars[B1_FULL0 + s];
                 const int t0 = c * kC;
                 const int row = (int)(bh * nch + c) * 64;
-                mbar_arrive_expect_tx(full, 3 * 16384 + 2 * 8192);
+                // the identity run needs neither dO nor the products that carry it (Q, P)
+                mbar_arrive_expect_tx(full, idrun ? 16384 + 8192 : 3 * 16384 + 2 * 8192);
                 for (int blk = 0; blk < 2; ++blk) {
-                    tma_load_4d(st + S1_DO + blk * 8192, &tm_do, full, blk * 64, h, t0, b);
-                    tma_load_4d(st + S1_Q + blk * 8192, &tm_q, full, blk * 64, h, t0, b);
+                    if (!idrun) {
+                        tma_load_4d(st + S1_DO + blk * 8192, &tm_do, full, blk * 64, h, t0, b);
+                        tma_load_4d(st + S1_Q + blk * 8192, &tm_q, full, blk * 64, h, t0, b);
+                    }
                     tma_load_4d(st + S1_K + blk * 8192, &tm_k, full, blk * 64, h, t0, b);
                 }
-                tma_load_2d(st + S1_P, &tm_p, full, 0, row);
+                if (!idrun) tma_load_2d(st + S1_P, &tm_p, full, 0, row);
                 tma_load_2d(st + S1_T, &tm_t, full, 0, row);
             }
         }
@@ -247,18 +311,30 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
         const uint32_t lb = (uint32_t)((warp & 3) * 32) << 16;
         bool ok = true;
         uint32_t mph = 0;  // phase of the next wait on B1_MMA
-        // dS <- dS_final (or zero)
+        // dS <- the adjoint leaving the walk: dS_final (or zero) for the last segment, the prefix's
+        // entry for the others; zero for the transfer's zero run, the identity for its identity run
+        const float *ent = nullptr;
+        if (p.mode == 0) {
+            if (seg == p.nseg - 1)
+                ent = p.dS_final ? p.dS_final + bh * kD * kD : nullptr;
+            else
+                ent = p.entry + (bh * (p.nseg - 1) + (p.nseg - 2 - seg)) * kD * kD;
+        }
 #pragma unroll 1
         for (int pc = 2 * ch; pc < 2 * ch + 2; ++pc) {
             uint32_t r[32];
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
                 float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (p.dS_final) x = *reinterpret_cast<const float4 *>(p.dS_final + (bh * kD + j) * kD + 32 * pc + i);
+                if (ent) x = *reinterpret_cast<const float4 *>(ent + (int64_t)j * kD + 32 * pc + i);
                 r[i] = __float_as_uint(x.x);
                 r[i + 1] = __float_as_uint(x.y);
                 r[i + 2] = __float_as_uint(x.z);
                 r[i + 3] = __float_as_uint(x.w);
+            }
+            if (idrun) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) r[i] = __float_as_uint((32 * pc + i == j) ? 1.f : 0.f);
             }
             tmem_st32(tm + lb + T1_DS + 32 * pc, r);
         }
@@ -280,7 +356,7 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
         // landed, its Q rows scaled by gamma_t in place (16-byte unit u: box u >> 9, row (u >> 3) & 63);
         // returns gamma_C
         auto prepare = [&](int idx) -> float {
-            const int c = nch - 1 - idx, s = idx & 1;
+            const int c = c_top - idx, s = idx & 1;
             const int t0 = c * kC;
             const int n = (T - t0 < kC) ? (int)(T - t0) : kC;
             chunk_gates(p.log_alpha, p.beta, (int64_t)b * T * H + h, H, t0, n, tid, g, bet, scratch, kBarP1,
@@ -293,7 +369,7 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             const bool w = wait_bar(&bars[B1_FULL0 + s], (idx >> 1) & 1, abort_flag);
             const bool r = bar_and(kBarP1, kP1Compute, w);  // also publishes gam, dl
             ok = ok && r;
-            if (r) {
+            if (r && !idrun) {
                 uint8_t *st = sm + s * S1_BYTES;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
@@ -309,10 +385,10 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             }
             return gc;
         };
-        float gC = (nch > 0) ? prepare(0) : 0.f;
+        float gC = (nrun > 0) ? prepare(0) : 0.f;
 #pragma unroll 1
-        for (int idx = 0; idx < nch && ok; ++idx) {
-            const int c = nch - 1 - idx, s = idx & 1;
+        for (int idx = 0; idx < nrun && ok; ++idx) {
+            const int c = c_top - idx, s = idx & 1;
             const int t0 = c * kC;
             const int n = (T - t0 < kC) ? (int)(T - t0) : kC;
             const int64_t item = bh * nch + c;
@@ -331,10 +407,12 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
                     for (int i = 0; i < 32; i += 2)
                         pk[i >> 1] = pack_bf16x2(__uint_as_float(r[i]), __uint_as_float(r[i + 1]));
                     tmem_st16(tm + lb + T1_DSB + 16 * pc, pk);
+                    if (p.mode == 0) {
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        reinterpret_cast<uint4 *>(dsg + 32 * pc)[i] =
-                            make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                        for (int i = 0; i < 4; ++i)
+                            reinterpret_cast<uint4 *>(dsg + 32 * pc)[i] =
+                                make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                    }
 #pragma unroll
                     for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(gC * __uint_as_float(r[i]));
                     tmem_st32(tm + lb + T1_DS + 32 * pc, r);
@@ -343,10 +421,12 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             sync_after_tmem_st();
             // ---- dO^T P and dS K^T ----
             if (tid == 0) {
+                if (!idrun) {
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ss(tm + T1_DU, smem_desc_sw128(sta + S1_DO + kk * 2048, 8192, 1024),
-                           smem_desc_sw128(sta + S1_P + kk * 2048, 8192, 1024), IDESC_64_MN_MN, kk > 0);
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss(tm + T1_DU, smem_desc_sw128(sta + S1_DO + kk * 2048, 8192, 1024),
+                               smem_desc_sw128(sta + S1_P + kk * 2048, 8192, 1024), IDESC_64_MN_MN, kk > 0);
+                }
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ts(tm + T1_D2, tm + T1_DSB + kk * 8,
@@ -363,6 +443,10 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
                 tmem_ld32(tm + lb + T1_DU + 32 * pc, a);
                 tmem_ld32(tm + lb + T1_D2 + 32 * pc, d2);
                 tmem_wait_ld();
+                if (idrun) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) a[i] = 0u;
+                }
                 uint32_t pk[16];
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
@@ -399,12 +483,14 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
                     for (int i = 0; i < 32; i += 2) {
                         const int t = 32 * pc + i;
                         const float x0 = __uint_as_float(r[i]), x1 = __uint_as_float(r[i + 1]);
-                        dr_row[i * kD] = __float2bfloat16_rn(x0);
-                        dr_row[(i + 1) * kD] = __float2bfloat16_rn(x1);
-                        if (t < n) *dv_row = __float2bfloat16_rn(bet[t] * x0);
-                        dv_row += vstr;
-                        if (t + 1 < n) *dv_row = __float2bfloat16_rn(bet[t + 1] * x1);
-                        dv_row += vstr;
+                        if (p.mode == 0) {
+                            dr_row[i * kD] = __float2bfloat16_rn(x0);
+                            dr_row[(i + 1) * kD] = __float2bfloat16_rn(x1);
+                            if (t < n) *dv_row = __float2bfloat16_rn(bet[t] * x0);
+                            dv_row += vstr;
+                            if (t + 1 < n) *dv_row = __float2bfloat16_rn(bet[t + 1] * x1);
+                            dv_row += vstr;
+                        }
                         pk[i >> 1] = pack_bf16x2(-bet[t] * gam[t] * x0, -bet[t + 1] * gam[t + 1] * x1);
                     }
                     tmem_st16(tm + lb + T1_DRB + 16 * pc, pk);
@@ -413,10 +499,12 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             sync_after_tmem_st();
             // ---- dS += dO^T (diag(gamma) Q) - dR^T diag(beta gamma) K ----
             if (tid == 0) {
+                if (!idrun) {
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk)
-                    mma_ss(tm + T1_DS, smem_desc_sw128(sta + S1_DO + kk * 2048, 8192, 1024),
-                           smem_desc_sw128(sta + S1_Q + kk * 2048, 8192, 1024), IDESC_128_MN_MN, 1u);
+                    for (int kk = 0; kk < 4; ++kk)
+                        mma_ss(tm + T1_DS, smem_desc_sw128(sta + S1_DO + kk * 2048, 8192, 1024),
+                               smem_desc_sw128(sta + S1_Q + kk * 2048, 8192, 1024), IDESC_128_MN_MN, 1u);
+                }
 #pragma unroll
                 for (int kk = 0; kk < 4; ++kk)
                     mma_ts(tm + T1_DS, tm + T1_DRB + kk * 8, smem_desc_sw128(sta + S1_K + kk * 2048, 8192, 1024),
@@ -426,17 +514,23 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             }
             // the next chunk's gates and Q while the state update runs (this chunk's epilogues are
             // done with the gate buffers, and its Q is in the other stage)
-            if (idx + 1 < nch) gC = prepare(idx + 1);
+            if (idx + 1 < nrun) gC = prepare(idx + 1);
             mma_round();
         }
-        // dS0: the adjoint of the state entering chunk 0
-        if (ok && p.dS0) {
+        // the adjoint reached at the walk's start: dS0 (the state entering chunk 0) for segment 0, B'_p or
+        // X_p for a transfer run
+        float *exitp = nullptr;
+        if (p.mode == 0)
+            exitp = (seg == 0 && p.dS0) ? p.dS0 + bh * kD * kD : nullptr;
+        else if (nrun > 0)
+            exitp = (idrun ? p.xm : p.xb) + slot * kD * kD;
+        if (ok && exitp) {
 #pragma unroll 1
             for (int pc = 2 * ch; pc < 2 * ch + 2; ++pc) {
                 uint32_t r[32];
                 tmem_ld32(tm + lb + T1_DS + 32 * pc, r);
                 tmem_wait_ld();
-                float4 *dst = reinterpret_cast<float4 *>(p.dS0 + (bh * kD + j) * kD + 32 * pc);
+                float4 *dst = reinterpret_cast<float4 *>(exitp + (int64_t)j * kD + 32 * pc);
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
                     dst[i] = make_float4(__uint_as_float(r[4 * i]), __uint_as_float(r[4 * i + 1]),
@@ -877,8 +971,9 @@ bool configure(const void *fn, uint32_t smem, std::atomic<uint64_t> &done) {
 }
 
 struct TcLayout {
-    size_t fwd_ws, fwd_out, ckpt, tt, ds, dr, total;
-    int nseg;
+    size_t fwd_ws, fwd_out, ckpt, tt, ds, dr, seg, total;
+    int nseg;               // segments asked of the forward recompute
+    int seg_len, nseg_run;  // chunks per segment and the segments they make (the forward's own rounding)
 };
 
 size_t round256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -894,7 +989,12 @@ TcLayout tc_layout(const BwdProblem &p, int sm_count) {
     l.tt = round256((size_t)items * kC * kC * 2);
     l.ds = round256((size_t)items * kD * kD * 2);
     l.dr = round256((size_t)items * kC * kD * 2);
-    l.total = l.fwd_ws + l.fwd_out + l.ckpt + l.tt + l.ds + l.dr;
+    l.seg_len = (int)((nch + l.nseg - 1) / l.nseg);
+    l.nseg_run = (int)((nch + l.seg_len - 1) / l.seg_len);
+    // reverse segments: B', X and the entry adjoints of every transfer slot, and their flags
+    const size_t slots = (size_t)(f.B * f.H) * (size_t)(l.nseg_run - 1);
+    l.seg = l.nseg_run > 1 ? round256(3 * slots * kD * kD * sizeof(float)) + round256(slots * sizeof(int)) : 0;
+    l.total = l.fwd_ws + l.fwd_out + l.ckpt + l.tt + l.ds + l.dr + l.seg;
     return l;
 }
 
@@ -934,7 +1034,7 @@ cudaError_t launch_bwd_tc(const BwdProblem &p, int sm_count, void *workspace, cu
     const int64_t nch = (f.T + kC - 1) / kC, items = f.B * f.H * nch;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     uint8_t *fwd_ws = ws, *fwd_out = ws + l.fwd_ws, *ckpt = fwd_out + l.fwd_out, *tt = ckpt + l.ckpt,
-            *dsw = tt + l.tt, *drw = dsw + l.ds;
+            *dsw = tt + l.tt, *drw = dsw + l.ds, *segw = drw + l.dr;
     cudaError_t e;
     // forward recompute: bf16 checkpoints, T of every chunk, P and T diag(beta) in the workspace
     if ((e = cudaMemsetAsync(tt, 0, (size_t)items * kC * kC * 2, stream)) != cudaSuccess) return e;
@@ -976,9 +1076,37 @@ cudaError_t launch_bwd_tc(const BwdProblem &p, int sm_count, void *workspace, cu
     a.H = f.H;
     a.items = items;
     a.chunks = (int)nch;
+    a.nseg = l.nseg_run;
+    a.seg_len = l.seg_len;
+    a.gate_rec = fwd_split_ws_gates(fwd_ws, items);
+    a.entry = nullptr;
+    a.xb = a.xm = nullptr;
+    a.xflag = nullptr;
+    const int64_t heads = f.B * f.H;
+    if (l.nseg_run > 1) {
+        // long sequences with few heads: the segments' reverse transfers, their prefix from dS_final
+        // (the adjoint leaving every segment), then every segment's walk at once
+        const size_t per = (size_t)heads * (size_t)(l.nseg_run - 1) * kD * kD;
+        a.xb = reinterpret_cast<float *>(segw);
+        a.xm = a.xb + per;
+        float *entry = a.xm + per;
+        a.xflag = reinterpret_cast<int *>(segw + round256(3 * per * sizeof(float)));
+        a.mode = 1;
+        {
+            TimedLaunch tl_(GDN_KERNEL_TRANSFER, stream);
+            bwd_chain_kernel<<<(unsigned)(heads * (l.nseg_run - 1) * 2), kP1Threads, SMEM_P1, stream>>>(
+                mdo, mq, mk, mp, mt, a);
+        }
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = launch_seg_prefix(p.dS_final, a.xb, a.xm, a.xflag, entry, heads, l.nseg_run, stream, nullptr)) !=
+            cudaSuccess)
+            return e;
+        a.entry = entry;
+    }
+    a.mode = 0;
     {
         TimedLaunch tl_(GDN_KERNEL_BACKWARD, stream);
-        bwd_chain_kernel<<<(unsigned)(f.B * f.H), kP1Threads, SMEM_P1, stream>>>(mdo, mq, mk, mp, mt, a);
+        bwd_chain_kernel<<<(unsigned)(heads * l.nseg_run), kP1Threads, SMEM_P1, stream>>>(mdo, mq, mk, mp, mt, a);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     {

@@ -135,6 +135,9 @@ struct PrepArgs {
     const int2 *ctab;  // packed chunk table, or nullptr for fixed-length problems
     int raw_inputs;    // q, k not yet L2-normalised; log_alpha, beta hold the gate logits
     int group;         // grouped heads: k and the gates have H / group heads (head h / group)
+    // one memory per key-value head (lead = group): only the items of query heads h % lead == 0 feed
+    // the chain, so the others form P and their gate record alone (no inverse, TB or W^T)
+    int lead;
     // or nullptr: T = (I + A)^{-1} of every item, bf16 [items][64][64] row-major (the backward's
     // recompute); only the lower triangle is written, the caller zeroes the rest
     __nv_bfloat16 *t_out;
@@ -150,6 +153,9 @@ __device__ __forceinline__ void store_tb_tbg(uint8_t *tb, uint8_t *tbg, int row,
     if (tout) *reinterpret_cast<uint32_t *>(tout + row * 64 + col) = pack_bf16x2(v0, v1);
 }
 
+// kLead: one memory per key-value head (PrepArgs::lead > 1), with P-only items; a separate
+// instantiation, so that the plain forward's kernel carries none of its branches.
+template <bool kLead>
 __global__ void __launch_bounds__(kPrepThreads, kPrepCtasPerSm)
 fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_p, const __grid_constant__ CUtensorMap tm_tb,
@@ -189,6 +195,13 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             t0 = (int)(gi - bh * (uint32_t)p.chunks) * kC;
             nt = (T - t0 < kC) ? (int)(T - t0) : kC;
         }
+    };
+    // items that form P and the gate record alone
+    auto p_only = [&](int it) -> bool {
+        if (!kLead) return false;
+        int b, h, t0, nt;
+        coords(it, b, h, t0, nt);
+        return h % p.lead != 0;
     };
     const uint32_t sbase = smem_u32(sm);
 
@@ -230,6 +243,7 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 load_q(0);
                 load_k(0);
             }
+            uint32_t nw = 0;  // items with W^T so far (the phases of TBREADY and WDONE)
             for (int it = 0; it < nit && ok; ++it) {
                 const uint32_t par = it & 1;
                 SDBG(0, 0)
@@ -246,7 +260,16 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 mma_commit(&bars[PB_GDONE]);
                 SDBG(0, 2)
-                if (!(ok = wait_bar(&bars[PB_TBREADY], par, abort_flag))) break;
+                if (p_only(it)) {
+                    // the Q block is free once the P tile staged in it has been stored, K once G is done
+                    if (!(ok = wait_bar(&bars[PB_QFREE], par, abort_flag))) break;
+                    if (it + 1 < nit) load_q(it + 1);
+                    if (!(ok = wait_bar(&bars[PB_GDONE], par, abort_flag))) break;
+                    if (it + 1 < nit) load_k(it + 1);
+                    continue;
+                }
+                const uint32_t wpar = kLead ? (nw & 1) : par;  // every item has W^T unless kLead
+                if (!(ok = wait_bar(&bars[PB_TBREADY], wpar, abort_flag))) break;
                 SDBG(0, 3)
                 tc_fence_after();
 #pragma unroll
@@ -257,8 +280,9 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 // the Q block is free once the P tile staged in it has been stored, K once W^T is done
                 if (!(ok = wait_bar(&bars[PB_QFREE], par, abort_flag))) break;
                 if (it + 1 < nit) load_q(it + 1);
-                if (!(ok = wait_bar(&bars[PB_WDONE], par, abort_flag))) break;
+                if (!(ok = wait_bar(&bars[PB_WDONE], wpar, abort_flag))) break;
                 if (it + 1 < nit) load_k(it + 1);
+                if (kLead) ++nw;
                 SDBG(0, 4)
             }
         }
@@ -343,9 +367,11 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             named_bar(kBarP, kNumPrep);
         };
         if (nit > 0) prep_gates(0);
+        uint32_t nw = 0;  // items with W^T so far (the phases of WDONE)
         for (int it = 0; it < nit && ok; ++it) {
             const uint32_t par = it & 1;
             const int gi = (int)item(it);
+            const bool ponly = p_only(it);
             __nv_bfloat16 *const tout = p.t_out ? p.t_out + (int64_t)gi * 4096 : nullptr;
             float *g = reinterpret_cast<float *>(sm + PO_PG) + par * kPG;
             // beta, gamma, e^{g - c}, e^{c - g}, beta gamma (the last two carry 1 / |k_s| once the input
@@ -412,8 +438,9 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 named_bar(kBarP, kNumPrep);
             }
-            // ---- epilogue of G: rows 0..63 -> P (bf16), rows 64..127 -> A (fp32); columns by half ----
-            {
+            // ---- epilogue of G: rows 0..63 -> P (bf16), rows 64..127 -> A (fp32; not for P-only items);
+            //      columns by half ----
+            if ((warp & 3) < 2 || !ponly) {
                 const int m = (warp & 3) * 32 + lane;  // TMEM lane = row of [Q; K]
                 const int t = m & 63;
                 // with the input stage fused, the factors 1 / |q_t| (rows of P) or 1 / |k_t| (rows of A)
@@ -477,6 +504,15 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 tma_store_2d(&tm_p, sm + PO_P, 0, (int)(gi * 64));
                 bulk_commit();
                 SDBG(1, 11)
+            }
+            if (ponly) {
+                // the Q block is free once the P store has read its staging
+                if (pt == 0) {
+                    bulk_wait_read0();
+                    arrive(&bars[PB_QFREE]);
+                }
+                if (it + 1 < nit) prep_gates(it + 1);
+                continue;
             }
             SDBG(1, 2)
             // ---- T = (I + A)^{-1} ----
@@ -605,7 +641,8 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (it + 1 < nit) prep_gates(it + 1);
             SDBG(1, 6)
             // ---- W^T (bf16, rows = key dim i, 64 tokens per row) from TMEM into the staging tile ----
-            if (!(ok = role_wait(&bars[PB_WDONE], par, abort_flag, kBarP, kNumPrep))) break;
+            if (!(ok = role_wait(&bars[PB_WDONE], kLead ? (nw & 1) : par, abort_flag, kBarP, kNumPrep))) break;
+            if (kLead) ++nw;
             tc_fence_after();
             {
                 const int i = (warp & 3) * 32 + lane;
@@ -1649,8 +1686,9 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
         !make_map_tiles(&mp, ws_p, items, 64) || !make_map_tiles(&mtb, ws_tb, items, 64) ||
         !make_map_tiles(&mw, ws_w, items, 128))
         return cudaErrorInvalidValue;
-    static std::atomic<uint64_t> conf_prep{0}, conf_chain{0}, conf_tr{0};
-    if (!configure_once((const void *)fwd_prep_kernel, SMEM_PREP, conf_prep) ||
+    static std::atomic<uint64_t> conf_prep{0}, conf_prep_lead{0}, conf_chain{0}, conf_tr{0};
+    if (!configure_once((const void *)fwd_prep_kernel<false>, SMEM_PREP, conf_prep) ||
+        !configure_once((const void *)fwd_prep_kernel<true>, SMEM_PREP, conf_prep_lead) ||
         !configure_once((const void *)fwd_chain_kernel, SMEM_CHAIN, conf_chain) ||
         !configure_once((const void *)fwd_transfer_kernel, SMEM_TR, conf_tr))
         return cudaErrorInvalidValue;
@@ -1666,12 +1704,16 @@ cudaError_t launch_fwd_split(const FwdProblem &p, int nseg, int sm_count, void *
     pa.ctab = nullptr;
     pa.raw_inputs = p.raw_inputs;
     pa.group = p.group;
+    pa.lead = p.lead;
     pa.t_out = static_cast<__nv_bfloat16 *>(p.t_out);
     const int64_t pgrid =
         items < kPrepCtasPerSm * (int64_t)sm_count ? items : kPrepCtasPerSm * (int64_t)sm_count;
     {
         TimedLaunch tl_(GDN_KERNEL_PREP, stream);
-        fwd_prep_kernel<<<(unsigned)pgrid, kPrepThreads, SMEM_PREP, stream>>>(mq, mk, mp, mtb, mw, pa);
+        if (p.lead > 1)
+            fwd_prep_kernel<true><<<(unsigned)pgrid, kPrepThreads, SMEM_PREP, stream>>>(mq, mk, mp, mtb, mw, pa);
+        else
+            fwd_prep_kernel<false><<<(unsigned)pgrid, kPrepThreads, SMEM_PREP, stream>>>(mq, mk, mp, mtb, mw, pa);
     }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -1885,8 +1927,9 @@ cudaError_t launch_fwd_split_packed(const FwdProblem &p, const PackedPlan &pl, v
         !make_map_tiles(&mp, ws_p, rows, 64) || !make_map_tiles(&mtb, ws_tb, rows, 64) ||
         !make_map_tiles(&mw, ws_w, rows, 128))
         return cudaErrorInvalidValue;
-    static std::atomic<uint64_t> conf_prep{0}, conf_chain{0}, conf_tr{0};
-    if (!configure_once((const void *)fwd_prep_kernel, SMEM_PREP, conf_prep) ||
+    static std::atomic<uint64_t> conf_prep{0}, conf_prep_lead{0}, conf_chain{0}, conf_tr{0};
+    if (!configure_once((const void *)fwd_prep_kernel<false>, SMEM_PREP, conf_prep) ||
+        !configure_once((const void *)fwd_prep_kernel<true>, SMEM_PREP, conf_prep_lead) ||
         !configure_once((const void *)fwd_chain_kernel, SMEM_CHAIN, conf_chain) ||
         !configure_once((const void *)fwd_transfer_kernel, SMEM_TR, conf_tr))
         return cudaErrorInvalidValue;
@@ -1903,11 +1946,12 @@ cudaError_t launch_fwd_split_packed(const FwdProblem &p, const PackedPlan &pl, v
         pa.ctab = d_ctab;
         pa.raw_inputs = p.raw_inputs;
         pa.group = 1;
+        pa.lead = 1;
         pa.t_out = nullptr;
         const int64_t pgrid =
             items < kPrepCtasPerSm * (int64_t)sm_count ? items : kPrepCtasPerSm * (int64_t)sm_count;
         TimedLaunch tl_(GDN_KERNEL_PREP, stream);
-        fwd_prep_kernel<<<(unsigned)pgrid, kPrepThreads, SMEM_PREP, stream>>>(mq, mk, mp, mtb, mw, pa);
+        fwd_prep_kernel<false><<<(unsigned)pgrid, kPrepThreads, SMEM_PREP, stream>>>(mq, mk, mp, mtb, mw, pa);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;

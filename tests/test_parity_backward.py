@@ -145,3 +145,43 @@ def test_tensor_core_and_cuda_core_backward_agree(monkeypatch):
     assert kinds["backward"][1] == 3, kinds
     for x, y in zip(a, b):
         assert rel_err(cpu_f64(x), cpu_f64(y)) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("final,s0", [(True, True), (False, False)])
+def test_tensor_core_backward_segments_negligible_and_exact(monkeypatch, final, s0):
+    """A long sequence cut into segments (four here): the reverse chain's transfers, their prefix from
+    dS_final, then every segment's walk at once.  Heads 0 and 2 decay fast, so the chunks past the head
+    of a segment reach its start scaled by at most e^-40: the zero run walks the head alone and the
+    identity run is skipped; heads 1 and 3 keep alpha close to 1, so both runs walk the whole segment
+    and the prefix multiplies by the exact transfer.  Ragged last chunk, with and without S0 and
+    dS_final; still two backward launches (the transfers are timed as transfer launches)."""
+    monkeypatch.setenv("GDN_SEGMENTS", "4")
+    monkeypatch.delenv("GDN_BWD_PATH", raising=False)
+    monkeypatch.delenv("GDN_BWD_RECOMPUTE", raising=False)
+    B, T, H = 1, 64 * 24 + 17, 4
+    inp = forward_inputs(B, T, H, 128, 128, "bf16", seed=91, s0_std=0.3 if s0 else None)
+    inp["log_alpha"][:, :, 1::2] = -1e-3 * torch.rand(inp["log_alpha"][:, :, 1::2].shape,
+                                                       generator=torch.Generator().manual_seed(6))
+    d_out, dSf = grads_in(B, T, H, 128, 128, "bf16", seed=92, final=final)
+    gdn.timing_start()
+    try:
+        check(inp, d_out, dSf, "bf16", 64, label="segments final=%s" % final)
+    finally:
+        kinds = gdn.timing_stop()
+    assert kinds["backward"][1] == 2, kinds
+    assert kinds["transfer"][1] == 2, kinds  # the recompute's forward transfers and the reverse ones
+
+
+def test_tensor_core_backward_segments_match_one_walk(monkeypatch):
+    """The segmented reverse chain gives the gradients of the single walk (GDN_SEGMENTS=1) to within
+    the bf16 bar, both against the oracle."""
+    monkeypatch.delenv("GDN_BWD_PATH", raising=False)
+    B, T, H = 1, 64 * 20, 2
+    inp = forward_inputs(B, T, H, 128, 128, "bf16", seed=93, s0_std=0.1, alpha_mu=-3.0)
+    d_out, dSf = grads_in(B, T, H, 128, 128, "bf16", seed=94)
+    monkeypatch.setenv("GDN_SEGMENTS", "5")
+    a = check(inp, d_out, dSf, "bf16", 64, label="five segments")
+    monkeypatch.setenv("GDN_SEGMENTS", "1")
+    b = check(inp, d_out, dSf, "bf16", 64, label="one walk")
+    for x, y in zip(a, b):
+        assert rel_err(cpu_f64(x), cpu_f64(y)) <= TOL["bf16"]
