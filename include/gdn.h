@@ -245,7 +245,12 @@ int gdn_decode_step_raw(const void *q, const void *k, const void *v, const float
  * adjoint of the state in tensor memory) and a chunk-parallel pass forming
  * every chunk's gradients (scratch about 136 KB per chunk and head: the
  * recompute's workspace, bf16 checkpoints, T of every chunk, and the
- * adjoints passed between the two).  Every other shape, or
+ * adjoints passed between the two).  Long sequences with few heads are cut
+ * into the forward's segments: the adjoint's map through each segment
+ * (affine: the transpose of the segment's forward transfer plus the
+ * segment's own term), a prefix over the segments from grad_S_final, then
+ * every segment's reverse walk at once (3 x 64 KB more scratch per segment
+ * boundary and head).  Every other shape, or
  * GDN_BWD_PATH=simt, walks the chunks backwards with the chunkwise adjoint in
  * float32 on the CUDA cores (checkpoints of dv * dk * 4 bytes per chunk and
  * head, and float32 accumulators of dq and dk for bf16).
@@ -281,7 +286,8 @@ int gdn_backward(const void *q, const void *k, const void *v, const float *log_a
  * runs each memory once as well: the two-kernel tensor-core forward runs the
  * memory of key-value head hk on query head hk * G's chunk items (writing
  * that head's outputs, and per chunk the bf16 state entering it and U^T, in
- * scratch), then one chunk-parallel kernel forms the other query heads'
+ * scratch; the other query heads' chunk items form only their P tiles and
+ * gate records), then one chunk-parallel kernel forms the other query heads'
  * outputs from them.  Other shapes run the CUDA-core forward with
  * per-query-head work items, where each query head recomputes its memory.
  */
