@@ -112,6 +112,7 @@ static_assert(PO_PG + 2 * kPG * 4 <= PO_NRM && PO_NRM + 3 * 64 * 4 <= PO_BARS,
               "prep-kernel gate buffers overflow their slot");
 static_assert(kPrepCtasPerSm * (SMEM_PREP + 1024) <= 233472, "three prep CTAs no longer fit an SM");
 constexpr int kBarMerge = 2;  // named barrier of the four 16->32 merge warps
+constexpr int kBarGates = 3;  // named barrier of the two warps that form an item's gates
 
 constexpr uint32_t TP_G = 0;   // 64 columns: [Q;K] K^T
 constexpr uint32_t TP_W = 64;  // 64 columns: W^T
@@ -318,6 +319,8 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 be_next = p.beta[x];
             }
         }
+        // (threads pt < 64 alone, with their own barrier; the role's next 256-thread barrier, which
+        // every caller reaches before the buffer is read, publishes what they write)
         auto prep_gates = [&](int it) {
             float *gb = reinterpret_cast<float *>(sm + PO_PG) + (it & 1) * kPG;
             if (pt < 64) {
@@ -330,7 +333,7 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
                 const float x = valid ? fmaxf(la, kLogAlphaFloor) : 0.f;
                 gb[64 + pt] = valid ? be : 0.f;
-                const float s = chunk_cumsum(x, pt, scan_tmp, kBarP, kNumPrep);
+                const float s = chunk_cumsum(x, pt, scan_tmp, kBarGates, 64);
                 SDBG(1, 8)
                 gb[pt] = s;
                 if (it + 1 < nit) {
@@ -338,12 +341,8 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     la_next = xn >= 0 ? p.log_alpha[xn] : 0.f;
                     be_next = xn >= 0 ? p.beta[xn] : 0.f;
                 }
-            } else {
-                named_bar(kBarP, kNumPrep);  // the barrier inside chunk_cumsum
-            }
-            named_bar(kBarP, kNumPrep);
-            SDBG(1, 9)
-            if (pt < 64) {
+                named_bar(kBarGates, 64);
+                SDBG(1, 9)
                 const float gt = gb[pt], cm = gb[31];
                 const float gm = expf(gt);
                 gb[128 + pt] = gm;
@@ -364,7 +363,6 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const bool nr = __all_sync(0xffffffffu, fabsf(gt - cm) < 60.f);
                 if (lane == 0) nflags[(it & 1) * 2 + (pt >> 5)] = nr ? 1 : 0;
             }
-            named_bar(kBarP, kNumPrep);
         };
         if (nit > 0) prep_gates(0);
         uint32_t nw = 0;  // items with W^T so far (the phases of WDONE)
@@ -377,7 +375,6 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             // beta, gamma, e^{g - c}, e^{c - g}, beta gamma (the last two carry 1 / |k_s| once the input
             // stage below has run)
             const float *bet = g + 64, *gam = g + 128, *ea = g + 192, *eb = g + 256, *bgm = g + 320;
-            const bool narrow = nflags[par * 2] && nflags[par * 2 + 1];
             // the stores of the previous item have finished reading P, TB and the W^T staging
             if (pt == 0) {
                 SDBG(1, 14)
@@ -394,6 +391,8 @@ fwd_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 if (!(ok = bar_and(kBarP, kNumPrep, w))) break;
             }
             tc_fence_after();
+            // this item's gates and flags, published by the barrier above
+            const bool narrow = nflags[par * 2] && nflags[par * 2 + 1];
             SDBG(1, 1)
             // ---- with the input stage fused: 1 / |q_t| and 1 / |k_s| (the thread pair of a row of
             //      [Q; K] reads its two 64-column boxes), folded into this item's gate buffers in place:
