@@ -57,6 +57,16 @@ constexpr int kRecFloats = 132;  // the forward prep kernel's gate record per ch
 
 __device__ int g_bwd_timeout;  // set when a bounded mbarrier wait gives up
 
+#ifdef GDN_TC_DEBUG
+// Debug builds only: per-phase clock stamps of the gradient pass's CTA 0 for its first 8 items, 16 int64
+// per item.
+__device__ long long *g_bwd_dbg;
+#define BDBG(i) \
+    if (dbgp != nullptr && nd < 8 && tid == 0) dbgp[nd * 16 + (i)] = clock64();
+#else
+#define BDBG(i)
+#endif
+
 // [rows][128] bf16 viewed as a 2-D tensor; box = 64 columns x box_rows rows, 128-byte swizzle.
 inline bool make_map_rows128(CUtensorMap *m, const void *base, int64_t rows, uint32_t box_rows) {
     EncodeTiledFn f = encode_fn();
@@ -561,8 +571,8 @@ constexpr uint32_t R_DS = 114688;   // 32 KB: dS' (bf16), same layout
 constexpr uint32_t R_UT = 147456;   // 16 KB: U^T [128 j][64 s]
 constexpr uint32_t R_TB = 163840;   // 8 KB:  T diag(beta) [t][s]
 constexpr uint32_t R_A1 = 172032;   // 32 KB: [[0, dP o E], [(dP o E)^T, F + F^T]], [128 m][64 k] x 2 boxes
-constexpr uint32_t R_F = 204800;    // floats: g, bet, gam, dl, dg, db, colsum [64 each], misc [16]
-constexpr uint32_t R_BARS = R_F + 7 * 256 + 64;
+constexpr uint32_t R_F = 204800;    // floats: g, bet, gam, dl, dg, db, colsum [64 each], misc [16], keep [64]
+constexpr uint32_t R_BARS = R_F + 8 * 256 + 64;
 constexpr uint32_t R_MISC = R_BARS + 64;
 constexpr uint32_t SMEM_P2 = R_MISC + 64 + 1024;
 static_assert(SMEM_P2 <= 232448, "pass-2 kernel exceeds the shared memory of a CTA");
@@ -583,14 +593,17 @@ __global__ void __launch_bounds__(kP2Threads, 1)
 bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                 const __grid_constant__ CUtensorMap tm_dr, const __grid_constant__ CUtensorMap tm_s,
-                const __grid_constant__ CUtensorMap tm_ds, const __grid_constant__ CUtensorMap tm_tb, BwdArgs p) {
+                const __grid_constant__ CUtensorMap tm_ds, const __grid_constant__ CUtensorMap tm_tb,
+                const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ CUtensorMap tm_dk, BwdArgs p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + R_BARS);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + R_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + R_MISC + 4);
     float *g = reinterpret_cast<float *>(sm + R_F), *bet = g + 64, *gam = g + 128, *dl = g + 192, *dg = g + 256,
-          *db = g + 320, *colsum = g + 384, *misc = g + 448;  // misc: scan scratch, <dS', S>, sum of w
+          *db = g + 320, *colsum = g + 384, *misc = g + 448;  // misc: scan scratch, <dS', S>, sum of w, ...
+    // keep: log alpha_t at or above the forward's floor (its gradient passes)
+    float *keep = g + 464;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t H = p.H, T = p.T;
@@ -631,6 +644,10 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tma_load_2d(sm + R_TB, &tm_tb, full, 0, (int)(item * 64));
     };
     if (tid == 0 && (int64_t)blockIdx.x < p.items) issue_loads(blockIdx.x);
+#ifdef GDN_TC_DEBUG
+    long long *const dbgp = (blockIdx.x == 0) ? g_bwd_dbg : nullptr;
+    int nd = 0;
+#endif
 
     bool ok = true;
     uint32_t lph = 0, mph = 0;
@@ -653,6 +670,7 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int c = (int)(item % nch), b = (int)(bh / H), h = (int)(bh % H), t0 = c * kC;
         const int n = (T - t0 < kC) ? (int)(T - t0) : kC;
         const int64_t gbase = (int64_t)b * T * H + h;
+        BDBG(0)
         // ---- gates (while the loads fly) ----
         chunk_gates(p.log_alpha, p.beta, gbase, H, t0, n, tid, g, bet, misc, 1, kP2Threads);
         if (tid < 64) {
@@ -661,6 +679,8 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             dg[tid] = 0.f;
             db[tid] = 0.f;
             colsum[tid] = 0.f;
+            // the clamp test of the d log alpha step below, its load in flight with the tiles'
+            keep[tid] = (tid < n && p.log_alpha[gbase + (int64_t)(t0 + tid) * H] >= kLogAlphaFloor) ? 1.f : 0.f;
         }
         if (tid == 0) {
             misc[1] = 0.f;
@@ -671,6 +691,7 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             lph ^= 1u;
             if (!(ok = __syncthreads_and(w))) break;  // also publishes the gates
         }
+        BDBG(1)
         const float gC = expf(g[63]);
         // ---- round 1: G = [Q; K] K^T, Z = [Q; K] S^T, D2 = dS' K^T ----
         if (tid == 0) {
@@ -707,6 +728,7 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         mma_round();
         if (!ok) break;
+        BDBG(2)
         // ---- epilogue 1: rows t: d g_t from the outputs' gamma_t Q S^T term; rows 64 + t: X, Y ----
         if (m < 64) {
             const int t = m;
@@ -757,6 +779,7 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             atomicAdd(&dg[t], -bt * rx);
         }
         publish_smem();
+        BDBG(3)
         // ---- round 2: U^T = Y^T (T diag(beta))^T ----
         if (tid == 0) {
 #pragma unroll
@@ -767,6 +790,7 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         mma_round();
         if (!ok) break;
+        BDBG(4)
         // ---- epilogue 2 (row j = tid): U^T into shared memory in bf16; w_s = dl_s sum_j U^T_js D2_js ----
         {
             const int j = m;
@@ -799,6 +823,9 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
             if ((tid & 31) == 0) atomicAdd(&misc[2], x);
         }
+        BDBG(5)
+        // the previous item's dQ / dK stores have read their staging in the A1 tile, which epilogue 3 writes
+        if (tid == 0) bulk_wait_read0();
         // ---- round 3: [dO; dR] U^T ----
         if (tid == 0) {
 #pragma unroll
@@ -809,6 +836,7 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         mma_round();
         if (!ok) break;
+        BDBG(6)
         // ---- epilogue 3: dP o E, F, their d g and dbeta terms; the A1 operand of round 4 ----
         if (m < 64) {
             const int t = m;
@@ -885,6 +913,7 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             atomicAdd(&db[t], bs);
         }
         publish_smem();  // A1 and colsum
+        BDBG(7)
         if (tid < 64) atomicAdd(&dg[tid], -colsum[tid]);
         // ---- round 4: [dQ; dK] = A1 [Q; K] + (scaled) [dO; dR] S + [*; U] dS' ----
         if (tid == 0) {
@@ -903,14 +932,16 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         mma_round();
         if (!ok) break;
+        BDBG(8)
         // every MMA of this item is done: the next item's tiles may land while this one finishes
         if (tid == 0 && item + gridDim.x < p.items) issue_loads(item + gridDim.x);
-        // ---- epilogue 4: dQ (rows t), dK (rows 64 + s) ----
+        // ---- epilogue 4: dQ (rows t), dK (rows 64 + s), staged in the A1 tile (free once round 4 is done:
+        //      [dQ box 0 | dQ box 1 | dK box 0 | dK box 1], 64 rows x 64 columns each) for TMA stores ----
         {
             const int r = m & 63;
             const bool isq = m < 64;
             const float f2 = isq ? gam[r] : -bet[r] * gam[r], f3 = dl[r];
-            __nv_bfloat16 *dst = (isq ? p.dq : p.dk) + (((int64_t)b * T + t0 + r) * H + h) * kD;
+            uint8_t *const stg = sm + R_A1 + ((isq ? 0 : 2) + ch) * 8192;
 #pragma unroll 1
             for (int pc = 2 * ch; pc < 2 * ch + 2; ++pc) {
                 uint32_t x1[32], x2[32], x3[32];
@@ -929,28 +960,51 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                     }
                     pk[i >> 1] = pack_bf16x2(v0, v1);
                 }
-                if (r < n) {
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        reinterpret_cast<uint4 *>(dst + 32 * pc)[q] =
-                            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
-                }
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4 *>(stg + sw128(r, 4 * (pc - 2 * ch) + q)) =
+                        make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
             }
         }
-        // ---- dbeta and d log alpha_r = sum_{t >= r} dg_t + dg_C (zero where log alpha was clamped) ----
-        if (tid < 64 && tid < n) {
-            const float dgC = gC * misc[1] + misc[2];
-            float s = dgC;
-            for (int t = tid; t < 64; ++t) s += dg[t];
-            const int64_t gi = gbase + (int64_t)(t0 + tid) * H;
-            p.dlog_alpha[gi] = (p.log_alpha[gi] >= kLogAlphaFloor) ? s : 0.f;
-            p.dbeta[gi] = db[tid];
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            // rows past the sequence's end are outside the tensor and not written
+            for (int blk = 0; blk < 2; ++blk) {
+                tma_store_4d(&tm_dq, sm + R_A1 + blk * 8192, blk * 64, h, t0, b);
+                tma_store_4d(&tm_dk, sm + R_A1 + (2 + blk) * 8192, blk * 64, h, t0, b);
+            }
+            bulk_commit();
+        }
+        BDBG(9)
+        // ---- dbeta and d log alpha_r = sum_{t >= r} dg_t + dg_C (zero where log alpha was clamped):
+        //      a suffix sum over the two warps' 32 tokens each, then warp 0 adds warp 1's total ----
+        if (tid < 64) {
+            float x = dg[tid];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y = __shfl_down_sync(0xffffffffu, x, o);
+                if (lane + o < 32) x += y;
+            }
+            if (tid == 32) misc[3] = x;
+            named_bar(2, 64);
+            if (tid < 32) x += misc[3];
+            if (tid < n) {
+                const int64_t gi = gbase + (int64_t)(t0 + tid) * H;
+                p.dlog_alpha[gi] = keep[tid] != 0.f ? x + (gC * misc[1] + misc[2]) : 0.f;
+                p.dbeta[gi] = db[tid];
+            }
         }
         tc_fence_before();
         __syncthreads();  // TMEM and the gate buffers are free for the next item
         tc_fence_after();
+        BDBG(10)
+#ifdef GDN_TC_DEBUG
+        ++nd;
+#endif
     }
     if (!ok) *abort_flag = 1;
+    if (tid == 0) bulk_wait0();  // every dQ / dK store has completed
     tc_fence_before();
     __syncthreads();
     if (tid == 0 && *abort_flag) atomicExch(&g_bwd_timeout, 1);
@@ -999,6 +1053,12 @@ TcLayout tc_layout(const BwdProblem &p, int sm_count) {
 }
 
 }  // namespace
+
+#ifdef GDN_TC_DEBUG
+extern "C" int gdn_debug_set_bwd_dump(long long *ptr) {
+    return cudaMemcpyToSymbol(g_bwd_dbg, &ptr, sizeof(ptr)) == cudaSuccess ? 0 : 1;
+}
+#endif
 
 bool take_bwd_timeout() {
     int v = 0;
@@ -1049,9 +1109,10 @@ cudaError_t launch_bwd_tc(const BwdProblem &p, int sm_count, void *workspace, cu
     void *p_tiles = nullptr, *tb_tiles = nullptr;
     fwd_split_ws_tiles(fwd_ws, items, &p_tiles, &tb_tiles);
 
-    CUtensorMap mq, mk, mv, mdo, mp, mt, mtb, mdr, ms, mds;
+    CUtensorMap mq, mk, mv, mdo, mp, mt, mtb, mdr, ms, mds, mdq, mdk;
     if (!make_map_bthd(&mq, f.q, f.B, f.T, f.H) || !make_map_bthd(&mk, f.k, f.B, f.T, f.H) ||
         !make_map_bthd(&mv, f.v, f.B, f.T, f.H) || !make_map_bthd(&mdo, p.d_out, f.B, f.T, f.H) ||
+        !make_map_bthd(&mdq, p.dq, f.B, f.T, f.H) || !make_map_bthd(&mdk, p.dk, f.B, f.T, f.H) ||
         !make_map_tiles(&mp, p_tiles, items, 64) || !make_map_tiles(&mt, tt, items, 64) ||
         !make_map_tiles(&mtb, tb_tiles, items, 64) || !make_map_rows128(&mdr, drw, items * 64, 64) ||
         !make_map_rows128(&ms, ckpt, items * 128, 128) || !make_map_rows128(&mds, dsw, items * 128, 128))
@@ -1112,7 +1173,8 @@ cudaError_t launch_bwd_tc(const BwdProblem &p, int sm_count, void *workspace, cu
     {
         const int64_t grid = items < (int64_t)sm_count ? items : (int64_t)sm_count;
         TimedLaunch tl_(GDN_KERNEL_BACKWARD, stream);
-        bwd_grad_kernel<<<(unsigned)grid, kP2Threads, SMEM_P2, stream>>>(mq, mk, mv, mdo, mdr, ms, mds, mtb, a);
+        bwd_grad_kernel<<<(unsigned)grid, kP2Threads, SMEM_P2, stream>>>(mq, mk, mv, mdo, mdr, ms, mds, mtb, mdq,
+                                                                          mdk, a);
     }
     return cudaGetLastError();
 }
