@@ -63,8 +63,13 @@ __device__ int g_bwd_timeout;  // set when a bounded mbarrier wait gives up
 __device__ long long *g_bwd_dbg;
 #define BDBG(i) \
     if (dbgp != nullptr && nd < 8 && tid == 0) dbgp[nd * 16 + (i)] = clock64();
+// and of the reverse chain's CTA 0 for its first 8 chunks
+__device__ long long *g_bwd1_dbg;
+#define B1DBG(i) \
+    if (blockIdx.x == 0 && g_bwd1_dbg != nullptr && idx < 8 && tid == 0) g_bwd1_dbg[idx * 16 + (i)] = clock64();
 #else
 #define BDBG(i)
+#define B1DBG(i)
 #endif
 
 // [rows][128] bf16 viewed as a 2-D tensor; box = 64 columns x box_rows rows, 128-byte swizzle.
@@ -398,6 +403,7 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
         float gC = (nrun > 0) ? prepare(0) : 0.f;
 #pragma unroll 1
         for (int idx = 0; idx < nrun && ok; ++idx) {
+            B1DBG(0)
             const int c = c_top - idx, s = idx & 1;
             const int t0 = c * kC;
             const int n = (T - t0 < kC) ? (int)(T - t0) : kC;
@@ -429,6 +435,7 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
                 }
             }
             sync_after_tmem_st();
+            B1DBG(1)
             // ---- dO^T P and dS K^T ----
             if (tid == 0) {
                 if (!idrun) {
@@ -445,6 +452,7 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
                 mma_commit(&bars[B1_MMA]);
             }
             mma_round();
+            B1DBG(2)
             if (!ok) break;
             // ---- dU^T = dO^T P + (dS K^T) diag(dl), in bf16 ----
             {
@@ -467,6 +475,7 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
                 tmem_st16(tm + lb + T1_DUB + 16 * pc, pk);
             }
             sync_after_tmem_st();
+            B1DBG(3)
             // ---- dR^T = dU^T T ----
             if (tid == 0) {
 #pragma unroll
@@ -476,6 +485,7 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
                 mma_commit(&bars[B1_MMA]);
             }
             mma_round();
+            B1DBG(4)
             if (!ok) break;
             // ---- dV = diag(beta) dR (output), dR (workspace), -beta gamma dR^T in bf16 ----
             {
@@ -507,6 +517,7 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
                 }
             }
             sync_after_tmem_st();
+            B1DBG(5)
             // ---- dS += dO^T (diag(gamma) Q) - dR^T diag(beta gamma) K ----
             if (tid == 0) {
                 if (!idrun) {
@@ -525,7 +536,9 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             // the next chunk's gates and Q while the state update runs (this chunk's epilogues are
             // done with the gate buffers, and its Q is in the other stage)
             if (idx + 1 < nrun) gC = prepare(idx + 1);
+            B1DBG(6)
             mma_round();
+            B1DBG(7)
         }
         // the adjoint reached at the walk's start: dS0 (the state entering chunk 0) for segment 0, B'_p or
         // X_p for a transfer run
@@ -577,7 +590,9 @@ constexpr uint32_t R_MISC = R_BARS + 64;
 constexpr uint32_t SMEM_P2 = R_MISC + 64 + 1024;
 static_assert(SMEM_P2 <= 232448, "pass-2 kernel exceeds the shared memory of a CTA");
 
-enum P2Bar { B2_LOAD = 0, B2_MMA, B2_COUNT };
+// B2_LOAD: Q, K, dO, dR, S, dS' of an item; B2_LOADE: its V and T diag(beta), which load as soon as the
+// previous item's round 2 has read its own
+enum P2Bar { B2_LOAD = 0, B2_LOADE, B2_MMA, B2_COUNT };
 
 // tensor memory of pass 2 (the last round reuses columns 0..383)
 constexpr uint32_t T2_G = 0;     // 64:  [Q; K] K^T
@@ -631,19 +646,28 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int64_t bh = item / nch;
         const int c = (int)(item % nch), b = (int)(bh / H), h = (int)(bh % H), t0 = c * kC;
         uint64_t *full = &bars[B2_LOAD];
-        mbar_arrive_expect_tx(full, 32768 * 4 + 16384 + 8192);
+        mbar_arrive_expect_tx(full, 32768 * 4);
         for (int blk = 0; blk < 2; ++blk) {
             tma_load_4d(sm + R_QK + blk * 16384, &tm_q, full, blk * 64, h, t0, b);
             tma_load_4d(sm + R_QK + blk * 16384 + 8192, &tm_k, full, blk * 64, h, t0, b);
             tma_load_4d(sm + R_DOR + blk * 16384, &tm_do, full, blk * 64, h, t0, b);
             tma_load_2d(sm + R_DOR + blk * 16384 + 8192, &tm_dr, full, blk * 64, (int)(item * 64));
-            tma_load_4d(sm + R_V + blk * 8192, &tm_v, full, blk * 64, h, t0, b);
             tma_load_2d(sm + R_S + blk * 16384, &tm_s, full, blk * 64, (int)(item * 128));
             tma_load_2d(sm + R_DS + blk * 16384, &tm_ds, full, blk * 64, (int)(item * 128));
         }
+    };
+    auto issue_loads_early = [&](int64_t item) {  // thread 0
+        const int64_t bh = item / nch;
+        const int c = (int)(item % nch), b = (int)(bh / H), h = (int)(bh % H), t0 = c * kC;
+        uint64_t *full = &bars[B2_LOADE];
+        mbar_arrive_expect_tx(full, 16384 + 8192);
+        for (int blk = 0; blk < 2; ++blk) tma_load_4d(sm + R_V + blk * 8192, &tm_v, full, blk * 64, h, t0, b);
         tma_load_2d(sm + R_TB, &tm_tb, full, 0, (int)(item * 64));
     };
-    if (tid == 0 && (int64_t)blockIdx.x < p.items) issue_loads(blockIdx.x);
+    if (tid == 0 && (int64_t)blockIdx.x < p.items) {
+        issue_loads_early(blockIdx.x);
+        issue_loads(blockIdx.x);
+    }
 #ifdef GDN_TC_DEBUG
     long long *const dbgp = (blockIdx.x == 0) ? g_bwd_dbg : nullptr;
     int nd = 0;
@@ -687,7 +711,7 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             misc[2] = 0.f;
         }
         {
-            const bool w = wait_bar(&bars[B2_LOAD], lph, abort_flag);
+            const bool w = wait_bar(&bars[B2_LOAD], lph, abort_flag) && wait_bar(&bars[B2_LOADE], lph, abort_flag);
             lph ^= 1u;
             if (!(ok = __syncthreads_and(w))) break;  // also publishes the gates
         }
@@ -790,6 +814,8 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         mma_round();
         if (!ok) break;
+        // round 2 has read this item's V (now Y) and T diag(beta): the next item's may land
+        if (tid == 0 && item + gridDim.x < p.items) issue_loads_early(item + gridDim.x);
         BDBG(4)
         // ---- epilogue 2 (row j = tid): U^T into shared memory in bf16; w_s = dl_s sum_j U^T_js D2_js ----
         {
@@ -1004,7 +1030,14 @@ bwd_grad_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #endif
     }
     if (!ok) *abort_flag = 1;
-    if (tid == 0) bulk_wait0();  // every dQ / dK store has completed
+    if (tid == 0) {
+        bulk_wait0();  // every dQ / dK store has completed
+        // after an abort, tile loads of the next item may still be in flight: bounded waits for them
+        if (!ok) {
+            mbar_wait(&bars[B2_LOADE], lph, 1u << 20);
+            mbar_wait(&bars[B2_LOAD], lph, 1u << 20);
+        }
+    }
     tc_fence_before();
     __syncthreads();
     if (tid == 0 && *abort_flag) atomicExch(&g_bwd_timeout, 1);
@@ -1057,6 +1090,9 @@ TcLayout tc_layout(const BwdProblem &p, int sm_count) {
 #ifdef GDN_TC_DEBUG
 extern "C" int gdn_debug_set_bwd_dump(long long *ptr) {
     return cudaMemcpyToSymbol(g_bwd_dbg, &ptr, sizeof(ptr)) == cudaSuccess ? 0 : 1;
+}
+extern "C" int gdn_debug_set_bwd1_dump(long long *ptr) {
+    return cudaMemcpyToSymbol(g_bwd1_dbg, &ptr, sizeof(ptr)) == cudaSuccess ? 0 : 1;
 }
 #endif
 
