@@ -125,14 +125,11 @@ __device__ __forceinline__ float warp_colsum32(float (&v)[32]) {
 // Chunk-local inclusive cumsum g_t of the clamped log-decays (zero past the n valid tokens) and
 // beta_t, by threads 0..63 of a group of `nthreads` that share named barrier `bar_id`; every thread
 // of the group calls it.  g[], bet[] receive 64 entries.
-__device__ __forceinline__ void chunk_gates(const float *log_alpha, const float *beta, int64_t gbase, int64_t H,
-                                            int t0, int n, int tid, float *g, float *bet, float *scratch,
-                                            int bar_id, int nthreads) {
-    float la = 0.f, be = 0.f;
-    if (tid < 64 && tid < n) {
-        la = fmaxf(log_alpha[gbase + (int64_t)(t0 + tid) * H], kLogAlphaFloor);
-        be = beta[gbase + (int64_t)(t0 + tid) * H];
-    }
+// chunk_gates_from takes this thread's raw gates (log alpha unclamped, zero past the valid tokens).
+__device__ __forceinline__ void chunk_gates_from(float la, float be, int n, int tid, float *g, float *bet,
+                                                 float *scratch, int bar_id, int nthreads) {
+    la = (tid < 64 && tid < n) ? fmaxf(la, kLogAlphaFloor) : 0.f;
+    be = (tid < 64 && tid < n) ? be : 0.f;
     float s = la;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
@@ -147,6 +144,16 @@ __device__ __forceinline__ void chunk_gates(const float *log_alpha, const float 
         bet[tid] = be;
     }
     named_bar(bar_id, nthreads);
+}
+__device__ __forceinline__ void chunk_gates(const float *log_alpha, const float *beta, int64_t gbase, int64_t H,
+                                            int t0, int n, int tid, float *g, float *bet, float *scratch,
+                                            int bar_id, int nthreads) {
+    float la = 0.f, be = 0.f;
+    if (tid < 64 && tid < n) {
+        la = log_alpha[gbase + (int64_t)(t0 + tid) * H];
+        be = beta[gbase + (int64_t)(t0 + tid) * H];
+    }
+    chunk_gates_from(la, be, n, tid, g, bet, scratch, bar_id, nthreads);
 }
 
 constexpr uint32_t IDESC_64_MN_MN = instr_desc_bf16(128, 64, 1, 1);
@@ -171,10 +178,16 @@ constexpr uint32_t S1_K = 32768;    // 16 KB: K
 constexpr uint32_t S1_P = 49152;    // 8 KB:  P [t][s]
 constexpr uint32_t S1_T = 57344;    // 8 KB:  T [s][t]
 constexpr uint32_t S1_BYTES = 65536;
-constexpr uint32_t O1_GATE = 2 * S1_BYTES;  // g[64], bet[64], gam[64], dl[64], scratch[16]
+// staging of the outputs for TMA stores (128-byte swizzle): dS' [128 j][128 i] as two [128][64] boxes,
+// dR and dV [64 t][128 j] as two [64][64] boxes each
+constexpr uint32_t O1_DSST = 2 * S1_BYTES;    // 32 KB
+constexpr uint32_t O1_DRST = O1_DSST + 32768;  // 16 KB
+constexpr uint32_t O1_DVST = O1_DRST + 16384;  // 16 KB
+constexpr uint32_t O1_GATE = O1_DVST + 16384;  // g[64], bet[64], gam[64], dl[64], scratch[16]
 constexpr uint32_t O1_BARS = O1_GATE + 1088;
 constexpr uint32_t O1_MISC = O1_BARS + 64;
 constexpr uint32_t SMEM_P1 = O1_MISC + 64 + 1024;
+static_assert(SMEM_P1 <= 232448, "pass-1 kernel exceeds the shared memory of a CTA");
 
 enum P1Bar { B1_FULL0 = 0, B1_FULL1, B1_EMPTY0, B1_EMPTY1, B1_MMA, B1_COUNT };
 static_assert(B1_COUNT * 8 <= O1_MISC - O1_BARS, "pass-1 mbarriers overflow their slot");
@@ -217,7 +230,8 @@ struct BwdArgs {
 __global__ void __launch_bounds__(kP1Threads, 1)
 bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_q,
                  const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_p,
-                 const __grid_constant__ CUtensorMap tm_t, BwdArgs p) {
+                 const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_dsw,
+                 const __grid_constant__ CUtensorMap tm_drw, const __grid_constant__ CUtensorMap tm_dv, BwdArgs p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + O1_BARS);
@@ -370,12 +384,24 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
         // the gates of chunk number idx (counted from the last) into the gate buffers, its stage
         // landed, its Q rows scaled by gamma_t in place (16-byte unit u: box u >> 9, row (u >> 3) & 63);
         // returns gamma_C
+        // the raw gates of the next chunk to prepare, loaded one chunk ahead (threads tid < 64)
+        float la_pf = 0.f, be_pf = 0.f;
+        auto fetch_gates = [&](int idx) {
+            if (idx < nrun && tid < 64) {
+                const int t0 = (c_top - idx) * kC;
+                const int n = (T - t0 < kC) ? (int)(T - t0) : kC;
+                const int64_t x = ((int64_t)b * T + t0 + tid) * H + h;
+                la_pf = tid < n ? p.log_alpha[x] : 0.f;
+                be_pf = tid < n ? p.beta[x] : 0.f;
+            }
+        };
+        fetch_gates(0);
         auto prepare = [&](int idx) -> float {
             const int c = c_top - idx, s = idx & 1;
             const int t0 = c * kC;
             const int n = (T - t0 < kC) ? (int)(T - t0) : kC;
-            chunk_gates(p.log_alpha, p.beta, (int64_t)b * T * H + h, H, t0, n, tid, g, bet, scratch, kBarP1,
-                        kP1Compute);
+            chunk_gates_from(la_pf, be_pf, n, tid, g, bet, scratch, kBarP1, kP1Compute);
+            fetch_gates(idx + 1);
             if (tid < 64) {
                 gam[tid] = expf(g[tid]);
                 dl[tid] = expf(g[63] - g[tid]);
@@ -406,13 +432,11 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             B1DBG(0)
             const int c = c_top - idx, s = idx & 1;
             const int t0 = c * kC;
-            const int n = (T - t0 < kC) ? (int)(T - t0) : kC;
             const int64_t item = bh * nch + c;
             const uint32_t sta = sbase + s * S1_BYTES;
             // ---- dS (the adjoint of the state leaving chunk c): bf16 copy into TMEM and to the
             //      workspace, then dS <- gamma_C dS ----
             {
-                __nv_bfloat16 *dsg = p.ds_ws + (item * kD + j) * kD;
 #pragma unroll 1
                 for (int pc = 2 * ch; pc < 2 * ch + 2; ++pc) {
                     uint32_t r[32];
@@ -426,7 +450,7 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
                     if (p.mode == 0) {
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
-                            reinterpret_cast<uint4 *>(dsg + 32 * pc)[i] =
+                            *reinterpret_cast<uint4 *>(sm + O1_DSST + ch * 16384 + sw128(j, (pc & 1) * 4 + i)) =
                                 make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
                     }
 #pragma unroll
@@ -434,7 +458,14 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
                     tmem_st32(tm + lb + T1_DS + 32 * pc, r);
                 }
             }
+            if (p.mode == 0) fence_proxy_async_smem();
             sync_after_tmem_st();
+            if (p.mode == 0 && tid == 0) {
+                // dS' of this chunk to the workspace (pass 2 reads it)
+                for (int blk = 0; blk < 2; ++blk)
+                    tma_store_2d(&tm_dsw, sm + O1_DSST + blk * 16384, blk * 64, (int)(item * 128));
+                bulk_commit();
+            }
             B1DBG(1)
             // ---- dO^T P and dS K^T ----
             if (tid == 0) {
@@ -489,34 +520,42 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             if (!ok) break;
             // ---- dV = diag(beta) dR (output), dR (workspace), -beta gamma dR^T in bf16 ----
             {
-                __nv_bfloat16 *drg = p.dr_ws + item * kC * kD + j;
-                __nv_bfloat16 *dvg = p.dv + (((int64_t)b * T + t0) * H + h) * kD + j;
+                // thread j holds column j of dR (tokens 32 pc ..): element (t, j) of the staged [64 t][128 j]
+                // tiles sits in box j / 64, row t, 16-byte chunk (j % 64) / 8
+                const uint32_t col = (uint32_t)(j >> 6) * 8192, cj = (uint32_t)((j & 63) >> 3), bj = (j & 7) * 2;
                 {
                     const int pc = ch;
                     uint32_t r[32];
                     tmem_ld32(tm + lb + T1_DR + 32 * pc, r);
                     tmem_wait_ld();
                     uint32_t pk[16];
-                    const int64_t vstr = H * kD;  // token stride of dV
-                    __nv_bfloat16 *dr_row = drg + (int64_t)(32 * pc) * kD, *dv_row = dvg + (int64_t)(32 * pc) * vstr;
 #pragma unroll
                     for (int i = 0; i < 32; i += 2) {
                         const int t = 32 * pc + i;
                         const float x0 = __uint_as_float(r[i]), x1 = __uint_as_float(r[i + 1]);
                         if (p.mode == 0) {
-                            dr_row[i * kD] = __float2bfloat16_rn(x0);
-                            dr_row[(i + 1) * kD] = __float2bfloat16_rn(x1);
-                            if (t < n) *dv_row = __float2bfloat16_rn(bet[t] * x0);
-                            dv_row += vstr;
-                            if (t + 1 < n) *dv_row = __float2bfloat16_rn(bet[t + 1] * x1);
-                            dv_row += vstr;
+                            const uint32_t o0 = col + sw128(t, cj) + bj, o1 = col + sw128(t + 1, cj) + bj;
+                            *reinterpret_cast<uint16_t *>(sm + O1_DRST + o0) = bf16_bits(x0);
+                            *reinterpret_cast<uint16_t *>(sm + O1_DRST + o1) = bf16_bits(x1);
+                            *reinterpret_cast<uint16_t *>(sm + O1_DVST + o0) = bf16_bits(bet[t] * x0);
+                            *reinterpret_cast<uint16_t *>(sm + O1_DVST + o1) = bf16_bits(bet[t + 1] * x1);
                         }
                         pk[i >> 1] = pack_bf16x2(-bet[t] * gam[t] * x0, -bet[t + 1] * gam[t + 1] * x1);
                     }
                     tmem_st16(tm + lb + T1_DRB + 16 * pc, pk);
                 }
             }
+            if (p.mode == 0) fence_proxy_async_smem();
             sync_after_tmem_st();
+            if (p.mode == 0 && tid == 0) {
+                // dR to the workspace, dV to the output (its rows past the sequence's end are outside the
+                // tensor and not written)
+                for (int blk = 0; blk < 2; ++blk) {
+                    tma_store_2d(&tm_drw, sm + O1_DRST + blk * 8192, blk * 64, (int)(item * 64));
+                    tma_store_4d(&tm_dv, sm + O1_DVST + blk * 8192, blk * 64, h, t0, b);
+                }
+                bulk_commit();
+            }
             B1DBG(5)
             // ---- dS += dO^T (diag(gamma) Q) - dR^T diag(beta gamma) K ----
             if (tid == 0) {
@@ -537,6 +576,9 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             // done with the gate buffers, and its Q is in the other stage)
             if (idx + 1 < nrun) gC = prepare(idx + 1);
             B1DBG(6)
+            // this chunk's stores have read their staging before the next chunk writes it (the barrier
+            // of the round below orders the other threads)
+            if (tid == 0) bulk_wait_read0();
             mma_round();
             B1DBG(7)
         }
@@ -561,6 +603,7 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             }
         }
         if (!ok) *abort_flag = 1;
+        if (tid == 0) bulk_wait0();  // every dS', dR and dV store has completed
     }
     tc_fence_before();
     __syncthreads();
@@ -1145,10 +1188,11 @@ cudaError_t launch_bwd_tc(const BwdProblem &p, int sm_count, void *workspace, cu
     void *p_tiles = nullptr, *tb_tiles = nullptr;
     fwd_split_ws_tiles(fwd_ws, items, &p_tiles, &tb_tiles);
 
-    CUtensorMap mq, mk, mv, mdo, mp, mt, mtb, mdr, ms, mds, mdq, mdk;
+    CUtensorMap mq, mk, mv, mdo, mp, mt, mtb, mdr, ms, mds, mdq, mdk, mdv;
     if (!make_map_bthd(&mq, f.q, f.B, f.T, f.H) || !make_map_bthd(&mk, f.k, f.B, f.T, f.H) ||
         !make_map_bthd(&mv, f.v, f.B, f.T, f.H) || !make_map_bthd(&mdo, p.d_out, f.B, f.T, f.H) ||
         !make_map_bthd(&mdq, p.dq, f.B, f.T, f.H) || !make_map_bthd(&mdk, p.dk, f.B, f.T, f.H) ||
+        !make_map_bthd(&mdv, p.dv, f.B, f.T, f.H) ||
         !make_map_tiles(&mp, p_tiles, items, 64) || !make_map_tiles(&mt, tt, items, 64) ||
         !make_map_tiles(&mtb, tb_tiles, items, 64) || !make_map_rows128(&mdr, drw, items * 64, 64) ||
         !make_map_rows128(&ms, ckpt, items * 128, 128) || !make_map_rows128(&mds, dsw, items * 128, 128))
@@ -1192,7 +1236,7 @@ cudaError_t launch_bwd_tc(const BwdProblem &p, int sm_count, void *workspace, cu
         {
             TimedLaunch tl_(GDN_KERNEL_TRANSFER, stream);
             bwd_chain_kernel<<<(unsigned)(heads * (l.nseg_run - 1) * 2), kP1Threads, SMEM_P1, stream>>>(
-                mdo, mq, mk, mp, mt, a);
+                mdo, mq, mk, mp, mt, mds, mdr, mdv, a);
         }
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         if ((e = launch_seg_prefix(p.dS_final, a.xb, a.xm, a.xflag, entry, heads, l.nseg_run, stream, nullptr)) !=
@@ -1203,7 +1247,8 @@ cudaError_t launch_bwd_tc(const BwdProblem &p, int sm_count, void *workspace, cu
     a.mode = 0;
     {
         TimedLaunch tl_(GDN_KERNEL_BACKWARD, stream);
-        bwd_chain_kernel<<<(unsigned)(heads * l.nseg_run), kP1Threads, SMEM_P1, stream>>>(mdo, mq, mk, mp, mt, a);
+        bwd_chain_kernel<<<(unsigned)(heads * l.nseg_run), kP1Threads, SMEM_P1, stream>>>(mdo, mq, mk, mp, mt, mds,
+                                                                                       mdr, mdv, a);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     {
