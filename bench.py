@@ -43,8 +43,8 @@ from gdn_inputs import (WORKLOADS, as_f32_numpy, decode_inputs, forward_inputs, 
                         varlen_inputs)
 
 FWD_WORKLOAD = "fwd_bf16_b1h16_t64k_d128"
-# the decode workload of the survey (state 67 MB, 134 MB read and written per step, partly served by the
-# 126 MB L2) and one whose state (268 MB, 537 MB per step) is twice L2, so that its HBM fraction is not
+# the serving decode workload at batch 64 (state 67 MB, 134 MB read and written per step, partly served by
+# the 126 MB L2) and one whose state (268 MB, 537 MB per step) is twice L2, so that its HBM fraction is not
 # helped by the cache
 DEC_WORKLOADS = ("decode_bf16_b64h16_d128_x1024", "decode_bf16_b256h16_d128_x256")
 METRIC = "gated-delta forward tokens/s & TFLOP/s vs BF16 roofline; decode GB/s vs HBM peak"
@@ -474,7 +474,7 @@ def run_gdn(args, world, rank, local):
                          "traffic_per_launch": tr}
         step_traffic = None if (step_traffic is None or tr is None) else step_traffic + tr * n / args.steps
     top = max(kernels, key=lambda k: ktimes[k][0]) if kernels else None
-    # SURVEY-style roofline of the whole step: the counted FLOP of the chunkwise method over the step's
+    # roofline of the whole step: the counted FLOP of the chunkwise method over the step's
     # device time against the measured dense bf16 peak (burst: the step is timed as a short burst of
     # launches), and the compulsory bytes against the measured copy bandwidth beside it.
     roof = {"bound": "tensor", "kernel": "forward step (%d launches)" % launches_per_fwd,
