@@ -167,8 +167,9 @@ constexpr uint32_t IDESC_128_KK = instr_desc_bf16(128, 128, 0, 0);
 // ============================================================================
 // pass 1: reverse chain
 // ============================================================================
-constexpr int kP1Threads = 288;  // warps 0-7: the chain, two per TMEM lane quadrant (value dim j = lane
-                                 // 32 (w & 3) + lane, column half w >> 2); warp 8: TMA
+constexpr int kP1Threads = 320;  // warps 0-7: the chain, two per TMEM lane quadrant (value dim j = lane
+                                 // 32 (w & 3) + lane, column half w >> 2); warp 8: TMA; warp 9: each chunk's
+                                 // gates and gamma-scaled Q, one chunk ahead of the chain
 constexpr int kP1Compute = 256;
 constexpr int kBarP1 = 1;
 
@@ -183,13 +184,26 @@ constexpr uint32_t S1_BYTES = 65536;
 constexpr uint32_t O1_DSST = 2 * S1_BYTES;    // 32 KB
 constexpr uint32_t O1_DRST = O1_DSST + 32768;  // 16 KB
 constexpr uint32_t O1_DVST = O1_DRST + 16384;  // 16 KB
-constexpr uint32_t O1_GATE = O1_DVST + 16384;  // g[64], bet[64], gam[64], dl[64], scratch[16]
-constexpr uint32_t O1_BARS = O1_GATE + 1088;
-constexpr uint32_t O1_MISC = O1_BARS + 64;
+constexpr uint32_t O1_GATE = O1_DVST + 16384;  // per chunk parity: bet[64], gam[64], dl[64], gamma_C (1 KB)
+constexpr uint32_t O1_BARS = O1_GATE + 2048;
+constexpr uint32_t O1_MISC = O1_BARS + 128;
 constexpr uint32_t SMEM_P1 = O1_MISC + 64 + 1024;
 static_assert(SMEM_P1 <= 232448, "pass-1 kernel exceeds the shared memory of a CTA");
 
-enum P1Bar { B1_FULL0 = 0, B1_FULL1, B1_EMPTY0, B1_EMPTY1, B1_MMA, B1_COUNT };
+// READY: a chunk's gates are in their buffer and its stage has landed with Q scaled; GFREE: the chain is done
+// with a gate buffer (both per chunk parity)
+enum P1Bar {
+    B1_FULL0 = 0,
+    B1_FULL1,
+    B1_EMPTY0,
+    B1_EMPTY1,
+    B1_MMA,
+    B1_READY0,
+    B1_READY1,
+    B1_GFREE0,
+    B1_GFREE1,
+    B1_COUNT
+};
 static_assert(B1_COUNT * 8 <= O1_MISC - O1_BARS, "pass-1 mbarriers overflow their slot");
 
 // tensor memory of pass 1
@@ -237,8 +251,7 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + O1_BARS);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + O1_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + O1_MISC + 4);
-    float *g = reinterpret_cast<float *>(sm + O1_GATE), *bet = g + 64, *gam = g + 128, *dl = g + 192,
-          *scratch = g + 256;
+    float *gbuf = reinterpret_cast<float *>(sm + O1_GATE);  // [2][256]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t H = p.H, T = p.T;
@@ -333,6 +346,65 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             }
         }
         __syncwarp();
+    } else if (warp == 9) {
+        // ============================ prepare ============================
+        // chunk idx's gates into buffer idx & 1 (once the chain is done with chunk idx - 2's), then its
+        // stage's Q rows scaled by gamma_t in place once the stage has landed (16-byte unit u: box u >> 9,
+        // row (u >> 3) & 63)
+        bool ok = true;
+        for (int idx = 0; idx < nrun && ok; ++idx) {
+            const int c = c_top - idx, s = idx & 1;
+            const int t0 = c * kC;
+            const int n = (T - t0 < kC) ? (int)(T - t0) : kC;
+            // the raw gates of tokens lane and lane + 32 (zero past the valid tokens)
+            float la[2], be[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int t = lane + 32 * k;
+                const int64_t x = ((int64_t)b * T + t0 + t) * H + h;
+                la[k] = t < n ? fmaxf(p.log_alpha[x], kLogAlphaFloor) : 0.f;
+                be[k] = t < n ? p.beta[x] : 0.f;
+            }
+            // inclusive cumsum over the 64 tokens: each half by shuffles, the first half's total then
+            // added to the second
+            float s0 = la[0], s1 = la[1];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const float y0 = __shfl_up_sync(0xffffffffu, s0, o), y1 = __shfl_up_sync(0xffffffffu, s1, o);
+                if (lane >= o) {
+                    s0 += y0;
+                    s1 += y1;
+                }
+            }
+            s1 += __shfl_sync(0xffffffffu, s0, 31);
+            const float g63 = __shfl_sync(0xffffffffu, s1, 31);
+            if (idx >= 2 && !(ok = wait_bar(&bars[B1_GFREE0 + s], ((idx - 2) >> 1) & 1, abort_flag))) break;
+            float *gb = gbuf + s * 256;
+            gb[lane] = be[0];
+            gb[32 + lane] = be[1];
+            gb[64 + lane] = expf(s0);
+            gb[96 + lane] = expf(s1);
+            gb[128 + lane] = expf(g63 - s0);
+            gb[160 + lane] = expf(g63 - s1);
+            if (lane == 0) gb[192] = expf(g63);
+            if (!(ok = wait_bar(&bars[B1_FULL0 + s], (idx >> 1) & 1, abort_flag))) break;
+            __syncwarp();
+            if (!idrun) {
+                uint4 *q = reinterpret_cast<uint4 *>(sm + s * S1_BYTES + S1_Q);
+#pragma unroll 4
+                for (int i = 0; i < 32; ++i) {
+                    const int u = lane + 32 * i;
+                    float f[8];
+                    unpack8(q[u], f);
+                    const float x = gb[64 + ((u >> 3) & 63)];
+                    q[u] = make_uint4(pack_bf16x2(f[0] * x, f[1] * x), pack_bf16x2(f[2] * x, f[3] * x),
+                                      pack_bf16x2(f[4] * x, f[5] * x), pack_bf16x2(f[6] * x, f[7] * x));
+                }
+                fence_proxy_async_smem();
+            }
+            __syncwarp();
+            if (lane == 0) arrive(&bars[B1_READY0 + s]);
+        }
     } else {
         // ============================ the chain ============================
         const int j = (warp & 3) * 32 + lane;  // value dim = TMEM lane
@@ -381,52 +453,6 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             named_bar(kBarP1, kP1Compute);
             tc_fence_after();
         };
-        // the gates of chunk number idx (counted from the last) into the gate buffers, its stage
-        // landed, its Q rows scaled by gamma_t in place (16-byte unit u: box u >> 9, row (u >> 3) & 63);
-        // returns gamma_C
-        // the raw gates of the next chunk to prepare, loaded one chunk ahead (threads tid < 64)
-        float la_pf = 0.f, be_pf = 0.f;
-        auto fetch_gates = [&](int idx) {
-            if (idx < nrun && tid < 64) {
-                const int t0 = (c_top - idx) * kC;
-                const int n = (T - t0 < kC) ? (int)(T - t0) : kC;
-                const int64_t x = ((int64_t)b * T + t0 + tid) * H + h;
-                la_pf = tid < n ? p.log_alpha[x] : 0.f;
-                be_pf = tid < n ? p.beta[x] : 0.f;
-            }
-        };
-        fetch_gates(0);
-        auto prepare = [&](int idx) -> float {
-            const int c = c_top - idx, s = idx & 1;
-            const int t0 = c * kC;
-            const int n = (T - t0 < kC) ? (int)(T - t0) : kC;
-            chunk_gates_from(la_pf, be_pf, n, tid, g, bet, scratch, kBarP1, kP1Compute);
-            fetch_gates(idx + 1);
-            if (tid < 64) {
-                gam[tid] = expf(g[tid]);
-                dl[tid] = expf(g[63] - g[tid]);
-            }
-            const float gc = expf(g[63]);
-            const bool w = wait_bar(&bars[B1_FULL0 + s], (idx >> 1) & 1, abort_flag);
-            const bool r = bar_and(kBarP1, kP1Compute, w);  // also publishes gam, dl
-            ok = ok && r;
-            if (r && !idrun) {
-                uint8_t *st = sm + s * S1_BYTES;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int u = tid + 256 * i;
-                    uint4 *ptr = reinterpret_cast<uint4 *>(st + S1_Q) + u;
-                    float f[8];
-                    unpack8(*ptr, f);
-                    const float x = gam[(u >> 3) & 63];
-                    *ptr = make_uint4(pack_bf16x2(f[0] * x, f[1] * x), pack_bf16x2(f[2] * x, f[3] * x),
-                                      pack_bf16x2(f[4] * x, f[5] * x), pack_bf16x2(f[6] * x, f[7] * x));
-                }
-                fence_proxy_async_smem();
-            }
-            return gc;
-        };
-        float gC = (nrun > 0) ? prepare(0) : 0.f;
 #pragma unroll 1
         for (int idx = 0; idx < nrun && ok; ++idx) {
             B1DBG(0)
@@ -434,6 +460,13 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             const int t0 = c * kC;
             const int64_t item = bh * nch + c;
             const uint32_t sta = sbase + s * S1_BYTES;
+            // this chunk's gates, and its stage (landed, Q scaled), from the prepare warp
+            {
+                const bool w = wait_bar(&bars[B1_READY0 + s], (idx >> 1) & 1, abort_flag);
+                if (!(ok = bar_and(kBarP1, kP1Compute, w) && ok)) break;
+            }
+            const float *bet = gbuf + s * 256, *gam = bet + 64, *dl = bet + 128;
+            const float gC = bet[192];
             // ---- dS (the adjoint of the state leaving chunk c): bf16 copy into TMEM and to the
             //      workspace, then dS <- gamma_C dS ----
             {
@@ -469,6 +502,9 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             B1DBG(1)
             // ---- dO^T P and dS K^T ----
             if (tid == 0) {
+                // the issuing thread observes the stage's loads itself (complete long since: the prepare
+                // warp saw them before this chunk was ready)
+                wait_bar(&bars[B1_FULL0 + s], (idx >> 1) & 1, abort_flag);
                 if (!idrun) {
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
@@ -547,6 +583,7 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             }
             if (p.mode == 0) fence_proxy_async_smem();
             sync_after_tmem_st();
+            if (tid == 0) arrive(&bars[B1_GFREE0 + s]);  // this chunk's gates are no longer read
             if (p.mode == 0 && tid == 0) {
                 // dR to the workspace, dV to the output (its rows past the sequence's end are outside the
                 // tensor and not written)
@@ -572,9 +609,6 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
                 mma_commit(&bars[B1_EMPTY0 + s]);
                 mma_commit(&bars[B1_MMA]);
             }
-            // the next chunk's gates and Q while the state update runs (this chunk's epilogues are
-            // done with the gate buffers, and its Q is in the other stage)
-            if (idx + 1 < nrun) gC = prepare(idx + 1);
             B1DBG(6)
             // this chunk's stores have read their staging before the next chunk writes it (the barrier
             // of the round below orders the other threads)
