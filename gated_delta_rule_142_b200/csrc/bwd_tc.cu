@@ -554,45 +554,24 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
             mma_round();
             B1DBG(4)
             if (!ok) break;
-            // ---- dV = diag(beta) dR (output), dR (workspace), -beta gamma dR^T in bf16 ----
+            // ---- -beta gamma dR^T in bf16 for the state update; then, while that runs, dV = diag(beta) dR
+            //      (output) and dR (workspace) ----
+            uint32_t r[32];
+            tmem_ld32(tm + lb + T1_DR + 32 * ch, r);
+            tmem_wait_ld();
             {
-                // thread j holds column j of dR (tokens 32 pc ..): element (t, j) of the staged [64 t][128 j]
-                // tiles sits in box j / 64, row t, 16-byte chunk (j % 64) / 8
-                const uint32_t col = (uint32_t)(j >> 6) * 8192, cj = (uint32_t)((j & 63) >> 3), bj = (j & 7) * 2;
-                {
-                    const int pc = ch;
-                    uint32_t r[32];
-                    tmem_ld32(tm + lb + T1_DR + 32 * pc, r);
-                    tmem_wait_ld();
-                    uint32_t pk[16];
+                uint32_t pk[16];
 #pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const int t = 32 * pc + i;
-                        const float x0 = __uint_as_float(r[i]), x1 = __uint_as_float(r[i + 1]);
-                        if (p.mode == 0) {
-                            const uint32_t o0 = col + sw128(t, cj) + bj, o1 = col + sw128(t + 1, cj) + bj;
-                            *reinterpret_cast<uint16_t *>(sm + O1_DRST + o0) = bf16_bits(x0);
-                            *reinterpret_cast<uint16_t *>(sm + O1_DRST + o1) = bf16_bits(x1);
-                            *reinterpret_cast<uint16_t *>(sm + O1_DVST + o0) = bf16_bits(bet[t] * x0);
-                            *reinterpret_cast<uint16_t *>(sm + O1_DVST + o1) = bf16_bits(bet[t + 1] * x1);
-                        }
-                        pk[i >> 1] = pack_bf16x2(-bet[t] * gam[t] * x0, -bet[t + 1] * gam[t + 1] * x1);
-                    }
-                    tmem_st16(tm + lb + T1_DRB + 16 * pc, pk);
+                for (int i = 0; i < 32; i += 2) {
+                    const int t = 32 * ch + i;
+                    pk[i >> 1] = pack_bf16x2(-bet[t] * gam[t] * __uint_as_float(r[i]),
+                                             -bet[t + 1] * gam[t + 1] * __uint_as_float(r[i + 1]));
                 }
+                tmem_st16(tm + lb + T1_DRB + 16 * ch, pk);
             }
-            if (p.mode == 0) fence_proxy_async_smem();
+            // the previous chunk's dR / dV stores have read their staging before it is written again below
+            if (tid == 0) bulk_wait_read0();
             sync_after_tmem_st();
-            if (tid == 0) arrive(&bars[B1_GFREE0 + s]);  // this chunk's gates are no longer read
-            if (p.mode == 0 && tid == 0) {
-                // dR to the workspace, dV to the output (its rows past the sequence's end are outside the
-                // tensor and not written)
-                for (int blk = 0; blk < 2; ++blk) {
-                    tma_store_2d(&tm_drw, sm + O1_DRST + blk * 8192, blk * 64, (int)(item * 64));
-                    tma_store_4d(&tm_dv, sm + O1_DVST + blk * 8192, blk * 64, h, t0, b);
-                }
-                bulk_commit();
-            }
             B1DBG(5)
             // ---- dS += dO^T (diag(gamma) Q) - dR^T diag(beta gamma) K ----
             if (tid == 0) {
@@ -609,10 +588,41 @@ bwd_chain_kernel(const __grid_constant__ CUtensorMap tm_do, const __grid_constan
                 mma_commit(&bars[B1_EMPTY0 + s]);
                 mma_commit(&bars[B1_MMA]);
             }
+            if (p.mode == 0) {
+                // thread j holds column j of dR (tokens 32 ch ..): element (t, j) of the staged [64 t][128 j]
+                // tiles sits in box j / 64, row t, 16-byte chunk (j % 64) / 8.  Lanes j, j ^ 1 trade one value
+                // per token pair so that each writes two adjacent columns of one row: the even lane columns
+                // j, j + 1 of row t, the odd lane columns j - 1, j of row t + 1.
+                const bool odd = (lane & 1) != 0;
+                const int j0 = j & ~1;
+                const uint32_t col = (uint32_t)(j0 >> 6) * 8192, cj = (uint32_t)((j0 & 63) >> 3), bj = (j0 & 7) * 2;
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    const int t = 32 * ch + i;
+                    const float x0 = __uint_as_float(r[i]), x1 = __uint_as_float(r[i + 1]);
+                    const float got = __shfl_xor_sync(0xffffffffu, odd ? x0 : x1, 1);
+                    const int row = odd ? t + 1 : t;
+                    const float lo = odd ? got : x0, hi = odd ? x1 : got, bt = bet[row];
+                    const uint32_t o = col + sw128(row, cj) + bj;
+                    *reinterpret_cast<uint32_t *>(sm + O1_DRST + o) = pack_bf16x2(lo, hi);
+                    *reinterpret_cast<uint32_t *>(sm + O1_DVST + o) = pack_bf16x2(bt * lo, bt * hi);
+                }
+                fence_proxy_async_smem();
+            }
+            named_bar(kBarP1, kP1Compute);
+            if (tid == 0) {
+                arrive(&bars[B1_GFREE0 + s]);  // this chunk's gates are no longer read
+                if (p.mode == 0) {
+                    // dR to the workspace, dV to the output (its rows past the sequence's end are outside
+                    // the tensor and not written)
+                    for (int blk = 0; blk < 2; ++blk) {
+                        tma_store_2d(&tm_drw, sm + O1_DRST + blk * 8192, blk * 64, (int)(item * 64));
+                        tma_store_4d(&tm_dv, sm + O1_DVST + blk * 8192, blk * 64, h, t0, b);
+                    }
+                    bulk_commit();
+                }
+            }
             B1DBG(6)
-            // this chunk's stores have read their staging before the next chunk writes it (the barrier
-            // of the round below orders the other threads)
-            if (tid == 0) bulk_wait_read0();
             mma_round();
             B1DBG(7)
         }
