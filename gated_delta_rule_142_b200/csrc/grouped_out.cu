@@ -14,7 +14,9 @@
 // with Q_r the query head's tile, P_r its decayed, masked Q_r K^T tile and
 // gamma its gate scales, both from the prep kernel's workspace item of that
 // query head.  Two MMAs into one 128 x 64 accumulator per chunk; persistent
-// CTAs, three per SM.
+// CTAs, three per SM, each over a contiguous range of (memory chunk, query
+// head) steps with the query head fastest, so that S and U^T load once for the
+// query heads of a group that a CTA takes in a row.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -55,7 +57,8 @@ __device__ int g_grp_timeout;
 struct GrpArgs {
     const float *gates;  // [items][kRecFloats]: the prep kernel's records, every query head
     __nv_bfloat16 *out;  // [B, T, H, 128]
-    int64_t T, H, items;  // items: B * Hkv * (G - 1) * chunks
+    int64_t T, H, items;  // items: B * Hkv * chunks * (G - 1), the query head fastest
+    int64_t per;          // items per CTA (a contiguous range)
     int chunks, group;
 };
 
@@ -91,17 +94,18 @@ grouped_out_kernel(const __grid_constant__ CUtensorMap tm_s, const __grid_consta
     tc_fence_after();
     const uint32_t tm = *tmem_slot;
 
-    // item -> (b, hk, r, c): query head h = hk * G + r, memory index m = b * Hkv + hk
+    // item -> (b, hk, c, r): query head h = hk * G + r, memory index m = b * Hkv + hk; the memory chunk
+    // m * nch + c is item / (G - 1)
     struct Coord {
         int b, h, c;
         int64_t m, wi;  // memory index, the query head's workspace item
     };
     auto coord = [&](int64_t it) {
         Coord x;
-        x.c = (int)(it % nch);
-        int64_t rest = it / nch;
-        const int r = 1 + (int)(rest % (G - 1));
-        rest /= (G - 1);
+        const int r = 1 + (int)(it % (G - 1));
+        int64_t rest = it / (G - 1);
+        x.c = (int)(rest % nch);
+        rest /= nch;
         const int hk = (int)(rest % Hkv);
         x.b = (int)(rest / Hkv);
         x.h = hk * G + r;
@@ -109,23 +113,30 @@ grouped_out_kernel(const __grid_constant__ CUtensorMap tm_s, const __grid_consta
         x.wi = ((int64_t)x.b * H + x.h) * nch + x.c;
         return x;
     };
+    // this CTA's range of items
+    const int64_t first = (int64_t)blockIdx.x * p.per;
+    const int64_t last = (first + p.per < p.items) ? first + p.per : p.items;
+    // S and U^T of item `it`'s memory chunk load unless the item before it in this range had them
     auto issue_loads = [&](int64_t it) {  // thread 0
         const Coord x = coord(it);
-        const int64_t ci = x.m * nch + x.c;  // checkpoint / U^T index of the memory
-        mbar_arrive_expect_tx(&bars[0], 32768 + 16384 + 16384 + 8192);
-        for (int blk = 0; blk < 2; ++blk) {
-            tma_load_2d(sm + G_S + blk * 16384, &tm_s, &bars[0], blk * 64, (int)(ci * 128));
-            tma_load_4d(sm + G_Q + blk * 8192, &tm_q, &bars[0], blk * 64, x.h, x.c * kC, x.b);
+        const bool su = it == first || it / (G - 1) != (it - 1) / (G - 1);
+        mbar_arrive_expect_tx(&bars[0], (su ? 32768 + 16384 : 0) + 16384 + 8192);
+        if (su) {
+            const int64_t ci = x.m * nch + x.c;  // checkpoint / U^T index of the memory
+            for (int blk = 0; blk < 2; ++blk)
+                tma_load_2d(sm + G_S + blk * 16384, &tm_s, &bars[0], blk * 64, (int)(ci * 128));
+            tma_load_2d(sm + G_U, &tm_u, &bars[0], 0, (int)(ci * 128));
         }
-        tma_load_2d(sm + G_U, &tm_u, &bars[0], 0, (int)(ci * 128));
+        for (int blk = 0; blk < 2; ++blk)
+            tma_load_4d(sm + G_Q + blk * 8192, &tm_q, &bars[0], blk * 64, x.h, x.c * kC, x.b);
         tma_load_2d(sm + G_P, &tm_p, &bars[0], 0, (int)(x.wi * 64));
     };
-    if (tid == 0 && (int64_t)blockIdx.x < p.items) issue_loads(blockIdx.x);
+    if (tid == 0 && first < last) issue_loads(first);
 
     bool ok = true;
     uint32_t ph = 0;
 #pragma unroll 1
-    for (int64_t it = blockIdx.x; it < p.items && ok; it += gridDim.x, ph ^= 1u) {
+    for (int64_t it = first; it < last && ok; ++it, ph ^= 1u) {
         const Coord x = coord(it);
         const int t0 = x.c * kC;
         const int n = (T - t0 < kC) ? (int)(T - t0) : kC;
@@ -165,7 +176,7 @@ grouped_out_kernel(const __grid_constant__ CUtensorMap tm_s, const __grid_consta
         if (!(ok = __syncthreads_and(wait_bar(&bars[1], ph, abort_flag)))) break;
         tc_fence_after();
         // the tiles are read: the next item's loads may land while this one's outputs leave
-        if (tid == 0 && it + gridDim.x < p.items) issue_loads(it + gridDim.x);
+        if (tid == 0 && it + 1 < last) issue_loads(it + 1);
         // O^T row j -> out[b, t0 + t, h, j]
         __nv_bfloat16 *dst = p.out + (((int64_t)x.b * T + t0) * H + x.h) * kD + j;
 #pragma unroll 1
@@ -250,7 +261,9 @@ cudaError_t launch_grouped_outputs(const FwdProblem &p, const void *ckpt, const 
     a.items = items;
     a.chunks = (int)nch;
     a.group = G;
-    const int64_t grid = items < 3 * (int64_t)sm_count ? items : 3 * (int64_t)sm_count;
+    const int64_t ctas = items < 3 * (int64_t)sm_count ? items : 3 * (int64_t)sm_count;
+    a.per = (items + ctas - 1) / ctas;
+    const int64_t grid = (items + a.per - 1) / a.per;
     {
         TimedLaunch tl_(GDN_KERNEL_GROUP_OUT, stream);
         grouped_out_kernel<<<(unsigned)grid, kGrpThreads, SMEM_GRP, stream>>>(ms, mu, mq, mp, a);
