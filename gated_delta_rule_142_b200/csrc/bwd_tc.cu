@@ -19,16 +19,22 @@
 // After a forward recompute (the two-kernel forward, asked for bf16
 // checkpoints of the state entering every chunk and for T of every chunk),
 // two passes:
-//   1. bwd_chain_kernel, one CTA per (b, h), walks the chunks backwards with
-//      dS in tensor memory: per chunk dU^T, dR^T and the dS update as three
-//      rounds of MMAs.  It writes dV, and for pass 2 dS' (bf16) and dR (bf16)
-//      of every chunk.
+//   1. bwd_chain_kernel, one CTA per (b, h) and segment, walks the chunks
+//      backwards with dS in tensor memory: per chunk dU^T, dR^T and the dS
+//      update as three rounds of MMAs, while a tenth warp prepares the next
+//      chunk's gates and gamma-scaled Q.  It writes dV, and for pass 2 dS'
+//      (bf16) and dR (bf16) of every chunk, through TMA stores.  Long
+//      sequences with few heads are cut into the forward's segments: a
+//      transfer launch of the same kernel gives each segment's map of the
+//      adjoint (dS -> dS X_p + B'_p, X_p the transpose of the segment's
+//      forward transfer), the forward's prefix kernel chains them from
+//      dS_final, and every segment then walks at once.
 //   2. bwd_grad_kernel, chunk-parallel (persistent CTAs over the chunks of
 //      every (b, h)): from S, dS', dR and the chunk's tiles it forms
 //      [Q;K] K^T, [Q;K] S^T, dS' K^T, U^T, [dO; dR] U^T and finally
 //      [dQ; dK] as one 128-row accumulator fed by three products, then dbeta
 //      and d log alpha.
-// Both kernels run their roles in lock step (one thread issues, all wait on
+// Both kernels run their rounds in lock step (one thread issues, all wait on
 // the MMA's mbarrier with a bounded wait), so each round's latency shows; the
 // chunk-parallel pass hides it behind the other SMs' chunks.
 #include <cuda.h>
