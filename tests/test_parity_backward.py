@@ -185,3 +185,18 @@ def test_tensor_core_backward_segments_match_one_walk(monkeypatch):
     b = check(inp, d_out, dSf, "bf16", 64, label="one walk")
     for x, y in zip(a, b):
         assert rel_err(cpu_f64(x), cpu_f64(y)) <= TOL["bf16"]
+
+
+def test_tensor_core_backward_many_segments(monkeypatch):
+    """Sixteen segments over 4,000 tokens (63 chunks, ragged last chunk): head 0 decays fast (every reverse
+    transfer negligible within a short head of its segment), head 1 keeps alpha close to 1 (every transfer
+    exact, the prefix chaining fifteen products)."""
+    monkeypatch.setenv("GDN_SEGMENTS", "16")
+    monkeypatch.delenv("GDN_BWD_PATH", raising=False)
+    monkeypatch.delenv("GDN_BWD_RECOMPUTE", raising=False)
+    B, T, H = 1, 4000, 2
+    inp = forward_inputs(B, T, H, 128, 128, "bf16", seed=95, s0_std=0.2)
+    inp["log_alpha"][:, :, 1] = -1e-3 * torch.rand(inp["log_alpha"][:, :, 1].shape,
+                                                    generator=torch.Generator().manual_seed(7))
+    d_out, dSf = grads_in(B, T, H, 128, 128, "bf16", seed=96)
+    check(inp, d_out, dSf, "bf16", 64, label="sixteen segments")
