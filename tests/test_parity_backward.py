@@ -200,3 +200,15 @@ def test_tensor_core_backward_many_segments(monkeypatch):
                                                     generator=torch.Generator().manual_seed(7))
     d_out, dSf = grads_in(B, T, H, 128, 128, "bf16", seed=96)
     check(inp, d_out, dSf, "bf16", 64, label="sixteen segments")
+
+
+def test_tensor_core_backward_segments_two_batch_rows(monkeypatch):
+    """Segments with two batch rows (the transfer slots, prefix chains and entry adjoints of every
+    (b, h)), a ragged last chunk, S0 and dS_final given."""
+    monkeypatch.setenv("GDN_SEGMENTS", "5")
+    monkeypatch.delenv("GDN_BWD_PATH", raising=False)
+    monkeypatch.delenv("GDN_BWD_RECOMPUTE", raising=False)
+    B, T, H = 2, 1500, 2
+    inp = forward_inputs(B, T, H, 128, 128, "bf16", seed=97, s0_std=0.3, alpha_mu=-4.0)
+    d_out, dSf = grads_in(B, T, H, 128, 128, "bf16", seed=98)
+    check(inp, d_out, dSf, "bf16", 64, label="segments, two batch rows")
